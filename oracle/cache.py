@@ -1,0 +1,96 @@
+"""Layer-level semantics of the quantized cache: anchors, effective bits, decode.
+
+Anchors ("Fourier Magnitude KV Cache Quantization" post 6, "Corrected semantics":
+"quantize ALL layers, anchors only protect"; "Minimal recipe": "fp16 anchors on layer 0
+alone (D=48)"; "The winning recipe": "keep the KV of the first N decoded tokens in high
+precision only on the quantization-sensitive layers"; "sliding window s64 (all layers)").
+Every row is quantized; a row in the anchor set is additionally kept as its original fp16
+row, and attention reads that fp16 row instead of the quantized one.  Rules, for layers in
+the anchor layer set:
+  first_n(n): tokens t < n
+  window(w):  tokens t >= L - w, L = the sequence's stored length
+  all:        every token of the layer
+
+Effective bits ("E21W" "Result": "Group scales are counted in the bit totals (3.5 bits
+per value for 3-bit at group 32, 4.5 for 4-bit)"; "E22L" "What I tested": "Bits per value
+are averaged over keys and values and include the scales"; post 6 "Corrected semantics":
+"NF4/g64 + dp32 anchors ALL layers: ... eff bits"): (code bits + 16 per scale + 16 per zero
+point + 16 D per anchored row + 16 D per channel-scale vector) / values, averaged over K
+and V.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import attention as A
+from .quant import Side, bits_per_value, quantize_rows, to_original_f64
+
+
+@dataclass
+class Spec:
+    n_layers: int
+    batch: int
+    n_kv: int
+    n_q: int
+    D: int
+    k: Side
+    v: Side
+    anchor_layers: frozenset = field(default_factory=frozenset)
+    anchor_rule: str = "none"  # none | first_n | window | all
+    anchor_n: int = 0
+    sm_scale: float | None = None
+
+
+def anchored(spec: Spec, layer: int, tokens: np.ndarray, seq_len: int) -> np.ndarray:
+    t = np.asarray(tokens)
+    if spec.anchor_rule == "none" or layer not in spec.anchor_layers:
+        return np.zeros(t.shape, dtype=bool)
+    if spec.anchor_rule == "first_n":
+        return t < spec.anchor_n
+    if spec.anchor_rule == "window":
+        return (t >= seq_len - spec.anchor_n) & (t < seq_len)
+    if spec.anchor_rule == "all":
+        return t < seq_len
+    raise ValueError(spec.anchor_rule)
+
+
+def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None):
+    """Quantize one (layer, sequence, kv-head) unit: K16, V16 [T, D]; c16 [D] or None."""
+    kq = quantize_rows(K16, spec.k, None if c16 is None else np.broadcast_to(c16, K16.shape))
+    vq = quantize_rows(V16, spec.v, None)
+    return kq, vq
+
+
+def reconstruct_unit(spec: Spec, layer: int, K16, V16, kq, vq, seq_len: int, c16=None):
+    """Keys and values attention sees for one unit (fp64 [T, D]); anchors override."""
+    T = K16.shape[0]
+    cK = None if c16 is None else np.broadcast_to(c16, K16.shape)
+    Kh = to_original_f64(kq["exact"], spec.k, cK)
+    Vh = to_original_f64(vq["exact"], spec.v, None)
+    an = anchored(spec, layer, np.arange(T), seq_len)
+    Kh[an] = np.asarray(K16, dtype=np.float16)[an].astype(np.float64)
+    Vh[an] = np.asarray(V16, dtype=np.float16)[an].astype(np.float64)
+    return Kh, Vh
+
+
+def decode_query(spec: Spec, layer: int, q16: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, kv_len: int):
+    """q16 [Hq, D]; Kh, Vh [Hkv, T, D] reconstructed; returns (o, lse, p)."""
+    return A.attention(np.asarray(q16, np.float16), Kh, Vh, kv_len, spec.sm_scale)
+
+
+def effective_bits(spec: Spec, seq_len: int) -> float:
+    """Average stored bits per K/V value over all layers of one sequence of length seq_len."""
+    D = spec.D
+    tot = 0.0
+    for layer in range(spec.n_layers):
+        an = anchored(spec, layer, np.arange(seq_len), seq_len).sum()
+        for side, is_k in ((spec.k, True), (spec.v, False)):
+            per_row = bits_per_value(side, D) * D
+            bits = (seq_len - an) * per_row + an * 16 * D
+            if is_k and side.chan_scale:
+                bits += 16 * D
+            tot += bits
+    return tot / (spec.n_layers * 2 * seq_len * D)

@@ -1,0 +1,474 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU needed).
+
+Each test checks the oracle against something other than itself: hand-worked fixtures, closed
+forms printed on the pages, textbook definitions, library routines, brute force in exact
+rational arithmetic, or invariants.  A plausible mistake (dropped term, wrong sign or index,
+transposed operand, wrong tie rule) fails at least one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import attention as A
+from oracle import cache as C
+from oracle import nf4 as N
+from oracle import quant as Q
+from oracle import transforms as T
+from oracle.quant import Side
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "packing.json")))
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------- packing
+@pytest.mark.parametrize("case", GOLD["pack_bits"])
+def test_pack_bits_golden(case):
+    got = Q.pack_bits(np.array([case["codes"]]), case["bits"])[0].tolist()
+    assert got == case["bytes"]
+    back = Q.unpack_bits(np.array([case["bytes"]], dtype=np.uint8), case["bits"], len(case["codes"]))
+    assert back[0].tolist() == case["codes"]
+
+
+def test_pack_trits_golden():
+    case = GOLD["pack_trits"][0]
+    t = np.array([case["t"]])
+    assert Q.pack_trits(t + 1)[0].tolist() == case["bytes"]
+    assert (Q.unpack_trits(np.array([case["bytes"]], np.uint8), 7) - 1)[0].tolist() == case["t"]
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 6, 8])
+def test_pack_roundtrip(b):
+    c = rng(b).integers(0, 2 ** b, size=(7, 128))
+    assert (Q.unpack_bits(Q.pack_bits(c, b), b, 128) == c).all()
+
+
+def test_row_bytes():
+    assert Side("int", 4).row_bytes(128) == 64
+    assert Side("int", 3).row_bytes(256) == 96
+    assert Side("int", 2).row_bytes(256) == 64
+    assert Side("ternary", group=8).row_bytes(128) == 26
+    assert Side("sign", group=4).row_bytes(128) == 16
+    assert Side("polar", 4, 8).row_bytes(128) == 96
+    assert Side("cart", 6).row_bytes(128) == 96
+
+
+# ----------------------------------------------------------------------------- grids: golden
+def _rows(x):
+    return np.array([x], dtype=np.float16)
+
+
+@pytest.mark.parametrize("case", GOLD["int_absmax"])
+def test_int_absmax_golden(case):
+    r = Q.quantize_rows(_rows(case["x"]), Side("int", case["bits"], group=4))
+    assert float(r["scales"][0, 0]) == case["d"]
+    assert r["q"][0].tolist() == case["q"]
+    assert r["bytes"][0].tolist() == [case["byte"]]
+
+
+def test_int_minmax_golden():
+    case = GOLD["int_minmax"][0]
+    r = Q.quantize_rows(_rows(case["x"]), Side("int", case["bits"], scale="minmax", group=4))
+    assert float(r["scales"][0, 0]) == case["d"] and float(r["zeros"][0, 0]) == case["z"]
+    assert r["q"][0].tolist() == case["q"]
+    assert r["bytes"][0].tolist() == [case["byte"]]
+
+
+def test_ternary_golden():
+    case = GOLD["ternary"][0]
+    r = Q.quantize_rows(_rows(case["x"]), Side("ternary", group=4))
+    assert float(r["scales"][0, 0]) == case["s"]
+    assert r["q"][0].tolist() == case["t"]
+    assert r["bytes"][0].tolist() == [case["byte"]]
+
+
+def test_nf4_golden():
+    case = GOLD["nf4"][0]
+    r = Q.quantize_rows(_rows(case["x"]), Side("nf4", group=4))
+    assert float(r["scales"][0, 0]) == case["s"]
+    assert r["q"][0].tolist() == case["codes"]
+    assert r["bytes"][0].tolist() == case["bytes"]
+
+
+def test_sign_golden():
+    case = GOLD["sign"][0]
+    r = Q.quantize_rows(_rows(case["x"]), Side("sign", group=4))
+    assert float(r["scales"][0, 0]) == case["s"]
+    assert r["q"][0].tolist() == case["t"]
+    assert r["bytes"][0].tolist() == [case["byte"]]
+
+
+# ----------------------------------------------------------------------------- grids: brute force
+def _nearest_exact(x: float, levels):
+    """Index of the nearest level in exact rational arithmetic, ties to the larger level."""
+    fx = Fraction(x)
+    best = None
+    for i, lv in enumerate(levels):
+        dist = abs(fx - lv)
+        if best is None or dist < best[0] or (dist == best[0] and lv > levels[best[1]]):
+            best = (dist, i)
+    return best[1]
+
+
+@pytest.mark.parametrize("b", [2, 3, 4, 8])
+def test_int_absmax_nearest_grid_point(b):
+    x = (rng(b).standard_normal((6, 64)) * 3).astype(np.float16)
+    side = Side("int", b, group=32, rot=0)
+    r = Q.quantize_rows(x, side)
+    qmin, qmax = -(2 ** (b - 1)), 2 ** (b - 1) - 1
+    for i in range(6):
+        for gi in range(2):
+            d = Fraction(float(r["scales"][i, gi]))
+            grp = x[i, gi * 32:(gi + 1) * 32].astype(np.float64)
+            # the extreme element maps to the full-range end of the grid
+            j = int(np.argmax(np.abs(grp)))
+            assert r["q"][i, gi * 32 + j] == qmin
+            levels = [k * d for k in range(qmin, qmax + 1)]
+            for jj in range(32):
+                if d == 0:
+                    continue
+                # levels are in k order; nearest in value with ties to larger code = larger k
+                fx = Fraction(float(grp[jj]))
+                dists = [abs(fx - lv) for lv in levels]
+                m = min(dists)
+                want = max(k for k, dd in zip(range(qmin, qmax + 1), dists) if dd == m)
+                assert r["q"][i, gi * 32 + jj] == want
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_int_minmax_nearest_grid_point(b):
+    x = (rng(10 + b).standard_normal((5, 64)) * 2 + 0.7).astype(np.float16)
+    r = Q.quantize_rows(x, Side("int", b, scale="minmax", group=32))
+    for i in range(5):
+        for gi in range(2):
+            d = Fraction(float(r["scales"][i, gi]))
+            z = Fraction(float(r["zeros"][i, gi]))
+            levels = [z + k * d for k in range(2 ** b)]
+            for jj in range(32):
+                want = _nearest_exact(float(x[i, gi * 32 + jj]), levels)
+                assert r["q"][i, gi * 32 + jj] == want
+
+
+def test_nf4_nearest_level():
+    x = (rng(3).standard_normal((4, 128))).astype(np.float16)
+    r = Q.quantize_rows(x, Side("nf4", group=64))
+    L = [Fraction(float(v)) for v in N.nf4_levels()]
+    for i in range(4):
+        for gi in range(2):
+            s = Fraction(float(r["scales"][i, gi]))
+            for jj in range(64):
+                want = _nearest_exact(float(x[i, gi * 64 + jj]), [lv * s for lv in L])
+                assert r["q"][i, gi * 64 + jj] == want
+
+
+def test_ternary_nearest_level():
+    x = (rng(4).standard_normal((4, 64))).astype(np.float16)
+    r = Q.quantize_rows(x, Side("ternary", group=8))
+    for i in range(4):
+        for gi in range(8):
+            s = Fraction(float(r["scales"][i, gi]))
+            for jj in range(8):
+                want = _nearest_exact(float(x[i, gi * 8 + jj]), [-s, Fraction(0), s]) - 1
+                assert r["q"][i, gi * 8 + jj] == want
+
+
+def test_round_half_up_exact_adversarial():
+    """Exact ties and values one fp32 ulp either side of a tie."""
+    d = np.float16(0.1).astype(np.float64)
+    xs, want = [], []
+    for k in range(-8, 8):
+        tie = (Fraction(2 * k + 1, 2)) * Fraction(float(d))
+        t32 = np.float32(float(tie))
+        for v in (np.nextafter(t32, np.float32(-1e9)), t32, np.nextafter(t32, np.float32(1e9))):
+            xs.append(float(v))
+            r = Fraction(float(v)) / Fraction(float(d)) + Fraction(1, 2)
+            want.append(math.floor(r))
+    got = Q.round_half_up_exact(np.array(xs), d)
+    assert got.tolist() == want
+
+
+def test_roundtrip_error_bound():
+    """|x - x_hat| <= |d|/2 inside the grid hull (the ggml grid clamps one side)."""
+    x = (rng(5).standard_normal((16, 128)) * 4).astype(np.float16)
+    for b in (2, 3, 4):
+        side = Side("int", b, group=32)
+        r = Q.quantize_rows(x, side)
+        d = np.repeat(r["scales"].astype(np.float64), 32, axis=1)
+        inside = (r["q"] > -(2 ** (b - 1))) & (r["q"] < 2 ** (b - 1) - 1)
+        err = np.abs(x.astype(np.float64) - r["exact"])
+        assert (err[inside] <= np.abs(d[inside]) / 2 + 1e-12).all()
+        assert (err <= np.abs(d) + 1e-12).all()
+
+
+def test_level_sets():
+    """Grids named on the pages: int2 -2..1 ("E22L"), ternary {-1,0,1}, sign {-1,1}."""
+    x = (rng(6).standard_normal((64, 128)) * 3).astype(np.float16)
+    assert set(np.unique(Q.quantize_rows(x, Side("int", 2, group=128))["q"])) == {-2, -1, 0, 1}
+    assert set(np.unique(Q.quantize_rows(x, Side("int", 4, group=32))["q"])) <= set(range(-8, 8))
+    assert set(np.unique(Q.quantize_rows(x, Side("ternary", group=8))["q"])) == {-1, 0, 1}
+    assert set(np.unique(Q.quantize_rows(x, Side("sign", group=4))["q"])) == {-1, 1}
+
+
+def test_sign_scale_least_squares_and_page_error():
+    """s = mean|x| minimises sum (x - s t)^2 for t = sign(x); on Gaussian rows the relative
+    error norm tends to sqrt(1 - 2/pi) = 0.603, inside the 0.54-0.63 K/V rel-err that post 6
+    ("Debunk audit") reports for sign KV."""
+    x = rng(7).standard_normal((256, 128)).astype(np.float16)
+    side = Side("sign", group=128)
+    r = Q.quantize_rows(x, side)
+    t = np.where(x >= 0, 1.0, -1.0)
+    s_ls = (x.astype(np.float64) * t).sum(axis=1) / 128.0
+    assert np.allclose(r["scales"][:, 0].astype(np.float64), s_ls, rtol=1e-3)
+    rel = math.sqrt(A.rel_sq_error(x, r["exact"]))
+    assert abs(rel - math.sqrt(1 - 2 / math.pi)) < 0.01
+    assert 0.54 <= rel <= 0.63
+
+
+# ----------------------------------------------------------------------------- NF4 construction
+def test_nf4_construction_properties():
+    L = N.nf4_levels()
+    assert len(L) == 16 and (np.diff(L) > 0).all()
+    assert L[0] == -1.0 and L[-1] == 1.0 and 0.0 in L
+    assert (L < 0).sum() == 7 and (L > 0).sum() == 8
+    # quantile spacing, checked through the normal CDF (erf), not the inverse used to build it
+    top = N.nf4_levels_f64()
+    z = statistics_inv(N.DELTA)
+    phi = lambda v: 0.5 * (1 + math.erf(v / math.sqrt(2)))
+    pos = sorted(v for v in top if v > 0)
+    neg = sorted(-v for v in top if v < 0)
+    assert np.allclose([phi(v * z) for v in pos], np.linspace(N.DELTA, 0.5, 9)[:-1][::-1], atol=1e-12)
+    assert np.allclose([phi(v * z) for v in neg], np.linspace(N.DELTA, 0.5, 8)[:-1][::-1], atol=1e-12)
+    # fp16 levels: midpoints times any fp16 scale are exact in fp32 (thresholds are exact)
+    mids = (L[:-1] + L[1:]) / 2
+    for s in np.float16([0.1, 3.7, 1000.0, 6e-5]).astype(np.float64):
+        assert ((mids * s).astype(np.float32).astype(np.float64) == mids * s).all()
+
+
+def statistics_inv(p):
+    import statistics
+    return statistics.NormalDist().inv_cdf(p)
+
+
+# ----------------------------------------------------------------------------- Hadamard
+@pytest.mark.parametrize("n", [128, 256])
+def test_hadamard_matrix(n):
+    H = T.sylvester(n)
+    ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+    pc = np.vectorize(lambda a: bin(a).count("1"))(ii & jj)
+    assert (H == (-1.0) ** pc).all()  # Sylvester = (-1)^popcount(i & j)
+    assert np.array_equal(H @ H.T, n * np.eye(n))
+
+
+@pytest.mark.parametrize("n", [128, 256])
+def test_fwht_matches_matrix_and_norm(n):
+    x = rng(n).standard_normal((5, n)).astype(np.float32)
+    y = T.fwht_f32(x, n).astype(np.float64)
+    ref = x.astype(np.float64) @ (T.sylvester(n) / math.sqrt(n)).T
+    assert np.allclose(y, ref, rtol=0, atol=1e-5 * np.abs(x).max())
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x.astype(np.float64), axis=1), rtol=1e-6)
+    e = np.eye(n, dtype=np.float32)[3:4]
+    col = T.fwht_f32(e, n)[0].astype(np.float64)
+    assert set(np.abs(col).tolist()) == {float(T.hadamard_scale(n))}
+    assert np.allclose(T.hadamard_inverse_f64(y, n), x, atol=1e-5)
+
+
+def test_hadamard_scale_is_nearest_fp32():
+    for n in (128, 256):
+        r = T.hadamard_scale(n)
+        exact = 1 / math.sqrt(n)
+        lo = np.nextafter(r, np.float32(0))
+        hi = np.nextafter(r, np.float32(1))
+        assert abs(float(r) - exact) <= abs(float(lo) - exact)
+        assert abs(float(r) - exact) <= abs(float(hi) - exact)
+
+
+def test_fwht_block_diagonal():
+    x = rng(9).standard_normal((3, 256)).astype(np.float32)
+    y = T.fwht_f32(x, 128)
+    assert np.array_equal(y[:, :128], T.fwht_f32(x[:, :128], 128))
+    assert np.array_equal(y[:, 128:], T.fwht_f32(x[:, 128:], 128))
+
+
+# ----------------------------------------------------------------------------- FFT
+def test_dft_matches_definition_and_library():
+    x = rng(11).standard_normal((4, 128)).astype(np.float32)
+    re, im = T.dft_dit_f32(x)
+    n = np.arange(128)
+    W = np.exp(-2j * np.pi * np.outer(n, n) / 128)
+    ref = x.astype(np.float64) @ W.T
+    scale = np.linalg.norm(x.astype(np.float64))
+    assert np.abs(re - ref.real).max() < 1e-5 * scale
+    assert np.abs(im - ref.imag).max() < 1e-5 * scale
+    lib = np.fft.fft(x.astype(np.float64), axis=-1)
+    assert np.abs((re + 1j * im) - lib).max() < 1e-5 * scale
+    # Hermitian symmetry of a real row's spectrum (the reply: "the FFT is Hermitian-symmetric")
+    X = re.astype(np.float64) + 1j * im.astype(np.float64)
+    assert np.abs(X[:, 1:] - np.conj(X[:, 1:][:, ::-1])).max() < 1e-5 * scale
+    # Parseval
+    assert np.allclose((np.abs(X) ** 2).sum(axis=1) / 128, (x.astype(np.float64) ** 2).sum(axis=1), rtol=1e-5)
+
+
+def test_fold_unfold_roundtrip():
+    x = rng(12).standard_normal((3, 128)).astype(np.float32)
+    a, b = T.fold_spectrum(*T.dft_dit_f32(x))
+    assert a.shape == (3, 64)
+    assert np.allclose(T.unfold_idft_f64(a, b), x, atol=1e-5)
+
+
+def test_polar_exact_phase_reduces_to_magnitude_error():
+    """Probe of the reply ("full FFT + magnitude quantization + exact phase"): with the
+    angle kept exact, the reconstruction error is the magnitude rounding alone."""
+    x = rng(13).standard_normal((8, 128)).astype(np.float16)
+    bm = 4
+    mc, pc, s = Q.quant_polar(x.astype(np.float32), bm, 8)
+    a, b = T.fold_spectrum(*T.dft_dit_f32(x.astype(np.float32)))
+    ang = np.arctan2(b.astype(np.float64), a.astype(np.float64))
+    m = mc * s[:, None]
+    xr = T.unfold_idft_f64(m * np.cos(ang), m * np.sin(ang))
+    mag = np.hypot(a.astype(np.float64), b.astype(np.float64))
+    assert (np.abs(m - mag) <= s[:, None] / 2 + 1e-6).all()
+    # error energy equals the magnitude error energy through Parseval on the folded slots
+    e_slot = (m - mag) ** 2
+    e_slot[:, 1:] *= 2
+    assert np.allclose(((xr - x.astype(np.float64)) ** 2).sum(axis=1), e_slot.sum(axis=1) / 128, rtol=1e-3, atol=1e-9)
+
+
+def test_polar_phase_codes_uniform_grid():
+    x = rng(14).standard_normal((32, 128)).astype(np.float16)
+    for bm, bp in ((4, 8), (5, 7), (6, 6), (7, 5), (8, 4)):
+        r = Q.quantize_rows(x, Side("polar", bm, bp))
+        mc, pc = r["q"][:, :64], r["q"][:, 64:]
+        assert mc.max() == 2 ** bm - 1 and mc.min() >= 0
+        assert pc.min() >= 0 and pc.max() < 2 ** bp
+        a, b = T.fold_spectrum(*T.dft_dit_f32(x.astype(np.float32)))
+        ang = np.arctan2(b.astype(np.float64), a.astype(np.float64))
+        phi = Q.phase_angles_f64(bp)[pc]
+        dphi = np.angle(np.exp(1j * (ang - phi)))
+        assert np.abs(dphi).max() <= math.pi / 2 ** bp + 1e-9
+
+
+# ----------------------------------------------------------------------------- effective bits
+def test_effective_bits_closed_forms():
+    D = 256
+    b = Q.bits_per_value
+    # "E21W" "Result": 3.5 bits for 3-bit at group 32, 4.5 for 4-bit
+    assert b(Side("int", 3, group=32), D) == 3.5
+    assert b(Side("int", 4, group=32), D) == 4.5
+    # "E22L" "What I tested": A 3.125, B 3.25, C 3.5, D 3.625 (averaged over K and V)
+    avg = lambda k, v: (b(k, D) + b(v, D)) / 2
+    assert avg(Side("int", 4, group=128, rot=256), Side("int", 2, group=128, rot=256)) == 3.125
+    assert avg(Side("int", 4, group=64, rot=256), Side("int", 2, group=64, rot=256)) == 3.25
+    assert avg(Side("int", 4, group=32), Side("int", 2, group=32, rot=256)) == 3.5
+    assert avg(Side("int", 4, group=128, rot=256), Side("int", 3, group=128, rot=256)) == 3.625
+    # post 6: NF4/g64 at 4.25 b, "NF4-K + int4-g64 V (4.25b)"
+    assert b(Side("nf4", group=64), 128) == 4.25
+    assert avg(Side("nf4", group=64), Side("int", 4, group=64)) == 4.25
+    # "E21W": the 3.19-bit allocation (K 2 bits in 2 layers, V 4 bits in 3 layers, 3 bits
+    # elsewhere, groups of 128, 8 layers)
+    Kb = [2, 2] + [3] * 6
+    Vb = [4] * 3 + [3] * 5
+    tot = sum(b(Side("int", k, group=128), D) for k in Kb) + sum(b(Side("int", v, group=128), D) for v in Vb)
+    assert tot / 16 == 3.1875 and round(tot / 16, 2) == 3.19
+    # the reply: (4 + 8) * 33 / 64 = 6.1875 payload bits at head_dim 64 with 33 one-sided
+    # bins; the folded 32-slot layout reaches the 6-bit asymptote, +16/128 for the scale at 128
+    assert (4 + 8) * (64 // 2 + 1) / 64 == 6.1875
+    assert Side("polar", 4, 8).row_bytes(64) * 8 / 64 == 6.0
+    for bm, bp in ((4, 8), (5, 7), (6, 6), (7, 5), (8, 4)):
+        assert b(Side("polar", bm, bp), 128) == 6.125
+    assert b(Side("cart", 6), 128) == 6.125
+    assert b(Side("int", 6, group=128, rot=128), 128) == 6.125
+
+
+def test_effective_bits_anchor_layer():
+    """Post 6 "Corrected semantics": NF4/g64 + L0-only anchors @ 4.69 eff bits, consistent
+    with one fully fp16 layer out of 26 (Gemma-3-1B depth): 4.25 + 11.75/26."""
+    s = C.Spec(26, 1, 1, 4, 256, Side("nf4", group=64), Side("nf4", group=64),
+               frozenset({0}), "all", 0)
+    assert abs(C.effective_bits(s, 4096) - 4.69) < 0.02
+
+
+def test_anchor_rules():
+    s = C.Spec(4, 1, 1, 1, 128, Side(), Side(), frozenset({0, 2}), "first_n", 48)
+    t = np.arange(100)
+    assert C.anchored(s, 0, t, 100).sum() == 48 and C.anchored(s, 1, t, 100).sum() == 0
+    s.anchor_rule, s.anchor_n = "window", 64
+    m = C.anchored(s, 2, t, 100)
+    assert m.sum() == 64 and m[36:].all() and not m[:36].any()
+    s.anchor_rule = "all"
+    assert C.anchored(s, 0, t, 100).all()
+
+
+# ----------------------------------------------------------------------------- attention
+def _brute_attention(q, K, V, kv_len):
+    """Pure-Python textbook softmax attention on tiny shapes."""
+    Hq, D = len(q), len(q[0])
+    Hkv = len(K)
+    G = Hq // Hkv
+    out = []
+    for h in range(Hq):
+        j = h // G
+        s = [sum(q[h][c] * K[j][t][c] for c in range(D)) / math.sqrt(D) for t in range(kv_len)]
+        m = max(s)
+        e = [math.exp(v - m) for v in s]
+        z = sum(e)
+        out.append([sum(e[t] / z * V[j][t][c] for t in range(kv_len)) for c in range(D)])
+    return out
+
+
+def test_attention_fp16_format_is_textbook():
+    r = rng(20)
+    Hkv, Hq, D, Tn = 2, 4, 16, 40
+    K = r.standard_normal((Hkv, Tn, D)).astype(np.float16)
+    V = r.standard_normal((Hkv, Tn, D)).astype(np.float16)
+    q = r.standard_normal((Hq, D)).astype(np.float16)
+    side = Side("fp16")
+    Kh = np.stack([Q.to_original_f64(Q.quantize_rows(K[j], side)["exact"], side) for j in range(Hkv)])
+    Vh = np.stack([Q.to_original_f64(Q.quantize_rows(V[j], side)["exact"], side) for j in range(Hkv)])
+    o, lse, p = A.attention(q, Kh, Vh, 33)
+    ref = _brute_attention(q.astype(float).tolist(), K.astype(float).tolist(), V.astype(float).tolist(), 33)
+    assert np.allclose(o, ref, atol=1e-12)
+    assert np.allclose(p.sum(axis=1), 1.0)
+
+
+def test_attention_split_merge_equals_one_pass():
+    r = rng(21)
+    K = r.standard_normal((1, 50, 8))
+    V = r.standard_normal((1, 50, 8))
+    q = r.standard_normal((2, 8))
+    o, lse, _ = A.attention(q, K, V, 50)
+    o1, l1, _ = A.attention(q, K[:, :20], V[:, :20], 20)
+    o2, l2, _ = A.attention(q, K[:, 20:], V[:, 20:], 30)
+    M = np.maximum(l1, l2)
+    w1, w2 = np.exp(l1 - M), np.exp(l2 - M)
+    om = (w1[:, None] * o1 + w2[:, None] * o2) / (w1 + w2)[:, None]
+    assert np.allclose(om, o) and np.allclose(M + np.log(w1 + w2), lse)
+
+
+def test_metrics_closed_forms():
+    p = np.array([0.5, 0.5])
+    qd = np.array([0.25, 0.75])
+    assert A.kl(p, p) == 0.0
+    assert abs(A.kl(p, qd) - (0.5 * math.log(2) + 0.5 * math.log(2 / 3))) < 1e-15
+    assert A.rel_l2([3.0, 4.0], [3.0, 4.0]) == 0.0
+    assert abs(A.rel_l2([3.0, 5.0], [3.0, 4.0]) - 0.2) < 1e-15
+    assert abs(A.rel_sq_error([1.0, 1.0], [1.0, 0.0]) - 0.5) < 1e-15
+
+
+def test_channel_scale_then_rotation_order():
+    """Variant D of "E21W": per-channel scale first, then rotation; dequant rotates back and
+    multiplies the scale back in."""
+    r = rng(22)
+    x = (r.standard_normal((4, 256)) * 3).astype(np.float16)
+    c = (np.abs(r.standard_normal(256)) + 0.5).astype(np.float16)
+    side = Side("int", 8, group=32, rot=256, chan_scale=True)
+    out = Q.quantize_rows(x, side, np.broadcast_to(c, x.shape))
+    xo = Q.to_original_f64(out["exact"], side, np.broadcast_to(c, x.shape))
+    assert A.rel_sq_error(x, xo) < 1e-4
+    y = T.fwht_f32(x.astype(np.float32) / c.astype(np.float32), 256)
+    assert np.array_equal(Q.transform_rows(x, side, np.broadcast_to(c, x.shape)), y)
