@@ -1,0 +1,182 @@
+/*
+ * kvq.h - low-bit KV-cache quantize-append and split-K decode attention for one B200 GPU.
+ *
+ * C ABI.  Every pointer is a plain device (or host, where stated) pointer; sizes are plain
+ * integers; streams are passed as `void*` holding a cudaStream_t (NULL = legacy default stream).
+ * No call allocates device memory except kvq_create (a small split-K workspace and nothing
+ * else); the cache itself lives in one caller-owned device arena.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [FMKQ]  "Fourier Magnitude KV Cache Quantization" forum thread: post 6 ("Corrected
+ *           semantics", "Minimal recipe", "Milestone", "The winning recipe") and the long
+ *           reply ("The three controls I would try first", "Fixed-rate magnitude/phase
+ *           allocation", "The finite-phase implementation and the physical codec may be
+ *           worth separating").
+ *   [E21W]  "PROVISIONAL: known 3-bit KV cache methods on the 4B ... (proxy queries)":
+ *           "What I tested", "Result".
+ *   [E22L]  "Can 4-bit keys and 2-bit values hit a 1M-token memory budget?": "What I
+ *           tested", "Result".
+ *   [LCPP]  llama.cpp issue #21385 "Per-head adaptive KV cache quantization": "Finding 1".
+ *
+ * Error behaviour: argument and configuration errors are detected on the host before any
+ * launch and returned as a status; launch failures come back as KVQ_ERR_CUDA.  No kernel
+ * traps or spins.  A device-side condition the host cannot see in advance (an append past
+ * the capacity while a CUDA graph replays) skips the offending writes and raises a bit in
+ * the cache's error word (kvq_error_flags).
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = -1,  /* null pointer, out-of-range index or size, inconsistent config */
+  KVQ_ERR_UNSUPPORTED = -2,  /* valid but not built (e.g. polar at head_dim != 128) */
+  KVQ_ERR_CAPACITY = -3,     /* append past capacity, or more queries than max_queries */
+  KVQ_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
+  KVQ_ERR_ALLOC = -5,        /* arena too small, or the workspace allocation failed */
+  KVQ_ERR_STATE = -6         /* call order violated (e.g. channel scale never set) */
+} kvq_status;
+
+/* Storage format of one side (K or V). */
+enum {
+  KVQ_FMT_FP16 = 0,     /* unquantized fp16 rows (the K-only arm's V [E22L]) */
+  KVQ_FMT_INT = 1,      /* b-bit integer grid; scale_mode ABSMAX (ggml signed -2^(b-1)..2^(b-1)-1,
+                           [E22L] "Result", [LCPP]) or MINMAX (asymmetric, [E21W] variant A) */
+  KVQ_FMT_NF4 = 2,      /* 16-level NormalFloat codebook, absmax scale [FMKQ] post 6 "NF4/g64" */
+  KVQ_FMT_TERNARY = 3,  /* {-s, 0, +s}, s = group absmax, 5 trits per byte [FMKQ] "Milestone" */
+  KVQ_FMT_SIGN = 4,     /* {-s, +s}, s = group mean |x| [FMKQ] "Minimal recipe" */
+  KVQ_FMT_POLAR = 5,    /* rFFT magnitude (bits) / phase (bits2) indices [FMKQ] reply */
+  KVQ_FMT_CART = 6      /* rFFT real/imag, signed absmax int-bits, one scale [FMKQ] reply control */
+};
+enum { KVQ_SCALE_ABSMAX = 0, KVQ_SCALE_MINMAX = 1 };
+enum { KVQ_ROT_NONE = 0, KVQ_ROT_H128 = 128, KVQ_ROT_H256 = 256 };
+enum { KVQ_ANCHOR_NONE = 0, KVQ_ANCHOR_FIRST_N = 1, KVQ_ANCHOR_WINDOW = 2, KVQ_ANCHOR_ALL = 3 };
+enum { KVQ_SIDE_K = 0, KVQ_SIDE_V = 1 };
+enum { KVQ_DOMAIN_STORED = 0, KVQ_DOMAIN_ORIGINAL = 1 };
+enum { KVQ_ERRF_CAPACITY = 1, KVQ_ERRF_SEQ_ID = 2 };
+
+typedef struct {
+  int32_t format;      /* KVQ_FMT_* */
+  int32_t bits;        /* INT: 2..8; CART: 2..8; POLAR: magnitude bits 1..8; else ignored */
+  int32_t bits2;       /* POLAR: phase bits 1..8; else ignored */
+  int32_t scale_mode;  /* INT: KVQ_SCALE_ABSMAX or KVQ_SCALE_MINMAX; else must be ABSMAX */
+  int32_t group;       /* channels per scale: 4, 8, 16, 32, 64 or 128, dividing head_dim
+                          (POLAR/CART: ignored, one scale per row; FP16: ignored) */
+  int32_t rotation;    /* KVQ_ROT_NONE / H128 / H256: orthonormal Sylvester Walsh-Hadamard over
+                          blocks of that many channels (block-diagonal if < head_dim)
+                          [E21W] variant B, [E22L] "What I tested".  Not with POLAR/CART. */
+  int32_t chan_scale;  /* K only: 1 = divide by a per-(layer, kv-head) fp16 channel scale
+                          before the rotation ([E21W] variants C/D); set with
+                          kvq_set_chan_scale before the first append. */
+} kvq_side;
+
+typedef struct {
+  int32_t n_layers;      /* 1..64 */
+  int32_t batch;         /* sequences, >= 1 */
+  int32_t n_kv_heads;    /* >= 1 */
+  int32_t n_q_heads;     /* multiple of n_kv_heads; query head h reads kv-head h / (Hq/Hkv) */
+  int32_t head_dim;      /* 64, 128 or 256 */
+  int32_t capacity;      /* tokens per sequence per layer, >= 1 */
+  int32_t max_queries;   /* largest n_q passed to kvq_decode_attention, >= 1 */
+  kvq_side k, v;
+  uint64_t anchor_layer_mask;  /* bit l set: layer l keeps fp16 anchor rows */
+  int32_t anchor_rule;         /* KVQ_ANCHOR_*; [FMKQ] post 6 "Corrected semantics" */
+  int32_t anchor_n;            /* FIRST_N: tokens t < n; WINDOW: the last n tokens */
+  float sm_scale;              /* softmax scale; 0 selects 1/sqrt(head_dim) */
+} kvq_config;
+
+/* Byte offsets (into the arena) and geometry of one (layer, side).  Rows of one
+ * (sequence, kv-head) are contiguous: row r of unit u = (b * n_kv_heads + h) is at
+ * codes + (u * row_stride_tokens + r) * row_bytes; scales (fp16) at
+ * scales + ((u * row_stride_tokens + r) * n_groups) * 2, zeros likewise (MINMAX only).
+ * Anchor rows (fp16, original domain) at anchors + ((u * anchor_rows + slot) * head_dim) * 2,
+ * slot = t (FIRST_N, ALL) or t mod anchor_n (WINDOW).  Offsets are -1 when absent. */
+typedef struct {
+  int64_t codes, scales, zeros, anchors, chan_scale, seq_len;
+  int32_t row_bytes, n_groups, row_stride_tokens, anchor_rows;
+} kvq_layout;
+
+typedef struct kvq_cache kvq_cache;
+
+/* Bytes of device memory the cache arena needs for `cfg` (256-byte aligned base).
+ * Returns KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config. Host only. */
+kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes);
+
+/* Validate `cfg`, bind the caller-owned device arena (>= kvq_arena_bytes, 256-byte aligned;
+ * owned by the caller, must outlive the handle), zero its sequence lengths, and allocate the
+ * handle plus a split-K workspace on the current device.  Synchronous. */
+kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out);
+
+/* Release the handle and its workspace (not the arena).  NULL is a no-op. */
+void kvq_free(kvq_cache* cache);
+
+/* Geometry of (layer, side) for inspection and tests.  Host only. */
+kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, int32_t side, kvq_layout* out);
+
+/* Copy the per-channel K scale c [n_kv_heads][head_dim] (fp16, device) of `layer` into the
+ * arena ([E21W] variants C/D: "calibrated offline").  Required before appending to a layer
+ * whose K side has chan_scale = 1. */
+kvq_status kvq_set_chan_scale(kvq_cache* cache, int32_t layer, const void* c_fp16, void* stream);
+
+/* Set the stored length of every sequence of `layer` (-1: all layers) to `len` (0..capacity).
+ * kvq_set_seq_len(cache, -1, 0, s) empties the cache. */
+kvq_status kvq_set_seq_len(kvq_cache* cache, int32_t layer, int32_t len, void* stream);
+
+/* Append n_new tokens to every sequence of `layer`: k, v are fp16 device [batch][n_kv_heads]
+ * [n_new][head_dim].  Token i of sequence b lands at position seq_len[b] + i (read on the
+ * device), every row is quantized (pre-transform, group scales, codes, packing), rows in
+ * the anchor set are also kept as fp16, and seq_len[b] += n_new.  n_new = prompt length is
+ * the bulk prefill; n_new = 1 is the decode-time append.  Errors: KVQ_ERR_CAPACITY if the
+ * host-side length bound would pass capacity; KVQ_ERR_STATE if a channel scale is required
+ * and was never set.  [E22L] "What I tested" ("Quantize ... keys and values as they enter
+ * the cache"), [FMKQ] post 6 "Corrected semantics" ("quantize ALL layers, anchors only
+ * protect"). */
+kvq_status kvq_quantize_append(kvq_cache* cache, int32_t layer, const void* k_fp16,
+                               const void* v_fp16, int32_t n_new, void* stream);
+
+/* Reconstruct tokens [t0, t0 + nt) of every (sequence, kv-head) of one side of `layer` into
+ * out [batch][n_kv_heads][nt][head_dim] (fp32 if out_fp32 else fp16).  STORED domain: the
+ * grid values (code x scale + zero; polar m cos(phi), m sin(phi) slot-interleaved) before
+ * any inverse transform, bit-exact by definition.  ORIGINAL domain: inverse DFT, inverse
+ * rotation and x channel scale applied, and anchored rows replaced by their fp16 copy. */
+kvq_status kvq_dequantize(const kvq_cache* cache, int32_t layer, int32_t side, int32_t domain,
+                          int32_t t0, int32_t nt, void* out, int32_t out_fp32, void* stream);
+
+/* Decode attention for n_q query positions on `layer`.  q: fp16 device [n_q][n_q_heads]
+ * [head_dim].  seq_ids: int32 device [n_q] (sequence each query reads) or NULL (query i reads
+ * sequence i; needs n_q <= batch); an id outside [0, batch) attends nothing and raises
+ * KVQ_ERRF_SEQ_ID in the error word.  kv_len: int32 device [n_q] (keys t < kv_len attended) or
+ * NULL (the sequence's stored length).  out: [n_q][n_q_heads][head_dim], fp32 if out_fp32 else
+ * fp16.  lse: fp32 device [n_q][n_q_heads] natural-log sum-exp of the scaled logits, or NULL.
+ * Split-K over tokens, dequantizing in registers, query pre-transformed once (q' = H(c . q)
+ * or the rFFT adjoint), partials merged by a second kernel that also undoes V's transform.
+ * An empty key range gives out = 0 and lse = -inf.  Errors: KVQ_ERR_CAPACITY if n_q >
+ * max_queries.  [E21W] "What I tested" (attention output, causal proxy queries). */
+kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q_fp16, int32_t n_q,
+                                const int32_t* seq_ids, const int32_t* kv_len, void* out,
+                                int32_t out_fp32, float* lse, void* stream);
+
+/* Read and clear the device error word (KVQ_ERRF_* bits) into *flags.  Synchronizes the
+ * device. */
+kvq_status kvq_error_flags(kvq_cache* cache, int32_t* flags);
+
+/* The 16 NF4 levels this library stores (fp16-exact values, ascending).  Host only. */
+kvq_status kvq_nf4_levels(float out[16]);
+
+/* Kernels launched by the last kvq_decode_attention / kvq_quantize_append call on this
+ * handle (for launch accounting).  Host only. */
+int32_t kvq_last_launch_count(const kvq_cache* cache);
+
+const char* kvq_status_str(kvq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -315,8 +315,8 @@ def quantize_rows(x16: np.ndarray, side: Side, c16=None) -> dict:
         mc, pc, s = quant_polar(x, bm, bp)
         out["bytes"] = np.concatenate([pack_bits(mc, bm), pack_bits(pc, bp)], axis=1)
         phi = phase_angles_f64(bp)
-        cos32 = np.cos(phi).astype(F32)
-        sin32 = np.sin(phi).astype(F32)
+        cos32 = np.array([math.cos(v) for v in phi], dtype=F64).astype(F32)  # libm, per entry
+        sin32 = np.array([math.sin(v) for v in phi], dtype=F64).astype(F32)
         m = (mc * s[:, None]).astype(F32)  # exact
         a32 = (m * cos32[pc]).astype(F32)
         b32 = (m * sin32[pc]).astype(F32)

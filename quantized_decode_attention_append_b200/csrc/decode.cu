@@ -1,0 +1,469 @@
+// kvq_decode_attention: split-K flash decode over the packed cache, then a merge kernel.
+//
+// Sources (page title, section): attention over the dequantized cache and the proxy-query setup
+// ("E21W" "What I tested": attention output, KL, causal proxy queries), the quantized-cache
+// simulation it stands in for ("E22L" "What I tested": keys and values quantized as they enter
+// the cache, "rotated" = 256-wide Hadamard), fp16 anchors ("Fourier Magnitude KV Cache
+// Quantization" post 6 "Corrected semantics").
+//
+// Pass 1 (one CTA per query x kv-head x split): the query group is transformed once into the
+// stored domain of K (q' = H(c . q), or the rFFT adjoint for polar/Cartesian K, pre-multiplied by
+// sm_scale * log2 e), then each tile of keys is scored against q' without reconstructing K,
+// online softmax runs in the log2 domain, and sum p * v is accumulated in V's stored domain.
+// Anchor rows (fp16, original domain) get their own split with the raw query.
+// Pass 2 (merge): log-sum-exp merge of the splits, V's inverse transform (Hadamard or inverse
+// DFT) applied once to the merged vector, anchors added, normalised.
+#include <math.h>
+
+#include "decode_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+__constant__ float d_nf4[16];
+__constant__ float d_tw_re[64];
+__constant__ float d_tw_im[64];
+__constant__ float d_ph_cos[512];
+__constant__ float d_ph_sin[512];
+
+cudaError_t upload_tables_decode(const HostTables& t) {
+  cudaError_t e;
+  if ((e = cudaMemcpyToSymbol(d_nf4, t.nf4, sizeof(t.nf4))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_tw_re, t.tw_re, sizeof(t.tw_re))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_tw_im, t.tw_im, sizeof(t.tw_im))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_ph_cos, t.ph_cos, sizeof(t.ph_cos))) != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(d_ph_sin, t.ph_sin, sizeof(t.ph_sin));
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kGenThreads = 128;
+constexpr int kGenTile = 128;
+constexpr int kMaxG = 8;  // GQA group size handled by the generic kernel
+
+struct QueryRange {
+  int seq, kv_len, len;
+  int qa, qb;  // quantized token range
+  int aa, ab;  // anchored token range
+};
+
+__device__ __forceinline__ QueryRange query_range(const LayerDev& L, int qi, const int* seq_ids, const int* kv_len) {
+  QueryRange r;
+  r.seq = seq_ids ? seq_ids[qi] : qi;
+  if (r.seq < 0 || r.seq >= L.B) {  // caller error: attend nothing, report it
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_SEQ_ID);
+    r.seq = 0;
+    r.len = 0;
+    r.kv_len = 0;
+    r.qa = r.qb = r.aa = r.ab = 0;
+    return r;
+  }
+  r.len = L.seq_len[r.seq];
+  int kl = kv_len ? kv_len[qi] : r.len;
+  kl = kl < 0 ? 0 : (kl > r.len ? r.len : kl);
+  r.kv_len = kl;
+  r.aa = 0;
+  r.ab = 0;
+  r.qa = 0;
+  r.qb = kl;
+  if (L.anchored) {
+    if (L.anchor_rule == KVQ_ANCHOR_FIRST_N) {
+      r.ab = L.anchor_n < kl ? L.anchor_n : kl;
+      r.qa = r.ab;
+    } else if (L.anchor_rule == KVQ_ANCHOR_WINDOW) {
+      int w0 = r.len - L.anchor_n;
+      w0 = w0 < 0 ? 0 : w0;
+      r.aa = w0 < kl ? w0 : kl;
+      r.ab = kl;
+      r.qb = r.aa;
+    } else if (L.anchor_rule == KVQ_ANCHOR_ALL) {
+      r.ab = kl;
+      r.qb = 0;
+    }
+  }
+  return r;
+}
+
+// q' for G heads into qs[G][D] (stored domain of K, x sm_scale log2 e) and qa[G][D] (raw, x same).
+template <int D>
+__device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, int qi, int kvh, int G,
+                              float* qs, float* qa) {
+  const SideDev& K = L.s[0];
+  const float scl = L.sm_scale * kLog2e;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < G * D; e += blockDim.x) {
+    const int h = e / D, j = e % D;
+    const float v = __half2float(q[((long long)qi * L.Hq + kvh * G + h) * D + j]);
+    qa[e] = v * scl;
+    qs[e] = K.chan_scale ? v * __half2float(K.chan[kvh * D + j]) : v;
+  }
+  __syncthreads();
+  if (K.rot == 128 || K.rot == 256) {
+    const int n = K.rot;
+    for (int h = 1; h < n; h <<= 1) {
+      for (int e = tid; e < G * D / 2; e += blockDim.x) {
+        // e-th pair: block of (i & ~h), index with bit h clear
+        const int row = e / (D / 2), p = e % (D / 2);
+        const int lo = p & (h - 1), hi = p >> __ffs(h) - 1;
+        const int i = (hi << (__ffs(h))) | lo;  // insert a 0 bit at position log2(h)
+        float* r = qs + row * D;
+        const float a = r[i], b = r[i + h];
+        r[i] = a + b;
+        r[i + h] = a - b;
+      }
+      __syncthreads();
+    }
+    const float rn = (n == 256) ? 0.0625f : 0.08838834764831845f;
+    for (int e = tid; e < G * D; e += blockDim.x) qs[e] *= rn;
+    __syncthreads();
+  } else if (K.fmt == KVQ_FMT_POLAR || K.fmt == KVQ_FMT_CART) {
+    // Parseval adjoint of the folded rFFT (N = 128): logit = sum_f alpha_f a_f + beta_f b_f,
+    // alpha_0 = Q_0/N, beta_0 = Q_64/N, alpha_f = 2 Re Q_f/N, beta_f = 2 Im Q_f/N.
+    __shared__ float tmp[kMaxG * 128];
+    for (int e = tid; e < G * 128; e += blockDim.x) tmp[e] = qs[e];
+    __syncthreads();
+    for (int e = tid; e < G * 64; e += blockDim.x) {
+      const int h = e / 64, f = e % 64;
+      const float* x = tmp + h * 128;
+      float re = 0.0f, im = 0.0f, re64 = 0.0f;
+      for (int n = 0; n < 128; ++n) {
+        const int k = (f * n) & 127;
+        const float c = k < 64 ? d_tw_re[k] : -d_tw_re[k - 64];
+        const float s = k < 64 ? d_tw_im[k] : -d_tw_im[k - 64];  // -sin
+        re += x[n] * c;
+        im += x[n] * s;
+        if (f == 0) re64 += (n & 1) ? -x[n] : x[n];
+      }
+      float* o = qs + h * 128;
+      if (f == 0) {
+        o[0] = re / 128.0f;
+        o[1] = re64 / 128.0f;
+      } else {
+        o[2 * f] = 2.0f * re / 128.0f;
+        o[2 * f + 1] = 2.0f * im / 128.0f;
+      }
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < G * D; e += blockDim.x) qs[e] *= scl;
+  __syncthreads();
+}
+
+// Generic pass 1: any format, any GQA group (<= 8), CUDA cores.  Thread-per-token scoring,
+// thread-per-channel value accumulation.
+template <int D>
+__global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L, const __half* __restrict__ q,
+                                                                     const int* __restrict__ seq_ids,
+                                                                     const int* __restrict__ kv_len, float* __restrict__ work,
+                                                                     int n_split, int nsp) {
+  constexpr int NCH = D > kGenThreads ? D / kGenThreads : 1;     // channels per thread
+  constexpr int TSUB = D < kGenThreads ? kGenThreads / D : 1;    // token subsets in PV
+  const int s = blockIdx.x, kvh = blockIdx.y, qi = blockIdx.z;
+  const int G = L.Hq / L.Hkv;
+  const int tid = threadIdx.x;
+  __shared__ float qs[kMaxG * D], qa[kMaxG * D];
+  __shared__ float sp[kMaxG][kGenTile];
+  __shared__ float m_run[kMaxG], l_run[kMaxG], alpha[kMaxG];
+  __shared__ float nf4[16], kcs[256], ksn[256], vcs[256], vsn[256];
+  __shared__ float red[kGenThreads / 32][kMaxG];
+
+  const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+  const SideDev& K = L.s[0];
+  const SideDev& V = L.s[1];
+  const bool anchor_split = (s == n_split);
+  int t0, t1;
+  if (anchor_split) {
+    t0 = R.aa;
+    t1 = R.ab;
+  } else {
+    const int n = R.qb - R.qa;
+    int chunk = (n + n_split - 1) / n_split;
+    chunk = ((chunk + kGenTile - 1) / kGenTile) * kGenTile;
+    t0 = R.qa + s * chunk;
+    t1 = t0 + chunk < R.qb ? t0 + chunk : R.qb;
+  }
+
+  if (tid < 16) nf4[tid] = d_nf4[tid];
+  if (K.fmt == KVQ_FMT_POLAR)
+    for (int k = tid; k < (1 << K.bits2); k += blockDim.x) {
+      kcs[k] = d_ph_cos[(1 << K.bits2) - 2 + k];
+      ksn[k] = d_ph_sin[(1 << K.bits2) - 2 + k];
+    }
+  if (V.fmt == KVQ_FMT_POLAR)
+    for (int k = tid; k < (1 << V.bits2); k += blockDim.x) {
+      vcs[k] = d_ph_cos[(1 << V.bits2) - 2 + k];
+      vsn[k] = d_ph_sin[(1 << V.bits2) - 2 + k];
+    }
+  if (tid < kMaxG) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.0f;
+  }
+  prepare_query<D>(L, q, qi, kvh, G, qs, qa);
+
+  const long long u = (long long)R.seq * L.Hkv + kvh;
+  float o[kMaxG][NCH];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) o[h][c] = 0.0f;
+
+  for (int tb = t0; tb < t1; tb += kGenTile) {
+    const int nt = (t1 - tb) < kGenTile ? (t1 - tb) : kGenTile;
+    // ---- scores: thread tid scores token tb + tid for all G heads
+    if (tid < nt) {
+      const int t = tb + tid;
+      float acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0f;
+      if (anchor_split) {
+        const __half* kr = K.anchors ? K.anchors + (u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t)) * D
+                                     : reinterpret_cast<const __half*>(K.codes + (u * L.Tcap + t) * K.row_bytes);
+        for (int j = 0; j < D; ++j) {
+          const float kv = __half2float(kr[j]);
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h)
+            if (h < G) acc[h] += qa[h * D + j] * kv;
+        }
+      } else {
+        const uint8_t* row = K.codes + (u * L.Tcap + t) * K.row_bytes;
+        const __half* sc = K.scales + (u * L.Tcap + t) * K.n_groups;
+        const __half* zr = K.zeros ? K.zeros + (u * L.Tcap + t) * K.n_groups : nullptr;
+        if (K.fmt == KVQ_FMT_POLAR) {
+          for (int f = 0; f < 64; ++f) {
+            const float2 ab = polar_slot(K, row, sc, f, kcs, ksn);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h)
+              if (h < G) acc[h] += qs[h * D + 2 * f] * ab.x + qs[h * D + 2 * f + 1] * ab.y;
+          }
+        } else {
+          for (int j = 0; j < D; ++j) {
+            const float kv = stored_value(K, row, sc, zr, j, nf4);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h)
+              if (h < G) acc[h] += qs[h * D + j] * kv;
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h)
+        if (h < G) sp[h][tid] = acc[h];
+    }
+    __syncthreads();
+    // ---- online softmax (log2 domain): per-head tile max, rescale factor, probabilities
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int h = 0; h < G; ++h) {
+        float mx = -INFINITY;
+        for (int t = tid; t < nt; t += blockDim.x) mx = fmaxf(mx, sp[h][t]);
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[warp][h] = mx;
+      }
+      __syncthreads();
+      if (tid < G) {
+        float mx = red[0][tid];
+        for (int w = 1; w < kGenThreads / 32; ++w) mx = fmaxf(mx, red[w][tid]);
+        const float mn = fmaxf(m_run[tid], mx);
+        alpha[tid] = exp2f(m_run[tid] - mn);  // m_run = -inf -> 0
+        m_run[tid] = mn;
+      }
+      __syncthreads();
+      for (int h = 0; h < G; ++h) {
+        float sum = 0.0f;
+        for (int t = tid; t < nt; t += blockDim.x) {
+          const float p = exp2f(sp[h][t] - m_run[h]);
+          sp[h][t] = p;
+          sum += p;
+        }
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0) red[warp][h] = sum;
+      }
+      __syncthreads();
+      if (tid < G) {
+        float sum = 0.0f;
+        for (int w = 0; w < kGenThreads / 32; ++w) sum += red[w][tid];
+        l_run[tid] = l_run[tid] * alpha[tid] + sum;
+      }
+    }
+    // ---- values: thread owns channels (tid % D) + 128 c, token subset tid / D
+    {
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          if (h < G) o[h][c] *= alpha[h];
+      const int ch0 = tid % (D < kGenThreads ? D : kGenThreads);
+      const int sub = tid / (D < kGenThreads ? D : kGenThreads);
+      for (int tt = sub; tt < nt; tt += TSUB) {
+        const int t = tb + tt;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          const int j = ch0 + c * kGenThreads;
+          float vv;
+          if (anchor_split) {
+            const __half* vr = V.anchors ? V.anchors + (u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t)) * D
+                                         : reinterpret_cast<const __half*>(V.codes + (u * L.Tcap + t) * V.row_bytes);
+            vv = __half2float(vr[j]);
+          } else {
+            const uint8_t* row = V.codes + (u * L.Tcap + t) * V.row_bytes;
+            const __half* sc = V.scales + (u * L.Tcap + t) * V.n_groups;
+            const __half* zr = V.zeros ? V.zeros + (u * L.Tcap + t) * V.n_groups : nullptr;
+            if (V.fmt == KVQ_FMT_POLAR) {
+              const float2 ab = polar_slot(V, row, sc, j >> 1, vcs, vsn);
+              vv = (j & 1) ? ab.y : ab.x;
+            } else {
+              vv = stored_value(V, row, sc, zr, j, nf4);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h)
+            if (h < G) o[h][c] += sp[h][tt] * vv;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // ---- write partials (combine token subsets through shared memory when TSUB > 1)
+  __shared__ float ored[kMaxG * D];
+  if (TSUB > 1) {
+    for (int e = tid; e < G * D; e += blockDim.x) ored[e] = 0.0f;
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+      if (h < G) atomicAdd(&ored[h * D + (tid % D)], o[h][0]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) {
+    if (h >= G) break;
+    float* P = work + (((long long)qi * L.Hq + kvh * G + h) * nsp + s) * (D + kPartStride);
+    if (tid == 0) {
+      P[0] = m_run[h];
+      P[1] = l_run[h];
+    }
+    if (TSUB > 1) {
+      for (int j = tid; j < D; j += blockDim.x) P[kPartStride + j] = ored[h * D + j];
+    } else {
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) P[kPartStride + tid + c * kGenThreads] = o[h][c];
+    }
+  }
+}
+
+// Pass 2: merge the splits of one (query, head), undo V's transform, add anchors, normalise.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(LayerDev L, const float* __restrict__ work, int n_split, int nsp,
+                                                    void* __restrict__ out, int out_fp32, float* __restrict__ lse) {
+  const int qh = blockIdx.x;  // qi * Hq + h
+  const int tid = threadIdx.x;
+  const SideDev& V = L.s[1];
+  const float* P = work + (long long)qh * nsp * (D + kPartStride);
+  __shared__ float w[kMaxSplit + 1];
+  __shared__ float Msh, Lsh;
+  __shared__ float ov[D], tmp[D];
+  if (tid == 0) {
+    float M = -INFINITY;
+    for (int s = 0; s < nsp; ++s) M = fmaxf(M, P[s * (D + kPartStride)]);
+    float Ls = 0.0f;
+    for (int s = 0; s < nsp; ++s) {
+      const float m = P[s * (D + kPartStride)];
+      const float ws = (m == -INFINITY) ? 0.0f : exp2f(m - M);
+      w[s] = ws;
+      Ls += ws * P[s * (D + kPartStride) + 1];
+    }
+    Msh = M;
+    Lsh = Ls;
+  }
+  __syncthreads();
+  for (int j = tid; j < D; j += blockDim.x) {
+    float acc = 0.0f;
+    for (int s = 0; s < n_split; ++s) acc += w[s] * P[s * (D + kPartStride) + kPartStride + j];
+    ov[j] = acc;
+  }
+  __syncthreads();
+  if (V.rot == 128 || V.rot == 256) {
+    const int n = V.rot;
+    for (int h = 1; h < n; h <<= 1) {
+      for (int p = tid; p < D / 2; p += blockDim.x) {
+        const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
+        const int i = (hi << __ffs(h)) | lo;
+        const float a = ov[i], b = ov[i + h];
+        ov[i] = a + b;
+        ov[i + h] = a - b;
+      }
+      __syncthreads();
+    }
+    const float rn = (n == 256) ? 0.0625f : 0.08838834764831845f;
+    for (int j = tid; j < D; j += blockDim.x) ov[j] *= rn;
+    __syncthreads();
+  } else if (V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART) {
+    // x_n = (1/N) [a_0 + b_0 (-1)^n + 2 sum_{f=1}^{63} (a_f cos(2 pi f n/N) - b_f sin(2 pi f n/N))]
+    for (int j = tid; j < D; j += blockDim.x) tmp[j] = ov[j];
+    __syncthreads();
+    for (int n = tid; n < 128; n += blockDim.x) {
+      float acc = tmp[0] + ((n & 1) ? -tmp[1] : tmp[1]);
+      float sacc = 0.0f;
+      for (int f = 1; f < 64; ++f) {
+        const int k = (f * n) & 127;
+        const float c = k < 64 ? d_tw_re[k] : -d_tw_re[k - 64];
+        const float sn = k < 64 ? -d_tw_im[k] : d_tw_im[k - 64];  // sin(2 pi k / N)
+        sacc += tmp[2 * f] * c - tmp[2 * f + 1] * sn;
+      }
+      ov[n] = (acc + 2.0f * sacc) / 128.0f;
+    }
+    __syncthreads();
+  }
+  const float Ls = Lsh;
+  const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
+  for (int j = tid; j < D; j += blockDim.x) {
+    float v = ov[j];
+    if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + j];
+    v *= inv;
+    if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + j] = v;
+    else reinterpret_cast<__half*>(out)[(long long)qh * D + j] = __float2half_rn(v);
+  }
+  if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (Msh + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+}
+
+// Split count: aim at ~4 CTAs per SM over the grid; each split keeps at least two tiles of keys.
+int decode_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
+  const long long units = (long long)n_q * Hkv;
+  long long s = (4LL * num_sms + units - 1) / units;
+  const long long max_by_len = (Tcap + 2 * kGenTile - 1) / (2 * kGenTile);
+  if (s > max_by_len) s = max_by_len;
+  if (s < 1) s = 1;
+  if (s > kMaxSplit) s = kMaxSplit;
+  return (int)s;
+}
+
+// Workspace floats for n_q queries with n_split splits (+1 anchor split).
+int decode_work_floats(int Hq, int D, int n_q, int n_split) {
+  return n_q * Hq * (n_split + 1) * (D + kPartStride);
+}
+
+template <int D>
+static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, const int* seq_ids, const int* kv_len,
+                                   void* out, int out_fp32, float* lse, float* work, int num_sms, cudaStream_t st,
+                                   int* launches) {
+  const int n_split = decode_split_count(L.Hkv, L.Tcap, n_q, num_sms);
+  const int nsp = n_split + (L.anchored ? 1 : 0);
+  dim3 grid(nsp, L.Hkv, n_q);
+  decode_generic_kernel<D><<<grid, kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  merge_kernel<D><<<n_q * L.Hq, 128, 0, st>>>(L, work, n_split, nsp, out, out_fp32, lse);
+  if (launches) *launches = 2;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int* seq_ids, const int* kv_len, void* out,
+                          int out_fp32, float* lse, float* work, int num_sms, int /*max_queries*/, cudaStream_t st,
+                          int* launches) {
+  switch (L.D) {
+    case 64: return launch_decode_d<64>(L, q, n_q, seq_ids, kv_len, out, out_fp32, lse, work, num_sms, st, launches);
+    case 128: return launch_decode_d<128>(L, q, n_q, seq_ids, kv_len, out, out_fp32, lse, work, num_sms, st, launches);
+    case 256: return launch_decode_d<256>(L, q, n_q, seq_ids, kv_len, out, out_fp32, lse, work, num_sms, st, launches);
+  }
+  return cudaErrorInvalidValue;
+}
+
+
+}  // namespace kvq

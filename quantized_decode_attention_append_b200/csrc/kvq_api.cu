@@ -1,0 +1,474 @@
+// C ABI of libkvq: configuration checks, arena layout, handle lifetime, launch wrappers.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <new>
+#include <set>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+int decode_split_count(int Hkv, int Tcap, int n_q, int num_sms);
+int decode_work_floats(int Hq, int D, int n_q, int n_split_max);
+}  // namespace kvq
+
+using namespace kvq;
+
+struct kvq_cache {
+  kvq_config cfg;
+  int Tcap;
+  char* arena;
+  uint64_t arena_bytes;
+  struct SideOff {
+    int64_t codes, scales, zeros, anchors;
+    int row_bytes, n_groups;
+  } off[64][2];
+  int64_t chan[64];
+  int64_t lens, tickets, err;
+  int anchor_rows;
+  int max_len[64];
+  bool chan_set[64];
+  float* work;
+  size_t work_floats;
+  int device, num_sms;
+  int last_launches;
+};
+
+namespace {
+
+constexpr uint64_t kAlign = 256;
+
+uint64_t align_up(uint64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool is_pow2_group(int g) { return g == 4 || g == 8 || g == 16 || g == 32 || g == 64 || g == 128; }
+
+kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
+  const int D = c.head_dim;
+  if (!is_k && s.chan_scale) return KVQ_ERR_INVALID_ARG;
+  if (s.chan_scale != 0 && s.chan_scale != 1) return KVQ_ERR_INVALID_ARG;
+  if (s.rotation != KVQ_ROT_NONE && s.rotation != KVQ_ROT_H128 && s.rotation != KVQ_ROT_H256)
+    return KVQ_ERR_INVALID_ARG;
+  if (s.rotation > D) return KVQ_ERR_INVALID_ARG;
+  switch (s.format) {
+    case KVQ_FMT_FP16:
+      if (s.rotation != KVQ_ROT_NONE || s.chan_scale) return KVQ_ERR_INVALID_ARG;
+      return KVQ_OK;
+    case KVQ_FMT_INT:
+      if (s.bits < 2 || s.bits > 8) return KVQ_ERR_INVALID_ARG;
+      if (s.scale_mode != KVQ_SCALE_ABSMAX && s.scale_mode != KVQ_SCALE_MINMAX) return KVQ_ERR_INVALID_ARG;
+      break;
+    case KVQ_FMT_NF4:
+    case KVQ_FMT_TERNARY:
+    case KVQ_FMT_SIGN:
+      if (s.scale_mode != KVQ_SCALE_ABSMAX) return KVQ_ERR_INVALID_ARG;
+      break;
+    case KVQ_FMT_POLAR:
+      if (s.bits < 1 || s.bits > 8 || s.bits2 < 1 || s.bits2 > 8) return KVQ_ERR_INVALID_ARG;
+      if (s.scale_mode != KVQ_SCALE_ABSMAX || s.rotation != KVQ_ROT_NONE) return KVQ_ERR_INVALID_ARG;
+      if (D != 128) return KVQ_ERR_UNSUPPORTED;
+      return KVQ_OK;
+    case KVQ_FMT_CART:
+      if (s.bits < 2 || s.bits > 8) return KVQ_ERR_INVALID_ARG;
+      if (s.scale_mode != KVQ_SCALE_ABSMAX || s.rotation != KVQ_ROT_NONE) return KVQ_ERR_INVALID_ARG;
+      if (D != 128) return KVQ_ERR_UNSUPPORTED;
+      return KVQ_OK;
+    default:
+      return KVQ_ERR_INVALID_ARG;
+  }
+  if (!is_pow2_group(s.group) || s.group > D) return KVQ_ERR_INVALID_ARG;
+  if (!append_supported(D, s)) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+kvq_status check_config(const kvq_config* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  if (c->n_layers < 1 || c->n_layers > 64) return KVQ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return KVQ_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads) return KVQ_ERR_INVALID_ARG;
+  if (c->n_q_heads / c->n_kv_heads > 8) return KVQ_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return KVQ_ERR_UNSUPPORTED;
+  if (c->capacity < 1 || c->capacity > (1 << 26)) return KVQ_ERR_INVALID_ARG;
+  if (c->max_queries < 1) return KVQ_ERR_INVALID_ARG;
+  if (!(c->sm_scale >= 0.0f) || isinf(c->sm_scale)) return KVQ_ERR_INVALID_ARG;
+  kvq_status st = check_side(*c, c->k, true);
+  if (st != KVQ_OK) return st;
+  st = check_side(*c, c->v, false);
+  if (st != KVQ_OK) return st;
+  if (c->anchor_rule < KVQ_ANCHOR_NONE || c->anchor_rule > KVQ_ANCHOR_ALL) return KVQ_ERR_INVALID_ARG;
+  if (c->n_layers < 64 && (c->anchor_layer_mask >> c->n_layers)) return KVQ_ERR_INVALID_ARG;
+  if (c->anchor_rule == KVQ_ANCHOR_FIRST_N || c->anchor_rule == KVQ_ANCHOR_WINDOW) {
+    if (c->anchor_n < 1 || c->anchor_n > c->capacity) return KVQ_ERR_INVALID_ARG;
+  }
+  return KVQ_OK;
+}
+
+void side_geometry(int D, const kvq_side& s, int* row_bytes, int* n_groups) {
+  switch (s.format) {
+    case KVQ_FMT_FP16: *row_bytes = 2 * D; *n_groups = 0; return;
+    case KVQ_FMT_INT: *row_bytes = D * s.bits / 8; *n_groups = D / s.group; return;
+    case KVQ_FMT_NF4: *row_bytes = D / 2; *n_groups = D / s.group; return;
+    case KVQ_FMT_TERNARY: *row_bytes = (D + 4) / 5; *n_groups = D / s.group; return;
+    case KVQ_FMT_SIGN: *row_bytes = D / 8; *n_groups = D / s.group; return;
+    case KVQ_FMT_POLAR: *row_bytes = (D / 2) * (s.bits + s.bits2) / 8; *n_groups = 1; return;
+    case KVQ_FMT_CART: *row_bytes = D * s.bits / 8; *n_groups = 1; return;
+  }
+  *row_bytes = 0;
+  *n_groups = 0;
+}
+
+bool layer_anchored(const kvq_config& c, int l) {
+  return c.anchor_rule != KVQ_ANCHOR_NONE && ((c.anchor_layer_mask >> l) & 1ULL);
+}
+
+// Lay out the arena; fills `h` offsets if non-null.  Returns total bytes.
+uint64_t layout(const kvq_config& c, kvq_cache* h) {
+  const int D = c.head_dim;
+  const int Tcap = (c.capacity + 127) / 128 * 128;
+  const uint64_t units = (uint64_t)c.batch * c.n_kv_heads;
+  const int anchor_rows = c.anchor_rule == KVQ_ANCHOR_ALL ? Tcap : c.anchor_n;
+  uint64_t off = 0;
+  for (int l = 0; l < c.n_layers; ++l) {
+    for (int s = 0; s < 2; ++s) {
+      const kvq_side& sd = s == 0 ? c.k : c.v;
+      int rb, ng;
+      side_geometry(D, sd, &rb, &ng);
+      kvq_cache::SideOff so{};
+      so.row_bytes = rb;
+      so.n_groups = ng;
+      so.codes = (int64_t)off;
+      off = align_up(off + units * Tcap * (uint64_t)rb);
+      so.scales = -1;
+      if (ng) {
+        so.scales = (int64_t)off;
+        off = align_up(off + units * Tcap * (uint64_t)ng * 2);
+      }
+      so.zeros = -1;
+      if (sd.format == KVQ_FMT_INT && sd.scale_mode == KVQ_SCALE_MINMAX) {
+        so.zeros = (int64_t)off;
+        off = align_up(off + units * Tcap * (uint64_t)ng * 2);
+      }
+      so.anchors = -1;
+      if (layer_anchored(c, l)) {
+        so.anchors = (int64_t)off;
+        off = align_up(off + units * (uint64_t)anchor_rows * D * 2);
+      }
+      if (h) h->off[l][s] = so;
+    }
+    int64_t ch = -1;
+    if (c.k.chan_scale) {
+      ch = (int64_t)off;
+      off = align_up(off + (uint64_t)c.n_kv_heads * D * 2);
+    }
+    if (h) h->chan[l] = ch;
+  }
+  const int64_t lens = (int64_t)off;
+  off = align_up(off + (uint64_t)c.n_layers * c.batch * 4);
+  const int64_t tickets = (int64_t)off;
+  off = align_up(off + (uint64_t)c.n_layers * 4);
+  const int64_t err = (int64_t)off;
+  off = align_up(off + 4);
+  if (h) {
+    h->Tcap = Tcap;
+    h->anchor_rows = anchor_rows;
+    h->lens = lens;
+    h->tickets = tickets;
+    h->err = err;
+  }
+  return off;
+}
+
+LayerDev layer_dev(const kvq_cache* h, int l) {
+  LayerDev L{};
+  const kvq_config& c = h->cfg;
+  for (int s = 0; s < 2; ++s) {
+    const kvq_side& sd = s == 0 ? c.k : c.v;
+    const kvq_cache::SideOff& so = h->off[l][s];
+    SideDev& S = L.s[s];
+    S.codes = reinterpret_cast<uint8_t*>(h->arena + so.codes);
+    S.scales = so.scales >= 0 ? reinterpret_cast<__half*>(h->arena + so.scales) : nullptr;
+    S.zeros = so.zeros >= 0 ? reinterpret_cast<__half*>(h->arena + so.zeros) : nullptr;
+    S.anchors = so.anchors >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchors) : nullptr;
+    S.chan = (s == 0 && h->chan[l] >= 0) ? reinterpret_cast<const __half*>(h->arena + h->chan[l]) : nullptr;
+    S.fmt = sd.format;
+    S.bits = sd.bits;
+    S.bits2 = sd.bits2;
+    S.scale_mode = sd.scale_mode;
+    S.group = sd.group;
+    S.rot = sd.rotation;
+    S.chan_scale = s == 0 ? sd.chan_scale : 0;
+    S.row_bytes = so.row_bytes;
+    S.n_groups = so.n_groups;
+  }
+  L.B = c.batch;
+  L.Hkv = c.n_kv_heads;
+  L.Hq = c.n_q_heads;
+  L.D = c.head_dim;
+  L.Tcap = h->Tcap;
+  L.anchored = layer_anchored(c, l) ? 1 : 0;
+  L.anchor_rule = c.anchor_rule;
+  L.anchor_n = c.anchor_n;
+  L.anchor_rows = h->anchor_rows;
+  L.seq_len = reinterpret_cast<int*>(h->arena + h->lens) + (size_t)l * c.batch;
+  L.ticket = reinterpret_cast<unsigned*>(h->arena + h->tickets) + l;
+  L.err = reinterpret_cast<unsigned*>(h->arena + h->err);
+  L.sm_scale = c.sm_scale > 0.0f ? c.sm_scale : (float)(1.0 / sqrt((double)c.head_dim));
+  return L;
+}
+
+// ----------------------------------------------------------------------------- host tables
+// Inverse of the standard normal CDF by bisection on Phi(x) = erfc(-x / sqrt 2) / 2.
+double inv_norm_cdf(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int it = 0; it < 400; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    const double ph = 0.5 * erfc(-mid / sqrt(2.0));
+    if (ph < p) lo = mid;
+    else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+HostTables build_tables() {
+  HostTables t{};
+  // NF4 (NormalFloat) construction: 8 quantiles above zero, 7 below, exact 0, ends at +-1.
+  const double delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+  double vals[16];
+  int n = 0;
+  const double step_p = (0.5 - delta) / 8.0, step_n = (0.5 - delta) / 7.0;
+  for (int i = 0; i < 8; ++i) vals[n++] = inv_norm_cdf((double)i * step_p + delta);
+  for (int i = 0; i < 7; ++i) vals[n++] = -inv_norm_cdf((double)i * step_n + delta);
+  vals[n++] = 0.0;
+  double mx = 0.0;
+  for (int i = 0; i < 16; ++i) mx = fabs(vals[i]) > mx ? fabs(vals[i]) : mx;
+  for (int i = 0; i < 16; ++i)
+    for (int j = i + 1; j < 16; ++j)
+      if (vals[j] < vals[i]) {
+        const double tmp = vals[i];
+        vals[i] = vals[j];
+        vals[j] = tmp;
+      }
+  for (int i = 0; i < 16; ++i) t.nf4[i] = __half2float(__double2half(vals[i] / mx));
+  for (int i = 0; i < 15; ++i) t.nf4_mid[i] = 0.5f * (t.nf4[i] + t.nf4[i + 1]);
+  for (int k = 0; k < 64; ++k) {
+    t.tw_re[k] = (float)cos(2.0 * M_PI * k / 128.0);
+    t.tw_im[k] = (float)(-sin(2.0 * M_PI * k / 128.0));
+  }
+  for (int bp = 1; bp <= 8; ++bp) {
+    const int nb = 1 << bp;
+    for (int k = 0; k < nb; ++k) {
+      const double phi = -M_PI + 2.0 * M_PI * k / (double)nb;
+      t.ph_cos[nb - 2 + k] = (float)cos(phi);
+      t.ph_sin[nb - 2 + k] = (float)sin(phi);
+    }
+  }
+  return t;
+}
+
+std::mutex g_mu;
+std::set<int> g_ready_devices;
+
+cudaError_t ensure_tables(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ready_devices.count(dev)) return cudaSuccess;
+  const HostTables& t = host_tables();
+  cudaError_t e = upload_tables_quant(t);
+  if (e == cudaSuccess) e = upload_tables_decode(t);
+  if (e == cudaSuccess) e = upload_tables_dequant(t);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) g_ready_devices.insert(dev);
+  return e;
+}
+
+}  // namespace
+
+namespace kvq {
+const HostTables& host_tables() {
+  static const HostTables t = build_tables();
+  return t;
+}
+}  // namespace kvq
+
+extern "C" {
+
+const char* kvq_status_str(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "capacity exceeded";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_ALLOC: return "allocation failed or arena too small";
+    case KVQ_ERR_STATE: return "invalid call order";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_nf4_levels(float out[16]) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  memcpy(out, host_tables().nf4, sizeof(float) * 16);
+  return KVQ_OK;
+}
+
+kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes) {
+  if (!bytes) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = check_config(cfg);
+  if (st != KVQ_OK) return st;
+  *bytes = layout(*cfg, nullptr);
+  return KVQ_OK;
+}
+
+kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  kvq_status st = check_config(cfg);
+  if (st != KVQ_OK) return st;
+  if (!arena || (reinterpret_cast<uintptr_t>(arena) % kAlign)) return KVQ_ERR_INVALID_ARG;
+  const uint64_t need = layout(*cfg, nullptr);
+  if (arena_bytes < need) return KVQ_ERR_ALLOC;
+  kvq_cache* h = new (std::nothrow) kvq_cache();
+  if (!h) return KVQ_ERR_ALLOC;
+  h->cfg = *cfg;
+  h->arena = reinterpret_cast<char*>(arena);
+  h->arena_bytes = arena_bytes;
+  layout(*cfg, h);
+  for (int l = 0; l < 64; ++l) {
+    h->max_len[l] = 0;
+    h->chan_set[l] = false;
+  }
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    delete h;
+    return KVQ_ERR_CUDA;
+  }
+  if (ensure_tables(h->device) != cudaSuccess) {
+    delete h;
+    return KVQ_ERR_CUDA;
+  }
+  // workspace for the largest split-K grid any n_q <= max_queries can use
+  size_t wf = 0;
+  for (int nq = 1; nq <= cfg->max_queries; ++nq) {
+    const int ns = decode_split_count(cfg->n_kv_heads, h->Tcap, nq, h->num_sms);
+    const size_t f = (size_t)decode_work_floats(cfg->n_q_heads, cfg->head_dim, nq, ns);
+    wf = f > wf ? f : wf;
+  }
+  h->work_floats = wf;
+  if (cudaMalloc(&h->work, wf * sizeof(float)) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return KVQ_ERR_ALLOC;
+  }
+  // zero lengths, tickets and the error word
+  if (cudaMemset(h->arena + h->lens, 0, (size_t)(need - (uint64_t)h->lens)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(h->work);
+    delete h;
+    return KVQ_ERR_CUDA;
+  }
+  *out = h;
+  return KVQ_OK;
+}
+
+void kvq_free(kvq_cache* h) {
+  if (!h) return;
+  if (h->work) cudaFree(h->work);
+  delete h;
+}
+
+kvq_status kvq_get_layout(const kvq_cache* h, int32_t layer, int32_t side, kvq_layout* out) {
+  if (!h || !out || layer < 0 || layer >= h->cfg.n_layers || (side != 0 && side != 1)) return KVQ_ERR_INVALID_ARG;
+  const kvq_cache::SideOff& so = h->off[layer][side];
+  out->codes = so.codes;
+  out->scales = so.scales;
+  out->zeros = so.zeros;
+  out->anchors = so.anchors;
+  out->chan_scale = side == 0 ? h->chan[layer] : -1;
+  out->seq_len = h->lens + (int64_t)layer * h->cfg.batch * 4;
+  out->row_bytes = so.row_bytes;
+  out->n_groups = so.n_groups;
+  out->row_stride_tokens = h->Tcap;
+  out->anchor_rows = so.anchors >= 0 ? h->anchor_rows : 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_chan_scale(kvq_cache* h, int32_t layer, const void* c, void* stream) {
+  if (!h || !c || layer < 0 || layer >= h->cfg.n_layers) return KVQ_ERR_INVALID_ARG;
+  if (h->chan[layer] < 0) return KVQ_ERR_STATE;
+  const size_t bytes = (size_t)h->cfg.n_kv_heads * h->cfg.head_dim * 2;
+  if (cudaMemcpyAsync(h->arena + h->chan[layer], c, bytes, cudaMemcpyDeviceToDevice,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  h->chan_set[layer] = true;
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_seq_len(kvq_cache* h, int32_t layer, int32_t len, void* stream) {
+  if (!h || layer < -1 || layer >= h->cfg.n_layers || len < 0 || len > h->cfg.capacity) return KVQ_ERR_INVALID_ARG;
+  int* lens = reinterpret_cast<int*>(h->arena + h->lens);
+  const int B = h->cfg.batch;
+  cudaError_t e;
+  if (layer < 0) {
+    e = launch_fill_len(lens, B * h->cfg.n_layers, len, reinterpret_cast<cudaStream_t>(stream));
+    for (int l = 0; l < h->cfg.n_layers; ++l) h->max_len[l] = len;
+  } else {
+    e = launch_fill_len(lens + (size_t)layer * B, B, len, reinterpret_cast<cudaStream_t>(stream));
+    h->max_len[layer] = len;
+  }
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const void* v, int32_t n_new,
+                               void* stream) {
+  if (!h || !k || !v || layer < 0 || layer >= h->cfg.n_layers || n_new < 1) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.k.chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
+  if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
+  if ((int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  const LayerDev L = layer_dev(h, layer);
+  int launches = 0;
+  const cudaError_t e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,
+                                      h->max_len[layer], reinterpret_cast<cudaStream_t>(stream), &launches);
+  h->last_launches = launches;
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  h->max_len[layer] += n_new;
+  return KVQ_OK;
+}
+
+kvq_status kvq_dequantize(const kvq_cache* h, int32_t layer, int32_t side, int32_t domain, int32_t t0, int32_t nt,
+                          void* out, int32_t out_fp32, void* stream) {
+  if (!h || !out || layer < 0 || layer >= h->cfg.n_layers || (side != 0 && side != 1)) return KVQ_ERR_INVALID_ARG;
+  if (domain != KVQ_DOMAIN_STORED && domain != KVQ_DOMAIN_ORIGINAL) return KVQ_ERR_INVALID_ARG;
+  if (t0 < 0 || nt < 1 || (int64_t)t0 + nt > h->cfg.capacity) return KVQ_ERR_INVALID_ARG;
+  const LayerDev L = layer_dev(h, layer);
+  const cudaError_t e = launch_dequant(L, side, domain, t0, nt, out, out_fp32 ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_decode_attention(kvq_cache* h, int32_t layer, const void* q, int32_t n_q, const int32_t* seq_ids,
+                                const int32_t* kv_len, void* out, int32_t out_fp32, float* lse, void* stream) {
+  if (!h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || n_q < 1) return KVQ_ERR_INVALID_ARG;
+  if (n_q > h->cfg.max_queries) return KVQ_ERR_CAPACITY;
+  if (!seq_ids && n_q > h->cfg.batch) return KVQ_ERR_INVALID_ARG;
+  const LayerDev L = layer_dev(h, layer);
+  int launches = 0;
+  const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_q, seq_ids, kv_len, out, out_fp32 ? 1 : 0,
+                                      lse, h->work, h->num_sms, h->cfg.max_queries,
+                                      reinterpret_cast<cudaStream_t>(stream), &launches);
+  h->last_launches = launches;
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_error_flags(kvq_cache* h, int32_t* flags) {
+  if (!h || !flags) return KVQ_ERR_INVALID_ARG;
+  unsigned v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaMemcpy(&v, h->arena + h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaMemset(h->arena + h->err, 0, 4) != cudaSuccess) return KVQ_ERR_CUDA;
+  *flags = (int32_t)v;
+  return KVQ_OK;
+}
+
+int32_t kvq_last_launch_count(const kvq_cache* h) { return h ? h->last_launches : 0; }
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Internal definitions shared by the translation units of libkvq (not part of the C ABI).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kMaxSplit = 256;     // split-K partitions per (query, kv-head)
+constexpr int kPartStride = 4;     // floats of (m, l, pad, pad) before o[D] in a partial
+
+// Device view of one (layer, side).
+struct SideDev {
+  uint8_t* codes;        // [B*Hkv][Tcap][row_bytes]
+  __half* scales;        // [B*Hkv][Tcap][n_groups]
+  __half* zeros;         // [B*Hkv][Tcap][n_groups] (MINMAX) or null
+  __half* anchors;       // [B*Hkv][anchor_rows][D] or null
+  const __half* chan;    // [Hkv][D] (K with chan_scale) or null
+  int fmt, bits, bits2, scale_mode, group, rot, chan_scale;
+  int row_bytes, n_groups;
+};
+
+// Device view of one layer.
+struct LayerDev {
+  SideDev s[2];
+  int B, Hkv, Hq, D, Tcap;
+  int anchored;          // this layer keeps anchor rows
+  int anchor_rule, anchor_n, anchor_rows;
+  int* seq_len;          // [B] stored lengths of this layer
+  unsigned* ticket;      // append completion counter of this layer
+  unsigned* err;         // error word (KVQ_ERRF_*)
+  float sm_scale;
+};
+
+// Tables the host builds once (NF4 levels, FFT twiddles, phase cos/sin) and every
+// translation unit uploads into its own constant memory.
+struct HostTables {
+  float nf4[16];
+  float nf4_mid[15];
+  float tw_re[64], tw_im[64];     // W_128^k = exp(-2 pi i k/128), k < 64
+  float ph_cos[512], ph_sin[512]; // phase angle -pi + 2 pi k / 2^bp at offset 2^bp - 2
+};
+
+const HostTables& host_tables();
+
+// Per-TU uploaders (called once per device by kvq_create).
+cudaError_t upload_tables_quant(const HostTables& t);
+cudaError_t upload_tables_decode(const HostTables& t);
+cudaError_t upload_tables_dequant(const HostTables& t);
+
+// Launchers (host side, validate nothing; the API validates first).
+cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new,
+                          int max_len_before, cudaStream_t st, int* launches);
+cudaError_t launch_dequant(const LayerDev& L, int side, int domain, int t0, int nt, void* out,
+                           int out_fp32, cudaStream_t st);
+cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int* seq_ids,
+                          const int* kv_len, void* out, int out_fp32, float* lse, float* work,
+                          int num_sms, int max_queries, cudaStream_t st, int* launches);
+cudaError_t launch_fill_len(int* lens, int n, int value, cudaStream_t st);
+
+// Which append kernels exist for a side (the API reports KVQ_ERR_UNSUPPORTED otherwise).
+bool append_supported(int D, const kvq_side& s);
+
+}  // namespace kvq

@@ -1,0 +1,295 @@
+"""Thin ctypes binding of libkvq (include/kvq.h): same names, argument marshalling only.
+
+Every step of quantize-append, dequantize and decode attention runs in the CUDA library; this
+module only converts Python/torch arguments to plain pointers and sizes.  If libkvq.so is
+missing the import of any call raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass, field
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvq.so")
+
+# enums (values fixed by include/kvq.h)
+FMT = {"fp16": 0, "int": 1, "nf4": 2, "ternary": 3, "sign": 4, "polar": 5, "cart": 6}
+SCALE = {"absmax": 0, "minmax": 1}
+ANCHOR = {"none": 0, "first_n": 1, "window": 2, "all": 3}
+SIDE_K, SIDE_V = 0, 1
+DOMAIN_STORED, DOMAIN_ORIGINAL = 0, 1
+ERRF_CAPACITY = 1
+
+STATUS = {0: "KVQ_OK", -1: "KVQ_ERR_INVALID_ARG", -2: "KVQ_ERR_UNSUPPORTED", -3: "KVQ_ERR_CAPACITY",
+          -4: "KVQ_ERR_CUDA", -5: "KVQ_ERR_ALLOC", -6: "KVQ_ERR_STATE"}
+
+
+class kvq_side(C.Structure):
+    _fields_ = [("format", C.c_int32), ("bits", C.c_int32), ("bits2", C.c_int32), ("scale_mode", C.c_int32),
+                ("group", C.c_int32), ("rotation", C.c_int32), ("chan_scale", C.c_int32)]
+
+
+class kvq_config(C.Structure):
+    _fields_ = [("n_layers", C.c_int32), ("batch", C.c_int32), ("n_kv_heads", C.c_int32), ("n_q_heads", C.c_int32),
+                ("head_dim", C.c_int32), ("capacity", C.c_int32), ("max_queries", C.c_int32),
+                ("k", kvq_side), ("v", kvq_side), ("anchor_layer_mask", C.c_uint64), ("anchor_rule", C.c_int32),
+                ("anchor_n", C.c_int32), ("sm_scale", C.c_float)]
+
+
+class kvq_layout(C.Structure):
+    _fields_ = [("codes", C.c_int64), ("scales", C.c_int64), ("zeros", C.c_int64), ("anchors", C.c_int64),
+                ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("row_bytes", C.c_int32),
+                ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32)]
+
+
+EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
+           "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_error_flags", "kvq_nf4_levels",
+           "kvq_last_launch_count", "kvq_status_str"]
+
+_LIB = None
+
+
+def lib() -> C.CDLL:
+    """Load libkvq.so (built in-tree by quantized_decode_attention_append_b200/build.py)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libkvq.so not built ({LIB_PATH}); run quantized_decode_attention_append_b200/build.py")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, u64p = C.c_void_p, C.c_int32, C.POINTER(C.c_uint64)
+        L.kvq_arena_bytes.argtypes = [C.POINTER(kvq_config), u64p]
+        L.kvq_create.argtypes = [C.POINTER(kvq_config), vp, C.c_uint64, C.POINTER(vp)]
+        L.kvq_free.argtypes = [vp]
+        L.kvq_free.restype = None
+        L.kvq_get_layout.argtypes = [vp, i32, i32, C.POINTER(kvq_layout)]
+        L.kvq_set_chan_scale.argtypes = [vp, i32, vp, vp]
+        L.kvq_set_seq_len.argtypes = [vp, i32, i32, vp]
+        L.kvq_quantize_append.argtypes = [vp, i32, vp, vp, i32, vp]
+        L.kvq_dequantize.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp]
+        L.kvq_decode_attention.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
+        L.kvq_error_flags.argtypes = [vp, C.POINTER(i32)]
+        L.kvq_nf4_levels.argtypes = [C.POINTER(C.c_float)]
+        L.kvq_last_launch_count.argtypes = [vp]
+        L.kvq_last_launch_count.restype = i32
+        L.kvq_status_str.argtypes = [i32]
+        L.kvq_status_str.restype = C.c_char_p
+        for name in EXPORTS:
+            if name not in ("kvq_free", "kvq_last_launch_count", "kvq_status_str"):
+                getattr(L, name).restype = i32
+        _LIB = L
+    return _LIB
+
+
+class KVQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({kvq_status_str(status)})")
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise KVQError(st, what)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+# ----------------------------------------------------------------------------- config
+@dataclass
+class Side:
+    fmt: str = "int"
+    bits: int = 4
+    bits2: int = 0
+    scale: str = "absmax"
+    group: int = 32
+    rot: int = 0
+    chan_scale: bool = False
+
+    def to_c(self) -> kvq_side:
+        return kvq_side(FMT[self.fmt], self.bits, self.bits2, SCALE[self.scale], self.group, self.rot,
+                        1 if self.chan_scale else 0)
+
+
+@dataclass
+class Config:
+    n_layers: int
+    batch: int
+    n_kv_heads: int
+    n_q_heads: int
+    head_dim: int
+    capacity: int
+    k: Side
+    v: Side
+    max_queries: int = 0
+    anchor_layers: tuple = ()
+    anchor_rule: str = "none"
+    anchor_n: int = 0
+    sm_scale: float = 0.0
+
+    def to_c(self) -> kvq_config:
+        mask = 0
+        for l in self.anchor_layers:
+            mask |= 1 << int(l)
+        return kvq_config(self.n_layers, self.batch, self.n_kv_heads, self.n_q_heads, self.head_dim, self.capacity,
+                          self.max_queries or self.batch, self.k.to_c(), self.v.to_c(), mask, ANCHOR[self.anchor_rule],
+                          self.anchor_n, self.sm_scale)
+
+
+# ----------------------------------------------------------------------------- C-ABI calls
+def kvq_status_str(status: int) -> str:
+    return lib().kvq_status_str(status).decode()
+
+
+def kvq_arena_bytes(cfg: Config) -> int:
+    c = cfg.to_c()
+    n = C.c_uint64(0)
+    _check(lib().kvq_arena_bytes(C.byref(c), C.byref(n)), "kvq_arena_bytes")
+    return n.value
+
+
+def kvq_create(cfg: Config, arena) -> C.c_void_p:
+    c = cfg.to_c()
+    h = C.c_void_p()
+    _check(lib().kvq_create(C.byref(c), C.c_void_p(arena.data_ptr()), arena.numel() * arena.element_size(),
+                            C.byref(h)), "kvq_create")
+    return h
+
+
+def kvq_free(h):
+    lib().kvq_free(h)
+
+
+def kvq_get_layout(h, layer: int, side: int) -> kvq_layout:
+    out = kvq_layout()
+    _check(lib().kvq_get_layout(h, layer, side, C.byref(out)), "kvq_get_layout")
+    return out
+
+
+def kvq_set_chan_scale(h, layer: int, c16, stream=None):
+    _check(lib().kvq_set_chan_scale(h, layer, _ptr(c16), _stream(stream)), "kvq_set_chan_scale")
+
+
+def kvq_set_seq_len(h, layer: int, length: int, stream=None):
+    _check(lib().kvq_set_seq_len(h, layer, length, _stream(stream)), "kvq_set_seq_len")
+
+
+def kvq_quantize_append(h, layer: int, k16, v16, n_new: int, stream=None):
+    _check(lib().kvq_quantize_append(h, layer, _ptr(k16), _ptr(v16), n_new, _stream(stream)), "kvq_quantize_append")
+
+
+def kvq_dequantize(h, layer: int, side: int, domain: int, t0: int, nt: int, out, stream=None):
+    import torch
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    _check(lib().kvq_dequantize(h, layer, side, domain, t0, nt, _ptr(out), fp32, _stream(stream)), "kvq_dequantize")
+
+
+def kvq_decode_attention(h, layer: int, q16, n_q: int, seq_ids, kv_len, out, lse=None, stream=None):
+    import torch
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    _check(lib().kvq_decode_attention(h, layer, _ptr(q16), n_q, _ptr(seq_ids), _ptr(kv_len), _ptr(out), fp32,
+                                      _ptr(lse), _stream(stream)), "kvq_decode_attention")
+
+
+def kvq_error_flags(h) -> int:
+    f = C.c_int32(0)
+    _check(lib().kvq_error_flags(h, C.byref(f)), "kvq_error_flags")
+    return f.value
+
+
+def kvq_nf4_levels() -> list:
+    arr = (C.c_float * 16)()
+    _check(lib().kvq_nf4_levels(arr), "kvq_nf4_levels")
+    return list(arr)
+
+
+def kvq_last_launch_count(h) -> int:
+    return lib().kvq_last_launch_count(h)
+
+
+# ----------------------------------------------------------------------------- convenience
+class KVCache:
+    """A cache handle plus its caller-owned device arena (a torch uint8 tensor)."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        import torch
+        self.cfg = cfg
+        nbytes = kvq_arena_bytes(cfg)
+        self.arena = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.arena.data_ptr()) % 256
+        self.arena = self.arena[off:off + nbytes]
+        self.h = kvq_create(cfg, self.arena)
+
+    def close(self):
+        if self.h:
+            kvq_free(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def layout(self, layer, side):
+        return kvq_get_layout(self.h, layer, side)
+
+    def view(self, layer: int, side: int, what: str):
+        """torch views into the arena: codes [B*Hkv, Tcap, row_bytes] uint8, scales/zeros
+        [B*Hkv, Tcap, n_groups] fp16, anchors [B*Hkv, anchor_rows, D] fp16, seq_len [B] int32."""
+        import torch
+        lo = self.layout(layer, side)
+        U = self.cfg.batch * self.cfg.n_kv_heads
+        T = lo.row_stride_tokens
+        if what == "codes":
+            return self.arena[lo.codes:lo.codes + U * T * lo.row_bytes].view(U, T, lo.row_bytes)
+        if what in ("scales", "zeros"):
+            o = lo.scales if what == "scales" else lo.zeros
+            if o < 0:
+                return None
+            n = U * T * lo.n_groups * 2
+            return self.arena[o:o + n].view(torch.float16).view(U, T, lo.n_groups)
+        if what == "anchors":
+            if lo.anchors < 0:
+                return None
+            n = U * lo.anchor_rows * self.cfg.head_dim * 2
+            return self.arena[lo.anchors:lo.anchors + n].view(torch.float16).view(U, lo.anchor_rows, self.cfg.head_dim)
+        if what == "seq_len":
+            return self.arena[lo.seq_len:lo.seq_len + 4 * self.cfg.batch].view(torch.int32)
+        raise ValueError(what)
+
+    def set_chan_scale(self, layer, c16, stream=None):
+        kvq_set_chan_scale(self.h, layer, c16, stream)
+
+    def set_seq_len(self, layer, length, stream=None):
+        kvq_set_seq_len(self.h, layer, length, stream)
+
+    def append(self, layer, k16, v16, stream=None):
+        assert k16.is_contiguous() and v16.is_contiguous() and k16.dtype == v16.dtype
+        kvq_quantize_append(self.h, layer, k16, v16, k16.shape[2], stream)
+
+    def dequantize(self, layer, side, t0, nt, domain=DOMAIN_STORED, fp32=True, stream=None):
+        import torch
+        c = self.cfg
+        out = torch.empty(c.batch, c.n_kv_heads, nt, c.head_dim, device=self.arena.device,
+                          dtype=torch.float32 if fp32 else torch.float16)
+        kvq_dequantize(self.h, layer, side, domain, t0, nt, out, stream)
+        return out
+
+    def decode(self, layer, q16, seq_ids=None, kv_len=None, fp32=True, lse=False, out=None, stream=None):
+        import torch
+        n_q = q16.shape[0]
+        if out is None:
+            out = torch.empty(n_q, self.cfg.n_q_heads, self.cfg.head_dim, device=q16.device,
+                              dtype=torch.float32 if fp32 else torch.float16)
+        l = torch.empty(n_q, self.cfg.n_q_heads, device=q16.device, dtype=torch.float32) if lse else None
+        kvq_decode_attention(self.h, layer, q16, n_q, seq_ids, kv_len, out, l, stream)
+        return (out, l) if lse else out

@@ -1,0 +1,112 @@
+"""The C-ABI library loads, exports every symbol include/kvq.h declares, and rejects bad
+configurations on the host (no GPU needed)."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import nf4 as ORACLE_NF4
+from quantized_decode_attention_append_b200 import kvq
+from quantized_decode_attention_append_b200.kvq import Config, Side
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = kvq.lib()
+    syms = header_symbols()
+    assert len(syms) >= 13
+    for s in syms:
+        assert hasattr(L, s), s
+    assert sorted(kvq.EXPORTS) == syms
+
+
+def base_cfg(**kw):
+    c = Config(n_layers=2, batch=2, n_kv_heads=2, n_q_heads=4, head_dim=128, capacity=512,
+               k=Side("int", 4, group=32, rot=128), v=Side("int", 4, group=32, rot=128))
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def status_of(cfg):
+    c = cfg.to_c()
+    n = C.c_uint64(0)
+    return kvq.lib().kvq_arena_bytes(C.byref(c), C.byref(n)), n.value
+
+
+def test_arena_bytes_matches_layout_arithmetic():
+    st, n = status_of(base_cfg())
+    assert st == 0
+    # per layer and side: codes 2*2*512*64, scales 2*2*512*4*2 (256-aligned), then metadata
+    per_side = 4 * 512 * 64 + 4 * 512 * 4 * 2
+    assert n >= 2 * 2 * per_side and n < 2 * 2 * per_side + 4096
+
+
+@pytest.mark.parametrize("mut,want", [
+    (dict(head_dim=96), -2),
+    (dict(n_q_heads=3), -1),
+    (dict(n_q_heads=2 * 16), -2),
+    (dict(capacity=0), -1),
+    (dict(k=Side("int", 9, group=32)), -1),
+    (dict(k=Side("int", 4, group=48)), -1),
+    (dict(k=Side("int", 4, group=256)), -1),
+    (dict(k=Side("int", 4, group=32, rot=256)), -1),
+    (dict(v=Side("int", 4, group=32, chan_scale=True)), -1),
+    (dict(k=Side("polar", 4, 8, rot=128)), -1),
+    (dict(head_dim=256, k=Side("polar", 4, 8), v=Side("polar", 4, 8)), -2),
+    (dict(head_dim=256, k=Side("ternary", group=8), v=Side("ternary", group=8)), -2),
+    (dict(k=Side("nf4", scale="minmax", group=64)), -1),
+    (dict(anchor_layers=(5,), anchor_rule="first_n", anchor_n=8), -1),
+    (dict(anchor_layers=(0,), anchor_rule="window", anchor_n=0), -1),
+    (dict(sm_scale=-1.0), -1),
+])
+def test_bad_configs_rejected_on_host(mut, want):
+    st, _ = status_of(base_cfg(**mut))
+    assert st == want
+
+
+@pytest.mark.parametrize("side", [
+    Side("int", 2, group=128, rot=128), Side("int", 3, group=32), Side("int", 8, scale="minmax", group=16),
+    Side("nf4", group=64), Side("ternary", group=8), Side("sign", group=4), Side("polar", 5, 7),
+    Side("cart", 6), Side("fp16"),
+])
+def test_good_configs_accepted(side):
+    st, n = status_of(base_cfg(k=side, v=side))
+    assert st == 0 and n > 0
+
+
+def test_create_rejects_before_touching_the_device():
+    L = kvq.lib()
+    c = base_cfg(head_dim=96).to_c()
+    h = C.c_void_p()
+    assert L.kvq_create(C.byref(c), C.c_void_p(256), 1 << 20, C.byref(h)) == -2
+    c = base_cfg().to_c()
+    assert L.kvq_create(C.byref(c), C.c_void_p(0), 1 << 20, C.byref(h)) == -1      # null arena
+    assert L.kvq_create(C.byref(c), C.c_void_p(4096 + 8), 1 << 30, C.byref(h)) == -1  # misaligned
+    assert L.kvq_create(C.byref(c), C.c_void_p(4096), 16, C.byref(h)) == -5         # too small
+    assert L.kvq_create(None, C.c_void_p(4096), 16, C.byref(h)) == -1
+
+
+def test_null_handle_calls_fail_cleanly():
+    L = kvq.lib()
+    assert L.kvq_quantize_append(None, 0, None, None, 1, None) == -1
+    assert L.kvq_decode_attention(None, 0, None, 1, None, None, None, 1, None, None) == -1
+    assert L.kvq_dequantize(None, 0, 0, 0, 0, 1, None, 1, None) == -1
+    assert L.kvq_set_seq_len(None, 0, 0, None) == -1
+    L.kvq_free(None)
+    assert kvq.kvq_status_str(-3) == "capacity exceeded"
+
+
+def test_library_nf4_table_equals_oracle_table():
+    """The two sides build the NF4 table independently (bisection on erfc vs the stdlib
+    inverse CDF); they must agree bit for bit after fp16 rounding."""
+    lib_levels = np.array(kvq.kvq_nf4_levels(), dtype=np.float64)
+    assert np.array_equal(lib_levels, ORACLE_NF4.nf4_levels())

@@ -1,0 +1,155 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on seeded inputs.
+
+Codes, scales and stored-domain dequantization are compared bit for bit; decode attention
+within max relative error 2e-3 per (query, head) vector.  Sizes span several 128-token tiles
+and a ragged tail, so split-K boundaries, partial tiles and the merge are all exercised.
+"""
+import numpy as np
+import pytest
+import torch
+
+from kvq_harness import TOL, Case
+from quantized_decode_attention_append_b200 import synth
+from quantized_decode_attention_append_b200.kvq import Config
+from quantized_decode_attention_append_b200.kvq import KVQError, Side
+
+pytestmark = pytest.mark.gpu
+
+
+def cfg_of(D, k, v, B=2, H=2, Hq=4, L=1, cap=None, T=300, **kw):
+    return Config(n_layers=L, batch=B, n_kv_heads=H, n_q_heads=Hq, head_dim=D, capacity=cap or T, k=k, v=v,
+                  max_queries=max(B, 16), **kw)
+
+
+def queries(cfg, n, pos, seed=1, layer=0):
+    return synth.queries(seed, layer, n, cfg.n_q_heads, cfg.head_dim, pos)
+
+
+# --------------------------------------------------------------------------------- Tiny (full size)
+def test_tiny_config_full():
+    """1 layer, 2 KV heads, 4 query heads, head_dim 128, 512 tokens; Hadamard-128 int4 absmax g32."""
+    s = Side("int", 4, group=32, rot=128)
+    cfg = cfg_of(128, s, s, B=1, H=2, Hq=4, T=512)
+    c = Case(cfg, 512)
+    c.check_codes(0)
+    c.check_dequant(0)
+    c.decode_and_compare(0, queries(cfg, 1, 512))
+
+
+FORMATS = [
+    (128, Side("int", 4, group=32), Side("int", 4, group=32)),
+    (128, Side("int", 2, group=128, rot=128), Side("int", 3, group=64, rot=128)),
+    (128, Side("int", 8, group=16), Side("int", 5, group=8)),
+    (128, Side("nf4", group=64), Side("int", 4, group=64)),
+    (128, Side("ternary", group=8), Side("ternary", group=8)),
+    (128, Side("sign", group=4), Side("sign", group=4)),
+    (128, Side("polar", 4, 8), Side("polar", 8, 4)),
+    (128, Side("polar", 5, 7), Side("polar", 6, 6)),
+    (128, Side("polar", 7, 5), Side("cart", 6)),
+    (128, Side("int", 6, group=128, rot=128), Side("int", 6, group=128, rot=128)),
+    (256, Side("int", 4, group=128, rot=256), Side("int", 2, group=128, rot=256)),
+    (256, Side("int", 4, group=128, rot=256), Side("int", 3, group=128, rot=256)),
+    (256, Side("int", 4, group=128, rot=256), Side("fp16")),
+    (256, Side("int", 4, group=32), Side("int", 4, group=32)),
+    (256, Side("int", 3, scale="minmax", group=32), Side("int", 3, scale="minmax", group=32)),
+    (256, Side("int", 4, scale="minmax", group=32, rot=256), Side("int", 4, scale="minmax", group=32, rot=256)),
+    (256, Side("int", 3, scale="minmax", group=32, chan_scale=True), Side("int", 3, scale="minmax", group=32)),
+    (256, Side("int", 4, scale="minmax", group=32, rot=256, chan_scale=True),
+     Side("int", 4, scale="minmax", group=32, rot=256)),
+    (256, Side("int", 4, group=64, rot=128), Side("nf4", group=32)),
+    (64, Side("int", 4, group=16), Side("sign", group=8)),
+    (64, Side("nf4", group=64), Side("ternary", group=4)),
+]
+
+
+@pytest.mark.parametrize("D,k,v", FORMATS, ids=[f"{d}-{k.fmt}{k.bits}g{k.group}r{k.rot}-{v.fmt}{v.bits}g{v.group}"
+                                                   for d, k, v in FORMATS])
+def test_format_parity(D, k, v):
+    cfg = cfg_of(D, k, v, T=300)
+    c = Case(cfg, 300)
+    c.check_codes(0)
+    c.check_dequant(0)
+    c.decode_and_compare(0, queries(cfg, 2, 300))
+
+
+def test_incremental_append_equals_bulk():
+    s = Side("nf4", group=64)
+    cfg = cfg_of(128, s, Side("int", 4, group=64), T=200)
+    bulk = Case(cfg, 200)
+    inc = Case(cfg, 200, chunks=[1] * 8 + [64, 1, 127])
+    for side in (0, 1):
+        for what in ("codes", "scales"):
+            a = bulk.cache.view(0, side, what)[:, :200].cpu()
+            b = inc.cache.view(0, side, what)[:, :200].cpu()
+            assert torch.equal(a, b)
+    assert inc.cache.view(0, 0, "seq_len").cpu().tolist() == [200, 200]
+    inc.check_codes(0)
+
+
+@pytest.mark.parametrize("rule,n", [("first_n", 48), ("window", 64), ("all", 0)])
+def test_anchor_rules(rule, n):
+    s = Side("ternary", group=8)
+    cfg = cfg_of(128, s, s, L=2, T=300, anchor_layers=(0,), anchor_rule=rule, anchor_n=n)
+    c = Case(cfg, 300)
+    for l in (0, 1):
+        c.check_codes(l)
+        c.check_dequant(l)
+        c.decode_and_compare(l, queries(cfg, 2, 300, layer=l), kv_len=[300, 299])
+
+
+def test_window_anchor_ring_wraps():
+    """A window smaller than the appended run: ring slots are reused as tokens arrive."""
+    s = Side("sign", group=4)
+    cfg = cfg_of(128, s, s, T=260, anchor_layers=(0,), anchor_rule="window", anchor_n=64)
+    c = Case(cfg, 260, chunks=[100, 1, 1, 30, 128])
+    c.check_dequant(0)
+    c.decode_and_compare(0, queries(cfg, 2, 260))
+
+
+def test_decode_ragged_lengths_and_seq_ids():
+    s = Side("int", 4, group=32, rot=128)
+    cfg = cfg_of(128, s, s, B=3, T=400)
+    c = Case(cfg, 400)
+    q = queries(cfg, 6, 400)
+    c.decode_and_compare(0, q, seq_ids=[0, 1, 2, 2, 1, 0], kv_len=[400, 1, 0, 129, 255, 37])
+
+
+def test_proxy_queries_share_a_sequence():
+    """Proxy queries ("E21W"): the post-RoPE key at position p as the query, causal over t < p."""
+    s = Side("int", 4, scale="minmax", group=32, rot=256)
+    cfg = Config(n_layers=1, batch=1, n_kv_heads=4, n_q_heads=4, head_dim=256, capacity=600, k=s, v=s,
+                 max_queries=16)
+    c = Case(cfg, 600)
+    pos = synth.proxy_positions(1, 16, 300, 600)
+    q = torch.from_numpy(c.K[0][0][:, pos].transpose(1, 0, 2).copy())  # [16, Hq=Hkv, D]
+    c.decode_and_compare(0, q, seq_ids=[0] * 16, kv_len=pos.tolist())
+
+
+def test_capacity_error_and_flags():
+    s = Side("int", 4, group=32)
+    cfg = cfg_of(128, s, s, T=100, cap=128)
+    c = Case(cfg, 100)
+    k = torch.zeros(2, 2, 29, 128, dtype=torch.float16, device="cuda")
+    with pytest.raises(KVQError) as e:
+        c.cache.append(0, k, k)
+    assert e.value.status == -3
+    assert c.cache.view(0, 0, "seq_len").cpu().tolist() == [100, 100]
+    from quantized_decode_attention_append_b200 import kvq
+    assert kvq.kvq_error_flags(c.cache.h) == 0
+
+
+def test_sm_scale_override():
+    s = Side("int", 8, group=32)
+    cfg = cfg_of(128, s, s, T=160, sm_scale=0.05)
+    c = Case(cfg, 160)
+    c.decode_and_compare(0, queries(cfg, 2, 160))
+
+
+def test_fp16_output_path():
+    s = Side("int", 4, group=32, rot=128)
+    cfg = cfg_of(128, s, s, T=256)
+    c = Case(cfg, 256)
+    q = queries(cfg, 2, 256).cuda()
+    o32 = c.cache.decode(0, q)
+    o16 = c.cache.decode(0, q, fp32=False)
+    assert torch.allclose(o16.float(), o32, rtol=1e-3, atol=1e-3)
