@@ -1,0 +1,375 @@
+"""Benchmark: quantized KV-cache decode steps/s on one B200 (replicas on N GPUs).
+
+Default workload (the throughput-stress configuration): 32 layers x 8 KV heads x 32 query
+heads, head_dim 128, batch 16 x 32768 tokens, NF4 K (group 64) + int4 V (group 64), 4.25 bits
+per value.  One step = append one new token per sequence to all 32 layers
+(kvq_quantize_append) and decode attention on all 32 layers (kvq_decode_attention).
+Other workloads: --workload names one of WORKLOADS below.
+
+Timing: W warm-up steps, then K steps between CUDA events on the launching stream, with a
+barrier and synchronize on both sides; the max over ranks is reported.  The per-layer KV
+working set (570 MB for the default) exceeds L2 (126 MB), so no flush is needed.  CUDA
+events around every decode call give the dominant kernel's duration for the roofline.
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (L, Hkv, Hq, D, B, T, k side, v side, anchors)
+    "stress-nf4": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
+                       k=dict(fmt="nf4", group=64), v=dict(fmt="int", bits=4, group=64),
+                       desc="32L x 8kv x 32q, hd128, B16 x 32768 tokens; NF4-K g64 + int4-g64 V (4.25 b)"),
+    "stress-ternary": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
+                           k=dict(fmt="ternary", group=8), v=dict(fmt="ternary", group=8),
+                           anchors=dict(layers=(0,), rule="first_n", n=48),
+                           desc="32L x 8kv x 32q, hd128, B16 x 32768; ternary g8, fp16 anchors layer 0, t < 48"),
+    "stress-sign": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
+                        k=dict(fmt="sign", group=4), v=dict(fmt="sign", group=4),
+                        desc="32L x 8kv x 32q, hd128, B16 x 32768; sign g4"),
+    "64k-A": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
+                  k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="int", bits=2, group=128, rot=256),
+                  desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K + H256 2-bit V, g128 (3.125 b)"),
+    "64k-konly": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
+                      k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="fp16"),
+                      desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K g128, fp16 V"),
+    "64k-v3": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
+                   k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="int", bits=3, group=128, rot=256),
+                   desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K + H256 3-bit V, g128 (3.625 b)"),
+}
+DEFAULT_WORKLOAD = "stress-nf4"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_PEAKS["hbm_gbs"], "fallback"
+
+
+def make_config(w, T_cap):
+    from quantized_decode_attention_append_b200.kvq import Config, Side
+    an = w.get("anchors")
+    return Config(n_layers=w["L"], batch=w["B"], n_kv_heads=w["Hkv"], n_q_heads=w["Hq"], head_dim=w["D"],
+                  capacity=T_cap, k=Side(**w["k"]), v=Side(**w["v"]), max_queries=w["B"],
+                  anchor_layers=an["layers"] if an else (), anchor_rule=an["rule"] if an else "none",
+                  anchor_n=an["n"] if an else 0)
+
+
+def row_bytes_of(cache, side):
+    """Stored bytes of one row of `side` (codes + fp16 scales + fp16 zero points), from the
+    library's own layout."""
+    lo = cache.layout(0, side)
+    return lo.row_bytes + 2 * lo.n_groups * (2 if lo.zeros >= 0 else 1)
+
+
+def decode_bytes(cache, w, kv_len, anchored_rows_per_unit):
+    """Algorithmic bytes of one decode call: packed K/V rows + scales for t < kv_len (fp16
+    rows for anchored tokens), the queries and the fp32 outputs."""
+    D, units = w["D"], w["B"] * w["Hkv"]
+    per_tok = row_bytes_of(cache, 0) + row_bytes_of(cache, 1)
+    a = anchored_rows_per_unit
+    kv = units * ((kv_len - a) * per_tok + a * 4 * D)
+    return kv + w["B"] * w["Hq"] * D * (2 + 4)
+
+
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/kvq_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def traffic_record(workload):
+    """dram bytes per decode launch from a committed ncu summary, if it matches this source."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    src = open(os.path.join(ROOT, "quantized_decode_attention_append_b200", "csrc", "decode.cu"), "rb").read()
+    if rec.get("decode_cu_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    return rec.get("per_launch_bytes", {}).get(workload)
+
+
+# ----------------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, budget_s=15.0, seed=0):
+    """Time the oracle, as it stands, on whole (layer, sequence, kv-head) units of one decode
+    step: quantize the unit's T rows (the appended token included), reconstruct them, attend with
+    the unit's query heads.  Input generation is outside the timed region.  Returns (seconds per
+    unit, units timed)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import cache as OC
+    from oracle import quant as OQ
+    from quantized_decode_attention_append_b200 import synth
+    D, T, G = w["D"], w["T"], w["Hq"] // w["Hkv"]
+    an = w.get("anchors")
+    spec = OC.Spec(w["L"], w["B"], w["Hkv"], w["Hq"], D, OQ.Side(**w["k"]), OQ.Side(**w["v"]),
+                   frozenset(an["layers"]) if an else frozenset(), an["rule"] if an else "none", an["n"] if an else 0)
+    done, spent = 0, 0.0
+    with threadpool_limits(1):
+        while spent < budget_s and done < 32:
+            layer, b, h = done % w["L"], (done // w["L"]) % w["B"], done % w["Hkv"]
+            K16 = synth.kv_rows(seed, "k", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
+            V16 = synth.kv_rows(seed, "v", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
+            q = synth.queries(1, layer, 1, G, D, T)[0].numpy()
+            t0 = time.perf_counter()
+            kq, vq = OC.quantize_unit(spec, K16, V16)
+            Kh, Vh = OC.reconstruct_unit(spec, layer, K16, V16, kq, vq, T)
+            OC.decode_query(spec, layer, q, Kh[None], Vh[None], T)
+            spent += time.perf_counter() - t0
+            done += 1
+    return spent / done, done
+
+
+def run_reference(args, w, name):
+    per_unit, n = oracle_sample(w, budget_s=args.ref_budget)
+    units_per_step = w["L"] * w["B"] * w["Hkv"]
+    sps = 1.0 / (per_unit * units_per_step)
+    rec = {"impl": "reference", "metric": "decode steps/s", "value": sps, "unit": "steps/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / sps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": f"{name}: {w['desc']}"},
+           "cpu_baseline": {"value": sps, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                            "sample": f"{n} (layer, seq, kv-head) units of one step (quantize + reconstruct "
+                                      f"{w['T']} rows, attend {w['Hq'] // w['Hkv']} heads), scaled by {units_per_step} "
+                                      f"units/step"},
+           "e2e": {"value": sps, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(rec), flush=True)
+
+
+# ----------------------------------------------------------------------------------- GPU arm
+def fill_cache(cache, w, T0, seed, device):
+    import torch
+    from quantized_decode_attention_append_b200 import synth
+    B, H, D = w["B"], w["Hkv"], w["D"]
+    chunk = max(1, min(T0, (1 << 28) // (B * H * D)))
+    for l in range(w["L"]):
+        t = 0
+        while t < T0:
+            n = min(chunk, T0 - t)
+            toks = list(range(t, t + n))
+            K = synth.kv_rows(seed, "k", l, list(range(B)), list(range(H)), toks, D, device)
+            V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), toks, D, device)
+            cache.append(l, K, V)
+            t += n
+            del K, V
+    torch.cuda.synchronize()
+
+
+def run_gpu(args, w, name):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_decode_attention_append_b200 import kvq, synth
+    from quantized_decode_attention_append_b200.kvq import KVCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    L, B, Hkv, Hq, D, T = w["L"], w["B"], w["Hkv"], w["Hq"], w["D"], w["T"]
+    K_, W_ = args.steps, args.warmup
+    T0 = T - K_ - W_
+    cfg = make_config(w, T)
+    cache = KVCache(cfg, dev)
+    fill_cache(cache, w, T0, seed=rank, device=dev)
+    # per-step inputs resident in HBM: one new K/V row per sequence and layer, queries per layer
+    steps_total = K_ + W_
+    knew = [synth.kv_rows(rank, "k", l, list(range(B)), list(range(Hkv)), [T0], D, dev) for l in range(L)]
+    vnew = [synth.kv_rows(rank, "v", l, list(range(B)), list(range(Hkv)), [T0], D, dev) for l in range(L)]
+    qs = [synth.queries(1, l, B, Hq, D, T0).to(dev) for l in range(L)]
+    outs = [torch.empty(B, Hq, D, device=dev, dtype=torch.float32) for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+    launches = {"n": 0}
+
+    def step(dec_events=None):
+        for l in range(L):
+            cache.append(l, knew[l], vnew[l])
+            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+            if dec_events is not None:
+                dec_events[l][0].record(stream)
+            cache.decode(l, qs[l], out=outs[l])
+            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+            if dec_events is not None:
+                dec_events[l][1].record(stream)
+
+    for _ in range(W_):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches["n"] = 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+          for _ in range(K_)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(K_):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = [ev[i][l][0].elapsed_time(ev[i][l][1]) for i in range(K_) for l in range(L)]
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        dist.barrier()
+    flags = kvq.kvq_error_flags(cache.h)
+    ms_step = ms / K_
+    # algorithmic bytes per decode call at the mean kv_len of the timed steps
+    an = w.get("anchors")
+    anchored = an["n"] if an and an["rule"] == "first_n" else 0
+    mean_len = T0 + W_ + (K_ + 1) / 2.0
+    dec_bytes_layer0 = decode_bytes(cache, w, mean_len, anchored)
+    dec_bytes_other = decode_bytes(cache, w, mean_len, 0)
+    dec_bytes_step = dec_bytes_layer0 + (L - 1) * dec_bytes_other if an else L * dec_bytes_other
+    dec_launch_ms = sum(dec_ms) / len(dec_ms)
+    achieved = (dec_bytes_step / L) / (dec_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    append_bytes_step = L * B * Hkv * (2 * 2 * D + row_bytes_of(cache, 0) + row_bytes_of(cache, 1))
+
+    # end to end through the public API with host buffers: H2D of the step's new rows and
+    # queries from pinned memory, D2H of the step's attention outputs
+    h_k = [x.cpu().pin_memory() for x in knew]
+    h_v = [x.cpu().pin_memory() for x in vnew]
+    h_q = [x.cpu().pin_memory() for x in qs]
+    h_o = [torch.empty(B, Hq, D, dtype=torch.float32).pin_memory() for _ in range(L)]
+    d_k = [torch.empty_like(x) for x in knew]
+    d_v = [torch.empty_like(x) for x in vnew]
+    d_q = [torch.empty_like(x) for x in qs]
+    cache.set_seq_len(-1, T0 + W_)
+    E = max(1, min(K_, 10))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        for l in range(L):
+            d_k[l].copy_(h_k[l], non_blocking=True)
+            d_v[l].copy_(h_v[l], non_blocking=True)
+            d_q[l].copy_(h_q[l], non_blocking=True)
+            cache.append(l, d_k[l], d_v[l])
+            cache.decode(l, d_q[l], out=outs[l])
+            h_o[l].copy_(outs[l], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(x.numel() * x.element_size() for x in h_k + h_v + h_q)
+    d2h = sum(x.numel() * x.element_size() for x in h_o)
+
+    rec = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            per_unit, n = oracle_sample(w, budget_s=args.ref_budget)
+            units_per_step = L * B * Hkv
+            cpu = {"value": 1.0 / (per_unit * units_per_step), "unit": "steps/s", "cores": 1, "kind": "oracle",
+                   "sample": f"{n} (layer, seq, kv-head) units of one step (quantize + reconstruct {T} rows, "
+                             f"attend {Hq // Hkv} heads), scaled by {units_per_step} units/step"}
+        rec = {"metric": "decode steps/s", "value": world * 1e3 / ms_step, "unit": "steps/s", "n_gpus": world,
+               "steps": K_, "warmup": W_, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+               "config": {"workload": f"{name}: {w['desc']}", "global_batch": world * B, "seq_len": T,
+                          "parallelism": f"replicas{world}", "l2": "per-layer KV working set exceeds L2; no flush"},
+               "kv_gbps": dec_bytes_step / (ms_step * 1e-3) / 1e9 * world,
+               "decode_ms_per_layer": dec_launch_ms,
+               "append_us_per_step": None,
+               "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                            "frac": achieved / peak, "traffic": traffic_record(name),
+                            "kernel": "kvq_decode_attention (split-K pass + merge)",
+                            "peak_kind": f"{peak_kind} hbm_gbs (burst copy)",
+                            "bytes_per_launch": dec_bytes_step / L},
+               "cpu_baseline": cpu,
+               "e2e": {"value": world * 1e3 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h},
+               "gpu_launches": launches["n"],
+               "clocks": clk, "error_flags": flags,
+               "append_bytes_per_step": append_bytes_step}
+        print(json.dumps(rec), flush=True)
+    cache.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return rec
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of CPU oracle work to sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args, w, args.workload)
+        return
+    run_gpu(args, w, args.workload)
+
+
+if __name__ == "__main__":
+    main()
