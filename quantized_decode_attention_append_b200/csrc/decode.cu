@@ -148,16 +148,18 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
   __syncthreads();
 }
 
+#include "decode_mma.cuh"
+
 // Generic pass 1: any format, any GQA group (<= 8), CUDA cores.  Thread-per-token scoring,
 // thread-per-channel value accumulation.
 template <int D>
 __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L, const __half* __restrict__ q,
                                                                      const int* __restrict__ seq_ids,
                                                                      const int* __restrict__ kv_len, float* __restrict__ work,
-                                                                     int n_split, int nsp) {
+                                                                     int n_split, int nsp, int split_base) {
   constexpr int NCH = D > kGenThreads ? D / kGenThreads : 1;     // channels per thread
   constexpr int TSUB = D < kGenThreads ? kGenThreads / D : 1;    // token subsets in PV
-  const int s = blockIdx.x, kvh = blockIdx.y, qi = blockIdx.z;
+  const int s = blockIdx.x + split_base, kvh = blockIdx.y, qi = blockIdx.z;
   const int G = L.Hq / L.Hkv;
   const int tid = threadIdx.x;
   __shared__ float qs[kMaxG * D], qa[kMaxG * D];
@@ -349,40 +351,51 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
 }
 
 // Pass 2: merge the splits of one (query, head), undo V's transform, add anchors, normalise.
+// One thread per channel; the split weights are computed in parallel first.
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(LayerDev L, const float* __restrict__ work, int n_split, int nsp,
-                                                    void* __restrict__ out, int out_fp32, float* __restrict__ lse) {
+__global__ void __launch_bounds__(D) merge_kernel(LayerDev L, const float* __restrict__ work, int n_split, int nsp,
+                                                  void* __restrict__ out, int out_fp32, float* __restrict__ lse) {
   const int qh = blockIdx.x;  // qi * Hq + h
   const int tid = threadIdx.x;
   const SideDev& V = L.s[1];
   const float* P = work + (long long)qh * nsp * (D + kPartStride);
   __shared__ float w[kMaxSplit + 1];
-  __shared__ float Msh, Lsh;
+  __shared__ float rm[D / 32], rl[D / 32];
   __shared__ float ov[D], tmp[D];
-  if (tid == 0) {
-    float M = -INFINITY;
-    for (int s = 0; s < nsp; ++s) M = fmaxf(M, P[s * (D + kPartStride)]);
-    float Ls = 0.0f;
-    for (int s = 0; s < nsp; ++s) {
-      const float m = P[s * (D + kPartStride)];
-      const float ws = (m == -INFINITY) ? 0.0f : exp2f(m - M);
-      w[s] = ws;
-      Ls += ws * P[s * (D + kPartStride) + 1];
-    }
-    Msh = M;
-    Lsh = Ls;
-  }
+  const int warp = tid >> 5, lane = tid & 31;
+  // max of the partial maxima
+  float M = -INFINITY;
+  for (int s = tid; s < nsp; s += D) M = fmaxf(M, P[s * (D + kPartStride)]);
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) rm[warp] = M;
   __syncthreads();
-  for (int j = tid; j < D; j += blockDim.x) {
+  M = rm[0];
+  for (int i = 1; i < D / 32; ++i) M = fmaxf(M, rm[i]);
+  // weights and the normaliser
+  float ls = 0.0f;
+  for (int s = tid; s < nsp; s += D) {
+    const float m = P[s * (D + kPartStride)];
+    const float ws = (m == -INFINITY) ? 0.0f : exp2f(m - M);
+    w[s] = ws;
+    ls += ws * P[s * (D + kPartStride) + 1];
+  }
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane == 0) rl[warp] = ls;
+  __syncthreads();
+  float Ls = 0.0f;
+  for (int i = 0; i < D / 32; ++i) Ls += rl[i];
+  {
     float acc = 0.0f;
-    for (int s = 0; s < n_split; ++s) acc += w[s] * P[s * (D + kPartStride) + kPartStride + j];
-    ov[j] = acc;
+    const float* pj = P + kPartStride + tid;
+#pragma unroll 8
+    for (int s = 0; s < n_split; ++s) acc += w[s] * pj[s * (D + kPartStride)];
+    ov[tid] = acc;
   }
   __syncthreads();
   if (V.rot == 128 || V.rot == 256) {
     const int n = V.rot;
     for (int h = 1; h < n; h <<= 1) {
-      for (int p = tid; p < D / 2; p += blockDim.x) {
+      for (int p = tid; p < D / 2; p += D) {
         const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
         const int i = (hi << __ffs(h)) | lo;
         const float a = ov[i], b = ov[i + h];
@@ -392,14 +405,15 @@ __global__ void __launch_bounds__(128) merge_kernel(LayerDev L, const float* __r
       __syncthreads();
     }
     const float rn = (n == 256) ? 0.0625f : 0.08838834764831845f;
-    for (int j = tid; j < D; j += blockDim.x) ov[j] *= rn;
+    ov[tid] *= rn;
     __syncthreads();
   } else if (V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART) {
     // x_n = (1/N) [a_0 + b_0 (-1)^n + 2 sum_{f=1}^{63} (a_f cos(2 pi f n/N) - b_f sin(2 pi f n/N))]
-    for (int j = tid; j < D; j += blockDim.x) tmp[j] = ov[j];
+    tmp[tid] = ov[tid];
     __syncthreads();
-    for (int n = tid; n < 128; n += blockDim.x) {
-      float acc = tmp[0] + ((n & 1) ? -tmp[1] : tmp[1]);
+    if (tid < 128) {
+      const int n = tid;
+      const float acc = tmp[0] + ((n & 1) ? -tmp[1] : tmp[1]);
       float sacc = 0.0f;
       for (int f = 1; f < 64; ++f) {
         const int k = (f * n) & 127;
@@ -411,20 +425,20 @@ __global__ void __launch_bounds__(128) merge_kernel(LayerDev L, const float* __r
     }
     __syncthreads();
   }
-  const float Ls = Lsh;
   const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
-  for (int j = tid; j < D; j += blockDim.x) {
-    float v = ov[j];
-    if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + j];
-    v *= inv;
-    if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + j] = v;
-    else reinterpret_cast<__half*>(out)[(long long)qh * D + j] = __float2half_rn(v);
-  }
-  if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (Msh + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  float v = ov[tid];
+  if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + tid];
+  v *= inv;
+  if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + tid] = v;
+  else reinterpret_cast<__half*>(out)[(long long)qh * D + tid] = __float2half_rn(v);
+  if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
 }
 
-// Split count: aim at ~4 CTAs per SM over the grid; each split keeps at least two tiles of keys.
-int decode_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
+// ----------------------------------------------------------------------------------------------
+// Planning and launch.
+
+// Generic path: ~4 CTAs per SM over the grid; each split keeps at least two tiles of keys.
+static int generic_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
   const long long units = (long long)n_q * Hkv;
   long long s = (4LL * num_sms + units - 1) / units;
   const long long max_by_len = (Tcap + 2 * kGenTile - 1) / (2 * kGenTile);
@@ -434,23 +448,127 @@ int decode_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
   return (int)s;
 }
 
-// Workspace floats for n_q queries with n_split splits (+1 anchor split).
-int decode_work_floats(int Hq, int D, int n_q, int n_split) {
-  return n_q * Hq * (n_split + 1) * (D + kPartStride);
+// Tensor-core path: pick the split count whose grid fills whole waves of resident CTAs and whose
+// splits hold whole tiles, preferring fewer splits on ties.
+static int mma_split_count(long long units, int ntiles, int slots) {
+  int best = 1;
+  double best_score = -1.0;
+  for (int n = 1; n <= 64 && n <= ntiles; ++n) {
+    const long long ctas = units * n;
+    const long long waves = (ctas + slots - 1) / slots;
+    const double eff = (double)ctas / (double)(waves * slots);
+    const int per = (ntiles + n - 1) / n;
+    const double bal = (double)ntiles / (double)(per * n);
+    const double score = eff * bal - (per < 4 ? 0.05 : 0.0);
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = n;
+    }
+  }
+  return best;
+}
+
+typedef void (*MmaKernel)(LayerDev, const __half*, const int*, const int*, float*, int, int);
+
+struct MmaPlan {
+  MmaKernel kern;
+  int smem, tile;
+};
+
+template <int D, int G, int KF, int GK, int VF, int GV, int TPW, int ST>
+static MmaPlan mma_plan_of() {
+  using C = MmaCfg<D, KF, GK, VF, GV, TPW, ST>;
+  return MmaPlan{decode_mma_kernel<D, G, KF, GK, VF, GV, TPW, ST>, C::SMEM, C::TILE};
+}
+
+static int code_fmt(const SideDev& S, bool is_v) {
+  if (S.fmt == KVQ_FMT_NF4 && !is_v) return CF_NF4;
+  if (S.fmt == KVQ_FMT_FP16 && is_v) return CF_FP16;
+  if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && (S.bits == 4 || S.bits == 2)) return S.bits;
+  return -1;
+}
+
+// The tensor-core instantiations (others use the generic kernel).
+static bool pick_mma(const LayerDev& L, MmaPlan* out) {
+  const int G = L.Hq / L.Hkv;
+  const int kf = code_fmt(L.s[0], false), vf = code_fmt(L.s[1], true);
+  if (kf < 0 || vf < 0) return false;
+  const int gk = L.s[0].group, gv = vf == CF_FP16 ? 128 : L.s[1].group;
+#define KVQ_MMA(D_, G_, KF_, GK_, VF_, GV_, TPW_, ST_)                                          \
+  if (L.D == D_ && G == G_ && kf == KF_ && gk == GK_ && vf == VF_ && gv == GV_) {                \
+    *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, TPW_, ST_>();                               \
+    return true;                                                                              \
+  }
+  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 64, 3)
+  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 64, 3)
+  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 64, 3)
+  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 64, 3)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 32, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 32, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 16, 4)
+  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 32, 4)
+#undef KVQ_MMA
+  return false;
+}
+
+static int mma_slots(const MmaPlan& p, int num_sms) {
+  static MmaKernel cached_k = nullptr;
+  static int cached_occ = 1;
+  if (cached_k != p.kern) {
+    cudaFuncSetAttribute(p.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+    int occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, p.kern, 128, p.smem) != cudaSuccess || occ < 1) occ = 1;
+    cudaGetLastError();
+    cached_k = p.kern;
+    cached_occ = occ;
+  }
+  return cached_occ * num_sms;
+}
+
+// Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).
+int decode_partials(const LayerDev& L, int n_q, int num_sms) {
+  MmaPlan p;
+  if (pick_mma(L, &p)) {
+    const int ntiles = L.Tcap / p.tile;
+    return mma_split_count((long long)n_q * L.Hkv, ntiles, mma_slots(p, num_sms)) + 1;
+  }
+  return generic_split_count(L.Hkv, L.Tcap, n_q, num_sms) + 1;
 }
 
 template <int D>
 static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, const int* seq_ids, const int* kv_len,
                                    void* out, int out_fp32, float* lse, float* work, int num_sms, cudaStream_t st,
                                    int* launches) {
-  const int n_split = decode_split_count(L.Hkv, L.Tcap, n_q, num_sms);
-  const int nsp = n_split + (L.anchored ? 1 : 0);
-  dim3 grid(nsp, L.Hkv, n_q);
-  decode_generic_kernel<D><<<grid, kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  merge_kernel<D><<<n_q * L.Hq, 128, 0, st>>>(L, work, n_split, nsp, out, out_fp32, lse);
-  if (launches) *launches = 2;
+  int nl = 0;
+  MmaPlan p;
+  int n_quant;  // quantized partials per (query, head)
+  if (pick_mma(L, &p)) {
+    const int slots = mma_slots(p, num_sms);
+    const int n_split = mma_split_count((long long)n_q * L.Hkv, L.Tcap / p.tile, slots);
+    n_quant = n_split;
+    const int nsp = n_quant + (L.anchored ? 1 : 0);
+    p.kern<<<dim3(n_split, L.Hkv, n_q), 128, p.smem, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
+    ++nl;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone
+      decode_generic_kernel<D><<<dim3(1, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp,
+                                                                           n_quant);
+      ++nl;
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  } else {
+    n_quant = generic_split_count(L.Hkv, L.Tcap, n_q, num_sms);
+    const int nsp = n_quant + (L.anchored ? 1 : 0);
+    decode_generic_kernel<D><<<dim3(nsp, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp, 0);
+    ++nl;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int nsp = n_quant + (L.anchored ? 1 : 0);
+  merge_kernel<D><<<n_q * L.Hq, D, 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse);
+  ++nl;
+  if (launches) *launches = nl;
   return cudaGetLastError();
 }
 
@@ -464,6 +582,5 @@ cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int
   }
   return cudaErrorInvalidValue;
 }
-
 
 }  // namespace kvq

@@ -9,11 +9,6 @@
 
 #include "kvq_internal.h"
 
-namespace kvq {
-int decode_split_count(int Hkv, int Tcap, int n_q, int num_sms);
-int decode_work_floats(int Hq, int D, int n_q, int n_split_max);
-}  // namespace kvq
-
 using namespace kvq;
 
 struct kvq_cache {
@@ -125,7 +120,7 @@ bool layer_anchored(const kvq_config& c, int l) {
 // Lay out the arena; fills `h` offsets if non-null.  Returns total bytes.
 uint64_t layout(const kvq_config& c, kvq_cache* h) {
   const int D = c.head_dim;
-  const int Tcap = (c.capacity + 127) / 128 * 128;
+  const int Tcap = (c.capacity + 255) / 256 * 256;  // whole 256-token decode tiles
   const uint64_t units = (uint64_t)c.batch * c.n_kv_heads;
   const int anchor_rows = c.anchor_rule == KVQ_ANCHOR_ALL ? Tcap : c.anchor_n;
   uint64_t off = 0;
@@ -349,10 +344,12 @@ kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, 
   }
   // workspace for the largest split-K grid any n_q <= max_queries can use
   size_t wf = 0;
-  for (int nq = 1; nq <= cfg->max_queries; ++nq) {
-    const int ns = decode_split_count(cfg->n_kv_heads, h->Tcap, nq, h->num_sms);
-    const size_t f = (size_t)decode_work_floats(cfg->n_q_heads, cfg->head_dim, nq, ns);
-    wf = f > wf ? f : wf;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const LayerDev L = layer_dev(h, l);
+    for (int nq = 1; nq <= cfg->max_queries; ++nq) {
+      const size_t f = (size_t)nq * cfg->n_q_heads * decode_partials(L, nq, h->num_sms) * (cfg->head_dim + kPartStride);
+      wf = f > wf ? f : wf;
+    }
   }
   h->work_floats = wf;
   if (cudaMalloc(&h->work, wf * sizeof(float)) != cudaSuccess) {

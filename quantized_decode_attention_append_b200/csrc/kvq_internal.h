@@ -61,6 +61,9 @@ cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int
                           int num_sms, int max_queries, cudaStream_t st, int* launches);
 cudaError_t launch_fill_len(int* lens, int n, int value, cudaStream_t st);
 
+// Split-K partials per (query, head) one decode call on `L` writes (workspace sizing).
+int decode_partials(const LayerDev& L, int n_q, int num_sms);
+
 // Which append kernels exist for a side (the API reports KVQ_ERR_UNSUPPORTED otherwise).
 bool append_supported(int D, const kvq_side& s);
 

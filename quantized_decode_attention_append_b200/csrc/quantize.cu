@@ -540,6 +540,208 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
 }
 
 // ------------------------------------------------------------------------------------------
+// Small appends (decode-time, a few hundred rows): one warp per row, V = D/32 contiguous values per
+// lane, compact loops over runtime format parameters.  The unrolled thread-per-row kernel above is
+// tens of thousands of straight-line instructions; with only a few warps resident its instruction
+// fetch, not its arithmetic, sets the time, so short appends take this path instead.  Every
+// decision is the same exact arithmetic as the row kernel (same helpers, same evaluation order:
+// Hadamard stages in order, sign sums in channel order), so codes are identical.
+constexpr int kSmallWarps = 4;
+
+template <int V>
+__global__ void __launch_bounds__(32 * kSmallWarps) append_small_kernel(LayerDev L, int side,
+                                                                         const __half* __restrict__ src, int n_new,
+                                                                         unsigned total_ctas) {
+  const SideDev& S = L.s[side];
+  constexpr int D = 32 * V;
+  __shared__ uint32_t words[kSmallWarps][D / 4];  // packed row (up to 8 bits per value)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long R = (long long)L.B * L.Hkv * n_new;
+  const long long row = (long long)blockIdx.x * kSmallWarps + warp;
+  bool ok = row < R;
+  int i = 0, u = 0, pos = 0, len_after = 0;
+  if (ok) {
+    i = (int)(row % n_new);
+    u = (int)(row / n_new);
+    const int len0 = L.seq_len[u / L.Hkv];
+    pos = len0 + i;
+    len_after = len0 + n_new;
+    if (pos >= L.Tcap) {
+      if (lane == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
+      ok = false;
+    }
+  }
+  if (ok) {
+    const __half* rp = src + ((long long)u * n_new + i) * D + lane * V;
+    float x[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) x[v] = __half2float(rp[v]);
+    if (in_anchor(L, pos, len_after)) {
+      __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + lane * V;
+#pragma unroll
+      for (int v = 0; v < V; ++v) ap[v] = rp[v];
+    }
+    if (S.chan_scale) {
+      const __half* cp = S.chan + (u % L.Hkv) * D + lane * V;
+#pragma unroll
+      for (int v = 0; v < V; ++v) x[v] = __fdiv_rn(x[v], __half2float(cp[v]));
+    }
+    if (S.rot) {  // stages h = 1 .. n/2 over element index j = lane*V + v
+      for (int h = 1; h < S.rot; h <<= 1) {
+        if (h < V) {
+#pragma unroll
+          for (int v = 0; v < V; ++v)
+            if ((v & h) == 0) {
+              const float a = x[v], b = x[v + h];
+              x[v] = __fadd_rn(a, b);
+              x[v + h] = __fsub_rn(a, b);
+            }
+        } else {
+          const int lm = h / V;
+          const bool upper = (lane & lm) != 0;
+#pragma unroll
+          for (int v = 0; v < V; ++v) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[v], lm);
+            x[v] = upper ? __fsub_rn(o, x[v]) : __fadd_rn(x[v], o);
+          }
+        }
+      }
+      const float rn = S.rot == 256 ? 0.0625f : __fdiv_rn(__fsqrt_rn(2.0f), 16.0f);
+#pragma unroll
+      for (int v = 0; v < V; ++v) x[v] = __fmul_rn(x[v], rn);
+    }
+    // groups: a lane holds ngl groups of epl values; a group spans lpg lanes
+    const int g = S.group;
+    const int epl = g < V ? g : V, ngl = V / epl, lpg = g / epl;
+    const int fam = (S.fmt == KVQ_FMT_INT) ? (S.scale_mode == KVQ_SCALE_MINMAX ? FAM_MINMAX : FAM_ABSMAX)
+                                           : (S.fmt == KVQ_FMT_NF4 ? FAM_NF4 : (S.fmt == KVQ_FMT_TERNARY ? FAM_TERNARY : FAM_SIGN));
+    const int bits = fam == FAM_SIGN ? 1 : (fam == FAM_NF4 ? 4 : S.bits);
+    const long long rix = (long long)u * L.Tcap + pos;
+    for (int w = lane; w < D / 4; w += 32) words[warp][w] = 0u;
+    __syncwarp();
+    uint32_t code[V];
+#pragma unroll
+    for (int gl = 0; gl < V; ++gl) {
+      if (gl >= ngl) break;
+      const int v0 = gl * epl;
+      // per-lane partial statistics over x[v0 .. v0+epl)
+      float m = 0.0f, am = -1.0f, mn = INFINITY, mx = -INFINITY, sum = 0.0f;
+      int mi = 1 << 30;
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        if (v < v0 || v >= v0 + epl) continue;
+        const float a = fabsf(x[v]);
+        if (a > am) { am = a; m = x[v]; mi = lane * V + v; }
+        mn = fminf(mn, x[v]);
+        mx = fmaxf(mx, x[v]);
+      }
+      if (fam == FAM_SIGN) {  // fp32 sum of |x| in channel order across the group's lanes
+        const int base = lane - (lane % lpg);
+        for (int k = 0; k < lpg; ++k) {
+          if (lane == base + k) {
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+              if (v >= v0 && v < v0 + epl) sum = __fadd_rn(sum, fabsf(x[v]));
+          }
+          sum = __shfl_sync(0xffffffffu, sum, base + k);
+        }
+      }
+      for (int o = 1; o < lpg; o <<= 1) {  // reductions inside the group (first index on ties)
+        const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, m, o);
+        const int omi = __shfl_xor_sync(0xffffffffu, mi, o);
+        if (oam > am || (oam == am && omi < mi)) { am = oam; m = om; mi = omi; }
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      __half sh, zh = __float2half_rn(0.0f);
+      float d = 0.0f, z = 0.0f, inv = 0.0f;
+      int half = 0, top = 0;
+      float t[15];
+      if (fam == FAM_ABSMAX) {
+        half = 1 << (bits - 1);
+        sh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
+        d = __half2float(sh);
+        inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+      } else if (fam == FAM_MINMAX) {
+        top = (1 << bits) - 1;
+        zh = __float2half_rn(mn);
+        sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)top));
+        z = __half2float(zh);
+        d = __half2float(sh);
+        inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+      } else if (fam == FAM_SIGN) {
+        sh = __float2half_rn(__fmul_rn(sum, 1.0f / (float)g));
+      } else {
+        sh = __float2half_rn(am);
+        d = __half2float(sh);
+        if (fam == FAM_NF4) {
+#pragma unroll
+          for (int k = 0; k < 15; ++k) t[k] = __fmul_rn(q_nf4_mid[k], d);
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        if (v < v0 || v >= v0 + epl) continue;
+        uint32_t cd;
+        if (fam == FAM_ABSMAX) {
+          float k = 0.0f;
+          if (d != 0.0f) k = fminf(fmaxf(round_exact_absmax(x[v], d, inv), (float)(-half)), (float)(half - 1));
+          cd = (uint32_t)((int)k + half);
+        } else if (fam == FAM_MINMAX) {
+          float k = 0.0f;
+          if (d != 0.0f) k = fminf(fmaxf(round_exact_minmax(x[v], z, d, inv), 0.0f), (float)top);
+          cd = (uint32_t)(int)k;
+        } else if (fam == FAM_NF4) {
+          int cc = 7;
+          if (d != 0.0f) {
+            cc = 0;
+#pragma unroll
+            for (int k = 0; k < 15; ++k) cc += (x[v] >= t[k]) ? 1 : 0;
+          }
+          cd = (uint32_t)cc;
+        } else if (fam == FAM_TERNARY) {
+          const float hh = __fmul_rn(d, 0.5f);
+          cd = d != 0.0f ? ((x[v] >= hh) ? 2u : ((x[v] < -hh) ? 0u : 1u)) : 1u;
+        } else {
+          cd = x[v] >= 0.0f ? 1u : 0u;
+        }
+        code[v] = cd;
+      }
+      // one scale (and zero point) per group, written by the group's first lane
+      if (lane % lpg == 0) {
+        const int gi = (lane * V + v0) / g;
+        S.scales[rix * S.n_groups + gi] = sh;
+        if (fam == FAM_MINMAX) S.zeros[rix * S.n_groups + gi] = zh;
+      }
+    }
+    // pack: LSB-first bit stream (ternary: 5 trits per byte) into shared words, then store
+    if (fam == FAM_TERNARY) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int j = lane * V + v, byte = j / 5, m5 = j % 5;
+        const uint32_t p3 = m5 == 0 ? 1u : m5 == 1 ? 3u : m5 == 2 ? 9u : m5 == 3 ? 27u : 81u;
+        atomicAdd(&words[warp][byte >> 2], (code[v] * p3) << (8 * (byte & 3)));
+      }
+      __syncwarp();
+      uint8_t* op = S.codes + rix * S.row_bytes;
+      for (int b = lane; b < S.row_bytes; b += 32) op[b] = (uint8_t)(words[warp][b >> 2] >> (8 * (b & 3)));
+    } else {
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int bit = (lane * V + v) * bits;
+        const uint64_t f = (uint64_t)code[v] << (bit & 31);
+        atomicOr(&words[warp][bit >> 5], (uint32_t)f);
+        if ((f >> 32) != 0ull) atomicOr(&words[warp][(bit >> 5) + 1], (uint32_t)(f >> 32));
+      }
+      __syncwarp();
+      uint32_t* op = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes);
+      for (int w = lane; w < S.row_bytes / 4; w += 32) op[w] = words[warp][w];
+    }
+  }
+  finish_append(L, n_new, total_ctas);
+}
+
+// ------------------------------------------------------------------------------------------
 // Dispatch.
 typedef void (*RowKernel)(LayerDev, int, const __half*, int, unsigned);
 
@@ -623,6 +825,9 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
   finish_append(L, n_new, total_ctas);
 }
 
+// Appends of at most this many rows (per side) use the warp-per-row kernel.
+constexpr long long kSmallRows = 8192;
+
 struct SidePlan {
   void (*kern)(LayerDev, int, const __half*, int, unsigned);
   unsigned blocks;
@@ -638,6 +843,9 @@ static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
   } else if (S.fmt == KVQ_FMT_POLAR || S.fmt == KVQ_FMT_CART) {
     p.kern = append_fft_kernel;
     p.blocks = (unsigned)((R + kFftWarps - 1) / kFftWarps);
+  } else if (R <= kSmallRows) {
+    p.kern = L.D == 64 ? append_small_kernel<2> : (L.D == 128 ? append_small_kernel<4> : append_small_kernel<8>);
+    p.blocks = (unsigned)((R + kSmallWarps - 1) / kSmallWarps);
   } else {
     int tpr = 1;
     p.kern = pick_row_kernel(L.D, S.group, fam_of(S), &tpr);

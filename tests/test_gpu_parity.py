@@ -72,18 +72,33 @@ def test_format_parity(D, k, v):
     c.decode_and_compare(0, queries(cfg, 2, 300))
 
 
-def test_incremental_append_equals_bulk():
-    s = Side("nf4", group=64)
-    cfg = cfg_of(128, s, Side("int", 4, group=64), T=200)
-    bulk = Case(cfg, 200)
-    inc = Case(cfg, 200, chunks=[1] * 8 + [64, 1, 127])
+BULK = [
+    (128, Side("nf4", group=64), Side("int", 4, group=64)),
+    (128, Side("ternary", group=8), Side("sign", group=4)),
+    (128, Side("int", 4, group=32, rot=128), Side("int", 3, scale="minmax", group=16)),
+    (256, Side("int", 4, group=128, rot=256), Side("int", 2, group=128, rot=256)),
+    (256, Side("int", 3, scale="minmax", group=32, rot=256, chan_scale=True), Side("sign", group=8)),
+    (64, Side("int", 8, group=64), Side("nf4", group=16)),
+]
+
+
+@pytest.mark.parametrize("D,k,v", BULK, ids=[f"{d}-{k.fmt}{k.bits}g{k.group}-{v.fmt}{v.bits}g{v.group}" for d, k, v in BULK])
+def test_bulk_prefill_and_token_appends_agree(D, k, v):
+    """A prefill above the small-append threshold (2 x 2 x 2100 rows) takes the unrolled
+    thread-per-row kernel; token-by-token appends take the warp-per-row kernel.  Both must give
+    the oracle's bytes."""
+    T = 2100
+    cfg = cfg_of(D, k, v, T=T)
+    bulk = Case(cfg, T)
+    inc = Case(cfg, T, chunks=[1] * 9 + [500, 1, 1590])
     for side in (0, 1):
-        for what in ("codes", "scales"):
-            a = bulk.cache.view(0, side, what)[:, :200].cpu()
-            b = inc.cache.view(0, side, what)[:, :200].cpu()
-            assert torch.equal(a, b)
-    assert inc.cache.view(0, 0, "seq_len").cpu().tolist() == [200, 200]
-    inc.check_codes(0)
+        for what in ("codes", "scales", "zeros"):
+            a, b = bulk.cache.view(0, side, what), inc.cache.view(0, side, what)
+            if a is not None:
+                assert torch.equal(a[:, :T].cpu(), b[:, :T].cpu()), (side, what)
+    assert inc.cache.view(0, 0, "seq_len").cpu().tolist() == [T, T]
+    bulk.check_codes(0)
+    bulk.decode_and_compare(0, queries(cfg, 2, T))
 
 
 @pytest.mark.parametrize("rule,n", [("first_n", 48), ("window", 64), ("all", 0)])
