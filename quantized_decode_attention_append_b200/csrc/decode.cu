@@ -499,14 +499,14 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
     *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, TPW_, ST_>();                               \
     return true;                                                                              \
   }
-  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 64, 3)
-  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 64, 3)
-  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 64, 3)
-  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 64, 3)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 32, 4)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 32, 4)
+  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 32, 3)
+  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 32, 3)
+  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 32, 3)
+  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 32, 3)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 16, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 16, 4)
-  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 32, 4)
+  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 16, 4)
 #undef KVQ_MMA
   return false;
 }

@@ -148,6 +148,29 @@ __device__ void prepare_query_rot(const LayerDev& L, const __half* __restrict__ 
   __syncthreads();
 }
 
+// Shared-memory XOR swizzle of 16-byte chunks within a staged row, chosen per row size and
+// per-thread chunk size so that the rows a warp reads in one instruction fall in distinct banks
+// (K: rows g = 0..7 of a 16-token block; V: rows c, c+4, c+8, c+12 of the permuted k order).
+template <int RB, int CB>
+__device__ __forceinline__ int swz_k(int r) {
+  if (RB == 64 && CB == 8) return ((r >> 1) & 1) << 1;
+  if (RB == 64 && CB == 4) return (r >> 1) & 3;
+  if (RB == 128 && CB == 16) return (r & 1) << 2;
+  if (RB == 128 && CB == 4) return r & 7;
+  return 0;
+}
+template <int RB, int CB>
+__device__ __forceinline__ int swz_v(int r) {
+  if (RB == 64 && (CB == 4 || CB == 2)) return ((r >> 1) & 1) << 1;
+  if (RB == 128 && CB == 8) return (r & 3) << 1;
+  if (RB == 512 && CB == 32) return (r & 1) | ((r & 2) << 1);
+  return 0;
+}
+template <int RB>
+__device__ __forceinline__ int swz_off(int r, int off, int sw) {  // byte offset within a row
+  return (((off >> 4) ^ sw) << 4) | (off & 15);
+}
+
 template <int D, int G, int KF, int GK, int VF, int GV, int TPW, int STAGES>
 __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __half* __restrict__ q,
                                                          const int* __restrict__ seq_ids, const int* __restrict__ kv_len,
@@ -155,7 +178,8 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
   using C = MmaCfg<D, KF, GK, VF, GV, TPW, STAGES>;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint32_t lut[KF == CF_NF4 ? 256 : 1];
-  __shared__ float pbuf[4][4][TPW];
+  // P' = p * d_v as fp16 (hi, lo) per V group, in mma k order: [warp][group][column n][16 k]
+  __shared__ __half pk[4][C::NGV][8][16];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -212,16 +236,23 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
   auto issue = [&](int tile_idx, int stage) {
     const int t0 = tstart + tile_idx * C::TILE;
     unsigned char* st = smem + stage * C::STAGE_BYTES;
-    constexpr int NKC = C::TILE * C::RBK / 16, NKS = C::KS_BYTES / 16, NVC = C::TILE * C::RBV / 16,
-                  NVS = C::VS_BYTES / 16;
+    constexpr int NCK = C::RBK / 16, NCV = C::RBV / 16;
+    constexpr int NKC = C::TILE * NCK, NKS = C::KS_BYTES / 16, NVC = C::TILE * NCV, NVS = C::VS_BYTES / 16;
     for (int i = tid; i < NKC + NKS + NVC + NVS; i += 128) {
-      if (i < NKC) cp_async16(st + C::OFF_KC + i * 16, gK + (long long)t0 * C::RBK + i * 16);
-      else if (i < NKC + NKS) cp_async16(st + C::OFF_KS + (i - NKC) * 16, gKs + (long long)t0 * C::NGK * 2 + (i - NKC) * 16);
-      else if (i < NKC + NKS + NVC)
-        cp_async16(st + C::OFF_VC + (i - NKC - NKS) * 16, gV + (long long)t0 * C::RBV + (i - NKC - NKS) * 16);
-      else
+      if (i < NKC) {
+        const int r = i / NCK, j = i % NCK;
+        cp_async16(st + C::OFF_KC + r * C::RBK + ((j ^ swz_k<C::RBK, C::KCB>(r)) << 4),
+                   gK + (long long)t0 * C::RBK + i * 16);
+      } else if (i < NKC + NKS) {
+        cp_async16(st + C::OFF_KS + (i - NKC) * 16, gKs + (long long)t0 * C::NGK * 2 + (i - NKC) * 16);
+      } else if (i < NKC + NKS + NVC) {
+        const int iv = i - NKC - NKS, r = iv / NCV, j = iv % NCV;
+        cp_async16(st + C::OFF_VC + r * C::RBV + ((j ^ swz_v<C::RBV, C::VCB>(r)) << 4),
+                   gV + (long long)t0 * C::RBV + iv * 16);
+      } else {
         cp_async16(st + C::OFF_VS + (i - NKC - NKS - NVC) * 16,
                    gVs + (long long)t0 * C::NGV * 2 + (i - NKC - NKS - NVC) * 16);
+      }
     }
   };
 
@@ -256,12 +287,15 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
 #pragma unroll
       for (int gk = 0; gk < C::NGK; ++gk) {
         uint32_t kw0[C::KCW], kw1[C::KCW];
-        const unsigned char* p0 = st + C::OFF_KC + r0 * C::RBK + (gk * GK + c * (GK / 4)) * C::KB / 8;
-        const unsigned char* p1 = p0 + 8 * C::RBK;
+        const int off = (gk * GK + c * (GK / 4)) * C::KB / 8;
+        const uint32_t* p0 = reinterpret_cast<const uint32_t*>(
+            st + C::OFF_KC + r0 * C::RBK + swz_off<C::RBK>(r0, off, swz_k<C::RBK, C::KCB>(r0)));
+        const uint32_t* p1 = reinterpret_cast<const uint32_t*>(
+            st + C::OFF_KC + r1 * C::RBK + swz_off<C::RBK>(r1, off, swz_k<C::RBK, C::KCB>(r1)));
 #pragma unroll
         for (int w = 0; w < C::KCW; ++w) {
-          kw0[w] = reinterpret_cast<const uint32_t*>(p0)[w];
-          kw1[w] = reinterpret_cast<const uint32_t*>(p1)[w];
+          kw0[w] = p0[w];
+          kw1[w] = p1[w];
         }
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -289,46 +323,52 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
     float alpha = 1.0f;
     if (m_new != -INFINITY) {
       alpha = exp2f(m_run - m_new);
+      l_run *= alpha;
 #pragma unroll
       for (int sb = 0; sb < C::NSB; ++sb) {
         sc[sb][0] = exp2f(sc[sb][0] - m_new);
         sc[sb][1] = exp2f(sc[sb][1] - m_new);
-        l_run = l_run * ((sb == 0) ? alpha : 1.0f) + sc[sb][0] + sc[sb][1];
+        l_run += sc[sb][0] + sc[sb][1];
       }
       m_run = m_new;
     } else {
 #pragma unroll
       for (int sb = 0; sb < C::NSB; ++sb) sc[sb][0] = sc[sb][1] = 0.0f;
     }
+    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-    for (int i = 0; i < D / 16; ++i) {
-      oacc[i][0] *= alpha;
-      oacc[i][1] *= alpha;
-      oacc[i][2] *= alpha;
-      oacc[i][3] *= alpha;
-    }
-    // ---- P transpose through shared memory
-    if (head_ok) {
-#pragma unroll
-      for (int sb = 0; sb < C::NSB; ++sb) {
-        pbuf[warp][c][sb * 16 + g] = sc[sb][0];
-        pbuf[warp][c][sb * 16 + g + 8] = sc[sb][1];
+      for (int i = 0; i < D / 16; ++i) {
+        oacc[i][0] *= alpha;
+        oacc[i][1] *= alpha;
+        oacc[i][2] *= alpha;
+        oacc[i][3] *= alpha;
       }
     }
-    __syncwarp();
-    // ---- values
-    const int hB = g >> 1, partB = g & 1;
+    // ---- values, one 16-token sub-block at a time.  k order of a sub-block: slot 2c, 2c+1,
+    // 2c+8, 2c+9 holds token c, c+4, c+8, c+12 (so the rows a warp loads together are adjacent).
 #pragma unroll
     for (int sb = 0; sb < C::NSB; ++sb) {
-      const int ta = sb * 16 + 2 * c;  // tokens ta, ta+1, ta+8, ta+9 (warp-relative)
-      float pv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (hB < G) {
-        pv[0] = pbuf[warp][hB][ta];
-        pv[1] = pbuf[warp][hB][ta + 1];
-        pv[2] = pbuf[warp][hB][ta + 8];
-        pv[3] = pbuf[warp][hB][ta + 9];
+      // P' (hi, lo) per V group from this thread's two tokens g, g+8 (head c)
+      {
+        const int tk[2] = {g, g + 8};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int t = tk[i];
+          const int kslot = 2 * (t & 3) + ((t >> 2) & 1) + 8 * (t >> 3);
+          const float p = head_ok ? sc[sb][i] : 0.0f;
+#pragma unroll
+          for (int gv = 0; gv < C::NGV; ++gv) {
+            float d = 1.0f;
+            if (C::VSCALE) d = __half2float(reinterpret_cast<const __half*>(st + C::OFF_VS)[(rb + sb * 16 + t) * C::NGV + gv]);
+            const float x = p == 0.0f ? 0.0f : p * d;
+            const __half hi = __float2half_rn(x);
+            pk[warp][gv][2 * c][kslot] = hi;
+            pk[warp][gv][2 * c + 1][kslot] = __float2half_rn(x - __half2float(hi));
+          }
+        }
       }
-      const int rr[4] = {rb + ta, rb + ta + 1, rb + ta + 8, rb + ta + 9};
+      __syncwarp();
+      const int rr[4] = {rb + sb * 16 + c, rb + sb * 16 + c + 4, rb + sb * 16 + c + 8, rb + sb * 16 + c + 12};
       uint32_t vmask_a = 0xFFFFFFFFu, vmask_c = 0xFFFFFFFFu;
       if (VF == CF_FP16) {  // unwritten fp16 rows may hold NaN; zero them (p is 0 there)
         auto ok = [&](int r) { const int t = tile_t0 + r; return t >= R.qa && t < R.qb; };
@@ -337,29 +377,23 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
       }
 #pragma unroll
       for (int gv = 0; gv < C::NGV; ++gv) {
-        float pp[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float d = 1.0f;
-          if (C::VSCALE) d = __half2float(reinterpret_cast<const __half*>(st + C::OFF_VS)[rr[i] * C::NGV + gv]);
-          const float x = pv[i] == 0.0f ? 0.0f : pv[i] * d;
-          const float hi = __half2float(__float2half_rn(x));
-          pp[i] = partB ? x - hi : hi;
-        }
-        const uint32_t b0 = pack_h2(pp[0], pp[1]), b1 = pack_h2(pp[2], pp[3]);
+        const uint32_t* pkw = reinterpret_cast<const uint32_t*>(&pk[warp][gv][g][0]);
+        const uint32_t b0 = pkw[c], b1 = pkw[c + 4];
         uint32_t vw[4][C::VCW];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint32_t* src = reinterpret_cast<const uint32_t*>(st + C::OFF_VC + rr[i] * C::RBV +
-                                                                   (gv * GV + g * (GV / 8)) * C::VB / 8);
+          const int off = (gv * GV + g * (GV / 8)) * C::VB / 8;
+          const int sw = swz_v<C::RBV, C::VCB>(rr[i]);
+          const unsigned char* rowp = st + C::OFF_VC + rr[i] * C::RBV;
           if (C::VCB == 2) {
-            vw[i][0] = *reinterpret_cast<const uint16_t*>(src);
+            vw[i][0] = *reinterpret_cast<const uint16_t*>(rowp + swz_off<C::RBV>(rr[i], off, sw));
           } else {
 #pragma unroll
-            for (int w = 0; w < C::VCW; ++w) vw[i][w] = src[w];
+            for (int w = 0; w < C::VCW; ++w)
+              vw[i][w] = *reinterpret_cast<const uint32_t*>(rowp + swz_off<C::RBV>(rr[i], off + 4 * w, sw));
           }
         }
-        // (t, t+1) pairs of each chunk element; element e -> M-tile e/2, row g (+8 if odd)
+        // (t, t') pairs of each chunk element; element e -> M-tile e/2, row g (+8 if odd)
         uint32_t pa[GV / 8], pc[GV / 8];
         if (VF == CF_FP16) {
 #pragma unroll
@@ -388,8 +422,8 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
         for (int mt = 0; mt < C::MT; ++mt)
           mma16816(oacc[gv * C::MT + mt], pa[2 * mt], pa[2 * mt + 1], pc[2 * mt], pc[2 * mt + 1], b0, b1);
       }
+      __syncwarp();
     }
-    __syncwarp();
   }
   cp_async_wait<0>();
   __syncthreads();  // stage buffers are free: reuse them to combine the four warps
