@@ -162,6 +162,24 @@ kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q_f
                                 const int32_t* seq_ids, const int32_t* kv_len, void* out,
                                 int32_t out_fp32, float* lse, void* stream);
 
+/* kvq_decode_attention without any device allocation behind it.  Same arguments, same results,
+ * same errors, plus KVQ_ERR_CAPACITY when the split-K partials of this call (n_q x n_q_heads x
+ * (splits + 1) x (head_dim + 4) floats) exceed the library's fixed scratch of 2^21 floats
+ * (8 MiB), and KVQ_ERR_INVALID_ARG when the current device is not the handle's.  The pages have
+ * no counterpart: this is an interface convenience.
+ * For callers that cannot call cudaMalloc where they decode: code running while a stream is
+ * captured into a CUDA graph in global mode (where cudaMalloc is illegal), or a serving runtime
+ * that hands nearly all of HBM to its own pool and budgets every other byte.  The scratch is a
+ * file-scope device array that every GPU loading this library holds until the process exits.
+ * The first call on a device looks up that array's device address (cudaGetSymbolAddress, with
+ * that device current); make the first call before any stream capture.  All calls share the
+ * array, so calls that overlap on the GPU (different streams, or different handles on one
+ * device) race; serialize them.  Each call writes every partial it reads, so nothing is cleared
+ * between calls.  The handle from kvq_create keeps its own workspace; this call leaves it alone. */
+kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q_fp16, int32_t n_q,
+                                        const int32_t* seq_ids, const int32_t* kv_len, void* out,
+                                        int32_t out_fp32, float* lse, void* stream);
+
 /* Read and clear the device error word (KVQ_ERRF_* bits) into *flags.  Synchronizes the
  * device. */
 kvq_status kvq_error_flags(kvq_cache* cache, int32_t* flags);

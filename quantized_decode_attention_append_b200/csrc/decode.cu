@@ -15,6 +15,8 @@
 // DFT) applied once to the merged vector, anchors added, normalised.
 #include <math.h>
 
+#include <mutex>
+
 #include "decode_common.cuh"
 #include "kvq_internal.h"
 
@@ -581,6 +583,34 @@ cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int
     case 256: return launch_decode_d<256>(L, q, n_q, seq_ids, kv_len, out, out_fp32, lse, work, num_sms, st, launches);
   }
   return cudaErrorInvalidValue;
+}
+
+
+// ----------------------------------------------------------------------------------------------
+// Fixed scratch for kvq_decode_attention_noalloc: split-K partials live in this file-scope device
+// array instead of a workspace from cudaMalloc.  Every GPU that loads the library holds it (8 MiB)
+// until the process exits.  Host code must not pass `g_static_work` itself to a kernel (on the
+// host that name is only a stand-in); its device address comes from cudaGetSymbolAddress, taken
+// once per device with that device current.
+constexpr size_t kStaticWorkFloats = size_t(2) << 20;
+static __device__ __align__(256) float g_static_work[kStaticWorkFloats];
+
+static std::mutex g_static_mu;
+static float* g_static_ptr[128] = {};
+
+size_t static_work_floats() { return kStaticWorkFloats; }
+
+cudaError_t static_work_ptr(int dev, float** out) {
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    float* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_static_work);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace kvq

@@ -456,6 +456,30 @@ kvq_status kvq_decode_attention(kvq_cache* h, int32_t layer, const void* q, int3
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+// Same computation as kvq_decode_attention; the split-K partials go to the library's fixed
+// device scratch instead of the handle's workspace, and nothing is allocated.
+kvq_status kvq_decode_attention_noalloc(kvq_cache* h, int32_t layer, const void* q, int32_t n_q,
+                                        const int32_t* seq_ids, const int32_t* kv_len, void* out, int32_t out_fp32,
+                                        float* lse, void* stream) {
+  if (!h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || n_q < 1) return KVQ_ERR_INVALID_ARG;
+  if (!seq_ids && n_q > h->cfg.batch) return KVQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (dev != h->device) return KVQ_ERR_INVALID_ARG;
+  const LayerDev L = layer_dev(h, layer);
+  const size_t need =
+      (size_t)n_q * h->cfg.n_q_heads * decode_partials(L, n_q, h->num_sms) * (h->cfg.head_dim + kPartStride);
+  if (need > static_work_floats()) return KVQ_ERR_CAPACITY;
+  float* ws = nullptr;
+  if (static_work_ptr(dev, &ws) != cudaSuccess) return KVQ_ERR_CUDA;
+  int launches = 0;
+  const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_q, seq_ids, kv_len, out, out_fp32 ? 1 : 0,
+                                      lse, ws, h->num_sms, h->cfg.max_queries, reinterpret_cast<cudaStream_t>(stream),
+                                      &launches);
+  h->last_launches = launches;
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 kvq_status kvq_error_flags(kvq_cache* h, int32_t* flags) {
   if (!h || !flags) return KVQ_ERR_INVALID_ARG;
   unsigned v = 0;

@@ -64,6 +64,10 @@ cudaError_t launch_fill_len(int* lens, int n, int value, cudaStream_t st);
 // Split-K partials per (query, head) one decode call on `L` writes (workspace sizing).
 int decode_partials(const LayerDev& L, int n_q, int num_sms);
 
+// Fixed device scratch for the no-allocation decode entry point (decode.cu).
+size_t static_work_floats();
+cudaError_t static_work_ptr(int dev, float** out);
+
 // Which append kernels exist for a side (the API reports KVQ_ERR_UNSUPPORTED otherwise).
 bool append_supported(int D, const kvq_side& s);
 

@@ -44,7 +44,8 @@ class kvq_layout(C.Structure):
 
 
 EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
-           "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_error_flags", "kvq_nf4_levels",
+           "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_decode_attention_noalloc",
+           "kvq_error_flags", "kvq_nf4_levels",
            "kvq_last_launch_count", "kvq_status_str"]
 
 _LIB = None
@@ -68,6 +69,7 @@ def lib() -> C.CDLL:
         L.kvq_quantize_append.argtypes = [vp, i32, vp, vp, i32, vp]
         L.kvq_dequantize.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp]
         L.kvq_decode_attention.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
+        L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
         L.kvq_error_flags.argtypes = [vp, C.POINTER(i32)]
         L.kvq_nf4_levels.argtypes = [C.POINTER(C.c_float)]
         L.kvq_last_launch_count.argtypes = [vp]
@@ -197,6 +199,14 @@ def kvq_decode_attention(h, layer: int, q16, n_q: int, seq_ids, kv_len, out, lse
     fp32 = 1 if out.dtype == torch.float32 else 0
     _check(lib().kvq_decode_attention(h, layer, _ptr(q16), n_q, _ptr(seq_ids), _ptr(kv_len), _ptr(out), fp32,
                                       _ptr(lse), _stream(stream)), "kvq_decode_attention")
+
+
+def kvq_decode_attention_noalloc(h, layer: int, q16, n_q: int, seq_ids, kv_len, out, lse=None, stream=None):
+    """kvq_decode_attention with the split-K scratch in the library's fixed device array."""
+    import torch
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    _check(lib().kvq_decode_attention_noalloc(h, layer, _ptr(q16), n_q, _ptr(seq_ids), _ptr(kv_len), _ptr(out), fp32,
+                                              _ptr(lse), _stream(stream)), "kvq_decode_attention_noalloc")
 
 
 def kvq_error_flags(h) -> int:
