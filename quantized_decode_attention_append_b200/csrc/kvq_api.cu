@@ -422,6 +422,7 @@ kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const
   if (h->cfg.k.chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
   if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
   if ((int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  if ((int64_t)h->cfg.batch * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
   const LayerDev L = layer_dev(h, layer);
   int launches = 0;
   const cudaError_t e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,

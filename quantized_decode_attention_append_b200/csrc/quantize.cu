@@ -15,9 +15,9 @@
 // absmax grids, whose thresholds are small odd integers times an fp16 scale; fp64 for min-max,
 // whose thresholds add an fp16 zero point), so no rounding in a division can flip a code.
 //
-// Work mapping: one thread per row (two for head_dim 256), the whole row in registers so the
-// Hadamard butterflies run without shuffles (one xor-shuffle stage for the 256-wide transform).
-// The polar/Cartesian codecs run one warp per row with the FFT in shared memory.
+// Work mapping: one warp per row (V = head_dim/32 contiguous values per lane, grid-stride over
+// rows); the Hadamard stages run in-lane then by xor-shuffles, group statistics reduce inside the
+// group's lanes.  The polar/Cartesian codecs run one warp per row with the FFT in shared memory.
 #include <math.h>
 #include <stdio.h>
 
@@ -39,24 +39,6 @@ cudaError_t upload_tables_quant(const HostTables& t) {
 
 enum Fam { FAM_ABSMAX = 0, FAM_MINMAX = 1, FAM_NF4 = 2, FAM_TERNARY = 3, FAM_SIGN = 4 };
 
-// ------------------------------------------------------------------------------------------
-// Bit packer: LSB-first stream of b-bit codes into 32-bit words (row chunks are whole words).
-struct Packer {
-  uint32_t* out;
-  uint64_t acc;
-  int nb;
-  int w;
-  __device__ __forceinline__ void put(uint32_t code, int b) {
-    acc |= (uint64_t)code << nb;
-    nb += b;
-    if (nb >= 32) {
-      out[w++] = (uint32_t)acc;
-      acc >>= 32;
-      nb -= 32;
-    }
-  }
-};
-
 // Exact k = floor(x/d + 1/2) for fp16 d != 0 (absmax grids, zero point 0), in fp32.
 // (2k +- 1) d is exact in fp32 for |k| <= 2^9, and 2x is exact, so the comparisons are exact.
 __device__ __forceinline__ float round_exact_absmax(float x, float d, float inv) {
@@ -72,6 +54,48 @@ __device__ __forceinline__ float round_exact_absmax(float x, float d, float inv)
     else if (t2 <= hi) k += 1.0f;
   }
   return k;
+}
+
+// Same decision as round_exact_absmax: the fp32 estimate r = x * (1/d) is within 2^-16 of x/d
+// (|x/d| <= 2^8), so away from a tie (fraction outside [2^-10, 1 - 2^-10] of the half-integer
+// grid) it already gives the exact k; only near a tie do the exact comparisons run.
+__device__ __forceinline__ float round_absmax(float x, float d, float inv) {
+  const float r = __fadd_rn(__fmul_rn(x, inv), 0.5f);
+  const float k = floorf(r);
+  const float fr = __fsub_rn(r, k);
+  if (fr < (1.0f / 1024.0f) || fr > (1.0f - 1.0f / 1024.0f)) return round_exact_absmax(x, d, inv);
+  return k;
+}
+
+// Pack 32 codes of `bits` bits (LSB-first) into bits words at out (skipped unless ok).
+template <int B>
+__device__ __forceinline__ void pack32(const uint32_t* code, uint32_t* out, bool ok) {
+  uint32_t w[B];
+#pragma unroll
+  for (int k = 0; k < B; ++k) w[k] = 0u;
+#pragma unroll
+  for (int v = 0; v < 32; ++v) {
+    const int bit = v * B, wi = bit >> 5, sh = bit & 31;
+    w[wi] |= code[v] << sh;
+    if (sh + B > 32) w[wi + 1] |= code[v] >> (32 - sh);
+  }
+  if (ok) {
+#pragma unroll
+    for (int k = 0; k < B; ++k) out[k] = w[k];
+  }
+}
+
+__device__ __forceinline__ void pack32_bits(const uint32_t* code, int bits, uint32_t* out, bool ok) {
+  switch (bits) {
+    case 1: pack32<1>(code, out, ok); break;
+    case 2: pack32<2>(code, out, ok); break;
+    case 3: pack32<3>(code, out, ok); break;
+    case 4: pack32<4>(code, out, ok); break;
+    case 5: pack32<5>(code, out, ok); break;
+    case 6: pack32<6>(code, out, ok); break;
+    case 7: pack32<7>(code, out, ok); break;
+    default: pack32<8>(code, out, ok); break;
+  }
 }
 
 // Exact k = floor((x - z)/d + 1/2), d > 0, z and d fp16.  Far from a tie the fp32 estimate is
@@ -94,121 +118,6 @@ __device__ __forceinline__ float round_exact_minmax(float x, float z, float d, f
     k = (float)kk;
   }
   return k;
-}
-
-// ------------------------------------------------------------------------------------------
-// In-register orthonormal Walsh-Hadamard over 128 values: stages h = 1 .. 64, then x fp32(1/sqrt n).
-template <int N>
-__device__ __forceinline__ void fwht_local(float* x) {
-#pragma unroll
-  for (int h = 1; h < N; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-      if ((i & h) == 0) {
-        const float a = x[i], b = x[i + h];
-        x[i] = __fadd_rn(a, b);
-        x[i + h] = __fsub_rn(a, b);
-      }
-    }
-  }
-}
-
-template <int DH>
-__device__ __forceinline__ void scale_all(float* x, float r) {
-#pragma unroll
-  for (int i = 0; i < DH; ++i) x[i] = __fmul_rn(x[i], r);
-}
-
-// Quantize one group of G values x[0..G) of family FAM; packs codes, returns scale (and zero).
-template <int G, int FAM>
-__device__ __forceinline__ void quant_group(const float* x, int bits, Packer& pk, uint8_t* trit_bytes,
-                                            int jbase, __half& s_out, __half& z_out) {
-  if (FAM == FAM_ABSMAX) {
-    float m = x[0], am = fabsf(x[0]);
-#pragma unroll
-    for (int j = 1; j < G; ++j) {
-      const float a = fabsf(x[j]);
-      if (a > am) { am = a; m = x[j]; }
-    }
-    const int half = 1 << (bits - 1);
-    const __half dh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
-    const float d = __half2float(dh);
-    s_out = dh;
-    const float inv = (d != 0.0f) ? __frcp_rn(d) : 0.0f;
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      float k = 0.0f;
-      if (d != 0.0f) {
-        k = round_exact_absmax(x[j], d, inv);
-        k = fminf(fmaxf(k, (float)(-half)), (float)(half - 1));
-      }
-      pk.put((uint32_t)((int)k + half), bits);
-    }
-  } else if (FAM == FAM_MINMAX) {
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int j = 1; j < G; ++j) { mn = fminf(mn, x[j]); mx = fmaxf(mx, x[j]); }
-    const int top = (1 << bits) - 1;
-    const __half zh = __float2half_rn(mn);
-    const __half dh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)top));
-    const float z = __half2float(zh), d = __half2float(dh);
-    s_out = dh;
-    z_out = zh;
-    const float inv = (d != 0.0f) ? __frcp_rn(d) : 0.0f;
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      float k = 0.0f;
-      if (d != 0.0f) {
-        k = round_exact_minmax(x[j], z, d, inv);
-        k = fminf(fmaxf(k, 0.0f), (float)top);
-      }
-      pk.put((uint32_t)(int)k, bits);
-    }
-  } else if (FAM == FAM_NF4) {
-    float am = fabsf(x[0]);
-#pragma unroll
-    for (int j = 1; j < G; ++j) am = fmaxf(am, fabsf(x[j]));
-    const __half sh = __float2half_rn(am);
-    const float s = __half2float(sh);
-    s_out = sh;
-    float t[15];
-#pragma unroll
-    for (int i = 0; i < 15; ++i) t[i] = __fmul_rn(q_nf4_mid[i], s);  // exact (<= 24 bits)
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      int c = 7;
-      if (s != 0.0f) {
-        c = 0;
-#pragma unroll
-        for (int i = 0; i < 15; ++i) c += (x[j] >= t[i]) ? 1 : 0;
-      }
-      pk.put((uint32_t)c, 4);
-    }
-  } else if (FAM == FAM_TERNARY) {
-    float am = fabsf(x[0]);
-#pragma unroll
-    for (int j = 1; j < G; ++j) am = fmaxf(am, fabsf(x[j]));
-    const __half sh = __float2half_rn(am);
-    const float s = __half2float(sh);
-    s_out = sh;
-    const float h = __fmul_rn(s, 0.5f);
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      int dgt = 1;
-      if (s != 0.0f) dgt = (x[j] >= h) ? 2 : ((x[j] < -h) ? 0 : 1);
-      const int e = jbase + j;  // static element index
-      const int p3 = (e % 5 == 0) ? 1 : (e % 5 == 1) ? 3 : (e % 5 == 2) ? 9 : (e % 5 == 3) ? 27 : 81;
-      trit_bytes[e / 5] = (uint8_t)(trit_bytes[e / 5] + dgt * p3);
-    }
-  } else {  // FAM_SIGN
-    float acc = 0.0f;
-#pragma unroll
-    for (int j = 0; j < G; ++j) acc = __fadd_rn(acc, fabsf(x[j]));
-    const __half sh = __float2half_rn(__fmul_rn(acc, 1.0f / (float)G));
-    s_out = sh;
-#pragma unroll
-    for (int j = 0; j < G; ++j) pk.put(x[j] >= 0.0f ? 1u : 0u, 1);
-  }
 }
 
 __device__ __forceinline__ bool in_anchor(const LayerDev& L, int pos, int len_after) {
@@ -241,116 +150,6 @@ __device__ __forceinline__ void finish_append(const LayerDev& L, int n_new, unsi
   }
 }
 
-template <int DH, int TPR, int G, int FAM>
-__device__ __forceinline__ void quantize_row(const LayerDev& L, const SideDev& S, const float* x, int u, int pos,
-                                             int part);
-
-// ------------------------------------------------------------------------------------------
-// Row kernel: DH values per thread, TPR threads per row (head_dim = DH * TPR).
-template <int DH, int TPR, int G, int FAM>
-__global__ void __launch_bounds__(128) append_rows_kernel(LayerDev L, int side, const __half* __restrict__ src,
-                                                          int n_new, unsigned total_ctas) {
-  const SideDev& S = L.s[side];
-  const int D = DH * TPR;
-  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long R = (long long)L.B * L.Hkv * n_new;
-  const long long row = gt / TPR;
-  const int part = (int)(gt % TPR);
-  const bool active = row < R;
-  int pos = 0, len_after = 0, u = 0, i = 0, b = 0;
-  if (active) {
-    i = (int)(row % n_new);
-    u = (int)(row / n_new);
-    b = u / L.Hkv;
-    const int len0 = L.seq_len[b];
-    pos = len0 + i;
-    len_after = len0 + n_new;
-  }
-  const bool ok = active && pos < L.Tcap;
-  if (active && !ok && part == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
-
-  // TPR = 2 rows must keep both lanes of the pair converged for the shuffle stage.
-  float x[DH];
-  const __half* rp = src + ((long long)u * n_new + i) * D + part * DH;
-  if (ok) {
-#pragma unroll
-    for (int c = 0; c < DH / 8; ++c) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(rp) + c);
-      const __half2* h2 = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h2[e]);
-        x[c * 8 + 2 * e] = f.x;
-        x[c * 8 + 2 * e + 1] = f.y;
-      }
-    }
-    if (in_anchor(L, pos, len_after)) {
-      __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + part * DH;
-#pragma unroll
-      for (int c = 0; c < DH / 8; ++c)
-        reinterpret_cast<uint4*>(ap)[c] = __ldg(reinterpret_cast<const uint4*>(rp) + c);
-    }
-    if (S.chan_scale) {
-      const __half* cp = S.chan + (u % L.Hkv) * D + part * DH;
-#pragma unroll
-      for (int j = 0; j < DH; ++j) x[j] = __fdiv_rn(x[j], __half2float(cp[j]));
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < DH; ++j) x[j] = 0.0f;
-  }
-
-  if (S.rot == 128 && DH == 128) {
-    fwht_local<128>(x);
-    scale_all<DH>(x, __fdiv_rn(__fsqrt_rn(2.0f), 16.0f));
-  } else if (S.rot == 256 && DH == 128 && TPR == 2) {
-    fwht_local<128>(x);
-    // stage h = 128 pairs element j of the first half with element j of the second half
-#pragma unroll
-    for (int j = 0; j < DH; ++j) {
-      const float other = __shfl_xor_sync(0xffffffffu, x[j], 1);
-      x[j] = part == 0 ? __fadd_rn(x[j], other) : __fsub_rn(other, x[j]);
-    }
-    scale_all<DH>(x, 0.0625f);
-  }
-  if (ok) quantize_row<DH, TPR, G, FAM>(L, S, x, u, pos, part);
-  // one barrier for every thread of the CTA (inactive rows included)
-  finish_append(L, n_new, total_ctas);
-}
-
-template <int DH, int TPR, int G, int FAM>
-__device__ __forceinline__ void quantize_row(const LayerDev& L, const SideDev& S, const float* x, int u, int pos,
-                                             int part) {
-  const int D = DH * TPR;
-  const long long rix = (long long)u * L.Tcap + pos;
-  const int ng = D / G;
-  __half* sp = S.scales + rix * ng + part * (DH / G);
-  __half* zp = S.zeros ? S.zeros + rix * ng + part * (DH / G) : nullptr;
-  const int b_eff = (FAM == FAM_SIGN) ? 1 : (FAM == FAM_NF4) ? 4 : S.bits;
-  Packer pk;
-  pk.out = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes + (part * DH * b_eff) / 8);
-  pk.acc = 0;
-  pk.nb = 0;
-  pk.w = 0;
-  uint8_t tb[(DH + 4) / 5 + 1];
-  if (FAM == FAM_TERNARY) {
-#pragma unroll
-    for (int j = 0; j < (DH + 4) / 5 + 1; ++j) tb[j] = 0;
-  }
-#pragma unroll
-  for (int g = 0; g < DH / G; ++g) {
-    __half s, z = __float2half_rn(0.0f);
-    quant_group<G, FAM>(x + g * G, S.bits, pk, tb, g * G, s, z);
-    sp[g] = s;
-    if (FAM == FAM_MINMAX) zp[g] = z;
-  }
-  if (FAM == FAM_TERNARY) {
-    uint8_t* op = S.codes + rix * S.row_bytes;
-#pragma unroll
-    for (int j = 0; j < (DH + 4) / 5; ++j) op[j] = tb[j];
-  }
-}
-
 // ------------------------------------------------------------------------------------------
 // rFFT polar / Cartesian codecs (head_dim 128): one warp per row, the radix-2 DIT FFT in shared
 // memory in the evaluation order the format fixes (bit-reversed input; spans 2..128; t = w*b
@@ -366,10 +165,10 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
   __shared__ uint32_t scode[kFftWarps][128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long R = (long long)L.B * L.Hkv * n_new;
-  const long long row = (long long)blockIdx.x * kFftWarps + warp;
-  bool ok = row < R;
+  for (long long row = (long long)blockIdx.x * kFftWarps + warp; row < R; row += (long long)gridDim.x * kFftWarps) {
+  bool ok = true;
   int pos = 0, len_after = 0, u = 0, i = 0;
-  if (ok) {
+  {
     i = (int)(row % n_new);
     u = (int)(row / n_new);
     const int len0 = L.seq_len[u / L.Hkv];
@@ -536,206 +335,242 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
       if (lane == 0) S.scales[rix] = dh;
     }
   }
+  __syncwarp();  // scode/sre/sim are reused by this warp's next row
+  }
   finish_append(L, n_new, total_ctas);
 }
 
 // ------------------------------------------------------------------------------------------
-// Small appends (decode-time, a few hundred rows): one warp per row, V = D/32 contiguous values per
-// lane, compact loops over runtime format parameters.  The unrolled thread-per-row kernel above is
-// tens of thousands of straight-line instructions; with only a few warps resident its instruction
-// fetch, not its arithmetic, sets the time, so short appends take this path instead.  Every
-// decision is the same exact arithmetic as the row kernel (same helpers, same evaluation order:
-// Hadamard stages in order, sign sums in channel order), so codes are identical.
-constexpr int kSmallWarps = 4;
+// Row formats (int, NF4, ternary, sign): each row is split over D/32 lanes, each lane holding 32
+// contiguous values in registers; a warp covers 32/(D/32) consecutive rows, so loads are
+// coalesced 64-byte pieces and a lane's codes fill whole 32-bit words of the packed row.  The
+// kernel is grid-stride (a few hundred CTAs, so only a few hundred completion tickets) and is
+// specialised on the grid family and group size only, which keeps it small.  Hadamard stages run
+// in-lane (h < 32) and by xor-shuffles between the row's lanes (h >= 32); groups of 64/128 reduce
+// across 2/4 lanes.  Evaluation order follows the format: Hadamard stages h = 1, 2, ..., n/2,
+// sign sums in channel order.
+constexpr int kRowThreads = 128;
 
-template <int V>
-__global__ void __launch_bounds__(32 * kSmallWarps) append_small_kernel(LayerDev L, int side,
-                                                                         const __half* __restrict__ src, int n_new,
-                                                                         unsigned total_ctas) {
+// NF4 code of x: number of thresholds th[0..14] (ascending) that x reaches, by a 4-step search.
+__device__ __forceinline__ uint32_t nf4_code(float x, const float* th) {
+  const bool b3 = x >= th[7];
+  const bool b2 = x >= (b3 ? th[11] : th[3]);
+  const float t1 = b3 ? (b2 ? th[13] : th[9]) : (b2 ? th[5] : th[1]);
+  const bool b1 = x >= t1;
+  const int i0 = (b3 ? 8 : 0) + (b2 ? 4 : 0) + (b1 ? 2 : 0);
+  float t0 = th[0];
+#pragma unroll
+  for (int k = 2; k <= 14; k += 2) t0 = (i0 == k) ? th[k] : t0;
+  const bool b0 = x >= t0;
+  return (uint32_t)(i0 + (b0 ? 1 : 0));
+}
+
+template <int FAM, int G>
+__global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, int side, const __half* __restrict__ src,
+                                                                  int n_new, unsigned total_ctas) {
   const SideDev& S = L.s[side];
-  constexpr int D = 32 * V;
-  __shared__ uint32_t words[kSmallWarps][D / 4];  // packed row (up to 8 bits per value)
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long R = (long long)L.B * L.Hkv * n_new;
-  const long long row = (long long)blockIdx.x * kSmallWarps + warp;
-  bool ok = row < R;
-  int i = 0, u = 0, pos = 0, len_after = 0;
-  if (ok) {
-    i = (int)(row % n_new);
-    u = (int)(row / n_new);
-    const int len0 = L.seq_len[u / L.Hkv];
-    pos = len0 + i;
-    len_after = len0 + n_new;
-    if (pos >= L.Tcap) {
-      if (lane == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
-      ok = false;
+  const int D = L.D, lpr = D >> 5;                    // lanes per row
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = kRowThreads / 32;
+  const int rpw = 32 / lpr;                           // rows per warp
+  const int li = lane % lpr;                          // this lane's 32-value slice of its row
+  const int R = L.B * L.Hkv * n_new;                  // < 2^31 (checked on the host)
+  constexpr int LG = G > 32 ? G / 32 : 1;             // lanes per group
+  constexpr int GPL = G > 32 ? 1 : 32 / G;            // groups per lane
+  const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : S.bits);
+  __shared__ uint32_t tw[NW][64];                     // ternary byte accumulation, one row slot at a time
+
+  for (int rb = (blockIdx.x * NW + warp) * rpw; rb < R; rb += gridDim.x * NW * rpw) {
+    const int row = rb + lane / lpr;
+    int i = 0, u = 0, pos = 0, len_after = 0;
+    bool ok = row < R;
+    if (ok) {
+      u = row / n_new;
+      i = row - u * n_new;
+      const int len0 = L.seq_len[u / L.Hkv];
+      pos = len0 + i;
+      len_after = len0 + n_new;
+      if (pos >= L.Tcap) {
+        if (li == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
+        ok = false;
+      }
     }
-  }
-  if (ok) {
-    const __half* rp = src + ((long long)u * n_new + i) * D + lane * V;
-    float x[V];
+    float x[32];
+    const __half* rp = src + ((long long)u * n_new + i) * D + li * 32;
+    if (ok) {
 #pragma unroll
-    for (int v = 0; v < V; ++v) x[v] = __half2float(rp[v]);
-    if (in_anchor(L, pos, len_after)) {
-      __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + lane * V;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(rp) + c4);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&w);
 #pragma unroll
-      for (int v = 0; v < V; ++v) ap[v] = rp[v];
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h2[e]);
+          x[c4 * 8 + 2 * e] = f.x;
+          x[c4 * 8 + 2 * e + 1] = f.y;
+        }
+      }
+      if (in_anchor(L, pos, len_after)) {
+        __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + li * 32;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = __ldg(reinterpret_cast<const uint4*>(rp) + c4);
+      }
+      if (S.chan_scale) {
+        const __half* cp = S.chan + (u % L.Hkv) * D + li * 32;
+#pragma unroll
+        for (int v = 0; v < 32; ++v) x[v] = __fdiv_rn(x[v], __half2float(cp[v]));
+      }
+    } else {
+#pragma unroll
+      for (int v = 0; v < 32; ++v) x[v] = 0.0f;
     }
-    if (S.chan_scale) {
-      const __half* cp = S.chan + (u % L.Hkv) * D + lane * V;
+    if (S.rot) {  // stages h = 1 .. rot/2 (warp-uniform: every lane takes part in the shuffles)
 #pragma unroll
-      for (int v = 0; v < V; ++v) x[v] = __fdiv_rn(x[v], __half2float(cp[v]));
-    }
-    if (S.rot) {  // stages h = 1 .. n/2 over element index j = lane*V + v
-      for (int h = 1; h < S.rot; h <<= 1) {
-        if (h < V) {
+      for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-          for (int v = 0; v < V; ++v)
-            if ((v & h) == 0) {
-              const float a = x[v], b = x[v + h];
-              x[v] = __fadd_rn(a, b);
-              x[v + h] = __fsub_rn(a, b);
-            }
-        } else {
-          const int lm = h / V;
-          const bool upper = (lane & lm) != 0;
-#pragma unroll
-          for (int v = 0; v < V; ++v) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[v], lm);
-            x[v] = upper ? __fsub_rn(o, x[v]) : __fadd_rn(x[v], o);
+        for (int v = 0; v < 32; ++v)
+          if ((v & h) == 0) {
+            const float a = x[v], b = x[v + h];
+            x[v] = __fadd_rn(a, b);
+            x[v + h] = __fsub_rn(a, b);
           }
+      }
+      for (int h = 32; h < S.rot; h <<= 1) {
+        const int lm = h >> 5;
+        const bool upper = (li & lm) != 0;
+#pragma unroll
+        for (int v = 0; v < 32; ++v) {
+          const float o = __shfl_xor_sync(0xffffffffu, x[v], lm);
+          x[v] = upper ? __fsub_rn(o, x[v]) : __fadd_rn(x[v], o);
         }
       }
       const float rn = S.rot == 256 ? 0.0625f : __fdiv_rn(__fsqrt_rn(2.0f), 16.0f);
 #pragma unroll
-      for (int v = 0; v < V; ++v) x[v] = __fmul_rn(x[v], rn);
+      for (int v = 0; v < 32; ++v) x[v] = __fmul_rn(x[v], rn);
     }
-    // groups: a lane holds ngl groups of epl values; a group spans lpg lanes
-    const int g = S.group;
-    const int epl = g < V ? g : V, ngl = V / epl, lpg = g / epl;
-    const int fam = (S.fmt == KVQ_FMT_INT) ? (S.scale_mode == KVQ_SCALE_MINMAX ? FAM_MINMAX : FAM_ABSMAX)
-                                           : (S.fmt == KVQ_FMT_NF4 ? FAM_NF4 : (S.fmt == KVQ_FMT_TERNARY ? FAM_TERNARY : FAM_SIGN));
-    const int bits = fam == FAM_SIGN ? 1 : (fam == FAM_NF4 ? 4 : S.bits);
     const long long rix = (long long)u * L.Tcap + pos;
-    for (int w = lane; w < D / 4; w += 32) words[warp][w] = 0u;
-    __syncwarp();
-    uint32_t code[V];
+    uint32_t* wout = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes) + li * bits;  // this lane's words
+    uint32_t code[32];
+    if (FAM == FAM_TERNARY) {
+      for (int k = lane; k < 64; k += 32) tw[warp][k] = 0u;
+      __syncwarp();
+    }
 #pragma unroll
-    for (int gl = 0; gl < V; ++gl) {
-      if (gl >= ngl) break;
-      const int v0 = gl * epl;
-      // per-lane partial statistics over x[v0 .. v0+epl)
-      float m = 0.0f, am = -1.0f, mn = INFINITY, mx = -INFINITY, sum = 0.0f;
-      int mi = 1 << 30;
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        if (v < v0 || v >= v0 + epl) continue;
-        const float a = fabsf(x[v]);
-        if (a > am) { am = a; m = x[v]; mi = lane * V + v; }
-        mn = fminf(mn, x[v]);
-        mx = fmaxf(mx, x[v]);
-      }
-      if (fam == FAM_SIGN) {  // fp32 sum of |x| in channel order across the group's lanes
-        const int base = lane - (lane % lpg);
-        for (int k = 0; k < lpg; ++k) {
-          if (lane == base + k) {
-#pragma unroll
-            for (int v = 0; v < V; ++v)
-              if (v >= v0 && v < v0 + epl) sum = __fadd_rn(sum, fabsf(x[v]));
-          }
-          sum = __shfl_sync(0xffffffffu, sum, base + k);
-        }
-      }
-      for (int o = 1; o < lpg; o <<= 1) {  // reductions inside the group (first index on ties)
-        const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, m, o);
-        const int omi = __shfl_xor_sync(0xffffffffu, mi, o);
-        if (oam > am || (oam == am && omi < mi)) { am = oam; m = om; mi = omi; }
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
+    for (int gl = 0; gl < GPL; ++gl) {
+      const float* xg = x + gl * (G > 32 ? 32 : G);
+      constexpr int NV = G > 32 ? 32 : G;
       __half sh, zh = __float2half_rn(0.0f);
       float d = 0.0f, z = 0.0f, inv = 0.0f;
-      int half = 0, top = 0;
-      float t[15];
-      if (fam == FAM_ABSMAX) {
-        half = 1 << (bits - 1);
+      if (FAM == FAM_ABSMAX) {
+        float m = xg[0], am = fabsf(xg[0]);
+        int mi = li * 32 + gl * NV;
+#pragma unroll
+        for (int v = 1; v < NV; ++v) {
+          const float a = fabsf(xg[v]);
+          if (a > am) { am = a; m = xg[v]; mi = li * 32 + gl * NV + v; }
+        }
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) {  // first index on ties
+          const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, m, o);
+          const int omi = __shfl_xor_sync(0xffffffffu, mi, o);
+          if (oam > am || (oam == am && omi < mi)) { am = oam; m = om; mi = omi; }
+        }
+        const int half = 1 << (bits - 1);
         sh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
         d = __half2float(sh);
         inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
-      } else if (fam == FAM_MINMAX) {
-        top = (1 << bits) - 1;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float k = 0.0f;
+          if (d != 0.0f) k = fminf(fmaxf(round_absmax(xg[v], d, inv), (float)(-half)), (float)(half - 1));
+          code[gl * NV + v] = (uint32_t)((int)k + half);
+        }
+      } else if (FAM == FAM_MINMAX) {
+        float mn = xg[0], mx = xg[0];
+#pragma unroll
+        for (int v = 1; v < NV; ++v) { mn = fminf(mn, xg[v]); mx = fmaxf(mx, xg[v]); }
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const int top = (1 << bits) - 1;
         zh = __float2half_rn(mn);
         sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)top));
         z = __half2float(zh);
         d = __half2float(sh);
         inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
-      } else if (fam == FAM_SIGN) {
-        sh = __float2half_rn(__fmul_rn(sum, 1.0f / (float)g));
-      } else {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float k = 0.0f;
+          if (d != 0.0f) k = fminf(fmaxf(round_exact_minmax(xg[v], z, d, inv), 0.0f), (float)top);
+          code[gl * NV + v] = (uint32_t)(int)k;
+        }
+      } else if (FAM == FAM_SIGN) {
+        float sum = 0.0f;  // fp32 sum of |x| in channel order, lane by lane across the group
+        if (LG == 1) {
+#pragma unroll
+          for (int v = 0; v < NV; ++v) sum = __fadd_rn(sum, fabsf(xg[v]));
+        } else {
+          const int base = lane - (li % LG);
+#pragma unroll
+          for (int k = 0; k < LG; ++k) {
+            if ((li % LG) == k) {
+#pragma unroll
+              for (int v = 0; v < NV; ++v) sum = __fadd_rn(sum, fabsf(xg[v]));
+            }
+            sum = __shfl_sync(0xffffffffu, sum, base + k);
+          }
+        }
+        sh = __float2half_rn(__fmul_rn(sum, 1.0f / (float)G));
+#pragma unroll
+        for (int v = 0; v < NV; ++v) code[gl * NV + v] = xg[v] >= 0.0f ? 1u : 0u;
+      } else {  // NF4 and ternary: absmax magnitude scale
+        float am = fabsf(xg[0]);
+#pragma unroll
+        for (int v = 1; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
         sh = __float2half_rn(am);
         d = __half2float(sh);
-        if (fam == FAM_NF4) {
+        if (FAM == FAM_NF4) {
+          float th[15];
 #pragma unroll
-          for (int k = 0; k < 15; ++k) t[k] = __fmul_rn(q_nf4_mid[k], d);
-        }
-      }
+          for (int k = 0; k < 15; ++k) th[k] = __fmul_rn(q_nf4_mid[k], d);  // exact (<= 24 bits)
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        if (v < v0 || v >= v0 + epl) continue;
-        uint32_t cd;
-        if (fam == FAM_ABSMAX) {
-          float k = 0.0f;
-          if (d != 0.0f) k = fminf(fmaxf(round_exact_absmax(x[v], d, inv), (float)(-half)), (float)(half - 1));
-          cd = (uint32_t)((int)k + half);
-        } else if (fam == FAM_MINMAX) {
-          float k = 0.0f;
-          if (d != 0.0f) k = fminf(fmaxf(round_exact_minmax(x[v], z, d, inv), 0.0f), (float)top);
-          cd = (uint32_t)(int)k;
-        } else if (fam == FAM_NF4) {
-          int cc = 7;
-          if (d != 0.0f) {
-            cc = 0;
-#pragma unroll
-            for (int k = 0; k < 15; ++k) cc += (x[v] >= t[k]) ? 1 : 0;
-          }
-          cd = (uint32_t)cc;
-        } else if (fam == FAM_TERNARY) {
+          for (int v = 0; v < NV; ++v) code[gl * NV + v] = d != 0.0f ? nf4_code(xg[v], th) : 7u;
+        } else {  // ternary digits t + 1 into this row's byte accumulators (5 trits per byte)
           const float hh = __fmul_rn(d, 0.5f);
-          cd = d != 0.0f ? ((x[v] >= hh) ? 2u : ((x[v] < -hh) ? 0u : 1u)) : 1u;
-        } else {
-          cd = x[v] >= 0.0f ? 1u : 0u;
+          if (ok) {
+            uint32_t* rowacc = &tw[warp][(lane / lpr) * (((D + 4) / 5 + 3) / 4)];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+              const uint32_t dg = d != 0.0f ? ((xg[v] >= hh) ? 2u : ((xg[v] < -hh) ? 0u : 1u)) : 1u;
+              const int j = li * 32 + gl * NV + v, byte = j / 5, m5 = j % 5;
+              const uint32_t p3 = m5 == 0 ? 1u : m5 == 1 ? 3u : m5 == 2 ? 9u : m5 == 3 ? 27u : 81u;
+              atomicAdd(&rowacc[byte >> 2], (dg * p3) << (8 * (byte & 3)));
+            }
+          }
         }
-        code[v] = cd;
       }
-      // one scale (and zero point) per group, written by the group's first lane
-      if (lane % lpg == 0) {
-        const int gi = (lane * V + v0) / g;
+      if (ok && (LG == 1 || (li % LG) == 0)) {
+        const int gi = (li * 32 + gl * NV) / G;
         S.scales[rix * S.n_groups + gi] = sh;
-        if (fam == FAM_MINMAX) S.zeros[rix * S.n_groups + gi] = zh;
+        if (FAM == FAM_MINMAX) S.zeros[rix * S.n_groups + gi] = zh;
       }
     }
-    // pack: LSB-first bit stream (ternary: 5 trits per byte) into shared words, then store
-    if (fam == FAM_TERNARY) {
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int j = lane * V + v, byte = j / 5, m5 = j % 5;
-        const uint32_t p3 = m5 == 0 ? 1u : m5 == 1 ? 3u : m5 == 2 ? 9u : m5 == 3 ? 27u : 81u;
-        atomicAdd(&words[warp][byte >> 2], (code[v] * p3) << (8 * (byte & 3)));
+    if (FAM != FAM_TERNARY) {
+      if (FAM == FAM_SIGN) pack32<1>(code, wout, ok);
+      else if (FAM == FAM_NF4) pack32<4>(code, wout, ok);
+      else pack32_bits(code, bits, wout, ok);
+    }
+    if (FAM == FAM_TERNARY) {
+      __syncwarp();
+      if (ok) {
+        const uint32_t* rowacc = &tw[warp][(lane / lpr) * (((D + 4) / 5 + 3) / 4)];
+        uint8_t* op = S.codes + rix * S.row_bytes;
+        for (int b = li; b < S.row_bytes; b += lpr) op[b] = (uint8_t)(rowacc[b >> 2] >> (8 * (b & 3)));
       }
       __syncwarp();
-      uint8_t* op = S.codes + rix * S.row_bytes;
-      for (int b = lane; b < S.row_bytes; b += 32) op[b] = (uint8_t)(words[warp][b >> 2] >> (8 * (b & 3)));
-    } else {
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int bit = (lane * V + v) * bits;
-        const uint64_t f = (uint64_t)code[v] << (bit & 31);
-        atomicOr(&words[warp][bit >> 5], (uint32_t)f);
-        if ((f >> 32) != 0ull) atomicOr(&words[warp][(bit >> 5) + 1], (uint32_t)(f >> 32));
-      }
-      __syncwarp();
-      uint32_t* op = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes);
-      for (int w = lane; w < S.row_bytes / 4; w += 32) op[w] = words[warp][w];
     }
   }
   finish_append(L, n_new, total_ctas);
@@ -750,55 +585,42 @@ static int fam_of(const SideDev& s) {
     case KVQ_FMT_INT: return s.scale_mode == KVQ_SCALE_MINMAX ? FAM_MINMAX : FAM_ABSMAX;
     case KVQ_FMT_NF4: return FAM_NF4;
     case KVQ_FMT_TERNARY: return FAM_TERNARY;
-    case KVQ_FMT_SIGN: return FAM_SIGN;
-    default: return -1;
+    default: return FAM_SIGN;
   }
 }
 
-template <int DH, int TPR, int G>
-static RowKernel pick_fam(int fam) {
-  switch (fam) {
-    case FAM_ABSMAX: return append_rows_kernel<DH, TPR, G, FAM_ABSMAX>;
-    case FAM_MINMAX: return append_rows_kernel<DH, TPR, G, FAM_MINMAX>;
-    case FAM_NF4: return append_rows_kernel<DH, TPR, G, FAM_NF4>;
-    case FAM_TERNARY: return TPR == 1 ? append_rows_kernel<DH, 1, G, FAM_TERNARY> : nullptr;
-    case FAM_SIGN: return append_rows_kernel<DH, TPR, G, FAM_SIGN>;
-  }
-  return nullptr;
-}
-
-template <int DH, int TPR>
-static RowKernel pick_group(int g, int fam) {
+template <int FAM>
+static RowKernel pick_rows_g(int g) {
   switch (g) {
-    case 4: return pick_fam<DH, TPR, 4>(fam);
-    case 8: return pick_fam<DH, TPR, 8>(fam);
-    case 16: return pick_fam<DH, TPR, 16>(fam);
-    case 32: return pick_fam<DH, TPR, 32>(fam);
-    case 64: return pick_fam<DH, TPR, 64>(fam);
-    case 128: return DH >= 128 ? pick_fam<128, TPR, 128>(fam) : nullptr;
+    case 4: return append_rows_kernel<FAM, 4>;
+    case 8: return append_rows_kernel<FAM, 8>;
+    case 16: return append_rows_kernel<FAM, 16>;
+    case 32: return append_rows_kernel<FAM, 32>;
+    case 64: return append_rows_kernel<FAM, 64>;
+    case 128: return append_rows_kernel<FAM, 128>;
   }
   return nullptr;
 }
 
-static RowKernel pick_row_kernel(int D, int g, int fam, int* tpr) {
-  if (D == 64) { *tpr = 1; return pick_group<64, 1>(g, fam); }
-  if (D == 128) { *tpr = 1; return pick_group<128, 1>(g, fam); }
-  if (D == 256) { *tpr = 2; return pick_group<128, 2>(g, fam); }
+static RowKernel pick_rows_kernel(int fam, int g) {
+  switch (fam) {
+    case FAM_ABSMAX: return pick_rows_g<FAM_ABSMAX>(g);
+    case FAM_MINMAX: return pick_rows_g<FAM_MINMAX>(g);
+    case FAM_NF4: return pick_rows_g<FAM_NF4>(g);
+    case FAM_TERNARY: return pick_rows_g<FAM_TERNARY>(g);
+    case FAM_SIGN: return pick_rows_g<FAM_SIGN>(g);
+  }
   return nullptr;
 }
 
 bool append_supported(int D, const kvq_side& s) {
   if (s.format == KVQ_FMT_FP16) return true;
   if (s.format == KVQ_FMT_POLAR || s.format == KVQ_FMT_CART) return D == 128 && s.rotation == 0;
-  SideDev sd{};
-  sd.fmt = s.format;
-  sd.scale_mode = s.scale_mode;
-  const int fam = fam_of(sd);
-  if (fam < 0) return false;
-  if (s.rotation == 128 && D == 64) return false;
-  if (s.rotation == 256 && D != 256) return false;
-  int tpr = 0;
-  return pick_row_kernel(D, s.group, fam, &tpr) != nullptr;
+  if (s.format != KVQ_FMT_INT && s.format != KVQ_FMT_NF4 && s.format != KVQ_FMT_TERNARY && s.format != KVQ_FMT_SIGN)
+    return false;
+  if (D != 64 && D != 128 && D != 256) return false;
+  if (s.rotation > D || (s.rotation && D % s.rotation)) return false;
+  return s.group >= 4 && s.group <= 128 && s.group <= D;
 }
 
 // fp16 side: plain row copy (16-byte vectors), plus anchors are irrelevant (rows already fp16).
@@ -807,10 +629,11 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
   const SideDev& S = L.s[side];
   const int vec_per_row = L.D / 8;
   const long long R = (long long)L.B * L.Hkv * n_new;
-  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x; gt < R * vec_per_row;
+       gt += (long long)gridDim.x * blockDim.x) {
   const long long row = gt / vec_per_row;
   const int c = (int)(gt % vec_per_row);
-  if (row < R) {
+  {
     const int i = (int)(row % n_new), u = (int)(row / n_new);
     const int pos = L.seq_len[u / L.Hkv] + i;
     if (pos < L.Tcap) {
@@ -822,34 +645,36 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
       atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
     }
   }
+  }
   finish_append(L, n_new, total_ctas);
 }
 
-// Appends of at most this many rows (per side) use the warp-per-row kernel.
-constexpr long long kSmallRows = 8192;
+// Grid cap of the grid-stride append kernels (148 SMs x 8 CTAs of 8 warps).
+constexpr long long kMaxAppendCtas = 148 * 8;
 
 struct SidePlan {
   void (*kern)(LayerDev, int, const __half*, int, unsigned);
-  unsigned blocks;
+  unsigned blocks, threads;
 };
 
 static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
   const SideDev& S = L.s[side];
   const long long R = (long long)L.B * L.Hkv * n_new;
-  SidePlan p{nullptr, 0};
+  SidePlan p{nullptr, 0, 128};
   if (S.fmt == KVQ_FMT_FP16) {
     p.kern = append_fp16_kernel;
-    p.blocks = (unsigned)((R * (L.D / 8) + 127) / 128);
+    const long long want = (R * (L.D / 8) + 127) / 128;
+    p.blocks = (unsigned)(want < kMaxAppendCtas ? want : kMaxAppendCtas);
   } else if (S.fmt == KVQ_FMT_POLAR || S.fmt == KVQ_FMT_CART) {
     p.kern = append_fft_kernel;
-    p.blocks = (unsigned)((R + kFftWarps - 1) / kFftWarps);
-  } else if (R <= kSmallRows) {
-    p.kern = L.D == 64 ? append_small_kernel<2> : (L.D == 128 ? append_small_kernel<4> : append_small_kernel<8>);
-    p.blocks = (unsigned)((R + kSmallWarps - 1) / kSmallWarps);
+    const long long want = (R + kFftWarps - 1) / kFftWarps;
+    p.blocks = (unsigned)(want < kMaxAppendCtas ? want : kMaxAppendCtas);
   } else {
-    int tpr = 1;
-    p.kern = pick_row_kernel(L.D, S.group, fam_of(S), &tpr);
-    p.blocks = (unsigned)((R * tpr + 127) / 128);
+    p.kern = pick_rows_kernel(fam_of(S), S.group);
+    const long long rpc = (long long)(kRowThreads / 32) * (32 / (L.D / 32));  // rows per CTA pass
+    const long long want = (R + rpc - 1) / rpc;
+    p.blocks = (unsigned)(want < kMaxAppendCtas ? want : kMaxAppendCtas);
+    p.threads = kRowThreads;
   }
   return p;
 }
@@ -859,10 +684,10 @@ cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, i
   const SidePlan pk = plan_side(L, 0, n_new), pv = plan_side(L, 1, n_new);
   if (!pk.kern || !pv.kern) return cudaErrorInvalidValue;
   const unsigned total = pk.blocks + pv.blocks;
-  pk.kern<<<pk.blocks, 128, 0, st>>>(L, 0, k, n_new, total);
+  pk.kern<<<pk.blocks, pk.threads, 0, st>>>(L, 0, k, n_new, total);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  pv.kern<<<pv.blocks, 128, 0, st>>>(L, 1, v, n_new, total);
+  pv.kern<<<pv.blocks, pv.threads, 0, st>>>(L, 1, v, n_new, total);
   if (launches) *launches = 2;
   return cudaGetLastError();
 }

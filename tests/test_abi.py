@@ -62,7 +62,6 @@ def test_arena_bytes_matches_layout_arithmetic():
     (dict(v=Side("int", 4, group=32, chan_scale=True)), -1),
     (dict(k=Side("polar", 4, 8, rot=128)), -1),
     (dict(head_dim=256, k=Side("polar", 4, 8), v=Side("polar", 4, 8)), -2),
-    (dict(head_dim=256, k=Side("ternary", group=8), v=Side("ternary", group=8)), -2),
     (dict(k=Side("nf4", scale="minmax", group=64)), -1),
     (dict(anchor_layers=(5,), anchor_rule="first_n", anchor_n=8), -1),
     (dict(anchor_layers=(0,), anchor_rule="window", anchor_n=0), -1),

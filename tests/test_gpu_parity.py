@@ -59,6 +59,8 @@ FORMATS = [
     (256, Side("int", 4, group=64, rot=128), Side("nf4", group=32)),
     (64, Side("int", 4, group=16), Side("sign", group=8)),
     (64, Side("nf4", group=64), Side("ternary", group=4)),
+    (256, Side("ternary", group=8, rot=256), Side("sign", group=16, rot=128)),
+    (256, Side("int", 7, group=64), Side("int", 5, scale="minmax", group=32)),
 ]
 
 
