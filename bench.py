@@ -30,6 +30,9 @@ WORKLOADS = {
     "stress-nf4": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
                        k=dict(fmt="nf4", group=64), v=dict(fmt="int", bits=4, group=64),
                        desc="32L x 8kv x 32q, hd128, B16 x 32768 tokens; NF4-K g64 + int4-g64 V (4.25 b)"),
+    "stress-int4": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
+                        k=dict(fmt="int", bits=4, group=64), v=dict(fmt="int", bits=4, group=64),
+                        desc="32L x 8kv x 32q, hd128, B16 x 32768 tokens; int4-g64 K and V (4.25 b)"),
     "stress-ternary": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
                            k=dict(fmt="ternary", group=8), v=dict(fmt="ternary", group=8),
                            anchors=dict(layers=(0,), rule="first_n", n=48),
@@ -218,6 +221,22 @@ def fill_cache(cache, w, T0, seed, device, timed=False):
     return ms, rows
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (one all_reduce; replicas exchange nothing else)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_steps_per_s(ms_step_max: float, world: int) -> float:
+    """Whole-job throughput of `world` replicas, each doing one step per ms_step_max (the slowest)."""
+    return world * 1e3 / ms_step_max
+
+
 def run_gpu(args, w, name):
     import torch
     import torch.distributed as dist
@@ -291,10 +310,8 @@ def run_gpu(args, w, name):
     torch.cuda.synchronize()
     clk = clocks.stop()
     dec_launch_ms = d0.elapsed_time(d1) / (K_ * L)
+    ms, dec_launch_ms = max_over_ranks([ms, dec_launch_ms], dev)
     if world > 1:
-        tt = torch.tensor([ms, dec_launch_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, dec_launch_ms = float(tt[0].item()), float(tt[1].item())
         dist.barrier()
     flags = kvq.kvq_error_flags(cache.h)
     ms_step = ms / K_
@@ -343,10 +360,7 @@ def run_gpu(args, w, name):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / E
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
     h2d = sum(x.numel() * x.element_size() for x in h_k + h_v + h_q)
     d2h = sum(x.numel() * x.element_size() for x in h_o)
 
@@ -359,7 +373,8 @@ def run_gpu(args, w, name):
             cpu = {"value": 1.0 / (per_unit * units_per_step), "unit": "steps/s", "cores": 1, "kind": "oracle",
                    "sample": f"{n} (layer, seq, kv-head) units of one step (quantize + reconstruct {T} rows, "
                              f"attend {Hq // Hkv} heads), scaled by {units_per_step} units/step"}
-        rec = {"metric": "decode steps/s", "value": world * 1e3 / ms_step, "unit": "steps/s", "n_gpus": world,
+        rec = {"metric": "decode steps/s", "value": aggregate_steps_per_s(ms_step, world), "unit": "steps/s",
+               "n_gpus": world,
                "steps": K_, "warmup": W_, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                "config": {"workload": f"{name}: {w['desc']}", "global_batch": world * B, "seq_len": T,
@@ -377,7 +392,7 @@ def run_gpu(args, w, name):
                             "rows": q_rows, "bytes_per_row": row_io,
                             "what": "bulk prefill appends (fp16 K+V read, packed codes + scales written)"},
                "cpu_baseline": cpu,
-               "e2e": {"value": world * 1e3 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+               "e2e": {"value": aggregate_steps_per_s(e2e_ms, world), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h},
                "gpu_launches": per_step_launches * K_,
                "clocks": clk, "error_flags": flags}

@@ -134,9 +134,9 @@ kvq_status kvq_set_seq_len(kvq_cache* cache, int32_t layer, int32_t len, void* s
  * the anchor set are also kept as fp16, and seq_len[b] += n_new.  n_new = prompt length is
  * the bulk prefill; n_new = 1 is the decode-time append.  Errors: KVQ_ERR_CAPACITY if the
  * host-side length bound would pass capacity; KVQ_ERR_STATE if a channel scale is required
- * and was never set.  [E22L] "What I tested" ("Quantize ... keys and values as they enter
- * the cache"), [FMKQ] post 6 "Corrected semantics" ("quantize ALL layers, anchors only
- * protect"). */
+ * and was never set.  [E22L] "What I tested" (keys and values quantized on entry to the
+ * cache), [FMKQ] post 6 "Corrected semantics" (every layer quantized, anchors as extra
+ * protection). */
 kvq_status kvq_quantize_append(kvq_cache* cache, int32_t layer, const void* k_fp16,
                                const void* v_fp16, int32_t n_new, void* stream);
 

@@ -5,9 +5,9 @@ GQA groups), s_t = sm_scale * (q . k_t) for t < kv_len with sm_scale = 1/sqrt(D)
 p = softmax(s), o = sum_t p_t v_t.  The keys and values are the oracle's own reconstruction
 of the stored rows in the original domain; rows kept as fp16 anchors are used as stored.
 
-Metrics ("E21W" "What I tested": "K/V error is squared error over signal energy. Attention
-error is relative error of the attention output, KL is the divergence of the attention
-distribution from f16"; "E22L" "Result": "mean KL"):
+Metrics, as defined in "E21W" "What I tested" (K/V error as squared error relative to the
+signal energy, attention error as the relative error of the attention output, KL of the
+attention distribution against the fp16 one) and averaged as in "E22L" "Result":
   X1 = sum (x - x_hat)^2 / sum x^2
   X2 = ||o - o_f16||_2 / ||o_f16||_2
   X3 = sum_t p_f16(t) ln(p_f16(t) / p_q(t))

@@ -1,22 +1,21 @@
 """Layer-level semantics of the quantized cache: anchors, effective bits, decode.
 
-Anchors ("Fourier Magnitude KV Cache Quantization" post 6, "Corrected semantics":
-"quantize ALL layers, anchors only protect"; "Minimal recipe": "fp16 anchors on layer 0
-alone (D=48)"; "The winning recipe": "keep the KV of the first N decoded tokens in high
-precision only on the quantization-sensitive layers"; "sliding window s64 (all layers)").
-Every row is quantized; a row in the anchor set is additionally kept as its original fp16
-row, and attention reads that fp16 row instead of the quantized one.  Rules, for layers in
+Anchors ("Fourier Magnitude KV Cache Quantization" post 6: "Corrected semantics" -- every
+layer is quantized and anchors only add protection; "Minimal recipe" -- fp16 anchors on layer 0
+only, 48 tokens; "The winning recipe" -- the first decoded tokens stay high precision on
+selected layers; a 64-token sliding window is also reported).  Every row is quantized; a row in
+the anchor set is additionally kept as its original fp16 row, and attention reads that fp16 row
+instead of the quantized one.  Rules, for layers in
 the anchor layer set:
   first_n(n): tokens t < n
   window(w):  tokens t >= L - w, L = the sequence's stored length
   all:        every token of the layer
 
-Effective bits ("E21W" "Result": "Group scales are counted in the bit totals (3.5 bits
-per value for 3-bit at group 32, 4.5 for 4-bit)"; "E22L" "What I tested": "Bits per value
-are averaged over keys and values and include the scales"; post 6 "Corrected semantics":
-"NF4/g64 + dp32 anchors ALL layers: ... eff bits"): (code bits + 16 per scale + 16 per zero
-point + 16 D per anchored row + 16 D per channel-scale vector) / values, averaged over K
-and V.
+Effective bits ("E21W" "Result" counts group scales in the totals, 3.5 b for 3-bit g32 and
+4.5 b for 4-bit g32; "E22L" "What I tested" averages over K and V with scales included; post 6
+"Corrected semantics" reports anchored configurations in effective bits): (code bits + 16 per
+scale + 16 per zero point + 16 D per anchored row + 16 D per channel-scale vector) / values,
+averaged over K and V.
 """
 from __future__ import annotations
 

@@ -1,8 +1,9 @@
 """NF4 (4-bit NormalFloat) level table.
 
 The pages use NF4 as a K-cache grid ("Fourier Magnitude KV Cache Quantization", post 6:
-"NF4/g64, no anchors: 39.8% @ 4.25b", "NF4-K + int4-g64 V (4.25b)", "Tails are sacred ...
-fixed nonuniform codebooks (NF4) with intact range win") but print no table.  This follows
+"Corrected semantics" lists NF4 with groups of 64 at 4.25 b, the "Milestone" table pairs NF4 K
+with int4-g64 V, and "Mechanism findings" credits fixed non-uniform codebooks that keep the
+full range) but print no table.  This follows
 the published NormalFloat construction (Dettmers et al., QLoRA, 2023): normal quantiles, 8
 levels above zero and 7 below, an exact zero, extremes normalised to +-1.  The outer
 probability is delta = 1 - (1/(2*15) + 1/(2*16)) / 2, the mean of the 15- and 16-level

@@ -6,30 +6,29 @@ are exact in fp64 (small odd integers times an fp16 scale, plus an fp16 zero poi
 rounding in a division can never flip a code.
 
 Grids and scales (sources by page title and section):
-  * signed absmax int b, ggml-style: "E22L" "What I tested" ("absmax quantization with an
-    fp16 scale per group") and "Result" ("the ggml-style signed absmax grid (levels -2, -1,
-    0, 1 times the scale), which leaves one side with fewer levels"); q4_0 in llama.cpp
-    #21385 "Finding 1".  The group's largest-magnitude element m (first index on ties)
+  * signed absmax int b, ggml-style: "E22L" "What I tested" (absmax scaling, one fp16 scale
+    per group) and "Result" (the 2-bit grid is the ggml signed one, levels -2..1 times the
+    scale, one level fewer on the positive side); q4_0 in llama.cpp #21385 "Finding 1".  The group's largest-magnitude element m (first index on ties)
     maps to -2^(b-1): d = fp16(m / -2^(b-1)), q = clamp(round(x/d), -2^(b-1), 2^(b-1)-1),
     stored as the unsigned code q + 2^(b-1).
-  * per-token min-max (asymmetric): "E21W" "What I tested" variant A ("plain per-token
-    min-max").  z = fp16(min), d = fp16(fp32(max - min) / (2^b - 1)),
+  * per-token min-max (asymmetric): "E21W" "What I tested", variant A.  z = fp16(min), d = fp16(fp32(max - min) / (2^b - 1)),
     q = clamp(round((x - z)/d), 0, 2^b - 1).
-  * NF4: "Fourier Magnitude KV Cache Quantization" post 6 ("NF4/g64"); s = fp16(max|x|),
+  * NF4: "Fourier Magnitude KV Cache Quantization" post 6 (NF4 in groups of 64); s = fp16(max|x|),
     code = nearest level of x/s (see oracle.nf4).
-  * ternary {-s, 0, +s}: post 6 "Milestone" table ("ternary {-s,0,+s} g8/g4");
+  * ternary {-s, 0, +s}: post 6 "Milestone" table (ternary in groups of 8 and 4);
     s = fp16(max|x|), t = nearest of {-1, 0, 1} to x/s.
-  * sign {-s, +s}: post 6 "Minimal recipe" ("binary sign KV {-s,+s}");
+  * sign {-s, +s}: post 6 "Minimal recipe" (one-bit sign KV with a scale);
     s = fp16(fp32 sum of |x| in channel order / g) (least-squares scale for fixed signs),
     t = +1 if x >= 0 else -1.
   * rFFT polar: the reply, "Fixed-rate magnitude/phase allocation" (mag/phase splits
     4+8 .. 8+4 at 12 bits per coefficient) and "The finite-phase implementation and the
-    physical codec may be worth separating" (rFFT -> magnitude index -> one phase-angle
-    index).  Magnitude uniform over [0, max] with one fp16 scale per row:
+    physical codec may be worth separating" (a magnitude index and one phase-angle index per
+    rFFT coefficient).  Magnitude uniform over [0, max] with one fp16 scale per row:
     s = fp16(fp32(max_f |X_f|) / (2^bm - 1)); phase uniform over [-pi, pi):
     code = round((atan2 + pi) 2^bp / 2pi) mod 2^bp.
-  * FFT Cartesian control: the reply, "The three controls I would try first" item 2 ("FFT
-    Cartesian (real/imag)"): the n folded spectrum reals, signed absmax int-b, one scale.
+  * FFT Cartesian control: the reply, "The three controls I would try first" item 2 (real and
+    imaginary parts instead of polar): the n folded spectrum reals, signed absmax int-b, one
+    scale.
 
 Packing: per row an LSB-first bit stream (element j at bits [b j, b j + b)); ternary packs
 5 trits per byte (byte = sum_m d_m 3^m, d = t + 1, pad digits 0); polar stores the

@@ -3,15 +3,16 @@
 Forward transforms run in fp32 in a fixed evaluation order, because their outputs decide
 integer codes; the inverses (used only for reconstruction and attention) run in fp64.
 
-* Per-channel K scale: "E21W" "What I tested", variants C and D ("per-channel K scaling
-  ... scales divided back out after dequantizing").  x_j <- x_j / c_j (IEEE fp32 division).
-* Walsh-Hadamard rotation: "E21W" variant B ("rotated by a 256-dim Hadamard") and "E22L"
-  "What I tested" ("a 256-wide Hadamard rotation before quantizing").  Sylvester order,
-  no random signs, orthonormal (1/sqrt(n)); block-diagonal when n < D.
+* Per-channel K scale: "E21W" "What I tested", variants C and D (keys divided by calibrated
+  per-channel scales, multiplied back after dequantization).  x_j <- x_j / c_j (IEEE fp32
+  division).
+* Walsh-Hadamard rotation: "E21W" variant B and "E22L" "What I tested" (a 256-wide Hadamard
+  applied before quantizing).  Sylvester order, no random signs, orthonormal (1/sqrt(n));
+  block-diagonal when n < D.
 * rFFT polar / Cartesian split: "Fourier Magnitude KV Cache Quantization" reply, "The
-  finite-phase implementation and the physical codec may be worth separating" (rFFT ->
-  magnitude index + one phase-angle index -> irFFT) and "The three controls I would try
-  first" (FFT Cartesian real/imag control).
+  finite-phase implementation and the physical codec may be worth separating" (magnitude and
+  phase-angle indices per rFFT coefficient, inverted by an irFFT) and "The three controls I
+  would try first" (the real/imaginary control).
 """
 from __future__ import annotations
 
@@ -123,8 +124,8 @@ def fold_spectrum(re: np.ndarray, im: np.ndarray):
     """The n/2 complex slots of a real row's spectrum.
 
     Slot 0 carries the two real bins: (X_0, X_{n/2}); slots f = 1 .. n/2-1 carry X_f.  This
-    keeps exactly n reals (n/2 slots), the asymptote of the reply's one-sided-spectrum bit
-    count ("(4 magnitude bits + 8 phase bits) * 33 / 64 ... approaches one half").
+    keeps exactly n reals (n/2 slots), the limit the reply's one-sided-spectrum bit count
+    approaches for long rows (12 bits x (n/2 + 1) / n -> 6 bits).
     Returns (a, b) fp32 [.., n/2]: slot real and imaginary parts.
     """
     n = re.shape[-1]

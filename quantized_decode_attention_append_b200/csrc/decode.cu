@@ -2,8 +2,8 @@
 //
 // Sources (page title, section): attention over the dequantized cache and the proxy-query setup
 // ("E21W" "What I tested": attention output, KL, causal proxy queries), the quantized-cache
-// simulation it stands in for ("E22L" "What I tested": keys and values quantized as they enter
-// the cache, "rotated" = 256-wide Hadamard), fp16 anchors ("Fourier Magnitude KV Cache
+// simulation it stands in for ("E22L" "What I tested": keys and values quantized on entry to
+// the cache, the rotated variant being a 256-wide Hadamard), fp16 anchors ("Fourier Magnitude KV Cache
 // Quantization" post 6 "Corrected semantics").
 //
 // Pass 1 (one CTA per query x kv-head x split): the query group is transformed once into the

@@ -12,7 +12,8 @@
 //           (hi, lo) halves of p * d_v (the V group scale folded into the probability).
 // K/V codes are turned into exact fp16 operands in registers: b-bit integer fields with the
 // 0x6400 exponent trick (1024 + code, then - (1024 + 2^(b-1))), NF4 through a byte -> level-pair
-// table, fp16 V by byte permutes.  Because a dot product does not depend on the order of its
+// table in shared memory (a register-resident table read by byte permutes measured slower: it
+// costs more instructions than the shared-memory lookups save), fp16 V by byte permutes.  Because a dot product does not depend on the order of its
 // terms, each thread reads a contiguous chunk of a row and the query is permuted to match.
 // Tiles of keys are staged with cp.async (16-byte copies) in a multi-stage pipeline.
 //
@@ -106,15 +107,21 @@ __device__ __forceinline__ void k_pair_elems(int p, int& e1, int& e2) {
   }
 }
 
-template <int KF>
-__device__ __forceinline__ uint32_t k_pair(const uint32_t* kw, int p, const uint32_t* lut) {
-  if (KF == CF_NF4) {
-    const uint32_t byte = (kw[p >> 2] >> (8 * (p & 3))) & 0xFFu;
-    return lut[byte];
+// All element pairs of a thread's K chunk (pair p = the p-th mma half-pair of the chunk).
+template <int KF, int KCW>
+__device__ __forceinline__ void k_pairs(const uint32_t* kw, uint32_t* pr, const uint32_t* lut) {
+  if (KF == CF_NF4) {  // byte -> (level of low nibble, level of high nibble) table in shared memory
+#pragma unroll
+    for (int w = 0; w < KCW; ++w)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) pr[4 * w + b] = lut[(kw[w] >> (8 * b)) & 0xFFu];
   } else {
     constexpr int B = CodeBits<KF>::v;
     constexpr int PPW = 16 / B;
-    return int_pair<B>(kw[p / PPW], p % PPW);
+#pragma unroll
+    for (int w = 0; w < KCW; ++w)
+#pragma unroll
+      for (int k = 0; k < PPW; ++k) pr[w * PPW + k] = int_pair<B>(kw[w], k);
   }
 }
 
@@ -177,7 +184,6 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
                                                          float* __restrict__ work, int n_split, int nsp_total) {
   using C = MmaCfg<D, KF, GK, VF, GV, TPW, STAGES>;
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ uint32_t lut[KF == CF_NF4 ? 256 : 1];
   // P' = p * d_v as fp16 (hi, lo) per V group, in mma k order: [warp][group][column n][16 k]
   __shared__ __half pk[4][C::NGV][8][16];
 
@@ -189,6 +195,7 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
   const SideDev& V = L.s[1];
   const long long u = (long long)R.seq * L.Hkv + kvh;
 
+  __shared__ uint32_t lut[KF == CF_NF4 ? 256 : 1];
   if (KF == CF_NF4) {
     for (int b = tid; b < 256; b += 128) lut[b] = pack_h2(d_nf4[b & 15], d_nf4[b >> 4]);
   }
@@ -297,13 +304,14 @@ __global__ void __launch_bounds__(128) decode_mma_kernel(LayerDev L, const __hal
           kw0[w] = p0[w];
           kw1[w] = p1[w];
         }
+        uint32_t kp0[2 * C::KSTEPS], kp1[2 * C::KSTEPS];
+        k_pairs<KF, C::KCW>(kw0, kp0, lut);
+        k_pairs<KF, C::KCW>(kw1, kp1, lut);
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const uint32_t a0 = k_pair<KF>(kw0, 2 * ks, lut), a1 = k_pair<KF>(kw1, 2 * ks, lut);
-          const uint32_t a2 = k_pair<KF>(kw0, 2 * ks + 1, lut), a3 = k_pair<KF>(kw1, 2 * ks + 1, lut);
-          mma16816(acc, a0, a1, a2, a3, qreg[gk * C::KSTEPS + ks][0], qreg[gk * C::KSTEPS + ks][1]);
-        }
+        for (int ks = 0; ks < C::KSTEPS; ++ks)
+          mma16816(acc, kp0[2 * ks], kp1[2 * ks], kp0[2 * ks + 1], kp1[2 * ks + 1], qreg[gk * C::KSTEPS + ks][0],
+                   qreg[gk * C::KSTEPS + ks][1]);
         const __half* ks_ = reinterpret_cast<const __half*>(st + C::OFF_KS);
         s0 += __half2float(ks_[r0 * C::NGK + gk]) * (acc[0] + acc[1]);
         s1 += __half2float(ks_[r1 * C::NGK + gk]) * (acc[2] + acc[3]);

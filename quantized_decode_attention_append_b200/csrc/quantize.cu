@@ -15,9 +15,11 @@
 // absmax grids, whose thresholds are small odd integers times an fp16 scale; fp64 for min-max,
 // whose thresholds add an fp16 zero point), so no rounding in a division can flip a code.
 //
-// Work mapping: one warp per row (V = head_dim/32 contiguous values per lane, grid-stride over
-// rows); the Hadamard stages run in-lane then by xor-shuffles, group statistics reduce inside the
-// group's lanes.  The polar/Cartesian codecs run one warp per row with the FFT in shared memory.
+// Work mapping: head_dim/32 lanes per row, 32 contiguous values per lane, so a warp covers
+// 32*32/head_dim rows and the grid strides over rows.  The Hadamard stages run in-lane, then by
+// xor-shuffles across the row's lanes; group statistics reduce inside the group's lanes; codes are
+// packed at compile-time widths into 32-bit words.  The polar/Cartesian codecs run one warp per
+// row with the FFT in shared memory.
 #include <math.h>
 #include <stdio.h>
 

@@ -156,12 +156,14 @@ def rope_positions(x16: torch.Tensor, positions) -> torch.Tensor:
     return torch.cat([ra, rb], dim=-1).to(torch.float16)
 
 
-def kv_rows(seed: int, side: str, layer: int, seqs, heads, tokens, D: int, device="cpu") -> torch.Tensor:
-    """Synthetic K or V rows [S, H, T, D] (fp16) following the module law."""
+def kv_rows(seed: int, side: str, layer: int, seqs, heads, tokens, D: int, device="cpu",
+            outlier_seed: int | None = None) -> torch.Tensor:
+    """Synthetic K or V rows [S, H, T, D] (fp16) following the module law.  The outlier channels
+    are a property of the (layer, kv-head): `outlier_seed` (default `seed`) picks them."""
     tag = TAG_K if side == "k" else TAG_V
     otag = TAG_OUT_K if side == "k" else TAG_OUT_V
     x = gaussian_rows(seed, tag, layer, seqs, heads, tokens, D, device)
-    om = outlier_mask(seed, otag, layer, heads, D, device)  # [H, D]
+    om = outlier_mask(seed if outlier_seed is None else outlier_seed, otag, layer, heads, D, device)  # [H, D]
     gain = torch.where(om, torch.tensor(OUTLIER_GAIN, dtype=torch.float16, device=om.device),
                        torch.tensor(1.0, dtype=torch.float16, device=om.device))
     x = x * gain.view(1, len(heads), 1, D)
@@ -191,10 +193,11 @@ def proxy_positions(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
 def channel_scale(seed: int, layer: int, n_kv_heads: int, T: int, D: int) -> torch.Tensor:
     """Per-channel K scale c [Hkv, D] fp16: RMS over tokens of a calibration cache.
 
-    The calibration cache follows the same law with seed + 1000 (one sequence).  RMS rather
-    than absmax because the x50 sink token would otherwise set every channel's scale.
+    The calibration cache follows the same law with seed + 1000 (one sequence) and the same
+    outlier channels (those belong to the layer and head, not to the text).  RMS rather than
+    absmax because the x50 sink token would otherwise set every channel's scale.
     """
-    k = kv_rows(seed + 1000, "k", layer, [0], list(range(n_kv_heads)), list(range(T)), D, "cpu")
+    k = kv_rows(seed + 1000, "k", layer, [0], list(range(n_kv_heads)), list(range(T)), D, "cpu", outlier_seed=seed)
     k64 = k[0].double()  # [H, T, D]
     rms = torch.sqrt((k64 * k64).mean(dim=1))
     return rms.to(torch.float16)

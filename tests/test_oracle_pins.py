@@ -322,8 +322,8 @@ def test_fold_unfold_roundtrip():
 
 
 def test_polar_exact_phase_reduces_to_magnitude_error():
-    """Probe of the reply ("full FFT + magnitude quantization + exact phase"): with the
-    angle kept exact, the reconstruction error is the magnitude rounding alone."""
+    """The reply's first control (quantize only the spectrum magnitudes, keep the phase
+    exact): the reconstruction error is then the magnitude rounding alone."""
     x = rng(13).standard_normal((8, 128)).astype(np.float16)
     bm = 4
     mc, pc, s = Q.quant_polar(x.astype(np.float32), bm, 8)
@@ -386,8 +386,8 @@ def test_effective_bits_closed_forms():
 
 
 def test_effective_bits_anchor_layer():
-    """Post 6 "Corrected semantics": NF4/g64 + L0-only anchors @ 4.69 eff bits, consistent
-    with one fully fp16 layer out of 26 (Gemma-3-1B depth): 4.25 + 11.75/26."""
+    """Post 6 "Corrected semantics" gives 4.69 effective bits for NF4 g64 with layer-0-only
+    anchors, which matches one fully fp16 layer out of 26 (Gemma-3-1B depth): 4.25 + 11.75/26."""
     s = C.Spec(26, 1, 1, 4, 256, Side("nf4", group=64), Side("nf4", group=64),
                frozenset({0}), "all", 0)
     assert abs(C.effective_bits(s, 4096) - 4.69) < 0.02
