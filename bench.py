@@ -127,17 +127,29 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def traffic_record(workload):
-    """dram bytes per decode launch from a committed ncu summary, if it matches this source."""
+DECODE_SOURCES = ("decode.cu", "decode_mma.cuh", "decode_common.cuh", "kvq_internal.h")
+
+
+def decode_sources_sha256():
+    """One hash over the decode kernels' sources, in a fixed order."""
     import hashlib
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        h.update(open(os.path.join(ROOT, "quantized_decode_attention_append_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def traffic_record(workload):
+    """DRAM bytes (read + write) of one decode call -- split-K pass and merge -- from the committed
+    ncu summary, or None when that summary was taken on other decode sources."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p))
-    src = open(os.path.join(ROOT, "quantized_decode_attention_append_b200", "csrc", "decode.cu"), "rb").read()
-    if rec.get("decode_cu_sha256") != hashlib.sha256(src).hexdigest():
+    if rec.get("sources_sha256") != decode_sources_sha256():
         return None
-    return rec.get("per_launch_bytes", {}).get(workload)
+    w = rec.get("per_call", {}).get(workload)
+    return None if w is None else w["bytes"]
 
 
 # ----------------------------------------------------------------------------------- CPU oracle
