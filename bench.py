@@ -18,7 +18,6 @@ import argparse
 import json
 import math
 import os
-import subprocess
 import sys
 import time
 
@@ -89,45 +88,57 @@ def decode_bytes(cache, w, kv_len, anchored_rows_per_unit):
 
 
 class ClockSampler:
-    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
-             "clocks_event_reasons.sw_power_cap"
+    """SM clock and clock-event reasons of one GPU, polled through NVML every few milliseconds on a
+    host thread between start() and stop() (read-only queries)."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = f"/tmp/kvq_clocks_{os.getpid()}.csv"
+    def __init__(self, dev, period_s=0.004):
+        self.dev, self.period = dev, period_s
+        self.rows, self.thread, self.err = [], None, None
 
     def start(self):
+        import threading
+        import torch
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as N
+            N.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            self.h = N.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.N = N
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.err = f"nvml unavailable: {type(e).__name__}"
+            return
+        self.stop_flag = threading.Event()
+
+        def poll():
+            while not self.stop_flag.is_set():
+                try:
+                    self.rows.append((self.N.nvmlDeviceGetClockInfo(self.h, self.N.NVML_CLOCK_SM),
+                                      self.N.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+                except Exception as e:
+                    self.err = f"nvml query failed: {type(e).__name__}"
+                    return
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        self.proc.wait(timeout=10)
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
-        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "not started"]}
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [self.err or "no samples"]}
+        sm = sorted(r[0] for r in self.rows)
+        reasons = sorted({name for _, m in self.rows for bit, name in self.REASONS.items() if m & bit})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.rows), "period_ms": self.period * 1e3, "source": "nvml"}
 
 
-DECODE_SOURCES = ("decode.cu", "decode_mma.cuh", "decode_common.cuh", "kvq_internal.h")
+DECODE_SOURCES = ("decode.cu", "decode_tc.cuh", "decode_common.cuh", "kvq_internal.h")
 
 
 def decode_sources_sha256():
@@ -303,7 +314,7 @@ def run_gpu(args, w, name):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()

@@ -59,7 +59,9 @@ enum { KVQ_ROT_NONE = 0, KVQ_ROT_H128 = 128, KVQ_ROT_H256 = 256 };
 enum { KVQ_ANCHOR_NONE = 0, KVQ_ANCHOR_FIRST_N = 1, KVQ_ANCHOR_WINDOW = 2, KVQ_ANCHOR_ALL = 3 };
 enum { KVQ_SIDE_K = 0, KVQ_SIDE_V = 1 };
 enum { KVQ_DOMAIN_STORED = 0, KVQ_DOMAIN_ORIGINAL = 1 };
-enum { KVQ_ERRF_CAPACITY = 1, KVQ_ERRF_SEQ_ID = 2 };
+/* Error-word bits.  KVQ_ERRF_WAIT_TIMEOUT: a decode kernel gave up waiting for a staged tile of
+ * keys/values (a bounded wait on a shared-memory barrier ran out); its output is not valid. */
+enum { KVQ_ERRF_CAPACITY = 1, KVQ_ERRF_SEQ_ID = 2, KVQ_ERRF_WAIT_TIMEOUT = 4 };
 
 typedef struct {
   int32_t format;      /* KVQ_FMT_* */

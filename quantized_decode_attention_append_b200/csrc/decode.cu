@@ -150,7 +150,7 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
   __syncthreads();
 }
 
-#include "decode_mma.cuh"
+#include "decode_tc.cuh"
 
 // Generic pass 1: any format, any GQA group (<= 8), CUDA cores.  Thread-per-token scoring,
 // thread-per-channel value accumulation.
@@ -474,13 +474,13 @@ typedef void (*MmaKernel)(LayerDev, const __half*, const int*, const int*, float
 
 struct MmaPlan {
   MmaKernel kern;
-  int smem, tile;
+  int smem, tile, threads;
 };
 
-template <int D, int G, int KF, int GK, int VF, int GV, int TPW, int ST>
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int ST>
 static MmaPlan mma_plan_of() {
-  using C = MmaCfg<D, KF, GK, VF, GV, TPW, ST>;
-  return MmaPlan{decode_mma_kernel<D, G, KF, GK, VF, GV, TPW, ST>, C::SMEM, C::TILE};
+  using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, ST>;
+  return MmaPlan{decode_tc_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST>, C::SMEM, C::TILE, C::NT};
 }
 
 static int code_fmt(const SideDev& S, bool is_v) {
@@ -490,25 +490,28 @@ static int code_fmt(const SideDev& S, bool is_v) {
   return -1;
 }
 
-// The tensor-core instantiations (others use the generic kernel).
+// The tensor-core instantiations (others use the generic kernel): warps per CTA, tokens per warp
+// and tile, pipeline stages.  Measured on the 32K-token batch-16 workload: a warp's fixed cost per
+// tile (barrier, wait, softmax reduction) is amortised best by 32-64 tokens per warp and tile, with
+// two stages of 256 tokens; NF4's 32 KB per-lane table leaves room for 8 warps per CTA at most.
 static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   const int G = L.Hq / L.Hkv;
   const int kf = code_fmt(L.s[0], false), vf = code_fmt(L.s[1], true);
   if (kf < 0 || vf < 0) return false;
   const int gk = L.s[0].group, gv = vf == CF_FP16 ? 128 : L.s[1].group;
-#define KVQ_MMA(D_, G_, KF_, GK_, VF_, GV_, TPW_, ST_)                                          \
+#define KVQ_MMA(D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_)                                     \
   if (L.D == D_ && G == G_ && kf == KF_ && gk == GK_ && vf == VF_ && gv == GV_) {                \
-    *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, TPW_, ST_>();                               \
+    *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_>();                          \
     return true;                                                                              \
   }
-  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 32, 3)
-  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 32, 3)
-  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 32, 3)
-  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 32, 3)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 16, 4)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 16, 4)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 16, 4)
-  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 16, 4)
+  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 8, 32, 2)
+  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 4, 64, 2)
+  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
+  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 16, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)
+  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 4, 16, 3)
 #undef KVQ_MMA
   return false;
 }
@@ -519,7 +522,8 @@ static int mma_slots(const MmaPlan& p, int num_sms) {
   if (cached_k != p.kern) {
     cudaFuncSetAttribute(p.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
     int occ = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, p.kern, 128, p.smem) != cudaSuccess || occ < 1) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, p.kern, p.threads, p.smem) != cudaSuccess || occ < 1)
+      occ = 1;
     cudaGetLastError();
     cached_k = p.kern;
     cached_occ = occ;
@@ -549,7 +553,7 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     const int n_split = mma_split_count((long long)n_q * L.Hkv, L.Tcap / p.tile, slots);
     n_quant = n_split;
     const int nsp = n_quant + (L.anchored ? 1 : 0);
-    p.kern<<<dim3(n_split, L.Hkv, n_q), 128, p.smem, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
+    p.kern<<<dim3(n_split, L.Hkv, n_q), p.threads, p.smem, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
     ++nl;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

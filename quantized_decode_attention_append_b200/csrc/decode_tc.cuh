@@ -1,0 +1,651 @@
+// Tensor-core pass 1 of kvq_decode_attention for GQA groups of up to 4 query heads.
+//
+// Included by decode.cu inside namespace kvq (uses QueryRange, query_range, kLog2e and d_nf4).
+// Same contract as the generic pass: one CTA per (query, kv-head, split) writes one log2-domain
+// partial (m, l, o[D] in V's stored domain); the CTA's warps are combined in shared memory first.
+//
+// Staging.  A tile of TILE consecutive tokens of one (sequence, kv-head) is four contiguous byte
+// ranges of the cache: K codes, K scales, V codes, V scales.  One thread moves each range with a
+// bulk asynchronous copy (cp.async.bulk, the TMA engine's linear mode) into a stage of shared
+// memory and the copies count their bytes on that stage's mbarrier; every thread waits on the
+// barrier with a bounded poll.  STAGES - 1 tiles are in flight while one is consumed.  Stages are
+// recycled behind one CTA barrier per tile.
+//
+// Work mapping (mma.sync m16n8k16, fp16 operands, fp32 accumulate):
+//   scores  S[16 tokens x 8] = K[16 x 16 ch] . Q'^T[16 ch x 8]; the 8 columns are 4 heads x
+//           (hi, lo) fp16 halves of the pre-transformed query, so a logit keeps ~22 bits; one
+//           accumulator per K group, multiplied by the group's fp16 scale afterwards.
+//   values  O^T[16 ch x 8] += V^T[16 ch x 16 tokens] . P'^T[16 tokens x 8]; the columns are 4
+//           heads x (hi, lo) halves of p * d_v (the V group scale folded into the probability).
+// Codes become exact fp16 operands in registers.  b-bit fields use the 0x6400 exponent trick:
+// (field << s) | 0x6400 is 1024 + 2^s field, so one fused multiply-add by 2^-s with the offset
+// -(1024 2^-s + 2^(b-1)) yields the signed code exactly; fields at shifts 0..7 of a 16-bit half
+// need no shift instruction, only the upper byte does.  NF4 goes through a byte -> level-pair table
+// in shared memory with one copy per bank (entry e of lane l at word 32 e + l), so the lanes of a
+// warp never contend for a bank.  fp16 V is regrouped by byte permutes.
+//
+// Shared-memory banks.  Each of the four ranges of a tile is copied as two halves (tokens
+// [0, TILE/2) and [TILE/2, TILE)), the second one behind a small pad, so rows of the two halves
+// start on different banks.  A 16-token block takes 8 tokens from each half: score row rho is token
+// (half R(rho), index k(rho)) with k(rho + 8) = k(rho) + 4, and R, k chosen per row size so that the
+// rows one load phase touches fall on distinct banks (for 64-byte rows: R = bit 1 of rho,
+// k = bit 0 + 2 * (rho >> 2); for 128-byte rows: R = bit 0, k = rho >> 1).  In the V product the k
+// slots (2c, 2c+1) hold the two tokens of score row c and slots (2c+8, 2c+9) those of row c + 4, so
+// the pair of probabilities a score thread owns is one 32-bit word of P'.  P' is staged per warp in
+// rows of 12 words (16 halves + 4 pad), which keeps its stores and fragment loads conflict-free.
+
+enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32 };
+
+template <int F> struct CodeBits { static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : F); };
+
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// (x & mask) | magic
+__device__ __forceinline__ uint32_t and_or(uint32_t x, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(mask), "r"(magic));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ uint32_t pack_h2(float lo_part, float hi_part) {
+  return h2u(__floats2half2_rn(lo_part, hi_part));
+}
+
+// fp16 pair (x, x) from its bit pattern
+__device__ __forceinline__ __half2 h2c(unsigned short bits) {
+  const __half h = __ushort_as_half(bits);
+  return __halves2half2(h, h);
+}
+
+// The 16/B field pairs of a 32-bit word of B-bit offset-binary codes as signed fp16 pairs:
+// out[k] = (field k, field k + 16/B), i.e. field k of each 16-bit half.
+template <int B>
+__device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out) {
+  constexpr int PH = 16 / B;                 // fields per 16-bit half
+  constexpr int PB = 8 / B;                  // fields per byte
+  constexpr uint32_t M = ((1u << B) - 1u) * 0x00010001u;
+  const uint32_t w8 = w >> 8;
+#pragma unroll
+  for (int k = 0; k < PH; ++k) {
+    const int s = B * (k % PB);              // shift of the field inside its byte
+    const uint32_t x = and_or(k < PB ? w : w8, M << s, 0x64006400u);  // 1024 + 2^s field
+    // 2^-s and -(1024 2^-s + 2^(B-1)) as fp16 bit patterns
+    const unsigned short scl = (unsigned short)((15 - s) << 10);
+    const float off = -(1024.0f / (float)(1 << s) + (float)(1 << (B - 1)));
+    const __half2 r = __hfma2(u2h(x), h2c(scl), __float2half2_rn(off));
+    out[k] = h2u(r);
+  }
+}
+
+// 2^x by the special-function unit (ex2.approx, subnormal results flushed to zero; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Entry of byte `b` of `w` in the per-lane level-pair table at shared address `base` (lane's copy;
+// entries 128 bytes apart): byte extraction by permute, address by multiply-add.
+template <int b>
+__device__ __forceinline__ uint32_t lut_pair(uint32_t base, uint32_t w) {
+  uint32_t v;
+  asm volatile(
+      "{\n .reg .u32 i, a;\n prmt.b32 i, %1, 0, %3;\n mad.lo.u32 a, i, 128, %2;\n ld.shared.u32 %0, [a];\n}\n"
+      : "=r"(v)
+      : "r"(w), "r"(base), "n"(0x4440 | b));
+  return v;
+}
+
+// ---- mbarrier and bulk-copy primitives
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// Global -> shared bulk copy completing `bytes` on `bar` (16-byte aligned ends, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete; false after about one second of polling.
+constexpr long long kWaitCycles = 2000000000LL;
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity);
+}
+
+// N consecutive 32-bit words from 4N-byte aligned shared memory
+template <int N>
+__device__ __forceinline__ void lds_words(const unsigned char* p, uint32_t* w) {
+  if constexpr (N == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (N == 1) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) lds_words<4>(p + 4 * i, w + i);
+  }
+}
+
+template <int D, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
+struct TcCfg {
+  static constexpr int KB = CodeBits<KF>::v, VB = CodeBits<VF>::v;
+  static constexpr int NT = NW * 32;                   // threads
+  static constexpr int TILE = NW * TPW;                // tokens per stage
+  static constexpr int HALF = TILE / 2;                // tokens per half-tile range
+  static constexpr int NSB = TPW / 16;                 // 16-token blocks per warp and tile
+  static constexpr int RBK = D * KB / 8, RBV = D * VB / 8;
+  static constexpr int NGK = D / GK, NGV = D / GV;
+  static constexpr bool VSCALE = VF != CF_FP16;
+  static constexpr int NPV = VSCALE ? NGV : 1;         // distinct P' operands (one per V group)
+  static constexpr int GKB = GK * KB / 8, GVB = GV * VB / 8;  // bytes of a group in a row
+  static constexpr int KCB = GKB / 4, KCW = KCB / 4;   // a thread's K chunk of a group
+  static constexpr int VCB = GVB / 8;                  // a thread's V chunk of a group (bytes)
+  static constexpr int VCW = VCB >= 4 ? VCB / 4 : 1;
+  static constexpr int VCH = VCB / 2;                  // 16-bit halves of the V chunk
+  static constexpr int KSTEPS = GK / 16, MT = GV / 16;
+  static constexpr bool ALT = RBK >= 128;              // row -> (half, index) mapping
+  // log2 headroom of p over the running max: |d_v| <= 65504 / 2^(b-1) for b-bit absmax V, so
+  // p <= 2^(b-1) keeps p * d_v finite in fp16; fp16 V has no scale.
+  static constexpr float SLACK = VSCALE ? (float)(VB - 1) : 8.0f;
+  static constexpr int PADK = RBK >= 128 ? 64 : 32, PADV = RBV >= 128 ? 64 : 32, PADS = 16;
+  // stage: [K codes A | pad | K codes B][K scales A | pad | B][V codes A | pad | B][V scales A | pad | B]
+  static constexpr int KC_H = HALF * RBK, KS_H = HALF * NGK * 2;
+  static constexpr int VC_H = HALF * RBV, VS_H = VSCALE ? HALF * NGV * 2 : 0;
+  static constexpr int OFF_KA = 0, OFF_KB = OFF_KA + KC_H + PADK;
+  static constexpr int OFF_KSA = OFF_KB + KC_H, OFF_KSB = OFF_KSA + KS_H + PADS;
+  static constexpr int OFF_VA = OFF_KSB + KS_H, OFF_VB = OFF_VA + VC_H + PADV;
+  static constexpr int OFF_VSA = OFF_VB + VC_H, OFF_VSB = OFF_VSA + VS_H + PADS;
+  static constexpr int STAGE_RAW = OFF_VSB + VS_H;
+  static constexpr int STAGE_BYTES = (STAGE_RAW + 127) / 128 * 128;
+  static constexpr uint32_t TX_BYTES = 2 * (KC_H + KS_H + VC_H + VS_H);  // bytes one tile brings
+  static constexpr int RED_BYTES = NW * 4 * (D + 2) * 4;  // epilogue: per-warp (o, m, l)
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES > RED_BYTES ? STAGES * STAGE_BYTES : RED_BYTES;
+  static constexpr int PKS = 12;                       // words per staged P' row
+  static constexpr int PK_WORDS = NPV * 8 * PKS;       // per warp
+  static constexpr int PK_BYTES_RAW = NW * PK_WORDS * 4;
+  static constexpr int QS_BYTES = 4 * D * 4;           // query staging aliases the P' area
+  static constexpr int PK_BYTES = PK_BYTES_RAW > QS_BYTES ? PK_BYTES_RAW : QS_BYTES;
+  static constexpr int LUT_BYTES = KF == CF_NF4 ? 256 * 32 * 4 : 0;
+  static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_BAR = OFF_LUT + LUT_BYTES;
+  static constexpr int SMEM = OFF_BAR + STAGES * 8;
+
+  static_assert(KCB % 4 == 0, "K chunks must be whole words");
+  static_assert(VCB % 4 == 0 || VCB == 2, "V chunks must be whole words or one half");
+  static_assert(KC_H % 128 == 0 && VC_H % 128 == 0 && KS_H % 128 == 0 && VS_H % 128 == 0,
+                "half ranges keep the bank position of what follows them");
+  static_assert(STAGE_BYTES % 16 == 0 && RING_BYTES % 16 == 0 && PK_BYTES % 16 == 0, "16-byte aligned areas");
+  static_assert(TPW % 16 == 0 && 256 % TILE == 0, "tiles must divide the 256-token capacity unit");
+  static_assert(SMEM <= 227 * 1024, "stages exceed the shared memory of one CTA");
+
+  // Half and index (within this 16-token block's 8 tokens of that half) of score row rho.
+  __device__ static __forceinline__ int row_half(int rho) { return ALT ? (rho & 1) : ((rho >> 1) & 1); }
+  __device__ static __forceinline__ int row_index(int rho) { return ALT ? (rho >> 1) : ((rho & 1) + 2 * (rho >> 2)); }
+};
+
+template <int D>
+__device__ void prepare_query_rot(const LayerDev& L, const __half* __restrict__ q, int qi, int kvh, int G, float* qs) {
+  const SideDev& K = L.s[0];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < G * D; e += blockDim.x) {
+    const int h = e / D, j = e % D;
+    const float v = __half2float(q[((long long)qi * L.Hq + kvh * G + h) * D + j]);
+    qs[e] = K.chan_scale ? v * __half2float(K.chan[kvh * D + j]) : v;
+  }
+  __syncthreads();
+  if (K.rot == 128 || K.rot == 256) {
+    for (int h = 1; h < K.rot; h <<= 1) {
+      for (int e = tid; e < G * D / 2; e += blockDim.x) {
+        const int row = e / (D / 2), p = e % (D / 2);
+        const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
+        const int i = (hi << __ffs(h)) | lo;
+        float* r = qs + row * D;
+        const float a = r[i], b = r[i + h];
+        r[i] = a + b;
+        r[i + h] = a - b;
+      }
+      __syncthreads();
+    }
+  }
+  const float rn = K.rot == 256 ? 0.0625f : (K.rot == 128 ? 0.08838834764831845f : 1.0f);
+  const float scl = L.sm_scale * kLog2e * rn;
+  for (int e = tid; e < G * D; e += blockDim.x) qs[e] *= scl;
+  __syncthreads();
+}
+
+// Element pair (e1, e2) of a thread's K chunk that pair index p covers.
+template <int KF>
+__device__ __forceinline__ void k_pair_elems(int p, int& e1, int& e2) {
+  if (KF == CF_NF4) {
+    e1 = 2 * p;
+    e2 = 2 * p + 1;
+  } else {
+    constexpr int B = CodeBits<KF>::v;
+    constexpr int PPW = 16 / B;  // pairs per word
+    const int w = p / PPW, k = p % PPW;
+    e1 = w * (32 / B) + k;
+    e2 = e1 + PPW;
+  }
+}
+
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
+__global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
+                                                            const int* __restrict__ seq_ids,
+                                                            const int* __restrict__ kv_len, float* __restrict__ work,
+                                                            int n_split, int nsp_total) {
+  using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int split = blockIdx.x, kvh = blockIdx.y, qi = blockIdx.z;
+  const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+  const SideDev& K = L.s[0];
+  const SideDev& V = L.s[1];
+  const long long u = (long long)R.seq * L.Hkv + kvh;
+
+  // ---- token range of this split, in whole tiles
+  const int tstart = (R.qa / C::TILE) * C::TILE;
+  const int ntiles = R.qb > tstart ? (R.qb - tstart + C::TILE - 1) / C::TILE : 0;
+  const int per = (ntiles + n_split - 1) / n_split;
+  const int it0 = split * per;
+  const int nmy = max(0, min(ntiles, it0 + per) - it0);
+
+  const uint8_t* gK = K.codes + u * L.Tcap * C::RBK;
+  const uint8_t* gKs = reinterpret_cast<const uint8_t*>(K.scales + u * L.Tcap * C::NGK);
+  const uint8_t* gV = V.codes + u * L.Tcap * C::RBV;
+  const uint8_t* gVs = C::VSCALE ? reinterpret_cast<const uint8_t*>(V.scales + u * L.Tcap * C::NGV) : nullptr;
+
+  auto issue = [&](int tile_idx, int stage) {  // one thread: eight bulk copies (six for fp16 V)
+    const long long t0 = tstart + (long long)tile_idx * C::TILE, t1 = t0 + C::HALF;
+    unsigned char* st = smem + stage * C::STAGE_BYTES;
+    uint64_t* b = bar + stage;
+    fence_proxy_async();
+    mbar_expect_tx(b, C::TX_BYTES);
+    bulk_g2s(st + C::OFF_KA, gK + t0 * C::RBK, C::KC_H, b);
+    bulk_g2s(st + C::OFF_KB, gK + t1 * C::RBK, C::KC_H, b);
+    bulk_g2s(st + C::OFF_KSA, gKs + t0 * C::NGK * 2, C::KS_H, b);
+    bulk_g2s(st + C::OFF_KSB, gKs + t1 * C::NGK * 2, C::KS_H, b);
+    bulk_g2s(st + C::OFF_VA, gV + t0 * C::RBV, C::VC_H, b);
+    bulk_g2s(st + C::OFF_VB, gV + t1 * C::RBV, C::VC_H, b);
+    if (C::VSCALE) {
+      bulk_g2s(st + C::OFF_VSA, gVs + t0 * C::NGV * 2, C::VS_H, b);
+      bulk_g2s(st + C::OFF_VSB, gVs + t1 * C::NGV * 2, C::VS_H, b);
+    }
+  };
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) mbar_init(bar + s, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES - 1; ++s)
+      if (s < nmy) issue(it0 + s, s);
+  }
+
+  // ---- while the first tiles are in flight: NF4 table, query fragments
+  const uint32_t lut = smem_u32(smem + C::OFF_LUT) + 4 * lane;
+  if constexpr (KF == CF_NF4) {
+    uint32_t* t = reinterpret_cast<uint32_t*>(smem + C::OFF_LUT);
+    for (int b = warp * 32 + lane; b < 256; b += NW * 32) {
+      const uint32_t v = pack_h2(d_nf4[b & 15], d_nf4[b >> 4]);
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) t[b * 32 + ((lane + i) & 31)] = v;  // lanes write distinct banks
+    }
+  }
+  float* qs = reinterpret_cast<float*>(smem + C::OFF_PK);
+  prepare_query_rot<D>(L, q, qi, kvh, G, qs);
+  uint32_t qreg[C::NGK][C::KSTEPS][2];
+  {
+    const int h = g >> 1, part = g & 1;
+#pragma unroll
+    for (int j = 0; j < C::NGK; ++j) {
+      const int cb = j * GK + c * (GK / 4);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          int e1, e2;
+          k_pair_elems<KF>(2 * ks + r, e1, e2);
+          float v1 = 0.0f, v2 = 0.0f;
+          if (h < G) {
+            v1 = qs[h * D + cb + e1];
+            v2 = qs[h * D + cb + e2];
+          }
+          const float h1 = __half2float(__float2half_rn(v1)), h2 = __half2float(__float2half_rn(v2));
+          qreg[j][ks][r] = part ? pack_h2(v1 - h1, v2 - h2) : pack_h2(h1, h2);
+        }
+      }
+    }
+  }
+  __syncthreads();  // qs aliases the P' area; the table is complete
+
+  float oacc[D / 16][4];
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
+  float m_run = -INFINITY, l_run = 0.0f;
+  const bool head_ok = c < G;
+  uint32_t* pk = reinterpret_cast<uint32_t*>(smem + C::OFF_PK) + warp * C::PK_WORDS;
+  // Score rows g and g + 8 are tokens (sh, si) and (sh, si + 4) of each block's 8 tokens per half;
+  // V rows of lane c are tokens (vh, vi + {0, 4, 2, 6}).  Blocks of a warp start at index hb.
+  const int sh = C::row_half(g), si = C::row_index(g);
+  const int vh = C::row_half(c), vi = C::row_index(c);
+  const int hb0 = warp * (TPW / 2);
+  const int ks_off = (sh ? C::OFF_KSB : C::OFF_KSA) + (hb0 + si) * C::NGK * 2;   // K scales, row g
+  const int kc_off = (sh ? C::OFF_KB : C::OFF_KA) + (hb0 + si) * C::RBK + c * C::KCB;
+  const int vs_off = (sh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + si) * C::NGV * 2;
+  const int vc_off = (vh ? C::OFF_VB : C::OFF_VA) + (hb0 + vi) * C::RBV + g * C::VCB;
+  const int st_tok = sh * C::HALF + hb0 + si;  // tile-relative token of score row g, block 0
+  const int vt_tok = vh * C::HALF + hb0 + vi;  // tile-relative token of V row c, block 0
+  bool timed_out = false;
+  int it = 0;
+
+  for (; it < nmy; ++it) {
+    if (__syncthreads_or(timed_out)) break;  // every warp is done with tile it - 1: refill its stage
+    if (tid == 0 && it + STAGES - 1 < nmy) issue(it0 + it + STAGES - 1, (it + STAGES - 1) % STAGES);
+    const int stage = it % STAGES;
+    if (__any_sync(0xffffffffu, !mbar_wait(bar + stage, (uint32_t)(it / STAGES) & 1u))) {
+      if (lane == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_WAIT_TIMEOUT);
+      timed_out = true;
+      continue;
+    }
+
+    const unsigned char* st = smem + stage * C::STAGE_BYTES;
+    const int tile_t0 = tstart + (it0 + it) * C::TILE;
+    const bool full_tile = tile_t0 >= R.qa && tile_t0 + C::TILE <= R.qb;
+
+    // ---- scores: thread (g, c) gets head c's logits of score rows g and g + 8 of each block
+    float sc[C::NSB][2];
+#pragma unroll
+    for (int sb = 0; sb < C::NSB; ++sb) {
+      float kd0[C::NGK], kd1[C::NGK];
+      {
+        const __half* s0p = reinterpret_cast<const __half*>(st + ks_off + sb * 8 * C::NGK * 2);
+        const __half* s1p = s0p + 4 * C::NGK;
+        if constexpr (C::NGK == 2) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(s0p));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(s1p));
+          kd0[0] = a.x; kd0[1] = a.y; kd1[0] = b.x; kd1[1] = b.y;
+        } else {
+#pragma unroll
+          for (int j = 0; j < C::NGK; ++j) {
+            kd0[j] = __half2float(s0p[j]);
+            kd1[j] = __half2float(s1p[j]);
+          }
+        }
+      }
+      const unsigned char* k0p = st + kc_off + sb * 8 * C::RBK;
+      const unsigned char* k1p = k0p + 4 * C::RBK;
+      float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+      for (int j = 0; j < C::NGK; ++j) {
+        uint32_t kw0[C::KCW], kw1[C::KCW];
+        lds_words<C::KCW>(k0p + j * C::GKB, kw0);
+        lds_words<C::KCW>(k1p + j * C::GKB, kw1);
+        uint32_t kp0[2 * C::KSTEPS], kp1[2 * C::KSTEPS];
+        if constexpr (KF == CF_NF4) {
+#pragma unroll
+          for (int w = 0; w < C::KCW; ++w)
+#pragma unroll
+            {
+              kp0[4 * w + 0] = lut_pair<0>(lut, kw0[w]);
+              kp0[4 * w + 1] = lut_pair<1>(lut, kw0[w]);
+              kp0[4 * w + 2] = lut_pair<2>(lut, kw0[w]);
+              kp0[4 * w + 3] = lut_pair<3>(lut, kw0[w]);
+              kp1[4 * w + 0] = lut_pair<0>(lut, kw1[w]);
+              kp1[4 * w + 1] = lut_pair<1>(lut, kw1[w]);
+              kp1[4 * w + 2] = lut_pair<2>(lut, kw1[w]);
+              kp1[4 * w + 3] = lut_pair<3>(lut, kw1[w]);
+            }
+        } else {
+          constexpr int PPW = 16 / C::KB;
+#pragma unroll
+          for (int w = 0; w < C::KCW; ++w) {
+            code_pairs<C::KB>(kw0[w], kp0 + w * PPW);
+            code_pairs<C::KB>(kw1[w], kp1 + w * PPW);
+          }
+        }
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS; ++ks)
+          mma16816(acc, kp0[2 * ks], kp1[2 * ks], kp0[2 * ks + 1], kp1[2 * ks + 1], qreg[j][ks][0], qreg[j][ks][1]);
+        s0 = fmaf(kd0[j], acc[0] + acc[1], s0);
+        s1 = fmaf(kd1[j], acc[2] + acc[3], s1);
+      }
+      if (!full_tile) {
+        const int t0 = tile_t0 + st_tok + sb * 8, t1 = t0 + 4;
+        s0 = (t0 >= R.qa && t0 < R.qb) ? s0 : -INFINITY;
+        s1 = (t1 >= R.qa && t1 < R.qb) ? s1 : -INFINITY;
+      }
+      sc[sb][0] = s0;
+      sc[sb][1] = s1;
+    }
+
+    // ---- online softmax (log2 domain) for head c over this warp's TPW tokens.  The reference
+    // max moves only when the tile's max exceeds it by more than C::SLACK, so p <= 2^SLACK and the
+    // accumulators are rescaled rarely; p * d_v still fits fp16 for any stored V scale.
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int sb = 0; sb < C::NSB; ++sb) tmax = fmaxf(tmax, fmaxf(sc[sb][0], sc[sb][1]));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+    const bool move = tmax > m_run + C::SLACK;
+    if (__any_sync(0xffffffffu, move)) {
+      const float alpha = move ? ex2(m_run - tmax) : 1.0f;  // 0 when m_run = -inf
+      const float m_new = move ? tmax : m_run;
+      l_run *= alpha;
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) {
+        oacc[i][0] *= alpha;
+        oacc[i][1] *= alpha;
+        oacc[i][2] *= alpha;
+        oacc[i][3] *= alpha;
+      }
+      m_run = m_new;
+    }
+    if (m_run != -INFINITY) {
+#pragma unroll
+      for (int sb = 0; sb < C::NSB; ++sb) {
+        sc[sb][0] = ex2(sc[sb][0] - m_run);
+        sc[sb][1] = ex2(sc[sb][1] - m_run);
+        l_run += sc[sb][0] + sc[sb][1];
+      }
+    } else {
+#pragma unroll
+      for (int sb = 0; sb < C::NSB; ++sb) sc[sb][0] = sc[sb][1] = 0.0f;
+    }
+
+    // ---- values
+#pragma unroll
+    for (int sb = 0; sb < C::NSB; ++sb) {
+      {  // P' (hi, lo) of score rows g and g + 8 for head c: word g of rows 2c and 2c + 1
+        const float p0 = (G == 4 || head_ok) ? sc[sb][0] : 0.0f, p1 = (G == 4 || head_ok) ? sc[sb][1] : 0.0f;
+        float dv0[C::NPV], dv1[C::NPV];
+        if constexpr (C::VSCALE) {
+          const __half* d0p = reinterpret_cast<const __half*>(st + vs_off + sb * 8 * C::NGV * 2);
+          const __half* d1p = d0p + 4 * C::NGV;
+          if constexpr (C::NGV == 2) {
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(d0p));
+            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(d1p));
+            dv0[0] = a.x; dv0[1] = a.y; dv1[0] = b.x; dv1[1] = b.y;
+          } else {
+#pragma unroll
+            for (int v = 0; v < C::NGV; ++v) {
+              dv0[v] = __half2float(d0p[v]);
+              dv1[v] = __half2float(d1p[v]);
+            }
+          }
+        } else {
+          dv0[0] = dv1[0] = 1.0f;
+        }
+#pragma unroll
+        for (int v = 0; v < C::NPV; ++v) {
+          float x0 = p0 * dv0[v], x1 = p1 * dv1[v];
+          if (!full_tile) {  // masked tokens may carry unwritten (non-finite) scales
+            x0 = p0 == 0.0f ? 0.0f : x0;
+            x1 = p1 == 0.0f ? 0.0f : x1;
+          }
+          const __half2 hi = __floats2half2_rn(x0, x1);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+          pk[(v * 8 + 2 * c) * C::PKS + g] = h2u(hi);
+          pk[(v * 8 + 2 * c + 1) * C::PKS + g] = h2u(lo);
+        }
+      }
+      __syncwarp();
+      uint32_t vmask_a = 0xFFFFFFFFu, vmask_c = 0xFFFFFFFFu;
+      if (VF == CF_FP16 && !full_tile) {  // unwritten fp16 rows may hold NaN; zero them (p is 0 there)
+        const int t = tile_t0 + vt_tok + sb * 8;
+        auto ok = [&](int d) { return t + d >= R.qa && t + d < R.qb; };
+        vmask_a = (ok(0) ? 0x0000FFFFu : 0u) | (ok(4) ? 0xFFFF0000u : 0u);
+        vmask_c = (ok(2) ? 0x0000FFFFu : 0u) | (ok(6) ? 0xFFFF0000u : 0u);
+      }
+#pragma unroll
+      for (int gv = 0; gv < C::NGV; ++gv) {
+        const uint32_t* pr = pk + ((C::VSCALE ? gv : 0) * 8 + g) * C::PKS;
+        const uint32_t b0 = pr[c], b1 = pr[c + 4];
+        const unsigned char* vp = st + vc_off + sb * 8 * C::RBV + gv * C::GVB;
+        uint32_t vw[4][C::VCW];
+        constexpr int roff[4] = {0, 4, 2, 6};  // slots (2c, 2c+1) then (2c+8, 2c+9)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if constexpr (C::VCB == 2) {
+            vw[i][0] = *reinterpret_cast<const uint16_t*>(vp + roff[i] * C::RBV);
+          } else {
+            lds_words<C::VCW>(vp + roff[i] * C::RBV, vw[i]);
+          }
+        }
+        uint32_t pa[GV / 8], pc[GV / 8];
+        if constexpr (VF == CF_FP16) {
+#pragma unroll
+          for (int w = 0; w < C::VCW; ++w) {
+            pa[2 * w] = prmt(vw[0][w], vw[1][w], 0x5410) & vmask_a;
+            pa[2 * w + 1] = prmt(vw[0][w], vw[1][w], 0x7632) & vmask_a;
+            pc[2 * w] = prmt(vw[2][w], vw[3][w], 0x5410) & vmask_c;
+            pc[2 * w + 1] = prmt(vw[2][w], vw[3][w], 0x7632) & vmask_c;
+          }
+        } else {
+          constexpr int PH = 16 / C::VB;  // elements per 16-bit half
+#pragma unroll
+          for (int hh = 0; hh < C::VCH; ++hh) {
+            const int w = hh >> 1, hf = hh & 1;
+            code_pairs<C::VB>(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), pa + hh * PH);
+            code_pairs<C::VB>(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), pc + hh * PH);
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+          mma16816(oacc[gv * C::MT + mt], pa[2 * mt], pa[2 * mt + 1], pc[2 * mt], pc[2 * mt + 1], b0, b1);
+      }
+      __syncwarp();
+    }
+  }
+
+  // A tile that timed out, and the tiles issued after it, may still be landing: wait for them
+  // (bounded again) before the stage buffers are reused or the CTA exits.
+  timed_out = __syncthreads_or(timed_out);
+  if (timed_out && tid == 0) {
+    const int issued = min(nmy, it + STAGES - 1);
+    for (int i = max(it - 1, 0); i < issued; ++i) mbar_wait(bar + i % STAGES, (uint32_t)(i / STAGES) & 1u);
+  }
+  __syncthreads();  // stage buffers are free: reuse them to combine the warps
+
+  // ---- combine the warps' (m, l, o) into one partial per CTA
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+  float* red = reinterpret_cast<float*>(smem);  // [NW][4 heads][D]
+  float* ml = red + NW * 4 * D;                 // [NW][4 heads][2]
+  if (timed_out) {
+    m_run = -INFINITY;
+    l_run = 0.0f;
+  }
+  if (head_ok) {
+    if (g == 0) {
+      ml[(warp * 4 + c) * 2] = m_run;
+      ml[(warp * 4 + c) * 2 + 1] = l_run;
+    }
+#pragma unroll
+    for (int gv = 0; gv < C::NGV; ++gv)
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        const int ch = gv * GV + g * (GV / 8) + 2 * mt;
+        const float* o = oacc[gv * C::MT + mt];
+        *reinterpret_cast<float2*>(red + (warp * 4 + c) * D + ch) =
+            timed_out ? make_float2(0.0f, 0.0f) : make_float2(o[0] + o[1], o[2] + o[3]);
+      }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += C::NT) {
+    const int h = e / D, j = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * 4 + h) * 2]);
+    float lsum = 0.0f, osum = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float mw = ml[(w * 4 + h) * 2];
+        const float sc = mw == -INFINITY ? 0.0f : ex2(mw - M);
+        lsum += sc * ml[(w * 4 + h) * 2 + 1];
+        osum += sc * red[(w * 4 + h) * D + j];
+      }
+    }
+    float* P = work + (((long long)qi * L.Hq + kvh * G + h) * nsp_total + split) * (D + kPartStride);
+    if (j == 0) {
+      P[0] = M;
+      P[1] = lsum;
+    }
+    P[kPartStride + j] = osum;
+  }
+}

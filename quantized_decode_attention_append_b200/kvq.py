@@ -19,7 +19,7 @@ SCALE = {"absmax": 0, "minmax": 1}
 ANCHOR = {"none": 0, "first_n": 1, "window": 2, "all": 3}
 SIDE_K, SIDE_V = 0, 1
 DOMAIN_STORED, DOMAIN_ORIGINAL = 0, 1
-ERRF_CAPACITY = 1
+ERRF_CAPACITY, ERRF_SEQ_ID, ERRF_WAIT_TIMEOUT = 1, 2, 4
 
 STATUS = {0: "KVQ_OK", -1: "KVQ_ERR_INVALID_ARG", -2: "KVQ_ERR_UNSUPPORTED", -3: "KVQ_ERR_CAPACITY",
           -4: "KVQ_ERR_CUDA", -5: "KVQ_ERR_ALLOC", -6: "KVQ_ERR_STATE"}

@@ -68,7 +68,7 @@ def test_mma_kernel_is_the_one_that_runs():
         c.cache.decode(0, q)
         torch.cuda.synchronize()
     names = " ".join(e.name for e in prof.events())
-    assert "decode_mma_kernel" in names and "merge_kernel" in names
+    assert "decode_tc_kernel" in names and "merge_kernel" in names
     assert "decode_generic_kernel" not in names
 
 
