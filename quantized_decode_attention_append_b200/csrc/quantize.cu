@@ -76,9 +76,9 @@ __device__ __forceinline__ void pack32(const uint32_t* code, uint32_t* out, bool
 #pragma unroll
   for (int k = 0; k < B; ++k) w[k] = 0u;
 #pragma unroll
-  for (int v = 0; v < 32; ++v) {
+  for (int v = 0; v < 32; ++v) {  // fields are disjoint, so adding the shifted code is an OR
     const int bit = v * B, wi = bit >> 5, sh = bit & 31;
-    w[wi] |= code[v] << sh;
+    w[wi] += code[v] << sh;
     if (sh + B > 32) w[wi + 1] |= code[v] >> (32 - sh);
   }
   if (ok) {
@@ -353,23 +353,22 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
 // sign sums in channel order.
 constexpr int kRowThreads = 128;
 
-// NF4 code of x: number of thresholds th[0..14] (ascending) that x reaches, by a 4-step search.
+// NF4 code of x: number of thresholds th[0..14] (ascending) that x reaches, by a 4-step binary
+// search whose thresholds are picked by multiplexers on the decisions taken so far.
 __device__ __forceinline__ uint32_t nf4_code(float x, const float* th) {
   const bool b3 = x >= th[7];
   const bool b2 = x >= (b3 ? th[11] : th[3]);
-  const float t1 = b3 ? (b2 ? th[13] : th[9]) : (b2 ? th[5] : th[1]);
-  const bool b1 = x >= t1;
-  const int i0 = (b3 ? 8 : 0) + (b2 ? 4 : 0) + (b1 ? 2 : 0);
-  float t0 = th[0];
-#pragma unroll
-  for (int k = 2; k <= 14; k += 2) t0 = (i0 == k) ? th[k] : t0;
+  const bool b1 = x >= (b3 ? (b2 ? th[13] : th[9]) : (b2 ? th[5] : th[1]));
+  const float t0 = b3 ? (b2 ? (b1 ? th[14] : th[12]) : (b1 ? th[10] : th[8]))
+                      : (b2 ? (b1 ? th[6] : th[4]) : (b1 ? th[2] : th[0]));
   const bool b0 = x >= t0;
-  return (uint32_t)(i0 + (b0 ? 1 : 0));
+  return (b3 ? 8u : 0u) + (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (b0 ? 1u : 0u);
 }
 
+// Rows of one side over blocks bid = 0 .. nblk - 1 (grid-stride).
 template <int FAM, int G>
-__global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, int side, const __half* __restrict__ src,
-                                                                  int n_new, unsigned total_ctas) {
+__device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __half* __restrict__ src, int n_new,
+                                          int bid, int nblk) {
   const SideDev& S = L.s[side];
   const int D = L.D, lpr = D >> 5;                    // lanes per row
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -382,7 +381,7 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
   const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : S.bits);
   __shared__ uint32_t tw[NW][64];                     // ternary byte accumulation, one row slot at a time
 
-  for (int rb = (blockIdx.x * NW + warp) * rpw; rb < R; rb += gridDim.x * NW * rpw) {
+  for (int rb = (bid * NW + warp) * rpw; rb < R; rb += nblk * NW * rpw) {
     const int row = rb + lane / lpr;
     int i = 0, u = 0, pos = 0, len_after = 0;
     bool ok = row < R;
@@ -463,28 +462,42 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
       __half sh, zh = __float2half_rn(0.0f);
       float d = 0.0f, z = 0.0f, inv = 0.0f;
       if (FAM == FAM_ABSMAX) {
-        float m = xg[0], am = fabsf(xg[0]);
-        int mi = li * 32 + gl * NV;
+        // signed value of largest magnitude, first channel on ties: the magnitude maximum, then a
+        // backward scan that keeps the earliest element reaching it
+        float am = 0.0f;
 #pragma unroll
-        for (int v = 1; v < NV; ++v) {
-          const float a = fabsf(xg[v]);
-          if (a > am) { am = a; m = xg[v]; mi = li * 32 + gl * NV + v; }
-        }
+        for (int v = 0; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+        float m = 0.0f;
 #pragma unroll
-        for (int o = 1; o < LG; o <<= 1) {  // first index on ties
+        for (int v = NV - 1; v >= 0; --v) m = fabsf(xg[v]) == am ? xg[v] : m;
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) {  // the lane with the lower channels wins ties
           const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, m, o);
-          const int omi = __shfl_xor_sync(0xffffffffu, mi, o);
-          if (oam > am || (oam == am && omi < mi)) { am = oam; m = om; mi = omi; }
+          if (oam > am || (oam == am && (li & o))) { am = oam; m = om; }
         }
         const int half = 1 << (bits - 1);
         sh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
         d = __half2float(sh);
         inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        // code = floor(x/d + 1/2) + half from the estimate r = x * inv + half + 1/2, whose error is
+        // below 2^-19 (|x/d| <= half <= 2^7); a fraction within 2^-16 of an integer sends the
+        // lane's group through the exact comparisons instead.
+        const float c0 = 0.5f + (float)half;
+        bool near = false;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          float k = 0.0f;
-          if (d != 0.0f) k = fminf(fmaxf(round_absmax(xg[v], d, inv), (float)(-half)), (float)(half - 1));
-          code[gl * NV + v] = (uint32_t)((int)k + half);
+          const float r = fmaf(xg[v], inv, c0);
+          const float k = floorf(r);
+          const float fr = r - k;
+          near |= (fr < (1.0f / 65536.0f)) | (fr > (1.0f - 1.0f / 65536.0f));
+          code[gl * NV + v] = (uint32_t)(int)fminf(k, (float)(2 * half - 1));
+        }
+        if (near && d != 0.0f) {
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            const float k = fminf(fmaxf(round_exact_absmax(xg[v], d, inv), (float)(-half)), (float)(half - 1));
+            code[gl * NV + v] = (uint32_t)((int)k + half);
+          }
         }
       } else if (FAM == FAM_MINMAX) {
         float mn = xg[0], mx = xg[0];
@@ -539,7 +552,11 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
 #pragma unroll
           for (int k = 0; k < 15; ++k) th[k] = __fmul_rn(q_nf4_mid[k], d);  // exact (<= 24 bits)
 #pragma unroll
-          for (int v = 0; v < NV; ++v) code[gl * NV + v] = d != 0.0f ? nf4_code(xg[v], th) : 7u;
+          for (int v = 0; v < NV; ++v) code[gl * NV + v] = nf4_code(xg[v], th);
+          if (d == 0.0f) {  // all-zero group: the zero level
+#pragma unroll
+            for (int v = 0; v < NV; ++v) code[gl * NV + v] = 7u;
+          }
         } else {  // ternary digits t + 1 into this row's byte accumulators (5 trits per byte)
           const float hh = __fmul_rn(d, 0.5f);
           if (ok) {
@@ -575,7 +592,23 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
       __syncwarp();
     }
   }
+}
+
+template <int FAM, int G>
+__global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, int side, const __half* __restrict__ src,
+                                                                  int n_new, unsigned total_ctas) {
+  rows_body<FAM, G>(L, side, src, n_new, blockIdx.x, gridDim.x);
   finish_append(L, n_new, total_ctas);
+}
+
+// K and V in one launch: blocks [0, kblocks) take the K rows, the rest the V rows.
+template <int FK, int GK, int FV, int GV>
+__global__ void __launch_bounds__(kRowThreads) append_kv_kernel(LayerDev L, const __half* __restrict__ k,
+                                                                const __half* __restrict__ v, int n_new,
+                                                                unsigned kblocks) {
+  if (blockIdx.x < kblocks) rows_body<FK, GK>(L, 0, k, n_new, blockIdx.x, kblocks);
+  else rows_body<FV, GV>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
+  finish_append(L, n_new, gridDim.x);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -681,11 +714,39 @@ static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
   return p;
 }
 
+typedef void (*KvKernel)(LayerDev, const __half*, const __half*, int, unsigned);
+
+// The (K, V) format pairs that have a single-launch append kernel.
+static KvKernel pick_kv_kernel(const LayerDev& L) {
+  const SideDev& K = L.s[0];
+  const SideDev& V = L.s[1];
+  if (K.fmt == KVQ_FMT_FP16 || V.fmt == KVQ_FMT_FP16 || K.fmt == KVQ_FMT_POLAR || K.fmt == KVQ_FMT_CART ||
+      V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART)
+    return nullptr;
+  const int fk = fam_of(K), fv = fam_of(V), gk = K.group, gv = V.group;
+#define KVQ_KV(FK_, GK_, FV_, GV_) \
+  if (fk == FK_ && gk == GK_ && fv == FV_ && gv == GV_) return append_kv_kernel<FK_, GK_, FV_, GV_>;
+  KVQ_KV(FAM_NF4, 64, FAM_ABSMAX, 64)
+  KVQ_KV(FAM_ABSMAX, 64, FAM_ABSMAX, 64)
+  KVQ_KV(FAM_ABSMAX, 128, FAM_ABSMAX, 128)
+  KVQ_KV(FAM_ABSMAX, 32, FAM_ABSMAX, 32)
+  KVQ_KV(FAM_MINMAX, 32, FAM_MINMAX, 32)
+  KVQ_KV(FAM_TERNARY, 8, FAM_TERNARY, 8)
+  KVQ_KV(FAM_SIGN, 4, FAM_SIGN, 4)
+#undef KVQ_KV
+  return nullptr;
+}
+
 cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, int /*max_len_before*/,
                           cudaStream_t st, int* launches) {
   const SidePlan pk = plan_side(L, 0, n_new), pv = plan_side(L, 1, n_new);
   if (!pk.kern || !pv.kern) return cudaErrorInvalidValue;
   const unsigned total = pk.blocks + pv.blocks;
+  if (KvKernel kv = pick_kv_kernel(L)) {
+    kv<<<total, kRowThreads, 0, st>>>(L, k, v, n_new, pk.blocks);
+    if (launches) *launches = 1;
+    return cudaGetLastError();
+  }
   pk.kern<<<pk.blocks, pk.threads, 0, st>>>(L, 0, k, n_new, total);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from kvq_harness import Case
-from quantized_decode_attention_append_b200 import synth
+from quantized_decode_attention_append_b200 import kvq, synth
 from quantized_decode_attention_append_b200.kvq import Config, Side
 
 pytestmark = pytest.mark.gpu
@@ -70,6 +70,18 @@ def test_mma_kernel_is_the_one_that_runs():
     names = " ".join(e.name for e in prof.events())
     assert "decode_tc_kernel" in names and "merge_kernel" in names
     assert "decode_generic_kernel" not in names
+    assert kvq.kvq_last_launch_count(c.cache.h) == 2
+
+
+def test_append_is_one_launch_for_common_pairs():
+    cfg = Config(n_layers=1, batch=2, n_kv_heads=2, n_q_heads=8, head_dim=128, capacity=128,
+                 k=Side("nf4", group=64), v=Side("int", 4, group=64), max_queries=8)
+    c = Case(cfg, 64)
+    k = synth.kv_rows(3, "k", 0, list(range(cfg.batch)), list(range(cfg.n_kv_heads)), [64], 128, "cuda")
+    v = synth.kv_rows(3, "v", 0, list(range(cfg.batch)), list(range(cfg.n_kv_heads)), [64], 128, "cuda")
+    c.cache.append(0, k, v)
+    torch.cuda.synchronize()
+    assert kvq.kvq_last_launch_count(c.cache.h) == 1
 
 
 def test_mma_long_sequence_many_splits():
