@@ -34,9 +34,11 @@
 // the pair of probabilities a score thread owns is one 32-bit word of P'.  P' is staged per warp in
 // rows of 12 words (16 halves + 4 pad), which keeps its stores and fragment loads conflict-free.
 
-enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32 };
+enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64 };
 
-template <int F> struct CodeBits { static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : F); };
+template <int F> struct CodeBits {
+  static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : F));
+};
 
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
@@ -111,6 +113,33 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t base, uint32_t w) {
   return v;
 }
 
+// Sign codes carry their scale in the operand: a value is +d (bit set) or -d, exact in fp16, so the
+// sign bit of the duplicated fp16 scale is flipped per element.
+// K: pairs (channels 2p, 2p+1) of one word of sign bits (LSB first) with the scales of its 8
+// groups of 4 (sv: 4 words of fp16 pairs).  Odd bits are first moved 15 places up, so pair p's two
+// signs sit 16 bits apart and one shift brings them to bits 15 and 31.
+__device__ __forceinline__ void sign_pairs_k(uint32_t w, const uint32_t* sv, uint32_t* out) {
+  const uint32_t t = ~w, th = t >> 16;
+  const uint32_t lo = (t & 0x5555u) | ((t << 15) & 0x55550000u);
+  const uint32_t hi = (th & 0x5555u) | ((th << 15) & 0x55550000u);
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const uint32_t dd = prmt(sv[p >> 2], sv[p >> 2], ((p >> 1) & 1) ? 0x3232u : 0x1010u);
+    out[p] = (((p < 8 ? lo : hi) << (15 - 2 * (p & 7))) & 0x80008000u) ^ dd;
+  }
+}
+// V: pairs (row A, row B) of element e of 16 sign bits per row (ab: row A's bits in the low half,
+// row B's in the high half) with the rows' scales of 4 groups of 4 (sa, sb: 2 words each).
+__device__ __forceinline__ void sign_pairs_v(uint32_t ab, const uint32_t* sa, const uint32_t* sb, uint32_t* out) {
+  const uint32_t t = ~ab;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int k = e >> 2;
+    const uint32_t dd = prmt(sa[k >> 1], sb[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
+    out[e] = ((t << (15 - e)) & 0x80008000u) ^ dd;
+  }
+}
+
 // ---- mbarrier and bulk-copy primitives
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -180,23 +209,29 @@ struct TcCfg {
   static constexpr int HALF = TILE / 2;                // tokens per half-tile range
   static constexpr int NSB = TPW / 16;                 // 16-token blocks per warp and tile
   static constexpr int RBK = D * KB / 8, RBV = D * VB / 8;
-  static constexpr int NGK = D / GK, NGV = D / GV;
-  static constexpr bool VSCALE = VF != CF_FP16;
+  static constexpr int NGK = D / GK, NGV = D / GV;       // scale groups per row (storage)
+  static constexpr bool KSGN = KF == CF_SIGN, VSGN = VF == CF_SIGN;  // scale inside the operand
+  static constexpr bool VSCALE = VF != CF_FP16 && !VSGN;  // V scale folded into P'
+  static constexpr bool VSROW = VF != CF_FP16;            // V rows carry scales
+  static constexpr int GKM = KSGN ? D : GK, GVM = VSGN ? D : GV;  // channels per accumulation group
+  static constexpr int NGKM = D / GKM, NGVM = D / GVM;
   static constexpr int NPV = VSCALE ? NGV : 1;         // distinct P' operands (one per V group)
-  static constexpr int GKB = GK * KB / 8, GVB = GV * VB / 8;  // bytes of a group in a row
+  static constexpr int GKB = GKM * KB / 8, GVB = GVM * VB / 8;  // bytes of an accumulation group in a row
   static constexpr int KCB = GKB / 4, KCW = KCB / 4;   // a thread's K chunk of a group
   static constexpr int VCB = GVB / 8;                  // a thread's V chunk of a group (bytes)
   static constexpr int VCW = VCB >= 4 ? VCB / 4 : 1;
   static constexpr int VCH = VCB / 2;                  // 16-bit halves of the V chunk
-  static constexpr int KSTEPS = GK / 16, MT = GV / 16;
+  static constexpr int KSTEPS = GKM / 16, MT = GVM / 16;
+  static constexpr int KCS = KSGN ? (D / 4 / GK) * 2 : 0;  // bytes of a K chunk's scales (sign)
+  static constexpr int VCS = VSGN ? (D / 8 / GV) * 2 : 0;  // bytes of a V chunk's scales (sign)
   static constexpr bool ALT = RBK >= 128;              // row -> (half, index) mapping
   // log2 headroom of p over the running max: |d_v| <= 65504 / 2^(b-1) for b-bit absmax V, so
-  // p <= 2^(b-1) keeps p * d_v finite in fp16; fp16 V has no scale.
+  // p <= 2^(b-1) keeps p * d_v finite in fp16; P' carries no scale for fp16 and sign V.
   static constexpr float SLACK = VSCALE ? (float)(VB - 1) : 8.0f;
-  static constexpr int PADK = RBK >= 128 ? 64 : 32, PADV = RBV >= 128 ? 64 : 32, PADS = 16;
+  static constexpr int PADK = RBK == 64 ? 32 : 64, PADV = RBV == 64 ? 32 : 64, PADS = 16;
   // stage: [K codes A | pad | K codes B][K scales A | pad | B][V codes A | pad | B][V scales A | pad | B]
   static constexpr int KC_H = HALF * RBK, KS_H = HALF * NGK * 2;
-  static constexpr int VC_H = HALF * RBV, VS_H = VSCALE ? HALF * NGV * 2 : 0;
+  static constexpr int VC_H = HALF * RBV, VS_H = VSROW ? HALF * NGV * 2 : 0;
   static constexpr int OFF_KA = 0, OFF_KB = OFF_KA + KC_H + PADK;
   static constexpr int OFF_KSA = OFF_KB + KC_H, OFF_KSB = OFF_KSA + KS_H + PADS;
   static constexpr int OFF_VA = OFF_KSB + KS_H, OFF_VB = OFF_VA + VC_H + PADV;
@@ -261,7 +296,7 @@ __device__ void prepare_query_rot(const LayerDev& L, const __half* __restrict__ 
 // Element pair (e1, e2) of a thread's K chunk that pair index p covers.
 template <int KF>
 __device__ __forceinline__ void k_pair_elems(int p, int& e1, int& e2) {
-  if (KF == CF_NF4) {
+  if (KF == CF_NF4 || KF == CF_SIGN) {
     e1 = 2 * p;
     e2 = 2 * p + 1;
   } else {
@@ -300,7 +335,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   const uint8_t* gK = K.codes + u * L.Tcap * C::RBK;
   const uint8_t* gKs = reinterpret_cast<const uint8_t*>(K.scales + u * L.Tcap * C::NGK);
   const uint8_t* gV = V.codes + u * L.Tcap * C::RBV;
-  const uint8_t* gVs = C::VSCALE ? reinterpret_cast<const uint8_t*>(V.scales + u * L.Tcap * C::NGV) : nullptr;
+  const uint8_t* gVs = C::VSROW ? reinterpret_cast<const uint8_t*>(V.scales + u * L.Tcap * C::NGV) : nullptr;
 
   auto issue = [&](int tile_idx, int stage) {  // one thread: eight bulk copies (six for fp16 V)
     const long long t0 = tstart + (long long)tile_idx * C::TILE, t1 = t0 + C::HALF;
@@ -314,7 +349,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     bulk_g2s(st + C::OFF_KSB, gKs + t1 * C::NGK * 2, C::KS_H, b);
     bulk_g2s(st + C::OFF_VA, gV + t0 * C::RBV, C::VC_H, b);
     bulk_g2s(st + C::OFF_VB, gV + t1 * C::RBV, C::VC_H, b);
-    if (C::VSCALE) {
+    if (C::VSROW) {
       bulk_g2s(st + C::OFF_VSA, gVs + t0 * C::NGV * 2, C::VS_H, b);
       bulk_g2s(st + C::OFF_VSB, gVs + t1 * C::NGV * 2, C::VS_H, b);
     }
@@ -344,12 +379,12 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   }
   float* qs = reinterpret_cast<float*>(smem + C::OFF_PK);
   prepare_query_rot<D>(L, q, qi, kvh, G, qs);
-  uint32_t qreg[C::NGK][C::KSTEPS][2];
+  uint32_t qreg[C::NGKM][C::KSTEPS][2];
   {
     const int h = g >> 1, part = g & 1;
 #pragma unroll
-    for (int j = 0; j < C::NGK; ++j) {
-      const int cb = j * GK + c * (GK / 4);
+    for (int j = 0; j < C::NGKM; ++j) {
+      const int cb = j * C::GKM + c * (C::GKM / 4);
 #pragma unroll
       for (int ks = 0; ks < C::KSTEPS; ++ks) {
 #pragma unroll
@@ -384,6 +419,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   const int kc_off = (sh ? C::OFF_KB : C::OFF_KA) + (hb0 + si) * C::RBK + c * C::KCB;
   const int vs_off = (sh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + si) * C::NGV * 2;
   const int vc_off = (vh ? C::OFF_VB : C::OFF_VA) + (hb0 + vi) * C::RBV + g * C::VCB;
+  const int vsc_off = (vh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + vi) * C::NGV * 2 + g * C::VCS;  // sign V
   const int st_tok = sh * C::HALF + hb0 + si;  // tile-relative token of score row g, block 0
   const int vt_tok = vh * C::HALF + hb0 + vi;  // tile-relative token of V row c, block 0
   bool timed_out = false;
@@ -407,6 +443,33 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     float sc[C::NSB][2];
 #pragma unroll
     for (int sb = 0; sb < C::NSB; ++sb) {
+      if constexpr (C::KSGN) {  // scale inside the operand: one accumulator over the row
+        const unsigned char* k0p = st + kc_off + sb * 8 * C::RBK;
+        const unsigned char* s0p = st + ks_off + sb * 8 * C::NGK * 2 + c * C::KCS;
+        uint32_t kw0[C::KCW], kw1[C::KCW], sv0[C::KCS / 4], sv1[C::KCS / 4];
+        lds_words<C::KCW>(k0p, kw0);
+        lds_words<C::KCW>(k0p + 4 * C::RBK, kw1);
+        lds_words<C::KCS / 4>(s0p, sv0);
+        lds_words<C::KCS / 4>(s0p + 4 * C::NGK * 2, sv1);
+        uint32_t kp0[2 * C::KSTEPS], kp1[2 * C::KSTEPS];
+#pragma unroll
+        for (int w = 0; w < C::KCW; ++w) {
+          sign_pairs_k(kw0[w], sv0 + 4 * w, kp0 + 16 * w);
+          sign_pairs_k(kw1[w], sv1 + 4 * w, kp1 + 16 * w);
+        }
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS; ++ks)
+          mma16816(acc, kp0[2 * ks], kp1[2 * ks], kp0[2 * ks + 1], kp1[2 * ks + 1], qreg[0][ks][0], qreg[0][ks][1]);
+        float s0 = acc[0] + acc[1], s1 = acc[2] + acc[3];
+        if (!full_tile) {
+          const int t0 = tile_t0 + st_tok + sb * 8, t1 = t0 + 4;
+          s0 = (t0 >= R.qa && t0 < R.qb) ? s0 : -INFINITY;
+          s1 = (t1 >= R.qa && t1 < R.qb) ? s1 : -INFINITY;
+        }
+        sc[sb][0] = s0;
+        sc[sb][1] = s1;
+      } else {
       float kd0[C::NGK], kd1[C::NGK];
       {
         const __half* s0p = reinterpret_cast<const __half*>(st + ks_off + sb * 8 * C::NGK * 2);
@@ -434,9 +497,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
         uint32_t kp0[2 * C::KSTEPS], kp1[2 * C::KSTEPS];
         if constexpr (KF == CF_NF4) {
 #pragma unroll
-          for (int w = 0; w < C::KCW; ++w)
-#pragma unroll
-            {
+          for (int w = 0; w < C::KCW; ++w) {
               kp0[4 * w + 0] = lut_pair<0>(lut, kw0[w]);
               kp0[4 * w + 1] = lut_pair<1>(lut, kw0[w]);
               kp0[4 * w + 2] = lut_pair<2>(lut, kw0[w]);
@@ -468,6 +529,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       }
       sc[sb][0] = s0;
       sc[sb][1] = s1;
+      }
     }
 
     // ---- online softmax (log2 domain) for head c over this warp's TPW tokens.  The reference
@@ -544,14 +606,15 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       }
       __syncwarp();
       uint32_t vmask_a = 0xFFFFFFFFu, vmask_c = 0xFFFFFFFFu;
-      if (VF == CF_FP16 && !full_tile) {  // unwritten fp16 rows may hold NaN; zero them (p is 0 there)
+      if ((VF == CF_FP16 || C::VSGN) && !full_tile) {  // unwritten rows may hold NaN (fp16 values or sign
+                                                        // scales); zero them (p is 0 there)
         const int t = tile_t0 + vt_tok + sb * 8;
         auto ok = [&](int d) { return t + d >= R.qa && t + d < R.qb; };
         vmask_a = (ok(0) ? 0x0000FFFFu : 0u) | (ok(4) ? 0xFFFF0000u : 0u);
         vmask_c = (ok(2) ? 0x0000FFFFu : 0u) | (ok(6) ? 0xFFFF0000u : 0u);
       }
 #pragma unroll
-      for (int gv = 0; gv < C::NGV; ++gv) {
+      for (int gv = 0; gv < C::NGVM; ++gv) {
         const uint32_t* pr = pk + ((C::VSCALE ? gv : 0) * 8 + g) * C::PKS;
         const uint32_t b0 = pr[c], b1 = pr[c + 4];
         const unsigned char* vp = st + vc_off + sb * 8 * C::RBV + gv * C::GVB;
@@ -565,8 +628,26 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
             lds_words<C::VCW>(vp + roff[i] * C::RBV, vw[i]);
           }
         }
-        uint32_t pa[GV / 8], pc[GV / 8];
-        if constexpr (VF == CF_FP16) {
+        uint32_t pa[C::GVM / 8], pc[C::GVM / 8];
+        if constexpr (C::VSGN) {  // rows (vi, vi+4) -> pa, (vi+2, vi+6) -> pc, scales of each row's 4 groups per half
+          const unsigned char* sp = st + vsc_off + sb * 8 * C::NGV * 2;
+          uint32_t s4[4][C::VCS / 4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) lds_words<C::VCS / 4>(sp + roff[i] * C::NGV * 2, s4[i]);
+#pragma unroll
+          for (int hh = 0; hh < C::VCH; ++hh) {
+            const int w = hh >> 1, hf = hh & 1;
+            sign_pairs_v(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), s4[0] + 2 * hh, s4[1] + 2 * hh, pa + 16 * hh);
+            sign_pairs_v(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), s4[2] + 2 * hh, s4[3] + 2 * hh, pc + 16 * hh);
+          }
+          if (!full_tile) {
+#pragma unroll
+            for (int e = 0; e < C::GVM / 8; ++e) {
+              pa[e] &= vmask_a;
+              pc[e] &= vmask_c;
+            }
+          }
+        } else if constexpr (VF == CF_FP16) {
 #pragma unroll
           for (int w = 0; w < C::VCW; ++w) {
             pa[2 * w] = prmt(vw[0][w], vw[1][w], 0x5410) & vmask_a;
@@ -616,10 +697,10 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       ml[(warp * 4 + c) * 2 + 1] = l_run;
     }
 #pragma unroll
-    for (int gv = 0; gv < C::NGV; ++gv)
+    for (int gv = 0; gv < C::NGVM; ++gv)
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt) {
-        const int ch = gv * GV + g * (GV / 8) + 2 * mt;
+        const int ch = gv * C::GVM + g * (C::GVM / 8) + 2 * mt;
         const float* o = oacc[gv * C::MT + mt];
         *reinterpret_cast<float2*>(red + (warp * 4 + c) * D + ch) =
             timed_out ? make_float2(0.0f, 0.0f) : make_float2(o[0] + o[1], o[2] + o[3]);

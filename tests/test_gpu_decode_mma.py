@@ -25,6 +25,7 @@ MMA_CASES = [
     (256, 4, Side("int", 4, group=128, rot=256), Side("fp16")),
     (256, 4, Side("int", 4, group=32), Side("int", 4, group=32)),
     (256, 4, Side("int", 4, group=128, rot=256, chan_scale=True), Side("int", 2, group=128, rot=256)),
+    (128, 4, Side("sign", group=4), Side("sign", group=4)),
 ]
 
 
@@ -58,8 +59,10 @@ def test_mma_decode_with_anchors(rule, n):
         c.decode_and_compare(l, q, kv_len=[600, 555])
 
 
-def test_mma_kernel_is_the_one_that_runs():
-    cfg, c = make(128, 4, Side("nf4", group=64), Side("int", 4, group=64), 512)
+@pytest.mark.parametrize("k,v", [(Side("nf4", group=64), Side("int", 4, group=64)),
+                                 (Side("sign", group=4), Side("sign", group=4))], ids=["nf4-int4", "sign"])
+def test_mma_kernel_is_the_one_that_runs(k, v):
+    cfg, c = make(128, 4, k, v, 512)
     q = synth.queries(1, 0, 2, cfg.n_q_heads, 128, 512).cuda()
     c.cache.decode(0, q)
     torch.cuda.synchronize()
