@@ -487,6 +487,7 @@ static int code_fmt(const SideDev& S, bool is_v) {
   if (S.fmt == KVQ_FMT_NF4 && !is_v) return CF_NF4;
   if (S.fmt == KVQ_FMT_FP16 && is_v) return CF_FP16;
   if (S.fmt == KVQ_FMT_SIGN) return CF_SIGN;
+  if (S.fmt == KVQ_FMT_TERNARY) return CF_TERN;
   if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && (S.bits == 4 || S.bits == 2)) return S.bits;
   return -1;
 }
@@ -510,6 +511,7 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
   KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
   KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2)
+  KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)

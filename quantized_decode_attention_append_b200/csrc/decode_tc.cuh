@@ -34,10 +34,11 @@
 // the pair of probabilities a score thread owns is one 32-bit word of P'.  P' is staged per warp in
 // rows of 12 words (16 halves + 4 pad), which keeps its stores and fragment loads conflict-free.
 
-enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64 };
+enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64, CF_TERN = 128 };
 
 template <int F> struct CodeBits {
-  static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : F));
+  // bits per value in the layout the operands are built from (ternary: transcoded 2-bit digits)
+  static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : (F == CF_TERN ? 2 : F)));
 };
 
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -76,7 +77,7 @@ __device__ __forceinline__ __half2 h2c(unsigned short bits) {
 
 // The 16/B field pairs of a 32-bit word of B-bit offset-binary codes as signed fp16 pairs:
 // out[k] = (field k, field k + 16/B), i.e. field k of each 16-bit half.
-template <int B>
+template <int B, int OFS = (1 << (B - 1))>
 __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out) {
   constexpr int PH = 16 / B;                 // fields per 16-bit half
   constexpr int PB = 8 / B;                  // fields per byte
@@ -88,7 +89,7 @@ __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out) {
     const uint32_t x = and_or(k < PB ? w : w8, M << s, 0x64006400u);  // 1024 + 2^s field
     // 2^-s and -(1024 2^-s + 2^(B-1)) as fp16 bit patterns
     const unsigned short scl = (unsigned short)((15 - s) << 10);
-    const float off = -(1024.0f / (float)(1 << s) + (float)(1 << (B - 1)));
+    const float off = -(1024.0f / (float)(1 << s) + (float)OFS);
     const __half2 r = __hfma2(u2h(x), h2c(scl), __float2half2_rn(off));
     out[k] = h2u(r);
   }
@@ -138,6 +139,15 @@ __device__ __forceinline__ void sign_pairs_v(uint32_t ab, const uint32_t* sa, co
     const uint32_t dd = prmt(sa[k >> 1], sb[k >> 1], (k & 1) ? 0x7632u : 0x5410u);
     out[e] = ((t << (15 - e)) & 0x80008000u) ^ dd;
   }
+}
+
+// Ternary: digits d = t + 1 (2-bit fields after transcoding) -> (d - 1) x scale, exact in fp16;
+// dd holds the scales of the two elements of each pair (low, high half).
+__device__ __forceinline__ void tern_pairs(uint32_t w, uint32_t dd, uint32_t* out) {
+  uint32_t r[8];
+  code_pairs<2, 1>(w, r);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = h2u(__hmul2(u2h(r[k]), u2h(dd)));
 }
 
 // ---- mbarrier and bulk-copy primitives
@@ -210,10 +220,12 @@ struct TcCfg {
   static constexpr int NSB = TPW / 16;                 // 16-token blocks per warp and tile
   static constexpr int RBK = D * KB / 8, RBV = D * VB / 8;
   static constexpr int NGK = D / GK, NGV = D / GV;       // scale groups per row (storage)
-  static constexpr bool KSGN = KF == CF_SIGN, VSGN = VF == CF_SIGN;  // scale inside the operand
-  static constexpr bool VSCALE = VF != CF_FP16 && !VSGN;  // V scale folded into P'
+  static constexpr bool KSGN = KF == CF_SIGN, VSGN = VF == CF_SIGN;
+  static constexpr bool KTRN = KF == CF_TERN, VTRN = VF == CF_TERN;  // rows transcoded per warp
+  static constexpr bool KSCL = KSGN || KTRN, VSCL = VSGN || VTRN;    // scale inside the operand
+  static constexpr bool VSCALE = VF != CF_FP16 && !VSCL;  // V scale folded into P'
   static constexpr bool VSROW = VF != CF_FP16;            // V rows carry scales
-  static constexpr int GKM = KSGN ? D : GK, GVM = VSGN ? D : GV;  // channels per accumulation group
+  static constexpr int GKM = KSCL ? D : GK, GVM = VSCL ? D : GV;  // channels per accumulation group
   static constexpr int NGKM = D / GKM, NGVM = D / GVM;
   static constexpr int NPV = VSCALE ? NGV : 1;         // distinct P' operands (one per V group)
   static constexpr int GKB = GKM * KB / 8, GVB = GVM * VB / 8;  // bytes of an accumulation group in a row
@@ -222,16 +234,21 @@ struct TcCfg {
   static constexpr int VCW = VCB >= 4 ? VCB / 4 : 1;
   static constexpr int VCH = VCB / 2;                  // 16-bit halves of the V chunk
   static constexpr int KSTEPS = GKM / 16, MT = GVM / 16;
-  static constexpr int KCS = KSGN ? (D / 4 / GK) * 2 : 0;  // bytes of a K chunk's scales (sign)
-  static constexpr int VCS = VSGN ? (D / 8 / GV) * 2 : 0;  // bytes of a V chunk's scales (sign)
+  static constexpr int KCS = KSCL ? (D / 4 / GK) * 2 : 0;  // bytes of a K chunk's scales (scale in operand)
+  static constexpr int VCS = VSCL ? (D / 8 / GV) * 2 : 0;  // bytes of a V chunk's scales (scale in operand)
+  // stored row bytes (ternary: 5 digits per byte) and the per-warp transcode buffers
+  static constexpr int RSK = KTRN ? (D + 4) / 5 : RBK, RSV = VTRN ? (D + 4) / 5 : RBV;
+  static constexpr int XH = (TPW / 2) * 32, XB = XH + 64;   // transcoded half (TPW/2 rows of 32 bytes), B offset
+  static constexpr int XSIDE = XB + XH;
+  static constexpr int XW = (KTRN ? XSIDE : 0) + (VTRN ? XSIDE : 0);  // per warp
   static constexpr bool ALT = RBK >= 128;              // row -> (half, index) mapping
   // log2 headroom of p over the running max: |d_v| <= 65504 / 2^(b-1) for b-bit absmax V, so
   // p <= 2^(b-1) keeps p * d_v finite in fp16; P' carries no scale for fp16 and sign V.
   static constexpr float SLACK = VSCALE ? (float)(VB - 1) : 8.0f;
   static constexpr int PADK = RBK == 64 ? 32 : 64, PADV = RBV == 64 ? 32 : 64, PADS = 16;
   // stage: [K codes A | pad | K codes B][K scales A | pad | B][V codes A | pad | B][V scales A | pad | B]
-  static constexpr int KC_H = HALF * RBK, KS_H = HALF * NGK * 2;
-  static constexpr int VC_H = HALF * RBV, VS_H = VSROW ? HALF * NGV * 2 : 0;
+  static constexpr int KC_H = HALF * RSK, KS_H = HALF * NGK * 2;
+  static constexpr int VC_H = HALF * RSV, VS_H = VSROW ? HALF * NGV * 2 : 0;
   static constexpr int OFF_KA = 0, OFF_KB = OFF_KA + KC_H + PADK;
   static constexpr int OFF_KSA = OFF_KB + KC_H, OFF_KSB = OFF_KSA + KS_H + PADS;
   static constexpr int OFF_VA = OFF_KSB + KS_H, OFF_VB = OFF_VA + VC_H + PADV;
@@ -246,11 +263,14 @@ struct TcCfg {
   static constexpr int PK_BYTES_RAW = NW * PK_WORDS * 4;
   static constexpr int QS_BYTES = 4 * D * 4;           // query staging aliases the P' area
   static constexpr int PK_BYTES = PK_BYTES_RAW > QS_BYTES ? PK_BYTES_RAW : QS_BYTES;
-  static constexpr int LUT_BYTES = KF == CF_NF4 ? 256 * 32 * 4 : 0;
-  static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_BAR = OFF_LUT + LUT_BYTES;
+  static constexpr int LUT_BYTES = (KF == CF_NF4 || KTRN || VTRN) ? 256 * 32 * 4 : 0;
+  static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_X = OFF_LUT + LUT_BYTES;
+  static constexpr int OFF_BAR = OFF_X + NW * XW;
   static constexpr int SMEM = OFF_BAR + STAGES * 8;
 
   static_assert(KCB % 4 == 0, "K chunks must be whole words");
+  static_assert(!(KTRN || VTRN) || (D == 128 && TPW == 32 && GK == 8 && GV == 8), "ternary instance shape");
+  static_assert(KF != CF_NF4 || !(VTRN), "one table per kernel");
   static_assert(VCB % 4 == 0 || VCB == 2, "V chunks must be whole words or one half");
   static_assert(KC_H % 128 == 0 && VC_H % 128 == 0 && KS_H % 128 == 0 && VS_H % 128 == 0,
                 "half ranges keep the bank position of what follows them");
@@ -308,6 +328,28 @@ __device__ __forceinline__ void k_pair_elems(int p, int& e1, int& e2) {
   }
 }
 
+// One ternary row (26 bytes, 5 base-3 digits per byte, 2-byte aligned) -> 8 words of 2-bit digits
+// (channel j at bits 2j) through the per-lane byte table at shared address `lutb`.
+__device__ __forceinline__ void tern_transcode(const unsigned char* src, unsigned char* dst, uint32_t lutb) {
+  uint32_t out[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) out[i] = 0u;
+#pragma unroll
+  for (int h = 0; h < 13; ++h) {
+    const uint32_t two = *reinterpret_cast<const uint16_t*>(src + 2 * h);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int b = 2 * h + q, bit = 10 * b, w = bit >> 5, sh = bit & 31;
+      const uint32_t dg = q ? lut_pair<1>(lutb, two) : lut_pair<0>(lutb, two);
+      if (w < 8) out[w] |= dg << sh;
+      if (sh > 22 && w + 1 < 8) out[w + 1] |= dg >> (32 - sh);
+    }
+  }
+  uint4* o = reinterpret_cast<uint4*>(dst);
+  o[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  o[1] = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
 template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
                                                             const int* __restrict__ seq_ids,
@@ -332,9 +374,9 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   const int it0 = split * per;
   const int nmy = max(0, min(ntiles, it0 + per) - it0);
 
-  const uint8_t* gK = K.codes + u * L.Tcap * C::RBK;
+  const uint8_t* gK = K.codes + u * L.Tcap * C::RSK;
   const uint8_t* gKs = reinterpret_cast<const uint8_t*>(K.scales + u * L.Tcap * C::NGK);
-  const uint8_t* gV = V.codes + u * L.Tcap * C::RBV;
+  const uint8_t* gV = V.codes + u * L.Tcap * C::RSV;
   const uint8_t* gVs = C::VSROW ? reinterpret_cast<const uint8_t*>(V.scales + u * L.Tcap * C::NGV) : nullptr;
 
   auto issue = [&](int tile_idx, int stage) {  // one thread: eight bulk copies (six for fp16 V)
@@ -343,12 +385,12 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     uint64_t* b = bar + stage;
     fence_proxy_async();
     mbar_expect_tx(b, C::TX_BYTES);
-    bulk_g2s(st + C::OFF_KA, gK + t0 * C::RBK, C::KC_H, b);
-    bulk_g2s(st + C::OFF_KB, gK + t1 * C::RBK, C::KC_H, b);
+    bulk_g2s(st + C::OFF_KA, gK + t0 * C::RSK, C::KC_H, b);
+    bulk_g2s(st + C::OFF_KB, gK + t1 * C::RSK, C::KC_H, b);
     bulk_g2s(st + C::OFF_KSA, gKs + t0 * C::NGK * 2, C::KS_H, b);
     bulk_g2s(st + C::OFF_KSB, gKs + t1 * C::NGK * 2, C::KS_H, b);
-    bulk_g2s(st + C::OFF_VA, gV + t0 * C::RBV, C::VC_H, b);
-    bulk_g2s(st + C::OFF_VB, gV + t1 * C::RBV, C::VC_H, b);
+    bulk_g2s(st + C::OFF_VA, gV + t0 * C::RSV, C::VC_H, b);
+    bulk_g2s(st + C::OFF_VB, gV + t1 * C::RSV, C::VC_H, b);
     if (C::VSROW) {
       bulk_g2s(st + C::OFF_VSA, gVs + t0 * C::NGV * 2, C::VS_H, b);
       bulk_g2s(st + C::OFF_VSB, gVs + t1 * C::NGV * 2, C::VS_H, b);
@@ -369,10 +411,21 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
 
   // ---- while the first tiles are in flight: NF4 table, query fragments
   const uint32_t lut = smem_u32(smem + C::OFF_LUT) + 4 * lane;
-  if constexpr (KF == CF_NF4) {
+  if constexpr (C::LUT_BYTES > 0) {
     uint32_t* t = reinterpret_cast<uint32_t*>(smem + C::OFF_LUT);
     for (int b = warp * 32 + lane; b < 256; b += NW * 32) {
-      const uint32_t v = pack_h2(d_nf4[b & 15], d_nf4[b >> 4]);
+      uint32_t v;
+      if constexpr (KF == CF_NF4) {
+        v = pack_h2(d_nf4[b & 15], d_nf4[b >> 4]);
+      } else {  // ternary byte -> its five digits as 2-bit fields (bytes above 242 do not occur)
+        v = 0u;
+        int r = b < 243 ? b : 0;
+#pragma unroll
+        for (int m = 0; m < 5; ++m) {
+          v |= (uint32_t)(r % 3) << (2 * m);
+          r /= 3;
+        }
+      }
 #pragma unroll 8
       for (int i = 0; i < 32; ++i) t[b * 32 + ((lane + i) & 31)] = v;  // lanes write distinct banks
     }
@@ -416,9 +469,13 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   const int vh = C::row_half(c), vi = C::row_index(c);
   const int hb0 = warp * (TPW / 2);
   const int ks_off = (sh ? C::OFF_KSB : C::OFF_KSA) + (hb0 + si) * C::NGK * 2;   // K scales, row g
-  const int kc_off = (sh ? C::OFF_KB : C::OFF_KA) + (hb0 + si) * C::RBK + c * C::KCB;
+  // codes are read from the stage, or for ternary from this warp's transcoded rows (base `smem`)
+  const int kc_off = C::KTRN ? C::OFF_X + warp * C::XW + (sh ? C::XB : 0) + si * C::RBK + c * C::KCB
+                             : (sh ? C::OFF_KB : C::OFF_KA) + (hb0 + si) * C::RBK + c * C::KCB;
   const int vs_off = (sh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + si) * C::NGV * 2;
-  const int vc_off = (vh ? C::OFF_VB : C::OFF_VA) + (hb0 + vi) * C::RBV + g * C::VCB;
+  const int vc_off = C::VTRN ? C::OFF_X + warp * C::XW + (C::KTRN ? C::XSIDE : 0) + (vh ? C::XB : 0) + vi * C::RBV +
+                                   g * C::VCB
+                             : (vh ? C::OFF_VB : C::OFF_VA) + (hb0 + vi) * C::RBV + g * C::VCB;
   const int vsc_off = (vh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + vi) * C::NGV * 2 + g * C::VCS;  // sign V
   const int st_tok = sh * C::HALF + hb0 + si;  // tile-relative token of score row g, block 0
   const int vt_tok = vh * C::HALF + hb0 + vi;  // tile-relative token of V row c, block 0
@@ -438,13 +495,25 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     const unsigned char* st = smem + stage * C::STAGE_BYTES;
     const int tile_t0 = tstart + (it0 + it) * C::TILE;
     const bool full_tile = tile_t0 >= R.qa && tile_t0 + C::TILE <= R.qb;
+    const unsigned char* kb_ = C::KTRN ? smem : st;  // base of K code reads
+    const unsigned char* vb_ = C::VTRN ? smem : st;  // base of V code reads
+    if constexpr (C::KTRN || C::VTRN) {  // lane l transcodes row (half l / 16, index l % 16) of this warp
+      const int R2 = lane >> 4, li = lane & 15;
+      unsigned char* xw = smem + C::OFF_X + warp * C::XW;
+      if constexpr (C::KTRN)
+        tern_transcode(st + (R2 ? C::OFF_KB : C::OFF_KA) + (hb0 + li) * C::RSK, xw + (R2 ? C::XB : 0) + li * 32, lut);
+      if constexpr (C::VTRN)
+        tern_transcode(st + (R2 ? C::OFF_VB : C::OFF_VA) + (hb0 + li) * C::RSV,
+                       xw + (C::KTRN ? C::XSIDE : 0) + (R2 ? C::XB : 0) + li * 32, lut);
+      __syncwarp();
+    }
 
     // ---- scores: thread (g, c) gets head c's logits of score rows g and g + 8 of each block
     float sc[C::NSB][2];
 #pragma unroll
     for (int sb = 0; sb < C::NSB; ++sb) {
-      if constexpr (C::KSGN) {  // scale inside the operand: one accumulator over the row
-        const unsigned char* k0p = st + kc_off + sb * 8 * C::RBK;
+      if constexpr (C::KSCL) {  // scale inside the operand: one accumulator over the row
+        const unsigned char* k0p = kb_ + kc_off + sb * 8 * C::RBK;
         const unsigned char* s0p = st + ks_off + sb * 8 * C::NGK * 2 + c * C::KCS;
         uint32_t kw0[C::KCW], kw1[C::KCW], sv0[C::KCS / 4], sv1[C::KCS / 4];
         lds_words<C::KCW>(k0p, kw0);
@@ -452,10 +521,18 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
         lds_words<C::KCS / 4>(s0p, sv0);
         lds_words<C::KCS / 4>(s0p + 4 * C::NGK * 2, sv1);
         uint32_t kp0[2 * C::KSTEPS], kp1[2 * C::KSTEPS];
+        if constexpr (C::KSGN) {
 #pragma unroll
-        for (int w = 0; w < C::KCW; ++w) {
-          sign_pairs_k(kw0[w], sv0 + 4 * w, kp0 + 16 * w);
-          sign_pairs_k(kw1[w], sv1 + 4 * w, kp1 + 16 * w);
+          for (int w = 0; w < C::KCW; ++w) {
+            sign_pairs_k(kw0[w], sv0 + 4 * w, kp0 + 16 * w);
+            sign_pairs_k(kw1[w], sv1 + 4 * w, kp1 + 16 * w);
+          }
+        } else {  // ternary, groups of 8: word w of the chunk spans groups 2w, 2w + 1 (halves of sv[w])
+#pragma unroll
+          for (int w = 0; w < C::KCW; ++w) {
+            tern_pairs(kw0[w], sv0[w], kp0 + 8 * w);
+            tern_pairs(kw1[w], sv1[w], kp1 + 8 * w);
+          }
         }
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -486,7 +563,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
           }
         }
       }
-      const unsigned char* k0p = st + kc_off + sb * 8 * C::RBK;
+      const unsigned char* k0p = kb_ + kc_off + sb * 8 * C::RBK;
       const unsigned char* k1p = k0p + 4 * C::RBK;
       float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
@@ -606,7 +683,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       }
       __syncwarp();
       uint32_t vmask_a = 0xFFFFFFFFu, vmask_c = 0xFFFFFFFFu;
-      if ((VF == CF_FP16 || C::VSGN) && !full_tile) {  // unwritten rows may hold NaN (fp16 values or sign
+      if ((VF == CF_FP16 || C::VSCL) && !full_tile) {  // unwritten rows may hold NaN (fp16 values or sign
                                                         // scales); zero them (p is 0 there)
         const int t = tile_t0 + vt_tok + sb * 8;
         auto ok = [&](int d) { return t + d >= R.qa && t + d < R.qb; };
@@ -617,7 +694,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       for (int gv = 0; gv < C::NGVM; ++gv) {
         const uint32_t* pr = pk + ((C::VSCALE ? gv : 0) * 8 + g) * C::PKS;
         const uint32_t b0 = pr[c], b1 = pr[c + 4];
-        const unsigned char* vp = st + vc_off + sb * 8 * C::RBV + gv * C::GVB;
+        const unsigned char* vp = vb_ + vc_off + sb * 8 * C::RBV + gv * C::GVB;
         uint32_t vw[4][C::VCW];
         constexpr int roff[4] = {0, 4, 2, 6};  // slots (2c, 2c+1) then (2c+8, 2c+9)
 #pragma unroll
@@ -629,7 +706,25 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
           }
         }
         uint32_t pa[C::GVM / 8], pc[C::GVM / 8];
-        if constexpr (C::VSGN) {  // rows (vi, vi+4) -> pa, (vi+2, vi+6) -> pc, scales of each row's 4 groups per half
+        if constexpr (C::VTRN) {  // rows (vi, vi+4) -> pa, (vi+2, vi+6) -> pc; half hh is group 2g + hh
+          const unsigned char* sp = st + vsc_off + sb * 8 * C::NGV * 2;
+          uint32_t s4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) s4[i] = *reinterpret_cast<const uint32_t*>(sp + roff[i] * C::NGV * 2);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t sel = hh ? 0x7632u : 0x5410u;
+            tern_pairs(prmt(vw[0][0], vw[1][0], sel), prmt(s4[0], s4[1], sel), pa + 8 * hh);
+            tern_pairs(prmt(vw[2][0], vw[3][0], sel), prmt(s4[2], s4[3], sel), pc + 8 * hh);
+          }
+          if (!full_tile) {
+#pragma unroll
+            for (int e = 0; e < C::GVM / 8; ++e) {
+              pa[e] &= vmask_a;
+              pc[e] &= vmask_c;
+            }
+          }
+        } else if constexpr (C::VSGN) {  // rows (vi, vi+4) -> pa, (vi+2, vi+6) -> pc, scales of each row's 4 groups per half
           const unsigned char* sp = st + vsc_off + sb * 8 * C::NGV * 2;
           uint32_t s4[4][C::VCS / 4];
 #pragma unroll

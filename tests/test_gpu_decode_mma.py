@@ -26,6 +26,7 @@ MMA_CASES = [
     (256, 4, Side("int", 4, group=32), Side("int", 4, group=32)),
     (256, 4, Side("int", 4, group=128, rot=256, chan_scale=True), Side("int", 2, group=128, rot=256)),
     (128, 4, Side("sign", group=4), Side("sign", group=4)),
+    (128, 4, Side("ternary", group=8), Side("ternary", group=8)),
 ]
 
 
@@ -60,7 +61,9 @@ def test_mma_decode_with_anchors(rule, n):
 
 
 @pytest.mark.parametrize("k,v", [(Side("nf4", group=64), Side("int", 4, group=64)),
-                                 (Side("sign", group=4), Side("sign", group=4))], ids=["nf4-int4", "sign"])
+                                 (Side("sign", group=4), Side("sign", group=4)),
+                                 (Side("ternary", group=8), Side("ternary", group=8))],
+                         ids=["nf4-int4", "sign", "ternary"])
 def test_mma_kernel_is_the_one_that_runs(k, v):
     cfg, c = make(128, 4, k, v, 512)
     q = synth.queries(1, 0, 2, cfg.n_q_heads, 128, 512).cuda()
