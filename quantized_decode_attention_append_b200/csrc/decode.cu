@@ -353,29 +353,37 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
 }
 
 // Pass 2: merge the splits of one (query, head), undo V's transform, add anchors, normalise.
-// One thread per channel; the split weights are computed in parallel first.
+// D x SP threads: thread (group sg, channel j) sums the splits s = sg (mod SP) of channel j, so
+// many splits (long sequences, few queries) are read with SP times more loads in flight; the
+// split weights are computed in parallel first.
 template <int D>
-__global__ void __launch_bounds__(D) merge_kernel(LayerDev L, const float* __restrict__ work, int n_split, int nsp,
-                                                  void* __restrict__ out, int out_fp32, float* __restrict__ lse) {
+constexpr int merge_groups() { return D >= 256 ? 4 : 512 / D; }
+
+template <int D>
+__global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L, const float* __restrict__ work,
+                                                                     int n_split, int nsp, void* __restrict__ out,
+                                                                     int out_fp32, float* __restrict__ lse) {
+  constexpr int SP = merge_groups<D>(), NT = D * SP, NWP = NT / 32;
   const int qh = blockIdx.x;  // qi * Hq + h
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, j = tid % D, sg = tid / D;
   const SideDev& V = L.s[1];
   const float* P = work + (long long)qh * nsp * (D + kPartStride);
   __shared__ float w[kMaxSplit + 1];
-  __shared__ float rm[D / 32], rl[D / 32];
+  __shared__ float rm[NWP], rl[NWP];
+  __shared__ float po[SP][D];
   __shared__ float ov[D], tmp[D];
   const int warp = tid >> 5, lane = tid & 31;
   // max of the partial maxima
   float M = -INFINITY;
-  for (int s = tid; s < nsp; s += D) M = fmaxf(M, P[s * (D + kPartStride)]);
+  for (int s = tid; s < nsp; s += NT) M = fmaxf(M, P[s * (D + kPartStride)]);
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) rm[warp] = M;
   __syncthreads();
   M = rm[0];
-  for (int i = 1; i < D / 32; ++i) M = fmaxf(M, rm[i]);
+  for (int i = 1; i < NWP; ++i) M = fmaxf(M, rm[i]);
   // weights and the normaliser
   float ls = 0.0f;
-  for (int s = tid; s < nsp; s += D) {
+  for (int s = tid; s < nsp; s += NT) {
     const float m = P[s * (D + kPartStride)];
     const float ws = (m == -INFINITY) ? 0.0f : exp2f(m - M);
     w[s] = ws;
@@ -385,19 +393,26 @@ __global__ void __launch_bounds__(D) merge_kernel(LayerDev L, const float* __res
   if (lane == 0) rl[warp] = ls;
   __syncthreads();
   float Ls = 0.0f;
-  for (int i = 0; i < D / 32; ++i) Ls += rl[i];
+  for (int i = 0; i < NWP; ++i) Ls += rl[i];
   {
     float acc = 0.0f;
-    const float* pj = P + kPartStride + tid;
+    const float* pj = P + kPartStride + j;
 #pragma unroll 8
-    for (int s = 0; s < n_split; ++s) acc += w[s] * pj[s * (D + kPartStride)];
+    for (int s = sg; s < n_split; s += SP) acc += w[s] * pj[s * (D + kPartStride)];
+    po[sg][j] = acc;
+  }
+  __syncthreads();
+  if (tid < D) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int g = 0; g < SP; ++g) acc += po[g][tid];
     ov[tid] = acc;
   }
   __syncthreads();
   if (V.rot == 128 || V.rot == 256) {
     const int n = V.rot;
     for (int h = 1; h < n; h <<= 1) {
-      for (int p = tid; p < D / 2; p += D) {
+      for (int p = tid; p < D / 2; p += NT) {
         const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
         const int i = (hi << __ffs(h)) | lo;
         const float a = ov[i], b = ov[i + h];
@@ -407,11 +422,11 @@ __global__ void __launch_bounds__(D) merge_kernel(LayerDev L, const float* __res
       __syncthreads();
     }
     const float rn = (n == 256) ? 0.0625f : 0.08838834764831845f;
-    ov[tid] *= rn;
+    if (tid < D) ov[tid] *= rn;
     __syncthreads();
   } else if (V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART) {
     // x_n = (1/N) [a_0 + b_0 (-1)^n + 2 sum_{f=1}^{63} (a_f cos(2 pi f n/N) - b_f sin(2 pi f n/N))]
-    tmp[tid] = ov[tid];
+    if (tid < D) tmp[tid] = ov[tid];
     __syncthreads();
     if (tid < 128) {
       const int n = tid;
@@ -427,13 +442,15 @@ __global__ void __launch_bounds__(D) merge_kernel(LayerDev L, const float* __res
     }
     __syncthreads();
   }
-  const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
-  float v = ov[tid];
-  if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + tid];
-  v *= inv;
-  if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + tid] = v;
-  else reinterpret_cast<__half*>(out)[(long long)qh * D + tid] = __float2half_rn(v);
-  if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  if (tid < D) {
+    const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
+    float v = ov[tid];
+    if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + tid];
+    v *= inv;
+    if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + tid] = v;
+    else reinterpret_cast<__half*>(out)[(long long)qh * D + tid] = __float2half_rn(v);
+    if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  }
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -455,7 +472,7 @@ static int generic_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
 static int mma_split_count(long long units, int ntiles, int slots) {
   int best = 1;
   double best_score = -1.0;
-  for (int n = 1; n <= 64 && n <= ntiles; ++n) {
+  for (int n = 1; n <= kMaxSplit && n <= ntiles; ++n) {
     const long long ctas = units * n;
     const long long waves = (ctas + slots - 1) / slots;
     const double eff = (double)ctas / (double)(waves * slots);
@@ -512,7 +529,7 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
   KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2)
   KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 16, 4)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 32, 3)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)
   KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 4, 16, 3)
@@ -576,7 +593,7 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     if (e != cudaSuccess) return e;
   }
   const int nsp = n_quant + (L.anchored ? 1 : 0);
-  merge_kernel<D><<<n_q * L.Hq, D, 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse);
+  merge_kernel<D><<<n_q * L.Hq, D * merge_groups<D>(), 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse);
   ++nl;
   if (launches) *launches = nl;
   return cudaGetLastError();

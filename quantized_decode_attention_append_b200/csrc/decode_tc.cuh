@@ -283,33 +283,48 @@ struct TcCfg {
   __device__ static __forceinline__ int row_index(int rho) { return ALT ? (rho >> 1) : ((rho & 1) + 2 * (rho >> 2)); }
 };
 
+// q' = H(c . q) x sm_scale log2 e for the G heads of kv-head kvh into qs[G][D].  Warp h < G takes
+// head h with D/32 contiguous values per lane: Hadamard stages below D/32 run in-lane, the rest by
+// xor-shuffles (same fp32 butterflies, same order h = 1, 2, ..., rot/2).
 template <int D>
 __device__ void prepare_query_rot(const LayerDev& L, const __half* __restrict__ q, int qi, int kvh, int G, float* qs) {
   const SideDev& K = L.s[0];
-  const int tid = threadIdx.x;
-  for (int e = tid; e < G * D; e += blockDim.x) {
-    const int h = e / D, j = e % D;
-    const float v = __half2float(q[((long long)qi * L.Hq + kvh * G + h) * D + j]);
-    qs[e] = K.chan_scale ? v * __half2float(K.chan[kvh * D + j]) : v;
-  }
-  __syncthreads();
-  if (K.rot == 128 || K.rot == 256) {
-    for (int h = 1; h < K.rot; h <<= 1) {
-      for (int e = tid; e < G * D / 2; e += blockDim.x) {
-        const int row = e / (D / 2), p = e % (D / 2);
-        const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
-        const int i = (hi << __ffs(h)) | lo;
-        float* r = qs + row * D;
-        const float a = r[i], b = r[i + h];
-        r[i] = a + b;
-        r[i + h] = a - b;
-      }
-      __syncthreads();
+  constexpr int V = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < G) {
+    const int h = warp, j0 = lane * V;
+    float x[V];
+    const __half* qp = q + ((long long)qi * L.Hq + kvh * G + h) * D + j0;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      x[v] = __half2float(qp[v]);
+      if (K.chan_scale) x[v] = x[v] * __half2float(K.chan[kvh * D + j0 + v]);
     }
+    if (K.rot == 128 || K.rot == 256) {
+#pragma unroll
+      for (int hh = 1; hh < V; hh <<= 1)
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+          if ((v & hh) == 0) {
+            const float a = x[v], b = x[v + hh];
+            x[v] = a + b;
+            x[v + hh] = a - b;
+          }
+      for (int hh = V; hh < K.rot; hh <<= 1) {
+        const int lm = hh / V;
+        const bool upper = (lane & lm) != 0;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          const float o = __shfl_xor_sync(0xffffffffu, x[v], lm);
+          x[v] = upper ? o - x[v] : x[v] + o;
+        }
+      }
+    }
+    const float rn = K.rot == 256 ? 0.0625f : (K.rot == 128 ? 0.08838834764831845f : 1.0f);
+    const float scl = L.sm_scale * kLog2e * rn;
+#pragma unroll
+    for (int v = 0; v < V; ++v) qs[h * D + j0 + v] = x[v] * scl;
   }
-  const float rn = K.rot == 256 ? 0.0625f : (K.rot == 128 ? 0.08838834764831845f : 1.0f);
-  const float scl = L.sm_scale * kLog2e * rn;
-  for (int e = tid; e < G * D; e += blockDim.x) qs[e] *= scl;
   __syncthreads();
 }
 
