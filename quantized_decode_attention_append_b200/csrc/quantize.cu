@@ -27,6 +27,8 @@
 
 namespace kvq {
 
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
 __constant__ float q_nf4_mid[15];
 __constant__ float q_tw_re[64];
 __constant__ float q_tw_im[64];
@@ -397,6 +399,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       }
     }
     float x[32];
+    __half2 raw2[16];  // the lane's 32 input values as stored (fp16 pairs)
     const __half* rp = src + ((long long)u * n_new + i) * D + li * 32;
     if (ok) {
 #pragma unroll
@@ -405,6 +408,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         const __half2* h2 = reinterpret_cast<const __half2*>(&w);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          raw2[c4 * 4 + e] = h2[e];
           const float2 f = __half22float2(h2[e]);
           x[c4 * 8 + 2 * e] = f.x;
           x[c4 * 8 + 2 * e + 1] = f.y;
@@ -423,6 +427,8 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     } else {
 #pragma unroll
       for (int v = 0; v < 32; ++v) x[v] = 0.0f;
+#pragma unroll
+      for (int v = 0; v < 16; ++v) raw2[v] = __float2half2_rn(0.0f);
     }
     if (S.rot) {  // stages h = 1 .. rot/2 (warp-uniform: every lane takes part in the shuffles)
 #pragma unroll
@@ -548,11 +554,30 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         sh = __float2half_rn(am);
         d = __half2float(sh);
         if (FAM == FAM_NF4) {
-          float th[15];
+          if (!S.rot && !S.chan_scale) {
+            // x is the fp16 input itself, so x >= th <=> x >= th rounded up to fp16: count the
+            // thresholds reached two values at a time in fp16 (1024 + count keeps the count in
+            // the low mantissa bits)
+            __half2 t2[15];
 #pragma unroll
-          for (int k = 0; k < 15; ++k) th[k] = __fmul_rn(q_nf4_mid[k], d);  // exact (<= 24 bits)
+            for (int k = 0; k < 15; ++k) t2[k] = __half2half2(__float2half_ru(__fmul_rn(q_nf4_mid[k], d)));
 #pragma unroll
-          for (int v = 0; v < NV; ++v) code[gl * NV + v] = nf4_code(xg[v], th);
+            for (int p2 = 0; p2 < NV / 2; ++p2) {
+              const __half2 xv = raw2[(gl * NV) / 2 + p2];
+              __half2 acc = __float2half2_rn(1024.0f);
+#pragma unroll
+              for (int k = 0; k < 15; ++k) acc = __hadd2(acc, __hge2(xv, t2[k]));
+              const uint32_t b = h2u(acc);
+              code[gl * NV + 2 * p2] = b & 0xFu;
+              code[gl * NV + 2 * p2 + 1] = (b >> 16) & 0xFu;
+            }
+          } else {
+            float th[15];
+#pragma unroll
+            for (int k = 0; k < 15; ++k) th[k] = __fmul_rn(q_nf4_mid[k], d);  // exact (<= 24 bits)
+#pragma unroll
+            for (int v = 0; v < NV; ++v) code[gl * NV + v] = nf4_code(xg[v], th);
+          }
           if (d == 0.0f) {  // all-zero group: the zero level
 #pragma unroll
             for (int v = 0; v < NV; ++v) code[gl * NV + v] = 7u;
