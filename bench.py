@@ -351,24 +351,28 @@ def run_gpu(args, w, name):
     row_io = 2 * 2 * D + row_bytes_of(cache, 0) + row_bytes_of(cache, 1)  # fp16 in + packed out, K and V
     quant_gbps = (q_rows * row_io) / (q_ms * 1e-3) / 1e9 if q_ms > 0 else None
 
-    # end to end through the public API with host buffers: H2D of the step's new rows and
-    # queries from pinned memory, D2H of the step's attention outputs (captured with the step)
-    h_k = [x.cpu().pin_memory() for x in knew]
-    h_v = [x.cpu().pin_memory() for x in vnew]
-    h_q = [x.cpu().pin_memory() for x in qs]
-    h_o = [torch.empty(B, Hq, D, dtype=torch.float32).pin_memory() for _ in range(L)]
-    d_k = [torch.empty_like(x) for x in knew]
-    d_v = [torch.empty_like(x) for x in vnew]
-    d_q = [torch.empty_like(x) for x in qs]
+    # end to end through the public API with host buffers: one H2D copy of the step's new rows and
+    # queries (all layers, packed in one pinned buffer), the appends and decodes, and one D2H copy
+    # of all layers' attention outputs (captured with the step)
+    parts = [x for l in range(L) for x in (knew[l], vnew[l], qs[l])]
+    padded = [(x.numel() + 63) // 64 * 64 for x in parts]  # 128-byte aligned pieces
+    h_in = torch.zeros(sum(padded), dtype=torch.float16).pin_memory()
+    views, off = [], 0
+    d_in = torch.empty_like(h_in, device=dev)
+    for x, n in zip(parts, padded):
+        h_in[off:off + x.numel()] = x.reshape(-1).cpu()
+        views.append(d_in[off:off + x.numel()].view(x.shape))
+        off += n
+    d_k, d_v, d_q = views[0::3], views[1::3], views[2::3]
+    d_out = torch.empty(L, B, Hq, D, device=dev, dtype=torch.float32)
+    h_out = torch.empty(L, B, Hq, D, dtype=torch.float32).pin_memory()
 
     def e2e_step():
+        d_in.copy_(h_in, non_blocking=True)
         for l in range(L):
-            d_k[l].copy_(h_k[l], non_blocking=True)
-            d_v[l].copy_(h_v[l], non_blocking=True)
-            d_q[l].copy_(h_q[l], non_blocking=True)
             cache.append(l, d_k[l], d_v[l])
-            cache.decode(l, d_q[l], out=outs[l])
-            h_o[l].copy_(outs[l], non_blocking=True)
+            cache.decode(l, d_q[l], out=d_out[l])
+        h_out.copy_(d_out, non_blocking=True)
 
     E = max(1, min(K_, 10))
     cache.set_seq_len(-1, T0 + W_ - 1)
@@ -384,8 +388,8 @@ def run_gpu(args, w, name):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / E
     e2e_ms = max_over_ranks([e2e_ms], dev)[0]
-    h2d = sum(x.numel() * x.element_size() for x in h_k + h_v + h_q)
-    d2h = sum(x.numel() * x.element_size() for x in h_o)
+    h2d = h_in.numel() * h_in.element_size()
+    d2h = h_out.numel() * h_out.element_size()
 
     rec = None
     if rank == 0:

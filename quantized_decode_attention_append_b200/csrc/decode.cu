@@ -467,8 +467,10 @@ static int generic_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
   return (int)s;
 }
 
-// Tensor-core path: pick the split count whose grid fills whole waves of resident CTAs and whose
-// splits hold whole tiles, preferring fewer splits on ties.
+// Tensor-core path: the split count that maximises (busy fraction of the resident-CTA slots over
+// whole waves) x (balance of tiles across splits) x per / (per + F), where a CTA's fixed cost F
+// (query transform and fragments, table build, warp combine, partial write) is about 0.75 tiles of
+// streaming; ties go to fewer splits.
 static int mma_split_count(long long units, int ntiles, int slots) {
   int best = 1;
   double best_score = -1.0;
@@ -478,7 +480,7 @@ static int mma_split_count(long long units, int ntiles, int slots) {
     const double eff = (double)ctas / (double)(waves * slots);
     const int per = (ntiles + n - 1) / n;
     const double bal = (double)ntiles / (double)(per * n);
-    const double score = eff * bal - (per < 4 ? 0.05 : 0.0);
+    const double score = eff * bal * (double)per / ((double)per + 0.75);
     if (score > best_score + 1e-9) {
       best_score = score;
       best = n;
@@ -506,6 +508,7 @@ static int code_fmt(const SideDev& S, bool is_v) {
   if (S.fmt == KVQ_FMT_SIGN) return CF_SIGN;
   if (S.fmt == KVQ_FMT_TERNARY) return CF_TERN;
   if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && (S.bits == 4 || S.bits == 2)) return S.bits;
+  if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && S.bits == 3 && is_v) return CF_INT3;
   return -1;
 }
 
@@ -530,6 +533,7 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2)
   KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 32, 3)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT3, 128, 4, 32, 3)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)
   KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 4, 16, 3)

@@ -34,11 +34,12 @@
 // the pair of probabilities a score thread owns is one 32-bit word of P'.  P' is staged per warp in
 // rows of 12 words (16 halves + 4 pad), which keeps its stores and fragment loads conflict-free.
 
-enum CodeFmt { CF_INT2 = 2, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64, CF_TERN = 128 };
+enum CodeFmt { CF_INT2 = 2, CF_INT3 = 3, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64, CF_TERN = 128 };
 
 template <int F> struct CodeBits {
   // bits per value in the layout the operands are built from (ternary: transcoded 2-bit digits)
-  static constexpr int v = F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : (F == CF_TERN ? 2 : F)));
+  static constexpr int v =
+      F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : (F == CF_TERN ? 2 : (F == CF_INT3 ? 4 : F))));
 };
 
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -221,7 +222,10 @@ struct TcCfg {
   static constexpr int RBK = D * KB / 8, RBV = D * VB / 8;
   static constexpr int NGK = D / GK, NGV = D / GV;       // scale groups per row (storage)
   static constexpr bool KSGN = KF == CF_SIGN, VSGN = VF == CF_SIGN;
-  static constexpr bool KTRN = KF == CF_TERN, VTRN = VF == CF_TERN;  // rows transcoded per warp
+  static constexpr bool KTRN = KF == CF_TERN, VTRN = VF == CF_TERN;  // ternary rows transcoded per warp
+  static constexpr bool V3 = VF == CF_INT3;                          // int3 V rows transcoded to nibbles
+  static constexpr bool VX = VTRN || V3;                             // V read from the transcode buffer
+  static constexpr int VOFS = V3 ? 4 : (1 << (VB - 1));              // code offset of the V fields
   static constexpr bool KSCL = KSGN || KTRN, VSCL = VSGN || VTRN;    // scale inside the operand
   static constexpr bool VSCALE = VF != CF_FP16 && !VSCL;  // V scale folded into P'
   static constexpr bool VSROW = VF != CF_FP16;            // V rows carry scales
@@ -237,14 +241,15 @@ struct TcCfg {
   static constexpr int KCS = KSCL ? (D / 4 / GK) * 2 : 0;  // bytes of a K chunk's scales (scale in operand)
   static constexpr int VCS = VSCL ? (D / 8 / GV) * 2 : 0;  // bytes of a V chunk's scales (scale in operand)
   // stored row bytes (ternary: 5 digits per byte) and the per-warp transcode buffers
-  static constexpr int RSK = KTRN ? (D + 4) / 5 : RBK, RSV = VTRN ? (D + 4) / 5 : RBV;
-  static constexpr int XH = (TPW / 2) * 32, XB = XH + 64;   // transcoded half (TPW/2 rows of 32 bytes), B offset
-  static constexpr int XSIDE = XB + XH;
-  static constexpr int XW = (KTRN ? XSIDE : 0) + (VTRN ? XSIDE : 0);  // per warp
+  static constexpr int RSK = KTRN ? (D + 4) / 5 : RBK, RSV = VTRN ? (D + 4) / 5 : (V3 ? D * 3 / 8 : RBV);
+  // transcode buffers per warp: half A (TPW/2 rows), pad, half B, for K then V
+  static constexpr int XKH = (TPW / 2) * RBK, XKB = XKH + (RBK == 64 ? 32 : 64), XKS = KTRN ? XKB + XKH : 0;
+  static constexpr int XVH = (TPW / 2) * RBV, XVB = XVH + (RBV == 64 ? 32 : 64), XVS = VX ? XVB + XVH : 0;
+  static constexpr int XW = XKS + XVS;  // per warp
   static constexpr bool ALT = RBK >= 128;              // row -> (half, index) mapping
   // log2 headroom of p over the running max: |d_v| <= 65504 / 2^(b-1) for b-bit absmax V, so
   // p <= 2^(b-1) keeps p * d_v finite in fp16; P' carries no scale for fp16 and sign V.
-  static constexpr float SLACK = VSCALE ? (float)(VB - 1) : 8.0f;
+  static constexpr float SLACK = VSCALE ? (float)((V3 ? 3 : VB) - 1) : 8.0f;
   static constexpr int PADK = RBK == 64 ? 32 : 64, PADV = RBV == 64 ? 32 : 64, PADS = 16;
   // stage: [K codes A | pad | K codes B][K scales A | pad | B][V codes A | pad | B][V scales A | pad | B]
   static constexpr int KC_H = HALF * RSK, KS_H = HALF * NGK * 2;
@@ -270,6 +275,7 @@ struct TcCfg {
 
   static_assert(KCB % 4 == 0, "K chunks must be whole words");
   static_assert(!(KTRN || VTRN) || (D == 128 && TPW == 32 && GK == 8 && GV == 8), "ternary instance shape");
+  static_assert(!V3 || (TPW == 32 && GV >= 16), "int3 V instance shape");
   static_assert(KF != CF_NF4 || !(VTRN), "one table per kernel");
   static_assert(VCB % 4 == 0 || VCB == 2, "V chunks must be whole words or one half");
   static_assert(KC_H % 128 == 0 && VC_H % 128 == 0 && KS_H % 128 == 0 && VS_H % 128 == 0,
@@ -363,6 +369,33 @@ __device__ __forceinline__ void tern_transcode(const unsigned char* src, unsigne
   uint4* o = reinterpret_cast<uint4*>(dst);
   o[0] = make_uint4(out[0], out[1], out[2], out[3]);
   o[1] = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+// One int3 row (D fields of 3 bits, LSB first, 16-byte aligned) -> D 4-bit fields (nibble j =
+// field j).  Each output word takes 24 input bits (a funnel shift), splits them into two 12-bit
+// halves at bits 0 and 16, and spreads 3-bit fields to nibbles in two shift-and-mask steps.
+template <int D>
+__device__ __forceinline__ void int3_transcode(const unsigned char* src, unsigned char* dst) {
+  constexpr int NIN = D * 3 / 32, NOUT = D / 8;
+  uint32_t in[NIN + 1];
+#pragma unroll
+  for (int i = 0; i < NIN; i += 4) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i / 4];
+    in[i] = v.x; in[i + 1] = v.y; in[i + 2] = v.z; in[i + 3] = v.w;
+  }
+  in[NIN] = 0u;
+  uint32_t out[NOUT];
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    const int bit = 24 * o, wi = bit >> 5, sh = bit & 31;
+    const uint32_t g = __funnelshift_r(in[wi], in[wi + 1], sh);              // fields 8o .. 8o + 7 in bits 0..23
+    const uint32_t t = (g & 0x00000FFFu) | ((g << 4) & 0x0FFF0000u);          // halves at bits 0 and 16
+    const uint32_t x1 = (t & 0x003F003Fu) | ((t << 2) & 0x3F003F00u);         // fields 2, 3 up by 2
+    out[o] = (x1 & 0x07070707u) | ((x1 << 1) & 0x70707070u);                  // fields 1, 3 up by 1
+  }
+#pragma unroll
+  for (int o = 0; o < NOUT; o += 4)
+    reinterpret_cast<uint4*>(dst)[o / 4] = make_uint4(out[o], out[o + 1], out[o + 2], out[o + 3]);
 }
 
 template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
@@ -485,10 +518,10 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   const int hb0 = warp * (TPW / 2);
   const int ks_off = (sh ? C::OFF_KSB : C::OFF_KSA) + (hb0 + si) * C::NGK * 2;   // K scales, row g
   // codes are read from the stage, or for ternary from this warp's transcoded rows (base `smem`)
-  const int kc_off = C::KTRN ? C::OFF_X + warp * C::XW + (sh ? C::XB : 0) + si * C::RBK + c * C::KCB
+  const int kc_off = C::KTRN ? C::OFF_X + warp * C::XW + (sh ? C::XKB : 0) + si * C::RBK + c * C::KCB
                              : (sh ? C::OFF_KB : C::OFF_KA) + (hb0 + si) * C::RBK + c * C::KCB;
   const int vs_off = (sh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + si) * C::NGV * 2;
-  const int vc_off = C::VTRN ? C::OFF_X + warp * C::XW + (C::KTRN ? C::XSIDE : 0) + (vh ? C::XB : 0) + vi * C::RBV +
+  const int vc_off = C::VX ? C::OFF_X + warp * C::XW + C::XKS + (vh ? C::XVB : 0) + vi * C::RBV +
                                    g * C::VCB
                              : (vh ? C::OFF_VB : C::OFF_VA) + (hb0 + vi) * C::RBV + g * C::VCB;
   const int vsc_off = (vh ? C::OFF_VSB : C::OFF_VSA) + (hb0 + vi) * C::NGV * 2 + g * C::VCS;  // sign V
@@ -511,15 +544,18 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     const int tile_t0 = tstart + (it0 + it) * C::TILE;
     const bool full_tile = tile_t0 >= R.qa && tile_t0 + C::TILE <= R.qb;
     const unsigned char* kb_ = C::KTRN ? smem : st;  // base of K code reads
-    const unsigned char* vb_ = C::VTRN ? smem : st;  // base of V code reads
-    if constexpr (C::KTRN || C::VTRN) {  // lane l transcodes row (half l / 16, index l % 16) of this warp
+    const unsigned char* vb_ = C::VX ? smem : st;    // base of V code reads
+    if constexpr (C::KTRN || C::VX) {  // lane l transcodes row (half l / 16, index l % 16) of this warp
       const int R2 = lane >> 4, li = lane & 15;
       unsigned char* xw = smem + C::OFF_X + warp * C::XW;
       if constexpr (C::KTRN)
-        tern_transcode(st + (R2 ? C::OFF_KB : C::OFF_KA) + (hb0 + li) * C::RSK, xw + (R2 ? C::XB : 0) + li * 32, lut);
+        tern_transcode(st + (R2 ? C::OFF_KB : C::OFF_KA) + (hb0 + li) * C::RSK, xw + (R2 ? C::XKB : 0) + li * 32, lut);
       if constexpr (C::VTRN)
         tern_transcode(st + (R2 ? C::OFF_VB : C::OFF_VA) + (hb0 + li) * C::RSV,
-                       xw + (C::KTRN ? C::XSIDE : 0) + (R2 ? C::XB : 0) + li * 32, lut);
+                       xw + C::XKS + (R2 ? C::XVB : 0) + li * 32, lut);
+      if constexpr (C::V3)
+        int3_transcode<D>(st + (R2 ? C::OFF_VB : C::OFF_VA) + (hb0 + li) * C::RSV,
+                           xw + C::XKS + (R2 ? C::XVB : 0) + li * C::RBV);
       __syncwarp();
     }
 
@@ -770,8 +806,8 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
 #pragma unroll
           for (int hh = 0; hh < C::VCH; ++hh) {
             const int w = hh >> 1, hf = hh & 1;
-            code_pairs<C::VB>(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), pa + hh * PH);
-            code_pairs<C::VB>(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), pc + hh * PH);
+            code_pairs<C::VB, C::VOFS>(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), pa + hh * PH);
+            code_pairs<C::VB, C::VOFS>(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), pc + hh * PH);
           }
         }
 #pragma unroll

@@ -564,10 +564,12 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
 #pragma unroll
             for (int p2 = 0; p2 < NV / 2; ++p2) {
               const __half2 xv = raw2[(gl * NV) / 2 + p2];
-              __half2 acc = __float2half2_rn(1024.0f);
+              // four short chains instead of one long one (the one-token append is latency-bound)
+              __half2 a[4] = {__float2half2_rn(1024.0f), __float2half2_rn(0.0f), __float2half2_rn(0.0f),
+                              __float2half2_rn(0.0f)};
 #pragma unroll
-              for (int k = 0; k < 15; ++k) acc = __hadd2(acc, __hge2(xv, t2[k]));
-              const uint32_t b = h2u(acc);
+              for (int k = 0; k < 15; ++k) a[k & 3] = __hadd2(a[k & 3], __hge2(xv, t2[k]));
+              const uint32_t b = h2u(__hadd2(__hadd2(a[0], a[1]), __hadd2(a[2], a[3])));
               code[gl * NV + 2 * p2] = b & 0xFu;
               code[gl * NV + 2 * p2 + 1] = (b >> 16) & 0xFu;
             }

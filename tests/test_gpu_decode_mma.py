@@ -27,6 +27,7 @@ MMA_CASES = [
     (256, 4, Side("int", 4, group=128, rot=256, chan_scale=True), Side("int", 2, group=128, rot=256)),
     (128, 4, Side("sign", group=4), Side("sign", group=4)),
     (128, 4, Side("ternary", group=8), Side("ternary", group=8)),
+    (256, 4, Side("int", 4, group=128, rot=256), Side("int", 3, group=128, rot=256)),
 ]
 
 
