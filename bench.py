@@ -351,28 +351,46 @@ def run_gpu(args, w, name):
     row_io = 2 * 2 * D + row_bytes_of(cache, 0) + row_bytes_of(cache, 1)  # fp16 in + packed out, K and V
     quant_gbps = (q_rows * row_io) / (q_ms * 1e-3) / 1e9 if q_ms > 0 else None
 
-    # end to end through the public API with host buffers: one H2D copy of the step's new rows and
-    # queries (all layers, packed in one pinned buffer), the appends and decodes, and one D2H copy
-    # of all layers' attention outputs (captured with the step)
-    parts = [x for l in range(L) for x in (knew[l], vnew[l], qs[l])]
-    padded = [(x.numel() + 63) // 64 * 64 for x in parts]  # 128-byte aligned pieces
-    h_in = torch.zeros(sum(padded), dtype=torch.float16).pin_memory()
-    views, off = [], 0
+    # end to end through the public API with host buffers: every step copies its new rows and
+    # queries in from pinned memory and its attention outputs back out.  A copy stream moves layer
+    # l's inputs in (one copy per layer) and layer l's outputs out while other layers compute; the
+    # compute stream waits for each layer's inputs (captured with the step, fork/join in the graph).
+    parts = [[knew[l], vnew[l], qs[l]] for l in range(L)]
+    lay = [sum((x.numel() + 63) // 64 * 64 for x in p) for p in parts]  # 128-byte aligned pieces
+    h_in = torch.zeros(sum(lay), dtype=torch.float16).pin_memory()
     d_in = torch.empty_like(h_in, device=dev)
-    for x, n in zip(parts, padded):
-        h_in[off:off + x.numel()] = x.reshape(-1).cpu()
-        views.append(d_in[off:off + x.numel()].view(x.shape))
-        off += n
-    d_k, d_v, d_q = views[0::3], views[1::3], views[2::3]
+    d_k, d_v, d_q, spans, off = [], [], [], [], 0
+    for l in range(L):
+        start = off
+        for x, dst in zip(parts[l], (d_k, d_v, d_q)):
+            h_in[off:off + x.numel()] = x.reshape(-1).cpu()
+            dst.append(d_in[off:off + x.numel()].view(x.shape))
+            off += (x.numel() + 63) // 64 * 64
+        spans.append((start, off))
     d_out = torch.empty(L, B, Hq, D, device=dev, dtype=torch.float32)
     h_out = torch.empty(L, B, Hq, D, dtype=torch.float32).pin_memory()
+    copy_stream = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(L)]
+    ev_out = [torch.cuda.Event() for _ in range(L)]
 
     def e2e_step():
-        d_in.copy_(h_in, non_blocking=True)
+        main = torch.cuda.current_stream(dev)
+        copy_stream.wait_stream(main)
+        with torch.cuda.stream(copy_stream):
+            for l in range(L):
+                a, b = spans[l]
+                d_in[a:b].copy_(h_in[a:b], non_blocking=True)
+                ev_in[l].record(copy_stream)
         for l in range(L):
+            main.wait_event(ev_in[l])
             cache.append(l, d_k[l], d_v[l])
             cache.decode(l, d_q[l], out=d_out[l])
-        h_out.copy_(d_out, non_blocking=True)
+            ev_out[l].record(main)
+        with torch.cuda.stream(copy_stream):
+            for l in range(L):
+                copy_stream.wait_event(ev_out[l])
+                h_out[l].copy_(d_out[l], non_blocking=True)
+        main.wait_stream(copy_stream)
 
     E = max(1, min(K_, 10))
     cache.set_seq_len(-1, T0 + W_ - 1)
