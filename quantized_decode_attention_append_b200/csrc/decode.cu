@@ -499,7 +499,7 @@ struct MmaPlan {
 template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int ST>
 static MmaPlan mma_plan_of() {
   using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, ST>;
-  return MmaPlan{decode_tc_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST>, C::SMEM, C::TILE, C::NT};
+  return MmaPlan{decode_tc_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST>, C::SMEM, C::TILE, C::NTH};
 }
 
 static int code_fmt(const SideDev& S, bool is_v) {

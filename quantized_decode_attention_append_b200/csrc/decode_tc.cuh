@@ -161,6 +161,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
@@ -215,7 +218,12 @@ __device__ __forceinline__ void lds_words(const unsigned char* p, uint32_t* w) {
 template <int D, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
 struct TcCfg {
   static constexpr int KB = CodeBits<KF>::v, VB = CodeBits<VF>::v;
-  static constexpr int NT = NW * 32;                   // threads
+  static constexpr int NT = NW * 32;                   // consumer threads
+  // A dedicated producer warp recycles stages through per-stage "empty" barriers, so consumer
+  // warps never meet at a CTA barrier.  Measured: faster for head_dim 256 (4 consumer warps),
+  // slightly slower for the head_dim-128 instances, which keep one CTA barrier per tile.
+  static constexpr bool PROD = D >= 256;
+  static constexpr int NTH = NT + (PROD ? 32 : 0);
   static constexpr int TILE = NW * TPW;                // tokens per stage
   static constexpr int HALF = TILE / 2;                // tokens per half-tile range
   static constexpr int NSB = TPW / 16;                 // 16-token blocks per warp and tile
@@ -271,7 +279,7 @@ struct TcCfg {
   static constexpr int LUT_BYTES = (KF == CF_NF4 || KTRN || VTRN) ? 256 * 32 * 4 : 0;
   static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_X = OFF_LUT + LUT_BYTES;
   static constexpr int OFF_BAR = OFF_X + NW * XW;
-  static constexpr int SMEM = OFF_BAR + STAGES * 8;
+  static constexpr int SMEM = OFF_BAR + 2 * STAGES * 8;  // full and empty barriers
 
   static_assert(KCB % 4 == 0, "K chunks must be whole words");
   static_assert(!(KTRN || VTRN) || (D == 128 && TPW == 32 && GK == 8 && GV == 8), "ternary instance shape");
@@ -399,13 +407,14 @@ __device__ __forceinline__ void int3_transcode(const unsigned char* src, unsigne
 }
 
 template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
-__global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
+__global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
                                                             const int* __restrict__ seq_ids,
                                                             const int* __restrict__ kv_len, float* __restrict__ work,
                                                             int n_split, int nsp_total) {
   using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // full[s]: tile landed (bytes)
+  uint64_t* ebar = bar + STAGES;                                      // empty[s]: every consumer warp done
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -445,13 +454,21 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     }
   };
 
+  const bool producer = C::PROD && warp == NW;  // lane 0 of the extra warp moves the tiles
   if (tid == 0) {
 #pragma unroll
-    for (int s = 0; s < STAGES; ++s) mbar_init(bar + s, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar + s, 1);
+      mbar_init(ebar + s, NW);
+    }
     mbar_init_fence();
   }
   __syncthreads();
-  if (tid == 0) {
+  int issued = 0;  // tiles the producer has issued
+  if constexpr (C::PROD) {
+    if (producer && lane == 0)
+      for (; issued < STAGES && issued < nmy; ++issued) issue(it0 + issued, issued);
+  } else if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s)
       if (s < nmy) issue(it0 + s, s);
@@ -530,13 +547,30 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
   bool timed_out = false;
   int it = 0;
 
-  for (; it < nmy; ++it) {
-    if (__syncthreads_or(timed_out)) break;  // every warp is done with tile it - 1: refill its stage
-    if (tid == 0 && it + STAGES - 1 < nmy) issue(it0 + it + STAGES - 1, (it + STAGES - 1) % STAGES);
+  if (producer) {  // refill a stage once every consumer warp has released it (bounded waits)
+    if (lane == 0) {
+      for (; issued < nmy; ++issued) {
+        const int s = issued % STAGES;
+        if (!mbar_wait(ebar + s, (uint32_t)(issued / STAGES - 1) & 1u)) {
+          atomicOr(L.err, (unsigned)KVQ_ERRF_WAIT_TIMEOUT);
+          timed_out = true;
+          break;
+        }
+        issue(it0 + issued, s);
+      }
+    }
+  } else for (; it < nmy; ++it) {
+    if constexpr (!C::PROD) {
+      if (__syncthreads_or(timed_out)) break;  // every warp is done with tile it - 1: refill its stage
+      if (tid == 0 && it + STAGES - 1 < nmy) issue(it0 + it + STAGES - 1, (it + STAGES - 1) % STAGES);
+    }
     const int stage = it % STAGES;
-    if (__any_sync(0xffffffffu, !mbar_wait(bar + stage, (uint32_t)(it / STAGES) & 1u))) {
+    if (!timed_out && __any_sync(0xffffffffu, !mbar_wait(bar + stage, (uint32_t)(it / STAGES) & 1u))) {
       if (lane == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_WAIT_TIMEOUT);
       timed_out = true;
+    }
+    if (timed_out) {  // release the stage without reading it
+      if (C::PROD && lane == 0) mbar_arrive(ebar + stage);
       continue;
     }
 
@@ -816,14 +850,22 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       }
       __syncwarp();
     }
+    if (C::PROD && lane == 0) mbar_arrive(ebar + stage);  // this warp no longer reads the stage
   }
 
-  // A tile that timed out, and the tiles issued after it, may still be landing: wait for them
-  // (bounded again) before the stage buffers are reused or the CTA exits.
+  // After a timed-out wait the last tile issued into each stage may still be landing: the
+  // producer waits for them (bounded again) before the stage buffers are reused or the CTA exits.
   timed_out = __syncthreads_or(timed_out);
-  if (timed_out && tid == 0) {
-    const int issued = min(nmy, it + STAGES - 1);
-    for (int i = max(it - 1, 0); i < issued; ++i) mbar_wait(bar + i % STAGES, (uint32_t)(i / STAGES) & 1u);
+  if constexpr (C::PROD) {
+    if (timed_out && producer && lane == 0) {
+      for (int s = 0; s < STAGES; ++s) {
+        const int last = issued - 1 - ((issued - 1 - s) % STAGES + STAGES) % STAGES;  // last tile issued into s
+        if (last >= 0) mbar_wait(bar + s, (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+  } else if (timed_out && tid == 0) {
+    const int iss = min(nmy, it + STAGES - 1);
+    for (int i = max(it - 1, 0); i < iss; ++i) mbar_wait(bar + i % STAGES, (uint32_t)(i / STAGES) & 1u);
   }
   __syncthreads();  // stage buffers are free: reuse them to combine the warps
 
@@ -837,7 +879,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
     m_run = -INFINITY;
     l_run = 0.0f;
   }
-  if (head_ok) {
+  if (head_ok && !producer) {
     if (g == 0) {
       ml[(warp * 4 + c) * 2] = m_run;
       ml[(warp * 4 + c) * 2 + 1] = l_run;
@@ -853,7 +895,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(LayerDev L, const __
       }
   }
   __syncthreads();
-  for (int e = tid; e < G * D; e += C::NT) {
+  for (int e = tid; e < G * D && tid < C::NT; e += C::NT) {
     const int h = e / D, j = e % D;
     float M = -INFINITY;
 #pragma unroll
