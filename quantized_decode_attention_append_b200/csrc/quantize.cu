@@ -381,10 +381,32 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   constexpr int LG = G > 32 ? G / 32 : 1;             // lanes per group
   constexpr int GPL = G > 32 ? 1 : 32 / G;            // groups per lane
   const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : S.bits);
-  __shared__ uint32_t tw[NW][64];                     // ternary byte accumulation, one row slot at a time
 
-  for (int rb = (bid * NW + warp) * rpw; rb < R; rb += nblk * NW * rpw) {
+  // The next pass's input slice is loaded before this pass's arithmetic, so each warp keeps its
+  // loads in flight while it computes (the arithmetic per row is long).
+  const int stride = nblk * NW * rpw;
+  uint4 nx[4];
+  {
+    const long long r0 = (long long)(bid * NW + warp) * rpw + lane / lpr;
+    if (r0 < R) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + r0 * D + li * 32);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
+    }
+  }
+  for (int rb = (bid * NW + warp) * rpw; rb < R; rb += stride) {
     const int row = rb + lane / lpr;
+    uint4 cw[4];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) cw[c4] = nx[c4];
+    {
+      const long long rn = (long long)row + stride;
+      if (rn < R) {
+        const uint4* p = reinterpret_cast<const uint4*>(src + rn * D + li * 32);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
+      }
+    }
     int i = 0, u = 0, pos = 0, len_after = 0;
     bool ok = row < R;
     if (ok) {
@@ -400,12 +422,10 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     }
     float x[32];
     __half2 raw2[16];  // the lane's 32 input values as stored (fp16 pairs)
-    const __half* rp = src + ((long long)u * n_new + i) * D + li * 32;
     if (ok) {
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(rp) + c4);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&w);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&cw[c4]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           raw2[c4 * 4 + e] = h2[e];
@@ -417,7 +437,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       if (in_anchor(L, pos, len_after)) {
         __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + li * 32;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = __ldg(reinterpret_cast<const uint4*>(rp) + c4);
+        for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
       }
       if (S.chan_scale) {
         const __half* cp = S.chan + (u % L.Hkv) * D + li * 32;
@@ -457,10 +477,6 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     const long long rix = (long long)u * L.Tcap + pos;
     uint32_t* wout = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes) + li * bits;  // this lane's words
     uint32_t code[32];
-    if (FAM == FAM_TERNARY) {
-      for (int k = lane; k < 64; k += 32) tw[warp][k] = 0u;
-      __syncwarp();
-    }
 #pragma unroll
     for (int gl = 0; gl < GPL; ++gl) {
       const float* xg = x + gl * (G > 32 ? 32 : G);
@@ -584,18 +600,11 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
 #pragma unroll
             for (int v = 0; v < NV; ++v) code[gl * NV + v] = 7u;
           }
-        } else {  // ternary digits t + 1 into this row's byte accumulators (5 trits per byte)
+        } else {  // ternary digits t + 1 (packed into bytes after the groups)
           const float hh = __fmul_rn(d, 0.5f);
-          if (ok) {
-            uint32_t* rowacc = &tw[warp][(lane / lpr) * (((D + 4) / 5 + 3) / 4)];
 #pragma unroll
-            for (int v = 0; v < NV; ++v) {
-              const uint32_t dg = d != 0.0f ? ((xg[v] >= hh) ? 2u : ((xg[v] < -hh) ? 0u : 1u)) : 1u;
-              const int j = li * 32 + gl * NV + v, byte = j / 5, m5 = j % 5;
-              const uint32_t p3 = m5 == 0 ? 1u : m5 == 1 ? 3u : m5 == 2 ? 9u : m5 == 3 ? 27u : 81u;
-              atomicAdd(&rowacc[byte >> 2], (dg * p3) << (8 * (byte & 3)));
-            }
-          }
+          for (int v = 0; v < NV; ++v)
+            code[gl * NV + v] = d != 0.0f ? ((xg[v] >= hh) ? 2u : ((xg[v] < -hh) ? 0u : 1u)) : 1u;
         }
       }
       if (ok && (LG == 1 || (li % LG) == 0)) {
@@ -610,13 +619,34 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       else pack32_bits(code, bits, wout, ok);
     }
     if (FAM == FAM_TERNARY) {
-      __syncwarp();
-      if (ok) {
-        const uint32_t* rowacc = &tw[warp][(lane / lpr) * (((D + 4) / 5 + 3) / 4)];
-        uint8_t* op = S.codes + rix * S.row_bytes;
-        for (int b = li; b < S.row_bytes; b += lpr) op[b] = (uint8_t)(rowacc[b >> 2] >> (8 * (b & 3)));
+      // Bytes hold 5 digits (byte = sum d_m 3^m), so they straddle lanes.  A lane writes the
+      // bytes whose first digit is its own: [ceil(32 li / 5), ceil(32 (li + 1) / 5)); the last
+      // one may need up to 4 digits of the next lane (zero past the row's end).
+      uint32_t dlo = 0u, dhi = 0u;  // the lane's 32 digits as 2-bit fields
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        dlo += code[v] << (2 * v);
+        dhi += code[16 + v] << (2 * v);
       }
-      __syncwarp();
+      uint32_t nlo = __shfl_down_sync(0xffffffffu, dlo, 1);
+      if (li == lpr - 1) nlo = 0u;
+      const int b0 = (32 * li + 4) / 5, nb = (32 * li + 36) / 5 - b0;
+      const int o2 = 2 * (5 * b0 - 32 * li);  // bit of the first owned digit in the lane's stream
+      const uint32_t s0 = __funnelshift_r(dlo, dhi, o2), s1 = __funnelshift_r(dhi, nlo, o2), s2 = nlo >> o2;
+      uint8_t* op = S.codes + rix * S.row_bytes + b0;
+#pragma unroll
+      for (int j = 0; j < 7; ++j) {
+        const int bit = 10 * j;
+        const uint32_t f = bit <= 22 ? (s0 >> bit)
+                                    : (bit < 32 ? __funnelshift_r(s0, s1, bit)
+                                                : (bit <= 54 ? (s1 >> (bit - 32)) : __funnelshift_r(s1, s2, bit - 32)));
+        uint32_t t = (f >> 8) & 3u;
+        t = t * 3u + ((f >> 6) & 3u);
+        t = t * 3u + ((f >> 4) & 3u);
+        t = t * 3u + ((f >> 2) & 3u);
+        t = t * 3u + (f & 3u);
+        if (ok && j < nb) op[j] = (uint8_t)t;
+      }
     }
   }
 }
