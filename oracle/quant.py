@@ -12,7 +12,8 @@ Grids and scales (sources by page title and section):
     maps to -2^(b-1): d = fp16(m / -2^(b-1)), q = clamp(round(x/d), -2^(b-1), 2^(b-1)-1),
     stored as the unsigned code q + 2^(b-1).
   * per-token min-max (asymmetric): "E21W" "What I tested", variant A.  z = fp16(min), d = fp16(fp32(max - min) / (2^b - 1)),
-    q = clamp(round((x - z)/d), 0, 2^b - 1).
+    q = clamp(round((x - z)/d), 0, 2^b - 1).  The minimum orders -0 below +0 (IEEE 754
+    minimum), so a group whose smallest value is zero stores z = -0 if it holds a -0.
   * NF4: "Fourier Magnitude KV Cache Quantization" post 6 (NF4 in groups of 64); s = fp16(max|x|),
     code = nearest level of x/s (see oracle.nf4).
   * ternary {-s, 0, +s}: post 6 "Milestone" table (ternary in groups of 8 and 4);
@@ -167,6 +168,9 @@ def quant_int_minmax(x32: np.ndarray, b: int, g: int):
     xg = x32.reshape(R, D // g, g).astype(F32)
     mn = xg.min(axis=-1)
     mx = xg.max(axis=-1)
+    # a zero minimum is -0 when the group holds a -0 (IEEE 754 minimum: -0 orders below +0)
+    negz = np.any((xg == 0) & np.signbit(xg), axis=-1)
+    mn = np.where(mn == 0, np.where(negz, F32(-0.0), F32(0.0)), mn).astype(F32)
     z = f16(mn)
     d = f16((mx - mn).astype(F32) / F32(2 ** b - 1))
     q = round_half_up_exact(xg.astype(F64), d[..., None], z[..., None])

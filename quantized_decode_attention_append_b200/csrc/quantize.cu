@@ -28,6 +28,9 @@
 namespace kvq {
 
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+// Bitwise choice: bits of a where m is set, of b elsewhere (one 3-input logic op).
+__device__ __forceinline__ uint32_t bsel(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
 
 __constant__ float q_nf4_mid[15];
 __constant__ float q_tw_re[64];
@@ -484,35 +487,52 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       __half sh, zh = __float2half_rn(0.0f);
       float d = 0.0f, z = 0.0f, inv = 0.0f;
       if (FAM == FAM_ABSMAX) {
-        // signed value of largest magnitude, first channel on ties: the magnitude maximum, then a
-        // backward scan that keeps the earliest element reaching it
-        float am = 0.0f;
+        // signed value of largest magnitude, first channel on ties: the group's maximum or minimum,
+        // whichever is larger in magnitude; only a group holding both +a and -a (or only zeros)
+        // needs the earliest channel reaching a, found by a backward scan
+        float mx = xg[0], mn = xg[0];
 #pragma unroll
-        for (int v = 0; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
-        float m = 0.0f;
+        for (int v = 1; v < NV; ++v) { mx = fmaxf(mx, xg[v]); mn = fminf(mn, xg[v]); }
 #pragma unroll
-        for (int v = NV - 1; v >= 0; --v) m = fabsf(xg[v]) == am ? xg[v] : m;
+        for (int o = 1; o < LG; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        }
+        float m = mx > -mn ? mx : mn;
+        const bool tie = !(mx > -mn) && !(-mn > mx);
+        if (__any_sync(0xffffffffu, tie)) {  // warp-uniform, so the shuffles below see every lane
+          float am = 0.0f;
 #pragma unroll
-        for (int o = 1; o < LG; o <<= 1) {  // the lane with the lower channels wins ties
-          const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, m, o);
-          if (oam > am || (oam == am && (li & o))) { am = oam; m = om; }
+          for (int v = 0; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+          float me = 0.0f;
+#pragma unroll
+          for (int v = NV - 1; v >= 0; --v) me = fabsf(xg[v]) == am ? xg[v] : me;
+#pragma unroll
+          for (int o = 1; o < LG; o <<= 1) {  // the lane with the lower channels wins ties
+            const float oam = __shfl_xor_sync(0xffffffffu, am, o), om = __shfl_xor_sync(0xffffffffu, me, o);
+            if (oam > am || (oam == am && (li & o))) { am = oam; me = om; }
+          }
+          if (tie) m = me;
         }
         const int half = 1 << (bits - 1);
         sh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
         d = __half2float(sh);
         inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
-        // code = floor(x/d + 1/2) + half from the estimate r = x * inv + half + 1/2, whose error is
-        // below 2^-19 (|x/d| <= half <= 2^7); a fraction within 2^-16 of an integer sends the
-        // lane's group through the exact comparisons instead.
-        const float c0 = 0.5f + (float)half;
+        // code = floor(x/d + 1/2) + half.  x * inv + half + 1.5 * 2^23, rounded once by the fma,
+        // is 1.5 * 2^23 + the integer nearest to the estimate x * inv + half (error below 2^-17,
+        // as |x/d| <= half <= 2^7), so the code sits in the low mantissa bits with no conversion
+        // instruction.  A remainder within 2^-16 of +-1/2 sends the lane's group through the
+        // exact comparisons instead.
+        constexpr float kMagic = 12582912.0f;
+        const float c1 = (float)half + kMagic;
+        const uint32_t top = 2u * half - 1u;
         bool near = false;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          const float r = fmaf(xg[v], inv, c0);
-          const float k = floorf(r);
-          const float fr = r - k;
-          near |= (fr < (1.0f / 65536.0f)) | (fr > (1.0f - 1.0f / 65536.0f));
-          code[gl * NV + v] = (uint32_t)(int)fminf(k, (float)(2 * half - 1));
+          const float t = fmaf(xg[v], inv, c1);
+          const float fr = fmaf(xg[v], inv, c1 - t);  // c1 - t = half - k exactly
+          near |= fabsf(fr) > 0.5f - 1.0f / 65536.0f;
+          code[gl * NV + v] = min(__float_as_uint(t) - 0x4B400000u, top);
         }
         if (near && d != 0.0f) {
 #pragma unroll
@@ -529,6 +549,14 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         for (int o = 1; o < LG; o <<= 1) {
           mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (__any_sync(0xffffffffu, mn == 0.0f)) {  // a zero minimum is -0 iff the group holds a -0
+          bool negz = false;
+#pragma unroll
+          for (int v = 0; v < NV; ++v) negz |= __float_as_uint(xg[v]) == 0x80000000u;
+#pragma unroll
+          for (int o = 1; o < LG; o <<= 1) negz |= __shfl_xor_sync(0xffffffffu, (int)negz, o) != 0;
+          if (mn == 0.0f) mn = negz ? -0.0f : 0.0f;
         }
         const int top = (1 << bits) - 1;
         zh = __float2half_rn(mn);
@@ -577,17 +605,25 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
             __half2 t2[15];
 #pragma unroll
             for (int k = 0; k < 15; ++k) t2[k] = __half2half2(__float2half_ru(__fmul_rn(q_nf4_mid[k], d)));
+            uint32_t tw[15];
+#pragma unroll
+            for (int k = 0; k < 15; ++k) tw[k] = h2u(t2[k]);
 #pragma unroll
             for (int p2 = 0; p2 < NV / 2; ++p2) {
+              // the thresholds reached form a prefix, so its length comes from a 4-step binary
+              // search, run on both halves at once: each step compares with the threshold that
+              // the decisions so far select (bit masks, one 3-input logic op per 2-way choice)
               const __half2 xv = raw2[(gl * NV) / 2 + p2];
-              // four short chains instead of one long one (the one-token append is latency-bound)
-              __half2 a[4] = {__float2half2_rn(1024.0f), __float2half2_rn(0.0f), __float2half2_rn(0.0f),
-                              __float2half2_rn(0.0f)};
-#pragma unroll
-              for (int k = 0; k < 15; ++k) a[k & 3] = __hadd2(a[k & 3], __hge2(xv, t2[k]));
-              const uint32_t b = h2u(__hadd2(__hadd2(a[0], a[1]), __hadd2(a[2], a[3])));
+              const uint32_t m3 = __hge2_mask(xv, t2[7]);
+              const uint32_t m2 = __hge2_mask(xv, u2h(bsel(m3, tw[11], tw[3])));
+              const uint32_t m1 = __hge2_mask(
+                  xv, u2h(bsel(m3, bsel(m2, tw[13], tw[9]), bsel(m2, tw[5], tw[1]))));
+              const uint32_t m0 = __hge2_mask(
+                  xv, u2h(bsel(m3, bsel(m2, bsel(m1, tw[14], tw[12]), bsel(m1, tw[10], tw[8])),
+                               bsel(m2, bsel(m1, tw[6], tw[4]), bsel(m1, tw[2], tw[0])))));
+              const uint32_t b = (m3 & 0x00080008u) | (m2 & 0x00040004u) | (m1 & 0x00020002u) | (m0 & 0x00010001u);
               code[gl * NV + 2 * p2] = b & 0xFu;
-              code[gl * NV + 2 * p2 + 1] = (b >> 16) & 0xFu;
+              code[gl * NV + 2 * p2 + 1] = b >> 16;
             }
           } else {
             float th[15];

@@ -28,15 +28,20 @@ def oracle_spec(cfg: Config) -> OC.Spec:
 class Case:
     """A filled cache plus the fp16 inputs that went into it (kept on the host)."""
 
-    def __init__(self, cfg: Config, T: int, seed: int = 0, chunks=None, layers=None, calib_T: int = 512):
+    def __init__(self, cfg: Config, T: int, seed: int = 0, chunks=None, layers=None, calib_T: int = 512,
+                 inputs=None):
+        """inputs: optional callable l -> (K, V) fp16 arrays [B, H, T, D] replacing the seeded law."""
         self.cfg, self.T, self.seed = cfg, T, seed
         self.cache = KVCache(cfg)
         self.K, self.V, self.C = {}, {}, {}
         B, H, D = cfg.batch, cfg.n_kv_heads, cfg.head_dim
         layers = range(cfg.n_layers) if layers is None else layers
         for l in layers:
-            K = synth.kv_rows(seed, "k", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
-            V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
+            if inputs is None:
+                K = synth.kv_rows(seed, "k", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
+                V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
+            else:
+                K, V = (torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in inputs(l))
             if cfg.k.chan_scale:
                 c = synth.channel_scale(seed, l, H, calib_T, D).cuda()
                 self.cache.set_chan_scale(l, c)

@@ -170,3 +170,31 @@ def test_fp16_output_path():
     o32 = c.cache.decode(0, q)
     o16 = c.cache.decode(0, q, fp32=False)
     assert torch.allclose(o16.float(), o32, rtol=1e-3, atol=1e-3)
+
+
+# ------------------------------------------------------------------- decision-boundary inputs
+ADVERSARIAL = [
+    (128, Side("int", 4, group=32), Side("int", 3, group=64)),
+    (128, Side("int", 2, group=128), Side("int", 8, group=16)),
+    (128, Side("int", 4, group=64), Side("int", 4, group=64)),
+    (128, Side("nf4", group=64), Side("int", 4, group=64)),
+    (128, Side("ternary", group=8), Side("sign", group=4)),
+    (128, Side("nf4", group=16), Side("ternary", group=4)),
+    (256, Side("int", 4, scale="minmax", group=32), Side("int", 3, scale="minmax", group=16)),
+    (64, Side("int", 3, group=16), Side("nf4", group=32)),
+]
+
+
+@pytest.mark.parametrize("D,k,v", ADVERSARIAL, ids=[f"{d}-{k.fmt}{k.bits}g{k.group}-{v.fmt}{v.bits}g{v.group}"
+                                                       for d, k, v in ADVERSARIAL])
+@pytest.mark.parametrize("chunks", [None, [1] * 6 + [58]], ids=["bulk", "tokens"])
+def test_decision_boundaries(D, k, v, chunks):
+    """Rows whose values sit exactly on rounding ties, NF4 thresholds, both-sign maxima and
+    signed zeros: codes and scales still bit-identical to the oracle."""
+    import adversarial
+    T = 64
+    cfg = cfg_of(D, k, v, T=T)
+    c = Case(cfg, T, chunks=chunks, inputs=lambda l: (adversarial.rows(11 + l, 2, 2, T, D),
+                                                      adversarial.rows(97 + l, 2, 2, T, D)))
+    c.check_codes(0)
+    c.check_dequant(0)

@@ -155,6 +155,19 @@ def test_int_minmax_nearest_grid_point(b):
                 assert r["q"][i, gi * 32 + jj] == want
 
 
+def test_minmax_zero_point_signed_zero():
+    """IEEE 754 minimum orders -0 below +0: a group whose smallest value is zero stores z = -0
+    exactly when it holds a -0, +0 otherwise (the sign bit is all that differs)."""
+    x = np.zeros((3, 8), dtype=np.float16)
+    x[0, 5] = np.float16(-0.0)          # +0 ... -0 ... : min is -0
+    x[1, :] = np.float16(-0.0)          # all -0
+    x[2, 3] = np.float16(1.5)           # +0 and a positive value: min is +0
+    r = Q.quantize_rows(x, Side("int", 4, scale="minmax", group=8))
+    assert r["zeros"][:, 0].view(np.uint16).tolist() == [0x8000, 0x8000, 0x0000]
+    assert r["scales"][:, 0].view(np.uint16).tolist()[:2] == [0x0000, 0x0000]
+    assert r["scales"][2, 0] == np.float16(0.1)  # fp16(1.5 / 15)
+
+
 def test_nf4_nearest_level():
     x = (rng(3).standard_normal((4, 128))).astype(np.float16)
     r = Q.quantize_rows(x, Side("nf4", group=64))
