@@ -230,6 +230,9 @@ def fill_cache(cache, w, T0, seed, device, timed=False):
             if timed and not first:
                 torch.cuda.synchronize()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                # a ~0.5 ms device-side delay ahead of the start event lets the host queue the
+                # append before the device reaches it, so the events bracket the kernel alone
+                torch.cuda._sleep(1_000_000)
                 e0.record(stream)
             cache.append(l, K, V)
             if timed and not first:

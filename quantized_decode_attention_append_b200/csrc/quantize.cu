@@ -92,6 +92,28 @@ __device__ __forceinline__ void pack32(const uint32_t* code, uint32_t* out, bool
   }
 }
 
+// Same, for codes held as fp32 bit patterns 1.5 * 2^23 + code (B divides 32, so no field crosses a
+// word): the patterns' constant parts are added with the codes and taken off once per word.
+template <int B>
+__device__ __forceinline__ void pack32_biased(const uint32_t* code, uint32_t* out, bool ok) {
+  static_assert(32 % B == 0, "fields must not cross words");
+  constexpr int PW = 32 / B;
+  constexpr uint32_t bias = [] {
+    uint32_t t = 0u;
+    for (int j = 0; j < PW; ++j) t += 0x4B400000u << (j * B);
+    return t;
+  }();
+  uint32_t w[B];
+#pragma unroll
+  for (int k = 0; k < B; ++k) w[k] = 0u - bias;
+#pragma unroll
+  for (int v = 0; v < 32; ++v) w[v / PW] += code[v] << ((v % PW) * B);
+  if (ok) {
+#pragma unroll
+    for (int k = 0; k < B; ++k) out[k] = w[k];
+  }
+}
+
 __device__ __forceinline__ void pack32_bits(const uint32_t* code, int bits, uint32_t* out, bool ok) {
   switch (bits) {
     case 1: pack32<1>(code, out, ok); break;
@@ -371,7 +393,7 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const float* th) {
 }
 
 // Rows of one side over blocks bid = 0 .. nblk - 1 (grid-stride).
-template <int FAM, int G>
+template <int FAM, int G, int BITS = 0>
 __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __half* __restrict__ src, int n_new,
                                           int bid, int nblk) {
   const SideDev& S = L.s[side];
@@ -383,7 +405,8 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   const int R = L.B * L.Hkv * n_new;                  // < 2^31 (checked on the host)
   constexpr int LG = G > 32 ? G / 32 : 1;             // lanes per group
   constexpr int GPL = G > 32 ? 1 : 32 / G;            // groups per lane
-  const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : S.bits);
+  // code bits: fixed by the family, by the instance (BITS > 0), or read from the side
+  const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : (BITS > 0 ? BITS : S.bits));
 
   // The next pass's input slice is loaded before this pass's arithmetic, so each warp keeps its
   // loads in flight while it computes (the arithmetic per row is long).
@@ -430,11 +453,14 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       for (int c4 = 0; c4 < 4; ++c4) {
         const __half2* h2 = reinterpret_cast<const __half2*>(&cw[c4]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          raw2[c4 * 4 + e] = h2[e];
-          const float2 f = __half22float2(h2[e]);
-          x[c4 * 8 + 2 * e] = f.x;
-          x[c4 * 8 + 2 * e + 1] = f.y;
+        for (int e = 0; e < 4; ++e) raw2[c4 * 4 + e] = h2[e];
+      }
+      if (!(FAM == FAM_NF4 && !S.rot && !S.chan_scale)) {  // NF4 on untransformed rows reads raw2 only
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 f = __half22float2(raw2[e]);
+          x[2 * e] = f.x;
+          x[2 * e + 1] = f.y;
         }
       }
       if (in_anchor(L, pos, len_after)) {
@@ -490,9 +516,20 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         // signed value of largest magnitude, first channel on ties: the group's maximum or minimum,
         // whichever is larger in magnitude; only a group holding both +a and -a (or only zeros)
         // needs the earliest channel reaching a, found by a backward scan
-        float mx = xg[0], mn = xg[0];
+        float mx, mn;
+        if (NV >= 2 && !S.rot && !S.chan_scale) {  // x is the fp16 input: max and min two at a time
+          const __half2* rg = raw2 + (gl * NV) / 2;
+          __half2 hx = rg[0], hn = rg[0];
 #pragma unroll
-        for (int v = 1; v < NV; ++v) { mx = fmaxf(mx, xg[v]); mn = fminf(mn, xg[v]); }
+          for (int p2 = 1; p2 < NV / 2; ++p2) { hx = __hmax2(hx, rg[p2]); hn = __hmin2(hn, rg[p2]); }
+          mx = fmaxf(__low2float(hx), __high2float(hx));
+          mn = fminf(__low2float(hn), __high2float(hn));
+        } else {
+          mx = xg[0];
+          mn = xg[0];
+#pragma unroll
+          for (int v = 1; v < NV; ++v) { mx = fmaxf(mx, xg[v]); mn = fminf(mn, xg[v]); }
+        }
 #pragma unroll
         for (int o = 1; o < LG; o <<= 1) {
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -523,22 +560,25 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         // as |x/d| <= half <= 2^7), so the code sits in the low mantissa bits with no conversion
         // instruction.  A remainder within 2^-16 of +-1/2 sends the lane's group through the
         // exact comparisons instead.
+        // With BIASED the codes stay as the fp32 patterns (pack32_biased removes the constant).
+        constexpr bool BIASED = BITS == 2 || BITS == 4 || BITS == 8;
         constexpr float kMagic = 12582912.0f;
         const float c1 = (float)half + kMagic;
         const uint32_t top = 2u * half - 1u;
+        const float ctop = kMagic + (float)top;
         bool near = false;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
           const float t = fmaf(xg[v], inv, c1);
           const float fr = fmaf(xg[v], inv, c1 - t);  // c1 - t = half - k exactly
           near |= fabsf(fr) > 0.5f - 1.0f / 65536.0f;
-          code[gl * NV + v] = min(__float_as_uint(t) - 0x4B400000u, top);
+          code[gl * NV + v] = BIASED ? __float_as_uint(fminf(t, ctop)) : min(__float_as_uint(t) - 0x4B400000u, top);
         }
         if (near && d != 0.0f) {
 #pragma unroll
           for (int v = 0; v < NV; ++v) {
             const float k = fminf(fmaxf(round_exact_absmax(xg[v], d, inv), (float)(-half)), (float)(half - 1));
-            code[gl * NV + v] = (uint32_t)((int)k + half);
+            code[gl * NV + v] = (uint32_t)((int)k + half) + (BIASED ? 0x4B400000u : 0u);
           }
         }
       } else if (FAM == FAM_MINMAX) {
@@ -590,9 +630,18 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
 #pragma unroll
         for (int v = 0; v < NV; ++v) code[gl * NV + v] = xg[v] >= 0.0f ? 1u : 0u;
       } else {  // NF4 and ternary: absmax magnitude scale
-        float am = fabsf(xg[0]);
+        float am;
+        if (FAM == FAM_NF4 && NV >= 2 && !S.rot && !S.chan_scale) {  // from the fp16 input pairs
+          const __half2* rg = raw2 + (gl * NV) / 2;
+          __half2 hx = rg[0], hn = rg[0];
 #pragma unroll
-        for (int v = 1; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+          for (int p2 = 1; p2 < NV / 2; ++p2) { hx = __hmax2(hx, rg[p2]); hn = __hmin2(hn, rg[p2]); }
+          am = fabsf(fmaxf(fmaxf(__low2float(hx), __high2float(hx)), -fminf(__low2float(hn), __high2float(hn))));
+        } else {
+          am = fabsf(xg[0]);
+#pragma unroll
+          for (int v = 1; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+        }
 #pragma unroll
         for (int o = 1; o < LG; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
         sh = __float2half_rn(am);
@@ -652,6 +701,9 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     if (FAM != FAM_TERNARY) {
       if (FAM == FAM_SIGN) pack32<1>(code, wout, ok);
       else if (FAM == FAM_NF4) pack32<4>(code, wout, ok);
+      else if (FAM == FAM_ABSMAX && (BITS == 2 || BITS == 4 || BITS == 8))
+        pack32_biased<(BITS == 2 || BITS == 4 || BITS == 8) ? BITS : 8>(code, wout, ok);
+      else if (BITS > 0) pack32<(BITS > 0 ? BITS : 8)>(code, wout, ok);
       else pack32_bits(code, bits, wout, ok);
     }
     if (FAM == FAM_TERNARY) {
@@ -695,12 +747,12 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
 }
 
 // K and V in one launch: blocks [0, kblocks) take the K rows, the rest the V rows.
-template <int FK, int GK, int FV, int GV>
+template <int FK, int GK, int BK, int FV, int GV, int BV>
 __global__ void __launch_bounds__(kRowThreads) append_kv_kernel(LayerDev L, const __half* __restrict__ k,
                                                                 const __half* __restrict__ v, int n_new,
                                                                 unsigned kblocks) {
-  if (blockIdx.x < kblocks) rows_body<FK, GK>(L, 0, k, n_new, blockIdx.x, kblocks);
-  else rows_body<FV, GV>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
+  if (blockIdx.x < kblocks) rows_body<FK, GK, BK>(L, 0, k, n_new, blockIdx.x, kblocks);
+  else rows_body<FV, GV, BV>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
   finish_append(L, n_new, gridDim.x);
 }
 
@@ -817,15 +869,21 @@ static KvKernel pick_kv_kernel(const LayerDev& L) {
       V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART)
     return nullptr;
   const int fk = fam_of(K), fv = fam_of(V), gk = K.group, gv = V.group;
-#define KVQ_KV(FK_, GK_, FV_, GV_) \
-  if (fk == FK_ && gk == GK_ && fv == FV_ && gv == GV_) return append_kv_kernel<FK_, GK_, FV_, GV_>;
-  KVQ_KV(FAM_NF4, 64, FAM_ABSMAX, 64)
-  KVQ_KV(FAM_ABSMAX, 64, FAM_ABSMAX, 64)
-  KVQ_KV(FAM_ABSMAX, 128, FAM_ABSMAX, 128)
-  KVQ_KV(FAM_ABSMAX, 32, FAM_ABSMAX, 32)
-  KVQ_KV(FAM_MINMAX, 32, FAM_MINMAX, 32)
-  KVQ_KV(FAM_TERNARY, 8, FAM_TERNARY, 8)
-  KVQ_KV(FAM_SIGN, 4, FAM_SIGN, 4)
+  // bits 0: fixed by the family (NF4, ternary, sign)
+#define KVQ_KV(FK_, GK_, BK_, FV_, GV_, BV_)                                                      \
+  if (fk == FK_ && gk == GK_ && (BK_ == 0 || K.bits == BK_) && fv == FV_ && gv == GV_ &&        \
+      (BV_ == 0 || V.bits == BV_))                                                               \
+    return append_kv_kernel<FK_, GK_, BK_, FV_, GV_, BV_>;
+  KVQ_KV(FAM_NF4, 64, 0, FAM_ABSMAX, 64, 4)
+  KVQ_KV(FAM_ABSMAX, 64, 4, FAM_ABSMAX, 64, 4)
+  KVQ_KV(FAM_ABSMAX, 128, 4, FAM_ABSMAX, 128, 2)
+  KVQ_KV(FAM_ABSMAX, 128, 4, FAM_ABSMAX, 128, 3)
+  KVQ_KV(FAM_ABSMAX, 128, 4, FAM_ABSMAX, 128, 4)
+  KVQ_KV(FAM_ABSMAX, 32, 4, FAM_ABSMAX, 32, 4)
+  KVQ_KV(FAM_MINMAX, 32, 3, FAM_MINMAX, 32, 3)
+  KVQ_KV(FAM_MINMAX, 32, 4, FAM_MINMAX, 32, 4)
+  KVQ_KV(FAM_TERNARY, 8, 0, FAM_TERNARY, 8, 0)
+  KVQ_KV(FAM_SIGN, 4, 0, FAM_SIGN, 4, 0)
 #undef KVQ_KV
   return nullptr;
 }
