@@ -115,6 +115,17 @@ kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes);
  * handle plus a split-K workspace on the current device.  Synchronous. */
 kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out);
 
+/* Per-layer formats ("E21W" "What I tested" and "Result": a per-layer K/V bit allocation
+ * under an average budget, e.g. 2-bit K in two layers and 4-bit V in three, 3-bit elsewhere).
+ * layer_k / layer_v: host arrays of cfg->n_layers sides, read during the call only; NULL
+ * means cfg->k / cfg->v on every layer (and only then is that field read).  Every side is
+ * checked as in kvq_create; otherwise identical to kvq_arena_bytes / kvq_create (the same
+ * kernels run, each layer with its own format). */
+kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v,
+                                  uint64_t* bytes);
+kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
+                             uint64_t arena_bytes, kvq_cache** out);
+
 /* Release the handle and its workspace (not the arena).  NULL is a no-op. */
 void kvq_free(kvq_cache* cache);
 

@@ -11,6 +11,11 @@ the anchor layer set:
   window(w):  tokens t >= L - w, L = the sequence's stored length
   all:        every token of the layer
 
+Per-layer formats ("E21W" "What I tested": a per-layer K/V bit allocation, 2 to 4 bits in groups
+of 128, under a 3.2-bit average; "Result": 2-bit K in layers 2 and 7, 4-bit V in layers 1, 3
+and 4, 3 bits elsewhere, 3.19 bits on average).  A Spec may give one Side per layer for K and for
+V; layers are numbered from 0 (the same result calls layer 7 the last of the 8).
+
 Effective bits ("E21W" "Result" counts group scales in the totals, 3.5 b for 3-bit g32 and
 4.5 b for 4-bit g32; "E22L" "What I tested" averages over K and V with scales included; post 6
 "Corrected semantics" reports anchored configurations in effective bits): (code bits + 16 per
@@ -41,6 +46,13 @@ class Spec:
     anchor_rule: str = "none"  # none | first_n | window | all
     anchor_n: int = 0
     sm_scale: float | None = None
+    layer_k: tuple = ()  # one Side per layer, or empty: k on every layer
+    layer_v: tuple = ()
+
+
+def side_of(spec: Spec, layer: int, is_k: bool) -> Side:
+    per = spec.layer_k if is_k else spec.layer_v
+    return per[layer] if per else (spec.k if is_k else spec.v)
 
 
 def anchored(spec: Spec, layer: int, tokens: np.ndarray, seq_len: int) -> np.ndarray:
@@ -56,10 +68,10 @@ def anchored(spec: Spec, layer: int, tokens: np.ndarray, seq_len: int) -> np.nda
     raise ValueError(spec.anchor_rule)
 
 
-def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None):
+def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None, layer: int = 0):
     """Quantize one (layer, sequence, kv-head) unit: K16, V16 [T, D]; c16 [D] or None."""
-    kq = quantize_rows(K16, spec.k, None if c16 is None else np.broadcast_to(c16, K16.shape))
-    vq = quantize_rows(V16, spec.v, None)
+    kq = quantize_rows(K16, side_of(spec, layer, True), None if c16 is None else np.broadcast_to(c16, K16.shape))
+    vq = quantize_rows(V16, side_of(spec, layer, False), None)
     return kq, vq
 
 
@@ -67,8 +79,8 @@ def reconstruct_unit(spec: Spec, layer: int, K16, V16, kq, vq, seq_len: int, c16
     """Keys and values attention sees for one unit (fp64 [T, D]); anchors override."""
     T = K16.shape[0]
     cK = None if c16 is None else np.broadcast_to(c16, K16.shape)
-    Kh = to_original_f64(kq["exact"], spec.k, cK)
-    Vh = to_original_f64(vq["exact"], spec.v, None)
+    Kh = to_original_f64(kq["exact"], side_of(spec, layer, True), cK)
+    Vh = to_original_f64(vq["exact"], side_of(spec, layer, False), None)
     an = anchored(spec, layer, np.arange(T), seq_len)
     Kh[an] = np.asarray(K16, dtype=np.float16)[an].astype(np.float64)
     Vh[an] = np.asarray(V16, dtype=np.float16)[an].astype(np.float64)
@@ -86,7 +98,7 @@ def effective_bits(spec: Spec, seq_len: int) -> float:
     tot = 0.0
     for layer in range(spec.n_layers):
         an = anchored(spec, layer, np.arange(seq_len), seq_len).sum()
-        for side, is_k in ((spec.k, True), (spec.v, False)):
+        for side, is_k in ((side_of(spec, layer, True), True), (side_of(spec, layer, False), False)):
             per_row = bits_per_value(side, D) * D
             bits = (seq_len - an) * per_row + an * 16 * D
             if is_k and side.chan_scale:

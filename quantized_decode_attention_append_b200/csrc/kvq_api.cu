@@ -13,6 +13,7 @@ using namespace kvq;
 
 struct kvq_cache {
   kvq_config cfg;
+  kvq_side side[64][2];  // format of each (layer, side): cfg.k / cfg.v unless set per layer
   int Tcap;
   char* arena;
   uint64_t arena_bytes;
@@ -77,7 +78,19 @@ kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
   return KVQ_OK;
 }
 
-kvq_status check_config(const kvq_config* c) {
+// The (layer, side) formats of a cache: the per-layer arrays where given, else cfg.k / cfg.v.
+struct LayerSides {
+  kvq_side s[64][2];
+};
+
+void fill_sides(const kvq_config& c, const kvq_side* lk, const kvq_side* lv, LayerSides* out) {
+  for (int l = 0; l < c.n_layers && l < 64; ++l) {
+    out->s[l][0] = lk ? lk[l] : c.k;
+    out->s[l][1] = lv ? lv[l] : c.v;
+  }
+}
+
+kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side* lv) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->n_layers > 64) return KVQ_ERR_INVALID_ARG;
   if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return KVQ_ERR_INVALID_ARG;
@@ -87,10 +100,14 @@ kvq_status check_config(const kvq_config* c) {
   if (c->capacity < 1 || c->capacity > (1 << 26)) return KVQ_ERR_INVALID_ARG;
   if (c->max_queries < 1) return KVQ_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || isinf(c->sm_scale)) return KVQ_ERR_INVALID_ARG;
-  kvq_status st = check_side(*c, c->k, true);
-  if (st != KVQ_OK) return st;
-  st = check_side(*c, c->v, false);
-  if (st != KVQ_OK) return st;
+  for (int l = 0; l < (lk ? c->n_layers : 1); ++l) {
+    const kvq_status st = check_side(*c, lk ? lk[l] : c->k, true);
+    if (st != KVQ_OK) return st;
+  }
+  for (int l = 0; l < (lv ? c->n_layers : 1); ++l) {
+    const kvq_status st = check_side(*c, lv ? lv[l] : c->v, false);
+    if (st != KVQ_OK) return st;
+  }
   if (c->anchor_rule < KVQ_ANCHOR_NONE || c->anchor_rule > KVQ_ANCHOR_ALL) return KVQ_ERR_INVALID_ARG;
   if (c->n_layers < 64 && (c->anchor_layer_mask >> c->n_layers)) return KVQ_ERR_INVALID_ARG;
   if (c->anchor_rule == KVQ_ANCHOR_FIRST_N || c->anchor_rule == KVQ_ANCHOR_WINDOW) {
@@ -118,7 +135,7 @@ bool layer_anchored(const kvq_config& c, int l) {
 }
 
 // Lay out the arena; fills `h` offsets if non-null.  Returns total bytes.
-uint64_t layout(const kvq_config& c, kvq_cache* h) {
+uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
   const int D = c.head_dim;
   const int Tcap = (c.capacity + 255) / 256 * 256;  // whole 256-token decode tiles
   const uint64_t units = (uint64_t)c.batch * c.n_kv_heads;
@@ -126,7 +143,7 @@ uint64_t layout(const kvq_config& c, kvq_cache* h) {
   uint64_t off = 0;
   for (int l = 0; l < c.n_layers; ++l) {
     for (int s = 0; s < 2; ++s) {
-      const kvq_side& sd = s == 0 ? c.k : c.v;
+      const kvq_side& sd = sides.s[l][s];
       int rb, ng;
       side_geometry(D, sd, &rb, &ng);
       kvq_cache::SideOff so{};
@@ -152,7 +169,7 @@ uint64_t layout(const kvq_config& c, kvq_cache* h) {
       if (h) h->off[l][s] = so;
     }
     int64_t ch = -1;
-    if (c.k.chan_scale) {
+    if (sides.s[l][0].chan_scale) {
       ch = (int64_t)off;
       off = align_up(off + (uint64_t)c.n_kv_heads * D * 2);
     }
@@ -178,7 +195,7 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
   LayerDev L{};
   const kvq_config& c = h->cfg;
   for (int s = 0; s < 2; ++s) {
-    const kvq_side& sd = s == 0 ? c.k : c.v;
+    const kvq_side& sd = h->side[l][s];
     const kvq_cache::SideOff& so = h->off[l][s];
     SideDev& S = L.s[s];
     S.codes = reinterpret_cast<uint8_t*>(h->arena + so.codes);
@@ -307,28 +324,39 @@ kvq_status kvq_nf4_levels(float out[16]) {
   return KVQ_OK;
 }
 
-kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes) {
+kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v,
+                                  uint64_t* bytes) {
   if (!bytes) return KVQ_ERR_INVALID_ARG;
-  const kvq_status st = check_config(cfg);
+  const kvq_status st = check_config(cfg, layer_k, layer_v);
   if (st != KVQ_OK) return st;
-  *bytes = layout(*cfg, nullptr);
+  LayerSides sides;
+  fill_sides(*cfg, layer_k, layer_v, &sides);
+  *bytes = layout(*cfg, sides, nullptr);
   return KVQ_OK;
 }
 
-kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out) {
+kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes) {
+  return kvq_arena_bytes_layers(cfg, nullptr, nullptr, bytes);
+}
+
+kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
+                             uint64_t arena_bytes, kvq_cache** out) {
   if (!out) return KVQ_ERR_INVALID_ARG;
   *out = nullptr;
-  kvq_status st = check_config(cfg);
+  kvq_status st = check_config(cfg, layer_k, layer_v);
   if (st != KVQ_OK) return st;
   if (!arena || (reinterpret_cast<uintptr_t>(arena) % kAlign)) return KVQ_ERR_INVALID_ARG;
-  const uint64_t need = layout(*cfg, nullptr);
+  LayerSides sides;
+  fill_sides(*cfg, layer_k, layer_v, &sides);
+  const uint64_t need = layout(*cfg, sides, nullptr);
   if (arena_bytes < need) return KVQ_ERR_ALLOC;
   kvq_cache* h = new (std::nothrow) kvq_cache();
   if (!h) return KVQ_ERR_ALLOC;
   h->cfg = *cfg;
+  memcpy(h->side, sides.s, sizeof(h->side));
   h->arena = reinterpret_cast<char*>(arena);
   h->arena_bytes = arena_bytes;
-  layout(*cfg, h);
+  layout(*cfg, sides, h);
   for (int l = 0; l < 64; ++l) {
     h->max_len[l] = 0;
     h->chan_set[l] = false;
@@ -366,6 +394,10 @@ kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, 
   }
   *out = h;
   return KVQ_OK;
+}
+
+kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out) {
+  return kvq_create_layers(cfg, nullptr, nullptr, arena, arena_bytes, out);
 }
 
 void kvq_free(kvq_cache* h) {
@@ -419,7 +451,7 @@ kvq_status kvq_set_seq_len(kvq_cache* h, int32_t layer, int32_t len, void* strea
 kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const void* v, int32_t n_new,
                                void* stream) {
   if (!h || !k || !v || layer < 0 || layer >= h->cfg.n_layers || n_new < 1) return KVQ_ERR_INVALID_ARG;
-  if (h->cfg.k.chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
+  if (h->side[layer][0].chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
   if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
   if ((int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
   if ((int64_t)h->cfg.batch * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;

@@ -43,7 +43,7 @@ class kvq_layout(C.Structure):
                 ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32)]
 
 
-EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
+EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_arena_bytes_layers", "kvq_create_layers", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
            "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_decode_attention_noalloc",
            "kvq_error_flags", "kvq_nf4_levels",
            "kvq_last_launch_count", "kvq_status_str"]
@@ -61,6 +61,9 @@ def lib() -> C.CDLL:
         vp, i32, u64p = C.c_void_p, C.c_int32, C.POINTER(C.c_uint64)
         L.kvq_arena_bytes.argtypes = [C.POINTER(kvq_config), u64p]
         L.kvq_create.argtypes = [C.POINTER(kvq_config), vp, C.c_uint64, C.POINTER(vp)]
+        sp = C.POINTER(kvq_side)
+        L.kvq_arena_bytes_layers.argtypes = [C.POINTER(kvq_config), sp, sp, u64p]
+        L.kvq_create_layers.argtypes = [C.POINTER(kvq_config), sp, sp, vp, C.c_uint64, C.POINTER(vp)]
         L.kvq_free.argtypes = [vp]
         L.kvq_free.restype = None
         L.kvq_get_layout.argtypes = [vp, i32, i32, C.POINTER(kvq_layout)]
@@ -136,6 +139,22 @@ class Config:
     anchor_rule: str = "none"
     anchor_n: int = 0
     sm_scale: float = 0.0
+    layer_k: tuple = ()  # per-layer K formats (n_layers Sides); empty: k on every layer
+    layer_v: tuple = ()  # per-layer V formats; empty: v on every layer
+
+    def side(self, layer: int, side: int) -> Side:
+        """Format of (layer, side)."""
+        per = self.layer_k if side == SIDE_K else self.layer_v
+        return per[layer] if per else (self.k if side == SIDE_K else self.v)
+
+    def layer_arrays(self):
+        """(layer_k, layer_v) as C arrays of kvq_side, or None where uniform."""
+        def arr(per):
+            if not per:
+                return None
+            assert len(per) == self.n_layers
+            return (kvq_side * self.n_layers)(*[s.to_c() for s in per])
+        return arr(self.layer_k), arr(self.layer_v)
 
     def to_c(self) -> kvq_config:
         mask = 0
@@ -154,15 +173,23 @@ def kvq_status_str(status: int) -> str:
 def kvq_arena_bytes(cfg: Config) -> int:
     c = cfg.to_c()
     n = C.c_uint64(0)
-    _check(lib().kvq_arena_bytes(C.byref(c), C.byref(n)), "kvq_arena_bytes")
+    if cfg.layer_k or cfg.layer_v:
+        lk, lv = cfg.layer_arrays()
+        _check(lib().kvq_arena_bytes_layers(C.byref(c), lk, lv, C.byref(n)), "kvq_arena_bytes_layers")
+    else:
+        _check(lib().kvq_arena_bytes(C.byref(c), C.byref(n)), "kvq_arena_bytes")
     return n.value
 
 
 def kvq_create(cfg: Config, arena) -> C.c_void_p:
     c = cfg.to_c()
     h = C.c_void_p()
-    _check(lib().kvq_create(C.byref(c), C.c_void_p(arena.data_ptr()), arena.numel() * arena.element_size(),
-                            C.byref(h)), "kvq_create")
+    base, nbytes = C.c_void_p(arena.data_ptr()), arena.numel() * arena.element_size()
+    if cfg.layer_k or cfg.layer_v:
+        lk, lv = cfg.layer_arrays()
+        _check(lib().kvq_create_layers(C.byref(c), lk, lv, base, nbytes, C.byref(h)), "kvq_create_layers")
+    else:
+        _check(lib().kvq_create(C.byref(c), base, nbytes, C.byref(h)), "kvq_create")
     return h
 
 

@@ -22,7 +22,8 @@ def oracle_side(s: Side) -> OQ.Side:
 def oracle_spec(cfg: Config) -> OC.Spec:
     return OC.Spec(cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.n_q_heads, cfg.head_dim, oracle_side(cfg.k),
                    oracle_side(cfg.v), frozenset(cfg.anchor_layers), cfg.anchor_rule, cfg.anchor_n,
-                   cfg.sm_scale or None)
+                   cfg.sm_scale or None, tuple(oracle_side(s) for s in cfg.layer_k),
+                   tuple(oracle_side(s) for s in cfg.layer_v))
 
 
 class Case:
@@ -59,7 +60,7 @@ class Case:
 
     def oracle_unit(self, l, b, h):
         c = self.C[l][h] if l in self.C else None
-        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c)
+        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c, layer=l)
 
     def check_codes(self, l, rows=None):
         """Packed codes, scales and zero points of every unit are bit-identical to the oracle."""
@@ -102,7 +103,7 @@ class Case:
                     o = kq if side == 0 else vq
                     assert np.array_equal(st[b, h].view(np.uint32), o["stored"].astype(np.float32).view(np.uint32)), \
                         f"stored dequant side {side} l{l} b{b} h{h}"
-                    sd = self.spec.k if side == 0 else self.spec.v
+                    sd = OC.side_of(self.spec, l, side == 0)
                     c = self.C[l][h] if (side == 0 and l in self.C) else None
                     want = OQ.to_original_f64(o["exact"], sd, None if c is None else np.broadcast_to(c, o["exact"].shape))
                     an = OC.anchored(self.spec, l, np.arange(self.T), self.T)

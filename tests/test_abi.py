@@ -109,3 +109,40 @@ def test_library_nf4_table_equals_oracle_table():
     inverse CDF); they must agree bit for bit after fp16 rounding."""
     lib_levels = np.array(kvq.kvq_nf4_levels(), dtype=np.float64)
     assert np.array_equal(lib_levels, ORACLE_NF4.nf4_levels())
+
+
+def layers_status(cfg):
+    c = cfg.to_c()
+    n = C.c_uint64(0)
+    lk, lv = cfg.layer_arrays()
+    return kvq.lib().kvq_arena_bytes_layers(C.byref(c), lk, lv, C.byref(n)), n.value
+
+
+def test_per_layer_formats_arena_bytes():
+    """A per-layer table equal to the uniform sides gives the uniform arena; 2-bit K in one
+    layer takes exactly the 2-bit codes' bytes there (same groups, same metadata)."""
+    s4 = Side("int", 4, group=32, rot=128)
+    s2 = Side("int", 2, group=32, rot=128)
+    st_u, n_u = status_of(base_cfg())
+    st_l, n_l = layers_status(base_cfg(layer_k=(s4, s4), layer_v=(s4, s4)))
+    assert st_u == 0 and st_l == 0 and n_u == n_l
+    st_m, n_m = layers_status(base_cfg(layer_k=(s2, s4)))
+    assert st_m == 0
+    units, T = 2 * 2, 512
+    assert n_u - n_m == units * T * (128 * 4 // 8 - 128 * 2 // 8)
+
+
+def test_per_layer_formats_checked_per_entry():
+    bad = Side("int", 9, group=32)
+    ok = Side("int", 3, group=32)
+    assert layers_status(base_cfg(layer_k=(ok, bad)))[0] == -1
+    assert layers_status(base_cfg(layer_v=(ok, Side("int", 4, group=32, chan_scale=True))))[0] == -1
+    assert layers_status(base_cfg(layer_v=(ok, Side("polar", 4, 8, rot=128))))[0] == -1
+    assert layers_status(base_cfg(layer_k=(ok, Side("nf4", group=64)), layer_v=(Side("sign", group=4), ok)))[0] == 0
+    # the uniform field is not read where a per-layer array is given
+    assert layers_status(base_cfg(k=bad, layer_k=(ok, ok)))[0] == 0
+    L = kvq.lib()
+    c = base_cfg(head_dim=96).to_c()
+    h = C.c_void_p()
+    lk, _ = base_cfg(layer_k=(ok, ok)).layer_arrays()
+    assert L.kvq_create_layers(C.byref(c), lk, None, C.c_void_p(256), 1 << 20, C.byref(h)) == -2

@@ -198,3 +198,35 @@ def test_decision_boundaries(D, k, v, chunks):
                                                       adversarial.rows(97 + l, 2, 2, T, D)))
     c.check_codes(0)
     c.check_dequant(0)
+
+
+# ------------------------------------------------------------------------------ per-layer formats
+def test_per_layer_bit_allocation():
+    """"E21W" "Result": rotated groups of 128 with 2-bit K in layers 2 and 7, 4-bit V in layers
+    1, 3 and 4, 3 bits elsewhere (3.19 bits on average).  Each layer is quantized with its own
+    grid and decoded from it."""
+    side = lambda b: Side("int", b, group=128, rot=256)
+    lk = tuple(side(2 if l in (2, 7) else 3) for l in range(8))
+    lv = tuple(side(4 if l in (1, 3, 4) else 3) for l in range(8))
+    cfg = cfg_of(256, side(4), side(4), B=1, H=2, Hq=4, L=8, T=300, layer_k=lk, layer_v=lv)
+    c = Case(cfg, 300)
+    for l in range(8):
+        assert c.cache.layout(l, 0).row_bytes == 256 * lk[l].bits // 8
+        assert c.cache.layout(l, 1).row_bytes == 256 * lv[l].bits // 8
+        c.check_codes(l)
+        c.decode_and_compare(l, queries(cfg, 1, 300, layer=l))
+
+
+def test_per_layer_format_families():
+    """Layers of one cache in different families: each layer takes its own append and decode
+    kernels (tensor-core and CUDA-core paths side by side)."""
+    lk = (Side("nf4", group=64), Side("sign", group=4), Side("int", 3, scale="minmax", group=32),
+          Side("ternary", group=8))
+    lv = (Side("int", 4, group=64), Side("sign", group=4), Side("int", 4, scale="minmax", group=32),
+          Side("ternary", group=8))
+    cfg = cfg_of(128, lk[0], lv[0], B=2, H=2, Hq=8, L=4, T=300, layer_k=lk, layer_v=lv)
+    c = Case(cfg, 300)
+    for l in range(4):
+        c.check_codes(l)
+        c.check_dequant(l)
+        c.decode_and_compare(l, queries(cfg, 2, 300, layer=l))

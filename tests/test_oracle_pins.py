@@ -398,6 +398,23 @@ def test_effective_bits_closed_forms():
     assert b(Side("int", 6, group=128, rot=128), 128) == 6.125
 
 
+def test_per_layer_spec_follows_the_allocation():
+    """"E21W" "Result": the rotated g128 allocation with 2-bit K in layers 2 and 7, 4-bit V in
+    layers 1, 3 and 4 and 3 bits elsewhere averages 3.19 bits (exactly 3.1875 with the scales);
+    each layer's unit is quantized with that layer's own grid."""
+    D = 256
+    side = lambda b: Side("int", b, group=128, rot=256)
+    lk = tuple(side(2 if l in (2, 7) else 3) for l in range(8))
+    lv = tuple(side(4 if l in (1, 3, 4) else 3) for l in range(8))
+    s = C.Spec(8, 1, 1, 1, D, side(4), side(4), layer_k=lk, layer_v=lv)
+    assert C.effective_bits(s, 6000) == 3.1875
+    x = (rng(21).standard_normal((3, D))).astype(np.float16)
+    for l, (kb, vb) in enumerate(zip((3, 3, 2, 3, 3, 3, 3, 2), (3, 4, 3, 4, 4, 3, 3, 3))):
+        kq, vq = C.quantize_unit(s, x, x, None, layer=l)
+        assert kq["bytes"].shape == (3, D * kb // 8) and vq["bytes"].shape == (3, D * vb // 8)
+        assert np.array_equal(kq["bytes"], Q.quantize_rows(x, side(kb))["bytes"])
+
+
 def test_effective_bits_anchor_layer():
     """Post 6 "Corrected semantics" gives 4.69 effective bits for NF4 g64 with layer-0-only
     anchors, which matches one fully fp16 layer out of 26 (Gemma-3-1B depth): 4.25 + 11.75/26."""
