@@ -63,17 +63,6 @@ __device__ __forceinline__ float round_exact_absmax(float x, float d, float inv)
   return k;
 }
 
-// Same decision as round_exact_absmax: the fp32 estimate r = x * (1/d) is within 2^-16 of x/d
-// (|x/d| <= 2^8), so away from a tie (fraction outside [2^-10, 1 - 2^-10] of the half-integer
-// grid) it already gives the exact k; only near a tie do the exact comparisons run.
-__device__ __forceinline__ float round_absmax(float x, float d, float inv) {
-  const float r = __fadd_rn(__fmul_rn(x, inv), 0.5f);
-  const float k = floorf(r);
-  const float fr = __fsub_rn(r, k);
-  if (fr < (1.0f / 1024.0f) || fr > (1.0f - 1.0f / 1024.0f)) return round_exact_absmax(x, d, inv);
-  return k;
-}
-
 // Pack 32 codes of `bits` bits (LSB-first) into bits words at out (skipped unless ok).
 template <int B>
 __device__ __forceinline__ void pack32(const uint32_t* code, uint32_t* out, bool ok) {
