@@ -48,7 +48,7 @@ WORKLOADS = {
     "polar-4+8": dict(L=32, Hkv=8, Hq=32, D=128, B=1, T=8192,
                       k=dict(fmt="polar", bits=4, bits2=8), v=dict(fmt="polar", bits=4, bits2=8),
                       desc="32L x 8kv x 32q, hd128, B1 x 8192; rFFT polar K and V, 4-bit magnitude + 8-bit phase "
-                           "(6.125 b)"),
+                           "(6.125 b); the config names no query-head count: GQA 4 as in the stress workloads"),
     "64k-v3": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
                    k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="int", bits=3, group=128, rot=256),
                    desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K + H256 3-bit V, g128 (3.625 b)"),
