@@ -45,6 +45,11 @@ WORKLOADS = {
     "64k-konly": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
                       k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="fp16"),
                       desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K g128, fp16 V"),
+    "qwen-minmax4": dict(L=8, Hkv=4, Hq=16, D=256, B=16, T=6000,
+                         k=dict(fmt="int", bits=4, scale="minmax", group=32),
+                         v=dict(fmt="int", bits=4, scale="minmax", group=32),
+                         desc="8L x 4kv x 16q, hd256, B16 x 6000; per-token min-max 4-bit g32 K and V (5.0 b); "
+                              "16 sequences so that a step's cache (0.98 GB) exceeds L2"),
     "polar-4+8": dict(L=32, Hkv=8, Hq=32, D=128, B=1, T=8192,
                       k=dict(fmt="polar", bits=4, bits2=8), v=dict(fmt="polar", bits=4, bits2=8),
                       desc="32L x 8kv x 32q, hd128, B1 x 8192; rFFT polar K and V, 4-bit magnitude + 8-bit phase "
