@@ -329,7 +329,7 @@ kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k
   if (!bytes) return KVQ_ERR_INVALID_ARG;
   const kvq_status st = check_config(cfg, layer_k, layer_v);
   if (st != KVQ_OK) return st;
-  LayerSides sides;
+  LayerSides sides{};
   fill_sides(*cfg, layer_k, layer_v, &sides);
   *bytes = layout(*cfg, sides, nullptr);
   return KVQ_OK;
@@ -346,7 +346,7 @@ kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, con
   kvq_status st = check_config(cfg, layer_k, layer_v);
   if (st != KVQ_OK) return st;
   if (!arena || (reinterpret_cast<uintptr_t>(arena) % kAlign)) return KVQ_ERR_INVALID_ARG;
-  LayerSides sides;
+  LayerSides sides{};
   fill_sides(*cfg, layer_k, layer_v, &sides);
   const uint64_t need = layout(*cfg, sides, nullptr);
   if (arena_bytes < need) return KVQ_ERR_ALLOC;
