@@ -309,8 +309,19 @@ class KVCache:
     def set_seq_len(self, layer, length, stream=None):
         kvq_set_seq_len(self.h, layer, length, stream)
 
+    def _check_rows(self, name, x, n=None):
+        """x must be a contiguous fp16 CUDA tensor [batch, n_kv_heads, n, head_dim]."""
+        import torch
+        c = self.cfg
+        if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
+            raise ValueError(f"{name}: need a contiguous fp16 CUDA tensor, got {x.dtype} on {x.device}")
+        if x.dim() != 4 or tuple(x.shape[:2]) != (c.batch, c.n_kv_heads) or x.shape[3] != c.head_dim or \
+                (n is not None and x.shape[2] != n):
+            raise ValueError(f"{name}: need [{c.batch}, {c.n_kv_heads}, n, {c.head_dim}], got {tuple(x.shape)}")
+
     def append(self, layer, k16, v16, stream=None):
-        assert k16.is_contiguous() and v16.is_contiguous() and k16.dtype == v16.dtype
+        self._check_rows("k", k16)
+        self._check_rows("v", v16, k16.shape[2])
         kvq_quantize_append(self.h, layer, k16, v16, k16.shape[2], stream)
 
     def dequantize(self, layer, side, t0, nt, domain=DOMAIN_STORED, fp32=True, stream=None):
@@ -323,6 +334,14 @@ class KVCache:
 
     def decode(self, layer, q16, seq_ids=None, kv_len=None, fp32=True, lse=False, out=None, stream=None):
         import torch
+        c = self.cfg
+        if q16.dtype != torch.float16 or not q16.is_cuda or not q16.is_contiguous() or q16.dim() != 3 or \
+                tuple(q16.shape[1:]) != (c.n_q_heads, c.head_dim):
+            raise ValueError(f"q: need a contiguous fp16 CUDA tensor [n_q, {c.n_q_heads}, {c.head_dim}], got "
+                             f"{q16.dtype} {tuple(q16.shape)} on {q16.device}")
+        for name, t in (("seq_ids", seq_ids), ("kv_len", kv_len)):
+            if t is not None and (t.dtype != torch.int32 or not t.is_cuda or t.numel() != q16.shape[0]):
+                raise ValueError(f"{name}: need an int32 CUDA tensor of n_q = {q16.shape[0]} entries")
         n_q = q16.shape[0]
         if out is None:
             out = torch.empty(n_q, self.cfg.n_q_heads, self.cfg.head_dim, device=q16.device,

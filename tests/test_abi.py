@@ -146,3 +146,19 @@ def test_per_layer_formats_checked_per_entry():
     h = C.c_void_p()
     lk, _ = base_cfg(layer_k=(ok, ok)).layer_arrays()
     assert L.kvq_create_layers(C.byref(c), lk, None, C.c_void_p(256), 1 << 20, C.byref(h)) == -2
+
+
+def test_binding_rejects_bad_tensors_before_the_library():
+    """KVCache checks dtype, device, layout and shape on the host (no handle is touched)."""
+    import torch
+    cache = kvq.KVCache.__new__(kvq.KVCache)
+    cache.cfg = base_cfg()
+    cache.h = None
+    k32 = torch.zeros(2, 2, 3, 128, dtype=torch.float32)
+    k16 = torch.zeros(2, 2, 3, 128, dtype=torch.float16)
+    with pytest.raises(ValueError, match="fp16 CUDA"):
+        cache.append(0, k32, k32)
+    with pytest.raises(ValueError, match="fp16 CUDA"):
+        cache.append(0, k16, k16)  # host tensor
+    with pytest.raises(ValueError, match="q: need"):
+        cache.decode(0, torch.zeros(2, 4, 128, dtype=torch.float16))
