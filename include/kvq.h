@@ -20,9 +20,13 @@
  *
  * Error behaviour: argument and configuration errors are detected on the host before any
  * launch and returned as a status; launch failures come back as KVQ_ERR_CUDA.  No kernel
- * traps or spins.  A device-side condition the host cannot see in advance (an append past
- * the capacity while a CUDA graph replays) skips the offending writes and raises a bit in
- * the cache's error word (kvq_error_flags).
+ * traps.  A device-side condition the host cannot see in advance (an append past the capacity
+ * while a CUDA graph replays, a bad sequence id) skips the offending writes and raises a bit in
+ * the cache's error word (kvq_error_flags).  The only wait in any kernel is the decode's poll
+ * for a staged tile, bounded (about one second; KVQ_ERRF_WAIT_TIMEOUT when it runs out).  Test
+ * hook: with the environment variable KVQ_TEST_STALL_FIRST_WAIT=<cycles> set when a handle is
+ * created, the first such wait of every tensor-core decode CTA of that handle polls a barrier
+ * that nothing arrives on for that many clock cycles and then takes the give-up path.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -126,7 +130,12 @@ kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k
 kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
                              uint64_t arena_bytes, kvq_cache** out);
 
-/* Release the handle and its workspace (not the arena).  NULL is a no-op. */
+/* Release the handle and its split-K workspace; the caller-owned arena (the packed cache itself)
+ * is left untouched and may be freed by the caller afterwards.  NULL is a no-op.  Synchronous
+ * (cudaFree).  The pages manage no handle: their cache memory is what the configuration budgets
+ * ([LCPP] "Finding 1": an f16 cache that no longer fits where the q4_0 one does; [E22L] "What I
+ * tested": the bytes per token a 1M-token budget allows), and that memory belongs to the caller
+ * here. */
 void kvq_free(kvq_cache* cache);
 
 /* Geometry of (layer, side) for inspection and tests.  Host only. */
@@ -141,23 +150,38 @@ kvq_status kvq_set_chan_scale(kvq_cache* cache, int32_t layer, const void* c_fp1
  * kvq_set_seq_len(cache, -1, 0, s) empties the cache. */
 kvq_status kvq_set_seq_len(kvq_cache* cache, int32_t layer, int32_t len, void* stream);
 
-/* Append n_new tokens to every sequence of `layer`: k, v are fp16 device [batch][n_kv_heads]
- * [n_new][head_dim].  Token i of sequence b lands at position seq_len[b] + i (read on the
- * device), every row is quantized (pre-transform, group scales, codes, packing), rows in
- * the anchor set are also kept as fp16, and seq_len[b] += n_new.  n_new = prompt length is
- * the bulk prefill; n_new = 1 is the decode-time append.  Errors: KVQ_ERR_CAPACITY if the
- * host-side length bound would pass capacity; KVQ_ERR_STATE if a channel scale is required
- * and was never set.  [E22L] "What I tested" (keys and values quantized on entry to the
- * cache), [FMKQ] post 6 "Corrected semantics" (every layer quantized, anchors as extra
- * protection). */
-kvq_status kvq_quantize_append(kvq_cache* cache, int32_t layer, const void* k_fp16,
-                               const void* v_fp16, int32_t n_new, void* stream);
+/* Append n_new tokens to n_seqs sequences of `layer`.
+ *   seq_ids: int32 device [n_seqs], the sequences that receive rows, distinct, in [0, batch);
+ *            or NULL: every sequence in order (then n_seqs must equal batch).
+ *   k, v:    fp16 device [n_seqs][n_kv_heads][n_new][head_dim] (16-byte aligned), row s for
+ *            sequence seq_ids[s] (or s).
+ * Token i of sequence b lands at position seq_len[b] + i (read on the device); every row is
+ * quantized (pre-transform, group scales, codes, packing), rows in the anchor set are also
+ * kept as fp16, and seq_len[b] += n_new.  Sequences not listed are untouched.  n_new = prompt
+ * length is the bulk prefill; n_new = 1 is the decode-time append.
+ * Errors: KVQ_ERR_INVALID_ARG for a bad pointer, layer or count; KVQ_ERR_CAPACITY if n_new >
+ * capacity or, with seq_ids NULL, if the host-side length bound would pass capacity;
+ * KVQ_ERR_STATE if a channel scale is required and was never set.  On the device (so also
+ * under graph replay): a listed sequence with no room for all n_new rows gets none of them and
+ * keeps its length (KVQ_ERRF_CAPACITY in the error word); an id outside [0, batch) is skipped
+ * (KVQ_ERRF_SEQ_ID).  A repeated id is a caller error: its rows race and its length advances
+ * once per listing.
+ * Sources: [E22L] "What I tested" (keys and values quantized on entry to the cache), [FMKQ]
+ * post 6 "Corrected semantics" (every layer quantized, anchors as extra protection). */
+kvq_status kvq_quantize_append(kvq_cache* cache, int32_t layer, const void* k_fp16, const void* v_fp16,
+                               const int32_t* seq_ids, int32_t n_seqs, int32_t n_new, void* stream);
 
 /* Reconstruct tokens [t0, t0 + nt) of every (sequence, kv-head) of one side of `layer` into
- * out [batch][n_kv_heads][nt][head_dim] (fp32 if out_fp32 else fp16).  STORED domain: the
- * grid values (code x scale + zero; polar m cos(phi), m sin(phi) slot-interleaved) before
- * any inverse transform, bit-exact by definition.  ORIGINAL domain: inverse DFT, inverse
- * rotation and x channel scale applied, and anchored rows replaced by their fp16 copy. */
+ * out [batch][n_kv_heads][nt][head_dim] (fp32 if out_fp32 else fp16), device, caller-owned.
+ * STORED domain: the grid values (code x scale + zero; polar m cos(phi), m sin(phi)
+ * slot-interleaved) before any inverse transform, bit-exact by definition.  ORIGINAL domain:
+ * inverse DFT, inverse rotation and x channel scale applied, and anchored rows replaced by
+ * their fp16 copy.  Rows at or past a sequence's stored length hold whatever the arena held.
+ * Errors: KVQ_ERR_INVALID_ARG for a bad layer, side, domain or range (t0 + nt > capacity).
+ * Sources: the dequantized cache is what the pages' simulations attend over ([E22L] "What I
+ * tested": keys and values quantized, then dequantized, on entry to the cache) and what their
+ * K/V error is measured on ([E21W] "What I tested": squared error over signal energy; [E21W]
+ * variants C/D: channel scales multiplied back after dequantizing). */
 kvq_status kvq_dequantize(const kvq_cache* cache, int32_t layer, int32_t side, int32_t domain,
                           int32_t t0, int32_t nt, void* out, int32_t out_fp32, void* stream);
 
@@ -170,25 +194,29 @@ kvq_status kvq_dequantize(const kvq_cache* cache, int32_t layer, int32_t side, i
  * Split-K over tokens, dequantizing in registers, query pre-transformed once (q' = H(c . q)
  * or the rFFT adjoint), partials merged by a second kernel that also undoes V's transform.
  * An empty key range gives out = 0 and lse = -inf.  Errors: KVQ_ERR_CAPACITY if n_q >
- * max_queries.  [E21W] "What I tested" (attention output, causal proxy queries). */
+ * max_queries.  The split-K partials go to the handle's one workspace, shared by all layers:
+ * decode calls on one handle must not overlap on the GPU (issue them on one stream, or order
+ * the streams).  [E21W] "What I tested" (attention output, causal proxy queries). */
 kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q_fp16, int32_t n_q,
                                 const int32_t* seq_ids, const int32_t* kv_len, void* out,
                                 int32_t out_fp32, float* lse, void* stream);
 
 /* kvq_decode_attention without any device allocation behind it.  Same arguments, same results,
- * same errors, plus KVQ_ERR_CAPACITY when the split-K partials of this call (n_q x n_q_heads x
- * (splits + 1) x (head_dim + 4) floats) exceed the library's fixed scratch of 2^21 floats
- * (8 MiB), and KVQ_ERR_INVALID_ARG when the current device is not the handle's.  The pages have
- * no counterpart: this is an interface convenience.
- * For callers that cannot call cudaMalloc where they decode: code running while a stream is
- * captured into a CUDA graph in global mode (where cudaMalloc is illegal), or a serving runtime
- * that hands nearly all of HBM to its own pool and budgets every other byte.  The scratch is a
- * file-scope device array that every GPU loading this library holds until the process exits.
- * The first call on a device looks up that array's device address (cudaGetSymbolAddress, with
- * that device current); make the first call before any stream capture.  All calls share the
- * array, so calls that overlap on the GPU (different streams, or different handles on one
- * device) race; serialize them.  Each call writes every partial it reads, so nothing is cleared
- * between calls.  The handle from kvq_create keeps its own workspace; this call leaves it alone. */
+ * same errors (KVQ_ERR_CAPACITY for n_q > max_queries included), plus KVQ_ERR_CAPACITY when the
+ * split-K partials of this call (n_q x n_q_heads x (splits + 1) x (head_dim + 4) floats) exceed
+ * the library's fixed scratch of 2^21 floats (8 MiB), and KVQ_ERR_INVALID_ARG when the current
+ * device is not the handle's.  The pages have no counterpart: this is an interface convenience.
+ * For callers that cannot call cudaMalloc where they decode: a serving runtime that hands
+ * nearly all of HBM to its own pool and budgets every other byte, or a latency-critical decode
+ * loop that must not make the implicit device synchronisation a cudaMalloc/cudaFree can cause.
+ * The scratch is a file-scope device array that every GPU loading this library holds until the
+ * process exits.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that first call before
+ * any stream capture, and do not use the call after a cudaDeviceReset (the kept address is then
+ * stale).  All calls share the array, so calls that overlap on the GPU (different streams, or
+ * different handles on one device) race; serialize them.  Each call writes every partial it
+ * reads, so nothing is cleared between calls.  The handle from kvq_create keeps its own
+ * workspace; this call leaves it alone. */
 kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q_fp16, int32_t n_q,
                                         const int32_t* seq_ids, const int32_t* kv_len, void* out,
                                         int32_t out_fp32, float* lse, void* stream);

@@ -186,16 +186,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete; false after about one second of polling.
+// Wait for phase `parity` of `bar` to complete; false after `limit` clock cycles of polling
+// (by default about one second).
 constexpr long long kWaitCycles = 2000000000LL;
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   return true;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity);
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kWaitCycles) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, limit);
 }
 
 // N consecutive 32-bit words from 4N-byte aligned shared memory
@@ -279,7 +280,7 @@ struct TcCfg {
   static constexpr int LUT_BYTES = (KF == CF_NF4 || KTRN || VTRN) ? 256 * 32 * 4 : 0;
   static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_X = OFF_LUT + LUT_BYTES;
   static constexpr int OFF_BAR = OFF_X + NW * XW;
-  static constexpr int SMEM = OFF_BAR + 2 * STAGES * 8;  // full and empty barriers
+  static constexpr int SMEM = OFF_BAR + 2 * STAGES * 8 + 16;  // full and empty barriers, test barrier, abort flag
 
   static_assert(KCB % 4 == 0, "K chunks must be whole words");
   static_assert(!(KTRN || VTRN) || (D == 128 && TPW == 32 && GK == 8 && GV == 8), "ternary instance shape");
@@ -415,6 +416,8 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // full[s]: tile landed (bytes)
   uint64_t* ebar = bar + STAGES;                                      // empty[s]: every consumer warp done
+  uint64_t* dummy = ebar + STAGES;                                    // never arrived on (test hook)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dummy + 1);  // a consumer gave up
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -461,6 +464,8 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
       mbar_init(bar + s, 1);
       mbar_init(ebar + s, NW);
     }
+    mbar_init(dummy, 1);
+    *abort_flag = 0;
     mbar_init_fence();
   }
   __syncthreads();
@@ -556,6 +561,7 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
           timed_out = true;
           break;
         }
+        if (*abort_flag) break;  // a consumer gave up: the stage may still be landing
         issue(it0 + issued, s);
       }
     }
@@ -565,12 +571,18 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
       if (tid == 0 && it + STAGES - 1 < nmy) issue(it0 + it + STAGES - 1, (it + STAGES - 1) % STAGES);
     }
     const int stage = it % STAGES;
-    if (!timed_out && __any_sync(0xffffffffu, !mbar_wait(bar + stage, (uint32_t)(it / STAGES) & 1u))) {
+    // (test hook: the first wait polls a barrier nothing arrives on, for L.test_stall cycles)
+    const bool stall = L.test_stall > 0 && it == 0;
+    if (!timed_out && __any_sync(0xffffffffu, !(stall ? mbar_wait(dummy, 0u, L.test_stall)
+                                                      : mbar_wait(bar + stage, (uint32_t)(it / STAGES) & 1u)))) {
       if (lane == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_WAIT_TIMEOUT);
       timed_out = true;
     }
-    if (timed_out) {  // release the stage without reading it
-      if (C::PROD && lane == 0) mbar_arrive(ebar + stage);
+    if (timed_out) {  // release the stage without reading it; the producer issues no more tiles
+      if (C::PROD && lane == 0) {
+        *abort_flag = 1;
+        mbar_arrive(ebar + stage);
+      }
       continue;
     }
 

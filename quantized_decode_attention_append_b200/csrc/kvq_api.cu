@@ -1,6 +1,7 @@
 // C ABI of libkvq: configuration checks, arena layout, handle lifetime, launch wrappers.
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -24,8 +25,10 @@ struct kvq_cache {
   int64_t chan[64];
   int64_t lens, tickets, err;
   int anchor_rows;
-  int max_len[64];
+  int max_len[64];       // host-side bound on every sequence's length (exact while len_exact)
+  bool len_exact[64];    // false once a per-sequence append made the bound inexact
   bool chan_set[64];
+  long long test_stall;  // decode test hook, from KVQ_TEST_STALL_FIRST_WAIT (0 = off)
   float* work;
   size_t work_floats;
   int device, num_sms;
@@ -214,6 +217,10 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
     S.n_groups = so.n_groups;
   }
   L.B = c.batch;
+  L.cap = c.capacity;
+  L.app_ids = nullptr;
+  L.app_n = c.batch;
+  L.test_stall = h->test_stall;
   L.Hkv = c.n_kv_heads;
   L.Hq = c.n_q_heads;
   L.D = c.head_dim;
@@ -359,7 +366,18 @@ kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, con
   layout(*cfg, sides, h);
   for (int l = 0; l < 64; ++l) {
     h->max_len[l] = 0;
+    h->len_exact[l] = true;
     h->chan_set[l] = false;
+  }
+  // Test hook: with KVQ_TEST_STALL_FIRST_WAIT=<cycles> set when the handle is created, the first
+  // staged-tile wait of every tensor-core decode CTA polls a barrier that nothing arrives on, for
+  // that many clock cycles, then takes the give-up path (KVQ_ERRF_WAIT_TIMEOUT, empty partial,
+  // copies already issued drained).  Unset or 0: off.
+  h->test_stall = 0;
+  if (const char* w = getenv("KVQ_TEST_STALL_FIRST_WAIT")) {
+    char* end = nullptr;
+    const long long v = strtoll(w, &end, 10);
+    if (end != w && v > 0 && v <= 2000000000LL) h->test_stall = v;
   }
   if (cudaGetDevice(&h->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
@@ -440,28 +458,40 @@ kvq_status kvq_set_seq_len(kvq_cache* h, int32_t layer, int32_t len, void* strea
   cudaError_t e;
   if (layer < 0) {
     e = launch_fill_len(lens, B * h->cfg.n_layers, len, reinterpret_cast<cudaStream_t>(stream));
-    for (int l = 0; l < h->cfg.n_layers; ++l) h->max_len[l] = len;
+    for (int l = 0; l < h->cfg.n_layers; ++l) {
+      h->max_len[l] = len;
+      h->len_exact[l] = true;
+    }
   } else {
     e = launch_fill_len(lens + (size_t)layer * B, B, len, reinterpret_cast<cudaStream_t>(stream));
     h->max_len[layer] = len;
+    h->len_exact[layer] = true;
   }
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
-kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const void* v, int32_t n_new,
-                               void* stream) {
+kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const void* v, const int32_t* seq_ids,
+                               int32_t n_seqs, int32_t n_new, void* stream) {
   if (!h || !k || !v || layer < 0 || layer >= h->cfg.n_layers || n_new < 1) return KVQ_ERR_INVALID_ARG;
+  if (seq_ids ? (n_seqs < 1 || n_seqs > h->cfg.batch) : n_seqs != h->cfg.batch) return KVQ_ERR_INVALID_ARG;
   if (h->side[layer][0].chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
   if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
-  if ((int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
-  if ((int64_t)h->cfg.batch * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
-  const LayerDev L = layer_dev(h, layer);
+  if (n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  // every sequence advances together: the host bound is exact and decides; otherwise the device
+  // checks each listed sequence
+  if (!seq_ids && h->len_exact[layer] && (int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  if ((int64_t)n_seqs * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
+  LayerDev L = layer_dev(h, layer);
+  L.app_ids = seq_ids;
+  L.app_n = n_seqs;
   int launches = 0;
   const cudaError_t e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,
-                                      h->max_len[layer], reinterpret_cast<cudaStream_t>(stream), &launches);
+                                      reinterpret_cast<cudaStream_t>(stream), &launches);
   h->last_launches = launches;
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
-  h->max_len[layer] += n_new;
+  const int64_t nl = (int64_t)h->max_len[layer] + n_new;
+  h->max_len[layer] = (int)(nl < h->cfg.capacity ? nl : h->cfg.capacity);
+  if (seq_ids) h->len_exact[layer] = false;
   return KVQ_OK;
 }
 
@@ -495,6 +525,7 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* h, int32_t layer, const void*
                                         const int32_t* seq_ids, const int32_t* kv_len, void* out, int32_t out_fp32,
                                         float* lse, void* stream) {
   if (!h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || n_q < 1) return KVQ_ERR_INVALID_ARG;
+  if (n_q > h->cfg.max_queries) return KVQ_ERR_CAPACITY;
   if (!seq_ids && n_q > h->cfg.batch) return KVQ_ERR_INVALID_ARG;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;

@@ -27,12 +27,18 @@ struct SideDev {
 struct LayerDev {
   SideDev s[2];
   int B, Hkv, Hq, D, Tcap;
+  int cap;               // configured capacity (tokens per sequence); appends never pass it
   int anchored;          // this layer keeps anchor rows
   int anchor_rule, anchor_n, anchor_rows;
   int* seq_len;          // [B] stored lengths of this layer
   unsigned* ticket;      // append completion counter of this layer
   unsigned* err;         // error word (KVQ_ERRF_*)
   float sm_scale;
+  // append call: sequences that receive rows (null: every sequence, in order) and how many
+  const int* app_ids;
+  int app_n;
+  long long test_stall;  // test hook (0 = off): the decode's first stage wait polls a barrier nothing
+                         // arrives on for this many clock cycles, then gives up
 };
 
 // Tables the host builds once (NF4 levels, FFT twiddles, phase cos/sin) and every
@@ -52,8 +58,8 @@ cudaError_t upload_tables_decode(const HostTables& t);
 cudaError_t upload_tables_dequant(const HostTables& t);
 
 // Launchers (host side, validate nothing; the API validates first).
-cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new,
-                          int max_len_before, cudaStream_t st, int* launches);
+cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, cudaStream_t st,
+                          int* launches);
 cudaError_t launch_dequant(const LayerDev& L, int side, int domain, int t0, int nt, void* out,
                            int out_fp32, cudaStream_t st);
 cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int* seq_ids,

@@ -150,17 +150,51 @@ __device__ __forceinline__ int anchor_slot(const LayerDev& L, int pos) {
   return (L.anchor_rule == KVQ_ANCHOR_WINDOW) ? (pos % L.anchor_n) : pos;
 }
 
-// Completion ticket: the last CTA of an append (over all its launches) advances seq_len.
-// Every CTA read seq_len before it takes its ticket, so the update cannot race a reader.
+// Where appended row `row` lands.  Input rows are ordered (listed sequence, kv-head, token);
+// the listed sequence is L.app_ids[s] (or s when the list is null).  A sequence whose rows would
+// pass the capacity, or an id outside [0, B), gets none of its rows written; `err` names why and
+// `first` marks the row (token 0 of kv-head 0) that reports it.
+struct RowDst {
+  int u, pos, len_after;
+  unsigned err;
+  bool first;
+};
+__device__ __forceinline__ RowDst row_dst(const LayerDev& L, long long row, int n_new) {
+  RowDst d{0, 0, 0, 0u, false};
+  const long long ul = row / n_new;
+  const int i = (int)(row - ul * n_new);
+  const int sl = (int)(ul / L.Hkv), h = (int)(ul - (long long)sl * L.Hkv);
+  const int b = L.app_ids ? L.app_ids[sl] : sl;
+  d.first = i == 0 && h == 0;
+  if (b < 0 || b >= L.B) {
+    d.err = KVQ_ERRF_SEQ_ID;
+    return d;
+  }
+  const int len0 = L.seq_len[b];
+  if (len0 + n_new > L.cap) {
+    d.err = KVQ_ERRF_CAPACITY;
+    return d;
+  }
+  d.u = b * L.Hkv + h;
+  d.pos = len0 + i;
+  d.len_after = len0 + n_new;
+  return d;
+}
+
+// Completion ticket: the last CTA of an append (over all its launches) advances the lengths of
+// the listed sequences that had room (the same test every row of theirs took).  Every CTA read
+// seq_len before it takes its ticket, so the update cannot race a reader.
 __device__ __forceinline__ void finish_append(const LayerDev& L, int n_new, unsigned total_ctas) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned t = atomicAdd(L.ticket, 1u);
     if (t == total_ctas - 1) {
-      for (int b = 0; b < L.B; ++b) {
+      for (int s = 0; s < L.app_n; ++s) {
+        const int b = L.app_ids ? L.app_ids[s] : s;
+        if (b < 0 || b >= L.B) continue;
         const int nl = L.seq_len[b] + n_new;
-        L.seq_len[b] = nl < L.Tcap ? nl : L.Tcap;
+        if (nl <= L.cap) L.seq_len[b] = nl;
       }
       *L.ticket = 0u;
       __threadfence();
@@ -182,23 +216,14 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
   __shared__ float sre[kFftWarps][128], sim[kFftWarps][128];
   __shared__ uint32_t scode[kFftWarps][128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long R = (long long)L.B * L.Hkv * n_new;
+  const long long R = (long long)L.app_n * L.Hkv * n_new;
   for (long long row = (long long)blockIdx.x * kFftWarps + warp; row < R; row += (long long)gridDim.x * kFftWarps) {
-  bool ok = true;
-  int pos = 0, len_after = 0, u = 0, i = 0;
-  {
-    i = (int)(row % n_new);
-    u = (int)(row / n_new);
-    const int len0 = L.seq_len[u / L.Hkv];
-    pos = len0 + i;
-    len_after = len0 + n_new;
-    if (pos >= L.Tcap) {
-      if (lane == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
-      ok = false;
-    }
-  }
+  const RowDst dst = row_dst(L, row, n_new);
+  const bool ok = dst.err == 0;
+  const int pos = dst.pos, len_after = dst.len_after, u = dst.u;
+  if (!ok && dst.first && lane == 0) atomicOr(L.err, dst.err);
   if (ok) {
-    const __half* rp = src + ((long long)u * n_new + i) * 128;
+    const __half* rp = src + row * 128;
     float* re = sre[warp];
     float* im = sim[warp];
     for (int j = lane; j < 128; j += 32) {
@@ -391,7 +416,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   constexpr int NW = kRowThreads / 32;
   const int rpw = 32 / lpr;                           // rows per warp
   const int li = lane % lpr;                          // this lane's 32-value slice of its row
-  const int R = L.B * L.Hkv * n_new;                  // < 2^31 (checked on the host)
+  const int R = L.app_n * L.Hkv * n_new;              // < 2^31 (checked on the host)
   constexpr int LG = G > 32 ? G / 32 : 1;             // lanes per group
   constexpr int GPL = G > 32 ? 1 : 32 / G;            // groups per lane
   // code bits: fixed by the family, by the instance (BITS > 0), or read from the side
@@ -422,18 +447,15 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
       }
     }
-    int i = 0, u = 0, pos = 0, len_after = 0;
+    int u = 0, pos = 0, len_after = 0;
     bool ok = row < R;
     if (ok) {
-      u = row / n_new;
-      i = row - u * n_new;
-      const int len0 = L.seq_len[u / L.Hkv];
-      pos = len0 + i;
-      len_after = len0 + n_new;
-      if (pos >= L.Tcap) {
-        if (li == 0 && i == 0) atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
-        ok = false;
-      }
+      const RowDst d = row_dst(L, row, n_new);
+      if (d.err && d.first && li == 0) atomicOr(L.err, d.err);
+      ok = d.err == 0;
+      u = d.u;
+      pos = d.pos;
+      len_after = d.len_after;
     }
     float x[32];
     __half2 raw2[16];  // the lane's 32 input values as stored (fp16 pairs)
@@ -797,22 +819,19 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
                                    unsigned total_ctas) {
   const SideDev& S = L.s[side];
   const int vec_per_row = L.D / 8;
-  const long long R = (long long)L.B * L.Hkv * n_new;
+  const long long R = (long long)L.app_n * L.Hkv * n_new;
   for (long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x; gt < R * vec_per_row;
        gt += (long long)gridDim.x * blockDim.x) {
   const long long row = gt / vec_per_row;
   const int c = (int)(gt % vec_per_row);
-  {
-    const int i = (int)(row % n_new), u = (int)(row / n_new);
-    const int pos = L.seq_len[u / L.Hkv] + i;
-    if (pos < L.Tcap) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + ((long long)u * n_new + i) * L.D) + c);
-      reinterpret_cast<uint4*>(S.codes + ((long long)u * L.Tcap + pos) * S.row_bytes)[c] = w;
-      if (in_anchor(L, pos, L.seq_len[u / L.Hkv] + n_new))
-        reinterpret_cast<uint4*>(S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * L.D)[c] = w;
-    } else if (c == 0 && i == 0) {
-      atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);
-    }
+  const RowDst d = row_dst(L, row, n_new);
+  if (d.err == 0) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + row * L.D) + c);
+    reinterpret_cast<uint4*>(S.codes + ((long long)d.u * L.Tcap + d.pos) * S.row_bytes)[c] = w;
+    if (in_anchor(L, d.pos, d.len_after))
+      reinterpret_cast<uint4*>(S.anchors + ((long long)d.u * L.anchor_rows + anchor_slot(L, d.pos)) * L.D)[c] = w;
+  } else if (c == 0 && d.first) {
+    atomicOr(L.err, d.err);
   }
   }
   finish_append(L, n_new, total_ctas);
@@ -828,7 +847,7 @@ struct SidePlan {
 
 static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
   const SideDev& S = L.s[side];
-  const long long R = (long long)L.B * L.Hkv * n_new;
+  const long long R = (long long)L.app_n * L.Hkv * n_new;
   SidePlan p{nullptr, 0, 128};
   if (S.fmt == KVQ_FMT_FP16) {
     p.kern = append_fp16_kernel;
@@ -877,8 +896,8 @@ static KvKernel pick_kv_kernel(const LayerDev& L) {
   return nullptr;
 }
 
-cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, int /*max_len_before*/,
-                          cudaStream_t st, int* launches) {
+cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, cudaStream_t st,
+                          int* launches) {
   const SidePlan pk = plan_side(L, 0, n_new), pv = plan_side(L, 1, n_new);
   if (!pk.kern || !pv.kern) return cudaErrorInvalidValue;
   const unsigned total = pk.blocks + pv.blocks;

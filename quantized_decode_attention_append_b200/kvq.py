@@ -69,7 +69,7 @@ def lib() -> C.CDLL:
         L.kvq_get_layout.argtypes = [vp, i32, i32, C.POINTER(kvq_layout)]
         L.kvq_set_chan_scale.argtypes = [vp, i32, vp, vp]
         L.kvq_set_seq_len.argtypes = [vp, i32, i32, vp]
-        L.kvq_quantize_append.argtypes = [vp, i32, vp, vp, i32, vp]
+        L.kvq_quantize_append.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp]
         L.kvq_dequantize.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp]
         L.kvq_decode_attention.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
         L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
@@ -211,8 +211,9 @@ def kvq_set_seq_len(h, layer: int, length: int, stream=None):
     _check(lib().kvq_set_seq_len(h, layer, length, _stream(stream)), "kvq_set_seq_len")
 
 
-def kvq_quantize_append(h, layer: int, k16, v16, n_new: int, stream=None):
-    _check(lib().kvq_quantize_append(h, layer, _ptr(k16), _ptr(v16), n_new, _stream(stream)), "kvq_quantize_append")
+def kvq_quantize_append(h, layer: int, k16, v16, seq_ids, n_seqs: int, n_new: int, stream=None):
+    _check(lib().kvq_quantize_append(h, layer, _ptr(k16), _ptr(v16), _ptr(seq_ids), n_seqs, n_new, _stream(stream)),
+           "kvq_quantize_append")
 
 
 def kvq_dequantize(h, layer: int, side: int, domain: int, t0: int, nt: int, out, stream=None):
@@ -309,20 +310,34 @@ class KVCache:
     def set_seq_len(self, layer, length, stream=None):
         kvq_set_seq_len(self.h, layer, length, stream)
 
-    def _check_rows(self, name, x, n=None):
-        """x must be a contiguous fp16 CUDA tensor [batch, n_kv_heads, n, head_dim]."""
+    def _check_device(self, name, x):
+        if x.device != self.arena.device:
+            raise ValueError(f"{name}: on {x.device}, the cache arena is on {self.arena.device}")
+
+    def _check_rows(self, name, x, n_seqs, n=None):
+        """x must be a contiguous fp16 tensor [n_seqs, n_kv_heads, n, head_dim] on the arena's device."""
         import torch
         c = self.cfg
         if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
             raise ValueError(f"{name}: need a contiguous fp16 CUDA tensor, got {x.dtype} on {x.device}")
-        if x.dim() != 4 or tuple(x.shape[:2]) != (c.batch, c.n_kv_heads) or x.shape[3] != c.head_dim or \
+        if x.dim() != 4 or tuple(x.shape[:2]) != (n_seqs, c.n_kv_heads) or x.shape[3] != c.head_dim or \
                 (n is not None and x.shape[2] != n):
-            raise ValueError(f"{name}: need [{c.batch}, {c.n_kv_heads}, n, {c.head_dim}], got {tuple(x.shape)}")
+            raise ValueError(f"{name}: need [{n_seqs}, {c.n_kv_heads}, n, {c.head_dim}], got {tuple(x.shape)}")
+        self._check_device(name, x)
 
-    def append(self, layer, k16, v16, stream=None):
-        self._check_rows("k", k16)
-        self._check_rows("v", v16, k16.shape[2])
-        kvq_quantize_append(self.h, layer, k16, v16, k16.shape[2], stream)
+    def append(self, layer, k16, v16, seq_ids=None, stream=None):
+        """Append k16/v16 [n_seqs, n_kv_heads, n, head_dim] to the sequences `seq_ids` (an int32
+        CUDA tensor of n_seqs distinct ids) or, with seq_ids None, to every sequence (n_seqs = batch)."""
+        import torch
+        n_seqs = self.cfg.batch
+        if seq_ids is not None:
+            if seq_ids.dtype != torch.int32 or not seq_ids.is_cuda or seq_ids.dim() != 1 or not seq_ids.is_contiguous():
+                raise ValueError("seq_ids: need a contiguous 1-D int32 CUDA tensor")
+            self._check_device("seq_ids", seq_ids)
+            n_seqs = seq_ids.numel()
+        self._check_rows("k", k16, n_seqs)
+        self._check_rows("v", v16, n_seqs, k16.shape[2])
+        kvq_quantize_append(self.h, layer, k16, v16, seq_ids, n_seqs, k16.shape[2], stream)
 
     def dequantize(self, layer, side, t0, nt, domain=DOMAIN_STORED, fp32=True, stream=None):
         import torch
@@ -339,13 +354,23 @@ class KVCache:
                 tuple(q16.shape[1:]) != (c.n_q_heads, c.head_dim):
             raise ValueError(f"q: need a contiguous fp16 CUDA tensor [n_q, {c.n_q_heads}, {c.head_dim}], got "
                              f"{q16.dtype} {tuple(q16.shape)} on {q16.device}")
+        self._check_device("q", q16)
         for name, t in (("seq_ids", seq_ids), ("kv_len", kv_len)):
-            if t is not None and (t.dtype != torch.int32 or not t.is_cuda or t.numel() != q16.shape[0]):
-                raise ValueError(f"{name}: need an int32 CUDA tensor of n_q = {q16.shape[0]} entries")
+            if t is not None and (t.dtype != torch.int32 or not t.is_cuda or t.numel() != q16.shape[0] or
+                                  not t.is_contiguous()):
+                raise ValueError(f"{name}: need a contiguous int32 CUDA tensor of n_q = {q16.shape[0]} entries")
+            if t is not None:
+                self._check_device(name, t)
         n_q = q16.shape[0]
         if out is None:
             out = torch.empty(n_q, self.cfg.n_q_heads, self.cfg.head_dim, device=q16.device,
                               dtype=torch.float32 if fp32 else torch.float16)
+        elif out.dtype not in (torch.float32, torch.float16) or not out.is_cuda or not out.is_contiguous() or \
+                tuple(out.shape) != (n_q, c.n_q_heads, c.head_dim):
+            raise ValueError(f"out: need a contiguous fp32 or fp16 CUDA tensor [{n_q}, {c.n_q_heads}, {c.head_dim}], "
+                             f"got {out.dtype} {tuple(out.shape)} on {out.device}")
+        else:
+            self._check_device("out", out)
         l = torch.empty(n_q, self.cfg.n_q_heads, device=q16.device, dtype=torch.float32) if lse else None
         kvq_decode_attention(self.h, layer, q16, n_q, seq_ids, kv_len, out, l, stream)
         return (out, l) if lse else out

@@ -63,3 +63,50 @@ def rows(seed: int, B: int, H: int, T: int, D: int) -> np.ndarray:
                             r[c0:c0 + 8] = np.where(rng.random(8) < 0.5, 0.0, -0.0)
                 out[b, h, t] = r.astype(np.float16)
     return out
+
+
+def spike_rows(seed: int, B: int, H: int, T: int, D: int, n: int) -> np.ndarray:
+    """Rows whose orthonormal Hadamard image (blocks of n) lands on absmax ties.
+
+    Each n-channel block holds three spikes (2^(b-1), 2^(b-1) - 1/2, 1/2) x u at random channels,
+    b in {2, 3, 4} and u a power of two drawn per row.  The block's image is
+    (+-2^(b-1) +- (2^(b-1) - 1/2) +- 1/2) u / sqrt(n): magnitudes 2^b u, (2^b - 1) u, u and 0
+    (over sqrt n), so a group's largest magnitude usually occurs with both signs (the first-index
+    rule decides) and the b-bit grid's x/d hits half-integers exactly when 1/sqrt(n) is exact
+    (n = 256) and within one rounding otherwise (n = 128).  A quarter of the rows add small
+    Gaussian noise so that near-ties are reached from both sides."""
+    rng = np.random.default_rng(seed)
+    out = np.zeros((B, H, T, D), dtype=np.float16)
+    for b_ in range(B):
+        for h in range(H):
+            for t in range(T):
+                r = np.zeros(D)
+                for blk in range(0, D, n):
+                    b = int(rng.integers(2, 5))
+                    u = 2.0 ** int(rng.integers(-3, 3))
+                    ch = blk + rng.choice(n, size=3, replace=False)
+                    r[ch] = np.array([2.0 ** (b - 1), 2.0 ** (b - 1) - 0.5, 0.5]) * u * rng.choice([-1.0, 1.0], 3)
+                if t % 4 == 3:
+                    r += rng.standard_normal(D) * 2.0 ** -12
+                out[b_, h, t] = r.astype(np.float16)
+    return out
+
+
+def polar_boundary_rows(seed: int, n_rows: int, bp: int, pool: int = 40000) -> np.ndarray:
+    """fp16 rows (head_dim 128) chosen from a seeded pool so that some folded-spectrum slot's angle
+    sits next to a phase-code boundary (k + 1/2) 2 pi / 2^bp.  The oracle's own fp32 FFT decides
+    where the angle is; half of the rows are the pool's closest cases (within the GPU's fp64
+    fallback band), the other half sit just outside that band (where fp32 atan2 decides)."""
+    from oracle import transforms as OT
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((pool, 128)) * 2.0).astype(np.float16)
+    a, b = OT.fold_spectrum(*OT.dft_dit_f32(x.astype(np.float32)))
+    th = np.arctan2(b.astype(np.float64), a.astype(np.float64))
+    v = (th + np.pi) * (2 ** bp) / (2.0 * np.pi) + 0.5
+    dist = np.abs(v - np.round(v))            # distance (in code steps) to a rounding boundary
+    dist[(a == 0) & (b == 0)] = 1.0
+    near = dist.min(axis=1)
+    edge = np.abs(dist - 1.05e-3).min(axis=1)  # just outside a 1e-3 guard band
+    k = n_rows // 2
+    pick = np.concatenate([np.argsort(near)[:k], np.argsort(edge)[:n_rows - k]])
+    return x[pick]

@@ -30,8 +30,9 @@ class Case:
     """A filled cache plus the fp16 inputs that went into it (kept on the host)."""
 
     def __init__(self, cfg: Config, T: int, seed: int = 0, chunks=None, layers=None, calib_T: int = 512,
-                 inputs=None):
-        """inputs: optional callable l -> (K, V) fp16 arrays [B, H, T, D] replacing the seeded law."""
+                 inputs=None, chan=None):
+        """inputs: optional callable l -> (K, V) fp16 arrays [B, H, T, D] replacing the seeded law;
+        chan: optional callable l -> fp16 array [H, D] replacing the calibrated channel scale."""
         self.cfg, self.T, self.seed = cfg, T, seed
         self.cache = KVCache(cfg)
         self.K, self.V, self.C = {}, {}, {}
@@ -43,8 +44,9 @@ class Case:
                 V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
             else:
                 K, V = (torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in inputs(l))
-            if cfg.k.chan_scale:
-                c = synth.channel_scale(seed, l, H, calib_T, D).cuda()
+            if cfg.side(l, 0).chan_scale:
+                c = (synth.channel_scale(seed, l, H, calib_T, D) if chan is None else
+                     torch.from_numpy(np.ascontiguousarray(chan(l), dtype=np.float16))).cuda()
                 self.cache.set_chan_scale(l, c)
                 self.C[l] = c.cpu().numpy()
             steps = chunks or [T]
@@ -122,12 +124,17 @@ class Case:
             Vs.append(Vh)
         return np.stack(Ks), np.stack(Vs)
 
-    def decode_and_compare(self, l, q16, seq_ids=None, kv_len=None, tol=TOL):
-        """Decode through the C ABI; compare every (query, head) output with the oracle."""
+    def decode_and_compare(self, l, q16, seq_ids=None, kv_len=None, tol=TOL, decode=None):
+        """Decode through the C ABI; compare every (query, head) output with the oracle.
+        decode: optional callable (layer, q, seq_ids, kv_len) -> (out, lse) replacing the cache's
+        kvq_decode_attention call (another entry point with the same contract)."""
         n_q = q16.shape[0]
         sid = None if seq_ids is None else torch.tensor(seq_ids, dtype=torch.int32, device="cuda")
         kl = None if kv_len is None else torch.tensor(kv_len, dtype=torch.int32, device="cuda")
-        out, lse = self.cache.decode(l, q16.cuda(), sid, kl, lse=True)
+        if decode is None:
+            out, lse = self.cache.decode(l, q16.cuda(), sid, kl, lse=True)
+        else:
+            out, lse = decode(l, q16.cuda(), sid, kl)
         out = out.cpu().numpy()
         lse = lse.cpu().numpy()
         qn = q16.cpu().numpy()

@@ -96,7 +96,7 @@ def test_create_rejects_before_touching_the_device():
 
 def test_null_handle_calls_fail_cleanly():
     L = kvq.lib()
-    assert L.kvq_quantize_append(None, 0, None, None, 1, None) == -1
+    assert L.kvq_quantize_append(None, 0, None, None, None, 1, 1, None) == -1
     assert L.kvq_decode_attention(None, 0, None, 1, None, None, None, 1, None, None) == -1
     assert L.kvq_dequantize(None, 0, 0, 0, 0, 1, None, 1, None) == -1
     assert L.kvq_set_seq_len(None, 0, 0, None) == -1
@@ -162,3 +162,24 @@ def test_binding_rejects_bad_tensors_before_the_library():
         cache.append(0, k16, k16)  # host tensor
     with pytest.raises(ValueError, match="q: need"):
         cache.decode(0, torch.zeros(2, 4, 128, dtype=torch.float16))
+
+
+def test_binding_checks_sequence_list_and_output():
+    """The per-sequence append's id list and a caller-supplied decode output are checked on the
+    host before the library sees them."""
+    import torch
+    cache = kvq.KVCache.__new__(kvq.KVCache)
+    cache.cfg = base_cfg()
+    cache.h = None
+    k16 = torch.zeros(1, 2, 3, 128, dtype=torch.float16)
+    with pytest.raises(ValueError, match="seq_ids"):
+        cache.append(0, k16, k16, seq_ids=torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError, match="seq_ids"):
+        cache.append(0, k16, k16, seq_ids=torch.zeros(1, dtype=torch.int32))  # host tensor
+
+
+def test_header_documents_the_sequence_list():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    decl = text[text.index("kvq_status kvq_quantize_append("):]
+    decl = decl[:decl.index(";")]
+    assert "const int32_t* seq_ids" in decl and "int32_t n_seqs" in decl and "int32_t n_new" in decl

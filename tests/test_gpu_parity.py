@@ -230,3 +230,63 @@ def test_per_layer_format_families():
         c.check_codes(l)
         c.check_dequant(l)
         c.decode_and_compare(l, queries(cfg, 2, 300, layer=l))
+
+
+# ---------------------------------------------- decision boundaries behind a pre-transform
+def _pow2_chan(seed, H, D):
+    r = np.random.default_rng(seed)
+    return (2.0 ** r.integers(-2, 3, size=(H, D))).astype(np.float16)
+
+
+ROTATED_TIES = [
+    (256, Side("int", 4, group=32, rot=256), Side("int", 2, group=128, rot=256)),
+    (256, Side("int", 3, group=64, rot=256), Side("int", 4, group=128, rot=128)),
+    (256, Side("int", 4, group=128, rot=256), Side("int", 3, group=128, rot=256)),
+    (128, Side("int", 4, group=32, rot=128), Side("int", 2, group=16, rot=128)),
+    (128, Side("int", 4, group=64, rot=128), Side("nf4", group=64, rot=128)),
+    (256, Side("int", 4, group=32, rot=256, chan_scale=True), Side("ternary", group=8, rot=256)),
+    (256, Side("int", 2, group=128, rot=128, chan_scale=True), Side("int", 4, scale="minmax", group=32, rot=256)),
+]
+
+
+@pytest.mark.parametrize("D,k,v", ROTATED_TIES, ids=[f"{d}-{k.fmt}{k.bits}g{k.group}r{k.rot}c{int(k.chan_scale)}-"
+                                                       f"{v.fmt}{v.bits}g{v.group}r{v.rot}" for d, k, v in ROTATED_TIES])
+@pytest.mark.parametrize("chunks", [None, [1] * 5 + [59]], ids=["bulk", "tokens"])
+def test_rotated_decision_boundaries(D, k, v, chunks):
+    """Rows whose Hadamard image (after an exact power-of-two channel scale for K) puts absmax ties
+    of both signs and x/d on half-integers: the rotated path's exact near-tie fallback must give
+    the oracle's codes and scales ("E21W" variants B and D, "E22L" "What I tested")."""
+    import adversarial
+    T = 64
+    cfg = cfg_of(D, k, v, T=T)
+    chan = _pow2_chan(5, 2, D)
+
+    def inputs(l):
+        K = adversarial.spike_rows(21 + l, 2, 2, T, D, k.rot)
+        if k.chan_scale:  # x = spike * c, so x / c is the spike exactly
+            K = (K.astype(np.float32) * chan[None, :, None, :].astype(np.float32)).astype(np.float16)
+        return K, adversarial.spike_rows(77 + l, 2, 2, T, D, v.rot)
+
+    c = Case(cfg, T, chunks=chunks, inputs=inputs, chan=lambda l: chan)
+    c.check_codes(0)
+    c.check_dequant(0)
+    c.decode_and_compare(0, queries(cfg, 2, T))
+
+
+@pytest.mark.parametrize("bm,bp", [(4, 8), (5, 7), (6, 6), (7, 5), (8, 4)])
+def test_polar_phase_boundaries(bm, bp):
+    """Spectrum slots whose angle sits next to a phase-code boundary (k + 1/2) 2 pi / 2^bp: inside
+    the GPU's fp64 fallback band and just outside it.  Phase codes must equal the oracle's
+    (the reply, "The finite-phase implementation and the physical codec may be worth
+    separating": one phase-angle index per coefficient)."""
+    import adversarial
+    T = 64
+    rows = adversarial.polar_boundary_rows(40 + bp, 2 * 2 * T, bp)
+    K = rows.reshape(2, 2, T, 128)
+    V = rows[::-1].copy().reshape(2, 2, T, 128)
+    s = Side("polar", bm, bp)
+    cfg = cfg_of(128, s, s, T=T)
+    c = Case(cfg, T, inputs=lambda l: (K, V))
+    c.check_codes(0)
+    c.check_dequant(0)
+    c.decode_and_compare(0, queries(cfg, 2, T))

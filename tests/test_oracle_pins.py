@@ -502,3 +502,108 @@ def test_channel_scale_then_rotation_order():
     assert A.rel_sq_error(x, xo) < 1e-4
     y = T.fwht_f32(x.astype(np.float32) / c.astype(np.float32), 256)
     assert np.array_equal(Q.transform_rows(x, side, np.broadcast_to(c, x.shape)), y)
+
+
+# ----------------------------------------------------------------------------- anchors in reconstruction
+def _rot_int8_bound(x16, side, out):
+    """Per-row bound on the original-domain error of a rotated absmax int grid: the rotation is
+    orthonormal, so the row error norm equals the stored-domain one, at most |d|/2 per element
+    inside the grid hull and |d| where the positive side clamps."""
+    d = np.repeat(np.abs(out["scales"].astype(np.float64)), side.group, axis=1)
+    return np.sqrt((d ** 2).sum(axis=1))
+
+
+@pytest.mark.parametrize("rule,n", [("first_n", 48), ("window", 40), ("all", 0)])
+def test_reconstruct_unit_anchor_substitution(rule, n):
+    """Post 6 "Corrected semantics": an anchored row is attended as its original fp16 row --
+    K's own row for keys, V's for values, unrotated -- and every other row is the dequantized
+    row in the original domain.  Keys and values are drawn independently, so substituting the
+    wrong side, the rotated row, or the wrong token set cannot pass."""
+    r = rng(31)
+    T, D = 120, 128
+    side = Side("int", 8, group=32, rot=128)
+    spec = C.Spec(1, 1, 1, 1, D, side, side, frozenset({0}), rule, n)
+    K16 = (r.standard_normal((T, D)) * 2).astype(np.float16)
+    V16 = (r.standard_normal((T, D)) * 3 + 1).astype(np.float16)
+    seq_len = 100  # a window protects the last n stored tokens, not the last rows of the buffer
+    kq, vq = C.quantize_unit(spec, K16, V16)
+    Kh, Vh = C.reconstruct_unit(spec, 0, K16, V16, kq, vq, seq_len)
+    t = np.arange(T)
+    want = {"first_n": t < n, "window": (t >= seq_len - n) & (t < seq_len), "all": t < seq_len}[rule]
+    assert want.sum() > 0
+    for Xh, X16, q in ((Kh, K16, kq), (Vh, V16, vq)):
+        x = X16.astype(np.float64)
+        assert np.array_equal(Xh[want], x[want])              # exact original rows
+        err = np.sqrt(((Xh - x) ** 2).sum(axis=1))
+        bound = _rot_int8_bound(X16, side, q)
+        assert (err[~want] <= bound[~want] * (1 + 1e-6) + 1e-9).all()  # dequantized, unrotated
+        assert (err[~want] > 0).all()                        # and really the quantized row
+    # a layer outside the anchor set is quantized everywhere
+    spec2 = C.Spec(2, 1, 1, 1, D, side, side, frozenset({0}), rule, n)
+    Kh1, Vh1 = C.reconstruct_unit(spec2, 1, K16, V16, kq, vq, seq_len)
+    assert (np.sqrt(((Kh1 - K16.astype(np.float64)) ** 2).sum(axis=1)) > 0).all()
+
+
+# ----------------------------------------------------------------------------- composite rFFT reconstruction
+def _folded_reference(x16):
+    """Folded slots (X_0, X_64 | X_f) of each row from numpy's FFT in fp64 (independent of the
+    oracle's fp32 DIT and fold)."""
+    X = np.fft.rfft(x16.astype(np.float64), axis=-1)  # 65 bins
+    a = X[:, :64].real.copy()
+    b = X[:, :64].imag.copy()
+    b[:, 0] = X[:, 64].real
+    return a, b
+
+
+def _parseval_folded(ea, eb):
+    """Energy of the real row whose folded-slot error is (ea, eb), N = 128."""
+    w = np.full(ea.shape, 2.0)
+    w[:, 0] = 1.0
+    return (w * (ea ** 2 + eb ** 2)).sum(axis=1) / 128.0
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_cartesian_reconstruction_matches_parseval(bits):
+    """The reply's Cartesian control: the stored reals are the folded spectrum's (re, im) pairs on
+    a signed grid, and the inverse transform's row error is the Parseval-weighted stored error.
+    Against numpy's FFT: a swapped (re, im) interleave, a misplaced Nyquist bin or a missing
+    factor 2 on the one-sided bins fails the equality."""
+    x16 = (rng(32).standard_normal((16, 128)) * 3).astype(np.float16)
+    side = Side("cart", bits)
+    out = Q.quantize_rows(x16, side)
+    a_ref, b_ref = _folded_reference(x16)
+    y = out["exact"]
+    ea, eb = y[:, 0::2] - a_ref, y[:, 1::2] - b_ref
+    d = np.abs(out["scales"].astype(np.float64))  # [R, 1]
+    assert (np.abs(ea) <= d * (1 + 1e-3)).all() and (np.abs(eb) <= d * (1 + 1e-3)).all()
+    xr = Q.to_original_f64(y, side)
+    got = ((xr - x16.astype(np.float64)) ** 2).sum(axis=1)
+    assert np.allclose(got, _parseval_folded(ea, eb), rtol=1e-6, atol=1e-10)
+    assert (got <= (254 / 128) * d[:, 0] ** 2 * (1 + 1e-3)).all()
+
+
+@pytest.mark.parametrize("bm,bp", [(4, 8), (5, 7), (6, 6), (7, 5), (8, 4)])
+def test_polar_reconstruction_within_magnitude_and_phase_bound(bm, bp):
+    """The reply's polar codec: per slot the reconstruction error is at most the magnitude step
+    error plus the chord of the phase step, |dm| + m^ * pi / 2^bp; through Parseval the row error
+    is bounded by those per-slot bounds.  The reference spectrum is numpy's, so the composite
+    (DIT FFT, fold, codes, cos/sin, unfold, inverse DFT) is checked end to end."""
+    x16 = (rng(33).standard_normal((16, 128)) * 2).astype(np.float16)
+    side = Side("polar", bm, bp)
+    out = Q.quantize_rows(x16, side)
+    a_ref, b_ref = _folded_reference(x16)
+    mag = np.hypot(a_ref, b_ref)
+    s = out["scales"].astype(np.float64)  # [R, 1]
+    mh = out["q"][:, :64] * s
+    dm = np.abs(mh - mag)
+    assert (dm <= s / 2 + 1e-3 * mag.max(axis=1, keepdims=True)).all()
+    slot_bound = dm + mh * (math.pi / 2 ** bp) + 1e-6 * mag.max(axis=1, keepdims=True)
+    y = out["exact"]
+    ea, eb = y[:, 0::2] - a_ref, y[:, 1::2] - b_ref
+    assert (np.hypot(ea, eb) <= slot_bound).all()
+    xr = Q.to_original_f64(y, side)
+    got = ((xr - x16.astype(np.float64)) ** 2).sum(axis=1)
+    assert np.allclose(got, _parseval_folded(ea, eb), rtol=1e-6, atol=1e-10)
+    w = np.full(slot_bound.shape, 2.0)
+    w[:, 0] = 1.0
+    assert (got <= (w * slot_bound ** 2).sum(axis=1) / 128.0).all()

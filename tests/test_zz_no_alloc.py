@@ -1,8 +1,9 @@
 """kvq_decode_attention_noalloc: decode attention with no device allocation behind it.
 
-Some callers cannot call cudaMalloc where they decode (a stream being captured into a CUDA graph
-in global mode, or a runtime that budgets all of HBM itself).  For them the split-K scratch of
-the decode lives in a fixed device array inside the library.  This file runs last so that a
+Some callers cannot call cudaMalloc where they decode: a serving runtime that hands nearly all of
+HBM to its own pool and budgets every other byte, or a latency-critical loop that must not take
+the device synchronisation an allocation can cause.  For them the split-K scratch of the decode
+lives in a fixed device array inside the library.  This file runs last so that a
 failure here leaves every other test already run; it passes alone in a fresh process and after
 the rest of the suite.
 """
@@ -33,13 +34,20 @@ def test_noalloc_decode_matches_regular_decode_twice(D, k, v):
     seq = torch.tensor([0, 1, 1], dtype=torch.int32, device="cuda")
     kl = torch.tensor([900, 517, 3], dtype=torch.int32, device="cuda")
     ref_out, ref_lse = c.cache.decode(0, q, seq, kl, lse=True)
-    for _ in range(2):  # two calls in a row share (and overwrite) the fixed scratch
+
+    def noalloc(layer, qq, sid, kvl):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
-        kvq.kvq_decode_attention_noalloc(c.cache.h, 0, q, 3, seq, kl, out, lse)
+        kvq.kvq_decode_attention_noalloc(c.cache.h, layer, qq, qq.shape[0], sid, kvl, out, lse)
         torch.cuda.synchronize()
+        return out, lse
+
+    for _ in range(2):  # two calls in a row share (and overwrite) the fixed scratch
+        out, lse = noalloc(0, q, seq, kl)
         assert _rel(out, ref_out) <= TOL
         assert torch.allclose(lse, ref_lse, rtol=1e-5, atol=1e-5)
+    # and against the CPU oracle's attention over the same packed cache
+    c.decode_and_compare(0, q.cpu(), seq_ids=[0, 1, 1], kv_len=[900, 517, 3], decode=noalloc)
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
@@ -53,4 +61,8 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     out = torch.empty(n_q, 32, 128, device="cuda")
     with pytest.raises(KVQError) as e:
         kvq.kvq_decode_attention_noalloc(c.cache.h, 0, q, n_q, seq, None, out)
+    assert e.value.status == -3
+    # more queries than the handle's max_queries: the same status as kvq_decode_attention
+    with pytest.raises(KVQError) as e:
+        kvq.kvq_decode_attention_noalloc(c.cache.h, 0, q, n_q + 1, seq, None, out)
     assert e.value.status == -3
