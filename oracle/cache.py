@@ -16,6 +16,16 @@ of 128, under a 3.2-bit average; "Result": 2-bit K in layers 2 and 7, 4-bit V in
 and 4, 3 bits elsewhere, 3.19 bits on average).  A Spec may give one Side per layer for K and for
 V; layers are numbered from 0 (the same result calls layer 7 the last of the 8).
 
+Key mean subtraction (llama.cpp #21385, the later comment on a per-head shared key mean that
+carries about half of the key energy: the running mean is subtracted before quantization and
+restored after).  Reading taken here: the mean of one (layer, sequence, kv-head) is the running
+mean of its keys at the end of the sequence's first append (normally the prefill), frozen for
+the tokens that follow, so that every stored key row of the sequence shares it.  It is exact
+before one rounding: mu = fp16(fp64(S) / n * 2^-24) with S the exact integer sum of the n fp16
+keys times 2^24.  Rows are quantized as fp32(k - mu); dequantized rows get mu added back (the
+attention logits of the sequence's quantized rows all shift by q . mu).  Anchored rows keep the
+raw key.
+
 Effective bits ("E21W" "Result" counts group scales in the totals, 3.5 b for 3-bit g32 and
 4.5 b for 4-bit g32; "E22L" "What I tested" averages over K and V with scales included; post 6
 "Corrected semantics" reports anchored configurations in effective bits): (code bits + 16 per
@@ -30,6 +40,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 from . import attention as A
+from .quant import F64
 from .quant import Side, bits_per_value, quantize_rows, to_original_f64
 
 
@@ -68,9 +79,21 @@ def anchored(spec: Spec, layer: int, tokens: np.ndarray, seq_len: int) -> np.nda
     raise ValueError(spec.anchor_rule)
 
 
-def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None, layer: int = 0):
-    """Quantize one (layer, sequence, kv-head) unit: K16, V16 [T, D]; c16 [D] or None."""
-    kq = quantize_rows(K16, side_of(spec, layer, True), None if c16 is None else np.broadcast_to(c16, K16.shape))
+def key_mean(K16: np.ndarray) -> np.ndarray:
+    """fp16 mean over the rows of K16 [n, D]: the exact sum rounded once (see the module text)."""
+    k = np.asarray(K16, dtype=np.float16).astype(F64)
+    S = np.round(k * 2.0 ** 24).astype(np.int64).sum(axis=0)  # fp16 values are multiples of 2^-24
+    return ((S.astype(F64) / F64(k.shape[0])) * 2.0 ** -24).astype(np.float16)
+
+
+def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None, layer: int = 0, first_rows=None):
+    """Quantize one (layer, sequence, kv-head) unit: K16, V16 [T, D]; c16 [D] or None;
+    first_rows: rows of the sequence's first append (the key mean's rows; default all)."""
+    ks = side_of(spec, layer, True)
+    mu = key_mean(K16[:first_rows or K16.shape[0]]) if ks.mean_sub else None
+    kq = quantize_rows(K16, ks, None if c16 is None else np.broadcast_to(c16, K16.shape),
+                       None if mu is None else np.broadcast_to(mu, K16.shape))
+    kq["mu"] = mu
     vq = quantize_rows(V16, side_of(spec, layer, False), None)
     return kq, vq
 
@@ -79,7 +102,9 @@ def reconstruct_unit(spec: Spec, layer: int, K16, V16, kq, vq, seq_len: int, c16
     """Keys and values attention sees for one unit (fp64 [T, D]); anchors override."""
     T = K16.shape[0]
     cK = None if c16 is None else np.broadcast_to(c16, K16.shape)
-    Kh = to_original_f64(kq["exact"], side_of(spec, layer, True), cK)
+    mu = kq.get("mu")
+    Kh = to_original_f64(kq["exact"], side_of(spec, layer, True), cK,
+                         None if mu is None else np.broadcast_to(mu, K16.shape))
     Vh = to_original_f64(vq["exact"], side_of(spec, layer, False), None)
     an = anchored(spec, layer, np.arange(T), seq_len)
     Kh[an] = np.asarray(K16, dtype=np.float16)[an].astype(np.float64)
@@ -102,6 +127,8 @@ def effective_bits(spec: Spec, seq_len: int) -> float:
             per_row = bits_per_value(side, D) * D
             bits = (seq_len - an) * per_row + an * 16 * D
             if is_k and side.chan_scale:
+                bits += 16 * D
+            if is_k and side.mean_sub:
                 bits += 16 * D
             tot += bits
     return tot / (spec.n_layers * 2 * seq_len * D)

@@ -21,6 +21,14 @@ Grids and scales (sources by page title and section):
   * sign {-s, +s}: post 6 "Minimal recipe" (one-bit sign KV with a scale);
     s = fp16(fp32 sum of |x| in channel order / g) (least-squares scale for fixed signs),
     t = +1 if x >= 0 else -1.
+  * symmetric int b: "E22L" "Result" (the ggml grid "leaves one side with fewer levels"; a
+    symmetric grid is the next candidate).  Levels (q - (2^b - 1)/2) d for q = 0 .. 2^b - 1, so
+    the outermost level is the group's largest magnitude m: d = fp16(fp32(m / (2^(b-1) - 1/2))),
+    q = clamp(floor(x/d) + 2^(b-1), 0, 2^b - 1) (nearest level, ties up); d = 0 gives q = 2^(b-1).
+  * Gaussian Lloyd-Max b: "E22L" "Result" (the other next candidate, "Gaussian Lloyd-Max levels
+    on rotated values"); levels from oracle.lloyd in units of the group's RMS,
+    s = fp16(sqrt(fp32(fp32 sum of x^2 in channel order / g))), code = nearest level of x/s
+    (ties up); s = 0 gives the level just above zero, 2^(b-1).
   * rFFT polar: the reply, "Fixed-rate magnitude/phase allocation" (mag/phase splits
     4+8 .. 8+4 at 12 bits per coefficient) and "The finite-phase implementation and the
     physical codec may be worth separating" (a magnitude index and one phase-angle index per
@@ -44,6 +52,7 @@ from dataclasses import dataclass
 import numpy as np
 
 from . import transforms as T
+from .lloyd import lloyd_max_levels
 from .nf4 import nf4_levels
 
 F32 = np.float32
@@ -52,13 +61,14 @@ F64 = np.float64
 
 @dataclass(frozen=True)
 class Side:
-    fmt: str = "int"          # int | nf4 | ternary | sign | polar | cart | fp16
+    fmt: str = "int"          # int | nf4 | ternary | sign | polar | cart | lloyd | fp16
     bits: int = 4             # code bits (magnitude bits for polar)
     bits2: int = 0            # phase bits (polar only)
-    scale: str = "absmax"     # absmax | minmax   (int only)
+    scale: str = "absmax"     # absmax | minmax | sym   (int only)
     group: int = 32           # channels per scale (polar/cart: the whole row)
     rot: int = 0              # 0 | 128 | 256 (Walsh-Hadamard block size)
     chan_scale: bool = False  # divide by a per-channel scale first (K only)
+    mean_sub: bool = False    # subtract the sequence's key mean first (K only; oracle.cache)
 
     def n_groups(self, D: int) -> int:
         if self.fmt in ("polar", "cart"):
@@ -78,7 +88,7 @@ class Side:
             return (D // 2) * (self.bits + self.bits2) // 8
         if self.fmt == "nf4":
             return D // 2
-        return -(-D * self.bits // 8)
+        return -(-D * self.bits // 8)  # int (absmax, minmax, sym), lloyd, cart
 
     def has_zero(self) -> bool:
         return self.fmt == "int" and self.scale == "minmax"
@@ -201,6 +211,47 @@ def quant_ternary(x32: np.ndarray, g: int):
     return t.reshape(R, D).astype(np.int64), s
 
 
+def floor_exact(x: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """k = floor(x / d) in exact arithmetic for d > 0 (x fp32, d fp16, |k| < 2^12): an fp64
+    estimate corrected by comparing x with the exact products k d and (k + 1) d."""
+    x = np.asarray(x, dtype=F64)
+    d = np.broadcast_to(np.asarray(d, dtype=F64), x.shape)
+    pos = d > 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        k = np.floor(np.where(pos, x / np.where(pos, d, 1.0), 0.0))
+    k = np.where(pos & (x < k * d), k - 1, k)
+    k = np.where(pos & (x >= (k + 1) * d), k + 1, k)
+    return np.where(pos, k, 0.0)
+
+
+def quant_int_sym(x32: np.ndarray, b: int, g: int):
+    """Symmetric grid (q - (2^b - 1)/2) d, q = 0 .. 2^b - 1; returns (q, d)."""
+    R, D = x32.shape
+    xg = x32.reshape(R, D // g, g).astype(F32)
+    m = np.abs(xg).max(axis=-1).astype(F32)
+    d = f16((m / F32(2 ** (b - 1) - 0.5)).astype(F32))
+    q = floor_exact(xg.astype(F64), d[..., None]) + 2 ** (b - 1)
+    q = np.clip(q, 0, 2 ** b - 1)
+    q = np.where(d[..., None] == 0, 2 ** (b - 1), q)
+    return q.reshape(R, D).astype(np.int64), d
+
+
+def quant_lloyd(x32: np.ndarray, b: int, g: int):
+    """Gaussian Lloyd-Max levels times the group RMS; returns (code, s)."""
+    R, D = x32.shape
+    L = lloyd_max_levels(b)
+    mids = (L[:-1] + L[1:]) / 2.0
+    xg = x32.reshape(R, D // g, g).astype(F32)
+    acc = np.zeros(xg.shape[:-1], dtype=F32)
+    for j in range(g):  # fp32 sum of the rounded squares, in channel order
+        acc = (acc + (xg[..., j] * xg[..., j]).astype(F32)).astype(F32)
+    s = f16(np.sqrt((acc / F32(g)).astype(F32)).astype(F32))
+    thr = mids[None, None, None, :] * s[..., None, None]
+    code = (xg.astype(F64)[..., None] >= thr).sum(axis=-1)
+    code = np.where(s[..., None] == 0, 2 ** (b - 1), code)
+    return code.reshape(R, D).astype(np.int64), s
+
+
 def quant_sign(x32: np.ndarray, g: int):
     R, D = x32.shape
     xg = x32.reshape(R, D // g, g).astype(F32)
@@ -242,9 +293,12 @@ def interleave_slots(a: np.ndarray, b: np.ndarray) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- rows
-def transform_rows(x16: np.ndarray, side: Side, c16=None) -> np.ndarray:
-    """fp16 rows -> fp32 rows in the domain the grid sees (channel scale, then rotation)."""
+def transform_rows(x16: np.ndarray, side: Side, c16=None, mu16=None) -> np.ndarray:
+    """fp16 rows -> fp32 rows in the domain the grid sees (key mean subtracted, then channel
+    scale, then rotation)."""
     x = np.asarray(x16, dtype=np.float16).astype(F32)
+    if side.mean_sub:
+        x = (x - np.asarray(mu16, dtype=np.float16).astype(F32)).astype(F32)
     if side.chan_scale:
         x = T.channel_divide(x, np.asarray(c16, dtype=np.float16))
     if side.rot:
@@ -252,8 +306,9 @@ def transform_rows(x16: np.ndarray, side: Side, c16=None) -> np.ndarray:
     return x
 
 
-def quantize_rows(x16: np.ndarray, side: Side, c16=None) -> dict:
-    """Quantize fp16 rows [R, D] of one side.  Returns a dict with
+def quantize_rows(x16: np.ndarray, side: Side, c16=None, mu16=None) -> dict:
+    """Quantize fp16 rows [R, D] of one side (mu16: the key mean, with side.mean_sub).  Returns
+    a dict with
     bytes  uint8 [R, row_bytes]  logical packed codes
     scales float16 [R, G]         (min-max also: zeros float16 [R, G])
     stored float32 [R, D]         stored-domain dequantization (bit-exact definition)
@@ -268,9 +323,27 @@ def quantize_rows(x16: np.ndarray, side: Side, c16=None) -> dict:
         out["stored"] = x16.astype(F32)
         out["exact"] = x16.astype(F64)
         return out
-    x = transform_rows(x16, side, c16)
+    x = transform_rows(x16, side, c16, mu16)
     g = side.group
-    if side.fmt == "int" and side.scale == "absmax":
+    if side.fmt == "int" and side.scale == "sym":
+        q, d = quant_int_sym(x, side.bits, g)
+        out["bytes"] = pack_bits(q, side.bits)
+        dd = np.repeat(d, g, axis=1)
+        lv = q - (2 ** side.bits - 1) / 2.0
+        out["stored"] = (lv * dd).astype(F32)
+        out["exact"] = lv * dd
+        out["scales"] = d.astype(np.float16)
+        out["q"] = q
+    elif side.fmt == "lloyd":
+        code, s = quant_lloyd(x, side.bits, g)
+        L = lloyd_max_levels(side.bits)
+        out["bytes"] = pack_bits(code, side.bits)
+        val = L[code] * np.repeat(s, g, axis=1)
+        out["stored"] = val.astype(F32)
+        out["exact"] = val
+        out["scales"] = s.astype(np.float16)
+        out["q"] = code
+    elif side.fmt == "int" and side.scale == "absmax":
         q, d = quant_int_absmax(x, side.bits, g)
         out["bytes"] = pack_bits(q + 2 ** (side.bits - 1), side.bits)
         dd = np.repeat(d, g, axis=1)
@@ -343,8 +416,9 @@ def quantize_rows(x16: np.ndarray, side: Side, c16=None) -> dict:
     return out
 
 
-def to_original_f64(stored64: np.ndarray, side: Side, c16=None) -> np.ndarray:
-    """Undo the pre-transform of stored-domain rows, fp64: (i)DFT, then rotation, then x c."""
+def to_original_f64(stored64: np.ndarray, side: Side, c16=None, mu16=None) -> np.ndarray:
+    """Undo the pre-transform of stored-domain rows, fp64: (i)DFT, then rotation, then x c,
+    then + the key mean."""
     y = np.asarray(stored64, dtype=F64)
     if side.fmt in ("polar", "cart"):
         y = T.unfold_idft_f64(y[..., 0::2], y[..., 1::2])
@@ -352,6 +426,8 @@ def to_original_f64(stored64: np.ndarray, side: Side, c16=None) -> np.ndarray:
         y = T.hadamard_inverse_f64(y, side.rot)
     if side.chan_scale:
         y = y * np.asarray(c16, dtype=np.float16).astype(F64)
+    if side.mean_sub:
+        y = y + np.asarray(mu16, dtype=np.float16).astype(F64)
     return y
 
 

@@ -159,11 +159,12 @@ struct RowDst {
   unsigned err;
   bool first;
 };
-__device__ __forceinline__ RowDst row_dst(const LayerDev& L, long long row, int n_new) {
+// (rows per call < 2^31, checked on the host, so 32-bit index arithmetic suffices)
+__device__ __forceinline__ RowDst row_dst(const LayerDev& L, int row, int n_new) {
   RowDst d{0, 0, 0, 0u, false};
-  const long long ul = row / n_new;
-  const int i = (int)(row - ul * n_new);
-  const int sl = (int)(ul / L.Hkv), h = (int)(ul - (long long)sl * L.Hkv);
+  const int ul = row / n_new;
+  const int i = row - ul * n_new;
+  const int sl = ul / L.Hkv, h = ul - sl * L.Hkv;
   const int b = L.app_ids ? L.app_ids[sl] : sl;
   d.first = i == 0 && h == 0;
   if (b < 0 || b >= L.B) {
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long R = (long long)L.app_n * L.Hkv * n_new;
   for (long long row = (long long)blockIdx.x * kFftWarps + warp; row < R; row += (long long)gridDim.x * kFftWarps) {
-  const RowDst dst = row_dst(L, row, n_new);
+  const RowDst dst = row_dst(L, (int)row, n_new);
   const bool ok = dst.err == 0;
   const int pos = dst.pos, len_after = dst.len_after, u = dst.u;
   if (!ok && dst.first && lane == 0) atomicOr(L.err, dst.err);
@@ -824,7 +825,7 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
        gt += (long long)gridDim.x * blockDim.x) {
   const long long row = gt / vec_per_row;
   const int c = (int)(gt % vec_per_row);
-  const RowDst d = row_dst(L, row, n_new);
+  const RowDst d = row_dst(L, (int)row, n_new);
   if (d.err == 0) {
     const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + row * L.D) + c);
     reinterpret_cast<uint4*>(S.codes + ((long long)d.u * L.Tcap + d.pos) * S.row_bytes)[c] = w;

@@ -607,3 +607,130 @@ def test_polar_reconstruction_within_magnitude_and_phase_bound(bm, bp):
     w = np.full(slot_bound.shape, 2.0)
     w[:, 0] = 1.0
     assert (got <= (w * slot_bound ** 2).sum(axis=1) / 128.0).all()
+
+
+# ----------------------------------------------------------------------------- value grids after E22L
+from oracle import lloyd as LM
+
+# J. Max, "Quantizing for minimum distortion" (1960), Table I, the Gaussian optimum (positive
+# half, 4 decimals) and its mean squared error (to the precision compared) -- a published table,
+# independent of the iteration.
+MAX_1960 = {2: ([0.4528, 1.5104], 0.1175), 3: ([0.2451, 0.7560, 1.3439, 2.1520], 0.03455),
+            4: ([0.1284, 0.3881, 0.6568, 0.9424, 1.2562, 1.6180, 2.0690, 2.7326], 0.00950)}
+
+
+def _gauss_mse(levels):
+    """Expected (X - nearest level)^2 for X ~ N(0, 1), by midpoint-rule integration."""
+    x = np.linspace(-12, 12, 2_400_001)
+    w = np.exp(-0.5 * x * x) / math.sqrt(2 * math.pi) * (x[1] - x[0])
+    idx = np.searchsorted((levels[:-1] + levels[1:]) / 2.0, x)
+    return float((w * (x - levels[idx]) ** 2).sum())
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_lloyd_max_levels(b):
+    """Gaussian Lloyd-Max levels ("E22L" "Result": the next value grid to test): Max's table, the
+    two optimality conditions (midpoint thresholds, centroid levels) at the fixed point, odd
+    symmetry, and the table's distortion."""
+    lv = LM.lloyd_max_levels_f64(b)
+    half, mse = MAX_1960[b]
+    assert np.allclose(lv[2 ** (b - 1):], half, atol=6e-5)
+    assert np.allclose(lv, -lv[::-1], atol=1e-12)
+    assert np.abs(LM.centroids((lv[:-1] + lv[1:]) / 2) - lv).max() < 1e-10
+    assert abs(_gauss_mse(lv) - mse) < 1e-3 * mse
+    # fp16 storage: every level is an fp16 value within half an fp16 ulp of the optimum
+    l16 = LM.lloyd_max_levels(b)
+    assert np.array_equal(l16, l16.astype(np.float16).astype(np.float64))
+    assert np.all(np.abs(l16 - lv) <= np.abs(lv) * 2 ** -11)
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_lloyd_nearest_level(b):
+    x = (rng(40 + b).standard_normal((4, 64)) * 1.7).astype(np.float16)
+    x[0, :8] = 0.0
+    r = Q.quantize_rows(x, Side("lloyd", b, group=16))
+    L = [Fraction(float(v)) for v in LM.lloyd_max_levels(b)]
+    for i in range(4):
+        for gi in range(4):
+            grp = x[i, gi * 16:(gi + 1) * 16].astype(np.float64)
+            # the scale is the group RMS (fp32 sum of rounded squares in channel order)
+            acc = np.float32(0)
+            for v in grp.astype(np.float32):
+                acc = np.float32(acc + np.float32(v * v))
+            s = np.float16(np.sqrt(np.float32(acc / np.float32(16))))
+            assert r["scales"][i, gi] == s
+            S = Fraction(float(s))
+            for jj in range(16):
+                want = _nearest_exact(float(grp[jj]), [lv * S for lv in L]) if S != 0 else 2 ** (b - 1)
+                assert r["q"][i, gi * 16 + jj] == want
+    assert set(np.unique(r["q"])) <= set(range(2 ** b))
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_symmetric_grid_nearest_level(b):
+    """The symmetric b-bit grid (levels +-(k + 1/2) d, "E22L" "Result"): nearest level in exact
+    arithmetic with ties up, the outermost level at the group's largest magnitude, and the level
+    set symmetric about zero (no zero level)."""
+    x = (rng(50 + b).standard_normal((4, 64)) * 2.3).astype(np.float16)
+    x[1, :16] = 0.0
+    # exact ties: multiples of d where d comes out exact (m = 2^(b-1) - 1/2 times a power of two)
+    x[2, 32:48] = np.array([(2 ** (b - 1) - 0.5) * 0.25] + [0.25 * k for k in range(-7, 8)], dtype=np.float16)
+    r = Q.quantize_rows(x, Side("int", b, scale="sym", group=16))
+    nlev = 2 ** b
+    for i in range(4):
+        for gi in range(4):
+            grp = x[i, gi * 16:(gi + 1) * 16].astype(np.float64)
+            d = Fraction(float(r["scales"][i, gi]))
+            m = np.abs(grp).max()
+            assert float(r["scales"][i, gi]) == float(np.float16(np.float32(m) / np.float32(2 ** (b - 1) - 0.5)))
+            levels = [(Fraction(2 * q - (nlev - 1), 2)) * d for q in range(nlev)]
+            for jj in range(16):
+                want = _nearest_exact(float(grp[jj]), levels) if d != 0 else 2 ** (b - 1)
+                assert r["q"][i, gi * 16 + jj] == want
+    lv = sorted({float(v) for v in (r["q"] - (nlev - 1) / 2.0).ravel()})
+    assert all(abs(v) >= 0.5 for v in lv) and max(lv) <= (nlev - 1) / 2.0
+    assert set(np.unique(Q.quantize_rows(x, Side("int", 2, scale="sym", group=64))["q"] - 1.5)) == {-1.5, -0.5, 0.5, 1.5}
+
+
+def test_key_mean_is_the_exact_mean_rounded():
+    """The key mean (llama.cpp #21385, the comment on subtracting a shared per-head key mean): the
+    exact rational mean of the fp16 keys, through fp64, rounded to fp16."""
+    K = (rng(60).standard_normal((777, 64)) * 3 + 5).astype(np.float16)
+    K[0] *= 50
+    mu = C.key_mean(K)
+    for j in range(64):
+        S = sum(Fraction(float(v)) for v in K[:, j])
+        assert mu[j] == np.float16(float(S / 777))
+
+
+def test_key_mean_subtraction_restores_and_helps():
+    """Keys with a large shared per-head mean (the comment: about half of the key energy): the
+    quantized rows are the residual k - mu, the restored row is residual + mu (within the grid's
+    error bound), and at 3 bits the K error is far below the same grid without the subtraction."""
+    r = rng(61)
+    n_tok, D = 300, 128
+    mean = r.standard_normal(D) * 4.0
+    K = (mean[None, :] + r.standard_normal((n_tok, D))).astype(np.float16)
+    V = r.standard_normal((n_tok, D)).astype(np.float16)
+    k_sub = Side("int", 3, group=32, rot=128, mean_sub=True)
+    k_raw = Side("int", 3, group=32, rot=128)
+    v = Side("int", 4, group=32)
+    errs = {}
+    for name, ks in (("sub", k_sub), ("raw", k_raw)):
+        spec = C.Spec(1, 1, 1, 1, D, ks, v)
+        kq, vq = C.quantize_unit(spec, K, V, first_rows=200)
+        Kh, _ = C.reconstruct_unit(spec, 0, K, V, kq, vq, n_tok)
+        if name == "sub":
+            mu = C.key_mean(K[:200])  # the first append's 200 rows
+            assert np.array_equal(kq["mu"], mu)
+            # the grid sees the fp32 residual k - mu, rotated after the subtraction
+            resid = (K.astype(np.float32) - mu.astype(np.float32)).astype(np.float32)
+            q, d = Q.quant_int_absmax(T.fwht_f32(resid, 128), 3, 32)
+            assert np.array_equal(kq["q"], q) and np.array_equal(kq["scales"].astype(np.float64), d)
+            # restored: the residual's reconstruction plus mu
+            assert np.allclose(Kh - mu.astype(np.float64), Q.to_original_f64(kq["exact"], k_raw), rtol=0, atol=1e-12)
+        errs[name] = A.rel_sq_error(K, Kh)
+    assert errs["sub"] < 0.25 * errs["raw"]
+    # bits: one fp16 mean vector per (sequence, kv-head), like a channel-scale vector
+    s = C.Spec(1, 1, 1, 1, D, k_sub, v)
+    assert C.effective_bits(s, 1000) == pytest.approx((Q.bits_per_value(k_sub, D) + 16 / 1000 + Q.bits_per_value(v, D)) / 2)
