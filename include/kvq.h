@@ -56,9 +56,14 @@ enum {
   KVQ_FMT_TERNARY = 3,  /* {-s, 0, +s}, s = group absmax, 5 trits per byte [FMKQ] "Milestone" */
   KVQ_FMT_SIGN = 4,     /* {-s, +s}, s = group mean |x| [FMKQ] "Minimal recipe" */
   KVQ_FMT_POLAR = 5,    /* rFFT magnitude (bits) / phase (bits2) indices [FMKQ] reply */
-  KVQ_FMT_CART = 6      /* rFFT real/imag, signed absmax int-bits, one scale [FMKQ] reply control */
+  KVQ_FMT_CART = 6,     /* rFFT real/imag, signed absmax int-bits, one scale [FMKQ] reply control */
+  KVQ_FMT_LLOYD = 7     /* Gaussian Lloyd-Max levels (bits 2..4) times the group RMS, [E22L] "Result":
+                           the value grid named for the next run */
 };
-enum { KVQ_SCALE_ABSMAX = 0, KVQ_SCALE_MINMAX = 1 };
+/* INT scale modes: ABSMAX = the ggml signed grid; MINMAX = asymmetric; SYMMETRIC = levels
+ * (q - (2^b - 1)/2) d, outermost level at the group's largest magnitude ([E22L] "Result": the
+ * signed grid "leaves one side with fewer levels"; a symmetric grid is the next candidate). */
+enum { KVQ_SCALE_ABSMAX = 0, KVQ_SCALE_MINMAX = 1, KVQ_SCALE_SYMMETRIC = 2 };
 enum { KVQ_ROT_NONE = 0, KVQ_ROT_H128 = 128, KVQ_ROT_H256 = 256 };
 enum { KVQ_ANCHOR_NONE = 0, KVQ_ANCHOR_FIRST_N = 1, KVQ_ANCHOR_WINDOW = 2, KVQ_ANCHOR_ALL = 3 };
 enum { KVQ_SIDE_K = 0, KVQ_SIDE_V = 1 };
@@ -80,6 +85,13 @@ typedef struct {
   int32_t chan_scale;  /* K only: 1 = divide by a per-(layer, kv-head) fp16 channel scale
                           before the rotation ([E21W] variants C/D); set with
                           kvq_set_chan_scale before the first append. */
+  int32_t mean_sub;    /* K only, quantized formats: 1 = subtract the sequence's key mean before
+                          everything else and add it back after dequantizing ([LCPP], the later
+                          comment on a per-head shared key mean: "subtracting the running mean
+                          before quantization and restoring it after").  The mean of a (sequence,
+                          kv-head) is the mean of the rows of the sequence's first append (its
+                          length was 0), rounded to fp16 once from the exact sum, and is kept for
+                          the rows that follow; anchored rows stay raw. */
 } kvq_side;
 
 typedef struct {
@@ -105,6 +117,7 @@ typedef struct {
  * slot = t (FIRST_N, ALL) or t mod anchor_n (WINDOW).  Offsets are -1 when absent. */
 typedef struct {
   int64_t codes, scales, zeros, anchors, chan_scale, seq_len;
+  int64_t key_mean;  /* K with mean_sub: fp16 [batch * n_kv_heads][head_dim], unit u at u * head_dim */
   int32_t row_bytes, n_groups, row_stride_tokens, anchor_rows;
 } kvq_layout;
 
@@ -227,6 +240,10 @@ kvq_status kvq_error_flags(kvq_cache* cache, int32_t* flags);
 
 /* The 16 NF4 levels this library stores (fp16-exact values, ascending).  Host only. */
 kvq_status kvq_nf4_levels(float out[16]);
+
+/* The 2^bits Gaussian Lloyd-Max levels (bits 2..4) this library stores, in units of the
+ * group RMS (fp16-exact values, ascending).  Host only. */
+kvq_status kvq_lloyd_levels(int32_t bits, float* out);
 
 /* Kernels launched by the last kvq_decode_attention / kvq_quantize_append call on this
  * handle (for launch accounting).  Host only. */

@@ -27,6 +27,7 @@ __constant__ float d_tw_re[64];
 __constant__ float d_tw_im[64];
 __constant__ float d_ph_cos[512];
 __constant__ float d_ph_sin[512];
+__constant__ float d_lloyd[3][16];
 
 cudaError_t upload_tables_decode(const HostTables& t) {
   cudaError_t e;
@@ -34,6 +35,7 @@ cudaError_t upload_tables_decode(const HostTables& t) {
   if ((e = cudaMemcpyToSymbol(d_tw_re, t.tw_re, sizeof(t.tw_re))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_tw_im, t.tw_im, sizeof(t.tw_im))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_ph_cos, t.ph_cos, sizeof(t.ph_cos))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_lloyd, t.lloyd, sizeof(t.lloyd))) != cudaSuccess) return e;
   return cudaMemcpyToSymbol(d_ph_sin, t.ph_sin, sizeof(t.ph_sin));
 }
 
@@ -83,6 +85,26 @@ __device__ __forceinline__ QueryRange query_range(const LayerDev& L, int qi, con
     }
   }
   return r;
+}
+
+// (q . mu) x sm_scale log2 e for the G heads of kv-head kvh, into qmu[G]: the logit every
+// quantized row of a key-mean-subtracted sequence gets back (the original-domain dot product of
+// the raw query with the sequence's fp16 key mean).  Zero without a key mean.  Warps take heads
+// in turn; the caller synchronizes before reading.
+__device__ void query_mean_term(const LayerDev& L, const __half* __restrict__ q, int qi, int seq, int kvh, int G,
+                                float* qmu) {
+  const SideDev& K = L.s[0];
+  const int lane = threadIdx.x & 31, D = L.D;
+  for (int h = threadIdx.x >> 5; h < G; h += blockDim.x >> 5) {
+    float acc = 0.0f;
+    if (K.mean_sub) {
+      const __half* qp = q + ((long long)qi * L.Hq + kvh * G + h) * D;
+      const __half* mp = K.kmean + ((long long)seq * L.Hkv + kvh) * D;
+      for (int j = lane; j < D; j += 32) acc = fmaf(__half2float(qp[j]), __half2float(mp[j]), acc);
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    }
+    if (lane == 0) qmu[h] = acc * (L.sm_scale * kLog2e);
+  }
 }
 
 // q' for G heads into qs[G][D] (stored domain of K, x sm_scale log2 e) and qa[G][D] (raw, x same).
@@ -167,8 +189,9 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
   __shared__ float qs[kMaxG * D], qa[kMaxG * D];
   __shared__ float sp[kMaxG][kGenTile];
   __shared__ float m_run[kMaxG], l_run[kMaxG], alpha[kMaxG];
-  __shared__ float nf4[16], kcs[256], ksn[256], vcs[256], vsn[256];
+  __shared__ float nf4[16], klm[16], vlm[16], kcs[256], ksn[256], vcs[256], vsn[256];
   __shared__ float red[kGenThreads / 32][kMaxG];
+  __shared__ float qmu[kMaxG];
 
   const QueryRange R = query_range(L, qi, seq_ids, kv_len);
   const SideDev& K = L.s[0];
@@ -187,6 +210,8 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
   }
 
   if (tid < 16) nf4[tid] = d_nf4[tid];
+  if (K.fmt == KVQ_FMT_LLOYD && tid < 16) klm[tid] = d_lloyd[K.bits - 2][tid];
+  if (V.fmt == KVQ_FMT_LLOYD && tid < 16) vlm[tid] = d_lloyd[V.bits - 2][tid];
   if (K.fmt == KVQ_FMT_POLAR)
     for (int k = tid; k < (1 << K.bits2); k += blockDim.x) {
       kcs[k] = d_ph_cos[(1 << K.bits2) - 2 + k];
@@ -201,6 +226,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.0f;
   }
+  query_mean_term(L, q, qi, R.seq, kvh, G, qmu);
   prepare_query<D>(L, q, qi, kvh, G, qs, qa);
 
   const long long u = (long long)R.seq * L.Hkv + kvh;
@@ -240,12 +266,15 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
           }
         } else {
           for (int j = 0; j < D; ++j) {
-            const float kv = stored_value(K, row, sc, zr, j, nf4);
+            const float kv = stored_value(K, row, sc, zr, j, nf4, klm);
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h)
               if (h < G) acc[h] += qs[h * D + j] * kv;
           }
         }
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+          if (h < G) acc[h] += qmu[h];
       }
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h)
@@ -314,7 +343,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
               const float2 ab = polar_slot(V, row, sc, j >> 1, vcs, vsn);
               vv = (j & 1) ? ab.y : ab.x;
             } else {
-              vv = stored_value(V, row, sc, zr, j, nf4);
+              vv = stored_value(V, row, sc, zr, j, nf4, vlm);
             }
           }
 #pragma unroll
@@ -509,6 +538,7 @@ static int code_fmt(const SideDev& S, bool is_v) {
   if (S.fmt == KVQ_FMT_TERNARY) return CF_TERN;
   if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && (S.bits == 4 || S.bits == 2)) return S.bits;
   if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_ABSMAX && S.bits == 3 && is_v) return CF_INT3;
+  if (S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_SYMMETRIC && S.bits == 2 && is_v) return CF_SYM2;
   return -1;
 }
 
@@ -533,6 +563,7 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2)
   KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 32, 3)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_SYM2, 128, 4, 32, 3)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT3, 128, 4, 32, 3)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
   KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)

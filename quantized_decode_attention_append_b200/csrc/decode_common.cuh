@@ -29,10 +29,11 @@ __device__ __forceinline__ int get_trit(const uint8_t* __restrict__ row, int j) 
 }
 
 // Stored-domain value of element j of a non-polar quantized row.
-//   row: packed codes; sc/zr: the row's fp16 scales / zero points; nf4: 16 levels.
+//   row: packed codes; sc/zr: the row's fp16 scales / zero points; nf4: 16 levels; lloyd: the
+//   2^bits Gaussian Lloyd-Max levels of the side's width.
 __device__ __forceinline__ float stored_value(const SideDev& S, const uint8_t* __restrict__ row,
                                               const __half* __restrict__ sc, const __half* __restrict__ zr,
-                                              int j, const float* nf4) {
+                                              int j, const float* nf4, const float* lloyd) {
   switch (S.fmt) {
     case KVQ_FMT_FP16:
       return __half2float(reinterpret_cast<const __half*>(row)[j]);
@@ -41,8 +42,11 @@ __device__ __forceinline__ float stored_value(const SideDev& S, const uint8_t* _
       const float d = __half2float(sc[g]);
       const int c = (int)get_bits(row, j * S.bits, S.bits);
       if (S.scale_mode == KVQ_SCALE_MINMAX) return __fadd_rn(__half2float(zr[g]), (float)c * d);
+      if (S.scale_mode == KVQ_SCALE_SYMMETRIC) return ((float)c - 0.5f * (float)((1 << S.bits) - 1)) * d;
       return (float)(c - (1 << (S.bits - 1))) * d;
     }
+    case KVQ_FMT_LLOYD:
+      return lloyd[get_bits(row, j * S.bits, S.bits)] * __half2float(sc[j / S.group]);
     case KVQ_FMT_NF4: {
       const float s = __half2float(sc[j / S.group]);
       return nf4[get_bits(row, j * 4, 4)] * s;

@@ -34,12 +34,14 @@
 // the pair of probabilities a score thread owns is one 32-bit word of P'.  P' is staged per warp in
 // rows of 12 words (16 halves + 4 pad), which keeps its stores and fragment loads conflict-free.
 
-enum CodeFmt { CF_INT2 = 2, CF_INT3 = 3, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64, CF_TERN = 128 };
+// CF_SYM2: 2-bit codes of the symmetric grid, value code - 3/2 (exact in fp16).
+enum CodeFmt { CF_INT2 = 2, CF_INT3 = 3, CF_INT4 = 4, CF_NF4 = 16, CF_FP16 = 32, CF_SIGN = 64, CF_TERN = 128,
+               CF_SYM2 = 256 };
 
 template <int F> struct CodeBits {
   // bits per value in the layout the operands are built from (ternary: transcoded 2-bit digits)
   static constexpr int v =
-      F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : (F == CF_TERN ? 2 : (F == CF_INT3 ? 4 : F))));
+      F == CF_NF4 ? 4 : (F == CF_FP16 ? 16 : (F == CF_SIGN ? 1 : (F == CF_TERN || F == CF_SYM2 ? 2 : (F == CF_INT3 ? 4 : F))));
 };
 
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -76,10 +78,11 @@ __device__ __forceinline__ __half2 h2c(unsigned short bits) {
   return __halves2half2(h, h);
 }
 
-// The 16/B field pairs of a 32-bit word of B-bit offset-binary codes as signed fp16 pairs:
+// The 16/B field pairs of a 32-bit word of B-bit offset-binary codes as signed fp16 pairs
+// (field - ofs, exact while ofs is a multiple of 1/2 below 2^9):
 // out[k] = (field k, field k + 16/B), i.e. field k of each 16-bit half.
-template <int B, int OFS = (1 << (B - 1))>
-__device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out) {
+template <int B>
+__device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out, float ofs = (float)(1 << (B - 1))) {
   constexpr int PH = 16 / B;                 // fields per 16-bit half
   constexpr int PB = 8 / B;                  // fields per byte
   constexpr uint32_t M = ((1u << B) - 1u) * 0x00010001u;
@@ -90,7 +93,7 @@ __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out) {
     const uint32_t x = and_or(k < PB ? w : w8, M << s, 0x64006400u);  // 1024 + 2^s field
     // 2^-s and -(1024 2^-s + 2^(B-1)) as fp16 bit patterns
     const unsigned short scl = (unsigned short)((15 - s) << 10);
-    const float off = -(1024.0f / (float)(1 << s) + (float)OFS);
+    const float off = -(1024.0f / (float)(1 << s) + ofs);
     const __half2 r = __hfma2(u2h(x), h2c(scl), __float2half2_rn(off));
     out[k] = h2u(r);
   }
@@ -146,7 +149,7 @@ __device__ __forceinline__ void sign_pairs_v(uint32_t ab, const uint32_t* sa, co
 // dd holds the scales of the two elements of each pair (low, high half).
 __device__ __forceinline__ void tern_pairs(uint32_t w, uint32_t dd, uint32_t* out) {
   uint32_t r[8];
-  code_pairs<2, 1>(w, r);
+  code_pairs<2>(w, r, 1.0f);
 #pragma unroll
   for (int k = 0; k < 8; ++k) out[k] = h2u(__hmul2(u2h(r[k]), u2h(dd)));
 }
@@ -234,7 +237,7 @@ struct TcCfg {
   static constexpr bool KTRN = KF == CF_TERN, VTRN = VF == CF_TERN;  // ternary rows transcoded per warp
   static constexpr bool V3 = VF == CF_INT3;                          // int3 V rows transcoded to nibbles
   static constexpr bool VX = VTRN || V3;                             // V read from the transcode buffer
-  static constexpr int VOFS = V3 ? 4 : (1 << (VB - 1));              // code offset of the V fields
+  static constexpr float VOFS = V3 ? 4.0f : (VF == CF_SYM2 ? 1.5f : (float)(1 << (VB - 1)));  // V code offset
   static constexpr bool KSCL = KSGN || KTRN, VSCL = VSGN || VTRN;    // scale inside the operand
   static constexpr bool VSCALE = VF != CF_FP16 && !VSCL;  // V scale folded into P'
   static constexpr bool VSROW = VF != CF_FP16;            // V rows carry scales
@@ -258,7 +261,8 @@ struct TcCfg {
   static constexpr bool ALT = RBK >= 128;              // row -> (half, index) mapping
   // log2 headroom of p over the running max: |d_v| <= 65504 / 2^(b-1) for b-bit absmax V, so
   // p <= 2^(b-1) keeps p * d_v finite in fp16; P' carries no scale for fp16 and sign V.
-  static constexpr float SLACK = VSCALE ? (float)((V3 ? 3 : VB) - 1) : 8.0f;
+  // (symmetric 2-bit: |d_v| <= 65504 / 1.5, so p <= 1)
+  static constexpr float SLACK = VSCALE ? (VF == CF_SYM2 ? 0.0f : (float)((V3 ? 3 : VB) - 1)) : 8.0f;
   static constexpr int PADK = RBK == 64 ? 32 : 64, PADV = RBV == 64 ? 32 : 64, PADS = 16;
   // stage: [K codes A | pad | K codes B][K scales A | pad | B][V codes A | pad | B][V scales A | pad | B]
   static constexpr int KC_H = HALF * RSK, KS_H = HALF * NGK * 2;
@@ -275,7 +279,7 @@ struct TcCfg {
   static constexpr int PKS = 12;                       // words per staged P' row
   static constexpr int PK_WORDS = NPV * 8 * PKS;       // per warp
   static constexpr int PK_BYTES_RAW = NW * PK_WORDS * 4;
-  static constexpr int QS_BYTES = 4 * D * 4;           // query staging aliases the P' area
+  static constexpr int QS_BYTES = (4 * D + 4) * 4;     // query staging (+ q . mu per head) aliases the P' area
   static constexpr int PK_BYTES = PK_BYTES_RAW > QS_BYTES ? PK_BYTES_RAW : QS_BYTES;
   static constexpr int LUT_BYTES = (KF == CF_NF4 || KTRN || VTRN) ? 256 * 32 * 4 : 0;
   static constexpr int OFF_PK = RING_BYTES, OFF_LUT = OFF_PK + PK_BYTES, OFF_X = OFF_LUT + LUT_BYTES;
@@ -407,6 +411,8 @@ __device__ __forceinline__ void int3_transcode(const unsigned char* src, unsigne
     reinterpret_cast<uint4*>(dst)[o / 4] = make_uint4(out[o], out[o + 1], out[o + 2], out[o + 3]);
 }
 
+__device__ __forceinline__ bool head_ok_of(int c, int G) { return c < G; }
+
 template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
 __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
                                                             const int* __restrict__ seq_ids,
@@ -501,7 +507,10 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
     }
   }
   float* qs = reinterpret_cast<float*>(smem + C::OFF_PK);
+  query_mean_term(L, q, qi, R.seq, kvh, G, qs + 4 * D);
   prepare_query_rot<D>(L, q, qi, kvh, G, qs);
+  // logit term of the sequence's key mean (0 without one): it starts every score accumulator
+  const float kmu = head_ok_of(c, G) ? qs[4 * D + c] : 0.0f;
   uint32_t qreg[C::NGKM][C::KSTEPS][2];
   {
     const int h = g >> 1, part = g & 1;
@@ -631,7 +640,7 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
             tern_pairs(kw1[w], sv1[w], kp1 + 8 * w);
           }
         }
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float acc[4] = {kmu, 0.0f, kmu, 0.0f};
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks)
           mma16816(acc, kp0[2 * ks], kp1[2 * ks], kp0[2 * ks + 1], kp1[2 * ks + 1], qreg[0][ks][0], qreg[0][ks][1]);
@@ -662,7 +671,7 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
       }
       const unsigned char* k0p = kb_ + kc_off + sb * 8 * C::RBK;
       const unsigned char* k1p = k0p + 4 * C::RBK;
-      float s0 = 0.0f, s1 = 0.0f;
+      float s0 = kmu, s1 = kmu;
 #pragma unroll
       for (int j = 0; j < C::NGK; ++j) {
         uint32_t kw0[C::KCW], kw1[C::KCW];
@@ -852,8 +861,8 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
 #pragma unroll
           for (int hh = 0; hh < C::VCH; ++hh) {
             const int w = hh >> 1, hf = hh & 1;
-            code_pairs<C::VB, C::VOFS>(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), pa + hh * PH);
-            code_pairs<C::VB, C::VOFS>(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), pc + hh * PH);
+            code_pairs<C::VB>(prmt(vw[0][w], vw[1][w], hf ? 0x7632 : 0x5410), pa + hh * PH, C::VOFS);
+            code_pairs<C::VB>(prmt(vw[2][w], vw[3][w], hf ? 0x7632 : 0x5410), pc + hh * PH, C::VOFS);
           }
         }
 #pragma unroll

@@ -11,6 +11,7 @@ __constant__ float dq_tw_re[64];
 __constant__ float dq_tw_im[64];
 __constant__ float dq_ph_cos[512];
 __constant__ float dq_ph_sin[512];
+__constant__ float dq_lloyd[3][16];
 
 cudaError_t upload_tables_dequant(const HostTables& t) {
   cudaError_t e;
@@ -18,6 +19,7 @@ cudaError_t upload_tables_dequant(const HostTables& t) {
   if ((e = cudaMemcpyToSymbol(dq_tw_re, t.tw_re, sizeof(t.tw_re))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(dq_tw_im, t.tw_im, sizeof(t.tw_im))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(dq_ph_cos, t.ph_cos, sizeof(t.ph_cos))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(dq_lloyd, t.lloyd, sizeof(t.lloyd))) != cudaSuccess) return e;
   return cudaMemcpyToSymbol(dq_ph_sin, t.ph_sin, sizeof(t.ph_sin));
 }
 
@@ -29,8 +31,9 @@ __global__ void __launch_bounds__(128) dequant_kernel(LayerDev L, int side, int 
   const int D = L.D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float buf[kDqWarps][256], tmp[kDqWarps][256];
-  __shared__ float nf4[16], cs[256], sn[256];
+  __shared__ float nf4[16], lloyd[16], cs[256], sn[256];
   if (threadIdx.x < 16) nf4[threadIdx.x] = dq_nf4[threadIdx.x];
+  if (S.fmt == KVQ_FMT_LLOYD && threadIdx.x < 16) lloyd[threadIdx.x] = dq_lloyd[S.bits - 2][threadIdx.x];
   if (S.fmt == KVQ_FMT_POLAR)
     for (int k = threadIdx.x; k < (1 << S.bits2); k += blockDim.x) {
       cs[k] = dq_ph_cos[(1 << S.bits2) - 2 + k];
@@ -55,7 +58,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(LayerDev L, int side, int 
       x[2 * f + 1] = ab.y;
     }
   } else {
-    for (int j = lane; j < D; j += 32) x[j] = stored_value(S, cr, sc, zr, j, nf4);
+    for (int j = lane; j < D; j += 32) x[j] = stored_value(S, cr, sc, zr, j, nf4, lloyd);
   }
   __syncwarp();
   if (domain == KVQ_DOMAIN_ORIGINAL) {
@@ -93,6 +96,8 @@ __global__ void __launch_bounds__(128) dequant_kernel(LayerDev L, int side, int 
     }
     if (S.chan_scale)
       for (int j = lane; j < D; j += 32) x[j] *= __half2float(S.chan[(u % L.Hkv) * D + j]);
+    if (S.mean_sub)
+      for (int j = lane; j < D; j += 32) x[j] += __half2float(S.kmean[u * D + j]);
     // anchored rows: attention reads the fp16 copy
     bool anc = false;
     if (L.anchored) {

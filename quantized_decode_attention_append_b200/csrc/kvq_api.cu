@@ -23,6 +23,7 @@ struct kvq_cache {
     int row_bytes, n_groups;
   } off[64][2];
   int64_t chan[64];
+  int64_t kmean[64];
   int64_t lens, tickets, err;
   int anchor_rows;
   int max_len[64];       // host-side bound on every sequence's length (exact while len_exact)
@@ -45,8 +46,10 @@ bool is_pow2_group(int g) { return g == 4 || g == 8 || g == 16 || g == 32 || g =
 
 kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
   const int D = c.head_dim;
-  if (!is_k && s.chan_scale) return KVQ_ERR_INVALID_ARG;
+  if (!is_k && (s.chan_scale || s.mean_sub)) return KVQ_ERR_INVALID_ARG;
   if (s.chan_scale != 0 && s.chan_scale != 1) return KVQ_ERR_INVALID_ARG;
+  if (s.mean_sub != 0 && s.mean_sub != 1) return KVQ_ERR_INVALID_ARG;
+  if (s.mean_sub && s.format == KVQ_FMT_FP16) return KVQ_ERR_INVALID_ARG;
   if (s.rotation != KVQ_ROT_NONE && s.rotation != KVQ_ROT_H128 && s.rotation != KVQ_ROT_H256)
     return KVQ_ERR_INVALID_ARG;
   if (s.rotation > D) return KVQ_ERR_INVALID_ARG;
@@ -56,7 +59,12 @@ kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
       return KVQ_OK;
     case KVQ_FMT_INT:
       if (s.bits < 2 || s.bits > 8) return KVQ_ERR_INVALID_ARG;
-      if (s.scale_mode != KVQ_SCALE_ABSMAX && s.scale_mode != KVQ_SCALE_MINMAX) return KVQ_ERR_INVALID_ARG;
+      if (s.scale_mode != KVQ_SCALE_ABSMAX && s.scale_mode != KVQ_SCALE_MINMAX && s.scale_mode != KVQ_SCALE_SYMMETRIC)
+        return KVQ_ERR_INVALID_ARG;
+      break;
+    case KVQ_FMT_LLOYD:
+      if (s.bits < 2 || s.bits > 4) return KVQ_ERR_INVALID_ARG;
+      if (s.scale_mode != KVQ_SCALE_ABSMAX) return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_FMT_NF4:
     case KVQ_FMT_TERNARY:
@@ -122,7 +130,8 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
 void side_geometry(int D, const kvq_side& s, int* row_bytes, int* n_groups) {
   switch (s.format) {
     case KVQ_FMT_FP16: *row_bytes = 2 * D; *n_groups = 0; return;
-    case KVQ_FMT_INT: *row_bytes = D * s.bits / 8; *n_groups = D / s.group; return;
+    case KVQ_FMT_INT:
+    case KVQ_FMT_LLOYD: *row_bytes = D * s.bits / 8; *n_groups = D / s.group; return;
     case KVQ_FMT_NF4: *row_bytes = D / 2; *n_groups = D / s.group; return;
     case KVQ_FMT_TERNARY: *row_bytes = (D + 4) / 5; *n_groups = D / s.group; return;
     case KVQ_FMT_SIGN: *row_bytes = D / 8; *n_groups = D / s.group; return;
@@ -177,6 +186,12 @@ uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
       off = align_up(off + (uint64_t)c.n_kv_heads * D * 2);
     }
     if (h) h->chan[l] = ch;
+    int64_t km = -1;
+    if (sides.s[l][0].mean_sub) {
+      km = (int64_t)off;
+      off = align_up(off + units * D * 2);
+    }
+    if (h) h->kmean[l] = km;
   }
   const int64_t lens = (int64_t)off;
   off = align_up(off + (uint64_t)c.n_layers * c.batch * 4);
@@ -206,6 +221,8 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
     S.zeros = so.zeros >= 0 ? reinterpret_cast<__half*>(h->arena + so.zeros) : nullptr;
     S.anchors = so.anchors >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchors) : nullptr;
     S.chan = (s == 0 && h->chan[l] >= 0) ? reinterpret_cast<const __half*>(h->arena + h->chan[l]) : nullptr;
+    S.kmean = (s == 0 && h->kmean[l] >= 0) ? reinterpret_cast<__half*>(h->arena + h->kmean[l]) : nullptr;
+    S.mean_sub = s == 0 ? sd.mean_sub : 0;
     S.fmt = sd.format;
     S.bits = sd.bits;
     S.bits2 = sd.bits2;
@@ -275,6 +292,31 @@ HostTables build_tables() {
     t.tw_re[k] = (float)cos(2.0 * M_PI * k / 128.0);
     t.tw_im[k] = (float)(-sin(2.0 * M_PI * k / 128.0));
   }
+  // Gaussian Lloyd-Max levels: thresholds at midpoints, levels at the centroids of their cells
+  // (standard normal: (phi(a) - phi(b)) / (Phi(b) - Phi(a))), alternated from evenly spaced levels
+  // until they stop moving; stored at fp16 precision.
+  for (int bi = 0; bi < 3; ++bi) {
+    const int n = 4 << bi;
+    double lv[16], nx[16];
+    for (int k = 0; k < n; ++k) lv[k] = -2.0 + 4.0 * k / (n - 1);
+    for (int it = 0; it < 200000; ++it) {
+      double delta = 0.0;
+      for (int k = 0; k < n; ++k) {
+        const double a = k == 0 ? -INFINITY : 0.5 * (lv[k - 1] + lv[k]);
+        const double b = k == n - 1 ? INFINITY : 0.5 * (lv[k] + lv[k + 1]);
+        const double pa = isinf(a) ? 0.0 : exp(-0.5 * a * a) / sqrt(2.0 * M_PI);
+        const double pb = isinf(b) ? 0.0 : exp(-0.5 * b * b) / sqrt(2.0 * M_PI);
+        const double Pa = isinf(a) ? 0.0 : 0.5 * erfc(-a / sqrt(2.0));
+        const double Pb = isinf(b) ? 1.0 : 0.5 * erfc(-b / sqrt(2.0));
+        nx[k] = (pa - pb) / (Pb - Pa);
+        delta = fmax(delta, fabs(nx[k] - lv[k]));
+      }
+      for (int k = 0; k < n; ++k) lv[k] = nx[k];
+      if (delta < 1e-12) break;
+    }
+    for (int k = 0; k < n; ++k) t.lloyd[bi][k] = __half2float(__double2half(lv[k]));
+    for (int k = 0; k + 1 < n; ++k) t.lloyd_mid[bi][k] = 0.5f * (t.lloyd[bi][k] + t.lloyd[bi][k + 1]);
+  }
   for (int bp = 1; bp <= 8; ++bp) {
     const int nb = 1 << bp;
     for (int k = 0; k < nb; ++k) {
@@ -328,6 +370,12 @@ const char* kvq_status_str(kvq_status s) {
 kvq_status kvq_nf4_levels(float out[16]) {
   if (!out) return KVQ_ERR_INVALID_ARG;
   memcpy(out, host_tables().nf4, sizeof(float) * 16);
+  return KVQ_OK;
+}
+
+kvq_status kvq_lloyd_levels(int32_t bits, float* out) {
+  if (!out || bits < 2 || bits > 4) return KVQ_ERR_INVALID_ARG;
+  memcpy(out, host_tables().lloyd[bits - 2], sizeof(float) << bits);
   return KVQ_OK;
 }
 
@@ -432,6 +480,7 @@ kvq_status kvq_get_layout(const kvq_cache* h, int32_t layer, int32_t side, kvq_l
   out->zeros = so.zeros;
   out->anchors = so.anchors;
   out->chan_scale = side == 0 ? h->chan[layer] : -1;
+  out->key_mean = side == 0 ? h->kmean[layer] : -1;
   out->seq_len = h->lens + (int64_t)layer * h->cfg.batch * 4;
   out->row_bytes = so.row_bytes;
   out->n_groups = so.n_groups;
@@ -485,8 +534,17 @@ kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const
   L.app_ids = seq_ids;
   L.app_n = n_seqs;
   int launches = 0;
-  const cudaError_t e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,
-                                      reinterpret_cast<cudaStream_t>(stream), &launches);
+  cudaError_t e = cudaSuccess;
+  if (L.s[0].mean_sub) {  // key means of the sequences this append starts, before their rows
+    e = launch_key_mean(L, reinterpret_cast<const __half*>(k), n_new, reinterpret_cast<cudaStream_t>(stream));
+    ++launches;
+  }
+  if (e == cudaSuccess) {
+    int n = 0;
+    e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,
+                      reinterpret_cast<cudaStream_t>(stream), &n);
+    launches += n;
+  }
   h->last_launches = launches;
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
   const int64_t nl = (int64_t)h->max_len[layer] + n_new;

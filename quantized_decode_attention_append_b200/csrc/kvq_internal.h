@@ -19,7 +19,8 @@ struct SideDev {
   __half* zeros;         // [B*Hkv][Tcap][n_groups] (MINMAX) or null
   __half* anchors;       // [B*Hkv][anchor_rows][D] or null
   const __half* chan;    // [Hkv][D] (K with chan_scale) or null
-  int fmt, bits, bits2, scale_mode, group, rot, chan_scale;
+  __half* kmean;         // [B*Hkv][D] key means (K with mean_sub) or null
+  int fmt, bits, bits2, scale_mode, group, rot, chan_scale, mean_sub;
   int row_bytes, n_groups;
 };
 
@@ -48,6 +49,8 @@ struct HostTables {
   float nf4_mid[15];
   float tw_re[64], tw_im[64];     // W_128^k = exp(-2 pi i k/128), k < 64
   float ph_cos[512], ph_sin[512]; // phase angle -pi + 2 pi k / 2^bp at offset 2^bp - 2
+  float lloyd[3][16];             // Gaussian Lloyd-Max levels for 2, 3, 4 bits (2^b used)
+  float lloyd_mid[3][15];         // their midpoints
 };
 
 const HostTables& host_tables();
@@ -66,6 +69,8 @@ cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int
                           const int* kv_len, void* out, int out_fp32, float* lse, float* work,
                           int num_sms, int max_queries, cudaStream_t st, int* launches);
 cudaError_t launch_fill_len(int* lens, int n, int value, cudaStream_t st);
+// Key means of the listed sequences whose first append this is (K side with mean_sub).
+cudaError_t launch_key_mean(const LayerDev& L, const __half* k, int n_new, cudaStream_t st);
 
 // Split-K partials per (query, head) one decode call on `L` writes (workspace sizing).
 int decode_partials(const LayerDev& L, int n_q, int num_sms);

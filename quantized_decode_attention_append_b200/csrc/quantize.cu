@@ -35,16 +35,19 @@ __device__ __forceinline__ uint32_t bsel(uint32_t m, uint32_t a, uint32_t b) { r
 __constant__ float q_nf4_mid[15];
 __constant__ float q_tw_re[64];
 __constant__ float q_tw_im[64];
+__constant__ float q_lloyd_mid[3][15];
 
 cudaError_t upload_tables_quant(const HostTables& t) {
   cudaError_t e = cudaMemcpyToSymbol(q_nf4_mid, t.nf4_mid, sizeof(t.nf4_mid));
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(q_lloyd_mid, t.lloyd_mid, sizeof(t.lloyd_mid));
   if (e != cudaSuccess) return e;
   e = cudaMemcpyToSymbol(q_tw_re, t.tw_re, sizeof(t.tw_re));
   if (e != cudaSuccess) return e;
   return cudaMemcpyToSymbol(q_tw_im, t.tw_im, sizeof(t.tw_im));
 }
 
-enum Fam { FAM_ABSMAX = 0, FAM_MINMAX = 1, FAM_NF4 = 2, FAM_TERNARY = 3, FAM_SIGN = 4 };
+enum Fam { FAM_ABSMAX = 0, FAM_MINMAX = 1, FAM_NF4 = 2, FAM_TERNARY = 3, FAM_SIGN = 4, FAM_SYM = 5, FAM_LLOYD = 6 };
 
 // Exact k = floor(x/d + 1/2) for fp16 d != 0 (absmax grids, zero point 0), in fp32.
 // (2k +- 1) d is exact in fp32 for |k| <= 2^9, and 2x is exact, so the comparisons are exact.
@@ -229,6 +232,7 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
     float* im = sim[warp];
     for (int j = lane; j < 128; j += 32) {
       float v = __half2float(rp[j]);
+      if (S.mean_sub) v = __fsub_rn(v, __half2float(S.kmean[(long long)u * 128 + j]));
       if (S.chan_scale) v = __fdiv_rn(v, __half2float(S.chan[(u % L.Hkv) * 128 + j]));
       re[bitrev7(j)] = v;
       im[bitrev7(j)] = 0.0f;
@@ -422,6 +426,8 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   constexpr int GPL = G > 32 ? 1 : 32 / G;            // groups per lane
   // code bits: fixed by the family, by the instance (BITS > 0), or read from the side
   const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : (BITS > 0 ? BITS : S.bits));
+  // the grid sees the fp16 input itself (no key mean, channel scale or rotation in between)
+  const bool raw = !S.rot && !S.chan_scale && !S.mean_sub;
 
   // The next pass's input slice is loaded before this pass's arithmetic, so each warp keeps its
   // loads in flight while it computes (the arithmetic per row is long).
@@ -467,7 +473,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
 #pragma unroll
         for (int e = 0; e < 4; ++e) raw2[c4 * 4 + e] = h2[e];
       }
-      if (!(FAM == FAM_NF4 && !S.rot && !S.chan_scale)) {  // NF4 on untransformed rows reads raw2 only
+      if (!(FAM == FAM_NF4 && raw)) {  // NF4 on untransformed rows reads raw2 only
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 f = __half22float2(raw2[e]);
@@ -479,6 +485,11 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + li * 32;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
+      }
+      if (S.mean_sub) {
+        const __half* mp = S.kmean + (long long)u * D + li * 32;
+#pragma unroll
+        for (int v = 0; v < 32; ++v) x[v] = __fsub_rn(x[v], __half2float(mp[v]));
       }
       if (S.chan_scale) {
         const __half* cp = S.chan + (u % L.Hkv) * D + li * 32;
@@ -529,7 +540,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         // whichever is larger in magnitude; only a group holding both +a and -a (or only zeros)
         // needs the earliest channel reaching a, found by a backward scan
         float mx, mn;
-        if (NV >= 2 && !S.rot && !S.chan_scale) {  // x is the fp16 input: max and min two at a time
+        if (NV >= 2 && raw) {  // x is the fp16 input: max and min two at a time
           const __half2* rg = raw2 + (gl * NV) / 2;
           __half2 hx = rg[0], hn = rg[0];
 #pragma unroll
@@ -622,6 +633,56 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
           if (d != 0.0f) k = fminf(fmaxf(round_exact_minmax(xg[v], z, d, inv), 0.0f), (float)top);
           code[gl * NV + v] = (uint32_t)(int)k;
         }
+      } else if (FAM == FAM_SYM) {
+        // levels (q - (2^b - 1)/2) d with the outermost at the group's largest magnitude:
+        // d = fp16(m / (2^(b-1) - 1/2)), q = floor(x/d) + 2^(b-1) clamped; floor(x/d) from an fp32
+        // estimate corrected by the exact products k d and (k + 1) d
+        float am = fabsf(xg[0]);
+#pragma unroll
+        for (int v = 1; v < NV; ++v) am = fmaxf(am, fabsf(xg[v]));
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        const int half = 1 << (bits - 1);
+        sh = __float2half_rn(__fdiv_rn(am, (float)half - 0.5f));
+        d = __half2float(sh);
+        inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float k = floorf(__fmul_rn(xg[v], inv));
+          if (xg[v] < __fmul_rn(k, d)) k -= 1.0f;
+          else if (xg[v] >= __fmul_rn(k + 1.0f, d)) k += 1.0f;
+          const float q = fminf(fmaxf(k + (float)half, 0.0f), (float)(2 * half - 1));
+          code[gl * NV + v] = d != 0.0f ? (uint32_t)(int)q : (uint32_t)half;
+        }
+      } else if (FAM == FAM_LLOYD) {
+        // Gaussian Lloyd-Max levels times the group RMS: s = fp16(sqrt(fp32(sum of rounded
+        // squares in channel order) / g)); the code counts the thresholds (level midpoints times s,
+        // exact in fp32) that x reaches
+        float sum = 0.0f;
+        if (LG == 1) {
+#pragma unroll
+          for (int v = 0; v < NV; ++v) sum = __fadd_rn(sum, __fmul_rn(xg[v], xg[v]));
+        } else {
+          const int base = lane - (li % LG);
+#pragma unroll
+          for (int k = 0; k < LG; ++k) {
+            if ((li % LG) == k) {
+#pragma unroll
+              for (int v = 0; v < NV; ++v) sum = __fadd_rn(sum, __fmul_rn(xg[v], xg[v]));
+            }
+            sum = __shfl_sync(0xffffffffu, sum, base + k);
+          }
+        }
+        sh = __float2half_rn(__fsqrt_rn(__fdiv_rn(sum, (float)G)));
+        d = __half2float(sh);
+        const int nl = 1 << bits;
+        const float* mid = q_lloyd_mid[bits - 2];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          uint32_t c = 0u;
+          for (int k = 0; k < nl - 1; ++k) c += xg[v] >= __fmul_rn(mid[k], d) ? 1u : 0u;
+          code[gl * NV + v] = d != 0.0f ? c : (uint32_t)(nl >> 1);
+        }
       } else if (FAM == FAM_SIGN) {
         float sum = 0.0f;  // fp32 sum of |x| in channel order, lane by lane across the group
         if (LG == 1) {
@@ -643,7 +704,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         for (int v = 0; v < NV; ++v) code[gl * NV + v] = xg[v] >= 0.0f ? 1u : 0u;
       } else {  // NF4 and ternary: absmax magnitude scale
         float am;
-        if (FAM == FAM_NF4 && NV >= 2 && !S.rot && !S.chan_scale) {  // from the fp16 input pairs
+        if (FAM == FAM_NF4 && NV >= 2 && raw) {  // from the fp16 input pairs
           const __half2* rg = raw2 + (gl * NV) / 2;
           __half2 hx = rg[0], hn = rg[0];
 #pragma unroll
@@ -659,7 +720,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         sh = __float2half_rn(am);
         d = __half2float(sh);
         if (FAM == FAM_NF4) {
-          if (!S.rot && !S.chan_scale) {
+          if (raw) {
             // x is the fp16 input itself, so x >= th <=> x >= th rounded up to fp16: count the
             // thresholds reached two values at a time in fp16 (1024 + count keeps the count in
             // the low mantissa bits)
@@ -774,9 +835,11 @@ typedef void (*RowKernel)(LayerDev, int, const __half*, int, unsigned);
 
 static int fam_of(const SideDev& s) {
   switch (s.fmt) {
-    case KVQ_FMT_INT: return s.scale_mode == KVQ_SCALE_MINMAX ? FAM_MINMAX : FAM_ABSMAX;
+    case KVQ_FMT_INT:
+      return s.scale_mode == KVQ_SCALE_MINMAX ? FAM_MINMAX : (s.scale_mode == KVQ_SCALE_SYMMETRIC ? FAM_SYM : FAM_ABSMAX);
     case KVQ_FMT_NF4: return FAM_NF4;
     case KVQ_FMT_TERNARY: return FAM_TERNARY;
+    case KVQ_FMT_LLOYD: return FAM_LLOYD;
     default: return FAM_SIGN;
   }
 }
@@ -801,6 +864,8 @@ static RowKernel pick_rows_kernel(int fam, int g) {
     case FAM_NF4: return pick_rows_g<FAM_NF4>(g);
     case FAM_TERNARY: return pick_rows_g<FAM_TERNARY>(g);
     case FAM_SIGN: return pick_rows_g<FAM_SIGN>(g);
+    case FAM_SYM: return pick_rows_g<FAM_SYM>(g);
+    case FAM_LLOYD: return pick_rows_g<FAM_LLOYD>(g);
   }
   return nullptr;
 }
@@ -808,7 +873,8 @@ static RowKernel pick_rows_kernel(int fam, int g) {
 bool append_supported(int D, const kvq_side& s) {
   if (s.format == KVQ_FMT_FP16) return true;
   if (s.format == KVQ_FMT_POLAR || s.format == KVQ_FMT_CART) return D == 128 && s.rotation == 0;
-  if (s.format != KVQ_FMT_INT && s.format != KVQ_FMT_NF4 && s.format != KVQ_FMT_TERNARY && s.format != KVQ_FMT_SIGN)
+  if (s.format != KVQ_FMT_INT && s.format != KVQ_FMT_NF4 && s.format != KVQ_FMT_TERNARY && s.format != KVQ_FMT_SIGN &&
+      s.format != KVQ_FMT_LLOYD)
     return false;
   if (D != 64 && D != 128 && D != 256) return false;
   if (s.rotation > D || (s.rotation && D % s.rotation)) return false;
@@ -836,6 +902,36 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
   }
   }
   finish_append(L, n_new, total_ctas);
+}
+
+// Key means (K with mean_sub) of the listed sequences this append starts (stored length 0): one
+// CTA per (listed sequence, kv-head).  Each fp16 key times 2^24 is an integer, so the sum is exact
+// in int64 in any order; the mean is rounded once through fp64 to fp16.  Runs before the append
+// kernels on the same stream, which then subtract it.
+constexpr int kMeanThreads = 256;
+
+__global__ void __launch_bounds__(kMeanThreads) key_mean_kernel(LayerDev L, const __half* __restrict__ k, int n_new) {
+  const int ul = blockIdx.x, sl = ul / L.Hkv, h = ul - sl * L.Hkv;
+  const int b = L.app_ids ? L.app_ids[sl] : sl;
+  if (b < 0 || b >= L.B || L.seq_len[b] != 0) return;  // not this sequence's first append
+  const int D = L.D, j = threadIdx.x % D, r0 = threadIdx.x / D, nr = kMeanThreads / D;
+  const __half* src = k + (long long)ul * n_new * D;
+  long long acc = 0;
+  for (int i = r0; i < n_new; i += nr) acc += __float2ll_rn(__fmul_rn(__half2float(src[(long long)i * D + j]), 16777216.0f));
+  __shared__ long long part[kMeanThreads];
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  if (r0 == 0) {
+    long long S = 0;
+    for (int r = 0; r < nr; ++r) S += part[r * D + j];
+    const double m = __dmul_rn(__ddiv_rn(__ll2double_rn(S), (double)n_new), 5.9604644775390625e-08);  // x 2^-24
+    L.s[0].kmean[((long long)b * L.Hkv + h) * D + j] = __double2half(m);
+  }
+}
+
+cudaError_t launch_key_mean(const LayerDev& L, const __half* k, int n_new, cudaStream_t st) {
+  key_mean_kernel<<<L.app_n * L.Hkv, kMeanThreads, 0, st>>>(L, k, n_new);
+  return cudaGetLastError();
 }
 
 // Grid cap of the grid-stride append kernels (148 SMs x 8 CTAs of 8 warps).

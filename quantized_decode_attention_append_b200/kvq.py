@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkvq.so")
 
 # enums (values fixed by include/kvq.h)
-FMT = {"fp16": 0, "int": 1, "nf4": 2, "ternary": 3, "sign": 4, "polar": 5, "cart": 6}
-SCALE = {"absmax": 0, "minmax": 1}
+FMT = {"fp16": 0, "int": 1, "nf4": 2, "ternary": 3, "sign": 4, "polar": 5, "cart": 6, "lloyd": 7}
+SCALE = {"absmax": 0, "minmax": 1, "sym": 2}
 ANCHOR = {"none": 0, "first_n": 1, "window": 2, "all": 3}
 SIDE_K, SIDE_V = 0, 1
 DOMAIN_STORED, DOMAIN_ORIGINAL = 0, 1
@@ -27,7 +27,7 @@ STATUS = {0: "KVQ_OK", -1: "KVQ_ERR_INVALID_ARG", -2: "KVQ_ERR_UNSUPPORTED", -3:
 
 class kvq_side(C.Structure):
     _fields_ = [("format", C.c_int32), ("bits", C.c_int32), ("bits2", C.c_int32), ("scale_mode", C.c_int32),
-                ("group", C.c_int32), ("rotation", C.c_int32), ("chan_scale", C.c_int32)]
+                ("group", C.c_int32), ("rotation", C.c_int32), ("chan_scale", C.c_int32), ("mean_sub", C.c_int32)]
 
 
 class kvq_config(C.Structure):
@@ -39,13 +39,13 @@ class kvq_config(C.Structure):
 
 class kvq_layout(C.Structure):
     _fields_ = [("codes", C.c_int64), ("scales", C.c_int64), ("zeros", C.c_int64), ("anchors", C.c_int64),
-                ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("row_bytes", C.c_int32),
+                ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("key_mean", C.c_int64), ("row_bytes", C.c_int32),
                 ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32)]
 
 
 EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_arena_bytes_layers", "kvq_create_layers", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
            "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_decode_attention_noalloc",
-           "kvq_error_flags", "kvq_nf4_levels",
+           "kvq_error_flags", "kvq_nf4_levels", "kvq_lloyd_levels",
            "kvq_last_launch_count", "kvq_status_str"]
 
 _LIB = None
@@ -75,6 +75,7 @@ def lib() -> C.CDLL:
         L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
         L.kvq_error_flags.argtypes = [vp, C.POINTER(i32)]
         L.kvq_nf4_levels.argtypes = [C.POINTER(C.c_float)]
+        L.kvq_lloyd_levels.argtypes = [i32, C.POINTER(C.c_float)]
         L.kvq_last_launch_count.argtypes = [vp]
         L.kvq_last_launch_count.restype = i32
         L.kvq_status_str.argtypes = [i32]
@@ -118,10 +119,11 @@ class Side:
     group: int = 32
     rot: int = 0
     chan_scale: bool = False
+    mean_sub: bool = False
 
     def to_c(self) -> kvq_side:
         return kvq_side(FMT[self.fmt], self.bits, self.bits2, SCALE[self.scale], self.group, self.rot,
-                        1 if self.chan_scale else 0)
+                        1 if self.chan_scale else 0, 1 if self.mean_sub else 0)
 
 
 @dataclass
@@ -249,6 +251,12 @@ def kvq_nf4_levels() -> list:
     return list(arr)
 
 
+def kvq_lloyd_levels(bits: int) -> list:
+    arr = (C.c_float * (1 << bits))()
+    _check(lib().kvq_lloyd_levels(bits, arr), "kvq_lloyd_levels")
+    return list(arr)
+
+
 def kvq_last_launch_count(h) -> int:
     return lib().kvq_last_launch_count(h)
 
@@ -302,6 +310,11 @@ class KVCache:
             return self.arena[lo.anchors:lo.anchors + n].view(torch.float16).view(U, lo.anchor_rows, self.cfg.head_dim)
         if what == "seq_len":
             return self.arena[lo.seq_len:lo.seq_len + 4 * self.cfg.batch].view(torch.int32)
+        if what == "key_mean":
+            if lo.key_mean < 0:
+                return None
+            n = U * self.cfg.head_dim * 2
+            return self.arena[lo.key_mean:lo.key_mean + n].view(torch.float16).view(U, self.cfg.head_dim)
         raise ValueError(what)
 
     def set_chan_scale(self, layer, c16, stream=None):

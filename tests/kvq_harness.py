@@ -37,6 +37,7 @@ class Case:
         self.cache = KVCache(cfg)
         self.K, self.V, self.C = {}, {}, {}
         B, H, D = cfg.batch, cfg.n_kv_heads, cfg.head_dim
+        self.first_rows = (chunks or [T])[0]  # rows of each sequence's first append (the key mean's rows)
         layers = range(cfg.n_layers) if layers is None else layers
         for l in layers:
             if inputs is None:
@@ -62,7 +63,7 @@ class Case:
 
     def oracle_unit(self, l, b, h):
         c = self.C[l][h] if l in self.C else None
-        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c, layer=l)
+        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c, layer=l, first_rows=self.first_rows)
 
     def check_codes(self, l, rows=None):
         """Packed codes, scales and zero points of every unit are bit-identical to the oracle."""
@@ -73,6 +74,8 @@ class Case:
             zeros = self.cache.view(l, side, "zeros")
             scales = None if scales is None else scales.cpu().numpy()
             zeros = None if zeros is None else zeros.cpu().numpy()
+            kmean = self.cache.view(l, 0, "key_mean")
+            kmean = None if kmean is None else kmean.cpu().numpy()
             for b in range(cfg.batch):
                 for h in range(cfg.n_kv_heads):
                     u = b * cfg.n_kv_heads + h
@@ -92,6 +95,8 @@ class Case:
                     if zeros is not None:
                         assert np.array_equal(zeros[u, :self.T][sel].view(np.uint16),
                                               o["zeros"][sel].view(np.uint16)), f"{name} zeros l{l} u{u}"
+                    if side == 0 and kmean is not None:
+                        assert np.array_equal(kmean[u].view(np.uint16), o["mu"].view(np.uint16)), f"key mean l{l} u{u}"
 
     def check_dequant(self, l):
         """Stored domain bit-exact; original domain within fp32 transform error."""
@@ -107,7 +112,9 @@ class Case:
                         f"stored dequant side {side} l{l} b{b} h{h}"
                     sd = OC.side_of(self.spec, l, side == 0)
                     c = self.C[l][h] if (side == 0 and l in self.C) else None
-                    want = OQ.to_original_f64(o["exact"], sd, None if c is None else np.broadcast_to(c, o["exact"].shape))
+                    mu = o.get("mu")
+                    want = OQ.to_original_f64(o["exact"], sd, None if c is None else np.broadcast_to(c, o["exact"].shape),
+                                              None if mu is None else np.broadcast_to(mu, o["exact"].shape))
                     an = OC.anchored(self.spec, l, np.arange(self.T), self.T)
                     src = self.K[l] if side == 0 else self.V[l]
                     want[an] = src[b, h][an].astype(np.float64)

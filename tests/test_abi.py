@@ -183,3 +183,43 @@ def test_header_documents_the_sequence_list():
     decl = text[text.index("kvq_status kvq_quantize_append("):]
     decl = decl[:decl.index(";")]
     assert "const int32_t* seq_ids" in decl and "int32_t n_seqs" in decl and "int32_t n_new" in decl
+
+
+def test_library_lloyd_tables_equal_oracle_tables():
+    """The library iterates Lloyd's conditions in C++ and the oracle in numpy; the fp16 levels
+    must agree bit for bit ("E22L" "Result": Gaussian Lloyd-Max levels)."""
+    from oracle import lloyd as OL
+    for b in (2, 3, 4):
+        assert np.array_equal(np.array(kvq.kvq_lloyd_levels(b), dtype=np.float64), OL.lloyd_max_levels(b))
+    assert kvq.lib().kvq_lloyd_levels(5, (C.c_float * 32)()) == -1
+
+
+@pytest.mark.parametrize("mut,want", [
+    (dict(v=Side("int", 4, group=32, mean_sub=True)), -1),          # values carry no key mean
+    (dict(k=Side("fp16", mean_sub=True)), -1),                     # nothing to subtract it from
+    (dict(k=Side("lloyd", 5, group=32)), -1),
+    (dict(k=Side("lloyd", 1, group=32)), -1),
+    (dict(k=Side("lloyd", 3, scale="minmax", group=32)), -1),
+    (dict(k=Side("nf4", scale="sym", group=64)), -1),
+])
+def test_bad_value_grid_configs(mut, want):
+    assert status_of(base_cfg(**mut))[0] == want
+
+
+@pytest.mark.parametrize("side", [
+    Side("int", 2, scale="sym", group=128, rot=128), Side("int", 3, scale="sym", group=32),
+    Side("lloyd", 2, group=128, rot=128), Side("lloyd", 4, group=16), Side("int", 4, group=32, mean_sub=True),
+])
+def test_value_grid_configs_accepted(side):
+    v = Side(**{**side.__dict__, "mean_sub": False})
+    st, n = status_of(base_cfg(k=side, v=v))
+    assert st == 0 and n > 0
+
+
+def test_key_mean_region_in_the_arena():
+    """A K side with mean_sub adds one fp16 vector per (sequence, kv-head) and layer."""
+    st0, n0 = status_of(base_cfg())
+    st1, n1 = status_of(base_cfg(k=Side("int", 4, group=32, rot=128, mean_sub=True)))
+    assert st0 == 0 and st1 == 0
+    per_layer = 2 * 2 * 128 * 2  # batch x kv-heads x head_dim x fp16
+    assert n1 - n0 == 2 * ((per_layer + 255) // 256 * 256)
