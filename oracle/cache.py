@@ -16,6 +16,12 @@ of 128, under a 3.2-bit average; "Result": 2-bit K in layers 2 and 7, 4-bit V in
 and 4, 3 bits elsewhere, 3.19 bits on average).  A Spec may give one Side per layer for K and for
 V; layers are numbered from 0 (the same result calls layer 7 the last of the 8).
 
+Anchor precision (post 6, "The winning recipe" item 4, the anchor-precision dial: fp16, int8
+or int4 anchors; "Best results" rows "ternboth_a8" and "signboth_a8" use int8 anchors).  Reading
+taken here: an int8 or int4 anchor row is the original fp16 row on the same signed absmax grid as
+the int format (largest-magnitude element at -2^(b-1), first index on ties), in groups of 32
+channels with one fp16 scale each, no pre-transform; attention reads its dequantized values.
+
 Key mean subtraction (llama.cpp #21385, the later comment on a per-head shared key mean that
 carries about half of the key energy: the running mean is subtracted before quantization and
 restored after).  Reading taken here: the mean of one (layer, sequence, kv-head) is the running
@@ -59,6 +65,7 @@ class Spec:
     sm_scale: float | None = None
     layer_k: tuple = ()  # one Side per layer, or empty: k on every layer
     layer_v: tuple = ()
+    anchor_bits: int = 16  # 16 (fp16 rows), 8 or 4 (signed absmax grid, groups of 32)
 
 
 def side_of(spec: Spec, layer: int, is_k: bool) -> Side:
@@ -77,6 +84,19 @@ def anchored(spec: Spec, layer: int, tokens: np.ndarray, seq_len: int) -> np.nda
     if spec.anchor_rule == "all":
         return t < seq_len
     raise ValueError(spec.anchor_rule)
+
+
+def anchor_side(spec: Spec) -> Side:
+    return Side("int", spec.anchor_bits, group=32)
+
+
+def anchor_rows(spec: Spec, X16: np.ndarray) -> dict:
+    """The stored anchor form of fp16 rows X16 [n, D]: for int anchors the quantize_rows dict of
+    the anchor grid, for fp16 anchors the rows themselves (as 'exact')."""
+    X16 = np.asarray(X16, dtype=np.float16)
+    if spec.anchor_bits == 16:
+        return {"exact": X16.astype(F64)}
+    return quantize_rows(X16, anchor_side(spec))
 
 
 def key_mean(K16: np.ndarray) -> np.ndarray:
@@ -107,8 +127,9 @@ def reconstruct_unit(spec: Spec, layer: int, K16, V16, kq, vq, seq_len: int, c16
                          None if mu is None else np.broadcast_to(mu, K16.shape))
     Vh = to_original_f64(vq["exact"], side_of(spec, layer, False), None)
     an = anchored(spec, layer, np.arange(T), seq_len)
-    Kh[an] = np.asarray(K16, dtype=np.float16)[an].astype(np.float64)
-    Vh[an] = np.asarray(V16, dtype=np.float16)[an].astype(np.float64)
+    if an.any():
+        Kh[an] = anchor_rows(spec, np.asarray(K16)[an])["exact"]
+        Vh[an] = anchor_rows(spec, np.asarray(V16)[an])["exact"]
     return Kh, Vh
 
 
@@ -123,9 +144,10 @@ def effective_bits(spec: Spec, seq_len: int) -> float:
     tot = 0.0
     for layer in range(spec.n_layers):
         an = anchored(spec, layer, np.arange(seq_len), seq_len).sum()
+        a_row = 16 * D if spec.anchor_bits == 16 else bits_per_value(anchor_side(spec), D) * D
         for side, is_k in ((side_of(spec, layer, True), True), (side_of(spec, layer, False), False)):
             per_row = bits_per_value(side, D) * D
-            bits = (seq_len - an) * per_row + an * 16 * D
+            bits = (seq_len - an) * per_row + an * a_row
             if is_k and side.chan_scale:
                 bits += 16 * D
             if is_k and side.mean_sub:

@@ -734,3 +734,35 @@ def test_key_mean_subtraction_restores_and_helps():
     # bits: one fp16 mean vector per (sequence, kv-head), like a channel-scale vector
     s = C.Spec(1, 1, 1, 1, D, k_sub, v)
     assert C.effective_bits(s, 1000) == pytest.approx((Q.bits_per_value(k_sub, D) + 16 / 1000 + Q.bits_per_value(v, D)) / 2)
+
+
+@pytest.mark.parametrize("abits", [8, 4])
+def test_int_anchor_rows(abits):
+    """Post 6, "The winning recipe" item 4 (the anchor-precision dial, fp16 -> int8 -> int4): an
+    anchored row is attended as the original row on a b-bit grid in groups of 32 (one fp16 scale
+    each), within that grid's error bound, far closer than the ternary rows around it, and the
+    effective bits count b + 16/32 per anchored value."""
+    r = rng(70 + abits)
+    n_tok, D = 100, 128
+    side = Side("ternary", group=8)
+    K16 = (r.standard_normal((n_tok, D)) * 2).astype(np.float16)
+    V16 = (r.standard_normal((n_tok, D)) * 3).astype(np.float16)
+    spec = C.Spec(1, 1, 1, 1, D, side, side, frozenset({0}), "first_n", 30, anchor_bits=abits)
+    kq, vq = C.quantize_unit(spec, K16, V16)
+    Kh, Vh = C.reconstruct_unit(spec, 0, K16, V16, kq, vq, n_tok)
+    for Xh, X16 in ((Kh, K16), (Vh, V16)):
+        x = X16.astype(np.float64)
+        a, rest = x[:30], x[30:]
+        g = a.reshape(30, D // 32, 32)
+        d = np.abs(g).max(axis=-1, keepdims=True) / 2 ** (abits - 1)    # |d| before fp16 rounding
+        err = np.abs(Xh[:30].reshape(30, D // 32, 32) - g)
+        assert (err <= d * (1 + 2 ** -10) + 1e-12).all()
+        assert (Xh[:30] != x[:30]).any()                                   # not the fp16 row itself
+        assert A.rel_sq_error(a, Xh[:30]) < 0.1 * A.rel_sq_error(rest, Xh[30:])
+        # the grid's level set: code values x / d are integers in [-2^(b-1), 2^(b-1) - 1]
+        dd = np.repeat(Q.quantize_rows(X16[:30], Side("int", abits, group=32))["scales"].astype(np.float64), 32, axis=1)
+        lv = Xh[:30] / np.where(dd == 0, 1, dd)
+        assert np.allclose(lv, np.round(lv)) and lv.min() >= -(2 ** (abits - 1)) and lv.max() <= 2 ** (abits - 1) - 1
+    eb = C.effective_bits(spec, n_tok)
+    base = Q.bits_per_value(side, D)
+    assert eb == pytest.approx((70 * base + 30 * (abits + 16 / 32)) / n_tok)
