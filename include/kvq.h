@@ -107,6 +107,12 @@ typedef struct {
   int32_t anchor_rule;         /* KVQ_ANCHOR_*; [FMKQ] post 6 "Corrected semantics" */
   int32_t anchor_n;            /* FIRST_N: tokens t < n; WINDOW: the last n tokens */
   float sm_scale;              /* softmax scale; 0 selects 1/sqrt(head_dim) */
+  int32_t anchor_bits;         /* anchor precision ([FMKQ] post 6 "The winning recipe" item 4, the
+                                  anchor-precision dial): 16 (or 0) keeps anchored rows as fp16;
+                                  8 or 4 stores them on the signed absmax grid (largest magnitude at
+                                  -2^(b-1)) in groups of 32 channels with an fp16 scale each, in the
+                                  original domain.  8/4 need row formats (INT, NF4, TERNARY, SIGN,
+                                  LLOYD) on both sides of anchored layers. */
 } kvq_config;
 
 /* Byte offsets (into the arena) and geometry of one (layer, side).  Rows of one
@@ -118,6 +124,8 @@ typedef struct {
 typedef struct {
   int64_t codes, scales, zeros, anchors, chan_scale, seq_len;
   int64_t key_mean;  /* K with mean_sub: fp16 [batch * n_kv_heads][head_dim], unit u at u * head_dim */
+  int64_t anchor_scales;  /* int anchors: fp16 [units][anchor_rows][head_dim / 32]; anchor rows then hold
+                             head_dim * anchor_bits / 8 code bytes each (LSB-first) instead of fp16 */
   int32_t row_bytes, n_groups, row_stride_tokens, anchor_rows;
 } kvq_layout;
 

@@ -245,10 +245,9 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0f;
       if (anchor_split) {
-        const __half* kr = K.anchors ? K.anchors + (u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t)) * D
-                                     : reinterpret_cast<const __half*>(K.codes + (u * L.Tcap + t) * K.row_bytes);
+        const long long arow = u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t);
         for (int j = 0; j < D; ++j) {
-          const float kv = __half2float(kr[j]);
+          const float kv = anchor_value(L, K, arow, j);
 #pragma unroll
           for (int h = 0; h < kMaxG; ++h)
             if (h < G) acc[h] += qa[h * D + j] * kv;
@@ -332,9 +331,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(LayerDev L,
           const int j = ch0 + c * kGenThreads;
           float vv;
           if (anchor_split) {
-            const __half* vr = V.anchors ? V.anchors + (u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t)) * D
-                                         : reinterpret_cast<const __half*>(V.codes + (u * L.Tcap + t) * V.row_bytes);
-            vv = __half2float(vr[j]);
+            vv = anchor_value(L, V, u * L.anchor_rows + (L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t), j);
           } else {
             const uint8_t* row = V.codes + (u * L.Tcap + t) * V.row_bytes;
             const __half* sc = V.scales + (u * L.Tcap + t) * V.n_groups;

@@ -67,6 +67,15 @@ __device__ __forceinline__ float stored_value(const SideDev& S, const uint8_t* _
   return 0.0f;
 }
 
+// Value j of anchor row `arow` (= unit x anchor_rows + slot) of a side, original domain: the fp16
+// row, or an int8/int4 anchor's code times its group-of-32 scale.
+__device__ __forceinline__ float anchor_value(const LayerDev& L, const SideDev& S, long long arow, int j) {
+  if (L.anchor_bits == 16) return __half2float(S.anchors[arow * L.D + j]);
+  const uint8_t* row = reinterpret_cast<const uint8_t*>(S.anchors) + arow * L.anchor_rb;
+  const float d = __half2float(S.anchor_scales[arow * (L.D / 32) + j / 32]);
+  return (float)((int)get_bits(row, j * L.anchor_bits, L.anchor_bits) - (1 << (L.anchor_bits - 1))) * d;
+}
+
 // Polar slot f of a row: (m cos phi, m sin phi); cs/sn: cos/sin tables for the row's phase bits.
 __device__ __forceinline__ float2 polar_slot(const SideDev& S, const uint8_t* __restrict__ row,
                                              const __half* __restrict__ sc, int f, const float* cs,

@@ -108,8 +108,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(LayerDev L, int side, int 
     }
     if (anc) {
       const int slot = L.anchor_rule == KVQ_ANCHOR_WINDOW ? t % L.anchor_n : t;
-      const __half* ar = S.anchors + (u * L.anchor_rows + slot) * D;
-      for (int j = lane; j < D; j += 32) x[j] = __half2float(ar[j]);
+      for (int j = lane; j < D; j += 32) x[j] = anchor_value(L, S, u * L.anchor_rows + slot, j);
     }
     __syncwarp();
   }

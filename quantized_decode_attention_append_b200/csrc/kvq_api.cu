@@ -19,7 +19,7 @@ struct kvq_cache {
   char* arena;
   uint64_t arena_bytes;
   struct SideOff {
-    int64_t codes, scales, zeros, anchors;
+    int64_t codes, scales, zeros, anchors, anchor_scales;
     int row_bytes, n_groups;
   } off[64][2];
   int64_t chan[64];
@@ -124,8 +124,22 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
   if (c->anchor_rule == KVQ_ANCHOR_FIRST_N || c->anchor_rule == KVQ_ANCHOR_WINDOW) {
     if (c->anchor_n < 1 || c->anchor_n > c->capacity) return KVQ_ERR_INVALID_ARG;
   }
+  if (c->anchor_bits != 0 && c->anchor_bits != 16 && c->anchor_bits != 8 && c->anchor_bits != 4)
+    return KVQ_ERR_INVALID_ARG;
+  if (c->anchor_bits == 8 || c->anchor_bits == 4) {  // anchors are quantized by the row kernels
+    for (int l = 0; l < c->n_layers; ++l) {
+      if (c->anchor_rule == KVQ_ANCHOR_NONE || !((c->anchor_layer_mask >> l) & 1ULL)) continue;
+      for (int sd = 0; sd < 2; ++sd) {
+        const kvq_side& x = sd == 0 ? (lk ? lk[l] : c->k) : (lv ? lv[l] : c->v);
+        if (x.format == KVQ_FMT_FP16 || x.format == KVQ_FMT_POLAR || x.format == KVQ_FMT_CART)
+          return KVQ_ERR_UNSUPPORTED;
+      }
+    }
+  }
   return KVQ_OK;
 }
+
+int anchor_bits_of(const kvq_config& c) { return (c.anchor_bits == 8 || c.anchor_bits == 4) ? c.anchor_bits : 16; }
 
 void side_geometry(int D, const kvq_side& s, int* row_bytes, int* n_groups) {
   switch (s.format) {
@@ -174,9 +188,15 @@ uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
         off = align_up(off + units * Tcap * (uint64_t)ng * 2);
       }
       so.anchors = -1;
+      so.anchor_scales = -1;
       if (layer_anchored(c, l)) {
+        const int ab = anchor_bits_of(c);
         so.anchors = (int64_t)off;
-        off = align_up(off + units * (uint64_t)anchor_rows * D * 2);
+        off = align_up(off + units * (uint64_t)anchor_rows * D * ab / 8);
+        if (ab != 16) {
+          so.anchor_scales = (int64_t)off;
+          off = align_up(off + units * (uint64_t)anchor_rows * (D / 32) * 2);
+        }
       }
       if (h) h->off[l][s] = so;
     }
@@ -220,6 +240,7 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
     S.scales = so.scales >= 0 ? reinterpret_cast<__half*>(h->arena + so.scales) : nullptr;
     S.zeros = so.zeros >= 0 ? reinterpret_cast<__half*>(h->arena + so.zeros) : nullptr;
     S.anchors = so.anchors >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchors) : nullptr;
+    S.anchor_scales = so.anchor_scales >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchor_scales) : nullptr;
     S.chan = (s == 0 && h->chan[l] >= 0) ? reinterpret_cast<const __half*>(h->arena + h->chan[l]) : nullptr;
     S.kmean = (s == 0 && h->kmean[l] >= 0) ? reinterpret_cast<__half*>(h->arena + h->kmean[l]) : nullptr;
     S.mean_sub = s == 0 ? sd.mean_sub : 0;
@@ -246,6 +267,8 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
   L.anchor_rule = c.anchor_rule;
   L.anchor_n = c.anchor_n;
   L.anchor_rows = h->anchor_rows;
+  L.anchor_bits = anchor_bits_of(c);
+  L.anchor_rb = c.head_dim * L.anchor_bits / 8;
   L.seq_len = reinterpret_cast<int*>(h->arena + h->lens) + (size_t)l * c.batch;
   L.ticket = reinterpret_cast<unsigned*>(h->arena + h->tickets) + l;
   L.err = reinterpret_cast<unsigned*>(h->arena + h->err);
@@ -481,6 +504,7 @@ kvq_status kvq_get_layout(const kvq_cache* h, int32_t layer, int32_t side, kvq_l
   out->anchors = so.anchors;
   out->chan_scale = side == 0 ? h->chan[layer] : -1;
   out->key_mean = side == 0 ? h->kmean[layer] : -1;
+  out->anchor_scales = so.anchor_scales;
   out->seq_len = h->lens + (int64_t)layer * h->cfg.batch * 4;
   out->row_bytes = so.row_bytes;
   out->n_groups = so.n_groups;

@@ -17,7 +17,8 @@ struct SideDev {
   uint8_t* codes;        // [B*Hkv][Tcap][row_bytes]
   __half* scales;        // [B*Hkv][Tcap][n_groups]
   __half* zeros;         // [B*Hkv][Tcap][n_groups] (MINMAX) or null
-  __half* anchors;       // [B*Hkv][anchor_rows][D] or null
+  __half* anchors;       // [B*Hkv][anchor_rows][D] fp16, or [..][anchor_rb] codes (int anchors), or null
+  __half* anchor_scales; // int anchors: [B*Hkv][anchor_rows][D/32] or null
   const __half* chan;    // [Hkv][D] (K with chan_scale) or null
   __half* kmean;         // [B*Hkv][D] key means (K with mean_sub) or null
   int fmt, bits, bits2, scale_mode, group, rot, chan_scale, mean_sub;
@@ -31,6 +32,7 @@ struct LayerDev {
   int cap;               // configured capacity (tokens per sequence); appends never pass it
   int anchored;          // this layer keeps anchor rows
   int anchor_rule, anchor_n, anchor_rows;
+  int anchor_bits, anchor_rb;  // 16 (fp16 rows) or 8/4 (code bytes per anchor row: anchor_rb)
   int* seq_len;          // [B] stored lengths of this layer
   unsigned* ticket;      // append completion counter of this layer
   unsigned* err;         // error word (KVQ_ERRF_*)

@@ -411,6 +411,40 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const float* th) {
   return (b3 ? 8u : 0u) + (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (b0 ? 1u : 0u);
 }
 
+// An int8/int4 anchor row's group `li` (channels 32 li .. 32 li + 31, the lane's own slice): the
+// signed absmax grid of the int format on the raw fp16 values (largest magnitude, first on ties,
+// at -2^(b-1)), one fp16 scale.  Anchored rows are rare, so this stays out of the main path.
+__device__ __noinline__ void anchor_quant32(const LayerDev& L, const SideDev& S, long long arow, int li,
+                                            const __half2* raw2) {
+  const int b = L.anchor_bits, half = 1 << (b - 1);
+  float x[32];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float2 f = __half22float2(raw2[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+  float best = -1.0f, m = 0.0f;
+#pragma unroll
+  for (int v = 0; v < 32; ++v)
+    if (fabsf(x[v]) > best) {
+      best = fabsf(x[v]);
+      m = x[v];
+    }
+  const __half sh = __float2half_rn(__fmul_rn(m, -1.0f / (float)half));
+  const float d = __half2float(sh), inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+  uint32_t code[32];
+#pragma unroll
+  for (int v = 0; v < 32; ++v) {
+    const float k = d != 0.0f ? fminf(fmaxf(round_exact_absmax(x[v], d, inv), (float)(-half)), (float)(half - 1)) : 0.0f;
+    code[v] = (uint32_t)((int)k + half);
+  }
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(S.anchors) + arow * L.anchor_rb) + li * b;
+  if (b == 8) pack32<8>(code, out, true);
+  else pack32<4>(code, out, true);
+  S.anchor_scales[arow * (L.D / 32) + li] = sh;
+}
+
 // Rows of one side over blocks bid = 0 .. nblk - 1 (grid-stride).
 template <int FAM, int G, int BITS = 0>
 __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __half* __restrict__ src, int n_new,
@@ -482,9 +516,14 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
         }
       }
       if (in_anchor(L, pos, len_after)) {
-        __half* ap = S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, pos)) * D + li * 32;
+        const long long arow = (long long)u * L.anchor_rows + anchor_slot(L, pos);
+        if (L.anchor_bits == 16) {
+          __half* ap = S.anchors + arow * D + li * 32;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
+          for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
+        } else {
+          anchor_quant32(L, S, arow, li, raw2);
+        }
       }
       if (S.mean_sub) {
         const __half* mp = S.kmean + (long long)u * D + li * 32;

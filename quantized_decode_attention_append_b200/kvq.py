@@ -34,12 +34,13 @@ class kvq_config(C.Structure):
     _fields_ = [("n_layers", C.c_int32), ("batch", C.c_int32), ("n_kv_heads", C.c_int32), ("n_q_heads", C.c_int32),
                 ("head_dim", C.c_int32), ("capacity", C.c_int32), ("max_queries", C.c_int32),
                 ("k", kvq_side), ("v", kvq_side), ("anchor_layer_mask", C.c_uint64), ("anchor_rule", C.c_int32),
-                ("anchor_n", C.c_int32), ("sm_scale", C.c_float)]
+                ("anchor_n", C.c_int32), ("sm_scale", C.c_float), ("anchor_bits", C.c_int32)]
 
 
 class kvq_layout(C.Structure):
     _fields_ = [("codes", C.c_int64), ("scales", C.c_int64), ("zeros", C.c_int64), ("anchors", C.c_int64),
-                ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("key_mean", C.c_int64), ("row_bytes", C.c_int32),
+                ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("key_mean", C.c_int64), ("anchor_scales", C.c_int64),
+                ("row_bytes", C.c_int32),
                 ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32)]
 
 
@@ -143,6 +144,7 @@ class Config:
     sm_scale: float = 0.0
     layer_k: tuple = ()  # per-layer K formats (n_layers Sides); empty: k on every layer
     layer_v: tuple = ()  # per-layer V formats; empty: v on every layer
+    anchor_bits: int = 16  # anchored rows as fp16 (16) or on an 8/4-bit grid in groups of 32
 
     def side(self, layer: int, side: int) -> Side:
         """Format of (layer, side)."""
@@ -164,7 +166,7 @@ class Config:
             mask |= 1 << int(l)
         return kvq_config(self.n_layers, self.batch, self.n_kv_heads, self.n_q_heads, self.head_dim, self.capacity,
                           self.max_queries or self.batch, self.k.to_c(), self.v.to_c(), mask, ANCHOR[self.anchor_rule],
-                          self.anchor_n, self.sm_scale)
+                          self.anchor_n, self.sm_scale, self.anchor_bits)
 
 
 # ----------------------------------------------------------------------------- C-ABI calls
@@ -303,11 +305,21 @@ class KVCache:
                 return None
             n = U * T * lo.n_groups * 2
             return self.arena[o:o + n].view(torch.float16).view(U, T, lo.n_groups)
-        if what == "anchors":
+        if what == "anchors":  # fp16 rows, or code bytes for int anchors
             if lo.anchors < 0:
                 return None
-            n = U * lo.anchor_rows * self.cfg.head_dim * 2
-            return self.arena[lo.anchors:lo.anchors + n].view(torch.float16).view(U, lo.anchor_rows, self.cfg.head_dim)
+            D, ab = self.cfg.head_dim, self.cfg.anchor_bits
+            if ab == 16:
+                n = U * lo.anchor_rows * D * 2
+                return self.arena[lo.anchors:lo.anchors + n].view(torch.float16).view(U, lo.anchor_rows, D)
+            n = U * lo.anchor_rows * D * ab // 8
+            return self.arena[lo.anchors:lo.anchors + n].view(U, lo.anchor_rows, D * ab // 8)
+        if what == "anchor_scales":
+            if lo.anchor_scales < 0:
+                return None
+            n = U * lo.anchor_rows * (self.cfg.head_dim // 32) * 2
+            return self.arena[lo.anchor_scales:lo.anchor_scales + n].view(torch.float16).view(
+                U, lo.anchor_rows, self.cfg.head_dim // 32)
         if what == "seq_len":
             return self.arena[lo.seq_len:lo.seq_len + 4 * self.cfg.batch].view(torch.int32)
         if what == "key_mean":

@@ -23,7 +23,7 @@ def oracle_spec(cfg: Config) -> OC.Spec:
     return OC.Spec(cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.n_q_heads, cfg.head_dim, oracle_side(cfg.k),
                    oracle_side(cfg.v), frozenset(cfg.anchor_layers), cfg.anchor_rule, cfg.anchor_n,
                    cfg.sm_scale or None, tuple(oracle_side(s) for s in cfg.layer_k),
-                   tuple(oracle_side(s) for s in cfg.layer_v))
+                   tuple(oracle_side(s) for s in cfg.layer_v), anchor_bits=cfg.anchor_bits)
 
 
 class Case:
@@ -98,6 +98,28 @@ class Case:
                     if side == 0 and kmean is not None:
                         assert np.array_equal(kmean[u].view(np.uint16), o["mu"].view(np.uint16)), f"key mean l{l} u{u}"
 
+    def check_anchors(self, l):
+        """Stored anchor rows of every unit equal the oracle's: fp16 rows, or int codes and scales."""
+        cfg = self.cfg
+        an = OC.anchored(self.spec, l, np.arange(self.T), self.T)
+        if not an.any():
+            return
+        slots = np.arange(self.T)[an] % cfg.anchor_n if cfg.anchor_rule == "window" else np.arange(self.T)[an]
+        for side in (0, 1):
+            codes = self.cache.view(l, side, "anchors").cpu().numpy()
+            sc = self.cache.view(l, side, "anchor_scales")
+            for b in range(cfg.batch):
+                for h in range(cfg.n_kv_heads):
+                    u = b * cfg.n_kv_heads + h
+                    src = (self.K[l] if side == 0 else self.V[l])[b, h][an]
+                    want = OC.anchor_rows(self.spec, src)
+                    if cfg.anchor_bits == 16:
+                        assert np.array_equal(codes[u, slots].view(np.uint16), src.view(np.uint16))
+                    else:
+                        assert np.array_equal(codes[u, slots], want["bytes"]), f"anchor codes side {side} u{u}"
+                        assert np.array_equal(sc[u, slots].cpu().numpy().view(np.uint16),
+                                              want["scales"].view(np.uint16)), f"anchor scales side {side} u{u}"
+
     def check_dequant(self, l):
         """Stored domain bit-exact; original domain within fp32 transform error."""
         cfg = self.cfg
@@ -117,7 +139,8 @@ class Case:
                                               None if mu is None else np.broadcast_to(mu, o["exact"].shape))
                     an = OC.anchored(self.spec, l, np.arange(self.T), self.T)
                     src = self.K[l] if side == 0 else self.V[l]
-                    want[an] = src[b, h][an].astype(np.float64)
+                    if an.any():
+                        want[an] = OC.anchor_rows(self.spec, src[b, h][an])["exact"]
                     scale = np.abs(want).max()
                     assert np.abs(org[b, h] - want).max() <= 1e-5 * scale, f"orig dequant side {side} l{l}"
 

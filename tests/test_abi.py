@@ -223,3 +223,24 @@ def test_key_mean_region_in_the_arena():
     assert st0 == 0 and st1 == 0
     per_layer = 2 * 2 * 128 * 2  # batch x kv-heads x head_dim x fp16
     assert n1 - n0 == 2 * ((per_layer + 255) // 256 * 256)
+
+
+@pytest.mark.parametrize("mut,want", [
+    (dict(anchor_layers=(0,), anchor_rule="first_n", anchor_n=8, anchor_bits=5), -1),
+    (dict(anchor_layers=(0,), anchor_rule="first_n", anchor_n=8, anchor_bits=8, v=Side("fp16")), -2),
+    (dict(anchor_layers=(1,), anchor_rule="window", anchor_n=8, anchor_bits=4, k=Side("polar", 4, 8)), -2),
+    (dict(anchor_layers=(0,), anchor_rule="first_n", anchor_n=8, anchor_bits=8), 0),
+    (dict(anchor_bits=8, v=Side("fp16")), 0),  # no anchored layer: nothing to quantize
+])
+def test_anchor_precision_configs(mut, want):
+    assert status_of(base_cfg(**mut))[0] == want
+
+
+def test_int_anchor_arena_is_smaller():
+    """int8 anchors take half a byte per value plus one fp16 scale per 32 channels, against 2 bytes."""
+    kw = dict(anchor_layers=(0, 1), anchor_rule="first_n", anchor_n=256)
+    n16 = status_of(base_cfg(**kw))[1]
+    n8 = status_of(base_cfg(anchor_bits=8, **kw))[1]
+    n4 = status_of(base_cfg(anchor_bits=4, **kw))[1]
+    assert n16 > n8 > n4
+    assert n16 - n8 == pytest.approx(2 * 2 * 4 * 256 * (128 * 2 - 128 - 8), abs=4 * 512)

@@ -118,3 +118,31 @@ def test_key_mean_is_recomputed_after_an_emptied_cache():
         want = OC.key_mean(K2[1, h])
         assert np.array_equal(now[2 + h].numpy().view(np.uint16), want.view(np.uint16))
     assert kvq.kvq_error_flags(c.cache.h) == 0
+
+
+ANCHOR_CASES = [
+    (128, 4, Side("ternary", group=8), Side("ternary", group=8), "first_n", 48, 8),   # "ternboth_a8"
+    (128, 4, Side("sign", group=4), Side("sign", group=4), "first_n", 48, 8),         # "signboth_a8"
+    (128, 4, Side("nf4", group=64), Side("int", 4, group=64), "window", 64, 4),
+    (256, 2, Side("int", 4, group=128, rot=256, mean_sub=True), Side("lloyd", 2, group=128, rot=256), "all", 0, 8),
+    (64, 2, Side("int", 3, scale="sym", group=16), Side("int", 4, scale="minmax", group=32), "first_n", 20, 4),
+]
+
+
+@pytest.mark.parametrize("D,G,k,v,rule,n,abits", ANCHOR_CASES,
+                         ids=[f"{d}-{k.fmt}-{v.fmt}-{r}{n}-a{a}" for d, g, k, v, r, n, a in ANCHOR_CASES])
+@pytest.mark.parametrize("chunks", [None, [130, 1, 1, 1, 67]], ids=["bulk", "tokens"])
+def test_int_anchor_parity(D, G, k, v, rule, n, abits, chunks):
+    """Post 6, "The winning recipe" item 4 (anchor-precision dial) and "Best results" (int8 anchors
+    with ternary and sign KV): anchored rows stored on an 8/4-bit grid; codes, scales, anchors,
+    dequantization and attention against the oracle."""
+    T = 200
+    cfg = Config(n_layers=2, batch=2, n_kv_heads=2, n_q_heads=2 * G, head_dim=D, capacity=T, k=k, v=v, max_queries=8,
+                 anchor_layers=(0,), anchor_rule=rule, anchor_n=n, anchor_bits=abits)
+    c = Case(cfg, T, chunks=chunks)
+    for l in (0, 1):
+        c.check_codes(l)
+        c.check_anchors(l)
+        c.check_dequant(l)
+        q = synth.queries(1, l, 2, cfg.n_q_heads, D, T)
+        c.decode_and_compare(l, q, kv_len=[200, 151])
