@@ -29,6 +29,13 @@ Grids and scales (sources by page title and section):
     on rotated values"); levels from oracle.lloyd in units of the group's RMS,
     s = fp16(sqrt(fp32(fp32 sum of x^2 in channel order / g))), code = nearest level of x/s
     (ties up); s = 0 gives the level just above zero, 2^(b-1).
+  * sorted groups: post 6, "The winning recipe" item 1 (titled magnitude-sorted grouping: "sort
+    each row descending, quantize groups; outliers share one wide group", g = 8 for K and 4 for
+    V, with 2-bit codes).  Reading taken here: a row is ordered by value, descending (equal values
+    keep channel order), and consecutive g values of that order form a group on the per-token
+    min-max grid (so the top group, where large outliers gather, gets its own wide range); the row
+    stores each channel's rank (its position in the order) in ceil(log2 D) bits -- the permutation
+    the page's bit counts leave out -- after the codes.
   * rFFT polar: the reply, "Fixed-rate magnitude/phase allocation" (mag/phase splits
     4+8 .. 8+4 at 12 bits per coefficient) and "The finite-phase implementation and the
     physical codec may be worth separating" (a magnitude index and one phase-angle index per
@@ -61,7 +68,7 @@ F64 = np.float64
 
 @dataclass(frozen=True)
 class Side:
-    fmt: str = "int"          # int | nf4 | ternary | sign | polar | cart | lloyd | fp16
+    fmt: str = "int"          # int | nf4 | ternary | sign | polar | cart | lloyd | sorted | fp16
     bits: int = 4             # code bits (magnitude bits for polar)
     bits2: int = 0            # phase bits (polar only)
     scale: str = "absmax"     # absmax | minmax | sym   (int only)
@@ -88,10 +95,17 @@ class Side:
             return (D // 2) * (self.bits + self.bits2) // 8
         if self.fmt == "nf4":
             return D // 2
+        if self.fmt == "sorted":
+            return -(-(D * self.bits + D * rank_bits(D)) // 8)
         return -(-D * self.bits // 8)  # int (absmax, minmax, sym), lloyd, cart
 
     def has_zero(self) -> bool:
-        return self.fmt == "int" and self.scale == "minmax"
+        return (self.fmt == "int" and self.scale == "minmax") or self.fmt == "sorted"
+
+
+def rank_bits(D: int) -> int:
+    """Bits of one stored rank (channel position in the magnitude order): ceil(log2 D)."""
+    return max(1, (D - 1).bit_length())
 
 
 def f16(x) -> np.ndarray:
@@ -252,6 +266,17 @@ def quant_lloyd(x32: np.ndarray, b: int, g: int):
     return code.reshape(R, D).astype(np.int64), s
 
 
+def quant_sorted(x32: np.ndarray, b: int, g: int):
+    """Sorted groups: returns (q at sorted positions, d and z per sorted group, rank per channel)."""
+    R, D = x32.shape
+    x = np.asarray(x32, dtype=F32)
+    order = np.argsort(-x, axis=1, kind="stable")  # channel at each sorted position (descending)
+    rank = np.empty_like(order)
+    rank[np.arange(R)[:, None], order] = np.arange(D)[None, :]
+    q, d, z = quant_int_minmax(np.take_along_axis(x, order, axis=1), b, g)
+    return q, d, z, rank
+
+
 def quant_sign(x32: np.ndarray, g: int):
     R, D = x32.shape
     xg = x32.reshape(R, D // g, g).astype(F32)
@@ -343,6 +368,17 @@ def quantize_rows(x16: np.ndarray, side: Side, c16=None, mu16=None) -> dict:
         out["exact"] = val
         out["scales"] = s.astype(np.float16)
         out["q"] = code
+    elif side.fmt == "sorted":
+        q, d, z, rank = quant_sorted(x, side.bits, g)
+        out["bytes"] = np.concatenate([pack_bits(q, side.bits), pack_bits(rank, rank_bits(D))], axis=1)
+        rows = np.arange(R)[:, None]
+        qq, dd, zz = q[rows, rank], d[rows, rank // g], z[rows, rank // g]  # channel order
+        out["stored"] = (zz.astype(F32) + (qq * dd).astype(F32)).astype(F32)
+        out["exact"] = zz + qq * dd
+        out["scales"] = d.astype(np.float16)
+        out["zeros"] = z.astype(np.float16)
+        out["q"] = q
+        out["rank"] = rank
     elif side.fmt == "int" and side.scale == "absmax":
         q, d = quant_int_absmax(x, side.bits, g)
         out["bytes"] = pack_bits(q + 2 ** (side.bits - 1), side.bits)
@@ -435,7 +471,7 @@ def bits_per_value(side: Side, D: int) -> float:
     """Storage bits per value of one quantized row: codes + fp16 scales (+ fp16 zeros)."""
     if side.fmt == "fp16":
         return 16.0
-    code_bits = side.row_bytes(D) * 8 if side.fmt == "ternary" else (
+    code_bits = side.row_bytes(D) * 8 if side.fmt in ("ternary", "sorted") else (
         (D // 2) * (side.bits + side.bits2) if side.fmt == "polar" else
         D * (1 if side.fmt == "sign" else (4 if side.fmt == "nf4" else side.bits)))
     meta = 16 * side.n_groups(D) * (2 if side.has_zero() else 1)
