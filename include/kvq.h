@@ -57,8 +57,12 @@ enum {
   KVQ_FMT_SIGN = 4,     /* {-s, +s}, s = group mean |x| [FMKQ] "Minimal recipe" */
   KVQ_FMT_POLAR = 5,    /* rFFT magnitude (bits) / phase (bits2) indices [FMKQ] reply */
   KVQ_FMT_CART = 6,     /* rFFT real/imag, signed absmax int-bits, one scale [FMKQ] reply control */
-  KVQ_FMT_LLOYD = 7     /* Gaussian Lloyd-Max levels (bits 2..4) times the group RMS, [E22L] "Result":
+  KVQ_FMT_LLOYD = 7,    /* Gaussian Lloyd-Max levels (bits 2..4) times the group RMS, [E22L] "Result":
                            the value grid named for the next run */
+  KVQ_FMT_SORTED = 8    /* sorted groups ([FMKQ] post 6 "The winning recipe" item 1): the row sorted
+                           descending (equal values in channel order), consecutive `group` values on
+                           the min-max grid at `bits` (2..4), and each channel's rank stored in
+                           ceil(log2 head_dim) bits after the codes; fp16 scale and zero per group */
 };
 /* INT scale modes: ABSMAX = the ggml signed grid; MINMAX = asymmetric; SYMMETRIC = levels
  * (q - (2^b - 1)/2) d, outermost level at the group's largest magnitude ([E22L] "Result": the

@@ -47,6 +47,12 @@ __device__ __forceinline__ float stored_value(const SideDev& S, const uint8_t* _
     }
     case KVQ_FMT_LLOYD:
       return lloyd[get_bits(row, j * S.bits, S.bits)] * __half2float(sc[j / S.group]);
+    case KVQ_FMT_SORTED: {  // channel j's rank p (after the codes), then code p of its sorted group
+      const int D = S.n_groups * S.group, rb = 32 - __clz(D - 1);
+      const int p = (int)get_bits(row, D * S.bits + j * rb, rb), g = p / S.group;
+      const int c = (int)get_bits(row, p * S.bits, S.bits);
+      return __fadd_rn(__half2float(zr[g]), (float)c * __half2float(sc[g]));
+    }
     case KVQ_FMT_NF4: {
       const float s = __half2float(sc[j / S.group]);
       return nf4[get_bits(row, j * 4, 4)] * s;

@@ -63,6 +63,7 @@ kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
         return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_FMT_LLOYD:
+    case KVQ_FMT_SORTED:
       if (s.bits < 2 || s.bits > 4) return KVQ_ERR_INVALID_ARG;
       if (s.scale_mode != KVQ_SCALE_ABSMAX) return KVQ_ERR_INVALID_ARG;
       break;
@@ -131,7 +132,8 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
       if (c->anchor_rule == KVQ_ANCHOR_NONE || !((c->anchor_layer_mask >> l) & 1ULL)) continue;
       for (int sd = 0; sd < 2; ++sd) {
         const kvq_side& x = sd == 0 ? (lk ? lk[l] : c->k) : (lv ? lv[l] : c->v);
-        if (x.format == KVQ_FMT_FP16 || x.format == KVQ_FMT_POLAR || x.format == KVQ_FMT_CART)
+        if (x.format == KVQ_FMT_FP16 || x.format == KVQ_FMT_POLAR || x.format == KVQ_FMT_CART ||
+            x.format == KVQ_FMT_SORTED)
           return KVQ_ERR_UNSUPPORTED;
       }
     }
@@ -141,11 +143,18 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
 
 int anchor_bits_of(const kvq_config& c) { return (c.anchor_bits == 8 || c.anchor_bits == 4) ? c.anchor_bits : 16; }
 
+int rank_bits(int D) { return 32 - __builtin_clz((unsigned)(D - 1)); }  // ceil(log2 D), D >= 2
+
+bool has_zero_points(const kvq_side& s) {
+  return (s.format == KVQ_FMT_INT && s.scale_mode == KVQ_SCALE_MINMAX) || s.format == KVQ_FMT_SORTED;
+}
+
 void side_geometry(int D, const kvq_side& s, int* row_bytes, int* n_groups) {
   switch (s.format) {
     case KVQ_FMT_FP16: *row_bytes = 2 * D; *n_groups = 0; return;
     case KVQ_FMT_INT:
     case KVQ_FMT_LLOYD: *row_bytes = D * s.bits / 8; *n_groups = D / s.group; return;
+    case KVQ_FMT_SORTED: *row_bytes = D * (s.bits + rank_bits(D)) / 8; *n_groups = D / s.group; return;
     case KVQ_FMT_NF4: *row_bytes = D / 2; *n_groups = D / s.group; return;
     case KVQ_FMT_TERNARY: *row_bytes = (D + 4) / 5; *n_groups = D / s.group; return;
     case KVQ_FMT_SIGN: *row_bytes = D / 8; *n_groups = D / s.group; return;
@@ -183,7 +192,7 @@ uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
         off = align_up(off + units * Tcap * (uint64_t)ng * 2);
       }
       so.zeros = -1;
-      if (sd.format == KVQ_FMT_INT && sd.scale_mode == KVQ_SCALE_MINMAX) {
+      if (has_zero_points(sd)) {
         so.zeros = (int64_t)off;
         off = align_up(off + units * Tcap * (uint64_t)ng * 2);
       }

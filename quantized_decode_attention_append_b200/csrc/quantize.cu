@@ -389,6 +389,112 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
 }
 
 // ------------------------------------------------------------------------------------------
+// Sorted groups: one warp per row, the row in shared memory.  A channel's rank (its position when
+// the row is sorted descending, equal values in channel order) is counted against every other
+// channel; values move to their ranks; consecutive groups of the sorted row take the min-max grid;
+// codes (sorted order) then ranks (channel order) are packed LSB-first.  Pre-transforms run first,
+// the Hadamard stages in the same butterfly order as the row kernel.
+constexpr int kSortWarps = 4;
+
+__global__ void __launch_bounds__(128) append_sorted_kernel(LayerDev L, int side, const __half* __restrict__ src,
+                                                            int n_new, unsigned total_ctas) {
+  const SideDev& S = L.s[side];
+  const int D = L.D, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ float sx[kSortWarps][256], sv[kSortWarps][256];
+  __shared__ uint32_t scode[kSortWarps][256], srank[kSortWarps][256];
+  const long long R = (long long)L.app_n * L.Hkv * n_new;
+  const int G = S.group, bits = S.bits, rb = 32 - __clz(D - 1), ng = D / G, top = (1 << bits) - 1;
+  for (long long row = (long long)blockIdx.x * kSortWarps + warp; row < R; row += (long long)gridDim.x * kSortWarps) {
+    const RowDst dst = row_dst(L, (int)row, n_new);
+    if (dst.err) {  // warp-uniform: the whole warp holds this row
+      if (dst.first && lane == 0) atomicOr(L.err, dst.err);
+      continue;
+    }
+    const __half* rp = src + row * D;
+    float* x = sx[warp];
+    for (int j = lane; j < D; j += 32) {
+      float v = __half2float(rp[j]);
+      if (S.mean_sub) v = __fsub_rn(v, __half2float(S.kmean[(long long)dst.u * D + j]));
+      if (S.chan_scale) v = __fdiv_rn(v, __half2float(S.chan[(dst.u % L.Hkv) * D + j]));
+      x[j] = v;
+    }
+    if (in_anchor(L, dst.pos, dst.len_after)) {  // fp16 anchors (int anchors are refused on the host)
+      __half* ap = S.anchors + ((long long)dst.u * L.anchor_rows + anchor_slot(L, dst.pos)) * D;
+      for (int j = lane; j < D; j += 32) ap[j] = rp[j];
+    }
+    __syncwarp();
+    if (S.rot) {  // stages h = 1 .. rot/2: (x_i, x_i+h) <- (x_i + x_i+h, x_i - x_i+h), bit h of i clear
+      for (int h = 1; h < S.rot; h <<= 1) {
+        for (int p = lane; p < D / 2; p += 32) {
+          const int i = ((p >> (__ffs(h) - 1)) << __ffs(h)) | (p & (h - 1));
+          const float a = x[i], b = x[i + h];
+          x[i] = __fadd_rn(a, b);
+          x[i + h] = __fsub_rn(a, b);
+        }
+        __syncwarp();
+      }
+      const float rn = S.rot == 256 ? 0.0625f : __fdiv_rn(__fsqrt_rn(2.0f), 16.0f);
+      for (int j = lane; j < D; j += 32) x[j] = __fmul_rn(x[j], rn);
+      __syncwarp();
+    }
+    float* v = sv[warp];
+    for (int j = lane; j < D; j += 32) {
+      const float xj = x[j];
+      int r = 0;
+      for (int k = 0; k < D; ++k) {
+        const float xk = x[k];
+        r += (xk > xj || (xk == xj && k < j)) ? 1 : 0;
+      }
+      srank[warp][j] = (uint32_t)r;
+      v[r] = xj;
+    }
+    __syncwarp();
+    const long long rix = (long long)dst.u * L.Tcap + dst.pos;
+    for (int gi = lane; gi < ng; gi += 32) {  // sorted descending: the group's max leads, its min ends it
+      const float* gv = v + gi * G;
+      const float mx = gv[0];
+      float mn = gv[G - 1];
+      if (mn == 0.0f) {  // a zero minimum is -0 iff the group holds a -0 (the min-max rule)
+        bool negz = false;
+        for (int e = 0; e < G; ++e) negz |= __float_as_uint(gv[e]) == 0x80000000u;
+        mn = negz ? -0.0f : 0.0f;
+      }
+      const __half zh = __float2half_rn(mn), sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)top));
+      const float z = __half2float(zh), d = __half2float(sh), inv = d != 0.0f ? __frcp_rn(d) : 0.0f;
+      for (int e = 0; e < G; ++e) {
+        const float k = d != 0.0f ? fminf(fmaxf(round_exact_minmax(gv[e], z, d, inv), 0.0f), (float)top) : 0.0f;
+        scode[warp][gi * G + e] = (uint32_t)(int)k;
+      }
+      S.scales[rix * ng + gi] = sh;
+      S.zeros[rix * ng + gi] = zh;
+    }
+    __syncwarp();
+    uint32_t* cw = reinterpret_cast<uint32_t*>(S.codes + rix * S.row_bytes);
+    const int nwords = D * (bits + rb) / 32, cbits = D * bits;
+    for (int w = lane; w < nwords; w += 32) {
+      uint32_t word = 0u;
+      const int b0 = w * 32;
+      for (int e = b0 / bits; e < D && e * bits < b0 + 32; ++e) {
+        const int off = e * bits - b0;
+        const uint64_t c = scode[warp][e];
+        word |= (uint32_t)(off >= 0 ? (c << off) : (c >> (-off)));
+      }
+      if (b0 + 32 > cbits) {
+        const int lo = b0 > cbits ? b0 - cbits : 0;
+        for (int e = lo / rb; e < D && cbits + e * rb < b0 + 32; ++e) {
+          const int off = cbits + e * rb - b0;
+          const uint64_t r = srank[warp][e];
+          word |= (uint32_t)(off >= 0 ? (r << off) : (r >> (-off)));
+        }
+      }
+      cw[w] = word;
+    }
+    __syncwarp();  // sx/sv/scode/srank are reused by this warp's next row
+  }
+  finish_append(L, n_new, total_ctas);
+}
+
+// ------------------------------------------------------------------------------------------
 // Row formats (int, NF4, ternary, sign): each row is split over D/32 lanes, each lane holding 32
 // contiguous values in registers; a warp covers 32/(D/32) consecutive rows, so loads are
 // coalesced 64-byte pieces and a lane's codes fill whole 32-bit words of the packed row.  The
@@ -912,6 +1018,9 @@ static RowKernel pick_rows_kernel(int fam, int g) {
 bool append_supported(int D, const kvq_side& s) {
   if (s.format == KVQ_FMT_FP16) return true;
   if (s.format == KVQ_FMT_POLAR || s.format == KVQ_FMT_CART) return D == 128 && s.rotation == 0;
+  if (s.format == KVQ_FMT_SORTED)
+    return (D == 64 || D == 128 || D == 256) && !(s.rotation > D || (s.rotation && D % s.rotation)) && s.group >= 4 &&
+           s.group <= D;
   if (s.format != KVQ_FMT_INT && s.format != KVQ_FMT_NF4 && s.format != KVQ_FMT_TERNARY && s.format != KVQ_FMT_SIGN &&
       s.format != KVQ_FMT_LLOYD)
     return false;
@@ -989,6 +1098,10 @@ static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
     p.kern = append_fp16_kernel;
     const long long want = (R * (L.D / 8) + 127) / 128;
     p.blocks = (unsigned)(want < kMaxAppendCtas ? want : kMaxAppendCtas);
+  } else if (S.fmt == KVQ_FMT_SORTED) {
+    p.kern = append_sorted_kernel;
+    const long long want = (R + kSortWarps - 1) / kSortWarps;
+    p.blocks = (unsigned)(want < kMaxAppendCtas ? want : kMaxAppendCtas);
   } else if (S.fmt == KVQ_FMT_POLAR || S.fmt == KVQ_FMT_CART) {
     p.kern = append_fft_kernel;
     const long long want = (R + kFftWarps - 1) / kFftWarps;
@@ -1010,7 +1123,7 @@ static KvKernel pick_kv_kernel(const LayerDev& L) {
   const SideDev& K = L.s[0];
   const SideDev& V = L.s[1];
   if (K.fmt == KVQ_FMT_FP16 || V.fmt == KVQ_FMT_FP16 || K.fmt == KVQ_FMT_POLAR || K.fmt == KVQ_FMT_CART ||
-      V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART)
+      V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART || K.fmt == KVQ_FMT_SORTED || V.fmt == KVQ_FMT_SORTED)
     return nullptr;
   const int fk = fam_of(K), fv = fam_of(V), gk = K.group, gv = V.group;
   // bits 0: fixed by the family (NF4, ternary, sign)

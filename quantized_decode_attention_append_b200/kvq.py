@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkvq.so")
 
 # enums (values fixed by include/kvq.h)
-FMT = {"fp16": 0, "int": 1, "nf4": 2, "ternary": 3, "sign": 4, "polar": 5, "cart": 6, "lloyd": 7}
+FMT = {"fp16": 0, "int": 1, "nf4": 2, "ternary": 3, "sign": 4, "polar": 5, "cart": 6, "lloyd": 7, "sorted": 8}
 SCALE = {"absmax": 0, "minmax": 1, "sym": 2}
 ANCHOR = {"none": 0, "first_n": 1, "window": 2, "all": 3}
 SIDE_K, SIDE_V = 0, 1

@@ -244,3 +244,17 @@ def test_int_anchor_arena_is_smaller():
     n4 = status_of(base_cfg(anchor_bits=4, **kw))[1]
     assert n16 > n8 > n4
     assert n16 - n8 == pytest.approx(2 * 2 * 4 * 256 * (128 * 2 - 128 - 8), abs=4 * 512)
+
+
+def test_sorted_group_configs():
+    """Sorted groups (post 6, "The winning recipe" item 1): 2..4 bits, a zero point per group, the
+    ranks in ceil(log2 D) bits per value after the codes."""
+    ok = Side("sorted", 2, group=8)
+    assert status_of(base_cfg(k=ok, v=Side("sorted", 2, group=4)))[0] == 0
+    assert status_of(base_cfg(k=Side("sorted", 5, group=8)))[0] == -1
+    assert status_of(base_cfg(k=Side("sorted", 2, scale="minmax", group=8)))[0] == -1
+    assert status_of(base_cfg(k=ok, anchor_layers=(0,), anchor_rule="first_n", anchor_n=8, anchor_bits=8))[0] == -2
+    st, n = status_of(base_cfg(k=ok, v=ok))
+    st4, n4 = status_of(base_cfg(k=Side("int", 2, scale="minmax", group=8), v=Side("int", 2, scale="minmax", group=8)))
+    # per row: the same codes and metadata plus 7 x 128 rank bits (112 bytes)
+    assert st == 0 and st4 == 0 and n - n4 == pytest.approx(2 * 2 * 4 * 512 * 112, abs=2 * 2 * 3 * 256)

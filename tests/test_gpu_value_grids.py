@@ -146,3 +146,29 @@ def test_int_anchor_parity(D, G, k, v, rule, n, abits, chunks):
         c.check_dequant(l)
         q = synth.queries(1, l, 2, cfg.n_q_heads, D, T)
         c.decode_and_compare(l, q, kv_len=[200, 151])
+
+
+SORTED = [
+    (128, 4, Side("sorted", 2, group=8), Side("sorted", 2, group=4), {}),                  # the page's g8 K / g4 V
+    (128, 2, Side("sorted", 3, group=8, rot=128), Side("sorted", 4, group=16), {}),
+    (256, 2, Side("sorted", 2, group=8, mean_sub=True), Side("sorted", 2, group=32, rot=256),
+     dict(anchor_layers=(0,), anchor_rule="first_n", anchor_n=33)),
+    (64, 1, Side("sorted", 2, group=4, chan_scale=True), Side("int", 4, group=16), {}),
+]
+
+
+@pytest.mark.parametrize("D,G,k,v,anc", SORTED, ids=[f"{d}-{k.fmt}{k.bits}g{k.group}r{k.rot}-{v.fmt}{v.bits}g{v.group}"
+                                                     for d, g, k, v, _ in SORTED])
+@pytest.mark.parametrize("chunks", [None, [1, 1, 120, 1, 77]], ids=["bulk", "tokens"])
+def test_sorted_group_parity(D, G, k, v, anc, chunks):
+    """Sorted groups with their stored ranks (post 6, "The winning recipe" item 1): codes, ranks,
+    scales and zero points bit for bit, dequantization, and attention from the generic decode."""
+    T = 200
+    cfg = cfg_of(D, k, v, G=G, T=T, **anc)
+    c = Case(cfg, T, chunks=chunks)
+    c.check_codes(0)
+    c.check_anchors(0)
+    c.check_dequant(0)
+    q = synth.queries(1, 0, 2, cfg.n_q_heads, D, T)
+    c.decode_and_compare(0, q)
+    c.decode_and_compare(0, q, kv_len=[200, 64])
