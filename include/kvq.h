@@ -119,8 +119,8 @@ typedef struct {
                                   LLOYD) on both sides of anchored layers. */
 } kvq_config;
 
-/* Byte offsets (into the arena) and geometry of one (layer, side).  Rows of one
- * (sequence, kv-head) are contiguous: row r of unit u = (b * n_kv_heads + h) is at
+/* Byte offsets (into the arena) and geometry of one (layer, side) of a head group.  Rows of one
+ * (sequence, kv-head) are contiguous: row r of unit u = (b * n_heads + h - head0) is at
  * codes + (u * row_stride_tokens + r) * row_bytes; scales (fp16) at
  * scales + ((u * row_stride_tokens + r) * n_groups) * 2, zeros likewise (MINMAX only).
  * Anchor rows (fp16, original domain) at anchors + ((u * anchor_rows + slot) * head_dim) * 2,
@@ -131,6 +131,9 @@ typedef struct {
   int64_t anchor_scales;  /* int anchors: fp16 [units][anchor_rows][head_dim / 32]; anchor rows then hold
                              head_dim * anchor_bits / 8 code bytes each (LSB-first) instead of fp16 */
   int32_t row_bytes, n_groups, row_stride_tokens, anchor_rows;
+  int32_t head0, n_heads;  /* the head group these regions hold: kv-heads [head0, head0 + n_heads) of
+                              the layer (all of them without per-head formats); unit u = b * n_heads
+                              + (h - head0) */
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache;
@@ -155,6 +158,20 @@ kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k
 kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
                              uint64_t arena_bytes, kvq_cache** out);
 
+/* Per-(layer, kv-head) formats (llama.cpp #21385 "Finding 2": per-head bit allocation from the
+ * Renyi entropy of each head's attention, b_h = b_avg + 0.25 (H_avg - H_2(h)), with the lowest-
+ * entropy ~2% of heads -- the sink heads -- kept unquantized; "Feature Request: Per-Head KV Cache
+ * Types": per-head type selection in the cache allocation and per-head dequantization dispatch).
+ * head_k / head_v: host arrays of n_layers * n_kv_heads sides, layer-major, read during the call
+ * only; NULL means cfg->k / cfg->v everywhere.  Consecutive heads of a layer with equal (K, V)
+ * formats form a head group with its own arena regions and launches (kvq_get_layout_head).
+ * Every side is checked as in kvq_create; otherwise identical to kvq_arena_bytes / kvq_create.
+ * The allocation itself (entropies, rounding, sink heads) is the caller's calibration. */
+kvq_status kvq_arena_bytes_heads(const kvq_config* cfg, const kvq_side* head_k, const kvq_side* head_v,
+                                 uint64_t* bytes);
+kvq_status kvq_create_heads(const kvq_config* cfg, const kvq_side* head_k, const kvq_side* head_v, void* arena,
+                            uint64_t arena_bytes, kvq_cache** out);
+
 /* Release the handle and its split-K workspace; the caller-owned arena (the packed cache itself)
  * is left untouched and may be freed by the caller afterwards.  NULL is a no-op.  Synchronous
  * (cudaFree).  The pages manage no handle: their cache memory is what the configuration budgets
@@ -163,8 +180,10 @@ kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, con
  * here. */
 void kvq_free(kvq_cache* cache);
 
-/* Geometry of (layer, side) for inspection and tests.  Host only. */
+/* Geometry of (layer, side) for inspection and tests: the head group holding kv-head `head`
+ * (kvq_get_layout: kv-head 0).  Host only. */
 kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, int32_t side, kvq_layout* out);
+kvq_status kvq_get_layout_head(const kvq_cache* cache, int32_t layer, int32_t side, int32_t head, kvq_layout* out);
 
 /* Copy the per-channel K scale c [n_kv_heads][head_dim] (fp16, device) of `layer` into the
  * arena ([E21W] variants C/D: "calibrated offline").  Required before appending to a layer

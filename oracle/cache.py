@@ -66,9 +66,14 @@ class Spec:
     layer_k: tuple = ()  # one Side per layer, or empty: k on every layer
     layer_v: tuple = ()
     anchor_bits: int = 16  # 16 (fp16 rows), 8 or 4 (signed absmax grid, groups of 32)
+    head_k: tuple = ()  # per (layer, kv-head): n_layers tuples of n_kv Sides, or empty
+    head_v: tuple = ()
 
 
-def side_of(spec: Spec, layer: int, is_k: bool) -> Side:
+def side_of(spec: Spec, layer: int, is_k: bool, head: int = 0) -> Side:
+    ph = spec.head_k if is_k else spec.head_v
+    if ph:
+        return ph[layer][head]
     per = spec.layer_k if is_k else spec.layer_v
     return per[layer] if per else (spec.k if is_k else spec.v)
 
@@ -106,15 +111,18 @@ def key_mean(K16: np.ndarray) -> np.ndarray:
     return ((S.astype(F64) / F64(k.shape[0])) * 2.0 ** -24).astype(np.float16)
 
 
-def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None, layer: int = 0, first_rows=None):
+def quantize_unit(spec: Spec, K16: np.ndarray, V16: np.ndarray, c16=None, layer: int = 0, first_rows=None,
+                  head: int = 0):
     """Quantize one (layer, sequence, kv-head) unit: K16, V16 [T, D]; c16 [D] or None;
     first_rows: rows of the sequence's first append (the key mean's rows; default all)."""
-    ks = side_of(spec, layer, True)
+    ks = side_of(spec, layer, True, head)
     mu = key_mean(K16[:first_rows or K16.shape[0]]) if ks.mean_sub else None
     kq = quantize_rows(K16, ks, None if c16 is None else np.broadcast_to(c16, K16.shape),
                        None if mu is None else np.broadcast_to(mu, K16.shape))
     kq["mu"] = mu
-    vq = quantize_rows(V16, side_of(spec, layer, False), None)
+    kq["side"] = ks
+    vq = quantize_rows(V16, side_of(spec, layer, False, head), None)
+    vq["side"] = side_of(spec, layer, False, head)
     return kq, vq
 
 
@@ -123,9 +131,9 @@ def reconstruct_unit(spec: Spec, layer: int, K16, V16, kq, vq, seq_len: int, c16
     T = K16.shape[0]
     cK = None if c16 is None else np.broadcast_to(c16, K16.shape)
     mu = kq.get("mu")
-    Kh = to_original_f64(kq["exact"], side_of(spec, layer, True), cK,
+    Kh = to_original_f64(kq["exact"], kq.get("side") or side_of(spec, layer, True), cK,
                          None if mu is None else np.broadcast_to(mu, K16.shape))
-    Vh = to_original_f64(vq["exact"], side_of(spec, layer, False), None)
+    Vh = to_original_f64(vq["exact"], vq.get("side") or side_of(spec, layer, False), None)
     an = anchored(spec, layer, np.arange(T), seq_len)
     if an.any():
         Kh[an] = anchor_rows(spec, np.asarray(K16)[an])["exact"]
@@ -139,18 +147,21 @@ def decode_query(spec: Spec, layer: int, q16: np.ndarray, Kh: np.ndarray, Vh: np
 
 
 def effective_bits(spec: Spec, seq_len: int) -> float:
-    """Average stored bits per K/V value over all layers of one sequence of length seq_len."""
+    """Average stored bits per K/V value over all layers (and kv-heads) of one sequence of length
+    seq_len."""
     D = spec.D
+    heads = spec.n_kv if (spec.head_k or spec.head_v) else 1
     tot = 0.0
     for layer in range(spec.n_layers):
         an = anchored(spec, layer, np.arange(seq_len), seq_len).sum()
         a_row = 16 * D if spec.anchor_bits == 16 else bits_per_value(anchor_side(spec), D) * D
-        for side, is_k in ((side_of(spec, layer, True), True), (side_of(spec, layer, False), False)):
-            per_row = bits_per_value(side, D) * D
-            bits = (seq_len - an) * per_row + an * a_row
-            if is_k and side.chan_scale:
-                bits += 16 * D
-            if is_k and side.mean_sub:
-                bits += 16 * D
-            tot += bits
-    return tot / (spec.n_layers * 2 * seq_len * D)
+        for h in range(heads):
+            for side, is_k in ((side_of(spec, layer, True, h), True), (side_of(spec, layer, False, h), False)):
+                per_row = bits_per_value(side, D) * D
+                bits = (seq_len - an) * per_row + an * a_row
+                if is_k and side.chan_scale:
+                    bits += 16 * D
+                if is_k and side.mean_sub:
+                    bits += 16 * D
+                tot += bits
+    return tot / (spec.n_layers * heads * 2 * seq_len * D)

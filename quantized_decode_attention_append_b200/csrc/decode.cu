@@ -98,7 +98,7 @@ __device__ void query_mean_term(const LayerDev& L, const __half* __restrict__ q,
   for (int h = threadIdx.x >> 5; h < G; h += blockDim.x >> 5) {
     float acc = 0.0f;
     if (K.mean_sub) {
-      const __half* qp = q + ((long long)qi * L.Hq + kvh * G + h) * D;
+      const __half* qp = q + query_row(L, qi, kvh, G, h) * D;
       const __half* mp = K.kmean + ((long long)seq * L.Hkv + kvh) * D;
       for (int j = lane; j < D; j += 32) acc = fmaf(__half2float(qp[j]), __half2float(mp[j]), acc);
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -116,7 +116,7 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
   const int tid = threadIdx.x;
   for (int e = tid; e < G * D; e += blockDim.x) {
     const int h = e / D, j = e % D;
-    const float v = __half2float(q[((long long)qi * L.Hq + kvh * G + h) * D + j]);
+    const float v = __half2float(q[query_row(L, qi, kvh, G, h) * D + j]);
     qa[e] = v * scl;
     qs[e] = K.chan_scale ? v * __half2float(K.chan[kvh * D + j]) : v;
   }
@@ -390,8 +390,9 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
                                                                      int n_split, int nsp, void* __restrict__ out,
                                                                      int out_fp32, float* __restrict__ lse) {
   constexpr int SP = merge_groups<D>(), NT = D * SP, NWP = NT / 32;
-  const int qh = blockIdx.x;  // qi * Hq + h
+  const int qh = blockIdx.x;  // qi * Hq + h (this view's heads)
   const int tid = threadIdx.x, j = tid % D, sg = tid / D;
+  const long long orow = (long long)(qh / L.Hq) * L.Hkv_all * (L.Hq / L.Hkv) + L.h0 * (L.Hq / L.Hkv) + qh % L.Hq;
   const SideDev& V = L.s[1];
   const float* P = work + (long long)qh * nsp * (D + kPartStride);
   __shared__ float w[kMaxSplit + 1];
@@ -473,9 +474,9 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
     float v = ov[tid];
     if (nsp > n_split) v += w[n_split] * P[n_split * (D + kPartStride) + kPartStride + tid];
     v *= inv;
-    if (out_fp32) reinterpret_cast<float*>(out)[(long long)qh * D + tid] = v;
-    else reinterpret_cast<__half*>(out)[(long long)qh * D + tid] = __float2half_rn(v);
-    if (lse && tid == 0) lse[qh] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+    if (out_fp32) reinterpret_cast<float*>(out)[orow * D + tid] = v;
+    else reinterpret_cast<__half*>(out)[orow * D + tid] = __float2half_rn(v);
+    if (lse && tid == 0) lse[orow] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
   }
 }
 

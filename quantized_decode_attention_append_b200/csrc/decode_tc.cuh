@@ -313,7 +313,7 @@ __device__ void prepare_query_rot(const LayerDev& L, const __half* __restrict__ 
   if (warp < G) {
     const int h = warp, j0 = lane * V;
     float x[V];
-    const __half* qp = q + ((long long)qi * L.Hq + kvh * G + h) * D + j0;
+    const __half* qp = q + query_row(L, qi, kvh, G, h) * D + j0;
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       x[v] = __half2float(qp[v]);

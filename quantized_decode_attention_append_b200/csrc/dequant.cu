@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(LayerDev L, int side, int 
     }
     __syncwarp();
   }
-  const long long ob = row * D;
+  const long long ob = (((u / L.Hkv) * L.Hkv_all + L.h0 + u % L.Hkv) * nt + i) * D;  // caller's [B][Hkv_all][nt]
   for (int j = lane; j < D; j += 32) {
     if (out_fp32) reinterpret_cast<float*>(out)[ob + j] = x[j];
     else reinterpret_cast<__half*>(out)[ob + j] = __float2half_rn(x[j]);

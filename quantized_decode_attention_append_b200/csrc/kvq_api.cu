@@ -7,23 +7,35 @@
 #include <mutex>
 #include <new>
 #include <set>
+#include <vector>
 
 #include "kvq_internal.h"
 
 using namespace kvq;
 
+// Arena offsets of one side of one head group.
+struct SideOff {
+  int64_t codes, scales, zeros, anchors, anchor_scales;
+  int row_bytes, n_groups;
+};
+
+// Consecutive kv-heads [h0, h0 + nh) of a layer with one (K, V) format pair: they share arena
+// regions (unit = b * nh + local head) and are appended, decoded and dequantized by one set of
+// launches.  A layer without per-head formats is one group.
+struct HeadGroup {
+  int h0, nh;
+  kvq_side side[2];
+  SideOff off[2];
+  int64_t kmean;  // K key means [B * nh][D] fp16, or -1
+};
+
 struct kvq_cache {
   kvq_config cfg;
-  kvq_side side[64][2];  // format of each (layer, side): cfg.k / cfg.v unless set per layer
+  std::vector<HeadGroup> grp[64];  // per layer
   int Tcap;
   char* arena;
   uint64_t arena_bytes;
-  struct SideOff {
-    int64_t codes, scales, zeros, anchors, anchor_scales;
-    int row_bytes, n_groups;
-  } off[64][2];
-  int64_t chan[64];
-  int64_t kmean[64];
+  int64_t chan[64];      // per layer [Hkv][D] fp16 channel scales (some K side of the layer has them), or -1
   int64_t lens, tickets, err;
   int anchor_rows;
   int max_len[64];       // host-side bound on every sequence's length (exact while len_exact)
@@ -90,19 +102,31 @@ kvq_status check_side(const kvq_config& c, const kvq_side& s, bool is_k) {
   return KVQ_OK;
 }
 
-// The (layer, side) formats of a cache: the per-layer arrays where given, else cfg.k / cfg.v.
-struct LayerSides {
-  kvq_side s[64][2];
+// The (layer, kv-head, side) formats of a cache: per-head arrays where given, else per-layer
+// arrays, else cfg.k / cfg.v.
+struct HeadSides {
+  std::vector<kvq_side> k, v;  // [n_layers * n_kv_heads]
+  const kvq_side& at(int side, int l, int h, int H) const { return (side ? v : k)[(size_t)l * H + h]; }
 };
 
-void fill_sides(const kvq_config& c, const kvq_side* lk, const kvq_side* lv, LayerSides* out) {
-  for (int l = 0; l < c.n_layers && l < 64; ++l) {
-    out->s[l][0] = lk ? lk[l] : c.k;
-    out->s[l][1] = lv ? lv[l] : c.v;
-  }
+bool fill_sides(const kvq_config* c, const kvq_side* lk, const kvq_side* lv, const kvq_side* hk, const kvq_side* hv,
+                HeadSides* out) {
+  if (!c || c->n_layers < 1 || c->n_layers > 64 || c->n_kv_heads < 1 || c->n_kv_heads > 4096) return false;
+  const int L = c->n_layers, H = c->n_kv_heads;
+  out->k.resize((size_t)L * H);
+  out->v.resize((size_t)L * H);
+  for (int l = 0; l < L; ++l)
+    for (int h = 0; h < H; ++h) {
+      const size_t i = (size_t)l * H + h;
+      out->k[i] = hk ? hk[i] : (lk ? lk[l] : c->k);
+      out->v[i] = hv ? hv[i] : (lv ? lv[l] : c->v);
+    }
+  return true;
 }
 
-kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side* lv) {
+bool same_side(const kvq_side& a, const kvq_side& b) { return memcmp(&a, &b, sizeof(kvq_side)) == 0; }
+
+kvq_status check_config(const kvq_config* c, const HeadSides& sides) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->n_layers > 64) return KVQ_ERR_INVALID_ARG;
   if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return KVQ_ERR_INVALID_ARG;
@@ -112,14 +136,13 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
   if (c->capacity < 1 || c->capacity > (1 << 26)) return KVQ_ERR_INVALID_ARG;
   if (c->max_queries < 1) return KVQ_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || isinf(c->sm_scale)) return KVQ_ERR_INVALID_ARG;
-  for (int l = 0; l < (lk ? c->n_layers : 1); ++l) {
-    const kvq_status st = check_side(*c, lk ? lk[l] : c->k, true);
-    if (st != KVQ_OK) return st;
-  }
-  for (int l = 0; l < (lv ? c->n_layers : 1); ++l) {
-    const kvq_status st = check_side(*c, lv ? lv[l] : c->v, false);
-    if (st != KVQ_OK) return st;
-  }
+  const int H = c->n_kv_heads;
+  for (int sd = 0; sd < 2; ++sd)
+    for (int l = 0; l < c->n_layers; ++l)
+      for (int h = 0; h < H; ++h) {
+        const kvq_status st = check_side(*c, sides.at(sd, l, h, H), sd == 0);
+        if (st != KVQ_OK) return st;
+      }
   if (c->anchor_rule < KVQ_ANCHOR_NONE || c->anchor_rule > KVQ_ANCHOR_ALL) return KVQ_ERR_INVALID_ARG;
   if (c->n_layers < 64 && (c->anchor_layer_mask >> c->n_layers)) return KVQ_ERR_INVALID_ARG;
   if (c->anchor_rule == KVQ_ANCHOR_FIRST_N || c->anchor_rule == KVQ_ANCHOR_WINDOW) {
@@ -130,12 +153,13 @@ kvq_status check_config(const kvq_config* c, const kvq_side* lk, const kvq_side*
   if (c->anchor_bits == 8 || c->anchor_bits == 4) {  // anchors are quantized by the row kernels
     for (int l = 0; l < c->n_layers; ++l) {
       if (c->anchor_rule == KVQ_ANCHOR_NONE || !((c->anchor_layer_mask >> l) & 1ULL)) continue;
-      for (int sd = 0; sd < 2; ++sd) {
-        const kvq_side& x = sd == 0 ? (lk ? lk[l] : c->k) : (lv ? lv[l] : c->v);
-        if (x.format == KVQ_FMT_FP16 || x.format == KVQ_FMT_POLAR || x.format == KVQ_FMT_CART ||
-            x.format == KVQ_FMT_SORTED)
-          return KVQ_ERR_UNSUPPORTED;
-      }
+      for (int sd = 0; sd < 2; ++sd)
+        for (int h = 0; h < H; ++h) {
+          const kvq_side& x = sides.at(sd, l, h, H);
+          if (x.format == KVQ_FMT_FP16 || x.format == KVQ_FMT_POLAR || x.format == KVQ_FMT_CART ||
+              x.format == KVQ_FMT_SORTED)
+            return KVQ_ERR_UNSUPPORTED;
+        }
     }
   }
   return KVQ_OK;
@@ -169,58 +193,73 @@ bool layer_anchored(const kvq_config& c, int l) {
   return c.anchor_rule != KVQ_ANCHOR_NONE && ((c.anchor_layer_mask >> l) & 1ULL);
 }
 
-// Lay out the arena; fills `h` offsets if non-null.  Returns total bytes.
-uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
-  const int D = c.head_dim;
+// Lay out the arena; fills `h` (head groups and offsets) if non-null.  Returns total bytes.
+uint64_t layout(const kvq_config& c, const HeadSides& sides, kvq_cache* h) {
+  const int D = c.head_dim, H = c.n_kv_heads;
   const int Tcap = (c.capacity + 255) / 256 * 256;  // whole 256-token decode tiles
-  const uint64_t units = (uint64_t)c.batch * c.n_kv_heads;
   const int anchor_rows = c.anchor_rule == KVQ_ANCHOR_ALL ? Tcap : c.anchor_n;
   uint64_t off = 0;
   for (int l = 0; l < c.n_layers; ++l) {
-    for (int s = 0; s < 2; ++s) {
-      const kvq_side& sd = sides.s[l][s];
-      int rb, ng;
-      side_geometry(D, sd, &rb, &ng);
-      kvq_cache::SideOff so{};
-      so.row_bytes = rb;
-      so.n_groups = ng;
-      so.codes = (int64_t)off;
-      off = align_up(off + units * Tcap * (uint64_t)rb);
-      so.scales = -1;
-      if (ng) {
-        so.scales = (int64_t)off;
-        off = align_up(off + units * Tcap * (uint64_t)ng * 2);
-      }
-      so.zeros = -1;
-      if (has_zero_points(sd)) {
-        so.zeros = (int64_t)off;
-        off = align_up(off + units * Tcap * (uint64_t)ng * 2);
-      }
-      so.anchors = -1;
-      so.anchor_scales = -1;
-      if (layer_anchored(c, l)) {
-        const int ab = anchor_bits_of(c);
-        so.anchors = (int64_t)off;
-        off = align_up(off + units * (uint64_t)anchor_rows * D * ab / 8);
-        if (ab != 16) {
-          so.anchor_scales = (int64_t)off;
-          off = align_up(off + units * (uint64_t)anchor_rows * (D / 32) * 2);
+    std::vector<HeadGroup> groups;
+    for (int hh = 0; hh < H;) {  // maximal runs of heads with equal (K, V) formats
+      HeadGroup g{};
+      g.h0 = hh;
+      g.side[0] = sides.at(0, l, hh, H);
+      g.side[1] = sides.at(1, l, hh, H);
+      int e = hh + 1;
+      while (e < H && same_side(sides.at(0, l, e, H), g.side[0]) && same_side(sides.at(1, l, e, H), g.side[1])) ++e;
+      g.nh = e - hh;
+      hh = e;
+      const uint64_t units = (uint64_t)c.batch * g.nh;
+      for (int s = 0; s < 2; ++s) {
+        const kvq_side& sd = g.side[s];
+        int rb, ng;
+        side_geometry(D, sd, &rb, &ng);
+        SideOff& so = g.off[s];
+        so.row_bytes = rb;
+        so.n_groups = ng;
+        so.codes = (int64_t)off;
+        off = align_up(off + units * Tcap * (uint64_t)rb);
+        so.scales = -1;
+        if (ng) {
+          so.scales = (int64_t)off;
+          off = align_up(off + units * Tcap * (uint64_t)ng * 2);
+        }
+        so.zeros = -1;
+        if (has_zero_points(sd)) {
+          so.zeros = (int64_t)off;
+          off = align_up(off + units * Tcap * (uint64_t)ng * 2);
+        }
+        so.anchors = -1;
+        so.anchor_scales = -1;
+        if (layer_anchored(c, l)) {
+          const int ab = anchor_bits_of(c);
+          so.anchors = (int64_t)off;
+          off = align_up(off + units * (uint64_t)anchor_rows * D * ab / 8);
+          if (ab != 16) {
+            so.anchor_scales = (int64_t)off;
+            off = align_up(off + units * (uint64_t)anchor_rows * (D / 32) * 2);
+          }
         }
       }
-      if (h) h->off[l][s] = so;
+      g.kmean = -1;
+      if (g.side[0].mean_sub) {
+        g.kmean = (int64_t)off;
+        off = align_up(off + units * D * 2);
+      }
+      groups.push_back(g);
     }
+    bool any_chan = false;
+    for (const HeadGroup& g : groups) any_chan |= g.side[0].chan_scale != 0;
     int64_t ch = -1;
-    if (sides.s[l][0].chan_scale) {
+    if (any_chan) {
       ch = (int64_t)off;
-      off = align_up(off + (uint64_t)c.n_kv_heads * D * 2);
+      off = align_up(off + (uint64_t)H * D * 2);
     }
-    if (h) h->chan[l] = ch;
-    int64_t km = -1;
-    if (sides.s[l][0].mean_sub) {
-      km = (int64_t)off;
-      off = align_up(off + units * D * 2);
+    if (h) {
+      h->grp[l] = groups;
+      h->chan[l] = ch;
     }
-    if (h) h->kmean[l] = km;
   }
   const int64_t lens = (int64_t)off;
   off = align_up(off + (uint64_t)c.n_layers * c.batch * 4);
@@ -238,20 +277,25 @@ uint64_t layout(const kvq_config& c, const LayerSides& sides, kvq_cache* h) {
   return off;
 }
 
-LayerDev layer_dev(const kvq_cache* h, int l) {
+// Device view of head group gi of layer l.
+LayerDev layer_dev(const kvq_cache* h, int l, int gi) {
   LayerDev L{};
   const kvq_config& c = h->cfg;
+  const HeadGroup& g = h->grp[l][gi];
+  const int D = c.head_dim;
   for (int s = 0; s < 2; ++s) {
-    const kvq_side& sd = h->side[l][s];
-    const kvq_cache::SideOff& so = h->off[l][s];
+    const kvq_side& sd = g.side[s];
+    const SideOff& so = g.off[s];
     SideDev& S = L.s[s];
     S.codes = reinterpret_cast<uint8_t*>(h->arena + so.codes);
     S.scales = so.scales >= 0 ? reinterpret_cast<__half*>(h->arena + so.scales) : nullptr;
     S.zeros = so.zeros >= 0 ? reinterpret_cast<__half*>(h->arena + so.zeros) : nullptr;
     S.anchors = so.anchors >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchors) : nullptr;
     S.anchor_scales = so.anchor_scales >= 0 ? reinterpret_cast<__half*>(h->arena + so.anchor_scales) : nullptr;
-    S.chan = (s == 0 && h->chan[l] >= 0) ? reinterpret_cast<const __half*>(h->arena + h->chan[l]) : nullptr;
-    S.kmean = (s == 0 && h->kmean[l] >= 0) ? reinterpret_cast<__half*>(h->arena + h->kmean[l]) : nullptr;
+    S.chan = (s == 0 && sd.chan_scale && h->chan[l] >= 0)
+                 ? reinterpret_cast<const __half*>(h->arena + h->chan[l]) + (size_t)g.h0 * D
+                 : nullptr;
+    S.kmean = (s == 0 && g.kmean >= 0) ? reinterpret_cast<__half*>(h->arena + g.kmean) : nullptr;
     S.mean_sub = s == 0 ? sd.mean_sub : 0;
     S.fmt = sd.format;
     S.bits = sd.bits;
@@ -263,14 +307,17 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
     S.row_bytes = so.row_bytes;
     S.n_groups = so.n_groups;
   }
+  const int G = c.n_q_heads / c.n_kv_heads;
   L.B = c.batch;
   L.cap = c.capacity;
   L.app_ids = nullptr;
   L.app_n = c.batch;
   L.test_stall = h->test_stall;
-  L.Hkv = c.n_kv_heads;
-  L.Hq = c.n_q_heads;
-  L.D = c.head_dim;
+  L.Hkv = g.nh;
+  L.Hq = g.nh * G;
+  L.Hkv_all = c.n_kv_heads;
+  L.h0 = g.h0;
+  L.D = D;
   L.Tcap = h->Tcap;
   L.anchored = layer_anchored(c, l) ? 1 : 0;
   L.anchor_rule = c.anchor_rule;
@@ -283,6 +330,12 @@ LayerDev layer_dev(const kvq_cache* h, int l) {
   L.err = reinterpret_cast<unsigned*>(h->arena + h->err);
   L.sm_scale = c.sm_scale > 0.0f ? c.sm_scale : (float)(1.0 / sqrt((double)c.head_dim));
   return L;
+}
+
+bool layer_needs_chan(const kvq_cache* h, int l) {
+  for (const HeadGroup& g : h->grp[l])
+    if (g.side[0].chan_scale) return true;
+  return false;
 }
 
 // ----------------------------------------------------------------------------- host tables
@@ -411,13 +464,24 @@ kvq_status kvq_lloyd_levels(int32_t bits, float* out) {
   return KVQ_OK;
 }
 
+kvq_status kvq_arena_bytes_heads(const kvq_config* cfg, const kvq_side* head_k, const kvq_side* head_v,
+                                 uint64_t* bytes) {
+  if (!bytes) return KVQ_ERR_INVALID_ARG;
+  HeadSides sides;
+  if (!fill_sides(cfg, nullptr, nullptr, head_k, head_v, &sides)) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = check_config(cfg, sides);
+  if (st != KVQ_OK) return st;
+  *bytes = layout(*cfg, sides, nullptr);
+  return KVQ_OK;
+}
+
 kvq_status kvq_arena_bytes_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v,
                                   uint64_t* bytes) {
   if (!bytes) return KVQ_ERR_INVALID_ARG;
-  const kvq_status st = check_config(cfg, layer_k, layer_v);
+  HeadSides sides;
+  if (!fill_sides(cfg, layer_k, layer_v, nullptr, nullptr, &sides)) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = check_config(cfg, sides);
   if (st != KVQ_OK) return st;
-  LayerSides sides{};
-  fill_sides(*cfg, layer_k, layer_v, &sides);
   *bytes = layout(*cfg, sides, nullptr);
   return KVQ_OK;
 }
@@ -426,21 +490,16 @@ kvq_status kvq_arena_bytes(const kvq_config* cfg, uint64_t* bytes) {
   return kvq_arena_bytes_layers(cfg, nullptr, nullptr, bytes);
 }
 
-kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
-                             uint64_t arena_bytes, kvq_cache** out) {
-  if (!out) return KVQ_ERR_INVALID_ARG;
-  *out = nullptr;
-  kvq_status st = check_config(cfg, layer_k, layer_v);
+static kvq_status create_impl(const kvq_config* cfg, const HeadSides& sides, void* arena, uint64_t arena_bytes,
+                              kvq_cache** out) {
+  kvq_status st = check_config(cfg, sides);
   if (st != KVQ_OK) return st;
   if (!arena || (reinterpret_cast<uintptr_t>(arena) % kAlign)) return KVQ_ERR_INVALID_ARG;
-  LayerSides sides{};
-  fill_sides(*cfg, layer_k, layer_v, &sides);
   const uint64_t need = layout(*cfg, sides, nullptr);
   if (arena_bytes < need) return KVQ_ERR_ALLOC;
   kvq_cache* h = new (std::nothrow) kvq_cache();
   if (!h) return KVQ_ERR_ALLOC;
   h->cfg = *cfg;
-  memcpy(h->side, sides.s, sizeof(h->side));
   h->arena = reinterpret_cast<char*>(arena);
   h->arena_bytes = arena_bytes;
   layout(*cfg, sides, h);
@@ -468,15 +527,16 @@ kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, con
     delete h;
     return KVQ_ERR_CUDA;
   }
-  // workspace for the largest split-K grid any n_q <= max_queries can use
+  // workspace for the largest split-K grid any head group and any n_q <= max_queries can use
   size_t wf = 0;
-  for (int l = 0; l < cfg->n_layers; ++l) {
-    const LayerDev L = layer_dev(h, l);
-    for (int nq = 1; nq <= cfg->max_queries; ++nq) {
-      const size_t f = (size_t)nq * cfg->n_q_heads * decode_partials(L, nq, h->num_sms) * (cfg->head_dim + kPartStride);
-      wf = f > wf ? f : wf;
+  for (int l = 0; l < cfg->n_layers; ++l)
+    for (int gi = 0; gi < (int)h->grp[l].size(); ++gi) {
+      const LayerDev L = layer_dev(h, l, gi);
+      for (int nq = 1; nq <= cfg->max_queries; ++nq) {
+        const size_t f = (size_t)nq * L.Hq * decode_partials(L, nq, h->num_sms) * (cfg->head_dim + kPartStride);
+        wf = f > wf ? f : wf;
+      }
     }
-  }
   h->work_floats = wf;
   if (cudaMalloc(&h->work, wf * sizeof(float)) != cudaSuccess) {
     cudaGetLastError();
@@ -494,6 +554,24 @@ kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, con
   return KVQ_OK;
 }
 
+kvq_status kvq_create_heads(const kvq_config* cfg, const kvq_side* head_k, const kvq_side* head_v, void* arena,
+                            uint64_t arena_bytes, kvq_cache** out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  HeadSides sides;
+  if (!fill_sides(cfg, nullptr, nullptr, head_k, head_v, &sides)) return KVQ_ERR_INVALID_ARG;
+  return create_impl(cfg, sides, arena, arena_bytes, out);
+}
+
+kvq_status kvq_create_layers(const kvq_config* cfg, const kvq_side* layer_k, const kvq_side* layer_v, void* arena,
+                             uint64_t arena_bytes, kvq_cache** out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  HeadSides sides;
+  if (!fill_sides(cfg, layer_k, layer_v, nullptr, nullptr, &sides)) return KVQ_ERR_INVALID_ARG;
+  return create_impl(cfg, sides, arena, arena_bytes, out);
+}
+
 kvq_status kvq_create(const kvq_config* cfg, void* arena, uint64_t arena_bytes, kvq_cache** out) {
   return kvq_create_layers(cfg, nullptr, nullptr, arena, arena_bytes, out);
 }
@@ -504,22 +582,33 @@ void kvq_free(kvq_cache* h) {
   delete h;
 }
 
-kvq_status kvq_get_layout(const kvq_cache* h, int32_t layer, int32_t side, kvq_layout* out) {
-  if (!h || !out || layer < 0 || layer >= h->cfg.n_layers || (side != 0 && side != 1)) return KVQ_ERR_INVALID_ARG;
-  const kvq_cache::SideOff& so = h->off[layer][side];
+kvq_status kvq_get_layout_head(const kvq_cache* h, int32_t layer, int32_t side, int32_t head, kvq_layout* out) {
+  if (!h || !out || layer < 0 || layer >= h->cfg.n_layers || (side != 0 && side != 1) || head < 0 ||
+      head >= h->cfg.n_kv_heads)
+    return KVQ_ERR_INVALID_ARG;
+  const HeadGroup* g = nullptr;
+  for (const HeadGroup& x : h->grp[layer])
+    if (head >= x.h0 && head < x.h0 + x.nh) g = &x;
+  const SideOff& so = g->off[side];
   out->codes = so.codes;
   out->scales = so.scales;
   out->zeros = so.zeros;
   out->anchors = so.anchors;
   out->chan_scale = side == 0 ? h->chan[layer] : -1;
-  out->key_mean = side == 0 ? h->kmean[layer] : -1;
-  out->anchor_scales = so.anchor_scales;
   out->seq_len = h->lens + (int64_t)layer * h->cfg.batch * 4;
+  out->key_mean = side == 0 ? g->kmean : -1;
+  out->anchor_scales = so.anchor_scales;
   out->row_bytes = so.row_bytes;
   out->n_groups = so.n_groups;
   out->row_stride_tokens = h->Tcap;
   out->anchor_rows = so.anchors >= 0 ? h->anchor_rows : 0;
+  out->head0 = g->h0;
+  out->n_heads = g->nh;
   return KVQ_OK;
+}
+
+kvq_status kvq_get_layout(const kvq_cache* h, int32_t layer, int32_t side, kvq_layout* out) {
+  return kvq_get_layout_head(h, layer, side, 0, out);
 }
 
 kvq_status kvq_set_chan_scale(kvq_cache* h, int32_t layer, const void* c, void* stream) {
@@ -556,27 +645,36 @@ kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const
                                int32_t n_seqs, int32_t n_new, void* stream) {
   if (!h || !k || !v || layer < 0 || layer >= h->cfg.n_layers || n_new < 1) return KVQ_ERR_INVALID_ARG;
   if (seq_ids ? (n_seqs < 1 || n_seqs > h->cfg.batch) : n_seqs != h->cfg.batch) return KVQ_ERR_INVALID_ARG;
-  if (h->side[layer][0].chan_scale && !h->chan_set[layer]) return KVQ_ERR_STATE;
+  if (layer_needs_chan(h, layer) && !h->chan_set[layer]) return KVQ_ERR_STATE;
   if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
   if (n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
   // every sequence advances together: the host bound is exact and decides; otherwise the device
   // checks each listed sequence
   if (!seq_ids && h->len_exact[layer] && (int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
   if ((int64_t)n_seqs * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
-  LayerDev L = layer_dev(h, layer);
-  L.app_ids = seq_ids;
-  L.app_n = n_seqs;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int ng = (int)h->grp[layer].size();
+  std::vector<LayerDev> views(ng);
+  unsigned total = 0;  // every view's CTAs take a ticket; the last one advances the lengths
+  for (int gi = 0; gi < ng; ++gi) {
+    views[gi] = layer_dev(h, layer, gi);
+    views[gi].app_ids = seq_ids;
+    views[gi].app_n = n_seqs;
+    total += append_ctas(views[gi], n_new);
+  }
   int launches = 0;
   cudaError_t e = cudaSuccess;
-  if (L.s[0].mean_sub) {  // key means of the sequences this append starts, before their rows
-    e = launch_key_mean(L, reinterpret_cast<const __half*>(k), n_new, reinterpret_cast<cudaStream_t>(stream));
-    ++launches;
-  }
-  if (e == cudaSuccess) {
-    int n = 0;
-    e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new,
-                      reinterpret_cast<cudaStream_t>(stream), &n);
-    launches += n;
+  for (int gi = 0; gi < ng && e == cudaSuccess; ++gi) {
+    const LayerDev& L = views[gi];
+    if (L.s[0].mean_sub) {  // key means of the sequences this append starts, before their rows
+      e = launch_key_mean(L, reinterpret_cast<const __half*>(k), n_new, st);
+      ++launches;
+    }
+    if (e == cudaSuccess) {
+      int n = 0;
+      e = launch_append(L, reinterpret_cast<const __half*>(k), reinterpret_cast<const __half*>(v), n_new, total, st, &n);
+      launches += n;
+    }
   }
   h->last_launches = launches;
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
@@ -591,9 +689,35 @@ kvq_status kvq_dequantize(const kvq_cache* h, int32_t layer, int32_t side, int32
   if (!h || !out || layer < 0 || layer >= h->cfg.n_layers || (side != 0 && side != 1)) return KVQ_ERR_INVALID_ARG;
   if (domain != KVQ_DOMAIN_STORED && domain != KVQ_DOMAIN_ORIGINAL) return KVQ_ERR_INVALID_ARG;
   if (t0 < 0 || nt < 1 || (int64_t)t0 + nt > h->cfg.capacity) return KVQ_ERR_INVALID_ARG;
-  const LayerDev L = layer_dev(h, layer);
-  const cudaError_t e = launch_dequant(L, side, domain, t0, nt, out, out_fp32 ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  for (int gi = 0; gi < (int)h->grp[layer].size(); ++gi) {
+    const LayerDev L = layer_dev(h, layer, gi);
+    const cudaError_t e =
+        launch_dequant(L, side, domain, t0, nt, out, out_fp32 ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
+}
+
+// Decode every head group of `layer` with `work` as the split-K scratch (the groups run one after
+// another on the stream, so they share it).
+static kvq_status decode_groups(kvq_cache* h, int32_t layer, const void* q, int32_t n_q, const int32_t* seq_ids,
+                                const int32_t* kv_len, void* out, int32_t out_fp32, float* lse, float* work,
+                                void* stream) {
+  int launches = 0;
+  for (int gi = 0; gi < (int)h->grp[layer].size(); ++gi) {
+    const LayerDev L = layer_dev(h, layer, gi);
+    int n = 0;
+    const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_q, seq_ids, kv_len, out,
+                                        out_fp32 ? 1 : 0, lse, work, h->num_sms, h->cfg.max_queries,
+                                        reinterpret_cast<cudaStream_t>(stream), &n);
+    launches += n;
+    if (e != cudaSuccess) {
+      h->last_launches = launches;
+      return KVQ_ERR_CUDA;
+    }
+  }
+  h->last_launches = launches;
+  return KVQ_OK;
 }
 
 kvq_status kvq_decode_attention(kvq_cache* h, int32_t layer, const void* q, int32_t n_q, const int32_t* seq_ids,
@@ -601,13 +725,7 @@ kvq_status kvq_decode_attention(kvq_cache* h, int32_t layer, const void* q, int3
   if (!h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || n_q < 1) return KVQ_ERR_INVALID_ARG;
   if (n_q > h->cfg.max_queries) return KVQ_ERR_CAPACITY;
   if (!seq_ids && n_q > h->cfg.batch) return KVQ_ERR_INVALID_ARG;
-  const LayerDev L = layer_dev(h, layer);
-  int launches = 0;
-  const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_q, seq_ids, kv_len, out, out_fp32 ? 1 : 0,
-                                      lse, h->work, h->num_sms, h->cfg.max_queries,
-                                      reinterpret_cast<cudaStream_t>(stream), &launches);
-  h->last_launches = launches;
-  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  return decode_groups(h, layer, q, n_q, seq_ids, kv_len, out, out_fp32, lse, h->work, stream);
 }
 
 // Same computation as kvq_decode_attention; the split-K partials go to the library's fixed
@@ -621,18 +739,16 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* h, int32_t layer, const void*
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   if (dev != h->device) return KVQ_ERR_INVALID_ARG;
-  const LayerDev L = layer_dev(h, layer);
-  const size_t need =
-      (size_t)n_q * h->cfg.n_q_heads * decode_partials(L, n_q, h->num_sms) * (h->cfg.head_dim + kPartStride);
+  size_t need = 0;
+  for (int gi = 0; gi < (int)h->grp[layer].size(); ++gi) {
+    const LayerDev L = layer_dev(h, layer, gi);
+    const size_t f = (size_t)n_q * L.Hq * decode_partials(L, n_q, h->num_sms) * (h->cfg.head_dim + kPartStride);
+    need = f > need ? f : need;
+  }
   if (need > static_work_floats()) return KVQ_ERR_CAPACITY;
   float* ws = nullptr;
   if (static_work_ptr(dev, &ws) != cudaSuccess) return KVQ_ERR_CUDA;
-  int launches = 0;
-  const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_q, seq_ids, kv_len, out, out_fp32 ? 1 : 0,
-                                      lse, ws, h->num_sms, h->cfg.max_queries, reinterpret_cast<cudaStream_t>(stream),
-                                      &launches);
-  h->last_launches = launches;
-  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  return decode_groups(h, layer, q, n_q, seq_ids, kv_len, out, out_fp32, lse, ws, stream);
 }
 
 kvq_status kvq_error_flags(kvq_cache* h, int32_t* flags) {

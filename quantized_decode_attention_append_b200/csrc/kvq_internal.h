@@ -25,10 +25,14 @@ struct SideDev {
   int row_bytes, n_groups;
 };
 
-// Device view of one layer.
+// Device view of the kv-heads [h0, h0 + Hkv) of one layer that share one (K, V) format pair (all of
+// its heads unless the layer has per-head formats).  Arena regions are the view's own: unit
+// u = b * Hkv + local head.  The caller's arrays (queries, outputs, append inputs, dequantized
+// rows) hold all Hkv_all heads of the layer.
 struct LayerDev {
   SideDev s[2];
   int B, Hkv, Hq, D, Tcap;
+  int Hkv_all, h0;       // kv-heads of the layer; first kv-head of this view
   int cap;               // configured capacity (tokens per sequence); appends never pass it
   int anchored;          // this layer keeps anchor rows
   int anchor_rule, anchor_n, anchor_rows;
@@ -43,6 +47,19 @@ struct LayerDev {
   long long test_stall;  // test hook (0 = off): the decode's first stage wait polls a barrier nothing
                          // arrives on for this many clock cycles, then gives up
 };
+
+// Row of query head h (of kv-head kvh of the view, G query heads per kv-head) of query qi in the
+// caller's [n_q][Hq_all][..] arrays.
+__device__ __forceinline__ long long query_row(const LayerDev& L, int qi, int kvh, int G, int h) {
+  return ((long long)qi * L.Hkv_all + L.h0 + kvh) * G + h;
+}
+
+// Caller row ([n_seqs][Hkv_all][n_new] order) of the view's append row `row` ([n_seqs][Hkv][n_new]).
+__device__ __forceinline__ long long input_row(const LayerDev& L, long long row, int n_new) {
+  if (L.Hkv == L.Hkv_all) return row;
+  const long long ul = row / n_new, sl = ul / L.Hkv;
+  return (sl * L.Hkv_all + L.h0 + (ul - sl * L.Hkv)) * n_new + (row - ul * n_new);
+}
 
 // Tables the host builds once (NF4 levels, FFT twiddles, phase cos/sin) and every
 // translation unit uploads into its own constant memory.
@@ -63,8 +80,11 @@ cudaError_t upload_tables_decode(const HostTables& t);
 cudaError_t upload_tables_dequant(const HostTables& t);
 
 // Launchers (host side, validate nothing; the API validates first).
-cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, cudaStream_t st,
-                          int* launches);
+// CTAs launch_append starts for `L` (the completion ticket of one append counts the CTAs of every
+// view of the layer: total_ctas).
+unsigned append_ctas(const LayerDev& L, int n_new);
+cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, unsigned total_ctas,
+                          cudaStream_t st, int* launches);
 cudaError_t launch_dequant(const LayerDev& L, int side, int domain, int t0, int nt, void* out,
                            int out_fp32, cudaStream_t st);
 cudaError_t launch_decode(const LayerDev& L, const __half* q, int n_q, const int* seq_ids,

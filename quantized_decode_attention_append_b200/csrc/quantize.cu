@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
   const int pos = dst.pos, len_after = dst.len_after, u = dst.u;
   if (!ok && dst.first && lane == 0) atomicOr(L.err, dst.err);
   if (ok) {
-    const __half* rp = src + row * 128;
+    const __half* rp = src + input_row(L, row, n_new) * 128;
     float* re = sre[warp];
     float* im = sim[warp];
     for (int j = lane; j < 128; j += 32) {
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(128) append_sorted_kernel(LayerDev L, int side
       if (dst.first && lane == 0) atomicOr(L.err, dst.err);
       continue;
     }
-    const __half* rp = src + row * D;
+    const __half* rp = src + input_row(L, row, n_new) * D;
     float* x = sx[warp];
     for (int j = lane; j < D; j += 32) {
       float v = __half2float(rp[j]);
@@ -576,7 +576,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   {
     const long long r0 = (long long)(bid * NW + warp) * rpw + lane / lpr;
     if (r0 < R) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + r0 * D + li * 32);
+      const uint4* p = reinterpret_cast<const uint4*>(src + input_row(L, r0, n_new) * D + li * 32);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
     }
@@ -589,7 +589,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     {
       const long long rn = (long long)row + stride;
       if (rn < R) {
-        const uint4* p = reinterpret_cast<const uint4*>(src + rn * D + li * 32);
+        const uint4* p = reinterpret_cast<const uint4*>(src + input_row(L, rn, n_new) * D + li * 32);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
       }
@@ -968,10 +968,10 @@ __global__ void __launch_bounds__(kRowThreads) append_rows_kernel(LayerDev L, in
 template <int FK, int GK, int BK, int FV, int GV, int BV>
 __global__ void __launch_bounds__(kRowThreads) append_kv_kernel(LayerDev L, const __half* __restrict__ k,
                                                                 const __half* __restrict__ v, int n_new,
-                                                                unsigned kblocks) {
+                                                                unsigned kblocks, unsigned total_ctas) {
   if (blockIdx.x < kblocks) rows_body<FK, GK, BK>(L, 0, k, n_new, blockIdx.x, kblocks);
   else rows_body<FV, GV, BV>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
-  finish_append(L, n_new, gridDim.x);
+  finish_append(L, n_new, total_ctas);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1041,7 +1041,7 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
   const int c = (int)(gt % vec_per_row);
   const RowDst d = row_dst(L, (int)row, n_new);
   if (d.err == 0) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + row * L.D) + c);
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + input_row(L, row, n_new) * L.D) + c);
     reinterpret_cast<uint4*>(S.codes + ((long long)d.u * L.Tcap + d.pos) * S.row_bytes)[c] = w;
     if (in_anchor(L, d.pos, d.len_after))
       reinterpret_cast<uint4*>(S.anchors + ((long long)d.u * L.anchor_rows + anchor_slot(L, d.pos)) * L.D)[c] = w;
@@ -1063,7 +1063,7 @@ __global__ void __launch_bounds__(kMeanThreads) key_mean_kernel(LayerDev L, cons
   const int b = L.app_ids ? L.app_ids[sl] : sl;
   if (b < 0 || b >= L.B || L.seq_len[b] != 0) return;  // not this sequence's first append
   const int D = L.D, j = threadIdx.x % D, r0 = threadIdx.x / D, nr = kMeanThreads / D;
-  const __half* src = k + (long long)ul * n_new * D;
+  const __half* src = k + input_row(L, (long long)ul * n_new, n_new) * D;
   long long acc = 0;
   for (int i = r0; i < n_new; i += nr) acc += __float2ll_rn(__fmul_rn(__half2float(src[(long long)i * D + j]), 16777216.0f));
   __shared__ long long part[kMeanThreads];
@@ -1116,7 +1116,7 @@ static SidePlan plan_side(const LayerDev& L, int side, int n_new) {
   return p;
 }
 
-typedef void (*KvKernel)(LayerDev, const __half*, const __half*, int, unsigned);
+typedef void (*KvKernel)(LayerDev, const __half*, const __half*, int, unsigned, unsigned);
 
 // The (K, V) format pairs that have a single-launch append kernel.
 static KvKernel pick_kv_kernel(const LayerDev& L) {
@@ -1145,13 +1145,16 @@ static KvKernel pick_kv_kernel(const LayerDev& L) {
   return nullptr;
 }
 
-cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, cudaStream_t st,
-                          int* launches) {
+unsigned append_ctas(const LayerDev& L, int n_new) {
+  return plan_side(L, 0, n_new).blocks + plan_side(L, 1, n_new).blocks;
+}
+
+cudaError_t launch_append(const LayerDev& L, const __half* k, const __half* v, int n_new, unsigned total,
+                          cudaStream_t st, int* launches) {
   const SidePlan pk = plan_side(L, 0, n_new), pv = plan_side(L, 1, n_new);
   if (!pk.kern || !pv.kern) return cudaErrorInvalidValue;
-  const unsigned total = pk.blocks + pv.blocks;
   if (KvKernel kv = pick_kv_kernel(L)) {
-    kv<<<total, kRowThreads, 0, st>>>(L, k, v, n_new, pk.blocks);
+    kv<<<pk.blocks + pv.blocks, kRowThreads, 0, st>>>(L, k, v, n_new, pk.blocks, total);
     if (launches) *launches = 1;
     return cudaGetLastError();
   }

@@ -41,10 +41,12 @@ class kvq_layout(C.Structure):
     _fields_ = [("codes", C.c_int64), ("scales", C.c_int64), ("zeros", C.c_int64), ("anchors", C.c_int64),
                 ("chan_scale", C.c_int64), ("seq_len", C.c_int64), ("key_mean", C.c_int64), ("anchor_scales", C.c_int64),
                 ("row_bytes", C.c_int32),
-                ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32)]
+                ("n_groups", C.c_int32), ("row_stride_tokens", C.c_int32), ("anchor_rows", C.c_int32),
+                ("head0", C.c_int32), ("n_heads", C.c_int32)]
 
 
-EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_arena_bytes_layers", "kvq_create_layers", "kvq_free", "kvq_get_layout", "kvq_set_chan_scale", "kvq_set_seq_len",
+EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_arena_bytes_layers", "kvq_create_layers", "kvq_arena_bytes_heads",
+           "kvq_create_heads", "kvq_free", "kvq_get_layout", "kvq_get_layout_head", "kvq_set_chan_scale", "kvq_set_seq_len",
            "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_decode_attention_noalloc",
            "kvq_error_flags", "kvq_nf4_levels", "kvq_lloyd_levels",
            "kvq_last_launch_count", "kvq_status_str"]
@@ -65,6 +67,9 @@ def lib() -> C.CDLL:
         sp = C.POINTER(kvq_side)
         L.kvq_arena_bytes_layers.argtypes = [C.POINTER(kvq_config), sp, sp, u64p]
         L.kvq_create_layers.argtypes = [C.POINTER(kvq_config), sp, sp, vp, C.c_uint64, C.POINTER(vp)]
+        L.kvq_arena_bytes_heads.argtypes = [C.POINTER(kvq_config), sp, sp, u64p]
+        L.kvq_create_heads.argtypes = [C.POINTER(kvq_config), sp, sp, vp, C.c_uint64, C.POINTER(vp)]
+        L.kvq_get_layout_head.argtypes = [vp, i32, i32, i32, C.POINTER(kvq_layout)]
         L.kvq_free.argtypes = [vp]
         L.kvq_free.restype = None
         L.kvq_get_layout.argtypes = [vp, i32, i32, C.POINTER(kvq_layout)]
@@ -145,11 +150,26 @@ class Config:
     layer_k: tuple = ()  # per-layer K formats (n_layers Sides); empty: k on every layer
     layer_v: tuple = ()  # per-layer V formats; empty: v on every layer
     anchor_bits: int = 16  # anchored rows as fp16 (16) or on an 8/4-bit grid in groups of 32
+    head_k: tuple = ()   # per-(layer, kv-head) K formats: n_layers tuples of n_kv_heads Sides; empty: per layer
+    head_v: tuple = ()   # per-(layer, kv-head) V formats
 
-    def side(self, layer: int, side: int) -> Side:
-        """Format of (layer, side)."""
+    def side(self, layer: int, side: int, head: int = 0) -> Side:
+        """Format of (layer, side) for kv-head `head`."""
+        ph = self.head_k if side == SIDE_K else self.head_v
+        if ph:
+            return ph[layer][head]
         per = self.layer_k if side == SIDE_K else self.layer_v
         return per[layer] if per else (self.k if side == SIDE_K else self.v)
+
+    def head_arrays(self):
+        """(head_k, head_v) as flat layer-major C arrays of kvq_side (every (layer, head) filled)."""
+        n = self.n_layers * self.n_kv_heads
+        out = []
+        for sd in (SIDE_K, SIDE_V):
+            arr = (kvq_side * n)(*[self.side(l, sd, h).to_c() for l in range(self.n_layers)
+                                   for h in range(self.n_kv_heads)])
+            out.append(arr)
+        return out[0], out[1]
 
     def layer_arrays(self):
         """(layer_k, layer_v) as C arrays of kvq_side, or None where uniform."""
@@ -177,7 +197,10 @@ def kvq_status_str(status: int) -> str:
 def kvq_arena_bytes(cfg: Config) -> int:
     c = cfg.to_c()
     n = C.c_uint64(0)
-    if cfg.layer_k or cfg.layer_v:
+    if cfg.head_k or cfg.head_v:
+        hk, hv = cfg.head_arrays()
+        _check(lib().kvq_arena_bytes_heads(C.byref(c), hk, hv, C.byref(n)), "kvq_arena_bytes_heads")
+    elif cfg.layer_k or cfg.layer_v:
         lk, lv = cfg.layer_arrays()
         _check(lib().kvq_arena_bytes_layers(C.byref(c), lk, lv, C.byref(n)), "kvq_arena_bytes_layers")
     else:
@@ -189,7 +212,10 @@ def kvq_create(cfg: Config, arena) -> C.c_void_p:
     c = cfg.to_c()
     h = C.c_void_p()
     base, nbytes = C.c_void_p(arena.data_ptr()), arena.numel() * arena.element_size()
-    if cfg.layer_k or cfg.layer_v:
+    if cfg.head_k or cfg.head_v:
+        hk, hv = cfg.head_arrays()
+        _check(lib().kvq_create_heads(C.byref(c), hk, hv, base, nbytes, C.byref(h)), "kvq_create_heads")
+    elif cfg.layer_k or cfg.layer_v:
         lk, lv = cfg.layer_arrays()
         _check(lib().kvq_create_layers(C.byref(c), lk, lv, base, nbytes, C.byref(h)), "kvq_create_layers")
     else:
@@ -204,6 +230,12 @@ def kvq_free(h):
 def kvq_get_layout(h, layer: int, side: int) -> kvq_layout:
     out = kvq_layout()
     _check(lib().kvq_get_layout(h, layer, side, C.byref(out)), "kvq_get_layout")
+    return out
+
+
+def kvq_get_layout_head(h, layer: int, side: int, head: int) -> kvq_layout:
+    out = kvq_layout()
+    _check(lib().kvq_get_layout_head(h, layer, side, head, C.byref(out)), "kvq_get_layout_head")
     return out
 
 
@@ -287,15 +319,21 @@ class KVCache:
         except Exception:
             pass
 
-    def layout(self, layer, side):
-        return kvq_get_layout(self.h, layer, side)
+    def layout(self, layer, side, head=0):
+        return kvq_get_layout_head(self.h, layer, side, head)
 
-    def view(self, layer: int, side: int, what: str):
-        """torch views into the arena: codes [B*Hkv, Tcap, row_bytes] uint8, scales/zeros
-        [B*Hkv, Tcap, n_groups] fp16, anchors [B*Hkv, anchor_rows, D] fp16, seq_len [B] int32."""
+    def unit(self, layer: int, b: int, h: int) -> int:
+        """Row of (sequence b, kv-head h) in the views of h's head group."""
+        lo = self.layout(layer, SIDE_K, h)
+        return b * lo.n_heads + (h - lo.head0)
+
+    def view(self, layer: int, side: int, what: str, head: int = 0):
+        """torch views into the arena regions of the head group holding kv-head `head`: codes
+        [B*nh, Tcap, row_bytes] uint8, scales/zeros [B*nh, Tcap, n_groups] fp16, anchors
+        [B*nh, anchor_rows, D] fp16 (or code bytes), key_mean [B*nh, D], seq_len [B] int32."""
         import torch
-        lo = self.layout(layer, side)
-        U = self.cfg.batch * self.cfg.n_kv_heads
+        lo = self.layout(layer, side, head)
+        U = self.cfg.batch * lo.n_heads
         T = lo.row_stride_tokens
         if what == "codes":
             return self.arena[lo.codes:lo.codes + U * T * lo.row_bytes].view(U, T, lo.row_bytes)

@@ -23,7 +23,9 @@ def oracle_spec(cfg: Config) -> OC.Spec:
     return OC.Spec(cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.n_q_heads, cfg.head_dim, oracle_side(cfg.k),
                    oracle_side(cfg.v), frozenset(cfg.anchor_layers), cfg.anchor_rule, cfg.anchor_n,
                    cfg.sm_scale or None, tuple(oracle_side(s) for s in cfg.layer_k),
-                   tuple(oracle_side(s) for s in cfg.layer_v), anchor_bits=cfg.anchor_bits)
+                   tuple(oracle_side(s) for s in cfg.layer_v), anchor_bits=cfg.anchor_bits,
+                   head_k=tuple(tuple(oracle_side(s) for s in row) for row in cfg.head_k),
+                   head_v=tuple(tuple(oracle_side(s) for s in row) for row in cfg.head_v))
 
 
 class Case:
@@ -45,7 +47,7 @@ class Case:
                 V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), list(range(T)), D, "cuda")
             else:
                 K, V = (torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in inputs(l))
-            if cfg.side(l, 0).chan_scale:
+            if any(cfg.side(l, 0, h).chan_scale for h in range(H)):
                 c = (synth.channel_scale(seed, l, H, calib_T, D) if chan is None else
                      torch.from_numpy(np.ascontiguousarray(chan(l), dtype=np.float16))).cuda()
                 self.cache.set_chan_scale(l, c)
@@ -63,22 +65,35 @@ class Case:
 
     def oracle_unit(self, l, b, h):
         c = self.C[l][h] if l in self.C else None
-        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c, layer=l, first_rows=self.first_rows)
+        return OC.quantize_unit(self.spec, self.K[l][b, h], self.V[l][b, h], c, layer=l, first_rows=self.first_rows,
+                                head=h)
+
+    def views(self, l, side, head, names):
+        """Host copies of the arena views of kv-head `head`'s group (None where absent), fetched
+        once per head group."""
+        key = (l, side, self.cache.layout(l, side, head).head0, tuple(names))
+        memo = self.__dict__.setdefault("_views", {})
+        if key not in memo:
+            out = []
+            for w in names:
+                t = self.cache.view(l, side, w, head=head)
+                out.append(None if t is None else t.cpu().numpy())
+            memo[key] = out
+        return memo[key]
+
+    def forget_views(self):
+        self.__dict__.pop("_views", None)
 
     def check_codes(self, l, rows=None):
         """Packed codes, scales and zero points of every unit are bit-identical to the oracle."""
         cfg = self.cfg
+        self.forget_views()
         for side, name in ((0, "k"), (1, "v")):
-            codes = self.cache.view(l, side, "codes").cpu().numpy()
-            scales = self.cache.view(l, side, "scales")
-            zeros = self.cache.view(l, side, "zeros")
-            scales = None if scales is None else scales.cpu().numpy()
-            zeros = None if zeros is None else zeros.cpu().numpy()
-            kmean = self.cache.view(l, 0, "key_mean")
-            kmean = None if kmean is None else kmean.cpu().numpy()
-            for b in range(cfg.batch):
-                for h in range(cfg.n_kv_heads):
-                    u = b * cfg.n_kv_heads + h
+            for h in range(cfg.n_kv_heads):
+                codes, scales, zeros = self.views(l, side, h, ("codes", "scales", "zeros"))
+                (kmean,) = self.views(l, 0, h, ("key_mean",))
+                for b in range(cfg.batch):
+                    u = self.cache.unit(l, b, h)
                     kq, vq = self.oracle_unit(l, b, h)
                     o = kq if side == 0 else vq
                     sel = slice(None) if rows is None else rows
@@ -105,19 +120,19 @@ class Case:
         if not an.any():
             return
         slots = np.arange(self.T)[an] % cfg.anchor_n if cfg.anchor_rule == "window" else np.arange(self.T)[an]
+        self.forget_views()
         for side in (0, 1):
-            codes = self.cache.view(l, side, "anchors").cpu().numpy()
-            sc = self.cache.view(l, side, "anchor_scales")
-            for b in range(cfg.batch):
-                for h in range(cfg.n_kv_heads):
-                    u = b * cfg.n_kv_heads + h
+            for h in range(cfg.n_kv_heads):
+                codes, sc = self.views(l, side, h, ("anchors", "anchor_scales"))
+                for b in range(cfg.batch):
+                    u = self.cache.unit(l, b, h)
                     src = (self.K[l] if side == 0 else self.V[l])[b, h][an]
                     want = OC.anchor_rows(self.spec, src)
                     if cfg.anchor_bits == 16:
                         assert np.array_equal(codes[u, slots].view(np.uint16), src.view(np.uint16))
                     else:
                         assert np.array_equal(codes[u, slots], want["bytes"]), f"anchor codes side {side} u{u}"
-                        assert np.array_equal(sc[u, slots].cpu().numpy().view(np.uint16),
+                        assert np.array_equal(sc[u, slots].view(np.uint16),
                                               want["scales"].view(np.uint16)), f"anchor scales side {side} u{u}"
 
     def check_dequant(self, l):
@@ -132,7 +147,7 @@ class Case:
                     o = kq if side == 0 else vq
                     assert np.array_equal(st[b, h].view(np.uint32), o["stored"].astype(np.float32).view(np.uint32)), \
                         f"stored dequant side {side} l{l} b{b} h{h}"
-                    sd = OC.side_of(self.spec, l, side == 0)
+                    sd = OC.side_of(self.spec, l, side == 0, h)
                     c = self.C[l][h] if (side == 0 and l in self.C) else None
                     mu = o.get("mu")
                     want = OQ.to_original_f64(o["exact"], sd, None if c is None else np.broadcast_to(c, o["exact"].shape),

@@ -258,3 +258,38 @@ def test_sorted_group_configs():
     st4, n4 = status_of(base_cfg(k=Side("int", 2, scale="minmax", group=8), v=Side("int", 2, scale="minmax", group=8)))
     # per row: the same codes and metadata plus 7 x 128 rank bits (112 bytes)
     assert st == 0 and st4 == 0 and n - n4 == pytest.approx(2 * 2 * 4 * 512 * 112, abs=2 * 2 * 3 * 256)
+
+
+def test_head_allocation_matches_the_oracle_rule():
+    """The package's calibration (torch) and the oracle's rule (numpy) agree: entropies of the same
+    attention, bits per head, and the sink heads (llama.cpp #21385 "Finding 2")."""
+    import torch
+    from oracle import attention as OA
+    from oracle import headalloc as OH
+    from quantized_decode_attention_append_b200 import headalloc as HA
+    r = np.random.default_rng(5)
+    L, H, G, T, D = 3, 4, 2, 60, 32
+    H2 = np.zeros((L, H))
+    for l in range(L):
+        K = (r.standard_normal((H, T, D)) * (1 + l)).astype(np.float16)
+        q = (r.standard_normal((6, H * G, D)) * np.linspace(0.2, 3, H * G)[None, :, None]).astype(np.float16)
+        kv = [60, 31, 7, 60, 45, 12]
+        got = HA.head_entropy(torch.from_numpy(q), torch.from_numpy(K), kv)
+        want = np.zeros(H)
+        for i in range(6):
+            _, _, P = OA.attention(q[i], K, K, kv[i])
+            for hq in range(H * G):
+                want[hq // G] += OH.renyi2(P[hq]) / (6 * G)
+        assert np.allclose(got.numpy(), want, rtol=1e-9, atol=1e-9)
+        H2[l] = want
+    hk, hv, bits = HA.allocate(H2, 4.0, sink_frac=0.1)
+    want_bits = OH.head_bits(H2.reshape(-1), 4.0).reshape(L, H)
+    sinks = set(OH.sink_heads(H2.reshape(-1), 0.1).tolist())
+    assert len(sinks) == 1
+    for l in range(L):
+        for h in range(H):
+            if l * H + h in sinks:
+                assert bits[l][h] == 16 and hk[l][h].fmt == "fp16"
+            else:
+                assert bits[l][h] == want_bits[l, h] and hk[l][h].bits == want_bits[l, h]
+    assert hk == hv

@@ -826,3 +826,51 @@ def test_sorted_groups_honest_bits_and_error():
     e_plain = A.rel_sq_error(x, Q.quantize_rows(x, Side("int", 2, group=8))["exact"])
     e_plain_mm = A.rel_sq_error(x, Q.quantize_rows(x, Side("int", 2, scale="minmax", group=8))["exact"])
     assert e_sorted < 0.6 * e_plain and e_sorted < 0.6 * e_plain_mm
+
+
+# ----------------------------------------------------------------------------- per-head allocation
+from oracle import headalloc as HA
+
+
+def test_renyi2_closed_forms():
+    """H_2 = -log2 sum p^2 ("Finding 2"): log2 n for n equal weights, 0 for one certain key,
+    -log2(p^2 + (1 - p)^2) for two."""
+    for n in (1, 2, 7, 64, 1000):
+        assert HA.renyi2(np.full(n, 1.0 / n)) == pytest.approx(math.log2(n), abs=1e-12)
+    assert HA.renyi2(np.array([1.0, 0.0, 0.0])) == 0.0
+    assert HA.renyi2(np.array([0.25, 0.75])) == pytest.approx(-math.log2(0.25 ** 2 + 0.75 ** 2))
+    r = rng(91).random(50)
+    p = r / r.sum()
+    assert 0.0 <= HA.renyi2(p) <= math.log2(50)
+
+
+def test_head_bits_rule_and_sink_count():
+    """b_h = b_avg + 0.25 (H_avg - H_2(h)): the average is kept before rounding, a head at the mean
+    entropy gets b_avg, one bit more entropy costs a quarter bit; the bottom 2% of heads are sinks:
+    3 of GPT-2's 144 heads ("Finding 2")."""
+    H2 = rng(92).uniform(0.5, 9.0, size=144)
+    raw = 4 + 0.25 * (H2.mean() - H2)
+    assert raw.mean() == pytest.approx(4.0, abs=1e-12)
+    b = HA.head_bits(H2, 4.0)
+    assert (np.abs(b - raw) <= 0.5).all() and b.min() >= 2 and b.max() <= 8
+    flat = np.full(12, 5.0)
+    assert (HA.head_bits(flat, 4.0) == 4).all()
+    two = np.array([3.0, 7.0])  # mean 5: the diffuse head loses half a bit, the sharp one gains it
+    assert HA.head_bits(two, 4.0).tolist() == [5, 4]  # 4.5 rounds up, 3.5 rounds up
+    s = HA.sink_heads(H2)
+    assert len(s) == 3 and set(s) == set(np.argsort(H2)[:3])
+    assert len(HA.sink_heads(np.ones(12))) == 0 and HA.sink_heads(np.arange(50.0)).tolist() == [0]
+
+
+def test_per_head_spec_bits():
+    """A layer with per-head formats averages its heads' bits; an fp16 sink head counts 16."""
+    D = 128
+    s3, s4, f16 = Side("int", 3, group=32), Side("int", 4, group=32), Side("fp16")
+    hk = ((s3, s4, f16, s4),)
+    spec = C.Spec(1, 1, 4, 4, D, s4, s4, head_k=hk, head_v=hk)
+    want = (3.5 + 4.5 + 16 + 4.5) / 4
+    assert C.effective_bits(spec, 100) == pytest.approx(want)
+    x = rng(93).standard_normal((5, D)).astype(np.float16)
+    for h, side in enumerate(hk[0]):
+        kq, _ = C.quantize_unit(spec, x, x, head=h)
+        assert np.array_equal(kq["bytes"], Q.quantize_rows(x, side)["bytes"])
