@@ -45,15 +45,30 @@ WORKLOADS = {
     "64k-konly": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
                       k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="fp16"),
                       desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K g128, fp16 V"),
-    "qwen-minmax4": dict(L=8, Hkv=4, Hq=16, D=256, B=16, T=6000,
-                         k=dict(fmt="int", bits=4, scale="minmax", group=32),
-                         v=dict(fmt="int", bits=4, scale="minmax", group=32),
-                         desc="8L x 4kv x 16q, hd256, B16 x 6000; per-token min-max 4-bit g32 K and V (5.0 b); "
-                              "16 sequences so that a step's cache (0.98 GB) exceeds L2"),
-    "polar-4+8": dict(L=32, Hkv=8, Hq=32, D=128, B=1, T=8192,
+    "qwen-proxy128": dict(L=8, Hkv=4, Hq=4, D=256, B=1, T=6000,
+                          k=dict(fmt="int", bits=4, scale="minmax", group=32),
+                          v=dict(fmt="int", bits=4, scale="minmax", group=32), proxy=(128, 3000, 6000),
+                          desc="8L x 4kv x 4q (G 1), hd256, B1 x 6000; per-token min-max 4-bit g32 K and V (arm A); "
+                               "128 proxy queries (post-RoPE keys at positions in [3000, 6000), causal)"),
+    "qwen-proxy128-h256": dict(L=8, Hkv=4, Hq=4, D=256, B=1, T=6000,
+                               k=dict(fmt="int", bits=4, scale="minmax", group=32, rot=256),
+                               v=dict(fmt="int", bits=4, scale="minmax", group=32, rot=256), proxy=(128, 3000, 6000),
+                               desc="8L x 4kv x 4q (G 1), hd256, B1 x 6000; H256 min-max 4-bit g32 K and V (arm B); "
+                                    "128 proxy queries, causal"),
+    "polar-4+8": dict(L=32, Hkv=8, Hq=8, D=128, B=1, T=8192,
                       k=dict(fmt="polar", bits=4, bits2=8), v=dict(fmt="polar", bits=4, bits2=8),
-                      desc="32L x 8kv x 32q, hd128, B1 x 8192; rFFT polar K and V, 4-bit magnitude + 8-bit phase "
-                           "(6.125 b); the config names no query-head count: GQA 4 as in the stress workloads"),
+                      desc="32L x 8kv x 8q (G 1), hd128, B1 x 8192; rFFT polar K and V, 4-bit magnitude + 8-bit "
+                           "phase (6.125 b)"),
+    "stress-ternary-a8": dict(L=32, Hkv=8, Hq=32, D=128, B=16, T=32768,
+                              k=dict(fmt="ternary", group=8), v=dict(fmt="ternary", group=8),
+                              anchors=dict(layers=(0,), rule="first_n", n=48, bits=8),
+                              desc="32L x 8kv x 32q, hd128, B16 x 32768; ternary g8, int8 anchors layer 0, t < 48 "
+                                   "('ternboth_a8')"),
+    "64k-sym2": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
+                     k=dict(fmt="int", bits=4, group=128, rot=256),
+                     v=dict(fmt="int", bits=2, scale="sym", group=128, rot=256),
+                     desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K + H256 symmetric 2-bit V, g128 "
+                          "(3.125 b; the E22L next-run grid)"),
     "64k-v3": dict(L=8, Hkv=4, Hq=16, D=256, B=1, T=65536,
                    k=dict(fmt="int", bits=4, group=128, rot=256), v=dict(fmt="int", bits=3, group=128, rot=256),
                    desc="8L x 4kv x 16q, hd256, B1 x 65536; H256 4-bit K + H256 3-bit V, g128 (3.625 b)"),
@@ -74,9 +89,20 @@ def make_config(w, T_cap):
     from quantized_decode_attention_append_b200.kvq import Config, Side
     an = w.get("anchors")
     return Config(n_layers=w["L"], batch=w["B"], n_kv_heads=w["Hkv"], n_q_heads=w["Hq"], head_dim=w["D"],
-                  capacity=T_cap, k=Side(**w["k"]), v=Side(**w["v"]), max_queries=w["B"],
+                  capacity=T_cap, k=Side(**w["k"]), v=Side(**w["v"]),
+                  max_queries=w["proxy"][0] if w.get("proxy") else w["B"],
                   anchor_layers=an["layers"] if an else (), anchor_rule=an["rule"] if an else "none",
-                  anchor_n=an["n"] if an else 0)
+                  anchor_n=an["n"] if an else 0, anchor_bits=an.get("bits", 16) if an else 16)
+
+
+def proxy_setup(w, T0, seed, layer, device):
+    """Proxy queries ("E21W" "What I tested"): the post-RoPE keys of sequence 0 at n positions drawn
+    from [lo, min(hi, T0)), each attending the keys before it.  Returns (q [n, Hq, D], positions)."""
+    from quantized_decode_attention_append_b200 import synth
+    n, lo, hi = w["proxy"]
+    pos = synth.proxy_positions(1, n, lo, min(hi, T0))
+    K = synth.kv_rows(seed, "k", layer, [0], list(range(w["Hkv"])), pos.tolist(), w["D"], device)[0]
+    return K.transpose(0, 1).contiguous(), pos
 
 
 def row_bytes_of(cache, side):
@@ -86,13 +112,20 @@ def row_bytes_of(cache, side):
     return lo.row_bytes + 2 * lo.n_groups * (2 if lo.zeros >= 0 else 1)
 
 
-def decode_bytes(cache, w, kv_len, anchored_rows_per_unit):
-    """Algorithmic bytes of one decode call: packed K/V rows + scales for t < kv_len (fp16
-    rows for anchored tokens), the queries and the fp32 outputs."""
+def decode_bytes(cache, w, kv_len, anchored_rows_per_unit, proxy_pos=None):
+    """Algorithmic bytes of one decode call: packed K/V rows + scales for t < kv_len (anchor rows
+    as stored for anchored tokens), the queries and the fp32 outputs.  With proxy queries each
+    query reads its own causal prefix of sequence 0."""
     D, units = w["D"], w["B"] * w["Hkv"]
     per_tok = row_bytes_of(cache, 0) + row_bytes_of(cache, 1)
+    if proxy_pos is not None:
+        n = len(proxy_pos)
+        return w["Hkv"] * per_tok * float(sum(proxy_pos)) + n * w["Hq"] * D * (2 + 4)
     a = anchored_rows_per_unit
-    kv = units * ((kv_len - a) * per_tok + a * 4 * D)
+    an = w.get("anchors") or {}
+    ab = an.get("bits", 16)
+    a_row = 2 * (2 * D if ab == 16 else D * ab // 8 + 2 * (D // 32))  # K and V anchor rows as stored
+    kv = units * ((kv_len - a) * per_tok + a * a_row)
     return kv + w["B"] * w["Hq"] * D * (2 + 4)
 
 
@@ -173,48 +206,107 @@ def traffic_record(workload):
 
 
 # ----------------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, budget_s=15.0, seed=0):
-    """Time the oracle, as it stands, on whole (layer, sequence, kv-head) units of one decode
-    step: quantize the unit's T rows (the appended token included), reconstruct them, attend with
-    the unit's query heads.  Input generation is outside the timed region.  Returns (seconds per
-    unit, units timed)."""
-    from threadpoolctl import threadpool_limits
-
+def _oracle_spec(w):
     from oracle import cache as OC
     from oracle import quant as OQ
+    an = w.get("anchors")
+    return OC.Spec(w["L"], w["B"], w["Hkv"], w["Hq"], w["D"], OQ.Side(**w["k"]), OQ.Side(**w["v"]),
+                   frozenset(an["layers"]) if an else frozenset(), an["rule"] if an else "none", an["n"] if an else 0,
+                   anchor_bits=an.get("bits", 16) if an else 16)
+
+
+def _oracle_unit(w, spec, idx, seed):
+    """Inputs of oracle unit `idx` (a (layer, sequence, kv-head) of one step) and the function that
+    runs it: quantize the unit's T rows, reconstruct them, attend its queries (the unit's query
+    heads, or every proxy query of the sequence)."""
+    from oracle import cache as OC
     from quantized_decode_attention_append_b200 import synth
     D, T, G = w["D"], w["T"], w["Hq"] // w["Hkv"]
-    an = w.get("anchors")
-    spec = OC.Spec(w["L"], w["B"], w["Hkv"], w["Hq"], D, OQ.Side(**w["k"]), OQ.Side(**w["v"]),
-                   frozenset(an["layers"]) if an else frozenset(), an["rule"] if an else "none", an["n"] if an else 0)
-    done, spent = 0, 0.0
+    layer, b, h = idx % w["L"], (idx // w["L"]) % w["B"], idx % w["Hkv"]
+    K16 = synth.kv_rows(seed, "k", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
+    V16 = synth.kv_rows(seed, "v", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
+    if w.get("proxy"):
+        n, lo, hi = w["proxy"]
+        pos = synth.proxy_positions(1, n, lo, min(hi, T))
+        qs = [(K16[p][None, :], int(p)) for p in pos]
+    else:
+        qs = [(synth.queries(1, layer, 1, G, D, T)[0].numpy()[:G], T)]
+
+    def run():
+        kq, vq = OC.quantize_unit(spec, K16, V16)
+        Kh, Vh = OC.reconstruct_unit(spec, layer, K16, V16, kq, vq, T)
+        for q, kl in qs:
+            OC.decode_query(spec, layer, q, Kh[None], Vh[None], kl)
+    return run
+
+
+def _oracle_worker(args):
+    """One process of the multi-process sample: time units start, start + stride, ... for
+    budget_s seconds (single-threaded numpy); returns (units, seconds)."""
+    w, start, stride, budget_s, seed = args
+    from threadpoolctl import threadpool_limits
+    spec = _oracle_spec(w)
+    done, spent, idx = 0, 0.0, start
     with threadpool_limits(1):
-        while spent < budget_s and done < 32:
-            layer, b, h = done % w["L"], (done // w["L"]) % w["B"], done % w["Hkv"]
-            K16 = synth.kv_rows(seed, "k", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
-            V16 = synth.kv_rows(seed, "v", layer, [b], [h], list(range(T)), D)[0, 0].numpy()
-            q = synth.queries(1, layer, 1, G, D, T)[0].numpy()
+        while spent < budget_s and done < 64:
+            run = _oracle_unit(w, spec, idx, seed)
             t0 = time.perf_counter()
-            kq, vq = OC.quantize_unit(spec, K16, V16)
-            Kh, Vh = OC.reconstruct_unit(spec, layer, K16, V16, kq, vq, T)
-            OC.decode_query(spec, layer, q, Kh[None], Vh[None], T)
+            run()
             spent += time.perf_counter() - t0
             done += 1
-    return spent / done, done
+            idx += stride
+    return done, spent
+
+
+def oracle_sample(w, budget_s=15.0, seed=0, processes=0):
+    """Time the oracle, as it stands, on whole units of one decode step (see _oracle_unit); input
+    generation is outside the timed region.  Single-threaded in this process for budget_s, then,
+    if processes > 1, the same work spread over that many spawned processes (one numpy thread
+    each) for budget_s of wall time.  Returns a dict of seconds per unit (single thread), units per
+    second (all processes), and the counts."""
+    single = _oracle_worker((w, 0, 1, budget_s, seed))
+    out = {"units_single": single[0], "s_per_unit_single": single[1] / single[0], "processes": 1,
+           "units_per_s_multi": single[0] / single[1], "units_multi": single[0]}
+    if processes > 1:
+        import concurrent.futures as cf
+        import multiprocessing as mp
+        with cf.ProcessPoolExecutor(max_workers=processes, mp_context=mp.get_context("spawn")) as ex:
+            res = list(ex.map(_oracle_worker, [(w, i, processes, budget_s, seed) for i in range(processes)]))
+        out["processes"] = processes
+        out["units_multi"] = sum(r[0] for r in res)
+        out["units_per_s_multi"] = sum(r[0] / r[1] for r in res)  # the processes ran concurrently
+    return out
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_record(w, budget_s, processes):
+    o = oracle_sample(w, budget_s=budget_s, processes=processes)
+    units_per_step = w["L"] * w["B"] * w["Hkv"]
+    what = (f"{w['proxy'][0]} proxy queries" if w.get("proxy") else f"{w['Hq'] // w['Hkv']} query heads")
+    sample = (f"whole (layer, sequence, kv-head) units of one step: quantize + reconstruct {w['T']} rows, attend "
+              f"{what}; {o['units_single']} units on 1 thread and {o['units_multi']} units over {o['processes']} "
+              f"processes, scaled by {units_per_step} units/step")
+    return {"value": o["units_per_s_multi"] / units_per_step, "unit": "steps/s", "cores": o["processes"],
+            "kind": "oracle", "sample": sample, "nproc": host_cores(),
+            "single_thread": {"value": 1.0 / (o["s_per_unit_single"] * units_per_step), "unit": "steps/s"},
+            "multi_process": {"value": o["units_per_s_multi"] / units_per_step, "unit": "steps/s",
+                              "processes": o["processes"]}}
 
 
 def run_reference(args, w, name):
-    per_unit, n = oracle_sample(w, budget_s=args.ref_budget)
-    units_per_step = w["L"] * w["B"] * w["Hkv"]
-    sps = 1.0 / (per_unit * units_per_step)
+    cpu = cpu_baseline_record(w, args.ref_budget, max(1, min(host_cores(), args.ref_processes)))
+    sps = cpu["value"]
     rec = {"impl": "reference", "metric": "decode steps/s", "value": sps, "unit": "steps/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / sps, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": f"{name}: {w['desc']}"},
-           "cpu_baseline": {"value": sps, "unit": "steps/s", "cores": 1, "kind": "oracle",
-                            "sample": f"{n} (layer, seq, kv-head) units of one step (quantize + reconstruct "
-                                      f"{w['T']} rows, attend {w['Hq'] // w['Hkv']} heads), scaled by {units_per_step} "
-                                      f"units/step"},
+           "cpu_baseline": cpu,
            "e2e": {"value": sps, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(rec), flush=True)
 
@@ -296,20 +388,30 @@ def run_gpu(args, w, name):
     # per-step inputs resident in HBM: one new K/V row per sequence and layer, queries per layer
     knew = [synth.kv_rows(rank, "k", l, list(range(B)), list(range(Hkv)), [T0], D, dev) for l in range(L)]
     vnew = [synth.kv_rows(rank, "v", l, list(range(B)), list(range(Hkv)), [T0], D, dev) for l in range(L)]
-    qs = [synth.queries(1, l, B, Hq, D, T0).to(dev) for l in range(L)]
-    outs = [torch.empty(B, Hq, D, device=dev, dtype=torch.float32) for _ in range(L)]
+    proxy = w.get("proxy")
+    if proxy:  # config-2 shape: one sequence, its proxy queries, each causal over earlier keys
+        pq = [proxy_setup(w, T0, rank, l, dev) for l in range(L)]
+        qs = [p[0] for p in pq]
+        proxy_pos = pq[0][1]
+        qsid = torch.zeros(len(proxy_pos), dtype=torch.int32, device=dev)
+        qlen = torch.tensor(proxy_pos.tolist(), dtype=torch.int32, device=dev)
+    else:
+        qs = [synth.queries(1, l, B, Hq, D, T0).to(dev) for l in range(L)]
+        proxy_pos, qsid, qlen = None, None, None
+    n_q = qs[0].shape[0]
+    outs = [torch.empty(n_q, Hq, D, device=dev, dtype=torch.float32) for _ in range(L)]
     launches = {"n": 0}
 
     def step():
         for l in range(L):
             cache.append(l, knew[l], vnew[l])
             launches["n"] += kvq.kvq_last_launch_count(cache.h)
-            cache.decode(l, qs[l], out=outs[l])
+            cache.decode(l, qs[l], seq_ids=qsid, kv_len=qlen, out=outs[l])
             launches["n"] += kvq.kvq_last_launch_count(cache.h)
 
     def decode_only():
         for l in range(L):
-            cache.decode(l, qs[l], out=outs[l])
+            cache.decode(l, qs[l], seq_ids=qsid, kv_len=qlen, out=outs[l])
 
     # one eager step (first-call set-up), then capture the step and the decode-only pass
     step()
@@ -355,7 +457,7 @@ def run_gpu(args, w, name):
     anchored = an["n"] if an and an["rule"] == "first_n" else 0
     dec_len = T0 + W_ + K_
     mean_len = T0 + W_ + (K_ + 1) / 2.0
-    per_layer = lambda n, a: decode_bytes(cache, w, n, a)
+    per_layer = lambda n, a: decode_bytes(cache, w, n, a, proxy_pos)
     dec_bytes_step = sum(per_layer(mean_len, anchored if (an and l in an["layers"]) else 0) for l in range(L))
     dec_bytes_launch = sum(per_layer(dec_len, anchored if (an and l in an["layers"]) else 0) for l in range(L)) / L
     achieved = dec_bytes_launch / (dec_launch_ms * 1e-3) / 1e9
@@ -383,8 +485,8 @@ def run_gpu(args, w, name):
             dst.append(d_in[off:off + x.numel()].view(x.shape))
             off += (x.numel() + 63) // 64 * 64
         spans.append((start, off))
-    d_out = torch.empty(L, B, Hq, D, device=dev, dtype=torch.float32)
-    h_out = torch.empty(L, B, Hq, D, dtype=torch.float32).pin_memory()
+    d_out = torch.empty(L, n_q, Hq, D, device=dev, dtype=torch.float32)
+    h_out = torch.empty(L, n_q, Hq, D, dtype=torch.float32).pin_memory()
     copy_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(L)]
     ev_out = [torch.cuda.Event() for _ in range(L)]
@@ -397,7 +499,7 @@ def run_gpu(args, w, name):
             d_in.copy_(h_in, non_blocking=True)
             for l in range(L):
                 cache.append(l, d_k[l], d_v[l])
-                cache.decode(l, d_q[l], out=d_out[l])
+                cache.decode(l, d_q[l], seq_ids=qsid, kv_len=qlen, out=d_out[l])
             h_out.copy_(d_out, non_blocking=True)
             return
         copy_stream.wait_stream(main)
@@ -409,7 +511,7 @@ def run_gpu(args, w, name):
         for l in range(L):
             main.wait_event(ev_in[l])
             cache.append(l, d_k[l], d_v[l])
-            cache.decode(l, d_q[l], out=d_out[l])
+            cache.decode(l, d_q[l], seq_ids=qsid, kv_len=qlen, out=d_out[l])
             ev_out[l].record(main)
         with torch.cuda.stream(copy_stream):
             for l in range(L):
@@ -438,11 +540,7 @@ def run_gpu(args, w, name):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            per_unit, n = oracle_sample(w, budget_s=args.ref_budget)
-            units_per_step = L * B * Hkv
-            cpu = {"value": 1.0 / (per_unit * units_per_step), "unit": "steps/s", "cores": 1, "kind": "oracle",
-                   "sample": f"{n} (layer, seq, kv-head) units of one step (quantize + reconstruct {T} rows, "
-                             f"attend {Hq // Hkv} heads), scaled by {units_per_step} units/step"}
+            cpu = cpu_baseline_record(w, args.ref_budget, max(1, min(host_cores(), args.ref_processes)))
         rec = {"metric": "decode steps/s", "value": aggregate_steps_per_s(ms_step, world), "unit": "steps/s",
                "n_gpus": world,
                "steps": K_, "warmup": W_, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -481,7 +579,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
-    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of CPU oracle work to sample")
+    ap.add_argument("--ref-budget", type=float, default=10.0,
+                    help="seconds of CPU oracle work to sample (single thread, then again over all processes)")
+    ap.add_argument("--ref-processes", type=int, default=16,
+                    help="oracle processes for the multi-process sample (capped by the host's cores; each one "
+                         "imports numpy and torch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="profiling only: fewer layers than the workload")
     ap.add_argument("--batch", type=int, default=0, help="profiling only: fewer sequences than the workload")
