@@ -54,10 +54,11 @@ __device__ __forceinline__ long long query_row(const LayerDev& L, int qi, int kv
   return ((long long)qi * L.Hkv_all + L.h0 + kvh) * G + h;
 }
 
-// Caller row ([n_seqs][Hkv_all][n_new] order) of the view's append row `row` ([n_seqs][Hkv][n_new]).
-__device__ __forceinline__ long long input_row(const LayerDev& L, long long row, int n_new) {
+// Caller row ([n_seqs][Hkv_all][n_new] order) of the view's append row `row` ([n_seqs][Hkv][n_new]);
+// rows of one call are fewer than 2^31 (checked on the host), so 32-bit arithmetic suffices.
+__device__ __forceinline__ int input_row(const LayerDev& L, int row, int n_new) {
   if (L.Hkv == L.Hkv_all) return row;
-  const long long ul = row / n_new, sl = ul / L.Hkv;
+  const int ul = row / n_new, sl = ul / L.Hkv;
   return (sl * L.Hkv_all + L.h0 + (ul - sl * L.Hkv)) * n_new + (row - ul * n_new);
 }
 

@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
   const int pos = dst.pos, len_after = dst.len_after, u = dst.u;
   if (!ok && dst.first && lane == 0) atomicOr(L.err, dst.err);
   if (ok) {
-    const __half* rp = src + input_row(L, row, n_new) * 128;
+    const __half* rp = src + (long long)input_row(L, (int)row, n_new) * 128;
     float* re = sre[warp];
     float* im = sim[warp];
     for (int j = lane; j < 128; j += 32) {
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(128) append_sorted_kernel(LayerDev L, int side
       if (dst.first && lane == 0) atomicOr(L.err, dst.err);
       continue;
     }
-    const __half* rp = src + input_row(L, row, n_new) * D;
+    const __half* rp = src + (long long)input_row(L, (int)row, n_new) * D;
     float* x = sx[warp];
     for (int j = lane; j < D; j += 32) {
       float v = __half2float(rp[j]);
@@ -519,16 +519,21 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const float* th) {
 
 // An int8/int4 anchor row's group `li` (channels 32 li .. 32 li + 31, the lane's own slice): the
 // signed absmax grid of the int format on the raw fp16 values (largest magnitude, first on ties,
-// at -2^(b-1)), one fp16 scale.  Anchored rows are rare, so this stays out of the main path.
-__device__ __noinline__ void anchor_quant32(const LayerDev& L, const SideDev& S, long long arow, int li,
-                                            const __half2* raw2) {
+// at -2^(b-1)), one fp16 scale (anchored rows are rare: a branch the row kernels seldom take).
+__device__ __forceinline__ void anchor_quant32(const LayerDev& L, const SideDev& S, long long arow, int li, uint4 c0,
+                                            uint4 c1, uint4 c2, uint4 c3) {
   const int b = L.anchor_bits, half = 1 << (b - 1);
+  const uint4 cw[4] = {c0, c1, c2, c3};  // the 32 fp16 values, by value (no address of the caller's registers)
   float x[32];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float2 f = __half22float2(raw2[e]);
-    x[2 * e] = f.x;
-    x[2 * e + 1] = f.y;
+  for (int c4 = 0; c4 < 4; ++c4) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&cw[c4]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      x[8 * c4 + 2 * e] = f.x;
+      x[8 * c4 + 2 * e + 1] = f.y;
+    }
   }
   float best = -1.0f, m = 0.0f;
 #pragma unroll
@@ -576,7 +581,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   {
     const long long r0 = (long long)(bid * NW + warp) * rpw + lane / lpr;
     if (r0 < R) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + input_row(L, r0, n_new) * D + li * 32);
+      const uint4* p = reinterpret_cast<const uint4*>(src + (long long)input_row(L, (int)r0, n_new) * D + li * 32);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
     }
@@ -589,7 +594,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     {
       const long long rn = (long long)row + stride;
       if (rn < R) {
-        const uint4* p = reinterpret_cast<const uint4*>(src + input_row(L, rn, n_new) * D + li * 32);
+        const uint4* p = reinterpret_cast<const uint4*>(src + (long long)input_row(L, (int)rn, n_new) * D + li * 32);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
       }
@@ -628,7 +633,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
         } else {
-          anchor_quant32(L, S, arow, li, raw2);
+          anchor_quant32(L, S, arow, li, cw[0], cw[1], cw[2], cw[3]);
         }
       }
       if (S.mean_sub) {
@@ -1041,7 +1046,7 @@ __global__ void append_fp16_kernel(LayerDev L, int side, const __half* __restric
   const int c = (int)(gt % vec_per_row);
   const RowDst d = row_dst(L, (int)row, n_new);
   if (d.err == 0) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + input_row(L, row, n_new) * L.D) + c);
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + (long long)input_row(L, (int)row, n_new) * L.D) + c);
     reinterpret_cast<uint4*>(S.codes + ((long long)d.u * L.Tcap + d.pos) * S.row_bytes)[c] = w;
     if (in_anchor(L, d.pos, d.len_after))
       reinterpret_cast<uint4*>(S.anchors + ((long long)d.u * L.anchor_rows + anchor_slot(L, d.pos)) * L.D)[c] = w;
@@ -1063,7 +1068,7 @@ __global__ void __launch_bounds__(kMeanThreads) key_mean_kernel(LayerDev L, cons
   const int b = L.app_ids ? L.app_ids[sl] : sl;
   if (b < 0 || b >= L.B || L.seq_len[b] != 0) return;  // not this sequence's first append
   const int D = L.D, j = threadIdx.x % D, r0 = threadIdx.x / D, nr = kMeanThreads / D;
-  const __half* src = k + input_row(L, (long long)ul * n_new, n_new) * D;
+  const __half* src = k + (long long)input_row(L, ul * n_new, n_new) * D;
   long long acc = 0;
   for (int i = r0; i < n_new; i += nr) acc += __float2ll_rn(__fmul_rn(__half2float(src[(long long)i * D + j]), 16777216.0f));
   __shared__ long long part[kMeanThreads];
