@@ -81,16 +81,21 @@ __device__ __forceinline__ __half2 h2c(unsigned short bits) {
 // The 16/B field pairs of a 32-bit word of B-bit offset-binary codes as signed fp16 pairs
 // (field - ofs, exact while ofs is a multiple of 1/2 below 2^9):
 // out[k] = (field k, field k + 16/B), i.e. field k of each 16-bit half.
+// A half-integer offset needs every field at a shift of at least 1: the constant 2^(10-s) + ofs
+// is then a multiple of 1/2 below 1024, an fp16 value; the word is pre-shifted left by one bit
+// (fields of each byte at bits 1..8 of their 16-bit half, still inside the 10-bit mantissa).
 template <int B>
 __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t* out, float ofs = (float)(1 << (B - 1))) {
   constexpr int PH = 16 / B;                 // fields per 16-bit half
   constexpr int PB = 8 / B;                  // fields per byte
   constexpr uint32_t M = ((1u << B) - 1u) * 0x00010001u;
-  const uint32_t w8 = w >> 8;
+  const bool half_ofs = ofs != floorf(ofs);  // folded at compile time (ofs is a constant)
+  const int s0 = half_ofs ? 1 : 0;
+  const uint32_t wl = half_ofs ? (w << 1) : w, w8 = half_ofs ? (w >> 7) : (w >> 8);
 #pragma unroll
   for (int k = 0; k < PH; ++k) {
-    const int s = B * (k % PB);              // shift of the field inside its byte
-    const uint32_t x = and_or(k < PB ? w : w8, M << s, 0x64006400u);  // 1024 + 2^s field
+    const int s = B * (k % PB) + s0;         // shift of the field inside its 16-bit half
+    const uint32_t x = and_or(k < PB ? wl : w8, M << s, 0x64006400u);  // 1024 + 2^s field
     // 2^-s and -(1024 2^-s + 2^(B-1)) as fp16 bit patterns
     const unsigned short scl = (unsigned short)((15 - s) << 10);
     const float off = -(1024.0f / (float)(1 << s) + ofs);
