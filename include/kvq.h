@@ -66,7 +66,8 @@ enum {
 };
 /* INT scale modes: ABSMAX = the ggml signed grid; MINMAX = asymmetric; SYMMETRIC = levels
  * (q - (2^b - 1)/2) d, outermost level at the group's largest magnitude ([E22L] "Result": the
- * signed grid "leaves one side with fewer levels"; a symmetric grid is the next candidate). */
+ * signed grid has one level fewer on its positive side; a symmetric grid is named as the next
+ * value grid to try). */
 enum { KVQ_SCALE_ABSMAX = 0, KVQ_SCALE_MINMAX = 1, KVQ_SCALE_SYMMETRIC = 2 };
 enum { KVQ_ROT_NONE = 0, KVQ_ROT_H128 = 128, KVQ_ROT_H256 = 256 };
 enum { KVQ_ANCHOR_NONE = 0, KVQ_ANCHOR_FIRST_N = 1, KVQ_ANCHOR_WINDOW = 2, KVQ_ANCHOR_ALL = 3 };
@@ -91,8 +92,8 @@ typedef struct {
                           kvq_set_chan_scale before the first append. */
   int32_t mean_sub;    /* K only, quantized formats: 1 = subtract the sequence's key mean before
                           everything else and add it back after dequantizing ([LCPP], the later
-                          comment on a per-head shared key mean: "subtracting the running mean
-                          before quantization and restoring it after").  The mean of a (sequence,
+                          comment on a per-head shared key mean, removed before quantizing and
+                          restored afterwards).  The mean of a (sequence,
                           kv-head) is the mean of the rows of the sequence's first append (its
                           length was 0), rounded to fp16 once from the exact sum, and is kept for
                           the rows that follow; anchored rows stay raw. */

@@ -1,7 +1,7 @@
 """Gaussian Lloyd-Max quantizer levels.
 
 "E22L" "Result" (last paragraphs) names the value grid to test next after the ggml signed
-2-bit grid: "a symmetric grid or Gaussian Lloyd-Max levels on rotated values".  The pages give
+2-bit grid: a symmetric grid, or Lloyd-Max levels for a Gaussian applied after rotation.  The pages give
 no table.  This builds the levels from their definition (the MSE-optimal fixed-rate quantizer
 of a density; S. P. Lloyd, "Least squares quantization in PCM", and J. Max, "Quantizing for
 minimum distortion", 1960): at the optimum every threshold is the midpoint of its two

@@ -21,17 +21,17 @@ Grids and scales (sources by page title and section):
   * sign {-s, +s}: post 6 "Minimal recipe" (one-bit sign KV with a scale);
     s = fp16(fp32 sum of |x| in channel order / g) (least-squares scale for fixed signs),
     t = +1 if x >= 0 else -1.
-  * symmetric int b: "E22L" "Result" (the ggml grid "leaves one side with fewer levels"; a
-    symmetric grid is the next candidate).  Levels (q - (2^b - 1)/2) d for q = 0 .. 2^b - 1, so
+  * symmetric int b: "E22L" "Result" (the ggml grid has one level fewer on its positive side;
+    the page names a symmetric grid as the next value grid to try).  Levels (q - (2^b - 1)/2) d for q = 0 .. 2^b - 1, so
     the outermost level is the group's largest magnitude m: d = fp16(fp32(m / (2^(b-1) - 1/2))),
     q = clamp(floor(x/d) + 2^(b-1), 0, 2^b - 1) (nearest level, ties up); d = 0 gives q = 2^(b-1).
   * Gaussian Lloyd-Max b: "E22L" "Result" (the other next candidate, "Gaussian Lloyd-Max levels
     on rotated values"); levels from oracle.lloyd in units of the group's RMS,
     s = fp16(sqrt(fp32(fp32 sum of x^2 in channel order / g))), code = nearest level of x/s
     (ties up); s = 0 gives the level just above zero, 2^(b-1).
-  * sorted groups: post 6, "The winning recipe" item 1 (titled magnitude-sorted grouping: "sort
-    each row descending, quantize groups; outliers share one wide group", g = 8 for K and 4 for
-    V, with 2-bit codes).  Reading taken here: a row is ordered by value, descending (equal values
+  * sorted groups: post 6, "The winning recipe" item 1 (titled magnitude-sorted grouping: each
+    row is sorted in descending order and quantized in groups, so the outliers end up together in
+    one wide group; g = 8 for K and 4 for V, with 2-bit codes).  Reading taken here: a row is ordered by value, descending (equal values
     keep channel order), and consecutive g values of that order form a group on the per-token
     min-max grid (so the top group, where large outliers gather, gets its own wide range); the row
     stores each channel's rank (its position in the order) in ceil(log2 D) bits -- the permutation

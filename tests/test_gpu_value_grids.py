@@ -1,5 +1,5 @@
 """GPU parity of the value grids named for the next run in "E22L" "Result" (a symmetric 2-bit grid
-and Gaussian Lloyd-Max levels on rotated values) and of key-mean subtraction (llama.cpp #21385,
+and Lloyd-Max levels for a Gaussian after rotation) and of key-mean subtraction (llama.cpp #21385,
 the comment on a shared per-head key mean: subtract the running mean before quantization,
 restore it after).
 

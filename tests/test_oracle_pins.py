@@ -772,7 +772,7 @@ def test_int_anchor_rows(abits):
 @pytest.mark.parametrize("D,b,g", [(128, 2, 8), (128, 2, 4), (64, 3, 8), (256, 2, 16)])
 def test_sorted_groups(D, b, g):
     """Post 6, "The winning recipe" item 1: rows sorted descending, consecutive groups quantized
-    ("outliers share one wide group").  The stored ranks form a permutation that orders the row
+    (the outliers land together in one wide group).  The stored ranks form a permutation that orders the row
     descending (equal values in channel order); every value is the nearest level of its group's
     min-max grid; the top group holds the row's largest values; the bytes are the codes then the
     ceil(log2 D)-bit ranks."""
