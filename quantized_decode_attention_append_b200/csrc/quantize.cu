@@ -556,8 +556,10 @@ __device__ __forceinline__ void anchor_quant32(const LayerDev& L, const SideDev&
   S.anchor_scales[arow * (L.D / 32) + li] = sh;
 }
 
-// Rows of one side over blocks bid = 0 .. nblk - 1 (grid-stride).
-template <int FAM, int G, int BITS = 0>
+// Rows of one side over blocks bid = 0 .. nblk - 1 (grid-stride).  EXT = false compiles out the key
+// mean, int anchors and head-group input mapping (the fused K+V kernel's common case), which
+// keeps the hot instances at 128 registers; callers needing them use the EXT instances.
+template <int FAM, int G, int BITS = 0, bool EXT = true>
 __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __half* __restrict__ src, int n_new,
                                           int bid, int nblk) {
   const SideDev& S = L.s[side];
@@ -572,7 +574,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   // code bits: fixed by the family, by the instance (BITS > 0), or read from the side
   const int bits = FAM == FAM_SIGN ? 1 : (FAM == FAM_NF4 ? 4 : (BITS > 0 ? BITS : S.bits));
   // the grid sees the fp16 input itself (no key mean, channel scale or rotation in between)
-  const bool raw = !S.rot && !S.chan_scale && !S.mean_sub;
+  const bool raw = !S.rot && !S.chan_scale && !(EXT && S.mean_sub);
 
   // The next pass's input slice is loaded before this pass's arithmetic, so each warp keeps its
   // loads in flight while it computes (the arithmetic per row is long).
@@ -581,7 +583,8 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
   {
     const long long r0 = (long long)(bid * NW + warp) * rpw + lane / lpr;
     if (r0 < R) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + (long long)input_row(L, (int)r0, n_new) * D + li * 32);
+      const uint4* p = reinterpret_cast<const uint4*>(src + (long long)(EXT ? input_row(L, (int)r0, n_new) : (int)r0) * D +
+                                                      li * 32);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
     }
@@ -594,7 +597,8 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
     {
       const long long rn = (long long)row + stride;
       if (rn < R) {
-        const uint4* p = reinterpret_cast<const uint4*>(src + (long long)input_row(L, (int)rn, n_new) * D + li * 32);
+        const uint4* p = reinterpret_cast<const uint4*>(src + (long long)(EXT ? input_row(L, (int)rn, n_new) : (int)rn) * D +
+                                                        li * 32);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) nx[c4] = __ldg(p + c4);
       }
@@ -628,7 +632,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
       }
       if (in_anchor(L, pos, len_after)) {
         const long long arow = (long long)u * L.anchor_rows + anchor_slot(L, pos);
-        if (L.anchor_bits == 16) {
+        if (!EXT || L.anchor_bits == 16) {
           __half* ap = S.anchors + arow * D + li * 32;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) reinterpret_cast<uint4*>(ap)[c4] = cw[c4];
@@ -636,7 +640,7 @@ __device__ __forceinline__ void rows_body(const LayerDev& L, int side, const __h
           anchor_quant32(L, S, arow, li, cw[0], cw[1], cw[2], cw[3]);
         }
       }
-      if (S.mean_sub) {
+      if (EXT && S.mean_sub) {
         const __half* mp = S.kmean + (long long)u * D + li * 32;
 #pragma unroll
         for (int v = 0; v < 32; ++v) x[v] = __fsub_rn(x[v], __half2float(mp[v]));
@@ -974,8 +978,8 @@ template <int FK, int GK, int BK, int FV, int GV, int BV>
 __global__ void __launch_bounds__(kRowThreads) append_kv_kernel(LayerDev L, const __half* __restrict__ k,
                                                                 const __half* __restrict__ v, int n_new,
                                                                 unsigned kblocks, unsigned total_ctas) {
-  if (blockIdx.x < kblocks) rows_body<FK, GK, BK>(L, 0, k, n_new, blockIdx.x, kblocks);
-  else rows_body<FV, GV, BV>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
+  if (blockIdx.x < kblocks) rows_body<FK, GK, BK, false>(L, 0, k, n_new, blockIdx.x, kblocks);
+  else rows_body<FV, GV, BV, false>(L, 1, v, n_new, blockIdx.x - kblocks, gridDim.x - kblocks);
   finish_append(L, n_new, total_ctas);
 }
 
@@ -1130,6 +1134,7 @@ static KvKernel pick_kv_kernel(const LayerDev& L) {
   if (K.fmt == KVQ_FMT_FP16 || V.fmt == KVQ_FMT_FP16 || K.fmt == KVQ_FMT_POLAR || K.fmt == KVQ_FMT_CART ||
       V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART || K.fmt == KVQ_FMT_SORTED || V.fmt == KVQ_FMT_SORTED)
     return nullptr;
+  if (K.mean_sub || L.anchor_bits != 16 || L.Hkv != L.Hkv_all) return nullptr;  // the fused kernel has no extras
   const int fk = fam_of(K), fv = fam_of(V), gk = K.group, gv = V.group;
   // bits 0: fixed by the family (NF4, ternary, sign)
 #define KVQ_KV(FK_, GK_, BK_, FV_, GV_, BV_)                                                      \

@@ -35,7 +35,7 @@ GRIDS = [
 
 @pytest.mark.parametrize("D,G,k,v", GRIDS, ids=[f"{d}G{g}-{k.fmt}{k.bits}{k.scale[:3]}g{k.group}-{v.fmt}{v.bits}"
                                                  f"{v.scale[:3]}g{v.group}r{v.rot}" for d, g, k, v in GRIDS])
-@pytest.mark.parametrize("chunks", [None, [1] * 3 + [150, 1, 145]], ids=["bulk", "mixed"])
+@pytest.mark.parametrize("chunks", [None, [1] * 3 + [150, 1, 146]], ids=["bulk", "mixed"])
 def test_value_grid_parity(D, G, k, v, chunks):
     T = 300
     cfg = cfg_of(D, k, v, G=G, T=T)
@@ -54,10 +54,14 @@ def test_symmetric_v_runs_on_tensor_cores():
     c.cache.decode(0, q)
     torch.cuda.synchronize()
     from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        c.cache.decode(0, q)
-        torch.cuda.synchronize()
-    names = " ".join(e.name for e in prof.events())
+    names = ""
+    for _ in range(3):  # the profiler's kernel records occasionally arrive empty: take another look
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            c.cache.decode(0, q)
+            torch.cuda.synchronize()
+        names = " ".join(e.name for e in prof.events())
+        if "merge_kernel" in names:
+            break
     assert "decode_tc_kernel" in names and "decode_generic_kernel" not in names
 
 
