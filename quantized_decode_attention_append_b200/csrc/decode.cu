@@ -173,6 +173,7 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
 }
 
 #include "decode_tc.cuh"
+#include "decode_mq.cuh"
 
 // Generic pass 1: any format, any GQA group (<= 8), CUDA cores.  Thread-per-token scoring,
 // thread-per-channel value accumulation.
@@ -585,8 +586,34 @@ static int mma_slots(const MmaPlan& p, int num_sms) {
   return cached_occ * num_sms;
 }
 
+// The multi-query kernel serves GQA groups of 1 or 2 when there are more queries than sequences
+// (so some queries share a sequence and a decoded tile can serve several of them).
+static bool use_mq(const LayerDev& L, int n_q) { return L.Hq / L.Hkv <= 2 && n_q > L.B; }
+
+// Splits of the multi-query kernel: about two waves of its CTAs, at least one 32-token tile each.
+template <int D>
+static int mq_split_count(const LayerDev& L, int n_q, int num_sms) {
+  const int G = L.Hq / L.Hkv, qpb = MqCfg<D>::QM / G;
+  const long long units = (long long)L.Hkv * ((n_q + qpb - 1) / qpb);
+  const int per_sm = D >= 256 ? 1 : 2;
+  long long s = (2LL * per_sm * num_sms + units - 1) / units;
+  const long long tiles = L.Tcap / MqCfg<D>::TK;
+  if (s > tiles) s = tiles;
+  if (s > kMaxSplit) s = kMaxSplit;
+  return s < 1 ? 1 : (int)s;
+}
+
+static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
+  switch (L.D) {
+    case 64: return mq_split_count<64>(L, n_q, num_sms);
+    case 128: return mq_split_count<128>(L, n_q, num_sms);
+    default: return mq_split_count<256>(L, n_q, num_sms);
+  }
+}
+
 // Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).
 int decode_partials(const LayerDev& L, int n_q, int num_sms) {
+  if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 1;
   MmaPlan p;
   if (pick_mma(L, &p)) {
     const int ntiles = L.Tcap / p.tile;
@@ -602,7 +629,29 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   int nl = 0;
   MmaPlan p;
   int n_quant;  // quantized partials per (query, head)
-  if (pick_mma(L, &p)) {
+  if (use_mq(L, n_q)) {
+    using MC = MqCfg<D>;
+    static bool attr_set = false;  // one per instantiation (the attribute is per kernel)
+    if (!attr_set) {
+      cudaFuncSetAttribute(decode_mq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, MC::SMEM);
+      attr_set = true;
+    }
+    const int n_split = mq_split_count<D>(L, n_q, num_sms);
+    n_quant = n_split;
+    const int nsp = n_quant + (L.anchored ? 1 : 0);
+    const int qpb = MC::QM / (L.Hq / L.Hkv);
+    decode_mq_kernel<D><<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, MC::SMEM, st>>>(L, q, seq_ids, kv_len,
+                                                                                           work, n_split, nsp, n_q);
+    ++nl;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone
+      decode_generic_kernel<D><<<dim3(1, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp,
+                                                                           n_quant);
+      ++nl;
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  } else if (pick_mma(L, &p)) {
     const int slots = mma_slots(p, num_sms);
     const int n_split = mma_split_count((long long)n_q * L.Hkv, L.Tcap / p.tile, slots);
     n_quant = n_split;
