@@ -484,17 +484,6 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
 // ----------------------------------------------------------------------------------------------
 // Planning and launch.
 
-// Generic path: ~4 CTAs per SM over the grid; each split keeps at least two tiles of keys.
-static int generic_split_count(int Hkv, int Tcap, int n_q, int num_sms) {
-  const long long units = (long long)n_q * Hkv;
-  long long s = (4LL * num_sms + units - 1) / units;
-  const long long max_by_len = (Tcap + 2 * kGenTile - 1) / (2 * kGenTile);
-  if (s > max_by_len) s = max_by_len;
-  if (s < 1) s = 1;
-  if (s > kMaxSplit) s = kMaxSplit;
-  return (int)s;
-}
-
 // Tensor-core path: the split count that maximises (busy fraction of the resident-CTA slots over
 // whole waves) x (balance of tiles across splits) x per / (per + F), where a CTA's fixed cost F
 // (query transform and fragments, table build, warp combine, partial write) is about 0.75 tiles of
@@ -586,9 +575,14 @@ static int mma_slots(const MmaPlan& p, int num_sms) {
   return cached_occ * num_sms;
 }
 
-// The multi-query kernel serves GQA groups of 1 or 2 when there are more queries than sequences
-// (so some queries share a sequence and a decoded tile can serve several of them).
-static bool use_mq(const LayerDev& L, int n_q) { return L.Hq / L.Hkv <= 2 && n_q > L.B; }
+// The multi-query kernel (tiles decoded once per CTA into shared memory, any format) serves every
+// quantized range that has no register-decode tensor-core instance, and GQA groups of 1 or 2 with
+// more queries than sequences (some queries share a sequence, so a decoded tile serves several).
+// The generic kernel is left with the anchor rows.
+static bool use_mq(const LayerDev& L, int n_q) {
+  MmaPlan p;
+  return !pick_mma(L, &p) || (L.Hq / L.Hkv <= 2 && n_q > L.B);
+}
 
 // Splits of the multi-query kernel: about two waves of its CTAs, at least one 32-token tile each.
 template <int D>
@@ -615,11 +609,9 @@ static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
 int decode_partials(const LayerDev& L, int n_q, int num_sms) {
   if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 1;
   MmaPlan p;
-  if (pick_mma(L, &p)) {
-    const int ntiles = L.Tcap / p.tile;
-    return mma_split_count((long long)n_q * L.Hkv, ntiles, mma_slots(p, num_sms)) + 1;
-  }
-  return generic_split_count(L.Hkv, L.Tcap, n_q, num_sms) + 1;
+  pick_mma(L, &p);
+  const int ntiles = L.Tcap / p.tile;
+  return mma_split_count((long long)n_q * L.Hkv, ntiles, mma_slots(p, num_sms)) + 1;
 }
 
 template <int D>
@@ -651,7 +643,8 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
       ++nl;
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-  } else if (pick_mma(L, &p)) {
+  } else {  // a register-decode tensor-core instance exists (use_mq said no)
+    pick_mma(L, &p);
     const int slots = mma_slots(p, num_sms);
     const int n_split = mma_split_count((long long)n_q * L.Hkv, L.Tcap / p.tile, slots);
     n_quant = n_split;
@@ -666,13 +659,6 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
       ++nl;
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-  } else {
-    n_quant = generic_split_count(L.Hkv, L.Tcap, n_q, num_sms);
-    const int nsp = n_quant + (L.anchored ? 1 : 0);
-    decode_generic_kernel<D><<<dim3(nsp, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp, 0);
-    ++nl;
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
   }
   const int nsp = n_quant + (L.anchored ? 1 : 0);
   merge_kernel<D><<<n_q * L.Hq, D * merge_groups<D>(), 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse);

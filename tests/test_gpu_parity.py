@@ -219,7 +219,7 @@ def test_per_layer_bit_allocation():
 
 def test_per_layer_format_families():
     """Layers of one cache in different families: each layer takes its own append and decode
-    kernels (tensor-core and CUDA-core paths side by side)."""
+    kernels (register-decode and shared-tile tensor-core paths side by side)."""
     lk = (Side("nf4", group=64), Side("sign", group=4), Side("int", 3, scale="minmax", group=32),
           Side("ternary", group=8))
     lv = (Side("int", 4, group=64), Side("sign", group=4), Side("int", 4, scale="minmax", group=32),

@@ -166,7 +166,7 @@ SORTED = [
 @pytest.mark.parametrize("chunks", [None, [1, 1, 120, 1, 77]], ids=["bulk", "tokens"])
 def test_sorted_group_parity(D, G, k, v, anc, chunks):
     """Sorted groups with their stored ranks (post 6, "The winning recipe" item 1): codes, ranks,
-    scales and zero points bit for bit, dequantization, and attention from the generic decode."""
+    scales and zero points bit for bit, dequantization, and attention from the shared-tile decode."""
     T = 200
     cfg = cfg_of(D, k, v, G=G, T=T, **anc)
     c = Case(cfg, T, chunks=chunks)

@@ -24,7 +24,7 @@ def _rel(a, b):
 @pytest.mark.parametrize("D,k,v", [
     (128, Side("nf4", group=64), Side("int", 4, group=64)),                      # tensor-core kernel
     (256, Side("int", 4, group=128, rot=256), Side("int", 2, group=128, rot=256)),
-    (128, Side("ternary", group=8), Side("ternary", group=8)),                   # generic kernel
+    (128, Side("int", 3, scale="minmax", group=32), Side("polar", 5, 7)),        # shared-tile kernel
 ])
 def test_noalloc_decode_matches_regular_decode_twice(D, k, v):
     T = 900
