@@ -607,7 +607,7 @@ static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
 
 // Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).
 int decode_partials(const LayerDev& L, int n_q, int num_sms) {
-  if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 1;
+  if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 2;  // + anchor split, + prepared queries
   MmaPlan p;
   pick_mma(L, &p);
   const int ntiles = L.Tcap / p.tile;
@@ -623,20 +623,32 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   int n_quant;  // quantized partials per (query, head)
   if (use_mq(L, n_q)) {
     using MC = MqCfg<D>;
-    static bool attr_set = false;  // one per instantiation (the attribute is per kernel)
-    if (!attr_set) {
-      cudaFuncSetAttribute(decode_mq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, MC::SMEM);
-      attr_set = true;
+    static int dyn_max = -1;  // one per instantiation (the attribute is per kernel)
+    if (dyn_max < 0) {  // the opt-in limit covers static + dynamic shared memory
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, decode_mq_kernel<D>);
+      if (e != cudaSuccess) return e;
+      const int lim = MC::SMEM_MAX - (int)fa.sharedSizeBytes;
+      e = cudaFuncSetAttribute(decode_mq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+      if (e != cudaSuccess) return e;
+      dyn_max = lim;
     }
+    const int smem = mq_smem_bytes<D>(L);
+    if (smem > dyn_max) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
     const int n_split = mq_split_count<D>(L, n_q, num_sms);
     n_quant = n_split;
     const int nsp = n_quant + (L.anchored ? 1 : 0);
-    const int qpb = MC::QM / (L.Hq / L.Hkv);
-    decode_mq_kernel<D><<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, MC::SMEM, st>>>(L, q, seq_ids, kv_len,
-                                                                                           work, n_split, nsp, n_q);
+    // the prepared queries take the workspace slot after the partials (decode_partials counts it)
+    float* prep = work + (size_t)n_q * L.Hq * nsp * (D + kPartStride);
+    mq_prep_kernel<D><<<dim3(L.Hkv, n_q), 256, 0, st>>>(L, q, seq_ids, kv_len, prep);
     ++nl;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    const int qpb = MC::QM / (L.Hq / L.Hkv);
+    decode_mq_kernel<D><<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, smem, st>>>(L, prep, seq_ids, kv_len,
+                                                                                        work, n_split, nsp, n_q);
+    ++nl;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone
       decode_generic_kernel<D><<<dim3(1, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp,
                                                                            n_quant);

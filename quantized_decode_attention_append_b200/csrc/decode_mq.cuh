@@ -1,27 +1,34 @@
-// Tensor-core pass 1 of kvq_decode_attention for many queries over few sequences: GQA groups of 1
-// or 2 with more queries than sequences, as in the proxy-query setup ("E21W" "What I tested": the
-// post-RoPE keys at many positions of one text, each attending the keys before it).  There the
-// queries of one (sequence, kv-head) form a real M dimension, so a tile of keys and values is
-// decoded once per CTA and shared by all of its query rows.
+// Tensor-core pass 1 of kvq_decode_attention for many queries over few sequences (GQA groups of 1
+// or 2 with more queries than sequences, as in the proxy-query setup: "E21W" "What I tested", the
+// post-RoPE keys at many positions of one text, each attending the keys before it), and for every
+// format that has no register-decode instance.  The queries of one (sequence, kv-head) form a
+// real M dimension, so a tile of keys and values is decoded once per CTA and shared by all of its
+// query rows.
 //
 // Included by decode.cu inside namespace kvq (uses QueryRange, query_range, prepare_query, kLog2e,
 // kMaxG, d_nf4, d_lloyd, d_ph_cos, d_ph_sin).  Same contract as the other pass-1 kernels: one
 // log2-domain partial (m, l, o[D] in V's stored domain) per (query, head) and split.
 //
+// Queries.  mq_prep_kernel transforms each (query, kv-head) once (q' x sm_scale log2 e, as the
+// other kernels build it, and the key-mean term) into a workspace row; the CTAs of the main kernel
+// load their rows from there instead of each transforming them again.
+//
 // Rows.  A CTA holds QM = 64 rows, row r = (query q0 + r / G, head r % G); each warp owns a 16-row
 // block (with head_dim 256 two warps share one, each accumulating half of the channels).  The
-// transformed queries (q' x sm_scale log2 e, as the other kernels build them) are split into fp16
-// hi + lo halves in shared memory.
+// transformed queries are split into fp16 hi + lo halves in shared memory.  A warp none of whose
+// rows attends the current sequence skips the products.
 //
-// Tiles.  Per tile of TK = 32 tokens every thread decodes its share of the K and V rows into shared
-// memory as fp16 hi + lo halves of the exact stored-domain value (any format: code x scale, + zero,
-// levels, polar m (cos phi, sin phi), ...; rows past the sequence's length are zero), so no format
-// logic remains in the products.  Scores S[16 rows x 8 tokens] = Q . K^T take three mma per 16
-// channels (hi.hi + lo.hi + hi.lo, ~22-bit products), fragments loaded by ldmatrix; each row masks
-// its own causal range; the online softmax runs per row across the quad that shares it; the score
-// fragments are reused directly as the A operand of O += P . V (hi + lo again), with V's B
-// fragments loaded transposed (ldmatrix .trans).  Queries of different sequences in one CTA are
-// served by one pass per sequence over that sequence's tiles, other rows masked.
+// Tiles.  The packed bytes of a tile of TK = 32 tokens (codes, scales, zero points: contiguous
+// ranges of the cache) are copied into shared memory by cp.async one tile ahead of their use.
+// Every thread then decodes 8-element chunks of the staged rows into fp16 hi + lo halves of the
+// exact stored-domain value (any format: code x scale, + zero, levels, polar m (cos phi, sin phi),
+// ...; rows past the sequence's length are zero), so no format logic remains in the products.
+// Scores S[16 rows x 8 tokens] = Q . K^T take three mma per 16 channels (hi.hi + lo.hi + hi.lo,
+// ~22-bit products), fragments loaded by ldmatrix; each row masks its own causal range; the online
+// softmax runs per row across the quad that shares it; the score fragments are reused directly as
+// the A operand of O += P . V (hi + lo again), with V's B fragments loaded transposed (ldmatrix
+// .trans).  Queries of different sequences in one CTA are served by one pass per sequence over
+// that sequence's tiles, other rows masked.
 
 template <int D>
 struct MqCfg {
@@ -40,14 +47,30 @@ struct MqCfg {
   static constexpr int OFF_KL = OFF_KH + TK * LD * 2;
   static constexpr int OFF_VH = OFF_KL + TK * LD * 2;
   static constexpr int OFF_VL = OFF_VH + TK * LD * 2;
-  static constexpr int OFF_QT = OFF_VL + TK * LD * 2;         // fp32 [kMaxG][D] transformed query
-  static constexpr int OFF_QA = OFF_QT + kMaxG * D * 4;       // fp32 [kMaxG][D] (prepare_query's raw copy)
-  static constexpr int OFF_META = OFF_QA + kMaxG * D * 4;     // per row: seq, qa, qb, q.mu
-  static constexpr int OFF_TAB = OFF_META + QM * 4 * 4;       // NF4 16, Lloyd-Max 2 x 16, phase cos/sin 2 x 2 x 256
-  static constexpr int SMEM = OFF_TAB + (16 + 32 + 1024) * 4;
-  static_assert(SMEM <= 227 * 1024, "multi-query tiles exceed one CTA's shared memory");
+  static constexpr int OFF_META = OFF_VL + TK * LD * 2;          // per row: seq, qa, qb, q.mu
+  static constexpr int OFF_TAB = OFF_META + QM * 4 * 4;          // NF4 16, Lloyd-Max 2 x 16, phase cos/sin 2 x 2 x 256
+  static constexpr int OFF_RAW = OFF_TAB + (16 + 32 + 1024) * 4;  // two staging buffers of packed tile bytes
+  static constexpr int SMEM_MAX = 227 * 1024;
+  static_assert(OFF_RAW % 16 == 0, "staging buffers must start 16-byte aligned");
   static_assert((LD * 2) % 16 == 0, "ldmatrix rows must stay 16-byte aligned");
 };
+
+__host__ __device__ __forceinline__ int mq_up16(int x) { return (x + 15) & ~15; }
+
+// Staged bytes of one side for one tile: codes, then scales, then zero points, each range
+// starting 16-byte aligned.
+template <int TK>
+__host__ __device__ __forceinline__ int mq_stage_bytes(const SideDev& S) {
+  const int sc = S.scales ? mq_up16(TK * S.n_groups * 2) : 0;
+  return mq_up16(TK * S.row_bytes) + sc + (S.zeros ? sc : 0);
+}
+
+// Dynamic shared memory of one decode_mq_kernel<D> launch on `L`.
+template <int D>
+inline int mq_smem_bytes(const LayerDev& L) {
+  using C = MqCfg<D>;
+  return C::OFF_RAW + 2 * (mq_stage_bytes<C::TK>(L.s[0]) + mq_stage_bytes<C::TK>(L.s[1]));
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -60,25 +83,169 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-// Stored-domain value of element j of a row of any format (polar: slot j / 2, cos or sin part).
-__device__ __forceinline__ float mq_value(const SideDev& S, const uint8_t* __restrict__ row, const __half* __restrict__ sc,
-                                          const __half* __restrict__ zr, int j, const float* nf4, const float* lloyd,
-                                          const float* cs, const float* sn) {
-  if (S.fmt == KVQ_FMT_POLAR) {
-    const float2 ab = polar_slot(S, row, sc, j >> 1, cs, sn);
-    return (j & 1) ? ab.y : ab.x;
-  }
-  return stored_value(S, row, sc, zr, j, nf4, lloyd);
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(__cvta_generic_to_global(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(__cvta_generic_to_global(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void split_store(__half* hi, __half* lo, int idx, float v) {
-  const __half h = __float2half_rn(v);
-  hi[idx] = h;
-  lo[idx] = __float2half_rn(v - __half2float(h));
+// n bytes from global `src` to shared `dst` (16-byte aligned): asynchronous 16- or 4-byte copies
+// where the source's alignment allows them, the remaining bytes by plain loads and stores.
+__device__ __forceinline__ void mq_stage(uint8_t* dst, const uint8_t* src, int n, int tid, int nt) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src);
+  int done = 0;
+  if ((a & 15) == 0) {
+    const int n16 = n >> 4;
+    for (int i = tid; i < n16; i += nt) cp_async16(smem_u32(dst + 16 * i), src + 16 * i);
+    done = n16 << 4;
+  } else if ((a & 3) == 0) {
+    const int n4 = n >> 2;
+    for (int i = tid; i < n4; i += nt) cp_async4(smem_u32(dst + 4 * i), src + 4 * i);
+    done = n4 << 2;
+  }
+  for (int i = done + tid; i < n; i += nt) dst[i] = src[i];
+}
+
+// Rows [rix0, rix0 + nrow) of side S (codes, scales, zero points) into the staging buffer `buf`.
+template <int TK>
+__device__ __forceinline__ void mq_stage_side(const SideDev& S, long long rix0, int nrow, uint8_t* buf, int tid,
+                                              int nt) {
+  const int cb = mq_up16(TK * S.row_bytes), sb = S.scales ? mq_up16(TK * S.n_groups * 2) : 0;
+  mq_stage(buf, S.codes + rix0 * S.row_bytes, nrow * S.row_bytes, tid, nt);
+  if (S.scales)
+    mq_stage(buf + cb, reinterpret_cast<const uint8_t*>(S.scales + rix0 * S.n_groups), nrow * S.n_groups * 2, tid, nt);
+  if (S.zeros)
+    mq_stage(buf + cb + sb, reinterpret_cast<const uint8_t*>(S.zeros + rix0 * S.n_groups), nrow * S.n_groups * 2,
+             tid, nt);
+}
+
+// The n (<= 8) bytes at p as a little-endian word: one load when p is aligned for it.
+__device__ __forceinline__ uint64_t mq_bytes(const uint8_t* p, int n) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  if (n == 4 && (a & 3) == 0) return *reinterpret_cast<const uint32_t*>(p);
+  if (n == 2 && (a & 1) == 0) return *reinterpret_cast<const uint16_t*>(p);
+  if (n == 8 && (a & 7) == 0) return *reinterpret_cast<const unsigned long long*>(p);
+  uint64_t w = 0;
+  for (int i = 0; i < n; ++i) w |= (uint64_t)p[i] << (8 * i);
+  return w;
+}
+
+// Stored-domain values of elements j0 .. j0 + 7 (j0 % 8 == 0) of one staged row, with the same
+// arithmetic as stored_value / polar_slot (polar: slots j0 / 2 .. j0 / 2 + 3, (cos, sin) parts).
+__device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, const __half* sc, const __half* zr,
+                                         int j0, float* v, const float* nf4, const float* lloyd, const float* cs,
+                                         const float* sn) {
+  const int f = S.fmt;
+  if (f == KVQ_FMT_FP16) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + 2 * j0);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __half22float2(u2h(u[i]));
+      v[2 * i] = x.x;
+      v[2 * i + 1] = x.y;
+    }
+    return;
+  }
+  if (f == KVQ_FMT_POLAR) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 ab = polar_slot(S, row, sc, (j0 >> 1) + i, cs, sn);
+      v[2 * i] = ab.x;
+      v[2 * i + 1] = ab.y;
+    }
+    return;
+  }
+  if (f == KVQ_FMT_TERNARY || f == KVQ_FMT_SORTED) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = stored_value(S, row, sc, zr, j0 + i, nf4, lloyd);
+    return;
+  }
+  const int b = f == KVQ_FMT_NF4 ? 4 : (f == KVQ_FMT_SIGN ? 1 : S.bits);
+  const uint64_t w = mq_bytes(row + b * (j0 >> 3), b);
+  const uint32_t M = (1u << b) - 1u;
+  if (f == KVQ_FMT_CART) {
+    const float d = __half2float(sc[0]);
+    const int half = 1 << (b - 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (float)((int)((w >> (b * i)) & M) - half) * d;
+    return;
+  }
+  const bool one = S.group >= 8;  // the chunk lies in one group
+  const int g0 = j0 / S.group;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = (int)((w >> (b * i)) & M);
+    const int g = one ? g0 : (j0 + i) / S.group;
+    const float d = __half2float(sc[g]);
+    float x;
+    if (f == KVQ_FMT_INT) {
+      if (S.scale_mode == KVQ_SCALE_MINMAX) x = __fadd_rn(__half2float(zr[g]), (float)c * d);
+      else if (S.scale_mode == KVQ_SCALE_SYMMETRIC) x = ((float)c - 0.5f * (float)M) * d;
+      else x = (float)(c - (1 << (b - 1))) * d;
+    } else if (f == KVQ_FMT_LLOYD) {
+      x = lloyd[c] * d;
+    } else if (f == KVQ_FMT_NF4) {
+      x = nf4[c] * d;
+    } else {  // sign
+      x = c ? d : -d;
+    }
+    v[i] = x;
+  }
+}
+
+// 8 values as fp16 hi halves and the fp16 roundings of their remainders, 16 bytes each.
+__device__ __forceinline__ void mq_store8(__half* hi, __half* lo, int idx, const float* v) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 a = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+    const float2 af = __half22float2(a);
+    h[i] = h2u(a);
+    l[i] = h2u(__floats2half2_rn(v[2 * i] - af.x, v[2 * i + 1] - af.y));
+  }
+  *reinterpret_cast<uint4*>(hi + idx) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(lo + idx) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Transformed queries of one (query, kv-head): row (qi, kvh G + h) of `prep` holds the key-mean
+// term (x sm_scale log2 e) at 0 and q'[D] from kPartStride on.
+template <int D>
+__global__ void __launch_bounds__(256) mq_prep_kernel(LayerDev L, const __half* __restrict__ q,
+                                                      const int* __restrict__ seq_ids,
+                                                      const int* __restrict__ kv_len, float* __restrict__ prep) {
+  __shared__ float qt[kMaxG * D], qa[kMaxG * D];
+  const int kvh = blockIdx.x, qi = blockIdx.y, G = L.Hq / L.Hkv, tid = threadIdx.x;
+  const SideDev& K = L.s[0];
+  if (tid == 0 && kvh == 0) {  // a sequence id out of range attends nothing; report it
+    const int s = seq_ids ? seq_ids[qi] : qi;
+    if (s < 0 || s >= L.B) atomicOr(L.err, (unsigned)KVQ_ERRF_SEQ_ID);
+  }
+  prepare_query<D>(L, q, qi, kvh, G, qt, qa);  // synchronizes internally
+  float* dst = prep + ((long long)qi * L.Hq + kvh * G) * (D + kPartStride);
+  for (int e = tid; e < G * D; e += blockDim.x) dst[(e / D) * (D + kPartStride) + kPartStride + e % D] = qt[e];
+  if (tid < G) {
+    float mu = 0.0f;
+    if (K.mean_sub) {
+      const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+      const __half* qp = q + query_row(L, qi, kvh, G, tid) * D;
+      const __half* mp = K.kmean + ((long long)R.seq * L.Hkv + kvh) * D;
+      for (int j = 0; j < D; ++j) mu = fmaf(__half2float(qp[j]), __half2float(mp[j]), mu);
+    }
+    dst[tid * (D + kPartStride)] = mu * (L.sm_scale * kLog2e);
+  }
 }
 
 template <int D>
-__global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, const __half* __restrict__ q,
+__global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, const float* __restrict__ prep,
                                                                  const int* __restrict__ seq_ids,
                                                                  const int* __restrict__ kv_len, float* __restrict__ work,
                                                                  int n_split, int nsp_total, int n_q) {
@@ -90,8 +257,6 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   __half* Kl = reinterpret_cast<__half*>(smem + C::OFF_KL);
   __half* Vh = reinterpret_cast<__half*>(smem + C::OFF_VH);
   __half* Vl = reinterpret_cast<__half*>(smem + C::OFF_VL);
-  float* qt = reinterpret_cast<float*>(smem + C::OFF_QT);
-  float* qraw = reinterpret_cast<float*>(smem + C::OFF_QA);
   int* r_seq = reinterpret_cast<int*>(smem + C::OFF_META);
   int* r_qa = r_seq + C::QM;
   int* r_qb = r_qa + C::QM;
@@ -103,6 +268,7 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   float* t_ks = t_kc + 256;
   float* t_vc = t_ks + 256;
   float* t_vs = t_vc + 256;
+  uint8_t* raw = smem + C::OFF_RAW;
   __shared__ int pass_seq[MqCfg<D>::QM];
   __shared__ int n_pass;
 
@@ -112,6 +278,9 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   const int q0 = blockIdx.z * QPB;
   const SideDev& K = L.s[0];
   const SideDev& V = L.s[1];
+  const int stK = mq_stage_bytes<C::TK>(K), stV = mq_stage_bytes<C::TK>(V);
+  const int cbK = mq_up16(C::TK * K.row_bytes), sbK = K.scales ? mq_up16(C::TK * K.n_groups * 2) : 0;
+  const int cbV = mq_up16(C::TK * V.row_bytes), sbV = V.scales ? mq_up16(C::TK * V.n_groups * 2) : 0;
 
   // ---- tables
   if (tid < 16) t_nf4[tid] = d_nf4[tid];
@@ -128,43 +297,35 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
       t_vs[k] = d_ph_sin[(1 << V.bits2) - 2 + k];
     }
 
-  // ---- rows: transformed queries as fp16 hi + lo; per-row sequence and causal range
-  for (int qq = 0; qq < QPB; ++qq) {
-    const int qi = q0 + qq;  // uniform over the CTA
-    if (qi < n_q) {
-      prepare_query<D>(L, q, qi, kvh, G, qt, qraw);  // synchronizes internally
-      for (int e = tid; e < G * D; e += C::NT) {
-        const int r = qq * G + e / D, j = e % D;
-        split_store(Qh, Ql, r * C::LD + j, qt[e]);
-      }
-      if (tid < G) {
-        const int r = qq * G + tid;
-        const QueryRange R = query_range(L, qi, seq_ids, kv_len);
-        r_seq[r] = R.qb > R.qa ? R.seq : -1;
-        r_qa[r] = R.qa;
-        r_qb[r] = R.qb;
-        float mu = 0.0f;
-        if (K.mean_sub) {
-          const __half* qp = q + query_row(L, qi, kvh, G, tid) * D;
-          const __half* mp = K.kmean + ((long long)R.seq * L.Hkv + kvh) * D;
-          for (int j = 0; j < D; ++j) mu = fmaf(__half2float(qp[j]), __half2float(mp[j]), mu);
-        }
-        r_mu[r] = mu * (L.sm_scale * kLog2e);
-      }
-    } else {
-      for (int e = tid; e < G * D; e += C::NT) {
-        const int r = qq * G + e / D, j = e % D;
-        split_store(Qh, Ql, r * C::LD + j, 0.0f);
-      }
-      if (tid < G) {
-        const int r = qq * G + tid;
-        r_seq[r] = -1;
-        r_qa[r] = r_qb[r] = 0;
-        r_mu[r] = 0.0f;
-      }
-    }
-    __syncthreads();  // qt / qraw are reused for the next query
+  // ---- rows: the prepared queries as fp16 hi + lo; per-row sequence, causal range, key-mean term
+  for (int e = tid; e < C::QM * (D / 4); e += C::NT) {
+    const int r = e / (D / 4), j = (e % (D / 4)) * 4;
+    const int qi = q0 + r / G, h = r % G;
+    float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (qi < n_q)
+      x = *reinterpret_cast<const float4*>(prep + ((long long)qi * L.Hq + kvh * G + h) * (D + kPartStride) +
+                                           kPartStride + j);
+    const __half2 a = __floats2half2_rn(x.x, x.y), b = __floats2half2_rn(x.z, x.w);
+    const float2 af = __half22float2(a), bf = __half22float2(b);
+    *reinterpret_cast<uint2*>(Qh + r * C::LD + j) = make_uint2(h2u(a), h2u(b));
+    *reinterpret_cast<uint2*>(Ql + r * C::LD + j) =
+        make_uint2(h2u(__floats2half2_rn(x.x - af.x, x.y - af.y)), h2u(__floats2half2_rn(x.z - bf.x, x.w - bf.y)));
   }
+  if (tid < C::QM) {
+    const int r = tid, qi = q0 + r / G, h = r % G;
+    if (qi < n_q) {
+      const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+      r_seq[r] = R.qb > R.qa ? R.seq : -1;
+      r_qa[r] = R.qa;
+      r_qb[r] = R.qb;
+      r_mu[r] = prep[((long long)qi * L.Hq + kvh * G + h) * (D + kPartStride)];
+    } else {
+      r_seq[r] = -1;
+      r_qa[r] = r_qb[r] = 0;
+      r_mu[r] = 0.0f;
+    }
+  }
+  __syncthreads();
   // distinct sequences among the rows that attend anything (in row order)
   if (tid == 0) {
     int n = 0;
@@ -209,117 +370,147 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
     const int per = (ntiles + n_split - 1) / n_split;
     const int it0 = split * per, it1 = min(ntiles, it0 + per);
     const bool a0 = r_seq[row0] == seq, a1 = r_seq[row1] == seq;
+    const bool wact = __any_sync(0xffffffffu, a0 || a1);  // some row of this warp's block attends seq
     const int qa0 = r_qa[row0], qb0 = a0 ? r_qb[row0] : 0, qa1 = r_qa[row1], qb1 = a1 ? r_qb[row1] : 0;
     const long long u = (long long)seq * L.Hkv + kvh;
-    for (int it = it0; it < it1; ++it) {
+    // tile it's packed rows (those below the length) into staging buffer `buf`
+    auto stage = [&](int it, int buf) {
       const int t0 = tstart + it * C::TK;
-      // ---- decode the tile: exact stored values as fp16 hi + lo (rows past the length: 0)
-      for (int e = tid; e < C::TK * D; e += C::NT) {
-        const int t = e / D, j = e % D, tok = t0 + t;
-        float kv = 0.0f, vv = 0.0f;
-        if (tok < len) {
-          const long long rix = u * L.Tcap + tok;
-          kv = mq_value(K, K.codes + rix * K.row_bytes, K.scales + rix * K.n_groups,
-                        K.zeros ? K.zeros + rix * K.n_groups : nullptr, j, t_nf4, t_lk, t_kc, t_ks);
-          vv = mq_value(V, V.codes + rix * V.row_bytes, V.scales + rix * V.n_groups,
-                        V.zeros ? V.zeros + rix * V.n_groups : nullptr, j, t_nf4, t_lv, t_vc, t_vs);
+      const int nrow = min(C::TK, len - t0);
+      uint8_t* bk = raw + buf * (stK + stV);
+      mq_stage_side<C::TK>(K, u * L.Tcap + t0, nrow, bk, tid, C::NT);
+      mq_stage_side<C::TK>(V, u * L.Tcap + t0, nrow, bk + stK, tid, C::NT);
+      cp_async_commit();
+    };
+    if (it0 < it1) stage(it0, 0);
+    for (int it = it0; it < it1; ++it) {
+      const int cur = (it - it0) & 1;
+      if (it + 1 < it1) {
+        stage(it + 1, cur ^ 1);  // its buffer was last read by the decode of tile it - 1
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();  // tile it staged; every warp is done with the previous tile's K and V
+      const int t0 = tstart + it * C::TK;
+      // ---- decode the staged tile: exact stored values as fp16 hi + lo (rows past the length: 0)
+      {
+        const uint8_t* bk = raw + cur * (stK + stV);
+        const uint8_t* bv = bk + stK;
+        const __half* sk = reinterpret_cast<const __half*>(bk + cbK);
+        const __half* zk = K.zeros ? reinterpret_cast<const __half*>(bk + cbK + sbK) : nullptr;
+        const __half* sv = reinterpret_cast<const __half*>(bv + cbV);
+        const __half* zv = V.zeros ? reinterpret_cast<const __half*>(bv + cbV + sbV) : nullptr;
+        for (int e = tid; e < C::TK * (D / 8); e += C::NT) {
+          const int t = e / (D / 8), j0 = (e % (D / 8)) * 8;
+          float kv[8], vv[8];
+          if (t0 + t < len) {
+            mq_chunk(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk ? zk + t * K.n_groups : nullptr, j0, kv, t_nf4,
+                     t_lk, t_kc, t_ks);
+            mq_chunk(V, bv + t * V.row_bytes, sv + t * V.n_groups, zv ? zv + t * V.n_groups : nullptr, j0, vv, t_nf4,
+                     t_lv, t_vc, t_vs);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) kv[i] = vv[i] = 0.0f;
+          }
+          mq_store8(Kh, Kl, t * C::LD + j0, kv);
+          mq_store8(Vh, Vl, t * C::LD + j0, vv);
         }
-        split_store(Kh, Kl, t * C::LD + j, kv);
-        split_store(Vh, Vl, t * C::LD + j, vv);
       }
       __syncthreads();
-      // ---- scores for this warp's 16 rows x 32 tokens
-      float s[C::TK / 8][4];
+      if (wact) {
+        // ---- scores for this warp's 16 rows x 32 tokens
+        float s[C::TK / 8][4];
 #pragma unroll
-      for (int nb = 0; nb < C::TK / 8; ++nb) {
-        s[nb][0] = s[nb][1] = mu0;
-        s[nb][2] = s[nb][3] = mu1;
-      }
+        for (int nb = 0; nb < C::TK / 8; ++nb) {
+          s[nb][0] = s[nb][1] = mu0;
+          s[nb][2] = s[nb][3] = mu1;
+        }
 #pragma unroll 4
-      for (int ks = 0; ks < D / 16; ++ks) {
-        uint32_t ah[4], al[4];
-        ldsm_x4(qh_s + 2 * (a_off + ks * 16), ah[0], ah[1], ah[2], ah[3]);
-        ldsm_x4(ql_s + 2 * (a_off + ks * 16), al[0], al[1], al[2], al[3]);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t ah[4], al[4];
+          ldsm_x4(qh_s + 2 * (a_off + ks * 16), ah[0], ah[1], ah[2], ah[3]);
+          ldsm_x4(ql_s + 2 * (a_off + ks * 16), al[0], al[1], al[2], al[3]);
 #pragma unroll
-        for (int nb = 0; nb < C::TK / 8; nb += 2) {
-          uint32_t bh[4], bl[4];
-          ldsm_x4(kh_s + 2 * (k_off + nb * 8 * C::LD + ks * 16), bh[0], bh[1], bh[2], bh[3]);
-          ldsm_x4(kl_s + 2 * (k_off + nb * 8 * C::LD + ks * 16), bl[0], bl[1], bl[2], bl[3]);
-          mma16816(s[nb], ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
-          mma16816(s[nb], al[0], al[1], al[2], al[3], bh[0], bh[1]);
-          mma16816(s[nb], ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
-          mma16816(s[nb + 1], ah[0], ah[1], ah[2], ah[3], bh[2], bh[3]);
-          mma16816(s[nb + 1], al[0], al[1], al[2], al[3], bh[2], bh[3]);
-          mma16816(s[nb + 1], ah[0], ah[1], ah[2], ah[3], bl[2], bl[3]);
+          for (int nb = 0; nb < C::TK / 8; nb += 2) {
+            uint32_t bh[4], bl[4];
+            ldsm_x4(kh_s + 2 * (k_off + nb * 8 * C::LD + ks * 16), bh[0], bh[1], bh[2], bh[3]);
+            ldsm_x4(kl_s + 2 * (k_off + nb * 8 * C::LD + ks * 16), bl[0], bl[1], bl[2], bl[3]);
+            mma16816(s[nb], ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+            mma16816(s[nb], al[0], al[1], al[2], al[3], bh[0], bh[1]);
+            mma16816(s[nb], ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+            mma16816(s[nb + 1], ah[0], ah[1], ah[2], ah[3], bh[2], bh[3]);
+            mma16816(s[nb + 1], al[0], al[1], al[2], al[3], bh[2], bh[3]);
+            mma16816(s[nb + 1], ah[0], ah[1], ah[2], ah[3], bl[2], bl[3]);
+          }
         }
-      }
-      // ---- causal masks per row, online softmax per row (the quad c = 0..3 shares a row)
-      float tm0 = -INFINITY, tm1 = -INFINITY;
+        // ---- causal masks per row, online softmax per row (the quad c = 0..3 shares a row)
+        float tm0 = -INFINITY, tm1 = -INFINITY;
 #pragma unroll
-      for (int nb = 0; nb < C::TK / 8; ++nb) {
+        for (int nb = 0; nb < C::TK / 8; ++nb) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = t0 + nb * 8 + 2 * c + e;
-          if (!(tok >= qa0 && tok < qb0)) s[nb][e] = -INFINITY;
-          if (!(tok >= qa1 && tok < qb1)) s[nb][2 + e] = -INFINITY;
-          tm0 = fmaxf(tm0, s[nb][e]);
-          tm1 = fmaxf(tm1, s[nb][2 + e]);
+          for (int e = 0; e < 2; ++e) {
+            const int tok = t0 + nb * 8 + 2 * c + e;
+            if (!(tok >= qa0 && tok < qb0)) s[nb][e] = -INFINITY;
+            if (!(tok >= qa1 && tok < qb1)) s[nb][2 + e] = -INFINITY;
+            tm0 = fmaxf(tm0, s[nb][e]);
+            tm1 = fmaxf(tm1, s[nb][2 + e]);
+          }
         }
-      }
-      tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, 1));
-      tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, 2));
-      tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, 1));
-      tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, 2));
-      const float n0 = fmaxf(m0, tm0), n1 = fmaxf(m1, tm1);
-      const float al0 = n0 == -INFINITY ? 1.0f : ex2(m0 - n0), al1 = n1 == -INFINITY ? 1.0f : ex2(m1 - n1);
-      m0 = n0;
-      m1 = n1;
-      l0 *= al0;
-      l1 *= al1;
+        tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, 1));
+        tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, 2));
+        tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, 1));
+        tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, 2));
+        const float n0 = fmaxf(m0, tm0), n1 = fmaxf(m1, tm1);
+        const float al0 = n0 == -INFINITY ? 1.0f : ex2(m0 - n0), al1 = n1 == -INFINITY ? 1.0f : ex2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        l0 *= al0;
+        l1 *= al1;
 #pragma unroll
-      for (int i = 0; i < C::NB; ++i) {
-        o[i][0] *= al0;
-        o[i][1] *= al0;
-        o[i][2] *= al1;
-        o[i][3] *= al1;
-      }
-#pragma unroll
-      for (int nb = 0; nb < C::TK / 8; ++nb) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          s[nb][e] = m0 == -INFINITY ? 0.0f : ex2(s[nb][e] - m0);
-          s[nb][2 + e] = m1 == -INFINITY ? 0.0f : ex2(s[nb][2 + e] - m1);
-          l0 += s[nb][e];
-          l1 += s[nb][2 + e];
-        }
-      }
-      // ---- O += P . V: the score fragments of tokens [16 kk, 16 kk + 16) are P's A fragment
-#pragma unroll
-      for (int kk = 0; kk < C::TK / 16; ++kk) {
-        uint32_t ph[4], pl[4];
-        const float* f[4] = {&s[2 * kk][0], &s[2 * kk][2], &s[2 * kk + 1][0], &s[2 * kk + 1][2]};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __half2 h = __floats2half2_rn(f[i][0], f[i][1]);
-          const float2 hf = __half22float2(h);
-          ph[i] = h2u(h);
-          pl[i] = h2u(__floats2half2_rn(f[i][0] - hf.x, f[i][1] - hf.y));
+        for (int i = 0; i < C::NB; ++i) {
+          o[i][0] *= al0;
+          o[i][1] *= al0;
+          o[i][2] *= al1;
+          o[i][3] *= al1;
         }
 #pragma unroll
-        for (int nb = 0; nb < C::NB; nb += 2) {
-          uint32_t bh[4], bl[4];
-          const int vo = v_off + kk * 16 * C::LD + ch0 + nb * 8;
-          ldsm_x4_t(vh_s + 2 * vo, bh[0], bh[1], bh[2], bh[3]);
-          ldsm_x4_t(vl_s + 2 * vo, bl[0], bl[1], bl[2], bl[3]);
-          mma16816(o[nb], ph[0], ph[1], ph[2], ph[3], bh[0], bh[1]);
-          mma16816(o[nb], pl[0], pl[1], pl[2], pl[3], bh[0], bh[1]);
-          mma16816(o[nb], ph[0], ph[1], ph[2], ph[3], bl[0], bl[1]);
-          mma16816(o[nb + 1], ph[0], ph[1], ph[2], ph[3], bh[2], bh[3]);
-          mma16816(o[nb + 1], pl[0], pl[1], pl[2], pl[3], bh[2], bh[3]);
-          mma16816(o[nb + 1], ph[0], ph[1], ph[2], ph[3], bl[2], bl[3]);
+        for (int nb = 0; nb < C::TK / 8; ++nb) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            s[nb][e] = m0 == -INFINITY ? 0.0f : ex2(s[nb][e] - m0);
+            s[nb][2 + e] = m1 == -INFINITY ? 0.0f : ex2(s[nb][2 + e] - m1);
+            l0 += s[nb][e];
+            l1 += s[nb][2 + e];
+          }
+        }
+        // ---- O += P . V: the score fragments of tokens [16 kk, 16 kk + 16) are P's A fragment
+#pragma unroll
+        for (int kk = 0; kk < C::TK / 16; ++kk) {
+          uint32_t ph[4], pl[4];
+          const float* f[4] = {&s[2 * kk][0], &s[2 * kk][2], &s[2 * kk + 1][0], &s[2 * kk + 1][2]};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __half2 h = __floats2half2_rn(f[i][0], f[i][1]);
+            const float2 hf = __half22float2(h);
+            ph[i] = h2u(h);
+            pl[i] = h2u(__floats2half2_rn(f[i][0] - hf.x, f[i][1] - hf.y));
+          }
+#pragma unroll
+          for (int nb = 0; nb < C::NB; nb += 2) {
+            uint32_t bh[4], bl[4];
+            const int vo = v_off + kk * 16 * C::LD + ch0 + nb * 8;
+            ldsm_x4_t(vh_s + 2 * vo, bh[0], bh[1], bh[2], bh[3]);
+            ldsm_x4_t(vl_s + 2 * vo, bl[0], bl[1], bl[2], bl[3]);
+            mma16816(o[nb], ph[0], ph[1], ph[2], ph[3], bh[0], bh[1]);
+            mma16816(o[nb], pl[0], pl[1], pl[2], pl[3], bh[0], bh[1]);
+            mma16816(o[nb], ph[0], ph[1], ph[2], ph[3], bl[0], bl[1]);
+            mma16816(o[nb + 1], ph[0], ph[1], ph[2], ph[3], bh[2], bh[3]);
+            mma16816(o[nb + 1], pl[0], pl[1], pl[2], pl[3], bh[2], bh[3]);
+            mma16816(o[nb + 1], ph[0], ph[1], ph[2], ph[3], bl[2], bl[3]);
+          }
         }
       }
-      __syncthreads();  // the next tile overwrites K and V
     }
   }
 

@@ -39,14 +39,15 @@ def eff_bits(cache, cfg, T, anchored_rows_by_layer):
 
 
 def measure(cfg: Config, T: int, layers, queries_fn, calib_T=512, seed=0):
-    """Fill `layers` of a cache, decode the queries queries_fn(layer) -> (q [n, Hq, D] fp16,
-    seq_ids, kv_len), and return the mean metrics over layers, units, queries and heads."""
+    """Fill `layers` of a cache, decode the queries queries_fn(layer, K) -> (q [n, Hq, D] fp16,
+    seq_ids, kv_len), or a dict of such query sets by suffix, and return the mean metrics over
+    layers, units, queries and heads (X2 and X3 once per query set, keys suffixed)."""
     dev = "cuda"
     cache = KVCache(cfg, dev)
     B, H, Hq, D = cfg.batch, cfg.n_kv_heads, cfg.n_q_heads, cfg.head_dim
     G = Hq // H
     sm = cfg.sm_scale or 1.0 / math.sqrt(D)
-    x1k, x1v, x2, x3 = [], [], [], []
+    x1k, x1v, x2, x3 = [], [], {}, {}
     for l in layers:
         K = synth.kv_rows(seed, "k", l, list(range(B)), list(range(H)), list(range(T)), D, dev)
         V = synth.kv_rows(seed, "v", l, list(range(B)), list(range(H)), list(range(T)), D, dev)
@@ -58,24 +59,27 @@ def measure(cfg: Config, T: int, layers, queries_fn, calib_T=512, seed=0):
         Kf, Vf = K.float(), V.float()
         x1k.append(((Kf - Kh) ** 2).sum(dim=(2, 3)) / (Kf ** 2).sum(dim=(2, 3)))
         x1v.append(((Vf - Vh) ** 2).sum(dim=(2, 3)) / (Vf ** 2).sum(dim=(2, 3)))
-        q, seq_ids, kv_len = queries_fn(l, K)
-        n = q.shape[0]
-        sid = torch.tensor(seq_ids, dtype=torch.int32, device=dev)
-        kl = torch.tensor(kv_len, dtype=torch.int32, device=dev)
-        out = cache.decode(l, q.to(dev), sid, kl)  # [n, Hq, D]
-        for i in range(n):
-            b, L_ = seq_ids[i], kv_len[i]
-            qi = q[i].to(dev).float()  # [Hq, D]
-            kh = Kh[b].repeat_interleave(G, dim=0)[:, :L_]  # [Hq, L, D]
-            kf = Kf[b].repeat_interleave(G, dim=0)[:, :L_]
-            vf = Vf[b].repeat_interleave(G, dim=0)[:, :L_]
-            lf = torch.einsum("hd,htd->ht", qi, kf) * sm
-            lq = torch.einsum("hd,htd->ht", qi, kh) * sm
-            pf = torch.softmax(lf.double(), dim=-1)
-            lpq = torch.log_softmax(lq.double(), dim=-1)
-            of = torch.einsum("ht,htd->hd", pf.float(), vf)
-            x2.append((torch.linalg.norm(out[i] - of, dim=-1) / torch.linalg.norm(of, dim=-1)).cpu())
-            x3.append((pf * (torch.log(pf.clamp_min(1e-300)) - lpq)).sum(dim=-1).cpu())
+        sets = queries_fn(l, K)
+        if not isinstance(sets, dict):
+            sets = {"": sets}
+        for tag, (q, seq_ids, kv_len) in sets.items():
+            n = q.shape[0]
+            sid = torch.tensor(seq_ids, dtype=torch.int32, device=dev)
+            kl = torch.tensor(kv_len, dtype=torch.int32, device=dev)
+            out = cache.decode(l, q.to(dev), sid, kl)  # [n, Hq, D]
+            for i in range(n):
+                b, L_ = seq_ids[i], kv_len[i]
+                qi = q[i].to(dev).float()  # [Hq, D]
+                kh = Kh[b].repeat_interleave(G, dim=0)[:, :L_]  # [Hq, L, D]
+                kf = Kf[b].repeat_interleave(G, dim=0)[:, :L_]
+                vf = Vf[b].repeat_interleave(G, dim=0)[:, :L_]
+                lf = torch.einsum("hd,htd->ht", qi, kf) * sm
+                lq = torch.einsum("hd,htd->ht", qi, kh) * sm
+                pf = torch.softmax(lf.double(), dim=-1)
+                lpq = torch.log_softmax(lq.double(), dim=-1)
+                of = torch.einsum("ht,htd->hd", pf.float(), vf)
+                x2.setdefault(tag, []).append((torch.linalg.norm(out[i] - of, dim=-1) / torch.linalg.norm(of, dim=-1)).cpu())
+                x3.setdefault(tag, []).append((pf * (torch.log(pf.clamp_min(1e-300)) - lpq)).sum(dim=-1).cpu())
     anchored = {}
     if cfg.anchor_rule == "first_n":
         anchored = {l: cfg.anchor_n for l in cfg.anchor_layers}
@@ -84,8 +88,19 @@ def measure(cfg: Config, T: int, layers, queries_fn, calib_T=512, seed=0):
     bits = eff_bits(cache, cfg, T, anchored)
     cache.close()
     cat = lambda xs: torch.cat([x.flatten().cpu() for x in xs])
-    return {"X1_K": cat(x1k).mean().item(), "X1_V": cat(x1v).mean().item(), "X2_attn_err": cat(x2).mean().item(),
-            "X3_KL": cat(x3).mean().item(), "X5_bits": bits}
+    res = {"X1_K": cat(x1k).mean().item(), "X1_V": cat(x1v).mean().item()}
+    for tag in x2:
+        res["X2_attn_err" + tag] = cat(x2[tag]).mean().item()
+        res["X3_KL" + tag] = cat(x3[tag]).mean().item()
+    res["X5_bits"] = bits
+    return res
+
+
+def proxy_queries(K, b, pos, G):
+    """Proxy queries ("E21W" "What I tested"): the keys of sequence b at positions `pos`, each
+    kv-head's key serving its G query heads, attending the keys before it."""
+    q = K[b][:, pos].transpose(0, 1).repeat_interleave(G, dim=1).contiguous().cpu()  # [n, Hq, D]
+    return q, [b] * len(pos), pos.tolist()
 
 
 def config2():
@@ -98,7 +113,7 @@ def config2():
             v = Side("int", bits, scale="minmax", group=32, rot=rot)
             cfg = Config(n_layers=8, batch=1, n_kv_heads=4, n_q_heads=4, head_dim=256, capacity=6000, k=k, v=v,
                          max_queries=128)
-            qf = lambda l, K: (K[0][:, pos].transpose(0, 1).contiguous().cpu(), [0] * 128, pos.tolist())
+            qf = lambda l, K: proxy_queries(K, 0, pos, 1)
             res[f"{bits}-bit {name}"] = measure(cfg, 6000, range(8), qf, calib_T=6000)
     return res
 
@@ -111,9 +126,12 @@ def config3():
         "D': H256 4-bit K + 3-bit V g128": (Side("int", 4, group=128, rot=256), Side("int", 3, group=128, rot=256)),
         "plain 4-bit g32 K and V": (Side("int", 4, group=32), Side("int", 4, group=32)),
     }
+    pos = synth.proxy_positions(1, 128, 32768, 65536)
     for name, (k, v) in arms.items():
-        cfg = Config(n_layers=8, batch=1, n_kv_heads=4, n_q_heads=16, head_dim=256, capacity=65536, k=k, v=v)
-        qf = lambda l, K: (synth.queries(1, l, 1, 16, 256, 65536), [0], [65536])
+        cfg = Config(n_layers=8, batch=1, n_kv_heads=4, n_q_heads=16, head_dim=256, capacity=65536, k=k, v=v,
+                     max_queries=128)
+        qf = lambda l, K: {"": (synth.queries(1, l, 1, 16, 256, 65536), [0], [65536]),
+                           "_proxy": proxy_queries(K, 0, pos, 4)}
         res[name] = measure(cfg, 65536, (0, 3, 7), qf)
     return res
 
@@ -146,8 +164,13 @@ def config5():
         "(iii) sign g4": (Side("sign", group=4), Side("sign", group=4), {}),
     }
     for name, (k, v, an) in arms.items():
-        cfg = Config(n_layers=32, batch=16, n_kv_heads=8, n_q_heads=32, head_dim=128, capacity=T, k=k, v=v, **an)
-        qf = lambda l, K: (synth.queries(1, l, 16, 32, 128, T), list(range(16)), [T] * 16)
+        cfg = Config(n_layers=32, batch=16, n_kv_heads=8, n_q_heads=32, head_dim=128, capacity=T, k=k, v=v,
+                     max_queries=128, **an)
+
+        def qf(l, K):
+            px = [proxy_queries(K, b, synth.proxy_positions(1 + b, 8, T // 2, T), 4) for b in range(16)]
+            return {"": (synth.queries(1, l, 16, 32, 128, T), list(range(16)), [T] * 16),
+                    "_proxy": (torch.cat([p[0] for p in px]), sum((p[1] for p in px), []), sum((p[2] for p in px), []))}
         res[name] = measure(cfg, T, (0, 1, 31), qf)
     return res
 

@@ -15,6 +15,22 @@ from quantized_decode_attention_append_b200.kvq import Config, KVCache, Side
 TOL = 2e-3  # max relative error (inf-norm per query-head vector) of decode attention
 
 
+def kernel_names(run, want, tries: int = 6) -> str:
+    """Names of the CUDA kernels `run()` launches, seen by the torch profiler.  Its kernel records
+    occasionally arrive incomplete, so it looks again (up to `tries` times) until every name in
+    `want` is present."""
+    from torch.profiler import ProfilerActivity, profile
+    names = ""
+    for _ in range(tries):
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            run()
+            torch.cuda.synchronize()
+        names = " ".join(e.name for e in prof.events())
+        if all(w in names for w in want):
+            break
+    return names
+
+
 def oracle_side(s: Side) -> OQ.Side:
     return OQ.Side(**asdict(s))
 

@@ -9,7 +9,7 @@ tensor-core kernel is the one that ran.
 import pytest
 import torch
 
-from kvq_harness import Case
+from kvq_harness import Case, kernel_names
 from quantized_decode_attention_append_b200 import kvq, synth
 from quantized_decode_attention_append_b200.kvq import Config, Side
 
@@ -70,11 +70,7 @@ def test_mma_kernel_is_the_one_that_runs(k, v):
     q = synth.queries(1, 0, 2, cfg.n_q_heads, 128, 512).cuda()
     c.cache.decode(0, q)
     torch.cuda.synchronize()
-    from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        c.cache.decode(0, q)
-        torch.cuda.synchronize()
-    names = " ".join(e.name for e in prof.events())
+    names = kernel_names(lambda: c.cache.decode(0, q), ["decode_tc_kernel", "merge_kernel"])
     assert "decode_tc_kernel" in names and "merge_kernel" in names
     assert "decode_generic_kernel" not in names
     assert kvq.kvq_last_launch_count(c.cache.h) == 2

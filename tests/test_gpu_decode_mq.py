@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from kvq_harness import Case
+from kvq_harness import Case, kernel_names
 from quantized_decode_attention_append_b200 import kvq, synth
 from quantized_decode_attention_append_b200.kvq import Config, Side
 
@@ -30,6 +30,7 @@ MQ = [
     (64, 1, Side("sorted", 2, group=8), Side("int", 2, scale="sym", group=16),
      dict(anchor_layers=(0,), anchor_rule="window", anchor_n=50)),
     (256, 2, Side("sign", group=4), Side("ternary", group=8), {}),
+    (128, 1, Side("int", 4, group=64), Side("fp16"), {}),
 ]
 
 
@@ -44,6 +45,18 @@ def test_many_proxy_queries_on_one_sequence(D, G, k, v, anc):
     pos = synth.proxy_positions(1, 100, 5, T)  # > 64 rows per CTA: several query blocks
     q = proxies(c, 0, pos, G)
     c.decode_and_compare(0, q, seq_ids=[0] * 100, kv_len=pos.tolist())
+
+
+def test_odd_capacity_unaligned_staging():
+    """Capacity 701 and three kv-heads: a tile's packed ranges start at every alignment, so the
+    staging copies take their 16-byte, 4-byte and plain-byte forms."""
+    D, T = 128, 701
+    cfg = Config(n_layers=1, batch=1, n_kv_heads=3, n_q_heads=3, head_dim=D, capacity=T,
+                 k=Side("polar", 4, 8), v=Side("int", 3, scale="minmax", group=32), max_queries=80)
+    c = Case(cfg, T, chunks=[333, 368])
+    pos = synth.proxy_positions(2, 80, 3, T)
+    q = proxies(c, 0, pos, 1)
+    c.decode_and_compare(0, q, seq_ids=[0] * 80, kv_len=pos.tolist())
 
 
 def test_queries_of_several_sequences_in_one_block():
@@ -68,14 +81,6 @@ def test_multi_query_kernel_is_the_one_that_runs():
     kl = torch.arange(100, 132, dtype=torch.int32, device="cuda")
     c.cache.decode(0, q, sid, kl)
     torch.cuda.synchronize()
-    from torch.profiler import ProfilerActivity, profile
-    names = ""
-    for _ in range(3):
-        with profile(activities=[ProfilerActivity.CUDA]) as prof:
-            c.cache.decode(0, q, sid, kl)
-            torch.cuda.synchronize()
-        names = " ".join(e.name for e in prof.events())
-        if "merge_kernel" in names:
-            break
-    assert "decode_mq_kernel" in names and "decode_generic_kernel" not in names
-    assert kvq.kvq_last_launch_count(c.cache.h) == 2
+    names = kernel_names(lambda: c.cache.decode(0, q, sid, kl), ["mq_prep_kernel", "decode_mq_kernel", "merge_kernel"])
+    assert "mq_prep_kernel" in names and "decode_mq_kernel" in names and "decode_generic_kernel" not in names
+    assert kvq.kvq_last_launch_count(c.cache.h) == 3  # query preparation, split pass, merge
