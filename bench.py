@@ -2,8 +2,10 @@
 
 Default workload (the throughput-stress configuration): 32 layers x 8 KV heads x 32 query
 heads, head_dim 128, batch 16 x 32768 tokens, NF4 K (group 64) + int4 V (group 64), 4.25 bits
-per value.  One step = append one new token per sequence to all 32 layers
-(kvq_quantize_append) and decode attention on all 32 layers (kvq_decode_attention).
+per value.  One step = append one new token per sequence and decode attention on all 32
+layers: kvq_append_decode per layer (one split-K launch that writes the new rows and decodes,
+then the merge; kvq_quantize_append + kvq_decode_attention where the formats have no fused
+kernel or the queries are proxy positions).
 Other workloads: --workload names one of WORKLOADS below.
 
 Timing: W warm-up steps, then K steps between CUDA events on the launching stream, with a
@@ -402,12 +404,23 @@ def run_gpu(args, w, name):
     outs = [torch.empty(n_q, Hq, D, device=dev, dtype=torch.float32) for _ in range(L)]
     launches = {"n": 0}
 
+    # one query per sequence: the decode step is kvq_append_decode (append and decode in one
+    # split-K launch where the layer's formats allow it); proxy queries append, then decode
+    fused_step = not proxy
+
+    def layer_step(l, k, v, q, out):
+        if fused_step:
+            cache.append_decode(l, k, v, q, out=out)
+            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+        else:
+            cache.append(l, k, v)
+            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+            cache.decode(l, q, seq_ids=qsid, kv_len=qlen, out=out)
+            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+
     def step():
         for l in range(L):
-            cache.append(l, knew[l], vnew[l])
-            launches["n"] += kvq.kvq_last_launch_count(cache.h)
-            cache.decode(l, qs[l], seq_ids=qsid, kv_len=qlen, out=outs[l])
-            launches["n"] += kvq.kvq_last_launch_count(cache.h)
+            layer_step(l, knew[l], vnew[l], qs[l], outs[l])
 
     def decode_only():
         for l in range(L):
@@ -498,8 +511,7 @@ def run_gpu(args, w, name):
         if not pipelined:  # small steps: one copy in, one copy out
             d_in.copy_(h_in, non_blocking=True)
             for l in range(L):
-                cache.append(l, d_k[l], d_v[l])
-                cache.decode(l, d_q[l], seq_ids=qsid, kv_len=qlen, out=d_out[l])
+                layer_step(l, d_k[l], d_v[l], d_q[l], d_out[l])
             h_out.copy_(d_out, non_blocking=True)
             return
         copy_stream.wait_stream(main)
@@ -510,8 +522,7 @@ def run_gpu(args, w, name):
                 ev_in[l].record(copy_stream)
         for l in range(L):
             main.wait_event(ev_in[l])
-            cache.append(l, d_k[l], d_v[l])
-            cache.decode(l, d_q[l], seq_ids=qsid, kv_len=qlen, out=d_out[l])
+            layer_step(l, d_k[l], d_v[l], d_q[l], d_out[l])
             ev_out[l].record(main)
         with torch.cuda.stream(copy_stream):
             for l in range(L):
@@ -548,7 +559,9 @@ def run_gpu(args, w, name):
                "config": {"workload": f"{name}: {w['desc']}", "global_batch": world * B, "seq_len": T,
                           "parallelism": f"replicas{world}", "layers": L,
                           "l2": l2_note,
-                          "step": f"append 1 token/seq + decode, all {L} layers, one CUDA graph"},
+                          "step": f"append 1 token/seq + decode, all {L} layers, one CUDA graph"
+                                  + ("; kvq_append_decode per layer" if fused_step else
+                                     "; kvq_quantize_append + kvq_decode_attention per layer")},
                "kv_gbps": dec_bytes_step / (ms_step * 1e-3) / 1e9 * world,
                "decode_ms_per_layer": dec_launch_ms,
                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

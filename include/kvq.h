@@ -266,6 +266,28 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const v
                                         const int32_t* seq_ids, const int32_t* kv_len, void* out,
                                         int32_t out_fp32, float* lse, void* stream);
 
+/* One decode step of `layer`: append n_new tokens to n_seqs sequences, then decode one query per
+ * listed sequence over its whole new length.  Same results as kvq_quantize_append(cache, layer,
+ * k, v, seq_ids, n_seqs, n_new) followed by kvq_decode_attention(cache, layer, q, n_seqs,
+ * seq_ids, NULL, out, out_fp32, lse): the same codes, lengths and outputs.
+ *   k, v, seq_ids, n_seqs, n_new: as kvq_quantize_append (ids distinct).
+ *   q: fp16 device [n_seqs][n_q_heads][head_dim], query s for sequence seq_ids[s] (or s).
+ *   out, out_fp32, lse: as kvq_decode_attention, one row per listed sequence.
+ * Where a register-decode tensor-core kernel serves the layer's formats and the append needs no
+ * key mean, int anchors or per-head formats, one split-K launch writes the new rows (each by the
+ * CTA that reads it, before its tile copies) and decodes, and the merge advances the lengths:
+ * two launches per layer instead of three (anchored layers add their anchor pass).  Elsewhere
+ * the two calls run in turn.  kvq_last_launch_count tells which.  Errors: those of the two
+ * calls (KVQ_ERR_CAPACITY also for n_seqs > max_queries); on the device, a listed sequence
+ * without room for its rows gets none of them, keeps its length and is decoded over its old
+ * rows (KVQ_ERRF_CAPACITY).  Shares the handle's workspace like kvq_decode_attention.
+ * [FMKQ] post 6 "The winning recipe", component 2 (decode anchoring: each generated token is
+ * appended, anchored or not, before the step attends over the cache); the single launch is an
+ * engineering choice of this library, not the pages'. */
+kvq_status kvq_append_decode(kvq_cache* cache, int32_t layer, const void* k_fp16, const void* v_fp16,
+                             const int32_t* seq_ids, int32_t n_seqs, int32_t n_new, const void* q_fp16,
+                             void* out, int32_t out_fp32, float* lse, void* stream);
+
 /* Read and clear the device error word (KVQ_ERRF_* bits) into *flags.  Synchronizes the
  * device. */
 kvq_status kvq_error_flags(kvq_cache* cache, int32_t* flags);

@@ -19,6 +19,7 @@
 
 #include "decode_common.cuh"
 #include "kvq_internal.h"
+#include "quantize_row.cuh"
 
 namespace kvq {
 
@@ -31,6 +32,7 @@ __constant__ float d_lloyd[3][16];
 
 cudaError_t upload_tables_decode(const HostTables& t) {
   cudaError_t e;
+  if ((e = upload_row_tables(t)) != cudaSuccess) return e;  // thresholds of the fused append
   if ((e = cudaMemcpyToSymbol(d_nf4, t.nf4, sizeof(t.nf4))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_tw_re, t.tw_re, sizeof(t.tw_re))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_tw_im, t.tw_im, sizeof(t.tw_im))) != cudaSuccess) return e;
@@ -48,8 +50,11 @@ struct QueryRange {
   int seq, kv_len, len;
   int qa, qb;  // quantized token range
   int aa, ab;  // anchored token range
+  int fresh;   // fused append + decode: rows [len - fresh, len) are this call's new rows
 };
 
+// FUSED: honour a fused append + decode call (L.fuse_n); the plain decode instances compile it out.
+template <bool FUSED = true>
 __device__ __forceinline__ QueryRange query_range(const LayerDev& L, int qi, const int* seq_ids, const int* kv_len) {
   QueryRange r;
   r.seq = seq_ids ? seq_ids[qi] : qi;
@@ -59,9 +64,19 @@ __device__ __forceinline__ QueryRange query_range(const LayerDev& L, int qi, con
     r.len = 0;
     r.kv_len = 0;
     r.qa = r.qb = r.aa = r.ab = 0;
+    r.fresh = 0;
     return r;
   }
   r.len = L.seq_len[r.seq];
+  r.fresh = 0;
+  if (FUSED && L.fuse_n > 0) {  // the stored length before the rows this call appends
+    if (r.len + L.fuse_n <= L.cap) {
+      r.fresh = L.fuse_n;
+      r.len += L.fuse_n;
+    } else if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) {
+      atomicOr(L.err, (unsigned)KVQ_ERRF_CAPACITY);  // no room: none of its rows, attend the old ones
+    }
+  }
   int kl = kv_len ? kv_len[qi] : r.len;
   kl = kl < 0 ? 0 : (kl > r.len ? r.len : kl);
   r.kv_len = kl;
@@ -142,8 +157,14 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
   } else if (K.fmt == KVQ_FMT_POLAR || K.fmt == KVQ_FMT_CART) {
     // Parseval adjoint of the folded rFFT (N = 128): logit = sum_f alpha_f a_f + beta_f b_f,
     // alpha_0 = Q_0/N, beta_0 = Q_64/N, alpha_f = 2 Re Q_f/N, beta_f = 2 Im Q_f/N.
-    __shared__ float tmp[kMaxG * 128];
+    // twiddles of all 128 angles in shared memory: the threads' indices (f n mod N) diverge,
+    // which constant memory would serialise
+    __shared__ float tmp[kMaxG * 128], tc[128], ts[128];
     for (int e = tid; e < G * 128; e += blockDim.x) tmp[e] = qs[e];
+    for (int k = tid; k < 128; k += blockDim.x) {
+      tc[k] = k < 64 ? d_tw_re[k] : -d_tw_re[k - 64];
+      ts[k] = k < 64 ? d_tw_im[k] : -d_tw_im[k - 64];  // -sin
+    }
     __syncthreads();
     for (int e = tid; e < G * 64; e += blockDim.x) {
       const int h = e / 64, f = e % 64;
@@ -151,8 +172,8 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
       float re = 0.0f, im = 0.0f, re64 = 0.0f;
       for (int n = 0; n < 128; ++n) {
         const int k = (f * n) & 127;
-        const float c = k < 64 ? d_tw_re[k] : -d_tw_re[k - 64];
-        const float s = k < 64 ? d_tw_im[k] : -d_tw_im[k - 64];  // -sin
+        const float c = tc[k];
+        const float s = ts[k];
         re += x[n] * c;
         im += x[n] * s;
         if (f == 0) re64 += (n & 1) ? -x[n] : x[n];
@@ -389,7 +410,8 @@ constexpr int merge_groups() { return D >= 256 ? 4 : 512 / D; }
 template <int D>
 __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L, const float* __restrict__ work,
                                                                      int n_split, int nsp, void* __restrict__ out,
-                                                                     int out_fp32, float* __restrict__ lse) {
+                                                                     int out_fp32, float* __restrict__ lse,
+                                                                     const int* __restrict__ seq_ids) {
   constexpr int SP = merge_groups<D>(), NT = D * SP, NWP = NT / 32;
   const int qh = blockIdx.x;  // qi * Hq + h (this view's heads)
   const int tid = threadIdx.x, j = tid % D, sg = tid / D;
@@ -454,7 +476,12 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
     __syncthreads();
   } else if (V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART) {
     // x_n = (1/N) [a_0 + b_0 (-1)^n + 2 sum_{f=1}^{63} (a_f cos(2 pi f n/N) - b_f sin(2 pi f n/N))]
+    __shared__ float tc[128], tsn[128];  // divergent indices: shared memory, not constant memory
     if (tid < D) tmp[tid] = ov[tid];
+    if (tid < 128) {
+      tc[tid] = tid < 64 ? d_tw_re[tid] : -d_tw_re[tid - 64];
+      tsn[tid] = tid < 64 ? -d_tw_im[tid] : d_tw_im[tid - 64];  // sin(2 pi k / N)
+    }
     __syncthreads();
     if (tid < 128) {
       const int n = tid;
@@ -462,8 +489,8 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
       float sacc = 0.0f;
       for (int f = 1; f < 64; ++f) {
         const int k = (f * n) & 127;
-        const float c = k < 64 ? d_tw_re[k] : -d_tw_re[k - 64];
-        const float sn = k < 64 ? -d_tw_im[k] : d_tw_im[k - 64];  // sin(2 pi k / N)
+        const float c = tc[k];
+        const float sn = tsn[k];
         sacc += tmp[2 * f] * c - tmp[2 * f + 1] * sn;
       }
       ov[n] = (acc + 2.0f * sacc) / 128.0f;
@@ -478,6 +505,15 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
     if (out_fp32) reinterpret_cast<float*>(out)[orow * D + tid] = v;
     else reinterpret_cast<__half*>(out)[orow * D + tid] = __float2half_rn(v);
     if (lse && tid == 0) lse[orow] = Ls > 0.0f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  }
+  // fused append + decode: every read of this call is done (the split pass ran before), so the
+  // query's sequence takes its new length here (one CTA per query; sequences are distinct)
+  if (L.fuse_n > 0 && tid == 0 && qh % L.Hq == 0) {
+    const int qi = qh / L.Hq, b = seq_ids ? seq_ids[qi] : qi;
+    if (b >= 0 && b < L.B) {
+      const int nl = L.seq_len[b] + L.fuse_n;
+      if (nl <= L.cap) L.seq_len[b] = nl;
+    }
   }
 }
 
@@ -509,14 +545,16 @@ static int mma_split_count(long long units, int ntiles, int slots) {
 typedef void (*MmaKernel)(LayerDev, const __half*, const int*, const int*, float*, int, int);
 
 struct MmaPlan {
-  MmaKernel kern;
+  MmaKernel kern;   // decode only
+  MmaKernel fkern;  // fused append + decode (same tiles and splits)
   int smem, tile, threads;
 };
 
-template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int ST>
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int ST, int MB>
 static MmaPlan mma_plan_of() {
   using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, ST>;
-  return MmaPlan{decode_tc_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST>, C::SMEM, C::TILE, C::NTH};
+  return MmaPlan{decode_tc_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST>,
+                 decode_tc_fused_kernel<D, G, KF, GK, VF, GV, NW, TPW, ST, MB>, C::SMEM, C::TILE, C::NTH};
 }
 
 static int code_fmt(const SideDev& S, bool is_v) {
@@ -539,23 +577,25 @@ static bool pick_mma(const LayerDev& L, MmaPlan* out) {
   const int kf = code_fmt(L.s[0], false), vf = code_fmt(L.s[1], true);
   if (kf < 0 || vf < 0) return false;
   const int gk = L.s[0].group, gv = vf == CF_FP16 ? 128 : L.s[1].group;
-#define KVQ_MMA(D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_)                                     \
+// Last argument: CTAs per SM of the plain instance (shared memory or registers), which its fused
+// append + decode twin is held to.
+#define KVQ_MMA(D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_, MB_)                                \
   if (L.D == D_ && G == G_ && kf == KF_ && gk == GK_ && vf == VF_ && gv == GV_) {                \
-    *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_>();                          \
+    *out = mma_plan_of<D_, G_, KF_, GK_, VF_, GV_, NW_, TPW_, ST_, MB_>();                     \
     return true;                                                                              \
   }
-  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 8, 32, 2)
-  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 4, 64, 2)
-  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
-  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 8, 32, 2)
-  KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2)
-  KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 32, 3)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_SYM2, 128, 4, 32, 3)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT3, 128, 4, 32, 3)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4)
-  KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2)
-  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 4, 16, 3)
+  KVQ_MMA(128, 4, CF_NF4, 64, CF_INT4, 64, 8, 32, 2, 2)
+  KVQ_MMA(128, 4, CF_INT4, 64, CF_INT4, 64, 4, 64, 2, 3)
+  KVQ_MMA(128, 4, CF_INT4, 32, CF_INT4, 32, 8, 32, 2, 2)
+  KVQ_MMA(128, 2, CF_INT4, 32, CF_INT4, 32, 8, 32, 2, 2)
+  KVQ_MMA(128, 4, CF_SIGN, 4, CF_SIGN, 4, 8, 32, 2, 2)
+  KVQ_MMA(128, 4, CF_TERN, 8, CF_TERN, 8, 8, 32, 2, 2)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT2, 128, 4, 32, 3, 2)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_SYM2, 128, 4, 32, 3, 2)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT3, 128, 4, 32, 3, 2)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_INT4, 128, 4, 16, 4, 3)
+  KVQ_MMA(256, 4, CF_INT4, 128, CF_FP16, 128, 4, 16, 2, 2)
+  KVQ_MMA(256, 4, CF_INT4, 32, CF_INT4, 32, 4, 16, 3, 2)
 #undef KVQ_MMA
   return false;
 }
@@ -605,6 +645,15 @@ static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
   }
 }
 
+// Whether one decode launch can also append this call's rows (fused append + decode): a
+// register-decode tensor-core instance serves the pair, and the append needs none of the extras
+// (key mean, int anchors, head groups) that only the standalone append kernels carry.
+bool fused_decode_ok(const LayerDev& L, int n_q) {
+  MmaPlan p;
+  return pick_mma(L, &p) && !use_mq(L, n_q) && !L.s[0].mean_sub && !L.s[1].mean_sub && L.anchor_bits == 16 &&
+         L.Hkv == L.Hkv_all;
+}
+
 // Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).
 int decode_partials(const LayerDev& L, int n_q, int num_sms) {
   if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 2;  // + anchor split, + prepared queries
@@ -622,6 +671,7 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   MmaPlan p;
   int n_quant;  // quantized partials per (query, head)
   if (use_mq(L, n_q)) {
+    if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
     using MC = MqCfg<D>;
     static int dyn_max = -1;  // one per instantiation (the attribute is per kernel)
     if (dyn_max < 0) {  // the opt-in limit covers static + dynamic shared memory
@@ -661,6 +711,21 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     const int n_split = mma_split_count((long long)n_q * L.Hkv, L.Tcap / p.tile, slots);
     n_quant = n_split;
     const int nsp = n_quant + (L.anchored ? 1 : 0);
+    if (L.fuse_n > 0) {  // the fused instance: same tiles and splits, the new rows written first
+      static MmaKernel fset[32] = {};
+      bool seen = false;
+      for (int i = 0; i < 32 && fset[i]; ++i) seen |= fset[i] == p.fkern;
+      if (!seen) {
+        cudaError_t e = cudaFuncSetAttribute(p.fkern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+        if (e != cudaSuccess) return e;
+        for (int i = 0; i < 32; ++i)
+          if (!fset[i]) {
+            fset[i] = p.fkern;
+            break;
+          }
+      }
+      p.kern = p.fkern;
+    }
     p.kern<<<dim3(n_split, L.Hkv, n_q), p.threads, p.smem, st>>>(L, q, seq_ids, kv_len, work, n_split, nsp);
     ++nl;
     cudaError_t e = cudaGetLastError();
@@ -673,7 +738,7 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     }
   }
   const int nsp = n_quant + (L.anchored ? 1 : 0);
-  merge_kernel<D><<<n_q * L.Hq, D * merge_groups<D>(), 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse);
+  merge_kernel<D><<<n_q * L.Hq, D * merge_groups<D>(), 0, st>>>(L, work, n_quant, nsp, out, out_fp32, lse, seq_ids);
   ++nl;
   if (launches) *launches = nl;
   return cudaGetLastError();

@@ -138,6 +138,18 @@ __device__ __forceinline__ uint64_t mq_bytes(const uint8_t* p, int n) {
   return w;
 }
 
+// The 64 bits that start at bit `bit` of the staged bytes at p (LSB-first), from three aligned
+// 32-bit shared-memory words.  May read up to 11 bytes past the field: the staging buffers are
+// followed by more staged data, so the reads stay inside the CTA's shared memory.
+__device__ __forceinline__ uint64_t mq_bits64(const uint8_t* p, int bit) {
+  const uint8_t* a = p + (bit >> 3);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(reinterpret_cast<uintptr_t>(a) & ~uintptr_t(3));
+  const int sh = (int)((reinterpret_cast<uintptr_t>(a) & 3) * 8) + (bit & 7);  // 0 .. 31
+  const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
+  const uint32_t lo = __funnelshift_r(w0, w1, sh), hi = __funnelshift_r(w1, w2, sh);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 // Stored-domain values of elements j0 .. j0 + 7 (j0 % 8 == 0) of one staged row, with the same
 // arithmetic as stored_value / polar_slot (polar: slots j0 / 2 .. j0 / 2 + 3, (cos, sin) parts).
 __device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, const __half* sc, const __half* zr,
@@ -155,12 +167,17 @@ __device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, c
     }
     return;
   }
-  if (f == KVQ_FMT_POLAR) {
+  if (f == KVQ_FMT_POLAR) {  // slots f0 .. f0 + 3: magnitude fields, then phase fields, read at once
+    const int bm = S.bits, bp = S.bits2, f0 = j0 >> 1;
+    const uint64_t mw = mq_bits64(row, f0 * bm), pw = mq_bits64(row, 64 * bm + f0 * bp);
+    const uint32_t mm = (1u << bm) - 1u, pm = (1u << bp) - 1u;
+    const float s = __half2float(sc[0]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 ab = polar_slot(S, row, sc, (j0 >> 1) + i, cs, sn);
-      v[2 * i] = ab.x;
-      v[2 * i + 1] = ab.y;
+      const float m = (float)(uint32_t)((mw >> (i * bm)) & mm) * s;
+      const int k = (int)((pw >> (i * bp)) & pm);
+      v[2 * i] = __fmul_rn(m, cs[k]);
+      v[2 * i + 1] = __fmul_rn(m, sn[k]);
     }
     return;
   }
@@ -235,7 +252,7 @@ __global__ void __launch_bounds__(256) mq_prep_kernel(LayerDev L, const __half* 
   if (tid < G) {
     float mu = 0.0f;
     if (K.mean_sub) {
-      const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+      const QueryRange R = query_range<false>(L, qi, seq_ids, kv_len);
       const __half* qp = q + query_row(L, qi, kvh, G, tid) * D;
       const __half* mp = K.kmean + ((long long)R.seq * L.Hkv + kvh) * D;
       for (int j = 0; j < D; ++j) mu = fmaf(__half2float(qp[j]), __half2float(mp[j]), mu);
@@ -314,7 +331,7 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   if (tid < C::QM) {
     const int r = tid, qi = q0 + r / G, h = r % G;
     if (qi < n_q) {
-      const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+      const QueryRange R = query_range<false>(L, qi, seq_ids, kv_len);
       r_seq[r] = R.qb > R.qa ? R.seq : -1;
       r_qa[r] = R.qa;
       r_qb[r] = R.qb;

@@ -65,8 +65,6 @@ __device__ __forceinline__ uint32_t and_or(uint32_t x, uint32_t mask, uint32_t m
   return r;
 }
 
-__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo_part, float hi_part) {
   return h2u(__floats2half2_rn(lo_part, hi_part));
@@ -418,11 +416,67 @@ __device__ __forceinline__ void int3_transcode(const unsigned char* src, unsigne
 
 __device__ __forceinline__ bool head_ok_of(int c, int G) { return c < G; }
 
-template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
-__global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH) decode_tc_kernel(LayerDev L, const __half* __restrict__ q,
-                                                            const int* __restrict__ seq_ids,
-                                                            const int* __restrict__ kv_len, float* __restrict__ work,
-                                                            int n_split, int nsp_total) {
+// Append family and code bits of a tensor-core code format (the grid its rows are written with).
+template <int F> struct TcFam { static constexpr int fam = FAM_ABSMAX, bits = F; };  // CF_INT2 / CF_INT4
+template <> struct TcFam<CF_INT3> { static constexpr int fam = FAM_ABSMAX, bits = 3; };
+template <> struct TcFam<CF_SYM2> { static constexpr int fam = FAM_SYM, bits = 2; };
+template <> struct TcFam<CF_NF4> { static constexpr int fam = FAM_NF4, bits = 0; };
+template <> struct TcFam<CF_SIGN> { static constexpr int fam = FAM_SIGN, bits = 0; };
+template <> struct TcFam<CF_TERN> { static constexpr int fam = FAM_TERNARY, bits = 0; };
+
+// Fused append + decode: the new rows of (query qi's sequence, kv-head kvh) that this CTA owns
+// are written by warp 0 before any tile is copied.  A new row inside the quantized range belongs
+// to the CTA whose tiles cover it (the only reader of its codes in this launch); the others
+// (anchored rows, read later from their anchor copies) to split 0.  One row per lane group of
+// head_dim / 32 lanes, as in the append kernels, with the same arithmetic (quantize_slice).
+// Not inlined: its registers then stay out of the decode loop's allocation (called once per CTA);
+// the fused kernel's LayerDev is a __grid_constant__ parameter, so the reference reads it in place.
+template <int D, int KF, int GK, int VF, int GV>
+__device__ __noinline__ void fused_append_rows(const LayerDev& L, const QueryRange& R, int qi, int kvh, int split,
+                                               int t_lo, int t_hi) {
+  constexpr int LPR = D / 32, RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31, li = lane % LPR;
+  const int p0 = R.len - R.fresh;
+  const int u = R.seq * L.Hkv + kvh;
+  for (int base = 0; base < R.fresh; base += RPW) {
+    const int i = base + lane / LPR, p = p0 + i;
+    const bool in_q = p >= R.qa && p < R.qb;
+    const bool mine = i < R.fresh && (in_q ? (p >= t_lo && p < t_hi) : split == 0);
+    if (!__any_sync(0xffffffffu, mine)) continue;
+    const long long in_row = ((long long)qi * L.Hkv_all + L.h0 + kvh) * L.fuse_n + (mine ? i : 0);
+    uint4 cw[4];
+    const uint4* pk = reinterpret_cast<const uint4*>(L.fuse_k + in_row * D) + li * 4;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) cw[c4] = mine ? __ldg(pk + c4) : make_uint4(0u, 0u, 0u, 0u);
+    quantize_slice<TcFam<KF>::fam, GK, TcFam<KF>::bits, false>(L, L.s[0], cw, mine, u, p, R.len);
+    const uint4* pv = reinterpret_cast<const uint4*>(L.fuse_v + in_row * D) + li * 4;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) cw[c4] = mine ? __ldg(pv + c4) : make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (VF == CF_FP16) {  // fp16 V: the row as it comes, and its anchor copy
+      const SideDev& S = L.s[1];
+      if (mine) {
+        uint4* dst = reinterpret_cast<uint4*>(S.codes + ((long long)u * L.Tcap + p) * S.row_bytes) + li * 4;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) dst[c4] = cw[c4];
+        if (in_anchor(L, p, R.len)) {
+          uint4* ap = reinterpret_cast<uint4*>(S.anchors + ((long long)u * L.anchor_rows + anchor_slot(L, p)) * D) + li * 4;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) ap[c4] = cw[c4];
+        }
+      }
+    } else {
+      quantize_slice<TcFam<VF>::fam, GV, TcFam<VF>::bits, false>(L, L.s[1], cw, mine, u, p, R.len);
+    }
+  }
+  // the rows were written through the generic proxy; the tile copies read them through the async one
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
+}
+
+// The split-K pass; FUSE: the fused append + decode step (see fused_append_rows).
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES, bool FUSE>
+__device__ __forceinline__ void decode_tc_body(const LayerDev& L, const __half* __restrict__ q,
+                                               const int* __restrict__ seq_ids, const int* __restrict__ kv_len,
+                                               float* __restrict__ work, int n_split, int nsp_total) {
   using C = TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // full[s]: tile landed (bytes)
@@ -433,7 +487,7 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int split = blockIdx.x, kvh = blockIdx.y, qi = blockIdx.z;
-  const QueryRange R = query_range(L, qi, seq_ids, kv_len);
+  const QueryRange R = query_range<FUSE>(L, qi, seq_ids, kv_len);
   const SideDev& K = L.s[0];
   const SideDev& V = L.s[1];
   const long long u = (long long)R.seq * L.Hkv + kvh;
@@ -469,6 +523,20 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
   };
 
   const bool producer = C::PROD && warp == NW;  // lane 0 of the extra warp moves the tiles
+  // Fused append + decode: this call's new rows that this CTA owns are written by warp 0 before a
+  // copy reads them.  Without a producer warp, when the first copies hold none of them, those
+  // copies go out first and the rows are written while they are in flight (the issuing thread is
+  // in warp 0, and every later copy follows a CTA barrier).
+  const int t_lo = tstart + it0 * C::TILE, t_hi = tstart + (it0 + nmy) * C::TILE;
+  bool fuse_late = false;
+  if constexpr (FUSE) {
+    if (R.fresh > 0) {
+      const int p0 = R.len - R.fresh, first_hi = min(t_hi, t_lo + (STAGES - 1) * C::TILE);
+      const int a = max(p0, max(R.qa, t_lo)), b = min(R.len, min(R.qb, first_hi));  // owned rows in the first copies
+      fuse_late = !C::PROD && a >= b;
+      if (!fuse_late && warp == 0) fused_append_rows<D, KF, GK, VF, GV>(L, R, qi, kvh, split, t_lo, t_hi);
+    }
+  }
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) {
@@ -488,6 +556,9 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s)
       if (s < nmy) issue(it0 + s, s);
+  }
+  if constexpr (FUSE) {
+    if (fuse_late && warp == 0) fused_append_rows<D, KF, GK, VF, GV>(L, R, qi, kvh, split, t_lo, t_hi);
   }
 
   // ---- while the first tiles are in flight: NF4 table, query fragments
@@ -943,4 +1014,22 @@ __global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH
     }
     P[kPartStride + j] = osum;
   }
+}
+
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES>
+__global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH)
+    decode_tc_kernel(LayerDev L, const __half* __restrict__ q, const int* __restrict__ seq_ids,
+                     const int* __restrict__ kv_len, float* __restrict__ work, int n_split, int nsp_total) {
+  decode_tc_body<D, G, KF, GK, VF, GV, NW, TPW, STAGES, false>(L, q, seq_ids, kv_len, work, n_split, nsp_total);
+}
+
+// The fused append + decode instance: held to MINB CTAs per SM (the plain instance's occupancy),
+// so that the once-per-CTA row quantization may spill but never costs residency; LayerDev is a
+// __grid_constant__ parameter, so the non-inlined row quantization reads it in place.
+template <int D, int G, int KF, int GK, int VF, int GV, int NW, int TPW, int STAGES, int MINB>
+__global__ void __launch_bounds__(TcCfg<D, KF, GK, VF, GV, NW, TPW, STAGES>::NTH, MINB)
+    decode_tc_fused_kernel(const __grid_constant__ LayerDev L, const __half* __restrict__ q,
+                           const int* __restrict__ seq_ids, const int* __restrict__ kv_len,
+                           float* __restrict__ work, int n_split, int nsp_total) {
+  decode_tc_body<D, G, KF, GK, VF, GV, NW, TPW, STAGES, true>(L, q, seq_ids, kv_len, work, n_split, nsp_total);
 }

@@ -751,6 +751,43 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* h, int32_t layer, const void*
   return decode_groups(h, layer, q, n_q, seq_ids, kv_len, out, out_fp32, lse, ws, stream);
 }
 
+// Append then decode in one split-K launch (plus the merge) where the layer allows it; otherwise
+// the two calls in turn.  Query i belongs to listed sequence i and attends its whole new length.
+kvq_status kvq_append_decode(kvq_cache* h, int32_t layer, const void* k, const void* v, const int32_t* seq_ids,
+                             int32_t n_seqs, int32_t n_new, const void* q, void* out, int32_t out_fp32, float* lse,
+                             void* stream) {
+  if (!h || !k || !v || !q || !out || layer < 0 || layer >= h->cfg.n_layers || n_new < 1) return KVQ_ERR_INVALID_ARG;
+  if (seq_ids ? (n_seqs < 1 || n_seqs > h->cfg.batch) : n_seqs != h->cfg.batch) return KVQ_ERR_INVALID_ARG;
+  if (n_seqs > h->cfg.max_queries) return KVQ_ERR_CAPACITY;
+  if (layer_needs_chan(h, layer) && !h->chan_set[layer]) return KVQ_ERR_STATE;
+  if ((uintptr_t)k % 16 || (uintptr_t)v % 16) return KVQ_ERR_INVALID_ARG;
+  if (n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  if (!seq_ids && h->len_exact[layer] && (int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
+  if ((int64_t)n_seqs * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
+  LayerDev L = layer_dev(h, layer, 0);
+  if (h->grp[layer].size() != 1 || !fused_decode_ok(L, n_seqs)) {
+    kvq_status s = kvq_quantize_append(h, layer, k, v, seq_ids, n_seqs, n_new, stream);
+    if (s != KVQ_OK) return s;
+    const int na = h->last_launches;
+    s = decode_groups(h, layer, q, n_seqs, seq_ids, nullptr, out, out_fp32, lse, h->work, stream);
+    h->last_launches += na;
+    return s;
+  }
+  L.fuse_k = reinterpret_cast<const __half*>(k);
+  L.fuse_v = reinterpret_cast<const __half*>(v);
+  L.fuse_n = n_new;
+  int n = 0;
+  const cudaError_t e = launch_decode(L, reinterpret_cast<const __half*>(q), n_seqs, seq_ids, nullptr, out,
+                                      out_fp32 ? 1 : 0, lse, h->work, h->num_sms, h->cfg.max_queries,
+                                      reinterpret_cast<cudaStream_t>(stream), &n);
+  h->last_launches = n;
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  const int64_t nl = (int64_t)h->max_len[layer] + n_new;
+  h->max_len[layer] = (int)(nl < h->cfg.capacity ? nl : h->cfg.capacity);
+  if (seq_ids) h->len_exact[layer] = false;
+  return KVQ_OK;
+}
+
 kvq_status kvq_error_flags(kvq_cache* h, int32_t* flags) {
   if (!h || !flags) return KVQ_ERR_INVALID_ARG;
   unsigned v = 0;

@@ -9,6 +9,10 @@
 
 namespace kvq {
 
+// fp16 pairs as 32-bit words and back
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
 constexpr int kMaxSplit = 256;     // split-K partitions per (query, kv-head)
 constexpr int kPartStride = 4;     // floats of (m, l, pad, pad) before o[D] in a partial
 
@@ -46,6 +50,12 @@ struct LayerDev {
   int app_n;
   long long test_stall;  // test hook (0 = off): the decode's first stage wait polls a barrier nothing
                          // arrives on for this many clock cycles, then gives up
+  // fused append + decode (fuse_n > 0): query i's sequence also receives fuse_n new rows, input
+  // rows [n_q][Hkv_all][fuse_n][D] fp16 of K (fuse_k) and V (fuse_v); the decode kernel writes
+  // them before it reads them and the merge advances the stored length
+  const __half* fuse_k;
+  const __half* fuse_v;
+  int fuse_n;
 };
 
 // Row of query head h (of kv-head kvh of the view, G query heads per kv-head) of query qi in the
@@ -97,6 +107,8 @@ cudaError_t launch_key_mean(const LayerDev& L, const __half* k, int n_new, cudaS
 
 // Split-K partials per (query, head) one decode call on `L` writes (workspace sizing).
 int decode_partials(const LayerDev& L, int n_q, int num_sms);
+// Fused append + decode is available for this view and query count (see decode.cu).
+bool fused_decode_ok(const LayerDev& L, int n_q);
 
 // Fixed device scratch for the no-allocation decode entry point (decode.cu).
 size_t static_work_floats();

@@ -48,6 +48,7 @@ class kvq_layout(C.Structure):
 EXPORTS = ["kvq_arena_bytes", "kvq_create", "kvq_arena_bytes_layers", "kvq_create_layers", "kvq_arena_bytes_heads",
            "kvq_create_heads", "kvq_free", "kvq_get_layout", "kvq_get_layout_head", "kvq_set_chan_scale", "kvq_set_seq_len",
            "kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention", "kvq_decode_attention_noalloc",
+           "kvq_append_decode",
            "kvq_error_flags", "kvq_nf4_levels", "kvq_lloyd_levels",
            "kvq_last_launch_count", "kvq_status_str"]
 
@@ -79,6 +80,7 @@ def lib() -> C.CDLL:
         L.kvq_dequantize.argtypes = [vp, i32, i32, i32, i32, i32, vp, i32, vp]
         L.kvq_decode_attention.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
         L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, vp, vp]
+        L.kvq_append_decode.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp]
         L.kvq_error_flags.argtypes = [vp, C.POINTER(i32)]
         L.kvq_nf4_levels.argtypes = [C.POINTER(C.c_float)]
         L.kvq_lloyd_levels.argtypes = [i32, C.POINTER(C.c_float)]
@@ -273,6 +275,15 @@ def kvq_decode_attention_noalloc(h, layer: int, q16, n_q: int, seq_ids, kv_len, 
                                               _ptr(lse), _stream(stream)), "kvq_decode_attention_noalloc")
 
 
+def kvq_append_decode(h, layer: int, k16, v16, seq_ids, n_seqs: int, n_new: int, q16, out, lse=None, stream=None):
+    """kvq_quantize_append then kvq_decode_attention (one query per listed sequence), in one
+    split-K launch where the layer allows it."""
+    import torch
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    _check(lib().kvq_append_decode(h, layer, _ptr(k16), _ptr(v16), _ptr(seq_ids), n_seqs, n_new, _ptr(q16), _ptr(out),
+                                   fp32, _ptr(lse), _stream(stream)), "kvq_append_decode")
+
+
 def kvq_error_flags(h) -> int:
     f = C.c_int32(0)
     _check(lib().kvq_error_flags(h, C.byref(f)), "kvq_error_flags")
@@ -401,6 +412,38 @@ class KVCache:
         self._check_rows("k", k16, n_seqs)
         self._check_rows("v", v16, n_seqs, k16.shape[2])
         kvq_quantize_append(self.h, layer, k16, v16, seq_ids, n_seqs, k16.shape[2], stream)
+
+    def append_decode(self, layer, k16, v16, q16, seq_ids=None, fp32=True, lse=False, out=None, stream=None):
+        """One decode step: append k16/v16 [n_seqs, n_kv_heads, n, head_dim] to the sequences
+        `seq_ids` (or every sequence), then decode q16 [n_seqs, n_q_heads, head_dim], query s over
+        sequence seq_ids[s]'s whole new length.  Returns out (and lse)."""
+        import torch
+        c = self.cfg
+        n_seqs = c.batch
+        if seq_ids is not None:
+            if seq_ids.dtype != torch.int32 or not seq_ids.is_cuda or seq_ids.dim() != 1 or not seq_ids.is_contiguous():
+                raise ValueError("seq_ids: need a contiguous 1-D int32 CUDA tensor")
+            self._check_device("seq_ids", seq_ids)
+            n_seqs = seq_ids.numel()
+        self._check_rows("k", k16, n_seqs)
+        self._check_rows("v", v16, n_seqs, k16.shape[2])
+        if q16.dtype != torch.float16 or not q16.is_cuda or not q16.is_contiguous() or \
+                tuple(q16.shape) != (n_seqs, c.n_q_heads, c.head_dim):
+            raise ValueError(f"q: need a contiguous fp16 CUDA tensor [{n_seqs}, {c.n_q_heads}, {c.head_dim}], got "
+                             f"{q16.dtype} {tuple(q16.shape)} on {q16.device}")
+        self._check_device("q", q16)
+        if out is None:
+            out = torch.empty(n_seqs, c.n_q_heads, c.head_dim, device=q16.device,
+                              dtype=torch.float32 if fp32 else torch.float16)
+        elif out.dtype not in (torch.float32, torch.float16) or not out.is_cuda or not out.is_contiguous() or \
+                tuple(out.shape) != (n_seqs, c.n_q_heads, c.head_dim):
+            raise ValueError(f"out: need a contiguous fp32 or fp16 CUDA tensor [{n_seqs}, {c.n_q_heads}, "
+                             f"{c.head_dim}], got {out.dtype} {tuple(out.shape)} on {out.device}")
+        else:
+            self._check_device("out", out)
+        l = torch.empty(n_seqs, c.n_q_heads, device=q16.device, dtype=torch.float32) if lse else None
+        kvq_append_decode(self.h, layer, k16, v16, seq_ids, n_seqs, k16.shape[2], q16, out, l, stream)
+        return (out, l) if lse else out
 
     def dequantize(self, layer, side, t0, nt, domain=DOMAIN_STORED, fp32=True, stream=None):
         import torch
