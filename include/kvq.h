@@ -273,11 +273,12 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const v
  *   k, v, seq_ids, n_seqs, n_new: as kvq_quantize_append (ids distinct).
  *   q: fp16 device [n_seqs][n_q_heads][head_dim], query s for sequence seq_ids[s] (or s).
  *   out, out_fp32, lse: as kvq_decode_attention, one row per listed sequence.
- * Where a register-decode tensor-core kernel serves the layer's formats and the append needs no
- * key mean, int anchors or per-head formats, one split-K launch writes the new rows (each by the
- * CTA that reads it, before its tile copies) and decodes, and the merge advances the lengths:
- * two launches per layer instead of three (anchored layers add their anchor pass).  Elsewhere
- * the two calls run in turn.  kvq_last_launch_count tells which.  Errors: those of the two
+ * Where a register-decode tensor-core kernel serves the layer's formats, the append needs no
+ * key mean, int anchors or per-head formats, and the split-K grid fits in one wave of resident
+ * CTAs (a latency-bound step), one split-K launch writes the new rows (each by the CTA that
+ * reads it, before its tile copies) and decodes, and the merge advances the lengths: two
+ * launches per layer instead of three (anchored layers add their anchor pass).  Elsewhere the
+ * two calls run in turn.  kvq_last_launch_count tells which.  Errors: those of the two
  * calls (KVQ_ERR_CAPACITY also for n_seqs > max_queries); on the device, a listed sequence
  * without room for its rows gets none of them, keeps its length and is decoded over its old
  * rows (KVQ_ERRF_CAPACITY).  Shares the handle's workspace like kvq_decode_attention.

@@ -648,10 +648,18 @@ static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
 // Whether one decode launch can also append this call's rows (fused append + decode): a
 // register-decode tensor-core instance serves the pair, and the append needs none of the extras
 // (key mean, int anchors, head groups) that only the standalone append kernels carry.
-bool fused_decode_ok(const LayerDev& L, int n_q) {
+// It is also worth it only when the split-K grid fits in one wave of resident CTAs: there the step
+// is latency-bound and the saved launch shows (64K-token batch-1 step: +19 % steps/s), while on
+// multi-wave grids the fused instances' split pass measured slower than the plain pass plus the
+// one-token append (batch-16 NF4 + int4: 183 against 150 + 10 us per layer).
+bool fused_decode_ok(const LayerDev& L, int n_q, int num_sms) {
   MmaPlan p;
-  return pick_mma(L, &p) && !use_mq(L, n_q) && !L.s[0].mean_sub && !L.s[1].mean_sub && L.anchor_bits == 16 &&
-         L.Hkv == L.Hkv_all;
+  if (!pick_mma(L, &p) || use_mq(L, n_q) || L.s[0].mean_sub || L.s[1].mean_sub || L.anchor_bits != 16 ||
+      L.Hkv != L.Hkv_all)
+    return false;
+  const int slots = mma_slots(p, num_sms);
+  const long long units = (long long)n_q * L.Hkv;
+  return (long long)mma_split_count(units, L.Tcap / p.tile, slots) * units <= slots;
 }
 
 // Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).

@@ -765,7 +765,7 @@ kvq_status kvq_append_decode(kvq_cache* h, int32_t layer, const void* k, const v
   if (!seq_ids && h->len_exact[layer] && (int64_t)h->max_len[layer] + n_new > h->cfg.capacity) return KVQ_ERR_CAPACITY;
   if ((int64_t)n_seqs * h->cfg.n_kv_heads * n_new >= (int64_t)1 << 31) return KVQ_ERR_INVALID_ARG;
   LayerDev L = layer_dev(h, layer, 0);
-  if (h->grp[layer].size() != 1 || !fused_decode_ok(L, n_seqs)) {
+  if (h->grp[layer].size() != 1 || !fused_decode_ok(L, n_seqs, h->num_sms)) {
     kvq_status s = kvq_quantize_append(h, layer, k, v, seq_ids, n_seqs, n_new, stream);
     if (s != KVQ_OK) return s;
     const int na = h->last_launches;

@@ -107,8 +107,8 @@ cudaError_t launch_key_mean(const LayerDev& L, const __half* k, int n_new, cudaS
 
 // Split-K partials per (query, head) one decode call on `L` writes (workspace sizing).
 int decode_partials(const LayerDev& L, int n_q, int num_sms);
-// Fused append + decode is available for this view and query count (see decode.cu).
-bool fused_decode_ok(const LayerDev& L, int n_q);
+// Fused append + decode is available and chosen for this view and query count (see decode.cu).
+bool fused_decode_ok(const LayerDev& L, int n_q, int num_sms);
 
 // Fixed device scratch for the no-allocation decode entry point (decode.cu).
 size_t static_work_floats();

@@ -182,3 +182,25 @@ def test_fused_step_refuses_a_full_sequence():
     _same_cache(A, Bc, lens)
     A.close()
     Bc.close()
+
+
+def test_multi_wave_step_runs_the_two_calls():
+    """A split-K grid of more than one wave (batch 16 x 8 kv-heads, capacity 32768) takes the
+    two calls inside kvq_append_decode, with the same results."""
+    D, G, Bb, Hh, T0 = 128, 4, 16, 8, 1000
+    cfg = Config(n_layers=1, batch=Bb, n_kv_heads=Hh, n_q_heads=Hh * G, head_dim=D, capacity=32768,
+                 k=Side("nf4", group=64), v=Side("int", 4, group=64), max_queries=Bb)
+    A, Bc = KVCache(cfg), KVCache(cfg)
+    rows = lambda side, t0, n: synth.kv_rows(0, side, 0, list(range(Bb)), list(range(Hh)),
+                                             list(range(t0, t0 + n)), D, "cuda")
+    A.append(0, rows("k", 0, T0), rows("v", 0, T0))
+    Bc.append(0, rows("k", 0, T0), rows("v", 0, T0))
+    q = synth.queries(1, 0, Bb, cfg.n_q_heads, D, T0 + 1).cuda()
+    out_a = A.append_decode(0, rows("k", T0, 1), rows("v", T0, 1), q)
+    assert kvq.kvq_last_launch_count(A.h) == 3  # append, split pass, merge
+    Bc.append(0, rows("k", T0, 1), rows("v", T0, 1))
+    out_b = Bc.decode(0, q)
+    torch.testing.assert_close(out_a, out_b, rtol=0, atol=0)
+    assert A.view(0, 0, "seq_len").cpu().tolist() == [T0 + 1] * Bb
+    A.close()
+    Bc.close()
