@@ -182,7 +182,7 @@ class ClockSampler:
                 "samples": len(self.rows), "period_ms": self.period * 1e3, "source": "nvml"}
 
 
-DECODE_SOURCES = ("decode.cu", "decode_tc.cuh", "decode_common.cuh", "kvq_internal.h")
+DECODE_SOURCES = ("decode.cu", "decode_tc.cuh", "decode_mq.cuh", "decode_common.cuh", "quantize_row.cuh", "kvq_internal.h")
 
 
 def decode_sources_sha256():

@@ -423,9 +423,24 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
   __shared__ float po[SP][D];
   __shared__ float ov[D], tmp[D];
   const int warp = tid >> 5, lane = tid & 31;
+  static_assert(NT >= kMaxSplit + 1, "one thread per split's (m, l)");
+  // One round trip: every split's (m, l) (thread s takes split s) and this thread's first R
+  // partial-output values, loaded before the weights they are scaled by are known.
+  constexpr int R = 24;
+  float mv = -INFINITY, lv = 0.0f;
+  if (tid < nsp) {
+    mv = P[tid * (D + kPartStride)];
+    lv = P[tid * (D + kPartStride) + 1];
+  }
+  const float* pj = P + kPartStride + j;
+  float pre[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int s = sg + r * SP;
+    pre[r] = s < n_split ? pj[s * (D + kPartStride)] : 0.0f;
+  }
   // max of the partial maxima
-  float M = -INFINITY;
-  for (int s = tid; s < nsp; s += NT) M = fmaxf(M, P[s * (D + kPartStride)]);
+  float M = mv;
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) rm[warp] = M;
   __syncthreads();
@@ -433,11 +448,10 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
   for (int i = 1; i < NWP; ++i) M = fmaxf(M, rm[i]);
   // weights and the normaliser
   float ls = 0.0f;
-  for (int s = tid; s < nsp; s += NT) {
-    const float m = P[s * (D + kPartStride)];
-    const float ws = (m == -INFINITY) ? 0.0f : exp2f(m - M);
-    w[s] = ws;
-    ls += ws * P[s * (D + kPartStride) + 1];
+  if (tid < nsp) {
+    const float ws = (mv == -INFINITY) ? 0.0f : exp2f(mv - M);
+    w[tid] = ws;
+    ls = ws * lv;
   }
   for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
   if (lane == 0) rl[warp] = ls;
@@ -446,9 +460,13 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
   for (int i = 0; i < NWP; ++i) Ls += rl[i];
   {
     float acc = 0.0f;
-    const float* pj = P + kPartStride + j;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int s = sg + r * SP;
+      if (s < n_split) acc += w[s] * pre[r];
+    }
 #pragma unroll 8
-    for (int s = sg; s < n_split; s += SP) acc += w[s] * pj[s * (D + kPartStride)];
+    for (int s = sg + R * SP; s < n_split; s += SP) acc += w[s] * pj[s * (D + kPartStride)];
     po[sg][j] = acc;
   }
   __syncthreads();
@@ -461,7 +479,16 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
   __syncthreads();
   if (V.rot == 128 || V.rot == 256) {
     const int n = V.rot;
-    for (int h = 1; h < n; h <<= 1) {
+    if (tid < D) {  // stages h < 32 inside each warp (thread t holds channel t): same butterflies
+      float v = ov[tid];
+      for (int h = 1; h < 32; h <<= 1) {
+        const float p = __shfl_xor_sync(0xffffffffu, v, h);
+        v = (tid & h) ? p - v : v + p;
+      }
+      ov[tid] = v;
+    }
+    __syncthreads();
+    for (int h = 32; h < n; h <<= 1) {
       for (int p = tid; p < D / 2; p += NT) {
         const int lo = p & (h - 1), hi = p >> (__ffs(h) - 1);
         const int i = (hi << __ffs(h)) | lo;

@@ -312,8 +312,10 @@ LayerDev layer_dev(const kvq_cache* h, int l, int gi) {
   L.cap = c.capacity;
   L.app_ids = nullptr;
   L.app_n = c.batch;
+  L.div_new = fast_div(1u);
   L.test_stall = h->test_stall;
   L.Hkv = g.nh;
+  L.div_hkv = fast_div((unsigned)L.Hkv);
   L.Hq = g.nh * G;
   L.Hkv_all = c.n_kv_heads;
   L.h0 = g.h0;
@@ -660,6 +662,7 @@ kvq_status kvq_quantize_append(kvq_cache* h, int32_t layer, const void* k, const
     views[gi] = layer_dev(h, layer, gi);
     views[gi].app_ids = seq_ids;
     views[gi].app_n = n_seqs;
+    views[gi].div_new = fast_div((unsigned)n_new);
     total += append_ctas(views[gi], n_new);
   }
   int launches = 0;

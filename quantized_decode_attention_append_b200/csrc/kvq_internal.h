@@ -16,6 +16,25 @@ __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__
 constexpr int kMaxSplit = 256;     // split-K partitions per (query, kv-head)
 constexpr int kPartStride = 4;     // floats of (m, l, pad, pad) before o[D] in a partial
 
+// Division of n < 2^31 by a fixed d >= 1 as a multiply and a shift: m = ceil(2^(31 + l) / d),
+// l = ceil(log2 d), so 2^(31 + l) <= m d < 2^(31 + l) + 2^l, which makes floor(n m / 2^(31 + l))
+// equal floor(n / d) for every n < 2^31 (Granlund and Montgomery, "Division by invariant integers
+// using multiplication", PLDI 1994, Theorem 4.2).
+struct FastDiv {
+  unsigned long long m;
+  int sh;
+};
+inline FastDiv fast_div(unsigned d) {
+  if (d == 0) d = 1;  // callers pass counts >= 1; never divide by zero on the host
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  const int sh = 31 + l;
+  return FastDiv{((1ull << sh) + d - 1) / d, sh};
+}
+__device__ __forceinline__ int div_by(int n, const FastDiv& f) {
+  return (int)(((unsigned long long)(unsigned)n * f.m) >> f.sh);
+}
+
 // Device view of one (layer, side).
 struct SideDev {
   uint8_t* codes;        // [B*Hkv][Tcap][row_bytes]
@@ -48,6 +67,7 @@ struct LayerDev {
   // append call: sequences that receive rows (null: every sequence, in order) and how many
   const int* app_ids;
   int app_n;
+  FastDiv div_new, div_hkv;  // by the call's rows per sequence and by Hkv (row -> destination)
   long long test_stall;  // test hook (0 = off): the decode's first stage wait polls a barrier nothing
                          // arrives on for this many clock cycles, then gives up
   // fused append + decode (fuse_n > 0): query i's sequence also receives fuse_n new rows, input

@@ -53,9 +53,9 @@ struct RowDst {
 // (rows per call < 2^31, checked on the host, so 32-bit index arithmetic suffices)
 __device__ __forceinline__ RowDst row_dst(const LayerDev& L, int row, int n_new) {
   RowDst d{0, 0, 0, 0u, false};
-  const int ul = row / n_new;
+  const int ul = div_by(row, L.div_new);  // row / n_new
   const int i = row - ul * n_new;
-  const int sl = ul / L.Hkv, h = ul - sl * L.Hkv;
+  const int sl = div_by(ul, L.div_hkv), h = ul - sl * L.Hkv;
   const int b = L.app_ids ? L.app_ids[sl] : sl;
   d.first = i == 0 && h == 0;
   if (b < 0 || b >= L.B) {
@@ -609,7 +609,7 @@ cudaError_t launch_key_mean(const LayerDev& L, const __half* k, int n_new, cudaS
 }
 
 // Grid cap of the grid-stride append kernels (148 SMs x 8 CTAs of 8 warps).
-constexpr long long kMaxAppendCtas = 148 * 8;
+constexpr long long kMaxAppendCtas = 148 * 16;
 
 struct SidePlan {
   void (*kern)(LayerDev, int, const __half*, int, unsigned);
