@@ -186,7 +186,8 @@ def test_fused_step_refuses_a_full_sequence():
 
 def test_multi_wave_step_runs_the_two_calls():
     """A split-K grid of more than one wave (batch 16 x 8 kv-heads, capacity 32768) takes the
-    two calls inside kvq_append_decode, with the same results."""
+    two calls inside kvq_append_decode, with the same results, also for a subset of sequences
+    appending two tokens each."""
     D, G, Bb, Hh, T0 = 128, 4, 16, 8, 1000
     cfg = Config(n_layers=1, batch=Bb, n_kv_heads=Hh, n_q_heads=Hh * G, head_dim=D, capacity=32768,
                  k=Side("nf4", group=64), v=Side("int", 4, group=64), max_queries=Bb)
@@ -202,5 +203,24 @@ def test_multi_wave_step_runs_the_two_calls():
     out_b = Bc.decode(0, q)
     torch.testing.assert_close(out_a, out_b, rtol=0, atol=0)
     assert A.view(0, 0, "seq_len").cpu().tolist() == [T0 + 1] * Bb
+    # a second step on half of the sequences, two tokens each
+    ids = list(range(0, Bb, 2))
+    sid = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    k2 = synth.kv_rows(0, "k", 0, ids, list(range(Hh)), [T0 + 1, T0 + 2], D, "cuda")
+    v2 = synth.kv_rows(0, "v", 0, ids, list(range(Hh)), [T0 + 1, T0 + 2], D, "cuda")
+    q2 = synth.queries(1, 1, len(ids), cfg.n_q_heads, D, T0 + 3).cuda()
+    out_a = A.append_decode(0, k2, v2, q2, seq_ids=sid)
+    Bc.append(0, k2, v2, seq_ids=sid)
+    out_b = Bc.decode(0, q2, seq_ids=sid)
+    torch.testing.assert_close(out_a, out_b, rtol=0, atol=0)
+    lens = [T0 + 3 if b % 2 == 0 else T0 + 1 for b in range(Bb)]
+    assert A.view(0, 0, "seq_len").cpu().tolist() == Bc.view(0, 0, "seq_len").cpu().tolist() == lens
+    for side in (0, 1):
+        for what in ("codes", "scales"):
+            va, vb = A.view(0, side, what), Bc.view(0, side, what)
+            for b in range(Bb):
+                u = slice(b * Hh, (b + 1) * Hh)
+                assert torch.equal(va[u, :lens[b]], vb[u, :lens[b]]), (side, what, b)
+    assert kvq.kvq_error_flags(A.h) == 0
     A.close()
     Bc.close()
