@@ -425,12 +425,14 @@ template <> struct TcFam<CF_SIGN> { static constexpr int fam = FAM_SIGN, bits = 
 template <> struct TcFam<CF_TERN> { static constexpr int fam = FAM_TERNARY, bits = 0; };
 
 // Fused append + decode: the new rows of (query qi's sequence, kv-head kvh) that this CTA owns
-// are written by warp 0 before any tile is copied.  A new row inside the quantized range belongs
-// to the CTA whose tiles cover it (the only reader of its codes in this launch); the others
-// (anchored rows, read later from their anchor copies) to split 0.  One row per lane group of
-// head_dim / 32 lanes, as in the append kernels, with the same arithmetic (quantize_slice).
-// Not inlined: its registers then stay out of the decode loop's allocation (called once per CTA);
-// the fused kernel's LayerDev is a __grid_constant__ parameter, so the reference reads it in place.
+// are written by warp 0 before a tile copy reads them.  A new row inside the quantized range
+// belongs to the CTA whose tiles cover it (the only reader of its codes in this launch); the
+// others (anchored rows, read later from their anchor copies) to split 0.  One row per lane group
+// of head_dim / 32 lanes, as in the append kernels, with the same arithmetic (quantize_slice).
+// Not inlined (called once per CTA), so its working registers are not live in the decode loop;
+// the fused kernel's LayerDev is a __grid_constant__ parameter, so the reference reads it in
+// place.  Under the fused instances' register cap the call still makes the 8-warp loops spill,
+// which is why multi-wave grids take the separate append and decode calls (kvq_append_decode).
 template <int D, int KF, int GK, int VF, int GV>
 __device__ __noinline__ void fused_append_rows(const LayerDev& L, const QueryRange& R, int qi, int kvh, int split,
                                                int t_lo, int t_hi) {
