@@ -708,18 +708,30 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   if (use_mq(L, n_q)) {
     if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
     using MC = MqCfg<D>;
-    static int dyn_max = -1;  // one per instantiation (the attribute is per kernel)
-    if (dyn_max < 0) {  // the opt-in limit covers static + dynamic shared memory
+    // min-max int codes of 3 or 4 bits in groups of >= 8 on both sides (config 2): the specialised
+    // tile decode (head_dim 256 only)
+    auto mm_side = [](const SideDev& S) {
+      return S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_MINMAX && (S.bits == 3 || S.bits == 4) &&
+             S.group >= 8 && S.zeros;
+    };
+    const bool mm = D == 256 && mm_side(L.s[0]) && mm_side(L.s[1]);
+    auto kern = decode_mq_kernel<D, false>;
+    if constexpr (D == 256) {
+      if (mm) kern = decode_mq_kernel<D, true>;
+    }
+    static int dyn_max[2] = {-1, -1};  // per instantiation (the attribute is per kernel)
+    if (dyn_max[mm] < 0) {  // the opt-in limit covers static + dynamic shared memory
       cudaFuncAttributes fa;
-      cudaError_t e = cudaFuncGetAttributes(&fa, decode_mq_kernel<D>);
+      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return e;
       const int lim = MC::SMEM_MAX - (int)fa.sharedSizeBytes;
-      e = cudaFuncSetAttribute(decode_mq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
       if (e != cudaSuccess) return e;
-      dyn_max = lim;
+      dyn_max[mm] = lim;
     }
+    const int* dmax = dyn_max + mm;
     const int smem = mq_smem_bytes<D>(L);
-    if (smem > dyn_max) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
+    if (smem > *dmax) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
     const int n_split = mq_split_count<D>(L, n_q, num_sms);
     n_quant = n_split;
     const int nsp = n_quant + (L.anchored ? 1 : 0);
@@ -730,8 +742,8 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int qpb = MC::QM / (L.Hq / L.Hkv);
-    decode_mq_kernel<D><<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, smem, st>>>(L, prep, seq_ids, kv_len,
-                                                                                        work, n_split, nsp, n_q);
+    kern<<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, smem, st>>>(L, prep, seq_ids, kv_len, work, n_split,
+                                                                          nsp, n_q);
     ++nl;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone

@@ -219,6 +219,19 @@ __device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, c
   }
 }
 
+// mq_chunk for a side known to hold min-max int codes of 3 or 4 bits in groups of at least 8
+// (the config-2 formats): the same arithmetic without the format dispatch.
+__device__ __forceinline__ void mq_chunk_minmax(const SideDev& S, const uint8_t* row, const __half* sc,
+                                                const __half* zr, int j0, float* v) {
+  const int b = S.bits;
+  const uint64_t w = mq_bytes(row + b * (j0 >> 3), b);
+  const uint32_t M = (1u << b) - 1u;
+  const int g = j0 / S.group;
+  const float d = __half2float(sc[g]), z = __half2float(zr[g]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fadd_rn(z, (float)(int)((w >> (b * i)) & M) * d);
+}
+
 // 8 values as fp16 hi halves and the fp16 roundings of their remainders, 16 bytes each.
 __device__ __forceinline__ void mq_store8(__half* hi, __half* lo, int idx, const float* v) {
   uint32_t h[4], l[4];
@@ -261,7 +274,9 @@ __global__ void __launch_bounds__(256) mq_prep_kernel(LayerDev L, const __half* 
   }
 }
 
-template <int D>
+// MM: both sides hold min-max int codes of 3 or 4 bits in groups of at least 8 (decoded without
+// the format dispatch).
+template <int D, bool MM = false>
 __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, const float* __restrict__ prep,
                                                                  const int* __restrict__ seq_ids,
                                                                  const int* __restrict__ kv_len, float* __restrict__ work,
@@ -422,10 +437,15 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
           const int t = e / (D / 8), j0 = (e % (D / 8)) * 8;
           float kv[8], vv[8];
           if (t0 + t < len) {
-            mq_chunk(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk ? zk + t * K.n_groups : nullptr, j0, kv, t_nf4,
-                     t_lk, t_kc, t_ks);
-            mq_chunk(V, bv + t * V.row_bytes, sv + t * V.n_groups, zv ? zv + t * V.n_groups : nullptr, j0, vv, t_nf4,
-                     t_lv, t_vc, t_vs);
+            if constexpr (MM) {
+              mq_chunk_minmax(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk + t * K.n_groups, j0, kv);
+              mq_chunk_minmax(V, bv + t * V.row_bytes, sv + t * V.n_groups, zv + t * V.n_groups, j0, vv);
+            } else {
+              mq_chunk(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk ? zk + t * K.n_groups : nullptr, j0, kv,
+                       t_nf4, t_lk, t_kc, t_ks);
+              mq_chunk(V, bv + t * V.row_bytes, sv + t * V.n_groups, zv ? zv + t * V.n_groups : nullptr, j0, vv,
+                       t_nf4, t_lv, t_vc, t_vs);
+            }
           } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) kv[i] = vv[i] = 0.0f;

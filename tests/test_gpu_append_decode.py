@@ -224,3 +224,53 @@ def test_multi_wave_step_runs_the_two_calls():
     assert kvq.kvq_error_flags(A.h) == 0
     A.close()
     Bc.close()
+
+
+def test_per_head_formats_step_runs_the_two_calls():
+    """A layer with per-head formats (two head groups) takes the two calls inside
+    kvq_append_decode, with the results of kvq_quantize_append then kvq_decode_attention."""
+    a, s = Side("int", 4, group=32), Side("sign", group=4)
+    cfg = Config(n_layers=1, batch=3, n_kv_heads=2, n_q_heads=8, head_dim=128, capacity=256, k=a, v=a,
+                 max_queries=4, head_k=((a, s),), head_v=((a, s),))
+    A, Bc = KVCache(cfg), KVCache(cfg)
+    lens = [0] * 3
+    K, V = _step_rows(range(3), lens, 90, 128)
+    A.append(0, K, V)
+    Bc.append(0, K, V)
+    lens = [90] * 3
+    K, V = _step_rows(range(3), lens, 1, 128)
+    q = synth.queries(1, 0, 3, cfg.n_q_heads, 128, 91).cuda()
+    out_a = A.append_decode(0, K, V, q)
+    assert kvq.kvq_last_launch_count(A.h) > 3  # one append and one decode per head group
+    Bc.append(0, K, V)
+    out_b = Bc.decode(0, q)
+    torch.testing.assert_close(out_a, out_b, rtol=0, atol=0)
+    assert A.view(0, 0, "seq_len").cpu().tolist() == [91] * 3
+    A.close()
+    Bc.close()
+
+
+def test_append_decode_argument_errors():
+    """Host-side refusals of kvq_append_decode, before any launch."""
+    cfg = Config(n_layers=1, batch=2, n_kv_heads=2, n_q_heads=8, head_dim=128, capacity=64,
+                 k=Side("nf4", group=64), v=Side("int", 4, group=64), max_queries=2)
+    c = KVCache(cfg)
+    L = kvq.lib()
+    p = kvq._ptr
+    k = torch.zeros(2, 2, 1, 128, dtype=torch.float16, device="cuda")
+    q = torch.zeros(2, 8, 128, dtype=torch.float16, device="cuda")
+    out = torch.empty(2, 8, 128, dtype=torch.float32, device="cuda")
+    st = kvq._stream(None)
+    ids3 = torch.tensor([0, 1, 1], dtype=torch.int32, device="cuda")
+    assert L.kvq_append_decode(c.h, 0, p(k), p(k), None, 1, 1, p(q), p(out), 1, None, st) == -1      # NULL list: n_seqs = batch
+    assert L.kvq_append_decode(c.h, 1, p(k), p(k), None, 2, 1, p(q), p(out), 1, None, st) == -1      # no such layer
+    assert L.kvq_append_decode(c.h, 0, p(k), p(k), None, 2, 0, p(q), p(out), 1, None, st) == -1      # no rows
+    assert L.kvq_append_decode(c.h, 0, p(k), p(k), None, 2, 1, None, p(out), 1, None, st) == -1      # no queries
+    assert L.kvq_append_decode(c.h, 0, p(k), p(k), p(ids3), 3, 1, p(q), p(out), 1, None, st) == -1   # more ids than batch
+    assert L.kvq_append_decode(c.h, 0, p(k), p(k), None, 2, 65, p(q), p(out), 1, None, st) == -3     # more rows than capacity
+    with pytest.raises(ValueError):
+        c.append_decode(0, k, k, q[:1])  # one query for two sequences
+    assert kvq.kvq_last_launch_count(c.h) >= 0
+    torch.cuda.synchronize()
+    assert c.view(0, 0, "seq_len").cpu().tolist() == [0, 0]
+    c.close()
