@@ -708,28 +708,36 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   if (use_mq(L, n_q)) {
     if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
     using MC = MqCfg<D>;
-    // min-max int codes of 3 or 4 bits in groups of >= 8 on both sides (config 2): the specialised
-    // tile decode (head_dim 256 only)
+    // Tile decode without the format dispatch where both sides' class is known: min-max int codes
+    // of 3 or 4 bits in groups of >= 8 (config 2, head_dim 256), rFFT polar (config 4, head_dim 128).
     auto mm_side = [](const SideDev& S) {
       return S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_MINMAX && (S.bits == 3 || S.bits == 4) &&
              S.group >= 8 && S.zeros;
     };
-    const bool mm = D == 256 && mm_side(L.s[0]) && mm_side(L.s[1]);
-    auto kern = decode_mq_kernel<D, false>;
+    int fc = FC_ANY;
+    if (mm_side(L.s[0]) && mm_side(L.s[1])) fc = FC_MINMAX;
+    if (L.s[0].fmt == KVQ_FMT_POLAR && L.s[1].fmt == KVQ_FMT_POLAR) fc = FC_POLAR;
+    auto kern = decode_mq_kernel<D, FC_ANY>;
     if constexpr (D == 256) {
-      if (mm) kern = decode_mq_kernel<D, true>;
+      if (fc == FC_MINMAX) kern = decode_mq_kernel<D, FC_MINMAX>;
+      else fc = FC_ANY;
+    } else if constexpr (D == 128) {
+      if (fc == FC_POLAR) kern = decode_mq_kernel<D, FC_POLAR>;
+      else fc = FC_ANY;
+    } else {
+      fc = FC_ANY;
     }
-    static int dyn_max[2] = {-1, -1};  // per instantiation (the attribute is per kernel)
-    if (dyn_max[mm] < 0) {  // the opt-in limit covers static + dynamic shared memory
+    static int dyn_max[3] = {-1, -1, -1};  // per instantiation (the attribute is per kernel)
+    if (dyn_max[fc] < 0) {  // the opt-in limit covers static + dynamic shared memory
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return e;
       const int lim = MC::SMEM_MAX - (int)fa.sharedSizeBytes;
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
       if (e != cudaSuccess) return e;
-      dyn_max[mm] = lim;
+      dyn_max[fc] = lim;
     }
-    const int* dmax = dyn_max + mm;
+    const int* dmax = dyn_max + fc;
     const int smem = mq_smem_bytes<D>(L);
     if (smem > *dmax) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
     const int n_split = mq_split_count<D>(L, n_q, num_sms);

@@ -150,6 +150,23 @@ __device__ __forceinline__ uint64_t mq_bits64(const uint8_t* p, int bit) {
   return ((uint64_t)hi << 32) | lo;
 }
 
+// Polar slots j0 / 2 .. j0 / 2 + 3 of a staged row as (m cos phi, m sin phi) pairs, as polar_slot
+// computes them: the magnitude fields, then the phase fields, read at once.
+__device__ __forceinline__ void mq_chunk_polar(const SideDev& S, const uint8_t* row, const __half* sc, int j0,
+                                               float* v, const float* cs, const float* sn) {
+  const int bm = S.bits, bp = S.bits2, f0 = j0 >> 1;
+  const uint64_t mw = mq_bits64(row, f0 * bm), pw = mq_bits64(row, 64 * bm + f0 * bp);
+  const uint32_t mm = (1u << bm) - 1u, pm = (1u << bp) - 1u;
+  const float s = __half2float(sc[0]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float m = (float)(uint32_t)((mw >> (i * bm)) & mm) * s;
+    const int k = (int)((pw >> (i * bp)) & pm);
+    v[2 * i] = __fmul_rn(m, cs[k]);
+    v[2 * i + 1] = __fmul_rn(m, sn[k]);
+  }
+}
+
 // Stored-domain values of elements j0 .. j0 + 7 (j0 % 8 == 0) of one staged row, with the same
 // arithmetic as stored_value / polar_slot (polar: slots j0 / 2 .. j0 / 2 + 3, (cos, sin) parts).
 __device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, const __half* sc, const __half* zr,
@@ -167,18 +184,8 @@ __device__ __forceinline__ void mq_chunk(const SideDev& S, const uint8_t* row, c
     }
     return;
   }
-  if (f == KVQ_FMT_POLAR) {  // slots f0 .. f0 + 3: magnitude fields, then phase fields, read at once
-    const int bm = S.bits, bp = S.bits2, f0 = j0 >> 1;
-    const uint64_t mw = mq_bits64(row, f0 * bm), pw = mq_bits64(row, 64 * bm + f0 * bp);
-    const uint32_t mm = (1u << bm) - 1u, pm = (1u << bp) - 1u;
-    const float s = __half2float(sc[0]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float m = (float)(uint32_t)((mw >> (i * bm)) & mm) * s;
-      const int k = (int)((pw >> (i * bp)) & pm);
-      v[2 * i] = __fmul_rn(m, cs[k]);
-      v[2 * i + 1] = __fmul_rn(m, sn[k]);
-    }
+  if (f == KVQ_FMT_POLAR) {
+    mq_chunk_polar(S, row, sc, j0, v, cs, sn);
     return;
   }
   if (f == KVQ_FMT_TERNARY || f == KVQ_FMT_SORTED) {
@@ -274,9 +281,11 @@ __global__ void __launch_bounds__(256) mq_prep_kernel(LayerDev L, const __half* 
   }
 }
 
-// MM: both sides hold min-max int codes of 3 or 4 bits in groups of at least 8 (decoded without
-// the format dispatch).
-template <int D, bool MM = false>
+// Format class of both sides, decoded without the format dispatch when known: FC_ANY (any
+// format), FC_MINMAX (min-max int codes of 3 or 4 bits in groups of at least 8), FC_POLAR (rFFT
+// polar).
+enum MqFmtClass { FC_ANY = 0, FC_MINMAX = 1, FC_POLAR = 2 };
+template <int D, int FC = FC_ANY>
 __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, const float* __restrict__ prep,
                                                                  const int* __restrict__ seq_ids,
                                                                  const int* __restrict__ kv_len, float* __restrict__ work,
@@ -437,9 +446,12 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
           const int t = e / (D / 8), j0 = (e % (D / 8)) * 8;
           float kv[8], vv[8];
           if (t0 + t < len) {
-            if constexpr (MM) {
+            if constexpr (FC == FC_MINMAX) {
               mq_chunk_minmax(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk + t * K.n_groups, j0, kv);
               mq_chunk_minmax(V, bv + t * V.row_bytes, sv + t * V.n_groups, zv + t * V.n_groups, j0, vv);
+            } else if constexpr (FC == FC_POLAR) {
+              mq_chunk_polar(K, bk + t * K.row_bytes, sk + t * K.n_groups, j0, kv, t_kc, t_ks);
+              mq_chunk_polar(V, bv + t * V.row_bytes, sv + t * V.n_groups, j0, vv, t_vc, t_vs);
             } else {
               mq_chunk(K, bk + t * K.row_bytes, sk + t * K.n_groups, zk ? zk + t * K.n_groups : nullptr, j0, kv,
                        t_nf4, t_lk, t_kc, t_ks);
