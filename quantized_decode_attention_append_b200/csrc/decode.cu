@@ -651,17 +651,39 @@ static bool use_mq(const LayerDev& L, int n_q) {
   return !pick_mma(L, &p) || (L.Hq / L.Hkv <= 2 && n_q > L.B);
 }
 
-// Splits of the multi-query kernel: about two waves of its CTAs, at least one 32-token tile each.
+// Format class of a layer's (K, V) pair on the multi-query kernel (see MqFmtClass).
 template <int D>
-static int mq_split_count(const LayerDev& L, int n_q, int num_sms) {
-  const int G = L.Hq / L.Hkv, qpb = MqCfg<D>::QM / G;
+static int mq_class(const LayerDev& L) {
+  auto mm_side = [](const SideDev& S) {
+    return S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_MINMAX && (S.bits == 3 || S.bits == 4) && S.group >= 8 &&
+           S.zeros;
+  };
+  if (D == 256 && mm_side(L.s[0]) && mm_side(L.s[1])) return FC_MINMAX;
+  if (D == 128 && L.s[0].fmt == KVQ_FMT_POLAR && L.s[1].fmt == KVQ_FMT_POLAR) return FC_POLAR;
+  return FC_ANY;
+}
+
+// Splits of the multi-query kernel: about two waves of its CTAs, at least one tile each.
+template <int D, int FC>
+static int mq_split_count_fc(const LayerDev& L, int n_q, int num_sms) {
+  using C = MqCfg<D, FC>;
+  const int G = L.Hq / L.Hkv, qpb = C::QM / G;
   const long long units = (long long)L.Hkv * ((n_q + qpb - 1) / qpb);
-  const int per_sm = D >= 256 ? 1 : 2;
+  const int per_sm = (D >= 256 && FC != FC_MINMAX) ? 1 : 2;  // resident CTAs (shared memory)
   long long s = (2LL * per_sm * num_sms + units - 1) / units;
-  const long long tiles = L.Tcap / MqCfg<D>::TK;
+  const long long tiles = L.Tcap / C::TK;
   if (s > tiles) s = tiles;
   if (s > kMaxSplit) s = kMaxSplit;
   return s < 1 ? 1 : (int)s;
+}
+
+template <int D>
+static int mq_split_count(const LayerDev& L, int n_q, int num_sms) {
+  switch (mq_class<D>(L)) {
+    case FC_MINMAX: return mq_split_count_fc<D, FC_MINMAX>(L, n_q, num_sms);
+    case FC_POLAR: return mq_split_count_fc<D, FC_POLAR>(L, n_q, num_sms);
+    default: return mq_split_count_fc<D, FC_ANY>(L, n_q, num_sms);
+  }
 }
 
 static int mq_splits(const LayerDev& L, int n_q, int num_sms) {
@@ -707,39 +729,35 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   int n_quant;  // quantized partials per (query, head)
   if (use_mq(L, n_q)) {
     if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
-    using MC = MqCfg<D>;
     // Tile decode without the format dispatch where both sides' class is known: min-max int codes
     // of 3 or 4 bits in groups of >= 8 (config 2, head_dim 256), rFFT polar (config 4, head_dim 128).
-    auto mm_side = [](const SideDev& S) {
-      return S.fmt == KVQ_FMT_INT && S.scale_mode == KVQ_SCALE_MINMAX && (S.bits == 3 || S.bits == 4) &&
-             S.group >= 8 && S.zeros;
-    };
-    int fc = FC_ANY;
-    if (mm_side(L.s[0]) && mm_side(L.s[1])) fc = FC_MINMAX;
-    if (L.s[0].fmt == KVQ_FMT_POLAR && L.s[1].fmt == KVQ_FMT_POLAR) fc = FC_POLAR;
+    const int fc = mq_class<D>(L);
     auto kern = decode_mq_kernel<D, FC_ANY>;
+    int smem = mq_smem_bytes<D, FC_ANY>(L), nt = MqCfg<D, FC_ANY>::NT, qm = MqCfg<D, FC_ANY>::QM;
     if constexpr (D == 256) {
-      if (fc == FC_MINMAX) kern = decode_mq_kernel<D, FC_MINMAX>;
-      else fc = FC_ANY;
+      if (fc == FC_MINMAX) {
+        kern = decode_mq_kernel<D, FC_MINMAX>;
+        smem = mq_smem_bytes<D, FC_MINMAX>(L);
+        nt = MqCfg<D, FC_MINMAX>::NT;
+        qm = MqCfg<D, FC_MINMAX>::QM;
+      }
     } else if constexpr (D == 128) {
-      if (fc == FC_POLAR) kern = decode_mq_kernel<D, FC_POLAR>;
-      else fc = FC_ANY;
-    } else {
-      fc = FC_ANY;
+      if (fc == FC_POLAR) {
+        kern = decode_mq_kernel<D, FC_POLAR>;
+        smem = mq_smem_bytes<D, FC_POLAR>(L);
+      }
     }
     static int dyn_max[3] = {-1, -1, -1};  // per instantiation (the attribute is per kernel)
     if (dyn_max[fc] < 0) {  // the opt-in limit covers static + dynamic shared memory
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return e;
-      const int lim = MC::SMEM_MAX - (int)fa.sharedSizeBytes;
+      const int lim = MqCfg<D>::SMEM_MAX - (int)fa.sharedSizeBytes;
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
       if (e != cudaSuccess) return e;
       dyn_max[fc] = lim;
     }
-    const int* dmax = dyn_max + fc;
-    const int smem = mq_smem_bytes<D>(L);
-    if (smem > *dmax) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
+    if (smem > dyn_max[fc]) return cudaErrorInvalidValue;  // staged rows of this format pair do not fit
     const int n_split = mq_split_count<D>(L, n_q, num_sms);
     n_quant = n_split;
     const int nsp = n_quant + (L.anchored ? 1 : 0);
@@ -749,9 +767,9 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
     ++nl;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int qpb = MC::QM / (L.Hq / L.Hkv);
-    kern<<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), MC::NT, smem, st>>>(L, prep, seq_ids, kv_len, work, n_split,
-                                                                          nsp, n_q);
+    const int qpb = qm / (L.Hq / L.Hkv);
+    kern<<<dim3(n_split, L.Hkv, (n_q + qpb - 1) / qpb), nt, smem, st>>>(L, prep, seq_ids, kv_len, work, n_split, nsp,
+                                                                       n_q);
     ++nl;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone

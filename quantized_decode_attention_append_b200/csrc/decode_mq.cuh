@@ -30,14 +30,21 @@
 // .trans).  Queries of different sequences in one CTA are served by one pass per sequence over
 // that sequence's tiles, other rows masked.
 
-template <int D>
+// Format class of both sides, decoded without the format dispatch when known: FC_ANY (any
+// format), FC_MINMAX (min-max int codes of 3 or 4 bits in groups of at least 8), FC_POLAR (rFFT
+// polar).
+enum MqFmtClass { FC_ANY = 0, FC_MINMAX = 1, FC_POLAR = 2 };
+
+// Tile shapes per head_dim and format class.  The min-max class needs no level or phase tables and
+// takes 16-token tiles, which fits two CTAs per SM at head_dim 256.
+template <int D, int FC = FC_ANY>
 struct MqCfg {
   static constexpr int CS = D >= 256 ? 2 : 1;      // warps sharing a 16-row block (channel split)
   static constexpr int RB = 4;                     // 16-row blocks per CTA
   static constexpr int NW = RB * CS;
   static constexpr int NT = NW * 32;
   static constexpr int QM = 16 * RB;               // rows per CTA
-  static constexpr int TK = 32;                    // tokens per tile
+  static constexpr int TK = FC == FC_MINMAX ? 16 : 32;  // tokens per tile
   static constexpr int LD = D + 8;                 // halves per shared row: ldmatrix rows on distinct banks
   static constexpr int DC = D / CS;                // O channels per warp
   static constexpr int NB = DC / 8;                // O n-blocks per warp
@@ -49,7 +56,8 @@ struct MqCfg {
   static constexpr int OFF_VL = OFF_VH + TK * LD * 2;
   static constexpr int OFF_META = OFF_VL + TK * LD * 2;          // per row: seq, qa, qb, q.mu
   static constexpr int OFF_TAB = OFF_META + QM * 4 * 4;          // NF4 16, Lloyd-Max 2 x 16, phase cos/sin 2 x 2 x 256
-  static constexpr int OFF_RAW = OFF_TAB + (16 + 32 + 1024) * 4;  // two staging buffers of packed tile bytes
+  static constexpr int TAB_BYTES = FC == FC_MINMAX ? 0 : (16 + 32 + 1024) * 4;
+  static constexpr int OFF_RAW = OFF_TAB + TAB_BYTES;  // two staging buffers of packed tile bytes
   static constexpr int SMEM_MAX = 227 * 1024;
   static_assert(OFF_RAW % 16 == 0, "staging buffers must start 16-byte aligned");
   static_assert((LD * 2) % 16 == 0, "ldmatrix rows must stay 16-byte aligned");
@@ -65,10 +73,10 @@ __host__ __device__ __forceinline__ int mq_stage_bytes(const SideDev& S) {
   return mq_up16(TK * S.row_bytes) + sc + (S.zeros ? sc : 0);
 }
 
-// Dynamic shared memory of one decode_mq_kernel<D> launch on `L`.
-template <int D>
+// Dynamic shared memory of one decode_mq_kernel<D, FC> launch on `L`.
+template <int D, int FC>
 inline int mq_smem_bytes(const LayerDev& L) {
-  using C = MqCfg<D>;
+  using C = MqCfg<D, FC>;
   return C::OFF_RAW + 2 * (mq_stage_bytes<C::TK>(L.s[0]) + mq_stage_bytes<C::TK>(L.s[1]));
 }
 
@@ -281,16 +289,12 @@ __global__ void __launch_bounds__(256) mq_prep_kernel(LayerDev L, const __half* 
   }
 }
 
-// Format class of both sides, decoded without the format dispatch when known: FC_ANY (any
-// format), FC_MINMAX (min-max int codes of 3 or 4 bits in groups of at least 8), FC_POLAR (rFFT
-// polar).
-enum MqFmtClass { FC_ANY = 0, FC_MINMAX = 1, FC_POLAR = 2 };
 template <int D, int FC = FC_ANY>
-__global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, const float* __restrict__ prep,
+__global__ void __launch_bounds__(MqCfg<D, FC>::NT) decode_mq_kernel(LayerDev L, const float* __restrict__ prep,
                                                                  const int* __restrict__ seq_ids,
                                                                  const int* __restrict__ kv_len, float* __restrict__ work,
                                                                  int n_split, int nsp_total, int n_q) {
-  using C = MqCfg<D>;
+  using C = MqCfg<D, FC>;
   extern __shared__ __align__(128) unsigned char smem[];
   __half* Qh = reinterpret_cast<__half*>(smem + C::OFF_QH);
   __half* Ql = reinterpret_cast<__half*>(smem + C::OFF_QL);
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   float* t_vc = t_ks + 256;
   float* t_vs = t_vc + 256;
   uint8_t* raw = smem + C::OFF_RAW;
-  __shared__ int pass_seq[MqCfg<D>::QM];
+  __shared__ int pass_seq[MqCfg<D, FC>::QM];
   __shared__ int n_pass;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
@@ -323,7 +327,8 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
   const int cbK = mq_up16(C::TK * K.row_bytes), sbK = K.scales ? mq_up16(C::TK * K.n_groups * 2) : 0;
   const int cbV = mq_up16(C::TK * V.row_bytes), sbV = V.scales ? mq_up16(C::TK * V.n_groups * 2) : 0;
 
-  // ---- tables
+  // ---- tables (none for the min-max class)
+  if constexpr (FC != FC_MINMAX) {
   if (tid < 16) t_nf4[tid] = d_nf4[tid];
   if (K.fmt == KVQ_FMT_LLOYD && tid < 16) t_lk[tid] = d_lloyd[K.bits - 2][tid];
   if (V.fmt == KVQ_FMT_LLOYD && tid < 16) t_lv[tid] = d_lloyd[V.bits - 2][tid];
@@ -337,6 +342,7 @@ __global__ void __launch_bounds__(MqCfg<D>::NT) decode_mq_kernel(LayerDev L, con
       t_vc[k] = d_ph_cos[(1 << V.bits2) - 2 + k];
       t_vs[k] = d_ph_sin[(1 << V.bits2) - 2 + k];
     }
+  }
 
   // ---- rows: the prepared queries as fp16 hi + lo; per-row sequence, causal range, key-mean term
   for (int e = tid; e < C::QM * (D / 4); e += C::NT) {
