@@ -182,7 +182,8 @@ class ClockSampler:
                 "samples": len(self.rows), "period_ms": self.period * 1e3, "source": "nvml"}
 
 
-DECODE_SOURCES = ("decode.cu", "decode_tc.cuh", "decode_mq.cuh", "decode_common.cuh", "quantize_row.cuh", "kvq_internal.h")
+DECODE_SOURCES = ("decode.cu", "decode_tc.cuh", "decode_mq.cuh", "decode_polar.cuh", "decode_common.cuh", "fft128.cuh",
+                  "quantize_row.cuh", "kvq_internal.h")
 
 
 def decode_sources_sha256():

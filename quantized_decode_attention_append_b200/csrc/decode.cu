@@ -17,7 +17,10 @@
 
 #include <mutex>
 
+#include <vector>
+
 #include "decode_common.cuh"
+#include "fft128.cuh"
 #include "kvq_internal.h"
 #include "quantize_row.cuh"
 
@@ -30,8 +33,27 @@ __constant__ float d_ph_cos[512];
 __constant__ float d_ph_sin[512];
 __constant__ float d_lloyd[3][16];
 
+// The phase levels' (cos, sin) in the polar decode's layout: for phase width bp, level k, copy r
+// at entry ((2^bp - 2) + k) x 16 + r (16 copies, one per shared-memory bank pair once staged).
+__device__ __align__(16) float2 g_ph_rep[510 * 16];
+// W_128^k = exp(-2 pi i k / 128), k < 64, as (re[k], im[k]) in global memory: the register FFT's
+// lanes read divergent indices, which constant memory would serialise.
+__device__ float g_tw[2][64];
+
 cudaError_t upload_tables_decode(const HostTables& t) {
   cudaError_t e;
+  {
+    std::vector<float2> rep(510 * 16);
+    for (int k = 0; k < 510; ++k)
+      for (int r = 0; r < 16; ++r) rep[k * 16 + r] = make_float2(t.ph_cos[k], t.ph_sin[k]);
+    if ((e = cudaMemcpyToSymbol(g_ph_rep, rep.data(), rep.size() * sizeof(float2))) != cudaSuccess) return e;
+    float tw[2][64];
+    for (int k = 0; k < 64; ++k) {
+      tw[0][k] = t.tw_re[k];
+      tw[1][k] = t.tw_im[k];
+    }
+    if ((e = cudaMemcpyToSymbol(g_tw, tw, sizeof(tw))) != cudaSuccess) return e;
+  }
   if ((e = upload_row_tables(t)) != cudaSuccess) return e;  // thresholds of the fused append
   if ((e = cudaMemcpyToSymbol(d_nf4, t.nf4, sizeof(t.nf4))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_tw_re, t.tw_re, sizeof(t.tw_re))) != cudaSuccess) return e;
@@ -195,6 +217,7 @@ __device__ void prepare_query(const LayerDev& L, const __half* __restrict__ q, i
 
 #include "decode_tc.cuh"
 #include "decode_mq.cuh"
+#include "decode_polar.cuh"
 
 // Generic pass 1: any format, any GQA group (<= 8), CUDA cores.  Thread-per-token scoring,
 // thread-per-channel value accumulation.
@@ -651,6 +674,85 @@ static bool use_mq(const LayerDev& L, int n_q) {
   return !pick_mma(L, &p) || (L.Hq / L.Hkv <= 2 && n_q > L.B);
 }
 
+// rFFT polar K and V with one query per sequence (GQA 1, 2 or 4): the CUDA-core polar kernel,
+// whose lanes all work on the one live query row (the multi-query kernel's tiles would carry one
+// row in 64).  Queries sharing a sequence (proxy queries) stay on the multi-query kernel.
+static bool use_polar(const LayerDev& L, int n_q) {
+  const int G = L.Hq / L.Hkv;
+  return L.D == 128 && L.s[0].fmt == KVQ_FMT_POLAR && L.s[1].fmt == KVQ_FMT_POLAR && n_q <= L.B &&
+         (G == 1 || G == 2 || G == 4);
+}
+
+typedef void (*PolarKernel)(const LayerDev, const __half*, const int*, const int*, float*, int, int);
+
+template <int G>
+static PolarKernel polar_kernel_g(const LayerDev& L) {
+  const bool f48 = L.s[0].bits == 4 && L.s[0].bits2 == 8 && L.s[1].bits == 4 && L.s[1].bits2 == 8;
+  return f48 ? decode_polar_kernel<G, 4, 8> : decode_polar_kernel<G, 0, 0>;
+}
+static PolarKernel polar_kernel(const LayerDev& L) {
+  switch (L.Hq / L.Hkv) {
+    case 1: return polar_kernel_g<1>(L);
+    case 2: return polar_kernel_g<2>(L);
+    default: return polar_kernel_g<4>(L);
+  }
+}
+static int polar_smem(const LayerDev& L) {
+  switch (L.Hq / L.Hkv) {
+    case 1: return polar_smem_bytes<1>(L);
+    case 2: return polar_smem_bytes<2>(L);
+    default: return polar_smem_bytes<4>(L);
+  }
+}
+
+// Resident CTAs of the polar kernel on L's formats x SMs.  Each instance's opt-in shared-memory
+// limit is raised to the maximum once; occupancy is cached per (instance, bytes).
+static int polar_slots(const LayerDev& L, int num_sms) {
+  struct Occ {
+    PolarKernel k;
+    int smem, occ;
+  };
+  static PolarKernel raised[6] = {};
+  static Occ occs[32] = {};
+  static int n_occ = 0;
+  const PolarKernel k = polar_kernel(L);
+  const int smem = polar_smem(L);
+  for (int i = 0; i < n_occ; ++i)
+    if (occs[i].k == k && occs[i].smem == smem) return occs[i].occ * num_sms;
+  bool seen = false;
+  for (int i = 0; i < 6 && raised[i]; ++i) seen |= raised[i] == k;
+  if (!seen) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k) == cudaSuccess &&
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024 - (int)fa.sharedSizeBytes) == cudaSuccess)
+      for (int i = 0; i < 6; ++i)
+        if (!raised[i]) {
+          raised[i] = k;
+          break;
+        }
+    cudaGetLastError();
+  }
+  int occ = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, PolarCfg::NT, smem) != cudaSuccess || occ < 1) occ = 1;
+  cudaGetLastError();
+  if (n_occ < 32) occs[n_occ++] = Occ{k, smem, occ};
+  return occ * num_sms;
+}
+
+// Splits of the polar kernel: one wave of resident CTAs (every CTA has the same work), at least
+// one tile each.
+static int polar_splits(const LayerDev& L, int n_q, int num_sms) {
+  const long long units = (long long)L.Hkv * n_q;
+  const long long tiles = L.Tcap / PolarCfg::TT;  // capacities are whole multiples of 256 tokens
+  long long s = polar_slots(L, num_sms) / units;
+  if (s > kMaxSplit) s = kMaxSplit;
+  if (s > tiles) s = tiles;
+  if (s < 1) s = 1;
+  const long long per = (tiles + s - 1) / s;  // the same tiles over fewer splits: none left idle
+  return (int)((tiles + per - 1) / per);
+}
+
 // Format class of a layer's (K, V) pair on the multi-query kernel (see MqFmtClass).
 template <int D>
 static int mq_class(const LayerDev& L) {
@@ -713,7 +815,8 @@ bool fused_decode_ok(const LayerDev& L, int n_q, int num_sms) {
 
 // Partials per (query, head) the decode of `L` writes for n_q queries (the workspace bound).
 int decode_partials(const LayerDev& L, int n_q, int num_sms) {
-  if (use_mq(L, n_q)) return mq_splits(L, n_q, num_sms) + 2;  // + anchor split, + prepared queries
+  if (use_mq(L, n_q))  // + anchor split (+ prepared queries on the multi-query kernel)
+    return use_polar(L, n_q) ? polar_splits(L, n_q, num_sms) + 1 : mq_splits(L, n_q, num_sms) + 2;
   MmaPlan p;
   pick_mma(L, &p);
   const int ntiles = L.Tcap / p.tile;
@@ -727,7 +830,23 @@ static cudaError_t launch_decode_d(const LayerDev& L, const __half* q, int n_q, 
   int nl = 0;
   MmaPlan p;
   int n_quant;  // quantized partials per (query, head)
-  if (use_mq(L, n_q)) {
+  if (D == 128 && use_mq(L, n_q) && use_polar(L, n_q)) {
+    if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
+    const int n_split = polar_splits(L, n_q, num_sms);  // raises the kernel's shared-memory limit
+    n_quant = n_split;
+    const int nsp = n_quant + (L.anchored ? 1 : 0);
+    polar_kernel(L)<<<dim3(n_split, L.Hkv, n_q), PolarCfg::NT, polar_smem(L), st>>>(L, q, seq_ids, kv_len, work,
+                                                                                   n_split, nsp);
+    ++nl;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (L.anchored) {  // anchor rows: the generic kernel's anchor split alone
+      decode_generic_kernel<D><<<dim3(1, L.Hkv, n_q), kGenThreads, 0, st>>>(L, q, seq_ids, kv_len, work, n_quant, nsp,
+                                                                           n_quant);
+      ++nl;
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  } else if (use_mq(L, n_q)) {
     if (L.fuse_n > 0) return cudaErrorInvalidValue;  // the caller checks fused_decode_ok first
     // Tile decode without the format dispatch where both sides' class is known: min-max int codes
     // of 3 or 4 bits in groups of >= 8 (config 2, head_dim 256), rFFT polar (config 4, head_dim 128).

@@ -25,6 +25,7 @@
 #include <stdio.h>
 
 #include "kvq_internal.h"
+#include "fft128.cuh"
 #include "quantize_row.cuh"
 
 namespace kvq {
@@ -104,45 +105,8 @@ __device__ __forceinline__ void finish_append(const LayerDev& L, int n_new, unsi
 
 // ------------------------------------------------------------------------------------------
 // rFFT polar / Cartesian codecs (head_dim 128): one warp per row, the radix-2 DIT FFT in
-// registers, in the evaluation order the format fixes (bit-reversed input; spans 2..128;
-// t = w*b with separately rounded products; (a, b) <- (a + t, a - t)).  Lane l holds elements
-// 4l .. 4l + 3 of the transform: spans 2 and 4 pair elements inside a lane, spans 8 .. 128 pair
-// lane l with lane l ^ (span / 8), and both lanes of a pair form the same t from the same
-// operands, so every element takes exactly the operations of the sequential transform.
+// registers (fft128.cuh), in the evaluation order the format fixes.
 constexpr int kFftWarps = 4;
-
-// One butterfly stage with half-span `half` >= 4 across lanes (partner lane ^ half / 4).
-__device__ __forceinline__ void fft_stage_x(float (&re)[4], float (&im)[4], int half, int lane, const float* twr,
-                                            const float* twi) {
-  const int m = half >> 2, step = 64 / half;
-  const bool up = (lane & m) != 0;  // this lane holds the i1 = i0 + half side
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int j = (4 * lane + r) & (half - 1);
-    const float wr = twr[j * step], wi = twi[j * step];
-    const float ore = __shfl_xor_sync(0xffffffffu, re[r], m), oim = __shfl_xor_sync(0xffffffffu, im[r], m);
-    const float br = up ? re[r] : ore, bi = up ? im[r] : oim;
-    const float ar = up ? ore : re[r], ai = up ? oim : im[r];
-    const float tr = __fsub_rn(__fmul_rn(wr, br), __fmul_rn(wi, bi));
-    const float ti = __fadd_rn(__fmul_rn(wr, bi), __fmul_rn(wi, br));
-    re[r] = up ? __fsub_rn(ar, tr) : __fadd_rn(ar, tr);
-    im[r] = up ? __fsub_rn(ai, ti) : __fadd_rn(ai, ti);
-  }
-}
-
-// In-lane butterfly of elements (p, q = p + half) with twiddle index j * step.
-__device__ __forceinline__ void fft_bfly(float (&re)[4], float (&im)[4], int p, int q, int tw, const float* twr,
-                                         const float* twi) {
-  const float wr = twr[tw], wi = twi[tw];
-  const float br = re[q], bi = im[q];
-  const float tr = __fsub_rn(__fmul_rn(wr, br), __fmul_rn(wi, bi));
-  const float ti = __fadd_rn(__fmul_rn(wr, bi), __fmul_rn(wi, br));
-  const float ar = re[p], ai = im[p];
-  re[p] = __fadd_rn(ar, tr);
-  im[p] = __fadd_rn(ai, ti);
-  re[q] = __fsub_rn(ar, tr);
-  im[q] = __fsub_rn(ai, ti);
-}
 
 // OR a field of `nb` (<= 32) bits at stream bit `bit` into the shared words w.
 __device__ __forceinline__ void or_field(uint32_t* w, int bit, uint32_t v, int nb) {
@@ -189,13 +153,7 @@ __global__ void __launch_bounds__(128) append_fft_kernel(LayerDev L, int side, c
 #pragma unroll
       for (int r = 0; r < 4; ++r) ap[lane + 32 * r] = rp[lane + 32 * r];
     }
-    // spans 2 and 4 inside the lane (element index 4 lane + r: j = r mod half)
-    fft_bfly(re, im, 0, 1, 0, twr, twi);
-    fft_bfly(re, im, 2, 3, 0, twr, twi);
-    fft_bfly(re, im, 0, 2, 0, twr, twi);
-    fft_bfly(re, im, 1, 3, 32, twr, twi);
-#pragma unroll
-    for (int half = 4; half <= 64; half <<= 1) fft_stage_x(re, im, half, lane, twr, twi);
+    fft128_warp(re, im, lane, twr, twi);
     // folded slots f = 2 lane, 2 lane + 1: slot f = X_f (slot 0: (X_0, X_64)); X_f is element f & 3
     // of lane f >> 2
     float a[2], bb[2];
