@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
   __shared__ float w[kMaxSplit + 1];
   __shared__ float rm[NWP], rl[NWP];
   __shared__ float po[SP][D];
-  __shared__ float ov[D], tmp[D];
+  __shared__ float ov[D];
   const int warp = tid >> 5, lane = tid & 31;
   static_assert(NT >= kMaxSplit + 1, "one thread per split's (m, l)");
   // One round trip: every split's (m, l) (thread s takes split s) and this thread's first R
@@ -526,24 +526,28 @@ __global__ void __launch_bounds__(D * merge_groups<D>()) merge_kernel(LayerDev L
     __syncthreads();
   } else if (V.fmt == KVQ_FMT_POLAR || V.fmt == KVQ_FMT_CART) {
     // x_n = (1/N) [a_0 + b_0 (-1)^n + 2 sum_{f=1}^{63} (a_f cos(2 pi f n/N) - b_f sin(2 pi f n/N))]
-    __shared__ float tc[128], tsn[128];  // divergent indices: shared memory, not constant memory
-    if (tid < D) tmp[tid] = ov[tid];
-    if (tid < 128) {
-      tc[tid] = tid < 64 ? d_tw_re[tid] : -d_tw_re[tid - 64];
-      tsn[tid] = tid < 64 ? -d_tw_im[tid] : d_tw_im[tid - 64];  // sin(2 pi k / N)
-    }
-    __syncthreads();
-    if (tid < 128) {
-      const int n = tid;
-      const float acc = tmp[0] + ((n & 1) ? -tmp[1] : tmp[1]);
-      float sacc = 0.0f;
-      for (int f = 1; f < 64; ++f) {
-        const int k = (f * n) & 127;
-        const float c = tc[k];
-        const float sn = tsn[k];
-        sacc += tmp[2 * f] * c - tmp[2 * f + 1] * sn;
+    //     = (1/N) Re FFT(conj Y)_n for the Hermitian spectrum Y (Y_0 = a_0, Y_64 = b_0,
+    //       Y_f = a_f + i b_f, Y_{N-f} = conj Y_f): one warp, the register FFT (bit-reversed input)
+    if (tid < 32) {
+      const int brl = (int)(__brev((unsigned)tid) >> 27);
+      float re[4], im[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int f = brl + 32 * (((r & 1) << 1) | (r >> 1));  // spectrum index of element 4 tid + r
+        if (f == 0 || f == 64) {
+          re[r] = ov[f == 0 ? 0 : 1];
+          im[r] = 0.0f;
+        } else if (f < 64) {
+          re[r] = ov[2 * f];
+          im[r] = -ov[2 * f + 1];
+        } else {
+          re[r] = ov[2 * (128 - f)];
+          im[r] = ov[2 * (128 - f) + 1];
+        }
       }
-      ov[n] = (acc + 2.0f * sacc) / 128.0f;
+      fft128_warp(re, im, tid, g_tw[0], g_tw[1]);  // its shuffles order every lane's reads first
+#pragma unroll
+      for (int r = 0; r < 4; ++r) ov[4 * tid + r] = re[r] / 128.0f;
     }
     __syncthreads();
   }
