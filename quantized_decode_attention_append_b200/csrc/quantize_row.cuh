@@ -101,25 +101,22 @@ __device__ __forceinline__ void pack32_bits(const uint32_t* code, int bits, uint
   }
 }
 
+// The exact code from an estimate k within one of it: the midpoints z + (k -+ 1/2) d, exact in
+// fp64 (fp16 values are multiples of 2^-25 below 2^25), decide (ties toward the larger code).
+__device__ __forceinline__ float settle_minmax(float x, float z, float d, float k) {
+  const double X = x, Z = z, Dd = d;
+  if (X < fma((double)k - 0.5, Dd, Z)) return k - 1.0f;
+  if (X >= fma((double)k + 0.5, Dd, Z)) return k + 1.0f;
+  return k;
+}
+
 // Exact k = floor((x - z)/d + 1/2), d > 0, z and d fp16.  Far from a tie the fp32 estimate is
-// exact (its error is < 2^-14); near one, fp64 thresholds z + (k +- 1/2) d are exact (fp16
-// values are multiples of 2^-25 below 2^25) and decide.
+// exact (its error is < 2^-14); near one it is within one, and settle_minmax decides.
 __device__ __forceinline__ float round_exact_minmax(float x, float z, float d, float inv) {
   const float r = __fmul_rn(__fsub_rn(x, z), inv);
   float k = floorf(__fadd_rn(r, 0.5f));
   const float fr = __fsub_rn(__fadd_rn(r, 0.5f), k);
-  if (fr < (1.0f / 1024.0f) || fr > (1.0f - 1.0f / 1024.0f)) {
-    const double X = x, Z = z, Dd = d;
-    double kk = floor(__dadd_rn(__ddiv_rn(__dsub_rn(X, Z), Dd), 0.5));
-    const double lo = __dadd_rn(Z, __dmul_rn(__dsub_rn(kk, 0.5), Dd));
-    if (X < lo) {
-      kk -= 1.0;
-    } else {
-      const double hi = __dadd_rn(Z, __dmul_rn(__dadd_rn(kk, 0.5), Dd));
-      if (X >= hi) kk += 1.0;
-    }
-    k = (float)kk;
-  }
+  if (fr < (1.0f / 1024.0f) || fr > (1.0f - 1.0f / 1024.0f)) k = settle_minmax(x, z, d, k);
   return k;
 }
 

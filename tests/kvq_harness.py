@@ -15,19 +15,24 @@ from quantized_decode_attention_append_b200.kvq import Config, KVCache, Side
 TOL = 2e-3  # max relative error (inf-norm per query-head vector) of decode attention
 
 
-def kernel_names(run, want, tries: int = 6) -> str:
+def kernel_names(run, want, tries: int = 8, repeat: int = 3) -> str:
     """Names of the CUDA kernels `run()` launches, seen by the torch profiler.  Its kernel records
-    occasionally arrive incomplete, so it looks again (up to `tries` times) until every name in
-    `want` is present."""
+    sometimes arrive incomplete -- the first launches of a session can be missing -- so each
+    session calls `run()` `repeat` times (the same launches each time), and it looks again, up to
+    `tries` times with a short pause, until every name in `want` is present."""
+    import time
+
     from torch.profiler import ProfilerActivity, profile
     names = ""
-    for _ in range(tries):
+    for i in range(tries):
         with profile(activities=[ProfilerActivity.CUDA]) as prof:
-            run()
+            for _ in range(repeat):
+                run()
             torch.cuda.synchronize()
         names = " ".join(e.name for e in prof.events())
         if all(w in names for w in want):
             break
+        time.sleep(0.05 * (i + 1))
     return names
 
 
