@@ -25,6 +25,7 @@ def kernel_names(run, want, tries: int = 8, repeat: int = 3) -> str:
     from torch.profiler import ProfilerActivity, profile
     names = ""
     for i in range(tries):
+        torch.cuda.empty_cache()  # room for the profiler's activity buffers after large tests
         with profile(activities=[ProfilerActivity.CUDA]) as prof:
             for _ in range(repeat):
                 run()

@@ -76,6 +76,19 @@ def test_mma_kernel_is_the_one_that_runs(k, v):
     assert kvq.kvq_last_launch_count(c.cache.h) == 2
 
 
+def test_symmetric_v_runs_on_tensor_cores():
+    """The symmetric 2-bit V grid ("E22L" "Result") under a 256-wide rotation has a register-decode
+    instance."""
+    cfg = Config(n_layers=1, batch=2, n_kv_heads=2, n_q_heads=8, head_dim=256, capacity=512,
+                 k=Side("int", 4, group=128, rot=256), v=Side("int", 2, scale="sym", group=128, rot=256), max_queries=8)
+    c = Case(cfg, 512)
+    q = synth.queries(1, 0, 2, cfg.n_q_heads, 256, 512).cuda()
+    c.cache.decode(0, q)
+    torch.cuda.synchronize()
+    names = kernel_names(lambda: c.cache.decode(0, q), ["decode_tc_kernel", "merge_kernel"])
+    assert "decode_tc_kernel" in names and "decode_generic_kernel" not in names
+
+
 def test_append_is_one_launch_for_common_pairs():
     cfg = Config(n_layers=1, batch=2, n_kv_heads=2, n_q_heads=8, head_dim=128, capacity=128,
                  k=Side("nf4", group=64), v=Side("int", 4, group=64), max_queries=8)
