@@ -293,3 +293,22 @@ def test_head_allocation_matches_the_oracle_rule():
             else:
                 assert bits[l][h] == want_bits[l, h] and hk[l][h].bits == want_bits[l, h]
     assert hk == hv
+
+
+def test_decode_source_hash_covers_every_local_header_of_the_decode_unit():
+    """bench.py keys the committed DRAM-traffic summary to a hash of the decode kernels' sources:
+    every csrc header the decode translation unit includes (directly or through another header)
+    must be in that list, or a kernel change could leave a stale traffic number in the bench line."""
+    import bench
+    csrc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "quantized_decode_attention_append_b200", "csrc")
+    seen, todo = set(), ["decode.cu"]
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        for inc in re.findall(r'^#include "([^"/]+)"', open(os.path.join(csrc, f)).read(), re.M):
+            if os.path.exists(os.path.join(csrc, inc)):
+                todo.append(inc)
+    assert seen <= set(bench.DECODE_SOURCES), sorted(seen - set(bench.DECODE_SOURCES))
